@@ -1,0 +1,693 @@
+"""Plain, slow, fp64 CPU oracle for the JoLT compress -> decompress path.
+
+TEST INFRASTRUCTURE ONLY. Only the test suite, the package's smoke check and
+the benchmark's CPU-baseline leg may import this module. It shares no code
+with the CUDA library, and the library never calls it.
+
+What it follows: "A JoLT for the KV Cache: Near-Lossless KV Cache Compression
+via Joint Rank-bit Allocation" (Krishnan & Schulz), Section 3:
+  * "Partial Tucker backbone"       -> token_spectrum, feature_spectrum, fit
+  * "Rotated low-bit residual"      -> rotate / quantize / pack, residual_*
+  * "Joint Lagrangian allocation"   -> Eq. (1) cost_bytes, Eq. (2) error model,
+                                       eps2_table
+  * "Solving the allocation"        -> Eqs. (3)-(4): argmin_cell, allocate,
+                                       greedy_cell (the page's own heuristic)
+  * Section 3.1 "FlashJoLT", Eq. (5) -> q_cap (the randomized mode itself is
+                                       not in the oracle: the oracle is exact)
+and, for keys, the pre-RoPE handling of Section 3 (keys decomposed before the
+rotary embedding; the rotation re-applied to the reconstruction).
+
+Readings taken where the pages leave a step open (each is a knob of the
+library as well):
+  R1 quantizer: symmetric, mid-tread, absmax scaling, q_max = 2^(b-1)-1,
+     scale = fl32(absmax / q_max), code = clamp(rint(fl32(r / scale))),
+     stored as u = code + 2^(b-1) in b bits, LSB first, per row of D values.
+     One fp32 scale per group of g_q consecutive rotated values (g_q = D is
+     the page's "one fp32 scale per row"). The Gaussian round trip of this
+     quantizer reproduces the printed eps^2 values (see the tests).
+  R2 rotation: seeded randomized Hadamard R = D^(-1/2) H_D diag(s), s in
+     {+1,-1}^D from Philox4x32-10; the fast transform runs in fp32 with stages
+     h = 1, 2, 4, ..., D/2 and butterflies (a, b) -> (a + b, a - b), then one
+     multiply by fl32(1/sqrt(D)).
+  R3 per-cell minimizer: exact enumeration (b ascending, r_T ascending, r_d
+     ascending; strict < keeps the first minimum), which is what the
+     multiplier theorem needs; the page's greedy search is `greedy_cell`.
+  R4 bisection: lambda in [1e-30, 1], lambda_mid = sqrt(lo * hi), stop when
+     (1 - tol) B <= sum s <= B or after max_iters; otherwise the feasible
+     (hi) side is returned. e + lambda*s is two separately rounded operations.
+  R5 stored factors are bf16 (c = 2 in Eq. 1): U_T^ = bf16(U_T),
+     Y = X x_T U_T^T, U_d from the feature Gram of Y, U_d^ = bf16(U_d),
+     G^ = bf16(Y x_d U_d^T), and the decoder's per-(layer, head) product
+     M^ = bf16(G^ U_d^^T). The residual is taken against U_T^ M^, the
+     reconstruction the decoder actually forms, so storage rounding lands in
+     the residual.
+  R6 keys with a RoPE base theta: X = RoPE^{-1}(K) in fp32 from an fp32
+     cos/sin table (angles computed in fp64), rotate-half pairing; decode
+     re-applies RoPE in fp32 before the final bf16 rounding.
+  R7 sign of every singular/eigen vector: its largest-magnitude entry is
+     positive (first such entry on ties).
+  R8 budget C: B = floor(dense bf16 bytes of K and V / C).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+# --------------------------------------------------------------------------
+# Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
+# as 1, 2, 3", SC'11), written from its published definition.
+# --------------------------------------------------------------------------
+_PHILOX_M0 = np.uint64(0xD2511F53)
+_PHILOX_M1 = np.uint64(0xCD9E8D57)
+_PHILOX_W0 = np.uint64(0x9E3779B9)
+_PHILOX_W1 = np.uint64(0xBB67AE85)
+_MASK32 = np.uint64(0xFFFFFFFF)
+
+# stream tags: the third counter word separates the random quantities
+STREAM_HADAMARD = 1
+STREAM_CALIB = 2
+STREAM_SKETCH = 3
+STREAM_QRGAUSS = 4
+
+
+def philox4x32_10(ctr: np.ndarray, key: Tuple[int, int]) -> np.ndarray:
+    """ctr: uint32 array [..., 4]; returns uint32 [..., 4]."""
+    c = [ctr[..., i].astype(np.uint64) for i in range(4)]
+    k0 = np.uint64(key[0] & 0xFFFFFFFF)
+    k1 = np.uint64(key[1] & 0xFFFFFFFF)
+    for _ in range(10):
+        p0 = _PHILOX_M0 * c[0]
+        p1 = _PHILOX_M1 * c[2]
+        hi0, lo0 = p0 >> np.uint64(32), p0 & _MASK32
+        hi1, lo1 = p1 >> np.uint64(32), p1 & _MASK32
+        c = [(hi1 ^ c[1] ^ k0) & _MASK32, lo1, (hi0 ^ c[3] ^ k1) & _MASK32, lo0]
+        k0 = (k0 + _PHILOX_W0) & _MASK32
+        k1 = (k1 + _PHILOX_W1) & _MASK32
+    return np.stack([x.astype(np.uint32) for x in c], axis=-1)
+
+
+def philox_block(n_ctr: int, seed: int, stream: int, hi: int = 0) -> np.ndarray:
+    """Words for counters (i, hi, stream, 0), i = 0..n_ctr-1, key = seed's two
+    32-bit halves. Returns uint32 [n_ctr, 4]."""
+    ctr = np.zeros((n_ctr, 4), dtype=np.uint32)
+    ctr[:, 0] = np.arange(n_ctr, dtype=np.uint64).astype(np.uint32)
+    ctr[:, 1] = np.uint32(hi & 0xFFFFFFFF)
+    ctr[:, 2] = np.uint32(stream)
+    return philox4x32_10(ctr, (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF))
+
+
+def gaussian_f64(n: int, seed: int, stream: int) -> np.ndarray:
+    """n standard normals: each Philox call gives 4 words, u = (w + 0.5) 2^-32,
+    and Box-Muller turns (u0, u1) and (u2, u3) into two pairs (fp64)."""
+    nc = (n + 3) // 4
+    w = philox_block(nc, seed, stream).astype(np.float64)
+    u = (w + 0.5) * (2.0 ** -32)
+    r0 = np.sqrt(-2.0 * np.log(u[:, 0]))
+    r1 = np.sqrt(-2.0 * np.log(u[:, 2]))
+    t0 = 2.0 * math.pi * u[:, 1]
+    t1 = 2.0 * math.pi * u[:, 3]
+    z = np.stack([r0 * np.cos(t0), r0 * np.sin(t0), r1 * np.cos(t1), r1 * np.sin(t1)], axis=1)
+    return z.reshape(-1)[:n]
+
+
+def hadamard_signs(D: int, seed: int) -> np.ndarray:
+    """s_i = +1 if bit 0 of word 0 of Philox((i, 0, STREAM_HADAMARD, 0)) is 0,
+    else -1. Returns fp32 [D]."""
+    w = philox_block(D, seed, STREAM_HADAMARD)[:, 0]
+    return np.where((w & 1) == 0, 1.0, -1.0).astype(np.float32)
+
+
+# --------------------------------------------------------------------------
+# rounding helpers
+# --------------------------------------------------------------------------
+def bf16_rne(x: np.ndarray) -> np.ndarray:
+    """Round fp64 (or fp32) values to the nearest bf16 (ties to even), directly
+    from the input precision, returned as fp64. Overflow is not handled (the
+    values here are far from the bf16 range limits)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                       # x = m 2^e, 0.5 <= |m| < 1
+    # bf16 keeps 8 significant bits; below 2^-126 the spacing is fixed 2^-133
+    e_eff = np.maximum(e, -125)
+    q = np.rint(np.ldexp(m, 8 + (e - e_eff)))
+    return np.ldexp(q, e_eff - 8)
+
+
+def f32(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float32)
+
+
+# --------------------------------------------------------------------------
+# RoPE (keys only), reading R6
+# --------------------------------------------------------------------------
+def rope_table(T: int, D: int, theta: float) -> Tuple[np.ndarray, np.ndarray]:
+    """cos, sin as fp32 [T, D/2]: angle(t, i) = t * theta^(-2i/D) in fp64."""
+    half = D // 2
+    inv = theta ** (-2.0 * np.arange(half, dtype=np.float64) / D)
+    ang = np.arange(T, dtype=np.float64)[:, None] * inv[None, :]
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def unrope_f32(y: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """Inverse rotate-half RoPE, fp32, no fused multiply-add:
+    x_i = y_i c + y_j s ; x_j = y_j c - y_i s, j = i + D/2."""
+    y = f32(y)
+    half = y.shape[-1] // 2
+    a, b = y[..., :half], y[..., half:]
+    xa = f32(a * cos) + f32(b * sin)
+    xb = f32(b * cos) - f32(a * sin)
+    return np.concatenate([f32(xa), f32(xb)], axis=-1)
+
+
+def rope_f32(x: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """Forward rotate-half RoPE, fp32: y_i = x_i c - x_j s ; y_j = x_j c + x_i s."""
+    x = f32(x)
+    half = x.shape[-1] // 2
+    a, b = x[..., :half], x[..., half:]
+    ya = f32(a * cos) - f32(b * sin)
+    yb = f32(b * cos) + f32(a * sin)
+    return np.concatenate([f32(ya), f32(yb)], axis=-1)
+
+
+# --------------------------------------------------------------------------
+# rotation, quantizer and bit packing (readings R1, R2)
+# --------------------------------------------------------------------------
+def fwht_f32(v: np.ndarray) -> np.ndarray:
+    """Unnormalised Walsh-Hadamard transform along the last axis (natural
+    order), fp32, stages h = 1, 2, ..., D/2."""
+    v = f32(v).copy()
+    D = v.shape[-1]
+    h = 1
+    while h < D:
+        w = v.reshape(v.shape[:-1] + (D // (2 * h), 2, h))
+        a = w[..., 0, :].copy()
+        b = w[..., 1, :].copy()
+        w[..., 0, :] = a + b
+        w[..., 1, :] = a - b
+        v = w.reshape(v.shape)
+        h *= 2
+    return v
+
+
+def rot_scale(D: int) -> np.float32:
+    return np.float32(1.0 / math.sqrt(D))
+
+
+def rotate(E: np.ndarray, signs: np.ndarray) -> np.ndarray:
+    """r = fl32( FWHT(s * E) * fl32(1/sqrt(D)) ) along the last axis (fp32)."""
+    return f32(fwht_f32(f32(E) * signs) * rot_scale(E.shape[-1]))
+
+
+def unrotate(r: np.ndarray, signs: np.ndarray) -> np.ndarray:
+    """R^T r = s * fl32( FWHT(r) * fl32(1/sqrt(D)) ) (fp32)."""
+    return f32(f32(fwht_f32(r) * rot_scale(r.shape[-1])) * signs)
+
+
+def qmax(b: int) -> int:
+    return (1 << (b - 1)) - 1
+
+
+def quantize(r: np.ndarray, b: int, g: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Rows [..., D] fp32 -> (codes int32 [..., D] in [-q_max, q_max],
+    scales fp32 [..., D/g])."""
+    r = f32(r)
+    D = r.shape[-1]
+    grp = r.reshape(r.shape[:-1] + (D // g, g))
+    a = np.max(np.abs(grp), axis=-1)
+    scale = f32(a / np.float32(qmax(b)))
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = np.rint(f32(grp / safe[..., None]))
+    q = np.clip(q, -qmax(b), qmax(b))
+    q = np.where(scale[..., None] > 0, q, 0.0)
+    return q.reshape(r.shape).astype(np.int32), scale
+
+
+def dequantize(codes: np.ndarray, scales: np.ndarray, g: int) -> np.ndarray:
+    D = codes.shape[-1]
+    c = codes.reshape(codes.shape[:-1] + (D // g, g)).astype(np.float32)
+    return f32(c * scales[..., None]).reshape(codes.shape)
+
+
+def pack_bits(codes: np.ndarray, b: int) -> np.ndarray:
+    """u = code + 2^(b-1); element i of a row occupies bits [i b, (i+1) b) of
+    that row's little-endian bit stream. Returns uint8 [..., b*D/8]."""
+    u = (codes.astype(np.int64) + (1 << (b - 1))).astype(np.uint64)
+    D = codes.shape[-1]
+    bits = ((u[..., :, None] >> np.arange(b, dtype=np.uint64)) & np.uint64(1)).astype(np.uint8)
+    bits = bits.reshape(codes.shape[:-1] + (D * b,))
+    return np.packbits(bits, axis=-1, bitorder="little")
+
+
+def unpack_bits(packed: np.ndarray, b: int, D: int) -> np.ndarray:
+    bits = np.unpackbits(packed, axis=-1, bitorder="little")[..., : D * b]
+    bits = bits.reshape(packed.shape[:-1] + (D, b)).astype(np.int64)
+    u = np.sum(bits << np.arange(b, dtype=np.int64), axis=-1)
+    return (u - (1 << (b - 1))).astype(np.int32)
+
+
+# --------------------------------------------------------------------------
+# eps^2(b): "calibrated once on a Gaussian round-trip", eps^2(0) = 1
+# --------------------------------------------------------------------------
+CALIB_SAMPLES = 1 << 20
+CALIB_SEED = 0
+
+
+def eps2_table(bits: Sequence[int], g: int, n: int = CALIB_SAMPLES,
+               seed: int = CALIB_SEED) -> Dict[int, float]:
+    """Fraction of a Gaussian's energy the b-bit quantizer fails to recover,
+    with groups of g values; the samples are rounded to fp32 first."""
+    x = f32(gaussian_f64(n, seed, STREAM_CALIB)).reshape(-1, g)
+    out = {}
+    for b in bits:
+        if b == 0:
+            out[b] = 1.0
+            continue
+        c, s = quantize(x, b, g)
+        xh = dequantize(c, s, g)
+        d = x.astype(np.float64) - xh.astype(np.float64)
+        out[b] = float(np.sum(d * d) / np.sum(x.astype(np.float64) ** 2))
+    return out
+
+
+# --------------------------------------------------------------------------
+# Eq. (1) cost and Eq. (5) cap
+# --------------------------------------------------------------------------
+def residual_row_bytes(b: int, D: int, g: int) -> int:
+    """b bits per value plus one fp32 scale per g values, for a row of D."""
+    if b == 0:
+        return 0
+    nbits = b * D + 32 * (D // g)
+    assert nbits % 8 == 0
+    return nbits // 8
+
+
+def cost_bytes(Lg: int, H: int, T: int, D: int, rT: int, rd: int, b: int,
+               g: int, c: int = 2) -> int:
+    """Eq. (1): (|g| n_h r_T r_d + T r_T + d_h r_d) c + [b>0] (b + 32/g)/8 |g| n_h T d_h."""
+    return (Lg * H * rT * rd + T * rT + D * rd) * c + residual_row_bytes(b, D, g) * Lg * H * T
+
+
+def q_cap(T: int, C: float) -> int:
+    """Eq. (5): min(max(q_min(C), ceil(T/32)), 512), q_min = 32 (C <= 4) or 64."""
+    qmin = 32 if C <= 4 else 64
+    return min(max(qmin, -(-T // 32)), 512)
+
+
+# --------------------------------------------------------------------------
+# spectra (exact mode)
+# --------------------------------------------------------------------------
+def fix_signs(U: np.ndarray) -> np.ndarray:
+    """Reading R7: each column's largest-|.| entry made positive (first on ties)."""
+    idx = np.argmax(np.abs(U), axis=0)
+    s = np.sign(U[idx, np.arange(U.shape[1])])
+    s[s == 0] = 1.0
+    return U * s[None, :]
+
+
+def token_unfolding(X: np.ndarray) -> np.ndarray:
+    """X [Lg, H, T, D] -> X_(T) [T, Lg*H*D], column index (l, h, d)."""
+    Lg, H, T, D = X.shape
+    return np.transpose(X, (2, 0, 1, 3)).reshape(T, Lg * H * D)
+
+
+def feature_gram(X: np.ndarray) -> np.ndarray:
+    """X_(d) X_(d)^T = sum over (l, h, t) of x x^T, D x D, fp64."""
+    D = X.shape[-1]
+    F = X.reshape(-1, D)
+    return F.T @ F
+
+
+def token_spectrum(X: np.ndarray, r_needed: Optional[int] = None):
+    """Squared singular values of X_(T) (descending, all min(T, N) of them) and
+    the left singular vectors (T x r_needed, signs fixed), from the Gram
+    matrix on the smaller side: X X^T when T <= N, else X^T X with
+    U = X V Sigma^-1."""
+    XT = token_unfolding(X)
+    T, N = XT.shape
+    if T <= N:
+        G = XT @ XT.T
+        w, U = np.linalg.eigh(G)
+        order = np.argsort(-w, kind="stable")
+        w, U = w[order], U[:, order]
+        w = np.maximum(w, 0.0)
+        U = fix_signs(U)
+        if r_needed is not None:
+            U = U[:, :r_needed]
+        return w, U
+    G = XT.T @ XT
+    w, V = np.linalg.eigh(G)
+    order = np.argsort(-w, kind="stable")
+    w, V = np.maximum(w[order], 0.0), V[:, order]
+    r = N if r_needed is None else r_needed
+    sv = np.sqrt(w[:r])
+    U = (XT @ V[:, :r]) / np.where(sv > 0, sv, 1.0)[None, :]
+    return w, fix_signs(U)
+
+
+def feature_spectrum(X: np.ndarray) -> np.ndarray:
+    w = np.linalg.eigvalsh(feature_gram(X))
+    return np.maximum(np.sort(w)[::-1], 0.0)
+
+
+def tail_fractions(sig2: np.ndarray, normsq: float) -> np.ndarray:
+    """t[r] = sum_{i > r} sig2_i / ||X||^2 for r = 0..n, summed smallest first."""
+    n = len(sig2)
+    t = np.zeros(n + 1)
+    acc = 0.0
+    for i in range(n - 1, -1, -1):
+        acc += float(sig2[i])
+        t[i] = acc / normsq
+    t[n] = 0.0
+    return t
+
+
+# --------------------------------------------------------------------------
+# rate-distortion table and allocation, Eqs. (1)-(4)
+# --------------------------------------------------------------------------
+@dataclasses.dataclass
+class CellTable:
+    Lg: int
+    H: int
+    T: int
+    D: int
+    g: int
+    normsq: float
+    tT: np.ndarray           # t_T[r], r = 0..len
+    tD: np.ndarray           # t_D[r], r = 0..D
+    rt_grid: np.ndarray      # candidate r_T values (ascending)
+    rd_grid: np.ndarray      # candidate r_d values (ascending)
+    bits: np.ndarray         # candidate b values (ascending)
+    eps2: np.ndarray         # eps^2(b) for each entry of `bits`
+
+    def options(self):
+        """(b, r_T, r_d, e, s) in enumeration order: b, then r_T, then r_d."""
+        for bi, b in enumerate(self.bits):
+            for rT in self.rt_grid:
+                for rd in self.rd_grid:
+                    e = float(self.eps2[bi]) * (float(self.tT[rT]) + float(self.tD[rd]))
+                    s = cost_bytes(self.Lg, self.H, self.T, self.D, int(rT), int(rd), int(b), self.g)
+                    yield int(b), int(rT), int(rd), e, s
+
+    def arrays(self):
+        """All options as arrays (same enumeration order)."""
+        bb, tt, dd = np.meshgrid(self.bits, self.rt_grid, self.rd_grid, indexing="ij")
+        ei = np.broadcast_to(self.eps2[:, None, None], bb.shape)
+        e = ei * (self.tT[tt] + self.tD[dd])
+        rb = np.array([residual_row_bytes(int(x), self.D, self.g) for x in self.bits], dtype=np.int64)
+        rbb = np.broadcast_to(rb[:, None, None], bb.shape)
+        s = (self.Lg * self.H * tt * dd + self.T * tt + self.D * dd) * 2 + rbb * (self.Lg * self.H * self.T)
+        return bb.ravel(), tt.ravel(), dd.ravel(), e.ravel().astype(np.float64), s.ravel().astype(np.int64)
+
+
+def argmin_cell(tab: CellTable, lam: float, arrays=None) -> int:
+    """Index (enumeration order) of the first option minimising e + lam*s; the
+    product and the sum are separately rounded fp64 operations."""
+    b, t, d, e, s = arrays if arrays is not None else tab.arrays()
+    v = e + (lam * s.astype(np.float64))
+    return int(np.argmin(v))          # numpy returns the first minimum
+
+
+@dataclasses.dataclass
+class Allocation:
+    choice: List[Tuple[int, int, int]]    # (r_T, r_d, b) per cell
+    bytes: List[int]
+    errors: List[float]                   # surrogate e per cell
+    lam: float
+    iters: int
+
+
+def allocate(tables: List[CellTable], budget: int, tol: float = 0.005,
+             max_iters: int = 50, lam_lo: float = 1e-30, lam_hi: float = 1.0) -> Allocation:
+    """Geometric bisection on the shared multiplier lambda (reading R4)."""
+    arrs = [t.arrays() for t in tables]
+
+    def at(lam):
+        idx = [argmin_cell(t, lam, a) for t, a in zip(tables, arrs)]
+        S = int(sum(int(a[4][i]) for a, i in zip(arrs, idx)))
+        return idx, S
+
+    def pack(idx, lam, it):
+        ch = [(int(a[1][i]), int(a[2][i]), int(a[0][i])) for a, i in zip(arrs, idx)]
+        by = [int(a[4][i]) for a, i in zip(arrs, idx)]
+        er = [float(a[3][i]) for a, i in zip(arrs, idx)]
+        return Allocation(ch, by, er, lam, it)
+
+    idx, S = at(lam_lo)
+    if S <= budget:
+        return pack(idx, lam_lo, 0)
+    idx_hi, S_hi = at(lam_hi)
+    if S_hi > budget:
+        raise ValueError("budget infeasible")
+    lo, hi = lam_lo, lam_hi
+    for it in range(1, max_iters + 1):
+        mid = math.sqrt(lo * hi)
+        idx, S = at(mid)
+        if (1.0 - tol) * budget <= S <= budget:
+            return pack(idx, mid, it)
+        if S > budget:
+            lo = mid
+        else:
+            hi, idx_hi = mid, idx
+    return pack(idx_hi, hi, max_iters)
+
+
+def greedy_cell(tab: CellTable, lam: float) -> Tuple[int, int, int, float]:
+    """The page's per-cell search under integer rank grids: for every b, start
+    at r_T = r_d = 1 and repeatedly take whichever single-step rank increment
+    has the steeper error decrease per byte, as long as that step lowers
+    e + lam*s; keep the b with the smallest e + lam*s. Returns
+    (r_T, r_d, b, value)."""
+    best = None
+    rmaxT = len(tab.tT) - 1
+    rmaxD = len(tab.tD) - 1
+    for bi, b in enumerate(tab.bits):
+        eps = float(tab.eps2[bi])
+        rT, rd = 1, 1
+
+        def val(a, c):
+            e = eps * (float(tab.tT[a]) + float(tab.tD[c]))
+            s = cost_bytes(tab.Lg, tab.H, tab.T, tab.D, a, c, int(b), tab.g)
+            return e + lam * s, e, s
+
+        while True:
+            v0, e0, s0 = val(rT, rd)
+            cands = []
+            if rT < rmaxT:
+                v1, e1, s1 = val(rT + 1, rd)
+                if v1 < v0:
+                    cands.append(((e0 - e1) / (s1 - s0), 0))
+            if rd < rmaxD:
+                v2, e2, s2 = val(rT, rd + 1)
+                if v2 < v0:
+                    cands.append(((e0 - e2) / (s2 - s0), 1))
+            if not cands:
+                break
+            cands.sort(key=lambda z: (-z[0], z[1]))
+            if cands[0][1] == 0:
+                rT += 1
+            else:
+                rd += 1
+        v, _, _ = val(rT, rd)
+        if best is None or v < best[3]:
+            best = (rT, rd, int(b), v)
+    return best
+
+
+# --------------------------------------------------------------------------
+# fit (ST-HOSVD with stored bf16 factors, reading R5)
+# --------------------------------------------------------------------------
+@dataclasses.dataclass
+class CellFit:
+    UT: np.ndarray      # T x r_T   (bf16 values as fp64)
+    Ud: np.ndarray      # D x r_d   (bf16 values)
+    G: np.ndarray       # Lg x H x r_T x r_d (bf16 values)
+    M: np.ndarray       # Lg x H x r_T x D   (bf16 values) = bf16(G Ud^T)
+
+
+def fit(X: np.ndarray, U_T: np.ndarray, rT: int, rd: int, store_f64: bool = False) -> CellFit:
+    """Token factor first, then the feature factor on the projected tensor."""
+    rnd = (lambda a: np.asarray(a, dtype=np.float64)) if store_f64 else bf16_rne
+    UT = rnd(U_T[:, :rT])
+    Y = np.einsum("tr,lhtd->lhrd", UT, X)                 # X x_T UT^T
+    C = feature_gram(Y)
+    w, V = np.linalg.eigh(C)
+    order = np.argsort(-w, kind="stable")
+    Ud = rnd(fix_signs(V[:, order])[:, :rd])
+    G = rnd(np.einsum("lhrd,de->lhre", Y, Ud))            # Y x_d Ud^T
+    M = rnd(np.einsum("lhre,de->lhrd", G, Ud))            # G Ud^T per (l, h)
+    return CellFit(UT, Ud, G, M)
+
+
+def backbone(f: CellFit) -> np.ndarray:
+    """X~ = U_T^ M^ per (layer, head), fp64."""
+    return np.einsum("tr,lhrd->lhtd", f.UT, f.M)
+
+
+# --------------------------------------------------------------------------
+# residual encode / decode
+# --------------------------------------------------------------------------
+@dataclasses.dataclass
+class Residual:
+    b: int
+    codes: Optional[np.ndarray]     # int32 [Lg, H, T, D]
+    packed: Optional[np.ndarray]    # uint8 [Lg, H, T, b*D/8]
+    scales: Optional[np.ndarray]    # fp32 [Lg, H, T, D/g]
+
+
+def residual_from(X: np.ndarray, Xt: np.ndarray) -> np.ndarray:
+    """E = X - X~ in fp64, rounded once to fp32."""
+    return f32(np.asarray(X, np.float64) - Xt)
+
+
+def encode_residual(E: np.ndarray, b: int, g: int, signs: np.ndarray) -> Residual:
+    if b == 0:
+        return Residual(0, None, None, None)
+    r = rotate(E, signs)
+    codes, scales = quantize(r, b, g)
+    return Residual(b, codes, pack_bits(codes, b), scales)
+
+
+def decode_residual(res: Residual, g: int, signs: np.ndarray, D: int) -> Optional[np.ndarray]:
+    if res.b == 0:
+        return None
+    codes = unpack_bits(res.packed, res.b, D)
+    return unrotate(dequantize(codes, res.scales, g), signs)
+
+
+# --------------------------------------------------------------------------
+# the whole path
+# --------------------------------------------------------------------------
+@dataclasses.dataclass
+class Options:
+    bits: Tuple[int, ...] = (0, 2, 4, 8)
+    rt_grid: Optional[Tuple[int, ...]] = None     # None: 1..r_max
+    rd_grid: Optional[Tuple[int, ...]] = None     # None: 1..D
+    rt_max: int = 0                               # 0: min(T, N)
+    scale_group: int = 0                          # 0: D (one scale per row)
+    tol: float = 0.005
+    max_iters: int = 50
+
+
+@dataclasses.dataclass
+class CellRef:
+    b: int          # sequence
+    g: int          # group
+    kind: int       # 0 = K, 1 = V
+    l0: int
+    l1: int
+
+
+def cells_of(batch: int, group_starts: Sequence[int]) -> List[CellRef]:
+    """Cell order: sequence, then group, then K before V."""
+    out = []
+    for b in range(batch):
+        for g in range(len(group_starts) - 1):
+            for kind in (0, 1):
+                out.append(CellRef(b, g, kind, group_starts[g], group_starts[g + 1]))
+    return out
+
+
+def cell_tensor(cache_k: np.ndarray, cache_v: np.ndarray, c: CellRef, rope_theta_k: float) -> np.ndarray:
+    """The cell's compression target X [Lg, H, T, D] as fp64 values."""
+    src = cache_k if c.kind == 0 else cache_v
+    X = f32(src[c.b, c.l0:c.l1])
+    if c.kind == 0 and rope_theta_k > 0:
+        cs, sn = rope_table(X.shape[2], X.shape[3], rope_theta_k)
+        X = unrope_f32(X, cs, sn)
+    return X.astype(np.float64)
+
+
+def build_table(X: np.ndarray, opt: Options, eps2: Dict[int, float]) -> Tuple[CellTable, np.ndarray, np.ndarray]:
+    Lg, H, T, D = X.shape
+    g = opt.scale_group or D
+    normsq = float(np.sum(X * X))
+    sT, UT = token_spectrum(X)
+    sD = feature_spectrum(X)
+    rmax = opt.rt_max or min(T, Lg * H * D)
+    rt = np.array(opt.rt_grid if opt.rt_grid else range(1, rmax + 1), dtype=np.int64)
+    rd = np.array(opt.rd_grid if opt.rd_grid else range(1, D + 1), dtype=np.int64)
+    tab = CellTable(Lg, H, T, D, g, normsq, tail_fractions(sT, normsq), tail_fractions(sD, normsq),
+                    rt, rd, np.array(opt.bits, dtype=np.int64),
+                    np.array([eps2[b] for b in opt.bits], dtype=np.float64))
+    return tab, sT, UT
+
+
+@dataclasses.dataclass
+class CompressedCell:
+    ref: CellRef
+    rT: int
+    rd: int
+    b: int
+    fit: CellFit
+    res: Residual
+    bytes: int
+
+
+@dataclasses.dataclass
+class Compressed:
+    cells: List[CompressedCell]
+    alloc: Allocation
+    shape: Tuple[int, ...]
+    rope_theta_k: float
+    seed: int
+    g_of_D: int
+
+
+def compress(cache_k: np.ndarray, cache_v: np.ndarray, group_starts: Sequence[int],
+             budget: int, seed: int, opt: Options = Options(), rope_theta_k: float = 0.0) -> Compressed:
+    """Exact JoLT: spectra of every cell, one shared-multiplier allocation over
+    all cells, then the ST-HOSVD fit and the rotated low-bit residual."""
+    B, L, H, T, D = cache_k.shape
+    g = opt.scale_group or D
+    eps2 = eps2_table(opt.bits, g)
+    refs = cells_of(B, group_starts)
+    tabs, Us, Xs = [], [], []
+    for c in refs:
+        X = cell_tensor(cache_k, cache_v, c, rope_theta_k)
+        tab, _, U = build_table(X, opt, eps2)
+        tabs.append(tab)
+        Us.append(U)
+        Xs.append(X)
+    al = allocate(tabs, budget, opt.tol, opt.max_iters)
+    out = []
+    for c, X, U, (rT, rd, b), nb in zip(refs, Xs, Us, al.choice, al.bytes):
+        f = fit(X, U, rT, rd)
+        sg = hadamard_signs(D, seed + c.b)
+        res = encode_residual(residual_from(X, backbone(f)), b, g, sg)
+        out.append(CompressedCell(c, rT, rd, b, f, res, nb))
+    return Compressed(out, al, (B, L, H, T, D), rope_theta_k, seed, g)
+
+
+def decompress_cell(cc: CompressedCell, D: int, g: int, seed: int, rope_theta_k: float) -> np.ndarray:
+    """X^ = bf16( [RoPE]( X~ + R^T dequant(codes) ) ), fp32 sum and RoPE."""
+    Xt = backbone(cc.fit)
+    sg = hadamard_signs(D, seed + cc.ref.b)
+    e = decode_residual(cc.res, g, sg, D)
+    x = f32(Xt) if e is None else f32(f32(Xt) + e)
+    if cc.ref.kind == 0 and rope_theta_k > 0:
+        cs, sn = rope_table(x.shape[2], D, rope_theta_k)
+        x = rope_f32(x, cs, sn)
+    return bf16_rne(x)
+
+
+def decompress(comp: Compressed) -> Tuple[np.ndarray, np.ndarray]:
+    B, L, H, T, D = comp.shape
+    K = np.zeros(comp.shape, np.float64)
+    V = np.zeros(comp.shape, np.float64)
+    for cc in comp.cells:
+        dst = K if cc.ref.kind == 0 else V
+        dst[cc.ref.b, cc.ref.l0:cc.ref.l1] = decompress_cell(cc, D, comp.g_of_D, comp.seed, comp.rope_theta_k)
+    return K, V
+
+
+def rel_frobenius(X: np.ndarray, Xh: np.ndarray) -> float:
+    X = np.asarray(X, np.float64)
+    d = X - np.asarray(Xh, np.float64)
+    return math.sqrt(float(np.sum(d * d)) / float(np.sum(X * X)))
+
+
+def budget_for_ratio(n_elems_kv: int, C: float) -> int:
+    """Reading R8: B = floor(2 bytes * (elements of K and V) / C)."""
+    return int(math.floor(2.0 * n_elems_kv / C))
