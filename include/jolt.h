@@ -1,0 +1,238 @@
+/*
+ * jolt.h -- C ABI of the B200 JoLT KV-cache compressor.
+ *
+ * JoLT ("A JoLT for the KV Cache: Near-Lossless KV Cache Compression via
+ * Joint Rank-bit Allocation", Krishnan & Schulz) compresses the prefill KV
+ * cache of every layer group, for keys and values separately (a "cell" is one
+ * (sequence, group, K|V) tensor X of shape [L_g, H, T, D]), with
+ *   1. a partial Tucker decomposition that truncates only the token and the
+ *      feature modes (Section 3, "Partial Tucker backbone"),
+ *   2. a randomly rotated low-bit residual (Section 3, "Rotated low-bit
+ *      residual"),
+ *   3. per-cell ranks and bit-widths chosen jointly for all cells by one
+ *      Lagrange multiplier under a single byte budget (Section 3, Eqs. 1-4),
+ *   4. optionally a randomized token-mode SVD (Section 3.1, "FlashJoLT",
+ *      Eq. 5 for the rank cap).
+ *
+ * Conventions for every entry point:
+ *   * Device pointers are CUDA device (or managed) memory of the current
+ *     device; host pointers are ordinary host memory. Each argument says which.
+ *   * Every call returns a jolt_status; none aborts or exits. On failure
+ *     jolt_last_error() gives a thread-local message.
+ *   * Work is enqueued on the given stream and is asynchronous unless the
+ *     entry point says it synchronises.
+ *   * The library never writes its input caches.
+ *   * Device memory the library needs (handles, workspace) comes from the
+ *     allocator set by jolt_set_allocator (default: cudaMallocAsync /
+ *     cudaFreeAsync on the call's stream).
+ */
+#ifndef JOLT_H
+#define JOLT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define JOLT_API __attribute__((visibility("default")))
+#else
+#define JOLT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* jolt_stream_t;   /* == cudaStream_t */
+
+typedef enum {
+  JOLT_OK = 0,
+  JOLT_ERR_INVALID_ARG = 1,        /* null pointer, bad enum, bad grid value  */
+  JOLT_ERR_UNSUPPORTED_SHAPE = 2,  /* D not 64/128, stride not aligned, ...    */
+  JOLT_ERR_BUDGET_INFEASIBLE = 3,  /* budget below the cheapest allocation     */
+  JOLT_ERR_OOM = 4,                /* the allocator returned NULL              */
+  JOLT_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed        */
+  JOLT_ERR_TIMEOUT = 6,            /* a bounded device wait expired            */
+  JOLT_ERR_NONFINITE = 7           /* a cell's squared norm is not finite      */
+} jolt_status;
+
+enum { JOLT_BF16 = 0, JOLT_F32 = 1 };             /* jolt_layout.dtype        */
+enum { JOLT_EXACT = 0, JOLT_RANDOMIZED = 1 };      /* jolt_options.mode        */
+enum { JOLT_ROT_HADAMARD = 0 };                    /* jolt_options.rotation    */
+
+/*
+ * Where the cache lives. Element (b, l, h, t, d) of K (and of V, same layout)
+ * is at base + b*stride_b + l*stride_l + h*stride_h + t*stride_t + d, strides
+ * in ELEMENTS, d contiguous. Layers [group_start[g], group_start[g+1]) form
+ * group g (contiguous groups, Section 3: "partition the L layers into G
+ * contiguous groups"). rope_theta_k > 0 means the keys were stored after a
+ * rotate-half rotary embedding with that base over positions 0..T-1: keys are
+ * compressed before RoPE and RoPE is re-applied on decompression (Section 3,
+ * "Keys are decomposed before the rotary position embedding").
+ */
+typedef struct {
+  int32_t batch, n_layers, n_heads, seq_len, head_dim;   /* head_dim in {64,128} */
+  int32_t n_groups;
+  const int32_t* group_start;    /* HOST, n_groups+1 entries, 0 .. n_layers    */
+  int32_t dtype;                 /* JOLT_BF16 | JOLT_F32                       */
+  int64_t stride_b, stride_l, stride_h, stride_t;
+  float rope_theta_k;            /* 0: no RoPE handling                        */
+} jolt_layout;
+
+/*
+ * Knobs. jolt_default_options() fills the paper's defaults:
+ *   mode JOLT_EXACT; bits {0,2,4,8} (Section 3, "Rotated low-bit residual");
+ *   rank grids = every integer from 1 (Section 3, "Solving the allocation");
+ *   rt_max 0 (exact: min(T, N); randomized: q_cap of Eq. 5);
+ *   oversample_p 8, power_iters 2 (randomized range finder);
+ *   scale_group 0 (= D: one fp32 scale per row, Eq. 1's 32/d_h term);
+ *   budget_tol 0.005 and max_iters 50 (Section 3: "stopping within 0.5% of
+ *   the target budget or after 50 iterations").
+ * Grids are HOST arrays of strictly increasing values >= 1, copied at plan
+ * time; NULL/0 means "every integer 1..max".
+ */
+typedef struct {
+  int32_t mode;
+  int32_t n_bits;
+  int32_t bits[8];               /* each in {0,2,3,4,8}, strictly increasing   */
+  int32_t n_rt;
+  const int32_t* rt_grid;
+  int32_t n_rd;
+  const int32_t* rd_grid;
+  int32_t rt_max;
+  int32_t oversample_p, power_iters;
+  int32_t scale_group;           /* 0 (= D), 32, 64 or 128; must divide D      */
+  int32_t rotation;              /* JOLT_ROT_HADAMARD                          */
+  double budget_tol;
+  int32_t max_iters;
+} jolt_options;
+
+typedef struct jolt_plan_s jolt_plan_t;
+typedef struct jolt_handle_s jolt_handle_t;
+
+/* Per-cell result of an allocation (one entry per cell, cell order =
+ * sequence, then group, then K before V). */
+typedef struct {
+  int32_t seq, group, kind;      /* kind 0 = K, 1 = V                          */
+  int32_t r_t, r_d, bits;
+  int64_t bytes;                 /* Eq. (1) for this cell                      */
+  double err_model;              /* Eq. (2) surrogate at the chosen point      */
+  double norm_sq;                /* ||X||_F^2 of the cell                      */
+} jolt_cell_info;
+
+/* Device views of one compressed cell (for tests and for consumers that
+ * decode without this library). All pointers are DEVICE pointers owned by
+ * the handle. */
+typedef struct {
+  int32_t r_t, r_d, bits, scale_group;
+  int32_t L, H, T, D, t_pitch;
+  const uint16_t* ut;   /* bf16 U_T^ transposed: [r_t][t_pitch], first T used */
+  const uint16_t* ud;   /* bf16 U_d^: [D][r_d]                                */
+  const uint16_t* core; /* bf16 G^: [L][H][r_t][r_d]                          */
+  const uint8_t* codes; /* [L][H][T][bits*D/8], NULL when bits == 0           */
+  const float* scales;  /* [L][H][T][D/scale_group], NULL when bits == 0      */
+} jolt_cell_view;
+
+JOLT_API void jolt_default_options(jolt_options* opt);
+
+/* Checks layout, budget and options, derives the cells, the rank grids and
+ * the Eq. (5) cap, and sizes the workspace. byte_budget B is the target of
+ * Eq. (3) for ALL cells together. Synchronises the legacy default stream once
+ * (ε² calibration, Section 3 text under Eq. 2). Returns
+ * JOLT_ERR_BUDGET_INFEASIBLE when B is below the sum of every cell's cheapest
+ * option, JOLT_ERR_UNSUPPORTED_SHAPE for D not in {64,128}, strides not
+ * multiples of 8 elements or a mode/shape pair the kernels do not cover. */
+JOLT_API jolt_status jolt_plan(const jolt_layout* layout, int64_t byte_budget,
+                      const jolt_options* opt, jolt_plan_t** out);
+JOLT_API void jolt_free_plan(jolt_plan_t* plan);
+
+/* Compress K and V (DEVICE pointers, layout of the plan) under byte_budget
+ * (<= 0: the plan's budget). seed selects the residual rotation and, in
+ * randomized mode, the Gaussian sketch (sequence b uses seed + b). The handle
+ * owns every compressed buffer. Asynchronous; the handle is usable by later
+ * work on the same stream. */
+JOLT_API jolt_status jolt_compress(jolt_plan_t* plan, const void* k, const void* v,
+                          int64_t byte_budget, uint64_t seed,
+                          jolt_stream_t stream, jolt_handle_t** out);
+
+/* Decompress into k_out / v_out (DEVICE, bf16, layout out_layout; NULL means
+ * the plan's layout with dtype bf16). Section 3: "Decoding inverts the
+ * rotation and adds the dequantized residual to the low-rank reconstruction";
+ * keys get RoPE re-applied. Asynchronous. */
+JOLT_API jolt_status jolt_decompress(const jolt_handle_t* h, void* k_out, void* v_out,
+                            const jolt_layout* out_layout, jolt_stream_t stream);
+
+/* Sum over cells of Eq. (1) at the chosen (r_T, r_d, b): the compressed size
+ * in bytes. Synchronises the handle's stream. */
+JOLT_API jolt_status jolt_bytes(const jolt_handle_t* h, int64_t* payload_bytes);
+
+/* Per-cell allocation (n >= number of cells) and the multiplier lambda of
+ * Eq. (4). HOST outputs. Synchronises the handle's stream. */
+JOLT_API jolt_status jolt_handle_info(const jolt_handle_t* h, jolt_cell_info* cells,
+                             int32_t n, double* lambda, int32_t* iterations);
+JOLT_API jolt_status jolt_handle_cell(const jolt_handle_t* h, int32_t cell,
+                             jolt_cell_view* view);
+JOLT_API int32_t jolt_num_cells(const jolt_plan_t* plan);
+JOLT_API void jolt_free_handle(jolt_handle_t* h);
+
+/* Rate-distortion inputs of every cell (Section 3, Eq. 2: the unprojected
+ * mode spectra and ||X||^2), computed on the device by the plan's mode.
+ * HOST outputs: norm_sq[n_cells]; sig_t[n_cells * n_t] (descending squared
+ * token singular values; in randomized mode the q_cap computed values
+ * followed by the synthetic tail entry of Section 3.1); sig_d[n_cells * D].
+ * n_t is written to *n_t (<= max_t). Synchronises the stream. */
+JOLT_API jolt_status jolt_rd_table(jolt_plan_t* plan, const void* k, const void* v,
+                          double* norm_sq, double* sig_t, int32_t max_t,
+                          int32_t* n_t, double* sig_d, jolt_stream_t stream);
+
+/* The allocator of Eqs. (3)-(4) alone, on the device, from HOST rate-distortion
+ * inputs: for cell c, t_t[c*ld_t + r] (r = 0..n_t) and t_d[c*ld_d + r]
+ * (r = 0..D) are the tail fractions (discarded energy / ||X||^2 at rank r),
+ * eps2[n_bits] the calibration of Eq. (2). Uses the plan's grids, shapes and
+ * bit list. HOST outputs: choice[3*c] = (r_t, r_d, bits), bytes[c], and
+ * lambda. Synchronises the stream. */
+JOLT_API jolt_status jolt_allocate(jolt_plan_t* plan, const double* t_t, int32_t ld_t,
+                          const double* t_d, int32_t ld_d, const double* eps2,
+                          int64_t byte_budget, int32_t* choice, int64_t* bytes,
+                          double* lambda, int32_t* iterations,
+                          jolt_stream_t stream);
+
+/* ε²(b) calibration of Section 3 (text under Eq. 2): the fraction of a
+ * Gaussian's energy the b-bit quantizer with groups of `group` values fails
+ * to recover, over 2^20 Philox4x32-10 / Box-Muller samples rounded to fp32.
+ * HOST output eps2[n]. Synchronises the stream. */
+JOLT_API jolt_status jolt_eps2(const int32_t* bits, int32_t n, int32_t group,
+                      double* eps2, jolt_stream_t stream);
+
+/* The residual stage alone (Section 3, "Rotated low-bit residual"), for
+ * rows of D fp32 values: r = D^-1/2 H_D diag(s) e with s from `seed`, then
+ * absmax quantization to `bits` with one fp32 scale per `group` values and
+ * LSB-first packing. DEVICE in/out: e[rows][D]; codes[rows][bits*D/8];
+ * scales[rows][D/group]. */
+JOLT_API jolt_status jolt_residual_encode(const float* e, int64_t rows, int32_t D,
+                                 int32_t bits, int32_t group, uint64_t seed,
+                                 uint8_t* codes, float* scales,
+                                 jolt_stream_t stream);
+/* Inverse: e_hat = diag(s) D^-1/2 H_D dequant(codes). DEVICE in/out. */
+JOLT_API jolt_status jolt_residual_decode(const uint8_t* codes, const float* scales,
+                                 int64_t rows, int32_t D, int32_t bits,
+                                 int32_t group, uint64_t seed, float* e_hat,
+                                 jolt_stream_t stream);
+
+/* Device allocator used for handles and workspace. alloc returns NULL on
+ * failure (-> JOLT_ERR_OOM). Passing NULLs restores the default. */
+typedef void* (*jolt_alloc_fn)(size_t bytes, jolt_stream_t stream, void* ctx);
+typedef void (*jolt_free_fn)(void* ptr, jolt_stream_t stream, void* ctx);
+JOLT_API jolt_status jolt_set_allocator(jolt_alloc_fn alloc, jolt_free_fn free_fn,
+                               void* ctx);
+
+/* Thread-local description of the last failure on this thread. */
+JOLT_API const char* jolt_last_error(void);
+
+/* Number of kernels this library has launched in this process (for
+ * launch-count reporting). */
+JOLT_API uint64_t jolt_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* JOLT_H */

@@ -605,9 +605,13 @@ def build_table(X: np.ndarray, opt: Options, eps2: Dict[int, float]) -> Tuple[Ce
     normsq = float(np.sum(X * X))
     sT, UT = token_spectrum(X)
     sD = feature_spectrum(X)
-    rmax = opt.rt_max or min(T, Lg * H * D)
-    rt = np.array(opt.rt_grid if opt.rt_grid else range(1, rmax + 1), dtype=np.int64)
-    rd = np.array(opt.rd_grid if opt.rd_grid else range(1, D + 1), dtype=np.int64)
+    # a token rank cannot exceed min(T, N) (nor rt_max when given), a feature
+    # rank cannot exceed D: grid values beyond those bounds are dropped
+    rmax = min(T, Lg * H * D)
+    if opt.rt_max:
+        rmax = min(rmax, opt.rt_max)
+    rt = np.array([r for r in (opt.rt_grid or range(1, rmax + 1)) if r <= rmax], dtype=np.int64)
+    rd = np.array([r for r in (opt.rd_grid or range(1, D + 1)) if r <= D], dtype=np.int64)
     tab = CellTable(Lg, H, T, D, g, normsq, tail_fractions(sT, normsq), tail_fractions(sD, normsq),
                     rt, rd, np.array(opt.bits, dtype=np.int64),
                     np.array([eps2[b] for b in opt.bits], dtype=np.float64))

@@ -1,0 +1,59 @@
+"""The C-ABI library loads on a machine without a GPU and exports every
+function include/jolt.h declares; host-side argument checks answer with
+status codes (no kernel runs)."""
+import ctypes as C
+
+import pytest
+
+from tucker_quantized_residual_b200 import jolt
+
+
+def test_library_exports_every_declared_symbol():
+    lib = jolt.load_library()
+    names = jolt.header_symbols()
+    assert len(names) >= 16
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(jolt._SIGS), "binding and header disagree"
+
+
+def test_default_options_are_the_papers():
+    o, _ = jolt.make_options()
+    assert list(o.bits[: o.n_bits]) == [0, 2, 4, 8]
+    assert o.budget_tol == 0.005 and o.max_iters == 50
+    assert o.oversample_p == 8 and o.power_iters == 2 and o.scale_group == 0
+
+
+def _layout(D=64, theta=0.0, groups=(0, 2)):
+    gs = (C.c_int32 * len(groups))(*groups)
+    L = jolt.jolt_layout(1, groups[-1], 2, 256, D, len(groups) - 1, C.cast(gs, C.POINTER(C.c_int32)),
+                         jolt.JOLT_F32, groups[-1] * 2 * 256 * D, 2 * 256 * D, 256 * D, D, theta)
+    return L, gs
+
+
+@pytest.mark.parametrize("bad", ["D", "bits", "group", "grid", "groups"])
+def test_plan_rejects_bad_arguments_before_touching_the_device(bad):
+    L, keep = _layout()
+    o, k2 = jolt.make_options()
+    if bad == "D":
+        L.head_dim = 96
+    elif bad == "bits":
+        o.bits[1] = 5
+    elif bad == "group":
+        o.scale_group = 48
+    elif bad == "grid":
+        o, k2 = jolt.make_options(rt_grid=[4, 2])
+    elif bad == "groups":
+        L, keep = _layout(groups=(0, 1))
+        L.n_layers = 2
+    with pytest.raises(jolt.JoltError) as ei:
+        jolt.jolt_plan(L, 10 ** 6, o)
+    assert ei.value.status in (1, 2)
+
+
+def test_plan_rejects_infeasible_budget():
+    L, keep = _layout()
+    o, k2 = jolt.make_options()
+    with pytest.raises(jolt.JoltError) as ei:
+        jolt.jolt_plan(L, 100, o)
+    assert ei.value.status == 3

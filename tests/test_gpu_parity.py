@@ -1,0 +1,250 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on the same
+seeded inputs. Bars:
+  * eps^2 calibration, spectra: relative 1e-12 / 1e-10 (fp64 sums, other order);
+  * residual codes, scales and packed bytes: bit-exact when fed the oracle's
+    residual; decoding bit-exact;
+  * allocation fed the oracle's rate-distortion tables: bit-exact choices,
+    bytes, lambda and iteration count;
+  * exact-mode reconstruction: relative Frobenius distance to the oracle's
+    reconstruction <= 1e-4, the same allocation, the same byte count.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import jolt_oracle as o
+from tucker_quantized_residual_b200 import jolt, synth
+
+from gpu_helpers import gpu_compress, oracle_compress
+
+pytestmark = pytest.mark.gpu
+
+RTOL_RECON = 1e-4
+
+
+def rel(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return math.sqrt(float(np.sum((a - b) ** 2)) / max(float(np.sum(b * b)), 1e-300))
+
+
+# ------------------------------------------------------------ calibration
+@pytest.mark.parametrize("g", [64, 128])
+def test_eps2_calibration_matches_oracle(g):
+    bits = (0, 2, 3, 4, 8)
+    gpu = jolt.jolt_eps2(bits, g)
+    ref = o.eps2_table(bits, g)
+    for b, x in zip(bits, gpu):
+        assert abs(x - ref[b]) <= 1e-12 * ref[b], (b, x, ref[b])
+
+
+# --------------------------------------------------------- residual stage
+def _oracle_residual_rows(D):
+    """The oracle's own residual of the tiny cache at (16, 16) plus rows that
+    hit the quantizer's edges: zeros, exact ties, huge and tiny scales."""
+    spec = synth.SPECS["tiny"]
+    K, V = synth.make_cache(spec, 0)
+    X = V.numpy()[0, 0:2].astype(np.float64)
+    w, U = o.token_spectrum(X)
+    f = o.fit(X, U, 16, 16)
+    E = o.residual_from(X, o.backbone(f)).reshape(-1, 64)
+    if D == 128:
+        E = E.reshape(-1, 128)
+    rng = np.random.default_rng(5)
+    extra = (rng.standard_normal((300, D)) * np.exp(rng.uniform(-30, 30, (300, 1)))).astype(np.float32)
+    extra[0] = 0.0
+    extra[1] = np.arange(D, dtype=np.float32) - D / 2          # many exact .5 quotients
+    extra[2, :] = 0.0
+    extra[2, 3] = -1e-30
+    return np.concatenate([E, extra]).astype(np.float32)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("b", [2, 3, 4, 8])
+@pytest.mark.parametrize("g", [32, 64, 128])
+def test_residual_codes_bit_exact_on_oracle_residual(D, b, g):
+    if g > D:
+        pytest.skip("group larger than D")
+    E = _oracle_residual_rows(D)
+    rows = E.shape[0]
+    seed = 1234
+    sg = o.hadamard_signs(D, seed)
+    ref = o.encode_residual(E, b, g, sg)
+    e_dev = torch.from_numpy(E).cuda()
+    codes = torch.zeros(rows, b * D // 8, dtype=torch.uint8, device="cuda")
+    scales = torch.zeros(rows, D // g, dtype=torch.float32, device="cuda")
+    jolt.jolt_residual_encode(e_dev, D, b, g, seed, codes, scales)
+    torch.cuda.synchronize()
+    assert np.array_equal(codes.cpu().numpy(), ref.packed)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ref.scales.view(np.uint32))
+    # decoding the oracle's payload
+    out = torch.empty(rows, D, dtype=torch.float32, device="cuda")
+    jolt.jolt_residual_decode(torch.from_numpy(ref.packed).cuda(), torch.from_numpy(ref.scales).cuda(),
+                              rows, D, b, g, seed, out)
+    torch.cuda.synchronize()
+    dec = o.decode_residual(ref, g, sg, D)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), dec.view(np.uint32))
+
+
+def test_residual_zero_rows_and_empty_call():
+    e = torch.zeros(0, 128, device="cuda")
+    codes = torch.zeros(0, 64, dtype=torch.uint8, device="cuda")
+    scales = torch.zeros(0, 1, device="cuda")
+    jolt.jolt_residual_encode(e, 128, 4, 128, 0, codes, scales)   # no rows: no launch, OK
+    with pytest.raises(jolt.JoltError):
+        jolt.jolt_residual_encode(e, 96, 4, 32, 0, codes, scales)
+
+
+# --------------------------------------------------------------- allocation
+def _synthetic_tables(nc, T, D, Lg, H, seed):
+    """Decaying spectra per cell (any tables exercise the allocator)."""
+    rng = np.random.default_rng(seed)
+    tabs = []
+    n = min(T, Lg * H * D)
+    for c in range(nc):
+        a = rng.uniform(0.6, 1.2)
+        sT = np.arange(1, n + 1, dtype=np.float64) ** (-2 * a) * rng.uniform(0.5, 1.5, n)
+        sD = np.arange(1, D + 1, dtype=np.float64) ** (-2 * a) * rng.uniform(0.5, 1.5, D)
+        sT = np.sort(sT)[::-1]
+        sD = np.sort(sD)[::-1]
+        ns = float(sT.sum()) * rng.uniform(1.0, 1.05)
+        sD *= ns / sD.sum()
+        tabs.append((ns, sT, sD))
+    return tabs
+
+
+def _plan_for(T, D, Lg, H, ngroups, budget, **kw):
+    shape = (1, Lg * ngroups, H, T, D)
+    x = torch.empty(0)
+    gs = [i * Lg for i in range(ngroups + 1)]
+    import ctypes as C
+    arr = (C.c_int32 * len(gs))(*gs)
+    lay = jolt.jolt_layout(1, Lg * ngroups, H, T, D, ngroups, C.cast(arr, C.POINTER(C.c_int32)),
+                           jolt.JOLT_BF16, Lg * ngroups * H * T * D, H * T * D, T * D, D, 0.0)
+    opt, keep = jolt.make_options(**kw)
+    return jolt.jolt_plan(lay, budget, opt), (arr, keep)
+
+
+@pytest.mark.parametrize("C_ratio", [1.5, 2.0, 3.0, 4.0, 8.0])
+def test_allocation_bit_exact_on_oracle_tables(C_ratio):
+    T, D, Lg, H, ng = 1024, 128, 4, 8, 8
+    raw = _synthetic_tables(2 * ng, T, D, Lg, H, seed=int(C_ratio * 10))
+    dense = 2 * 2 * ng * Lg * H * T * D
+    B = int(dense // C_ratio)
+    plan, keep = _plan_for(T, D, Lg, H, ng, B)
+    try:
+        eps = o.eps2_table((0, 2, 4, 8), D)
+        tabs = []
+        for ns, sT, sD in raw:
+            tabs.append(o.CellTable(Lg, H, T, D, D, ns, o.tail_fractions(sT, ns), o.tail_fractions(sD, ns),
+                                    np.arange(1, min(T, Lg * H * D) + 1), np.arange(1, D + 1),
+                                    np.array([0, 2, 4, 8]), np.array([eps[b] for b in (0, 2, 4, 8)])))
+        ref = o.allocate(tabs, B)
+        ch, by, lam, it = jolt.jolt_allocate(plan, [t.tT for t in tabs], [t.tD for t in tabs],
+                                             [eps[b] for b in (0, 2, 4, 8)], B)
+        assert ch == ref.choice
+        assert by == ref.bytes
+        assert lam == ref.lam and it == ref.iters
+    finally:
+        jolt.jolt_free_plan(plan)
+
+
+def test_allocation_tiny_grid_bit_exact():
+    spec = synth.SPECS["tiny"]
+    K, V = synth.make_cache(spec, 0)
+    opt = o.Options(bits=(0, 2, 3, 4, 8), rt_grid=(8, 16, 32, 64), rd_grid=(16, 32, 48))
+    eps = o.eps2_table(opt.bits, 64)
+    tabs = [o.build_table(src.numpy()[0, 0:2].astype(np.float64), opt, eps)[0] for src in (K, V)]
+    for C_ratio in (2.0, 3.0):
+        B = o.budget_for_ratio(2 * 256 * 64 * 2 * 2 // 2, C_ratio)
+        plan, keep = _plan_for(256, 64, 2, 2, 1, B, bits=opt.bits, rt_grid=opt.rt_grid, rd_grid=opt.rd_grid)
+        try:
+            ref = o.allocate(tabs, B)
+            ch, by, lam, it = jolt.jolt_allocate(plan, [t.tT for t in tabs], [t.tD for t in tabs],
+                                                 [eps[b] for b in opt.bits], B)
+            assert ch == ref.choice and by == ref.bytes and lam == ref.lam and it == ref.iters
+        finally:
+            jolt.jolt_free_plan(plan)
+
+
+# ----------------------------------------------------------------- spectra
+@pytest.mark.parametrize("name", ["tiny", "mistral"])
+def test_rd_spectra_match_oracle(name):
+    spec = synth.SPECS[name]
+    K, V = synth.make_cache(spec, 0)
+    gs = synth.group_starts(spec)
+    Kd, Vd = K.cuda(), V.cuda()
+    lay, keep = jolt.make_layout(Kd, gs, spec.rope_theta_k)
+    opt, k2 = jolt.make_options()
+    plan = jolt.jolt_plan(lay, 10 ** 12, opt)
+    try:
+        n = jolt.jolt_num_cells(plan)
+        nmin = min(spec.seq_len, spec.group_size * spec.n_heads * spec.head_dim)
+        ns, st, nt, sd = jolt.jolt_rd_table(plan, Kd, Vd, n, nmin, spec.head_dim)
+        refs = o.cells_of(1, gs)
+        for i, c in enumerate(refs[: min(n, 4)]):
+            X = o.cell_tensor(K.float().numpy(), V.float().numpy(), c, spec.rope_theta_k)
+            assert abs(ns[i] - float(np.sum(X * X))) <= 1e-12 * ns[i]
+            wT, _ = o.token_spectrum(X)
+            wD = o.feature_spectrum(X)
+            assert np.max(np.abs(np.array(st[i][:nt]) - wT[:nt])) <= 1e-10 * wT[0]
+            assert np.max(np.abs(np.array(sd[i]) - wD)) <= 1e-10 * wD[0]
+    finally:
+        jolt.jolt_free_plan(plan)
+
+
+# ------------------------------------------------------------- end to end
+def _compare(K, V, gs, B, rope=0.0, **kw):
+    Kh, Vh, cells, lam, it, nbytes = gpu_compress(K, V, gs, B, 0, rope, **kw)
+    Kn, Vn, Ko, Vo, comp = oracle_compress(K, V, gs, B, 0, rope, **kw)
+    got = [(c.r_t, c.r_d, c.bits) for c in cells]
+    assert got == comp.alloc.choice
+    assert nbytes == sum(comp.alloc.bytes) and nbytes <= B
+    assert lam == comp.alloc.lam and it == comp.alloc.iters
+    assert rel(Kh, Ko) <= RTOL_RECON, rel(Kh, Ko)
+    assert rel(Vh, Vo) <= RTOL_RECON, rel(Vh, Vo)
+    eK, eV = o.rel_frobenius(Kn, Kh), o.rel_frobenius(Vn, Vh)
+    rK, rV = o.rel_frobenius(Kn, Ko), o.rel_frobenius(Vn, Vo)
+    assert abs(eK - rK) <= 1e-4 and abs(eV - rV) <= 1e-4
+    return eK, eV
+
+
+def test_tiny_fixed_ranks():
+    spec = synth.SPECS["tiny"]
+    K, V = synth.make_cache(spec, 0)
+    _compare(K, V, [0, 2], 10 ** 9, bits=(4,), rt_grid=(32,), rd_grid=(32,))
+
+
+@pytest.mark.parametrize("C_ratio", [2.0, 3.0])
+def test_tiny_lagrangian_sweep(C_ratio):
+    spec = synth.SPECS["tiny"]
+    K, V = synth.make_cache(spec, 0)
+    B = o.budget_for_ratio(K.numel() * 2, C_ratio)
+    _compare(K, V, [0, 2], B, bits=(0, 2, 3, 4, 8), rt_grid=(8, 16, 32, 64), rd_grid=(16, 32, 48))
+
+
+@pytest.mark.parametrize("C_ratio", [2.0, 3.0])
+def test_mistral_exact(C_ratio):
+    spec = synth.SPECS["mistral"]
+    K, V = synth.make_cache(spec, 0)
+    B = o.budget_for_ratio(K.numel() * 2, C_ratio)
+    eK, eV = _compare(K, V, synth.group_starts(spec), B, spec.rope_theta_k)
+    assert eK < 0.05 and eV < 0.05
+
+
+@pytest.mark.parametrize("dtype,D,T,rope", [("f32", 64, 200, 1e4), ("bf16", 128, 136, 1e6),
+                                            ("bf16", 64, 72, 0.0), ("bf16", 64, 300, 1e4)])
+def test_ragged_and_small_shapes(dtype, D, T, rope):
+    spec = synth.CacheSpec("ragged", 1, 3, 2, T, D, 2, 8, 1.0, 0.02, rope_theta_k=rope, dtype=dtype)
+    K, V = synth.make_cache(spec, 3)
+    gs = synth.group_starts(spec)          # groups of 2 and 1 layers
+    B = o.budget_for_ratio(K.numel() * 2, 2.5)
+    _compare(K, V, gs, B, rope, bits=(0, 2, 3, 4, 8), scale_group=32)
+
+
+def test_all_zero_bits_and_generous_budget():
+    spec = synth.SPECS["tiny"]
+    K, V = synth.make_cache(spec, 1)
+    _compare(K, V, [0, 2], 10 ** 9, bits=(0,), rt_grid=(8, 64), rd_grid=(16, 64))

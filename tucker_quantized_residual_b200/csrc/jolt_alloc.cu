@@ -1,0 +1,297 @@
+// Rate-distortion tables and the Lagrangian allocator on the device.
+//
+// "A JoLT for the KV Cache", Section 3:
+//  * Eq. (1): s(r_T, r_d, b) = (|g| n_h r_T r_d + T r_T + d_h r_d) c
+//             + [b>0] (b + 32/g_q)/8 |g| n_h T d_h, c = 2 (bf16);
+//  * Eq. (2): e(r_T, r_d, b) = eps^2(b) tau(r_T, r_d), tau = discarded
+//             token-mode + feature-mode mass of the unprojected spectra,
+//             divided by ||X||^2;
+//  * Eqs. (3)-(4): min sum e s.t. sum s <= B through L(lambda) = sum(e + lambda s),
+//             every cell minimised independently (here by exhaustive, segmented
+//             argmin over the grid), lambda found by geometric bisection that
+//             stops within the tolerance of B or after max_iters.
+//  * eps^2(b): the fraction of a Gaussian's energy the b-bit rotated quantizer
+//             fails to recover, calibrated once on a Gaussian round trip.
+#include "jolt_internal.cuh"
+#include "jolt_kernels.cuh"
+
+namespace jolt {
+
+// ------------------------------------------------------- eps^2 calibration --
+constexpr int CALIB_SAMPLES = 1 << 20;
+
+template <int G>
+__global__ void __launch_bounds__(256) k_eps2(int nb, int4 bits_lo, int4 bits_hi, double* partial) {
+  const int grp = blockIdx.x * blockDim.x + threadIdx.x;     // one group of G samples
+  const int ngrp = CALIB_SAMPLES / G;
+  int bl[8] = {bits_lo.x, bits_lo.y, bits_lo.z, bits_lo.w, bits_hi.x, bits_hi.y, bits_hi.z, bits_hi.w};
+  double err[8], en = 0.0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) err[i] = 0.0;
+  if (grp < ngrp) {
+    float x[G];
+#pragma unroll 1
+    for (int m = 0; m < G / 4; ++m) {
+      u4 w = philox_at(0ull, STREAM_CALIB, (uint32_t)(grp * (G / 4) + m));
+      double u0 = ((double)w.x + 0.5) * 0x1p-32, u1 = ((double)w.y + 0.5) * 0x1p-32;
+      double u2 = ((double)w.z + 0.5) * 0x1p-32, u3 = ((double)w.w + 0.5) * 0x1p-32;
+      double r0 = sqrt(-2.0 * log(u0)), r1 = sqrt(-2.0 * log(u2));
+      double t0 = (2.0 * 3.141592653589793) * u1, t1 = (2.0 * 3.141592653589793) * u3;
+      x[4 * m + 0] = (float)(r0 * cos(t0));
+      x[4 * m + 1] = (float)(r0 * sin(t0));
+      x[4 * m + 2] = (float)(r1 * cos(t1));
+      x[4 * m + 3] = (float)(r1 * sin(t1));
+    }
+    float a = 0.0f;
+    for (int j = 0; j < G; ++j) {
+      a = fmaxf(a, fabsf(x[j]));
+      en += (double)x[j] * (double)x[j];
+    }
+    for (int bi = 0; bi < nb; ++bi) {
+      int b = bl[bi];
+      if (b == 0) continue;
+      float qm = (float)qmax_of(b);
+      float sc = __fdiv_rn(a, qm);
+      double acc = 0.0;
+      for (int j = 0; j < G; ++j) {
+        float q = 0.0f;
+        if (sc > 0.0f) q = fminf(fmaxf(rintf(__fdiv_rn(x[j], sc)), -qm), qm);
+        float xh = __fmul_rn(q, sc);
+        double d = (double)x[j] - (double)xh;
+        acc += d * d;
+      }
+      err[bi] = acc;
+    }
+  }
+  // block reduction in a fixed order
+  __shared__ double red[9][256];
+  for (int i = 0; i < 8; ++i) red[i][threadIdx.x] = err[i];
+  red[8][threadIdx.x] = en;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o)
+      for (int i = 0; i < 9; ++i) red[i][threadIdx.x] += red[i][threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x < 9) partial[blockIdx.x * 9 + threadIdx.x] = red[threadIdx.x][0];
+}
+
+__global__ void k_eps2_final(const double* partial, int nblk, int nb, int4 bits_lo, int4 bits_hi,
+                             double* eps2) {
+  int bl[8] = {bits_lo.x, bits_lo.y, bits_lo.z, bits_lo.w, bits_hi.x, bits_hi.y, bits_hi.z, bits_hi.w};
+  if (threadIdx.x != 0) return;
+  double en = 0.0;
+  for (int k = 0; k < nblk; ++k) en += partial[k * 9 + 8];
+  for (int bi = 0; bi < nb; ++bi) {
+    double e = 0.0;
+    for (int k = 0; k < nblk; ++k) e += partial[k * 9 + bi];
+    eps2[bi] = (bl[bi] == 0) ? 1.0 : e / en;
+  }
+}
+
+jolt_status launch_eps2(const int* bits_host, int nb, int G, double* eps2_dev, double* scratch,
+                        cudaStream_t s) {
+  int b[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int i = 0; i < nb && i < 8; ++i) b[i] = bits_host[i];
+  int4 lo = make_int4(b[0], b[1], b[2], b[3]), hi = make_int4(b[4], b[5], b[6], b[7]);
+  int ngrp = CALIB_SAMPLES / G;
+  int nblk = (ngrp + 255) / 256;
+  switch (G) {
+    case 32: k_eps2<32><<<nblk, 256, 0, s>>>(nb, lo, hi, scratch); break;
+    case 64: k_eps2<64><<<nblk, 256, 0, s>>>(nb, lo, hi, scratch); break;
+    case 128: k_eps2<128><<<nblk, 256, 0, s>>>(nb, lo, hi, scratch); break;
+    default: set_error("unsupported scale group %d", G); return JOLT_ERR_INVALID_ARG;
+  }
+  JOLT_LAUNCHED();
+  k_eps2_final<<<1, 32, 0, s>>>(scratch, nblk, nb, lo, hi, eps2_dev);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// ------------------------------------------------------ tail fractions -----
+// t[r] = sum_{i >= r} w_i / ||X||^2 (r = 0..n), summed smallest first, with
+// negative rounding noise in w clamped to 0. One thread per cell and table.
+__global__ void k_rd_tables(const CellRD* __restrict__ cells, int ncells,
+                            const double* const* __restrict__ wT, const double* const* __restrict__ wD,
+                            const double* const* __restrict__ normsq_in,
+                            double* const* __restrict__ tT, double* const* __restrict__ tD,
+                            const int* __restrict__ nt_used, int* status) {
+  int job = blockIdx.x * blockDim.x + threadIdx.x;
+  if (job >= 2 * ncells) return;
+  int c = job >> 1;
+  double ns = *normsq_in[c];
+  if (!isfinite(ns) || ns <= 0.0) {
+    if (!isfinite(ns)) atomicOr(status, DEV_ERR_NONFINITE);
+    ns = 1.0;
+  }
+  const double* w;
+  double* t;
+  int n;
+  if (job & 1) { w = wD[c]; t = tD[c]; n = cells[c].D; }
+  else { w = wT[c]; t = tT[c]; n = nt_used[c]; }
+  double acc = 0.0;
+  t[n] = 0.0;
+  for (int i = n - 1; i >= 0; --i) {
+    acc += fmax(w[i], 0.0);
+    t[i] = acc / ns;
+  }
+  t[n] = 0.0;
+}
+
+jolt_status launch_rd_tables(const CellRD* cells, int ncells, const double* const* wT,
+                             const double* const* wD, const double* /*unused*/,
+                             double* const* tT, double* const* tD, const int* nt_used,
+                             const double* const* normsq_in, int* status, cudaStream_t s) {
+  int n = 2 * ncells;
+  k_rd_tables<<<(n + 127) / 128, 128, 0, s>>>(cells, ncells, wT, wD, normsq_in, tT, tD, nt_used, status);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// ------------------------------------------------------------ allocation ----
+__device__ __forceinline__ void decode_opt(const AllocArgs& a, const CellRD& c, int idx, int& bi,
+                                           int& rt, int& rd) {
+  int per_b = c.n_rt * a.n_rd;
+  bi = idx / per_b;
+  int rem = idx - bi * per_b;
+  int ti = rem / a.n_rd;
+  int di = rem - ti * a.n_rd;
+  rt = a.rt_grid[ti];
+  rd = a.rd_grid[di];
+}
+
+__device__ __forceinline__ int64_t opt_bytes(const AllocArgs& a, const CellRD& c, int bi, int rt, int rd) {
+  const int64_t LH = (int64_t)c.Lg * c.H;
+  return 2 * (LH * rt * rd + (int64_t)c.T * rt + (int64_t)c.D * rd) + a.rowbytes[bi] * LH * c.T;
+}
+
+__device__ __forceinline__ double opt_err(const AllocArgs& a, const CellRD& c, int bi, int rt, int rd) {
+  return __dmul_rn(a.eps2[bi], __dadd_rn(c.tT[rt], c.tD[rd]));
+}
+
+__global__ void __launch_bounds__(256) k_alloc_eval(AllocArgs a) {
+  if (a.st->phase == 3) return;
+  const int cell = blockIdx.y;
+  const CellRD c = a.cells[cell];
+  const double lam = a.st->lam;
+  const int nopt = a.n_bits * c.n_rt * a.n_rd;
+  const int per = (nopt + a.nchunk - 1) / a.nchunk;
+  const int i0 = blockIdx.x * per, i1 = min(nopt, i0 + per);
+  double best = INFINITY;
+  int bidx = 0x7fffffff;
+  for (int idx = i0 + threadIdx.x; idx < i1; idx += blockDim.x) {
+    int bi, rt, rd;
+    decode_opt(a, c, idx, bi, rt, rd);
+    double e = opt_err(a, c, bi, rt, rd);
+    double v = __dadd_rn(e, __dmul_rn(lam, (double)opt_bytes(a, c, bi, rt, rd)));
+    if (v < best) { best = v; bidx = idx; }   // ascending idx per thread: first min kept
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    double ob = __shfl_xor_sync(0xffffffffu, best, o);
+    int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+    if (ob < best || (ob == best && oi < bidx)) { best = ob; bidx = oi; }
+  }
+  __shared__ double sv[8];
+  __shared__ int si[8];
+  if ((threadIdx.x & 31) == 0) { sv[threadIdx.x >> 5] = best; si[threadIdx.x >> 5] = bidx; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
+      if (sv[w] < best || (sv[w] == best && si[w] < bidx)) { best = sv[w]; bidx = si[w]; }
+    a.pv[cell * a.nchunk + blockIdx.x] = best;
+    a.pi[cell * a.nchunk + blockIdx.x] = bidx;
+  }
+}
+
+// One block: per-cell argmin over chunks, total bytes, one bisection step.
+__global__ void __launch_bounds__(512) k_alloc_decide(AllocArgs a) {
+  AllocState* st = a.st;
+  if (st->phase == 3) return;
+  __shared__ long long sbytes[512];
+  __shared__ int action;     // 0 none, 1 keep<-cur, 2 finish with cur, 3 finish with keep
+  long long mine = 0;
+  for (int c = threadIdx.x; c < a.ncells; c += blockDim.x) {
+    double best = INFINITY;
+    int bidx = 0x7fffffff;
+    for (int k = 0; k < a.nchunk; ++k) {
+      double v = a.pv[c * a.nchunk + k];
+      int i = a.pi[c * a.nchunk + k];
+      if (v < best || (v == best && i < bidx)) { best = v; bidx = i; }
+    }
+    a.cur[c] = bidx;
+    int bi, rt, rd;
+    decode_opt(a, a.cells[c], bidx, bi, rt, rd);
+    mine += opt_bytes(a, a.cells[c], bi, rt, rd);
+  }
+  sbytes[threadIdx.x] = mine;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long S = 0;
+    for (int i = 0; i < (int)blockDim.x; ++i) S += sbytes[i];
+    st->S = S;
+    const long long B = st->budget;
+    int act = 0;
+    if (st->phase == 0) {
+      if (S <= B) { act = 2; st->lam_final = st->lam; st->iters_final = 0; st->phase = 3; }
+      else { st->phase = 1; st->lam = st->hi; }
+    } else if (st->phase == 1) {
+      if (S > B) { atomicOr(a.status, DEV_ERR_INFEASIBLE); act = 2; st->lam_final = st->lam; st->iters_final = 0; st->phase = 3; }
+      else { act = 1; st->iter = 1; st->phase = 2; st->lam = sqrt(st->lo * st->hi); }
+    } else {
+      const double lo_ok = (1.0 - st->tol) * (double)B;
+      if ((double)S >= lo_ok && S <= B) {
+        act = 2; st->lam_final = st->lam; st->iters_final = st->iter; st->phase = 3;
+      } else {
+        if (S > B) st->lo = st->lam;
+        else { st->hi = st->lam; act = 1; }
+        if (st->iter >= st->max_iters) {
+          act = (act == 1) ? 4 : 3;   // 4: keep<-cur then finish with keep
+          st->lam_final = st->hi; st->iters_final = st->max_iters; st->phase = 3;
+        } else {
+          st->iter += 1;
+          st->lam = sqrt(st->lo * st->hi);
+        }
+      }
+    }
+    action = act;
+  }
+  __syncthreads();
+  const int act = action;
+  for (int c = threadIdx.x; c < a.ncells; c += blockDim.x) {
+    if (act == 1 || act == 4) a.keep[c] = a.cur[c];
+    if (act >= 2) {
+      int idx = (act == 2) ? a.cur[c] : a.keep[c];
+      const CellRD cc = a.cells[c];
+      int bi, rt, rd;
+      decode_opt(a, cc, idx, bi, rt, rd);
+      Choice ch;
+      ch.rT = rt; ch.rd = rd; ch.b = a.bits[bi]; ch.pad = 0;
+      ch.bytes = opt_bytes(a, cc, bi, rt, rd);
+      ch.err = opt_err(a, cc, bi, rt, rd);
+      a.out[c] = ch;
+    }
+  }
+}
+
+__global__ void k_alloc_init(AllocState* st, AllocState init) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) *st = init;
+}
+
+// Writes the initial state (phase 0, lambda = lo), then rounds of
+// evaluate + decide; each round tries one multiplier and rounds after the
+// decision return at once.
+jolt_status launch_alloc(const AllocArgs& a, const AllocState& init, cudaStream_t s) {
+  k_alloc_init<<<1, 32, 0, s>>>(a.st, init);
+  JOLT_LAUNCHED();
+  dim3 grid(a.nchunk, a.ncells);
+  for (int it = 0; it < init.max_iters + 2; ++it) {
+    k_alloc_eval<<<grid, 256, 0, s>>>(a);
+    JOLT_LAUNCHED();
+    k_alloc_decide<<<1, 512, 0, s>>>(a);
+    JOLT_LAUNCHED();
+  }
+  return JOLT_OK;
+}
+
+}  // namespace jolt

@@ -1,0 +1,743 @@
+// The C ABI of include/jolt.h: plans, handles and the order of the stages of
+// "A JoLT for the KV Cache" (Section 3): spectra of every cell -> rate-distortion
+// tables -> one shared-multiplier allocation over all cells -> ST-HOSVD fit
+// -> rotated low-bit residual; decompression rebuilds dense bf16.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "jolt_internal.cuh"
+#include "jolt_kernels.cuh"
+
+namespace jolt {
+
+// ---------------------------------------------------------------- errors ---
+static thread_local char g_err[512] = "";
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+static uint64_t g_launches = 0;
+uint64_t& launch_counter() { return g_launches; }
+
+// ------------------------------------------------------------- allocator ---
+static jolt_alloc_fn g_alloc = nullptr;
+static jolt_free_fn g_free = nullptr;
+static void* g_ctx = nullptr;
+
+void* dev_alloc(size_t bytes, cudaStream_t s) {
+  if (bytes == 0) bytes = 256;
+  if (g_alloc) return g_alloc(bytes, s, g_ctx);
+  void* p = nullptr;
+  if (cudaMallocAsync(&p, bytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return p;
+}
+void dev_free(void* p, cudaStream_t s) {
+  if (!p) return;
+  if (g_free) { g_free(p, s, g_ctx); return; }
+  cudaFreeAsync(p, s);
+}
+
+// A bump region carved out of one device allocation.
+struct Arena {
+  uint8_t* base = nullptr;
+  size_t size = 0, used = 0;
+  template <class T>
+  T* take(size_t n) {
+    size_t off = (used + 255) & ~(size_t)255;
+    used = off + n * sizeof(T);
+    return base ? reinterpret_cast<T*>(base + off) : nullptr;
+  }
+};
+
+}  // namespace jolt
+
+using namespace jolt;
+
+// ------------------------------------------------------------------ plan ---
+struct HostCell {
+  int seq, group, kind, l0, Lg;
+  int N, nmin;     // N = Lg*H*D, nmin = min(T, N)
+  int nt;          // token spectrum length fed to the allocator
+  int n_rt, rmax;  // usable rank-grid entries and the largest of them
+  int64_t min_bytes;
+};
+
+struct jolt_plan_s {
+  jolt_layout lay;
+  std::vector<int32_t> gstart;
+  jolt_options opt;
+  std::vector<int32_t> rt_grid, rd_grid, bits;
+  std::vector<int64_t> rowbytes;
+  int64_t budget = 0;
+  int G = 0, D = 0, T = 0, H = 0;
+  double C = 0.0;
+  int qcap = 0, k = 0;
+  int ncells = 0, nmin_max = 0, rmax_all = 0, lh_max = 0, nt_max = 0;
+  std::vector<HostCell> hc;
+  std::vector<CellDesc> cdesc;
+  // device
+  cudaStream_t init_stream = 0;
+  Arena ws;
+  int* d_status = nullptr;
+  double* d_eps2 = nullptr;
+  int64_t* d_rowbytes = nullptr;
+  int* d_bits = nullptr;
+  int* d_rt = nullptr;
+  int* d_rd = nullptr;
+  float2* d_cs = nullptr;
+  CellDesc* d_cells = nullptr;
+  CellRD* d_rd_cells = nullptr;
+  int* d_nt = nullptr;
+  int* d_rmax = nullptr;
+  int* d_nlh = nullptr;
+  int* d_rT_used = nullptr;      // r_T per cell (device copy for Y gram)
+  // per-cell arrays of pointers (device)
+  double** d_GT = nullptr;  double** d_ZT = nullptr;  double** d_VtT = nullptr;
+  double** d_wT = nullptr;  double** d_Cd = nullptr;  double** d_wD = nullptr;
+  double** d_nsq = nullptr; double** d_tT = nullptr;  double** d_tD = nullptr;
+  double** d_Y = nullptr;   double** d_CY = nullptr;  double** d_VtY = nullptr;
+  double** d_wY = nullptr;  double** d_ZY = nullptr;  double** d_Uf = nullptr;
+  uint16_t** d_M = nullptr; uint16_t** d_dst = nullptr;
+  EighJob* d_jobs_spec = nullptr;
+  EighJob* d_jobs_fit = nullptr;
+  double* d_fpart = nullptr;
+  int fchunk = 0;
+  double* d_apv = nullptr;
+  int* d_api = nullptr;
+  int* d_cur = nullptr;
+  int* d_keep = nullptr;
+  int achunk = 0;
+  // host mirrors of pointer arrays
+  std::vector<double*> h_tT, h_tD, h_wT, h_wD, h_nsq;
+  std::vector<uint16_t*> h_M;
+  void* ws_alloc = nullptr;
+};
+
+struct jolt_handle_s {
+  jolt_plan_t* plan = nullptr;
+  cudaStream_t stream = 0;
+  uint64_t seed = 0;
+  uint8_t* payload = nullptr;
+  int64_t capacity = 0;
+  CellOut* d_out = nullptr;
+  Choice* d_choice = nullptr;
+  AllocState* d_state = nullptr;
+  int* d_status = nullptr;
+  void* block = nullptr;
+};
+
+static jolt_status status_from_dev(int st) {
+  if (st == 0) return JOLT_OK;
+  if (st & DEV_ERR_INFEASIBLE) { set_error("byte budget infeasible for the rank/bit grids"); return JOLT_ERR_BUDGET_INFEASIBLE; }
+  if (st & DEV_ERR_NONFINITE) { set_error("a cell's squared Frobenius norm is not finite"); return JOLT_ERR_NONFINITE; }
+  if (st & DEV_ERR_TIMEOUT) { set_error("a bounded device wait expired"); return JOLT_ERR_TIMEOUT; }
+  if (st & DEV_ERR_EIG_NOCONV) { set_error("eigensolver did not converge"); return JOLT_ERR_CUDA; }
+  if (st & DEV_ERR_CHOL) { set_error("Cholesky factorization failed (rank-deficient sketch)"); return JOLT_ERR_CUDA; }
+  set_error("device status 0x%x", st);
+  return JOLT_ERR_CUDA;
+}
+
+static int64_t residual_row_bytes(int b, int D, int G) {
+  if (b == 0) return 0;
+  return ((int64_t)b * D + 32 * (D / G)) / 8;
+}
+
+static jolt_status plan_build_workspace(jolt_plan_s* p);
+
+extern "C" {
+
+void jolt_default_options(jolt_options* o) {
+  if (!o) return;
+  memset(o, 0, sizeof(*o));
+  o->mode = JOLT_EXACT;
+  o->n_bits = 4;
+  o->bits[0] = 0; o->bits[1] = 2; o->bits[2] = 4; o->bits[3] = 8;
+  o->oversample_p = 8;
+  o->power_iters = 2;
+  o->scale_group = 0;
+  o->rotation = JOLT_ROT_HADAMARD;
+  o->budget_tol = 0.005;
+  o->max_iters = 50;
+}
+
+const char* jolt_last_error(void) { return g_err; }
+uint64_t jolt_launch_count(void) { return g_launches; }
+
+jolt_status jolt_set_allocator(jolt_alloc_fn a, jolt_free_fn f, void* ctx) {
+  if ((a == nullptr) != (f == nullptr)) { set_error("alloc and free must both be set or both NULL"); return JOLT_ERR_INVALID_ARG; }
+  g_alloc = a; g_free = f; g_ctx = ctx;
+  return JOLT_OK;
+}
+
+int32_t jolt_num_cells(const jolt_plan_t* p) { return p ? p->ncells : 0; }
+
+static jolt_status validate(const jolt_layout* L, const jolt_options* o) {
+  if (!L || !o || !L->group_start) { set_error("null layout/options/group_start"); return JOLT_ERR_INVALID_ARG; }
+  if (L->batch < 1 || L->n_layers < 1 || L->n_heads < 1 || L->seq_len < 1 || L->n_groups < 1) {
+    set_error("non-positive layout dimension"); return JOLT_ERR_INVALID_ARG;
+  }
+  if (L->head_dim != 64 && L->head_dim != 128) { set_error("head_dim must be 64 or 128 (got %d)", L->head_dim); return JOLT_ERR_UNSUPPORTED_SHAPE; }
+  if (L->dtype != JOLT_BF16 && L->dtype != JOLT_F32) { set_error("dtype must be JOLT_BF16 or JOLT_F32"); return JOLT_ERR_INVALID_ARG; }
+  if (L->group_start[0] != 0 || L->group_start[L->n_groups] != L->n_layers) { set_error("groups must cover layers 0..n_layers"); return JOLT_ERR_INVALID_ARG; }
+  for (int g = 0; g < L->n_groups; ++g)
+    if (L->group_start[g + 1] <= L->group_start[g]) { set_error("group_start must increase"); return JOLT_ERR_INVALID_ARG; }
+  if (L->stride_t < L->head_dim || L->stride_h < 1 || L->stride_l < 1 || L->stride_b < 1) { set_error("bad strides"); return JOLT_ERR_INVALID_ARG; }
+  if (L->rope_theta_k < 0.0f) { set_error("rope_theta_k must be >= 0"); return JOLT_ERR_INVALID_ARG; }
+  if (o->mode != JOLT_EXACT && o->mode != JOLT_RANDOMIZED) { set_error("bad mode"); return JOLT_ERR_INVALID_ARG; }
+  if (o->rotation != JOLT_ROT_HADAMARD) { set_error("only the Hadamard rotation is implemented"); return JOLT_ERR_INVALID_ARG; }
+  if (o->n_bits < 1 || o->n_bits > 8) { set_error("n_bits must be 1..8"); return JOLT_ERR_INVALID_ARG; }
+  for (int i = 0; i < o->n_bits; ++i) {
+    int b = o->bits[i];
+    if (!(b == 0 || b == 2 || b == 3 || b == 4 || b == 8)) { set_error("bit width %d not in {0,2,3,4,8}", b); return JOLT_ERR_INVALID_ARG; }
+    if (i && b <= o->bits[i - 1]) { set_error("bits must increase"); return JOLT_ERR_INVALID_ARG; }
+  }
+  int G = o->scale_group ? o->scale_group : L->head_dim;
+  if (!(G == 32 || G == 64 || G == 128) || L->head_dim % G) { set_error("scale_group must be 32/64/128 and divide D"); return JOLT_ERR_INVALID_ARG; }
+  if (o->budget_tol < 0 || o->budget_tol >= 1 || o->max_iters < 1) { set_error("bad tolerance/max_iters"); return JOLT_ERR_INVALID_ARG; }
+  auto chk = [](int n, const int32_t* g) {
+    if (n < 0 || (n > 0 && !g)) return false;
+    for (int i = 0; i < n; ++i) if (g[i] < 1 || (i && g[i] <= g[i - 1])) return false;
+    return true;
+  };
+  if (!chk(o->n_rt, o->rt_grid) || !chk(o->n_rd, o->rd_grid)) { set_error("rank grids must be increasing positive integers"); return JOLT_ERR_INVALID_ARG; }
+  return JOLT_OK;
+}
+
+static int qcap_eq5(int T, double C) {
+  int qmin = (C <= 4.0) ? 32 : 64;
+  int q = std::max(qmin, (T + 31) / 32);
+  return std::min(q, 512);
+}
+
+jolt_status jolt_plan(const jolt_layout* L, int64_t byte_budget, const jolt_options* opt,
+                      jolt_plan_t** out) {
+  if (!out) { set_error("null out"); return JOLT_ERR_INVALID_ARG; }
+  *out = nullptr;
+  JOLT_TRY(validate(L, opt));
+  if (byte_budget <= 0) { set_error("byte budget must be positive"); return JOLT_ERR_INVALID_ARG; }
+  auto* p = new jolt_plan_s();
+  p->lay = *L;
+  p->gstart.assign(L->group_start, L->group_start + L->n_groups + 1);
+  p->lay.group_start = p->gstart.data();
+  p->opt = *opt;
+  p->rt_grid.assign(opt->rt_grid, opt->rt_grid + (opt->rt_grid ? opt->n_rt : 0));
+  p->rd_grid.assign(opt->rd_grid, opt->rd_grid + (opt->rd_grid ? opt->n_rd : 0));
+  p->opt.rt_grid = nullptr;
+  p->opt.rd_grid = nullptr;
+  p->bits.assign(opt->bits, opt->bits + opt->n_bits);
+  p->budget = byte_budget;
+  p->D = L->head_dim; p->T = L->seq_len; p->H = L->n_heads;
+  p->G = opt->scale_group ? opt->scale_group : p->D;
+  for (int b : p->bits) p->rowbytes.push_back(residual_row_bytes(b, p->D, p->G));
+  const double dense = 2.0 * 2.0 * (double)L->batch * L->n_layers * L->n_heads * (double)L->seq_len * p->D;
+  p->C = dense / (double)byte_budget;
+  p->qcap = qcap_eq5(p->T, p->C);
+  const bool rnd = opt->mode == JOLT_RANDOMIZED;
+  // rd grid: default every integer 1..D
+  if (p->rd_grid.empty()) for (int r = 1; r <= p->D; ++r) p->rd_grid.push_back(r);
+  while (!p->rd_grid.empty() && p->rd_grid.back() > p->D) p->rd_grid.pop_back();
+  if (p->rd_grid.empty()) { delete p; set_error("rd grid has no value <= D"); return JOLT_ERR_INVALID_ARG; }
+  // cells
+  int maxN = 0;
+  for (int b = 0; b < L->batch; ++b)
+    for (int g = 0; g < L->n_groups; ++g)
+      for (int kind = 0; kind < 2; ++kind) {
+        HostCell c{};
+        c.seq = b; c.group = g; c.kind = kind; c.l0 = p->gstart[g];
+        c.Lg = p->gstart[g + 1] - p->gstart[g];
+        c.N = c.Lg * p->H * p->D;
+        c.nmin = std::min(p->T, c.N);
+        maxN = std::max(maxN, c.N);
+        p->hc.push_back(c);
+      }
+  p->ncells = (int)p->hc.size();
+  // token-rank bound per cell and the shared rt grid
+  int rcap_all = 0;
+  for (auto& c : p->hc) {
+    int cap = rnd ? std::min(p->qcap, c.nmin) : c.nmin;
+    if (opt->rt_max > 0) cap = std::min(cap, opt->rt_max);
+    c.nt = rnd ? (std::min(p->qcap, c.nmin) + 1) : c.nmin;
+    c.rmax = cap;
+    rcap_all = std::max(rcap_all, cap);
+  }
+  if (p->rt_grid.empty()) for (int r = 1; r <= rcap_all; ++r) p->rt_grid.push_back(r);
+  for (auto& c : p->hc) {
+    c.n_rt = 0;
+    for (int r : p->rt_grid) if (r <= c.rmax) ++c.n_rt;
+    if (c.n_rt == 0) { delete p; set_error("rt grid has no value within the token-rank bound"); return JOLT_ERR_INVALID_ARG; }
+    c.rmax = p->rt_grid[c.n_rt - 1];
+    // cheapest option
+    int64_t best = INT64_MAX;
+    for (size_t bi = 0; bi < p->bits.size(); ++bi) {
+      int64_t LH = (int64_t)c.Lg * p->H;
+      int rt = p->rt_grid[0], rd = p->rd_grid[0];
+      int64_t s = 2 * (LH * rt * rd + (int64_t)p->T * rt + (int64_t)p->D * rd) + p->rowbytes[bi] * LH * p->T;
+      best = std::min(best, s);
+    }
+    c.min_bytes = best;
+    p->nmin_max = std::max(p->nmin_max, c.nmin);
+    p->rmax_all = std::max(p->rmax_all, c.rmax);
+    p->lh_max = std::max(p->lh_max, c.Lg * p->H);
+    p->nt_max = std::max(p->nt_max, c.nt);
+  }
+  if (!rnd && p->nmin_max > 2048) {
+    delete p;
+    set_error("exact mode needs min(T, L_g*H*D) <= 2048 (got %d); use JOLT_RANDOMIZED", p->nmin_max);
+    return JOLT_ERR_UNSUPPORTED_SHAPE;
+  }
+  int64_t minsum = 0;
+  for (auto& c : p->hc) minsum += c.min_bytes;
+  if (byte_budget < minsum) {
+    delete p;
+    set_error("budget %lld below the cheapest allocation %lld", (long long)byte_budget, (long long)minsum);
+    return JOLT_ERR_BUDGET_INFEASIBLE;
+  }
+  jolt_status st = plan_build_workspace(p);
+  if (st != JOLT_OK) { jolt_free_plan(p); return st; }
+  *out = p;
+  return JOLT_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------- workspace ---
+template <class T>
+static T* upload(Arena& A, const std::vector<T>& v) {
+  return A.take<T>(v.size());
+}
+
+static jolt_status plan_build_workspace(jolt_plan_s* p) {
+  const int nc = p->ncells, D = p->D, T = p->T;
+  p->fchunk = 64;
+  p->achunk = 32;
+  // two passes: size, then carve
+  for (int pass = 0; pass < 2; ++pass) {
+    Arena& A = p->ws;
+    A.used = 0;
+    p->d_status = A.take<int>(4);
+    p->d_eps2 = A.take<double>(8);
+    p->d_rowbytes = A.take<int64_t>(8);
+    p->d_bits = A.take<int>(8);
+    p->d_rt = A.take<int>(p->rt_grid.size());
+    p->d_rd = A.take<int>(p->rd_grid.size());
+    p->d_cs = p->lay.rope_theta_k > 0 ? A.take<float2>((size_t)T * (D / 2)) : nullptr;
+    p->d_cells = A.take<CellDesc>(nc);
+    p->d_rd_cells = A.take<CellRD>(nc);
+    p->d_nt = A.take<int>(nc);
+    p->d_rmax = A.take<int>(nc);
+    p->d_nlh = A.take<int>(nc);
+    p->d_rT_used = A.take<int>(nc);
+    p->d_GT = A.take<double*>(nc); p->d_ZT = A.take<double*>(nc); p->d_VtT = A.take<double*>(nc);
+    p->d_wT = A.take<double*>(nc); p->d_Cd = A.take<double*>(nc); p->d_wD = A.take<double*>(nc);
+    p->d_nsq = A.take<double*>(nc); p->d_tT = A.take<double*>(nc); p->d_tD = A.take<double*>(nc);
+    p->d_Y = A.take<double*>(nc); p->d_CY = A.take<double*>(nc); p->d_VtY = A.take<double*>(nc);
+    p->d_wY = A.take<double*>(nc); p->d_ZY = A.take<double*>(nc); p->d_Uf = A.take<double*>(nc);
+    p->d_M = A.take<uint16_t*>(nc); p->d_dst = A.take<uint16_t*>(nc);
+    p->d_jobs_spec = A.take<EighJob>(2 * nc);
+    p->d_jobs_fit = A.take<EighJob>(nc);
+    p->d_fpart = A.take<double>((size_t)nc * p->fchunk * (D * D + 1));
+    p->d_apv = A.take<double>((size_t)nc * p->achunk);
+    p->d_api = A.take<int>((size_t)nc * p->achunk);
+    p->d_cur = A.take<int>(nc);
+    p->d_keep = A.take<int>(nc);
+    // per-cell buffers
+    std::vector<double*> GT(nc), ZT(nc), VtT(nc), wT(nc), Cd(nc), wD(nc), nsq(nc), tT(nc), tD(nc),
+        Y(nc), CY(nc), VtY(nc), wY(nc), ZY(nc), Uf(nc), workT(nc), workD(nc), workY(nc);
+    std::vector<uint16_t*> M(nc);
+    const bool rnd = p->opt.mode == JOLT_RANDOMIZED;
+    for (int i = 0; i < nc; ++i) {
+      const HostCell& c = p->hc[i];
+      const int n = c.nmin;
+      const int64_t LH = (int64_t)c.Lg * p->H;
+      if (!rnd) {
+        GT[i] = A.take<double>((size_t)n * n);
+        ZT[i] = A.take<double>((size_t)n * n);
+        VtT[i] = A.take<double>((size_t)n * n);
+        wT[i] = A.take<double>(n);
+        workT[i] = A.take<double>(n);
+        Uf[i] = (T > c.N) ? A.take<double>((size_t)c.rmax * T) : nullptr;
+      } else {
+        GT[i] = ZT[i] = VtT[i] = Uf[i] = workT[i] = nullptr;
+        wT[i] = A.take<double>(c.nt);
+      }
+      Cd[i] = A.take<double>((size_t)D * D);
+      wD[i] = A.take<double>(D);
+      workD[i] = A.take<double>(D);
+      nsq[i] = A.take<double>(1);
+      tT[i] = A.take<double>(c.nt + 1);
+      tD[i] = A.take<double>(D + 1);
+      Y[i] = A.take<double>((size_t)LH * c.rmax * D);
+      CY[i] = A.take<double>((size_t)D * D);
+      VtY[i] = A.take<double>((size_t)D * D);
+      wY[i] = A.take<double>(D);
+      ZY[i] = A.take<double>((size_t)D * D);
+      workY[i] = A.take<double>(D);
+      M[i] = A.take<uint16_t>((size_t)LH * c.rmax * D);
+    }
+    if (pass == 0) {
+      A.size = A.used + 4096;
+      p->ws_alloc = dev_alloc(A.size, p->init_stream);
+      if (!p->ws_alloc) { set_error("workspace allocation of %zu bytes failed", A.size); return JOLT_ERR_OOM; }
+      A.base = reinterpret_cast<uint8_t*>(p->ws_alloc);
+      continue;
+    }
+    // ---- fill device tables
+    cudaStream_t s = p->init_stream;
+    JOLT_CUDA_TRY(cudaMemsetAsync(p->d_status, 0, 4 * sizeof(int), s));
+    std::vector<int> bits(8, 0);
+    for (size_t i = 0; i < p->bits.size(); ++i) bits[i] = p->bits[i];
+    std::vector<int64_t> rb(8, 0);
+    for (size_t i = 0; i < p->rowbytes.size(); ++i) rb[i] = p->rowbytes[i];
+    JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_bits, bits.data(), 8 * sizeof(int), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_rowbytes, rb.data(), 8 * sizeof(int64_t), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_rt, p->rt_grid.data(), p->rt_grid.size() * sizeof(int), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_rd, p->rd_grid.data(), p->rd_grid.size() * sizeof(int), cudaMemcpyHostToDevice, s));
+    std::vector<CellRD> rdc(nc);
+    std::vector<int> ntv(nc), rmaxv(nc), nlhv(nc);
+    std::vector<EighJob> js(2 * nc), jf(nc);
+    for (int i = 0; i < nc; ++i) {
+      const HostCell& c = p->hc[i];
+      rdc[i] = CellRD{c.Lg, p->H, T, D, c.n_rt, c.nt - 0, tT[i], tD[i]};
+      ntv[i] = c.nt;
+      rmaxv[i] = c.rmax;
+      nlhv[i] = c.Lg * p->H;
+      js[i] = EighJob{rnd ? 0 : c.nmin, 1, GT[i], wT[i], VtT[i], ZT[i], workT[i]};
+      js[nc + i] = EighJob{D, 0, Cd[i], wD[i], nullptr, nullptr, workD[i]};
+      jf[i] = EighJob{D, 1, CY[i], wY[i], VtY[i], ZY[i], workY[i]};
+    }
+    JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_rd_cells, rdc.data(), nc * sizeof(CellRD), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_nt, ntv.data(), nc * sizeof(int), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_rmax, rmaxv.data(), nc * sizeof(int), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_nlh, nlhv.data(), nc * sizeof(int), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_jobs_spec, js.data(), js.size() * sizeof(EighJob), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_jobs_fit, jf.data(), jf.size() * sizeof(EighJob), cudaMemcpyHostToDevice, s));
+#define UP(dst, v) JOLT_CUDA_TRY(cudaMemcpyAsync(dst, v.data(), nc * sizeof(v[0]), cudaMemcpyHostToDevice, s))
+    UP(p->d_GT, GT); UP(p->d_ZT, ZT); UP(p->d_VtT, VtT); UP(p->d_wT, wT); UP(p->d_Cd, Cd);
+    UP(p->d_wD, wD); UP(p->d_nsq, nsq); UP(p->d_tT, tT); UP(p->d_tD, tD); UP(p->d_Y, Y);
+    UP(p->d_CY, CY); UP(p->d_VtY, VtY); UP(p->d_wY, wY); UP(p->d_ZY, ZY); UP(p->d_Uf, Uf);
+    UP(p->d_M, M);
+#undef UP
+    p->h_tT = tT; p->h_tD = tD; p->h_wT = wT; p->h_wD = wD; p->h_nsq = nsq; p->h_M = M;
+    if (p->d_cs) JOLT_TRY(launch_rope_table(T, D, (double)p->lay.rope_theta_k, p->d_cs, s));
+    JOLT_TRY(launch_eps2(p->bits.data(), (int)p->bits.size(), p->G, p->d_eps2, p->d_fpart, s));
+    JOLT_CUDA_TRY(cudaStreamSynchronize(s));
+  }
+  return JOLT_OK;
+}
+
+// Device descriptors of the cells for given K/V base pointers.
+static jolt_status upload_cells(jolt_plan_s* p, const void* k, const void* v, cudaStream_t s) {
+  const jolt_layout& L = p->lay;
+  p->cdesc.resize(p->ncells);
+  const size_t esz = L.dtype == JOLT_F32 ? 4 : 2;
+  for (int i = 0; i < p->ncells; ++i) {
+    const HostCell& c = p->hc[i];
+    CellDesc d{};
+    const uint8_t* base = reinterpret_cast<const uint8_t*>(c.kind == 0 ? k : v);
+    d.src = base ? base + ((int64_t)c.seq * L.stride_b + (int64_t)c.l0 * L.stride_l) * esz : nullptr;
+    d.sl = L.stride_l; d.sh = L.stride_h; d.st = L.stride_t;
+    d.Lg = c.Lg; d.H = p->H; d.T = p->T; d.D = p->D;
+    d.kind = c.kind;
+    d.rope = (c.kind == 0 && L.rope_theta_k > 0) ? 1 : 0;
+    d.f32 = L.dtype == JOLT_F32;
+    d.seq = c.seq;
+    d.l0 = c.l0;
+    d.nt = c.nt;
+    d.rtmax = c.rmax;
+    p->cdesc[i] = d;
+  }
+  JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_cells, p->cdesc.data(), p->ncells * sizeof(CellDesc), cudaMemcpyHostToDevice, s));
+  return JOLT_OK;
+}
+
+// Spectra of every cell: ||X||^2, feature Gram eigenvalues, token spectrum.
+static jolt_status run_spectra(jolt_plan_s* p, int* status, cudaStream_t s) {
+  const int nc = p->ncells, D = p->D;
+  JOLT_TRY(launch_fgram_x(p->d_cells, nc, D, p->d_cs, p->fchunk, p->d_fpart, s));
+  JOLT_TRY(launch_sum_chunks(p->d_fpart, p->fchunk, D * D + 1, nc, p->d_Cd, p->d_nsq, s));
+  if (p->opt.mode == JOLT_EXACT) {
+    JOLT_TRY(launch_token_gram(p->d_cells, nc, p->nmin_max, p->d_cs, p->d_GT, s));
+    JOLT_TRY(launch_eigh(p->d_jobs_spec, 2 * nc, std::max(p->nmin_max, D), status, s));
+  } else {
+    set_error("randomized mode is not built yet");
+    return JOLT_ERR_UNSUPPORTED_SHAPE;
+  }
+  JOLT_TRY(launch_rd_tables(p->d_rd_cells, nc, p->d_wT, p->d_wD, nullptr, p->d_tT, p->d_tD, p->d_nt,
+                            p->d_nsq, status, s));
+  return JOLT_OK;
+}
+
+static jolt_status run_allocation(jolt_plan_s* p, int64_t budget, const double* eps2, AllocState* st_dev,
+                                  Choice* out, int* status, cudaStream_t s) {
+  AllocState st{};
+  st.lo = 1e-30; st.hi = 1.0; st.lam = st.lo;
+  st.tol = p->opt.budget_tol;
+  st.budget = budget;
+  st.max_iters = p->opt.max_iters;
+  st.phase = 0;
+  AllocArgs a{};
+  a.cells = p->d_rd_cells; a.ncells = p->ncells;
+  a.rt_grid = p->d_rt; a.rd_grid = p->d_rd; a.n_rd = (int)p->rd_grid.size();
+  a.bits = p->d_bits; a.eps2 = eps2; a.rowbytes = p->d_rowbytes; a.n_bits = (int)p->bits.size();
+  a.nchunk = p->achunk; a.pv = p->d_apv; a.pi = p->d_api; a.cur = p->d_cur; a.keep = p->d_keep;
+  a.st = st_dev; a.out = out; a.status = status;
+  return launch_alloc(a, st, s);
+}
+
+extern "C" {
+
+void jolt_free_plan(jolt_plan_t* p) {
+  if (!p) return;
+  if (p->ws_alloc) dev_free(p->ws_alloc, p->init_stream);
+  delete p;
+}
+
+jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t byte_budget,
+                          uint64_t seed, jolt_stream_t stream_, jolt_handle_t** out) {
+  cudaStream_t s = (cudaStream_t)stream_;
+  if (!p || !k || !v || !out) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
+  *out = nullptr;
+  const int64_t B = byte_budget > 0 ? byte_budget : p->budget;
+  int64_t minsum = 0, extra = 0;
+  for (auto& c : p->hc) {
+    minsum += c.min_bytes;
+    extra += 5 * 256 + (int64_t)c.rmax * 16;
+  }
+  if (B < minsum) { set_error("budget %lld below the cheapest allocation %lld", (long long)B, (long long)minsum); return JOLT_ERR_BUDGET_INFEASIBLE; }
+  const int nc = p->ncells;
+  auto* h = new jolt_handle_s();
+  h->plan = p;
+  h->stream = s;
+  h->seed = seed;
+  h->capacity = B + extra + 4096;
+  Arena A;
+  for (int pass = 0; pass < 2; ++pass) {
+    A.used = 0;
+    h->d_out = A.take<CellOut>(nc);
+    h->d_choice = A.take<Choice>(nc);
+    h->d_state = A.take<AllocState>(1);
+    h->d_status = A.take<int>(4);
+    h->payload = A.take<uint8_t>((size_t)h->capacity);
+    if (pass == 0) {
+      h->block = dev_alloc(A.used + 256, s);
+      if (!h->block) { delete h; set_error("handle allocation failed"); return JOLT_ERR_OOM; }
+      A.base = reinterpret_cast<uint8_t*>(h->block);
+    }
+  }
+  auto fail = [&](jolt_status st) { jolt_free_handle(h); return st; };
+  if (cudaMemsetAsync(h->d_status, 0, 4 * sizeof(int), s) != cudaSuccess) return fail(JOLT_ERR_CUDA);
+  jolt_status st;
+  if ((st = upload_cells(p, k, v, s)) != JOLT_OK) return fail(st);
+  if ((st = run_spectra(p, h->d_status, s)) != JOLT_OK) return fail(st);
+  if ((st = run_allocation(p, B, p->d_eps2, h->d_state, h->d_choice, h->d_status, s)) != JOLT_OK) return fail(st);
+  if ((st = launch_payload_layout(p->d_cells, h->d_choice, nc, p->G, h->payload, h->capacity, h->d_out,
+                                  h->d_status, s)) != JOLT_OK) return fail(st);
+  FitArgs fa{};
+  fa.cells = p->d_cells; fa.cs = p->d_cs; fa.out = h->d_out; fa.ncells = nc; fa.D = p->D;
+  fa.VtT = p->d_VtT; fa.wT = p->d_wT; fa.Uf = p->d_Uf; fa.Y = p->d_Y; fa.rmax_of = p->d_rmax;
+  fa.VtY = p->d_VtY; fa.M = p->d_M;
+  if (p->opt.mode == JOLT_EXACT) {
+    if ((st = launch_ut_exact(fa, p->T, p->rmax_all, s)) != JOLT_OK) return fail(st);
+    if ((st = launch_project_y(fa, p->T, p->rmax_all, p->lh_max, s)) != JOLT_OK) return fail(st);
+  }
+  // feature Gram of Y (rows r < r_T), then its eigenvectors
+  if ((st = launch_copy_rt(h->d_out, p->d_rT_used, nc, s)) != JOLT_OK) return fail(st);
+  if ((st = launch_fgram_rows(p->d_Y, p->d_rT_used, p->d_rmax, p->d_nlh, nc, p->D, p->fchunk, p->d_fpart, s)) != JOLT_OK) return fail(st);
+  if ((st = launch_sum_chunks(p->d_fpart, p->fchunk, p->D * p->D + 1, nc, p->d_CY, nullptr, s)) != JOLT_OK) return fail(st);
+  if ((st = launch_eigh(p->d_jobs_fit, nc, p->D, h->d_status, s)) != JOLT_OK) return fail(st);
+  if ((st = launch_core(fa, p->rmax_all, p->lh_max, s)) != JOLT_OK) return fail(st);
+  ResidArgs ra{};
+  ra.cells = p->d_cells; ra.cs = p->d_cs; ra.out = h->d_out; ra.M = p->d_M; ra.rmax_of = p->d_rmax;
+  ra.G = p->G; ra.seed = seed;
+  if ((st = launch_residual_simt(ra, nc, p->D, p->T, p->lh_max, s)) != JOLT_OK) return fail(st);
+  *out = h;
+  return JOLT_OK;
+}
+
+jolt_status jolt_decompress(const jolt_handle_t* h, void* k_out, void* v_out, const jolt_layout* ol,
+                            jolt_stream_t stream_) {
+  cudaStream_t s = (cudaStream_t)stream_;
+  if (!h || !k_out || !v_out) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
+  jolt_plan_s* p = h->plan;
+  const jolt_layout& L = ol ? *ol : p->lay;
+  if (L.batch != p->lay.batch || L.n_layers != p->lay.n_layers || L.n_heads != p->H || L.seq_len != p->T ||
+      L.head_dim != p->D) { set_error("output layout shape differs from the plan"); return JOLT_ERR_INVALID_ARG; }
+  if (L.stride_t < p->D || (L.stride_t % 2) || (L.stride_h % 2) || (L.stride_l % 2) || (L.stride_b % 2)) {
+    set_error("output strides must be even and stride_t >= head_dim"); return JOLT_ERR_UNSUPPORTED_SHAPE;
+  }
+  const int nc = p->ncells;
+  JOLT_TRY(launch_core_m(h->d_out, p->d_cells, p->d_M, p->d_rmax, nc, p->D, p->rmax_all, p->lh_max, s));
+  ResidArgs ra{};
+  ra.cells = p->d_cells; ra.cs = p->d_cs; ra.out = h->d_out; ra.M = p->d_M; ra.rmax_of = p->d_rmax;
+  ra.G = p->G; ra.seed = h->seed;
+  ra.out_k = reinterpret_cast<uint16_t*>(k_out); ra.out_v = reinterpret_cast<uint16_t*>(v_out);
+  ra.osb = L.stride_b; ra.osl = L.stride_l; ra.osh = L.stride_h; ra.ost = L.stride_t;
+  JOLT_TRY(launch_decompress_simt(ra, nc, p->D, p->T, p->lh_max, s));
+  return JOLT_OK;
+}
+
+static jolt_status handle_sync(const jolt_handle_t* h) {
+  JOLT_CUDA_TRY(cudaStreamSynchronize(h->stream));
+  int st = 0;
+  JOLT_CUDA_TRY(cudaMemcpy(&st, h->d_status, sizeof(int), cudaMemcpyDeviceToHost));
+  return status_from_dev(st);
+}
+
+jolt_status jolt_bytes(const jolt_handle_t* h, int64_t* nbytes) {
+  if (!h || !nbytes) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
+  JOLT_TRY(handle_sync(h));
+  std::vector<Choice> ch(h->plan->ncells);
+  JOLT_CUDA_TRY(cudaMemcpy(ch.data(), h->d_choice, ch.size() * sizeof(Choice), cudaMemcpyDeviceToHost));
+  int64_t s = 0;
+  for (auto& c : ch) s += c.bytes;
+  *nbytes = s;
+  return JOLT_OK;
+}
+
+jolt_status jolt_handle_info(const jolt_handle_t* h, jolt_cell_info* cells, int32_t n, double* lambda,
+                             int32_t* iterations) {
+  if (!h) { set_error("null handle"); return JOLT_ERR_INVALID_ARG; }
+  jolt_plan_s* p = h->plan;
+  if (cells && n < p->ncells) { set_error("need room for %d cells", p->ncells); return JOLT_ERR_INVALID_ARG; }
+  JOLT_TRY(handle_sync(h));
+  std::vector<Choice> ch(p->ncells);
+  JOLT_CUDA_TRY(cudaMemcpy(ch.data(), h->d_choice, ch.size() * sizeof(Choice), cudaMemcpyDeviceToHost));
+  AllocState st;
+  JOLT_CUDA_TRY(cudaMemcpy(&st, h->d_state, sizeof(st), cudaMemcpyDeviceToHost));
+  if (cells) {
+    for (int i = 0; i < p->ncells; ++i) {
+      const HostCell& c = p->hc[i];
+      double nsq = 0.0;
+      JOLT_CUDA_TRY(cudaMemcpy(&nsq, p->h_nsq[i], sizeof(double), cudaMemcpyDeviceToHost));
+      cells[i] = jolt_cell_info{c.seq, c.group, c.kind, ch[i].rT, ch[i].rd, ch[i].b, ch[i].bytes, ch[i].err, nsq};
+    }
+  }
+  if (lambda) *lambda = st.lam_final;
+  if (iterations) *iterations = st.iters_final;
+  return JOLT_OK;
+}
+
+jolt_status jolt_handle_cell(const jolt_handle_t* h, int32_t cell, jolt_cell_view* v) {
+  if (!h || !v) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
+  jolt_plan_s* p = h->plan;
+  if (cell < 0 || cell >= p->ncells) { set_error("cell %d out of range", cell); return JOLT_ERR_INVALID_ARG; }
+  JOLT_TRY(handle_sync(h));
+  CellOut o;
+  JOLT_CUDA_TRY(cudaMemcpy(&o, h->d_out + cell, sizeof(o), cudaMemcpyDeviceToHost));
+  const HostCell& c = p->hc[cell];
+  *v = jolt_cell_view{o.rT, o.rd, o.b, p->G, c.Lg, p->H, p->T, p->D, o.t_pitch,
+                      o.ut, o.ud, o.core, o.codes, o.scales};
+  return JOLT_OK;
+}
+
+void jolt_free_handle(jolt_handle_t* h) {
+  if (!h) return;
+  if (h->block) dev_free(h->block, h->stream);
+  delete h;
+}
+
+jolt_status jolt_rd_table(jolt_plan_t* p, const void* k, const void* v, double* norm_sq, double* sig_t,
+                          int32_t max_t, int32_t* n_t, double* sig_d, jolt_stream_t stream_) {
+  cudaStream_t s = (cudaStream_t)stream_;
+  if (!p || !k || !v || !norm_sq || !sig_t || !n_t || !sig_d) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
+  if (max_t < p->nt_max) { set_error("max_t must be >= %d", p->nt_max); return JOLT_ERR_INVALID_ARG; }
+  JOLT_CUDA_TRY(cudaMemsetAsync(p->d_status, 0, sizeof(int), s));
+  JOLT_TRY(upload_cells(p, k, v, s));
+  JOLT_TRY(run_spectra(p, p->d_status, s));
+  JOLT_CUDA_TRY(cudaStreamSynchronize(s));
+  int st = 0;
+  JOLT_CUDA_TRY(cudaMemcpy(&st, p->d_status, sizeof(int), cudaMemcpyDeviceToHost));
+  JOLT_TRY(status_from_dev(st));
+  for (int i = 0; i < p->ncells; ++i) {
+    const HostCell& c = p->hc[i];
+    JOLT_CUDA_TRY(cudaMemcpy(norm_sq + i, p->h_nsq[i], sizeof(double), cudaMemcpyDeviceToHost));
+    std::fill(sig_t + (size_t)i * max_t, sig_t + (size_t)(i + 1) * max_t, 0.0);
+    JOLT_CUDA_TRY(cudaMemcpy(sig_t + (size_t)i * max_t, p->h_wT[i], c.nt * sizeof(double), cudaMemcpyDeviceToHost));
+    JOLT_CUDA_TRY(cudaMemcpy(sig_d + (size_t)i * p->D, p->h_wD[i], p->D * sizeof(double), cudaMemcpyDeviceToHost));
+  }
+  *n_t = p->nt_max;
+  return JOLT_OK;
+}
+
+jolt_status jolt_allocate(jolt_plan_t* p, const double* t_t, int32_t ld_t, const double* t_d, int32_t ld_d,
+                          const double* eps2, int64_t byte_budget, int32_t* choice, int64_t* bytes,
+                          double* lambda, int32_t* iterations, jolt_stream_t stream_) {
+  cudaStream_t s = (cudaStream_t)stream_;
+  if (!p || !t_t || !t_d || !eps2 || !choice || !bytes) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
+  if (ld_t < p->nt_max + 1 || ld_d < p->D + 1) { set_error("ld_t >= %d and ld_d >= %d required", p->nt_max + 1, p->D + 1); return JOLT_ERR_INVALID_ARG; }
+  const int nc = p->ncells;
+  for (int i = 0; i < nc; ++i) {
+    JOLT_CUDA_TRY(cudaMemcpyAsync(p->h_tT[i], t_t + (size_t)i * ld_t, (p->hc[i].nt + 1) * sizeof(double), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemcpyAsync(p->h_tD[i], t_d + (size_t)i * ld_d, (p->D + 1) * sizeof(double), cudaMemcpyHostToDevice, s));
+  }
+  double* d_e = p->d_fpart;     // scratch for the given eps^2
+  JOLT_CUDA_TRY(cudaMemcpyAsync(d_e, eps2, p->bits.size() * sizeof(double), cudaMemcpyHostToDevice, s));
+  AllocState* d_st = reinterpret_cast<AllocState*>(p->d_fpart + 16);
+  Choice* d_out = reinterpret_cast<Choice*>(p->d_fpart + 64);
+  JOLT_CUDA_TRY(cudaMemsetAsync(p->d_status, 0, sizeof(int), s));
+  JOLT_TRY(run_allocation(p, byte_budget, d_e, d_st, d_out, p->d_status, s));
+  JOLT_CUDA_TRY(cudaStreamSynchronize(s));
+  int st = 0;
+  JOLT_CUDA_TRY(cudaMemcpy(&st, p->d_status, sizeof(int), cudaMemcpyDeviceToHost));
+  std::vector<Choice> ch(nc);
+  JOLT_CUDA_TRY(cudaMemcpy(ch.data(), d_out, nc * sizeof(Choice), cudaMemcpyDeviceToHost));
+  AllocState hs;
+  JOLT_CUDA_TRY(cudaMemcpy(&hs, d_st, sizeof(hs), cudaMemcpyDeviceToHost));
+  for (int i = 0; i < nc; ++i) {
+    choice[3 * i] = ch[i].rT; choice[3 * i + 1] = ch[i].rd; choice[3 * i + 2] = ch[i].b;
+    bytes[i] = ch[i].bytes;
+  }
+  if (lambda) *lambda = hs.lam_final;
+  if (iterations) *iterations = hs.iters_final;
+  return status_from_dev(st);
+}
+
+jolt_status jolt_eps2(const int32_t* bits, int32_t n, int32_t group, double* eps2, jolt_stream_t stream_) {
+  cudaStream_t s = (cudaStream_t)stream_;
+  if (!bits || !eps2 || n < 1 || n > 8) { set_error("bad arguments"); return JOLT_ERR_INVALID_ARG; }
+  for (int i = 0; i < n; ++i)
+    if (!(bits[i] == 0 || bits[i] == 2 || bits[i] == 3 || bits[i] == 4 || bits[i] == 8)) { set_error("bad bit width"); return JOLT_ERR_INVALID_ARG; }
+  if (!(group == 32 || group == 64 || group == 128)) { set_error("group must be 32, 64 or 128"); return JOLT_ERR_INVALID_ARG; }
+  size_t nblk = ((1 << 20) / group + 255) / 256;
+  double* buf = reinterpret_cast<double*>(dev_alloc((nblk * 9 + 16) * sizeof(double), s));
+  if (!buf) { set_error("allocation failed"); return JOLT_ERR_OOM; }
+  jolt_status st = launch_eps2(bits, n, group, buf, buf + 16, s);
+  if (st == JOLT_OK) {
+    if (cudaMemcpyAsync(eps2, buf, n * sizeof(double), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) { set_error("copy failed"); st = JOLT_ERR_CUDA; }
+  }
+  dev_free(buf, s);
+  return st;
+}
+
+static jolt_status check_rows(int32_t D, int32_t bits, int32_t group) {
+  if (D != 64 && D != 128) { set_error("D must be 64 or 128"); return JOLT_ERR_UNSUPPORTED_SHAPE; }
+  if (!(bits == 2 || bits == 3 || bits == 4 || bits == 8)) { set_error("bits must be 2, 3, 4 or 8"); return JOLT_ERR_INVALID_ARG; }
+  if (!(group == 32 || group == 64 || group == D) || D % group) { set_error("bad group"); return JOLT_ERR_INVALID_ARG; }
+  return JOLT_OK;
+}
+
+jolt_status jolt_residual_encode(const float* e, int64_t rows, int32_t D, int32_t bits, int32_t group,
+                                 uint64_t seed, uint8_t* codes, float* scales, jolt_stream_t stream_) {
+  JOLT_TRY(check_rows(D, bits, group));
+  if (rows < 0 || (rows > 0 && (!e || !codes || !scales))) { set_error("bad arguments"); return JOLT_ERR_INVALID_ARG; }
+  return launch_encode_rows(e, rows, D, bits, group, seed, codes, scales, (cudaStream_t)stream_);
+}
+
+jolt_status jolt_residual_decode(const uint8_t* codes, const float* scales, int64_t rows, int32_t D,
+                                 int32_t bits, int32_t group, uint64_t seed, float* e_hat,
+                                 jolt_stream_t stream_) {
+  JOLT_TRY(check_rows(D, bits, group));
+  if (rows < 0 || (rows > 0 && (!e_hat || !codes || !scales))) { set_error("bad arguments"); return JOLT_ERR_INVALID_ARG; }
+  return launch_decode_rows(codes, scales, rows, D, bits, group, seed, e_hat, (cudaStream_t)stream_);
+}
+
+}  // extern "C"

@@ -1,0 +1,153 @@
+// Kernel-side structures and host launchers shared across translation units.
+#pragma once
+#include "jolt_internal.cuh"
+
+namespace jolt {
+
+// ------------------------------------------------------------ eigensolver --
+struct EighJob {
+  int n;
+  int want_vec;
+  double* A;      // n*n, destroyed
+  double* w;      // n, descending
+  double* Vt;     // n*n, row j = eigenvector j (if want_vec)
+  double* Z;      // n*n scratch (if want_vec)
+  double* work;   // n scratch
+};
+
+jolt_status launch_eigh(const EighJob* jobs_dev, int njobs, int nmax, int* status, cudaStream_t s);
+size_t eigh_smem_bytes(int nmax);
+jolt_status launch_fgram_x(const CellDesc* cells, int ncells, int D, const float2* cs, int nchunk,
+                           double* partial, cudaStream_t s);
+jolt_status launch_fgram_rows(const double* const* Y, const int* nrow_used, const int* rmax_of,
+                              const int* nlh_of, int ncells, int D, int nchunk, double* partial,
+                              cudaStream_t s);
+jolt_status launch_sum_chunks(const double* partial, int nchunk, int len, int ncells,
+                              double* const* out, double* const* out_last, cudaStream_t s);
+jolt_status launch_token_gram(const CellDesc* cells, int ncells, int nmax, const float2* cs,
+                              double* const* G, cudaStream_t s);
+
+// ------------------------------------------------------------- allocation --
+// Per-cell data the allocator reads (device).
+struct CellRD {
+  int Lg, H, T, D;
+  int n_rt;             // grid entries usable by this cell
+  int nt;               // t_T has nt+1 entries
+  const double* tT;     // [nt+1]
+  const double* tD;     // [D+1]
+};
+
+struct AllocState {
+  double lo, hi, lam;   // bracket and the multiplier being evaluated
+  double tol;
+  int64_t budget;
+  int max_iters;
+  int phase;            // 0: lambda_lo, 1: lambda_hi, 2: bisection, 3: done
+  int iter;
+  int result_from_hi;   // 1 when the final answer is the kept feasible side
+  double lam_final;
+  int iters_final;
+  int64_t S;
+};
+
+// The chosen option of a cell (device).
+struct Choice {
+  int rT, rd, b, pad;
+  int64_t bytes;
+  double err;
+};
+
+struct AllocArgs {
+  const CellRD* cells;
+  int ncells;
+  const int* rt_grid;       // shared grid values
+  const int* rd_grid;
+  int n_rd;
+  const int* bits;
+  const double* eps2;
+  const int64_t* rowbytes;  // residual bytes per row for each bit entry
+  int n_bits;
+  int nchunk;               // option chunks per cell
+  double* pv;               // [ncells][nchunk] partial min values
+  int* pi;                  // [ncells][nchunk] partial argmins
+  int* cur;                 // [ncells] current argmin
+  int* keep;                // [ncells] feasible-side argmin
+  AllocState* st;
+  Choice* out;              // [ncells]
+  int* status;
+};
+
+jolt_status launch_alloc(const AllocArgs& a, const AllocState& init, cudaStream_t s);
+jolt_status launch_rd_tables(const CellRD* cells, int ncells, const double* const* wT,
+                             const double* const* wD, const double* normsq,
+                             double* const* tT, double* const* tD, const int* nt_used,
+                             const double* const* normsq_in, int* status, cudaStream_t s);
+jolt_status launch_eps2(const int* bits_host, int nb, int G, double* eps2_dev, double* scratch,
+                        cudaStream_t s);
+
+// ------------------------------------------------------------------ fit ----
+// Where one compressed cell lives in the handle's payload (device).
+struct CellOut {
+  uint16_t* ut;      // [rT][t_pitch] bf16 U_T^ transposed
+  uint16_t* ud;      // [D][rd] bf16
+  uint16_t* core;    // [Lg][H][rT][rd] bf16
+  uint8_t* codes;    // [Lg][H][T][b*D/8]
+  float* scales;     // [Lg][H][T][D/G]
+  int rT, rd, b, t_pitch;
+  int64_t bytes;
+};
+
+jolt_status launch_payload_layout(const CellDesc* cells, const Choice* ch, int ncells, int G,
+                                  uint8_t* base, int64_t capacity, CellOut* out, int* status,
+                                  cudaStream_t s);
+
+struct FitArgs {
+  const CellDesc* cells;
+  const float2* cs;
+  const CellOut* out;
+  int ncells;
+  int D;
+  // exact-mode token factor
+  const double* const* VtT;     // eigenvectors of the token Gram (rows)
+  const double* const* wT;      // eigenvalues
+  double* const* Uf;            // [rmax][T] fp64 scratch (T > N case)
+  // projection / feature factor / core
+  double* const* Y;             // [Lg*H][rmax][D] fp64
+  const int* rmax_of;
+  const double* const* VtY;     // eigenvectors of the projected feature Gram
+  uint16_t* const* M;           // [Lg*H][rmax][D] bf16 (decoder product M^)
+};
+
+jolt_status launch_ut_exact(const FitArgs& a, int Tmax, int rmax_all, cudaStream_t s);
+jolt_status launch_project_y(const FitArgs& a, int Tmax, int rmax_all, int lh_max, cudaStream_t s);
+jolt_status launch_core(const FitArgs& a, int rmax_all, int lh_max, cudaStream_t s);
+jolt_status launch_copy_rt(const CellOut* out, int* rt, int ncells, cudaStream_t s);
+jolt_status launch_core_m(const CellOut* out, const CellDesc* cells, uint16_t* const* M, const int* rmax_of,
+                          int ncells, int D, int rmax_all, int lh_max, cudaStream_t s);
+
+// ----------------------------------------------------------- residual ------
+struct ResidArgs {
+  const CellDesc* cells;
+  const float2* cs;
+  const CellOut* out;
+  uint16_t* const* M;           // [Lg*H][rmax][D] bf16 per cell
+  const int* rmax_of;
+  int G;
+  uint64_t seed;
+  // decompress outputs (bf16)
+  uint16_t* out_k;              // decompress outputs (bf16), NULL when encoding
+  uint16_t* out_v;
+  int64_t osb, osl, osh, ost;   // output strides (elements)
+};
+
+jolt_status launch_residual_simt(const ResidArgs& a, int ncells, int D, int Tmax, int lh_max,
+                                 cudaStream_t s);
+jolt_status launch_decompress_simt(const ResidArgs& a, int ncells, int D, int Tmax, int lh_max,
+                                   cudaStream_t s);
+jolt_status launch_encode_rows(const float* e, int64_t rows, int D, int b, int G, uint64_t seed,
+                               uint8_t* codes, float* scales, cudaStream_t s);
+jolt_status launch_decode_rows(const uint8_t* codes, const float* scales, int64_t rows, int D,
+                               int b, int G, uint64_t seed, float* e, cudaStream_t s);
+jolt_status launch_rope_table(int T, int D, double theta, float2* cs, cudaStream_t s);
+
+}  // namespace jolt

@@ -1,0 +1,481 @@
+// fp64 Gram matrices and the batched symmetric eigensolver.
+//
+// Section 3 of "A JoLT for the KV Cache" ("Partial Tucker backbone") needs the
+// mode-k singular values and vectors of the token unfolding X_(T) (T x N,
+// N = L_g H D) and of the feature unfolding X_(d) (D x L_g H T). They are
+// the eigenpairs of the Gram matrices X_(T) X_(T)^T (or X_(T)^T X_(T) when
+// T > N) and X_(d) X_(d)^T, formed here in fp64 from the fp32 cell values.
+#include "jolt_internal.cuh"
+#include "jolt_kernels.cuh"
+
+namespace jolt {
+
+// ------------------------------------------------------------ reductions ---
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Sum over the block; every thread gets the result. `red` >= 32 doubles.
+__device__ double block_sum(double v, double* red) {
+  int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  double s = 0.0;
+  for (int i = 0; i < nw; ++i) s += red[i];   // fixed order
+  return s;
+}
+
+// ---------------------------------------------------- feature Gram (fp64) --
+// partial[(cell*nchunk + chunk)*(D*D+1) + i*D + j] = sum over the chunk's rows
+// of x_i x_j; entry D*D holds the chunk's sum of squares. Rows are (l, h, t).
+template <int D>
+__global__ void __launch_bounds__(256) k_fgram_x(const CellDesc* __restrict__ cells,
+                                                 const float2* __restrict__ cs, int nchunk,
+                                                 double* __restrict__ partial) {
+  constexpr int RB = 32;               // rows per smem tile
+  constexpr int P = D / 16;            // outputs per thread per dim
+  __shared__ double xs[RB][D];
+  __shared__ double red[32];
+  const CellDesc c = cells[blockIdx.y];
+  const int64_t rows = (int64_t)c.Lg * c.H * c.T;
+  const int64_t per = (rows + nchunk - 1) / nchunk;
+  const int64_t r0 = blockIdx.x * per;
+  const int64_t r1 = min(rows, r0 + per);
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  double acc[P][P];
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+#pragma unroll
+    for (int j = 0; j < P; ++j) acc[i][j] = 0.0;
+  double sq = 0.0;
+  for (int64_t rb = r0; rb < r1; rb += RB) {
+    for (int e = threadIdx.x; e < RB * D; e += blockDim.x) {
+      int rr = e / D, d = e % D;
+      int64_t r = rb + rr;
+      double val = 0.0;
+      if (r < r1) {
+        int t = (int)(r % c.T);
+        int lh = (int)(r / c.T);
+        val = (double)x_elem(c, cs, lh / c.H, lh % c.H, t, d);
+      }
+      xs[rr][d] = val;
+      sq += val * val;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int k = 0; k < RB; ++k) {
+      double a[P], b[P];
+#pragma unroll
+      for (int i = 0; i < P; ++i) a[i] = xs[k][ty * P + i];
+#pragma unroll
+      for (int j = 0; j < P; ++j) b[j] = xs[k][tx * P + j];
+#pragma unroll
+      for (int i = 0; i < P; ++i)
+#pragma unroll
+        for (int j = 0; j < P; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  double* out = partial + ((int64_t)blockIdx.y * nchunk + blockIdx.x) * (D * D + 1);
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+#pragma unroll
+    for (int j = 0; j < P; ++j) out[(ty * P + i) * D + tx * P + j] = acc[i][j];
+  double s = block_sum(sq, red);
+  if (threadIdx.x == 0) out[D * D] = s;
+}
+
+// Same for rows of an fp64 matrix set: rows of Y[cell] = [L_g H][rmax][D],
+// only r < r_t(cell) counted.
+template <int D>
+__global__ void __launch_bounds__(256) k_fgram_rows(const double* const* __restrict__ Y,
+                                                    const int* __restrict__ nrow_used,
+                                                    const int* __restrict__ rmax_of, const int* __restrict__ nlh_of,
+                                                    int nchunk, double* __restrict__ partial) {
+  constexpr int RB = 32;
+  constexpr int P = D / 16;
+  __shared__ double xs[RB][D];
+  const int cell = blockIdx.y;
+  const double* src = Y[cell];
+  const int rmax = rmax_of[cell], ru = nrow_used[cell], nlh = nlh_of[cell];
+  const int64_t rows = (int64_t)nlh * rmax;
+  const int64_t per = (rows + nchunk - 1) / nchunk;
+  const int64_t r0 = blockIdx.x * per;
+  const int64_t r1 = min(rows, r0 + per);
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  double acc[P][P];
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+#pragma unroll
+    for (int j = 0; j < P; ++j) acc[i][j] = 0.0;
+  for (int64_t rb = r0; rb < r1; rb += RB) {
+    for (int e = threadIdx.x; e < RB * D; e += blockDim.x) {
+      int rr = e / D, d = e % D;
+      int64_t r = rb + rr;
+      double val = 0.0;
+      if (r < r1 && (int)(r % rmax) < ru) val = src[r * D + d];
+      xs[rr][d] = val;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int k = 0; k < RB; ++k) {
+      double a[P], b[P];
+#pragma unroll
+      for (int i = 0; i < P; ++i) a[i] = xs[k][ty * P + i];
+#pragma unroll
+      for (int j = 0; j < P; ++j) b[j] = xs[k][tx * P + j];
+#pragma unroll
+      for (int i = 0; i < P; ++i)
+#pragma unroll
+        for (int j = 0; j < P; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  double* out = partial + ((int64_t)cell * nchunk + blockIdx.x) * (D * D + 1);
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+#pragma unroll
+    for (int j = 0; j < P; ++j) out[(ty * P + i) * D + tx * P + j] = acc[i][j];
+  if (threadIdx.x == 0) out[D * D] = 0.0;
+}
+
+// out[cell][k] = sum over chunks (in chunk order) of partial[cell][chunk][k]
+__global__ void k_sum_chunks(const double* __restrict__ partial, int nchunk, int len,
+                             double* const* __restrict__ out, double* const* __restrict__ out_last) {
+  const int cell = blockIdx.y;
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < len; k += gridDim.x * blockDim.x) {
+    double s = 0.0;
+    for (int ch = 0; ch < nchunk; ++ch) s += partial[((int64_t)cell * nchunk + ch) * len + k];
+    if (k < len - 1) out[cell][k] = s;
+    else if (out_last) *out_last[cell] = s;
+  }
+}
+
+// ------------------------------------------------------ token Gram (fp64) --
+// Small side Gram of X_(T): if T <= N, G[t1][t2] = sum_n x(t1,n) x(t2,n);
+// else G[n1][n2] = sum_t x(t,n1) x(t,n2). n = (l*H + h)*D + d.
+__global__ void __launch_bounds__(256) k_token_gram(const CellDesc* __restrict__ cells,
+                                                    const float2* __restrict__ cs,
+                                                    double* const* __restrict__ G) {
+  constexpr int TB = 64, KB = 16;
+  __shared__ double As[KB][TB + 1];
+  __shared__ double Bs[KB][TB + 1];
+  const CellDesc c = cells[blockIdx.y];
+  const int N = c.Lg * c.H * c.D;
+  const bool tside = c.T <= N;
+  const int n = tside ? c.T : N;
+  const int K = tside ? N : c.T;
+  const int nt = (n + TB - 1) / TB;
+  // upper-triangular tile (ti <= tj) from the linear block index
+  int b = blockIdx.x, ti = 0;
+  while (ti < nt && b >= nt - ti) { b -= nt - ti; ++ti; }
+  if (ti >= nt) return;
+  const int tj = ti + b;
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  double acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+  for (int k0 = 0; k0 < K; k0 += KB) {
+    for (int e = threadIdx.x; e < KB * TB; e += blockDim.x) {
+      int kk = e / TB, ii = e % TB;
+      int k = k0 + kk;
+      int ia = ti * TB + ii, ib = tj * TB + ii;
+      double va = 0.0, vb = 0.0;
+      if (k < K) {
+        if (tside) {
+          int lh = k / c.D, d = k % c.D;
+          if (ia < n) va = x_elem(c, cs, lh / c.H, lh % c.H, ia, d);
+          if (ib < n) vb = x_elem(c, cs, lh / c.H, lh % c.H, ib, d);
+        } else {
+          if (ia < n) { int lh = ia / c.D; va = x_elem(c, cs, lh / c.H, lh % c.H, k, ia % c.D); }
+          if (ib < n) { int lh = ib / c.D; vb = x_elem(c, cs, lh / c.H, lh % c.H, k, ib % c.D); }
+        }
+      }
+      As[kk][ii] = va;
+      Bs[kk][ii] = vb;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < KB; ++kk) {
+      double a[4], bb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bb[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], bb[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  double* g = G[blockIdx.y];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int r = ti * TB + ty * 4 + i, q = tj * TB + tx * 4 + j;
+      if (r < n && q < n) {
+        g[(int64_t)r * n + q] = acc[i][j];
+        g[(int64_t)q * n + r] = acc[i][j];
+      }
+    }
+}
+
+// ------------------------------------------------------------ eigensolver --
+// One thread block per symmetric matrix A (n x n, row-major, destroyed):
+//  1. Householder reduction to tridiagonal form, A = Q T Q^T,
+//     Q = H_0 H_1 ... H_{n-3}, H_k = I - beta_k v_k v_k^T on rows k+1..n-1;
+//  2. implicit QL iterations with Wilkinson-type shifts on T; one thread
+//     computes each sweep's plane rotations and the whole block applies them
+//     to the eigenvector matrix, each thread owning rows;
+//  3. back-transformation z <- H_k z for k = n-3 .. 0;
+//  4. eigenvalues sorted descending, each eigenvector's largest-magnitude
+//     entry made positive (first on ties).
+// Outputs: w[n]; Vt[j*n + i] = component i of eigenvector j (if want_vec).
+constexpr int EIG_THREADS = 512;
+
+__global__ void __launch_bounds__(EIG_THREADS) k_eigh(const EighJob* __restrict__ jobs, int* status) {
+  const EighJob J = jobs[blockIdx.x];
+  const int n = J.n;
+  if (n <= 0) return;
+  extern __shared__ double sh[];
+  double* v = sh;            // n
+  double* p = v + n;         // n
+  double* dd = p + n;        // n   diagonal
+  double* ee = dd + n;       // n   off-diagonal
+  double* rc = ee + n;       // n   rotation cosines of the current sweep
+  double* rs = rc + n;       // n   rotation sines
+  double* red = rs + n;      // 32
+  __shared__ int ctl[4];
+  double* A = J.A;
+  double* tau = J.work;      // n
+  double* Z = J.Z;           // Z[j*n + i] = component i of vector j
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5, nwarp = nt >> 5;
+
+  // ---- 1. tridiagonalization
+  for (int k = 0; k + 2 < n; ++k) {
+    const int m = n - k - 1;
+    for (int i = tid; i < m; i += nt) v[i] = A[(int64_t)(k + 1 + i) * n + k];
+    __syncthreads();
+    double s = 0.0;
+    for (int i = 1 + tid; i < m; i += nt) s += v[i] * v[i];
+    s = block_sum(s, red);
+    const double x0 = v[0];
+    if (s == 0.0) {
+      if (tid == 0) { dd[k] = A[(int64_t)k * n + k]; ee[k] = x0; tau[k] = 0.0; }
+      __syncthreads();
+      continue;
+    }
+    const double nrm = sqrt(x0 * x0 + s);
+    const double alpha = (x0 <= 0.0) ? nrm : -nrm;
+    const double v0 = x0 - alpha;
+    const double beta = 2.0 / (s + v0 * v0);
+    __syncthreads();
+    if (tid == 0) v[0] = v0;
+    __syncthreads();
+    // p = beta A22 v
+    for (int i = warp; i < m; i += nwarp) {
+      const double* row = A + (int64_t)(k + 1 + i) * n + (k + 1);
+      double acc = 0.0;
+      for (int j = lane; j < m; j += 32) acc += row[j] * v[j];
+      acc = warp_sum(acc);
+      if (lane == 0) p[i] = beta * acc;
+    }
+    __syncthreads();
+    double pv = 0.0;
+    for (int i = tid; i < m; i += nt) pv += p[i] * v[i];
+    const double Kc = 0.5 * beta * block_sum(pv, red);
+    for (int i = tid; i < m; i += nt) p[i] -= Kc * v[i];
+    __syncthreads();
+    // A22 -= v w^T + w v^T
+    for (int i = warp; i < m; i += nwarp) {
+      double* row = A + (int64_t)(k + 1 + i) * n + (k + 1);
+      const double vi = v[i], wi = p[i];
+      for (int j = lane; j < m; j += 32) row[j] -= vi * p[j] + wi * v[j];
+    }
+    if (tid == 0) { dd[k] = A[(int64_t)k * n + k]; ee[k] = alpha; tau[k] = beta; }
+    for (int i = tid; i < m; i += nt) A[(int64_t)(k + 1 + i) * n + k] = v[i];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    if (n >= 2) {
+      dd[n - 2] = A[(int64_t)(n - 2) * n + (n - 2)];
+      ee[n - 2] = A[(int64_t)(n - 1) * n + (n - 2)];
+    }
+    dd[n - 1] = A[(int64_t)(n - 1) * n + (n - 1)];
+    ee[n - 1] = 0.0;
+  }
+  if (J.want_vec)
+    for (int64_t e = tid; e < (int64_t)n * n; e += nt) Z[e] = ((e / n) == (e % n)) ? 1.0 : 0.0;
+  __syncthreads();
+
+  // ---- 2. implicit QL
+  for (int l = 0; l < n; ++l) {
+    int iter = 0;
+    while (true) {
+      if (tid == 0) {
+        int m = l;
+        for (; m < n - 1; ++m) {
+          double s2 = fabs(dd[m]) + fabs(dd[m + 1]);
+          if (fabs(ee[m]) <= 2.220446049250313e-16 * s2) break;
+        }
+        if (m == l) {
+          ctl[0] = 1;
+        } else if (++iter > 90) {
+          atomicOr(status, DEV_ERR_EIG_NOCONV);
+          ctl[0] = 1;
+        } else {
+          double g = (dd[l + 1] - dd[l]) / (2.0 * ee[l]);
+          double r = hypot(g, 1.0);
+          g = dd[m] - dd[l] + ee[l] / (g + copysign(r, g));
+          double s = 1.0, cc = 1.0, pp = 0.0;
+          int i = m - 1;
+          bool early = false;
+          for (; i >= l; --i) {
+            double f = s * ee[i], b = cc * ee[i];
+            r = hypot(f, g);
+            ee[i + 1] = r;
+            if (r == 0.0) { dd[i + 1] -= pp; ee[m] = 0.0; early = true; break; }
+            s = f / r;
+            cc = g / r;
+            g = dd[i + 1] - pp;
+            r = (dd[i] - g) * s + 2.0 * cc * b;
+            pp = s * r;
+            dd[i + 1] = g + pp;
+            g = cc * r - b;
+            rc[i] = cc;
+            rs[i] = s;
+          }
+          if (!early) { dd[l] -= pp; ee[l] = g; ee[m] = 0.0; ctl[2] = l; }
+          else ctl[2] = i + 1;
+          ctl[0] = 0;
+          ctl[1] = m - 1;
+        }
+      }
+      __syncthreads();
+      if (ctl[0]) { __syncthreads(); break; }
+      if (J.want_vec) {
+        const int hi = ctl[1], lo = ctl[2];
+        for (int r = tid; r < n; r += nt) {
+          double z1 = Z[(int64_t)(hi + 1) * n + r];
+          for (int i = hi; i >= lo; --i) {
+            double zi = Z[(int64_t)i * n + r];
+            Z[(int64_t)(i + 1) * n + r] = rs[i] * zi + rc[i] * z1;
+            z1 = rc[i] * zi - rs[i] * z1;
+          }
+          if (hi >= lo) Z[(int64_t)lo * n + r] = z1;
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // ---- 3. back-transformation
+  if (J.want_vec) {
+    for (int k = n - 3; k >= 0; --k) {
+      const double beta = tau[k];
+      if (beta == 0.0) continue;
+      const int m = n - k - 1;
+      for (int i = tid; i < m; i += nt) v[i] = A[(int64_t)(k + 1 + i) * n + k];
+      __syncthreads();
+      for (int j = warp; j < n; j += nwarp) {
+        double* z = Z + (int64_t)j * n + (k + 1);
+        double acc = 0.0;
+        for (int i = lane; i < m; i += 32) acc += v[i] * z[i];
+        acc = beta * warp_sum(acc);
+        for (int i = lane; i < m; i += 32) z[i] -= acc * v[i];
+      }
+      __syncthreads();
+    }
+  }
+
+  // ---- 4. sort descending, fix signs, write out
+  for (int i = tid; i < n; i += nt) {
+    const double di = dd[i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) {
+      const double dj = dd[j];
+      rank += (dj > di) || (dj == di && j < i);
+    }
+    J.w[rank] = di;
+    p[i] = (double)rank;
+  }
+  __syncthreads();
+  if (J.want_vec) {
+    for (int j = warp; j < n; j += nwarp) {
+      const double* z = Z + (int64_t)j * n;
+      double best = -1.0;
+      int bi = 0x7fffffff;
+      for (int i = lane; i < n; i += 32) {
+        double a = fabs(z[i]);
+        if (a > best) { best = a; bi = i; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        double ob = __shfl_xor_sync(0xffffffffu, best, o);
+        int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+      }
+      const double sg = (z[bi] < 0.0) ? -1.0 : 1.0;
+      const int rank = (int)p[j];
+      double* dst = J.Vt + (int64_t)rank * n;
+      for (int i = lane; i < n; i += 32) dst[i] = sg * z[i];
+    }
+  }
+}
+
+size_t eigh_smem_bytes(int nmax) { return (size_t)(6 * nmax + 32) * sizeof(double); }
+
+jolt_status launch_eigh(const EighJob* jobs_dev, int njobs, int nmax, int* status, cudaStream_t s) {
+  size_t smem = eigh_smem_bytes(nmax);
+  JOLT_CUDA_TRY(cudaFuncSetAttribute(k_eigh, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  k_eigh<<<njobs, EIG_THREADS, smem, s>>>(jobs_dev, status);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+jolt_status launch_fgram_x(const CellDesc* cells, int ncells, int D, const float2* cs, int nchunk,
+                           double* partial, cudaStream_t s) {
+  dim3 grid(nchunk, ncells);
+  if (D == 128) k_fgram_x<128><<<grid, 256, 0, s>>>(cells, cs, nchunk, partial);
+  else k_fgram_x<64><<<grid, 256, 0, s>>>(cells, cs, nchunk, partial);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+jolt_status launch_fgram_rows(const double* const* Y, const int* nrow_used, const int* rmax_of,
+                              const int* nlh_of, int ncells, int D, int nchunk, double* partial,
+                              cudaStream_t s) {
+  dim3 grid(nchunk, ncells);
+  if (D == 128) k_fgram_rows<128><<<grid, 256, 0, s>>>(Y, nrow_used, rmax_of, nlh_of, nchunk, partial);
+  else k_fgram_rows<64><<<grid, 256, 0, s>>>(Y, nrow_used, rmax_of, nlh_of, nchunk, partial);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+jolt_status launch_sum_chunks(const double* partial, int nchunk, int len, int ncells,
+                              double* const* out, double* const* out_last, cudaStream_t s) {
+  dim3 grid((len + 255) / 256, ncells);
+  k_sum_chunks<<<grid, 256, 0, s>>>(partial, nchunk, len, out, out_last);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+jolt_status launch_token_gram(const CellDesc* cells, int ncells, int nmax, const float2* cs,
+                              double* const* G, cudaStream_t s) {
+  int nt = (nmax + 63) / 64;
+  dim3 grid(nt * (nt + 1) / 2, ncells);
+  k_token_gram<<<grid, 256, 0, s>>>(cells, cs, G);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+}  // namespace jolt

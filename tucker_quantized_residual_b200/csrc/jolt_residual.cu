@@ -1,0 +1,248 @@
+// Rotated low-bit residual and decompression ("A JoLT for the KV Cache",
+// Section 3, "Rotated low-bit residual"): E = X - X~, r = R E along the
+// feature axis with R = D^-1/2 H_D diag(s) (seeded randomized Hadamard), per
+// group absmax quantization to b bits with one fp32 scale, LSB-first
+// packing; decoding dequantizes, applies R^T and adds the backbone
+// X~ = U_T^ M^_lh. Keys get RoPE re-applied after decoding.
+//
+// This file holds the row-per-thread (SIMT) forms: the backbone product is
+// accumulated in fp32 registers, the transform runs inside the thread.
+#include "jolt_internal.cuh"
+#include "jolt_kernels.cuh"
+
+namespace jolt {
+
+// fl32(1/sqrt(D)): the quotient and the root are correctly rounded in fp64, then
+// rounded once to fp32.
+__device__ __forceinline__ float rot_scale_f(int D) { return (float)(1.0 / sqrt((double)D)); }
+
+template <int D>
+__device__ __forceinline__ void rotate_row(float* e, const float* sgn) {
+#pragma unroll
+  for (int d = 0; d < D; ++d) e[d] = __fmul_rn(e[d], sgn[d]);
+  fwht_row<D>(e);
+  const float rs = rot_scale_f(D);
+#pragma unroll
+  for (int d = 0; d < D; ++d) e[d] = __fmul_rn(e[d], rs);
+}
+
+template <int D>
+__device__ __forceinline__ void unrotate_row(float* v, const float* sgn) {
+  fwht_row<D>(v);
+  const float rs = rot_scale_f(D);
+#pragma unroll
+  for (int d = 0; d < D; ++d) v[d] = __fmul_rn(__fmul_rn(v[d], rs), sgn[d]);
+}
+
+template <int D>
+struct PackOp {
+  float* e;
+  uint8_t* codes;   // row base
+  float* scales;    // row base
+  template <int G, int B>
+  __device__ __forceinline__ void run() { quantize_pack_row<D, G, B>(e, codes, scales); }
+};
+
+template <int D>
+struct UnpackOp {
+  float* v;
+  const uint8_t* codes;
+  const float* scales;
+  template <int G, int B>
+  __device__ __forceinline__ void run() { unpack_dequant_row<D, G, B>(codes, scales, v); }
+};
+
+// X~ row t of (cell, lh) accumulated in fp32: acc[d] = sum_r U_T^[t][r] M^[r][d]
+template <int D>
+__device__ __forceinline__ void backbone_rows(const ResidArgs& a, int cell, const CellOut& o, int lh,
+                                              int t0, float* acc, float (*ms)[D], float (*us)[128]) {
+  const int rmax = a.rmax_of[cell];
+  const uint16_t* M = a.M[cell] + (int64_t)lh * rmax * D;
+#pragma unroll
+  for (int d = 0; d < D; ++d) acc[d] = 0.0f;
+  for (int r0 = 0; r0 < o.rT; r0 += 32) {
+    for (int e = threadIdx.x; e < 32 * D; e += blockDim.x) {
+      int rr = e / D, d = e % D;
+      ms[rr][d] = (r0 + rr < o.rT) ? bf16_bits_to_f32(M[(int64_t)(r0 + rr) * D + d]) : 0.0f;
+    }
+    for (int e = threadIdx.x; e < 32 * 128; e += blockDim.x) {
+      int rr = e / 128, tt = e % 128;
+      int t = t0 + tt;
+      us[rr][tt] = (r0 + rr < o.rT && t < o.t_pitch) ? bf16_bits_to_f32(o.ut[(int64_t)(r0 + rr) * o.t_pitch + t]) : 0.0f;
+    }
+    __syncthreads();
+    for (int rr = 0; rr < 32; ++rr) {
+      const float u = us[rr][threadIdx.x];
+#pragma unroll
+      for (int d = 0; d < D; ++d) acc[d] = fmaf(u, ms[rr][d], acc[d]);
+    }
+    __syncthreads();
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) k_residual_simt(ResidArgs a) {
+  const int cell = blockIdx.z, lh = blockIdx.y, t0 = blockIdx.x * 128;
+  const CellDesc c = a.cells[cell];
+  const CellOut o = a.out[cell];
+  if (o.b == 0 || lh >= c.Lg * c.H || t0 >= c.T) return;
+  __shared__ float ms[32][D];
+  __shared__ float us[32][128];
+  __shared__ float sg[D];
+  for (int d = threadIdx.x; d < D; d += blockDim.x) sg[d] = hadamard_sign(a.seed + c.seq, d);
+  __syncthreads();
+  float acc[D];
+  backbone_rows<D>(a, cell, o, lh, t0, acc, ms, us);
+  const int t = t0 + threadIdx.x;
+  if (t >= c.T) return;
+  const int l = lh / c.H, h = lh % c.H;
+#pragma unroll
+  for (int d = 0; d < D; ++d) acc[d] = __fsub_rn(x_elem(c, a.cs, l, h, t, d), acc[d]);
+  rotate_row<D>(acc, sg);
+  const int64_t row = (int64_t)lh * c.T + t;
+  PackOp<D> op{acc, o.codes + row * (o.b * D / 8), o.scales + row * (D / a.G)};
+  dispatch_gb<D>(a.G, o.b, op);
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) k_decompress_simt(ResidArgs a) {
+  const int cell = blockIdx.z, lh = blockIdx.y, t0 = blockIdx.x * 128;
+  const CellDesc c = a.cells[cell];
+  const CellOut o = a.out[cell];
+  if (lh >= c.Lg * c.H || t0 >= c.T) return;
+  __shared__ float ms[32][D];
+  __shared__ float us[32][128];
+  __shared__ float sg[D];
+  for (int d = threadIdx.x; d < D; d += blockDim.x) sg[d] = hadamard_sign(a.seed + c.seq, d);
+  __syncthreads();
+  float acc[D];
+  backbone_rows<D>(a, cell, o, lh, t0, acc, ms, us);
+  const int t = t0 + threadIdx.x;
+  if (t >= c.T) return;
+  const int l = lh / c.H, h = lh % c.H;
+  if (o.b > 0) {
+    float v[D];
+    const int64_t row = (int64_t)lh * c.T + t;
+    UnpackOp<D> op{v, o.codes + row * (o.b * D / 8), o.scales + row * (D / a.G)};
+    dispatch_gb<D>(a.G, o.b, op);
+    unrotate_row<D>(v, sg);
+#pragma unroll
+    for (int d = 0; d < D; ++d) acc[d] = __fadd_rn(acc[d], v[d]);
+  }
+  if (c.rope) {
+    constexpr int half = D / 2;
+    const float2* cs = a.cs + (int64_t)t * half;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float2 q = cs[i];
+      const float x0 = acc[i], x1 = acc[i + half];
+      acc[i] = __fsub_rn(__fmul_rn(x0, q.x), __fmul_rn(x1, q.y));
+      acc[i + half] = __fadd_rn(__fmul_rn(x1, q.x), __fmul_rn(x0, q.y));
+    }
+  }
+  uint16_t* dst = (c.kind == 0 ? a.out_k : a.out_v) + (int64_t)c.seq * a.osb + (int64_t)(c.l0 + l) * a.osl +
+                  (int64_t)h * a.osh + (int64_t)t * a.ost;
+#pragma unroll
+  for (int d = 0; d < D; d += 2) {
+    uint32_t lo = bf16_bits_from_f32(acc[d]), hi = bf16_bits_from_f32(acc[d + 1]);
+    *reinterpret_cast<uint32_t*>(dst + d) = lo | (hi << 16);
+  }
+}
+
+jolt_status launch_residual_simt(const ResidArgs& a, int ncells, int D, int Tmax, int lh_max,
+                                 cudaStream_t s) {
+  dim3 g((Tmax + 127) / 128, lh_max, ncells);
+  if (D == 128) k_residual_simt<128><<<g, 128, 0, s>>>(a);
+  else k_residual_simt<64><<<g, 128, 0, s>>>(a);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+jolt_status launch_decompress_simt(const ResidArgs& a, int ncells, int D, int Tmax, int lh_max,
+                                   cudaStream_t s) {
+  dim3 g((Tmax + 127) / 128, lh_max, ncells);
+  if (D == 128) k_decompress_simt<128><<<g, 128, 0, s>>>(a);
+  else k_decompress_simt<64><<<g, 128, 0, s>>>(a);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// ------------------------------------------------ residual stage alone -----
+template <int D>
+__global__ void __launch_bounds__(128) k_encode_rows(const float* __restrict__ e, int64_t rows, int b,
+                                                     int G, uint64_t seed, uint8_t* codes, float* scales) {
+  __shared__ float sg[D];
+  for (int d = threadIdx.x; d < D; d += blockDim.x) sg[d] = hadamard_sign(seed, d);
+  __syncthreads();
+  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= rows) return;
+  float v[D];
+#pragma unroll
+  for (int d = 0; d < D; d += 4) {
+    float4 q = *reinterpret_cast<const float4*>(e + row * D + d);
+    v[d] = q.x; v[d + 1] = q.y; v[d + 2] = q.z; v[d + 3] = q.w;
+  }
+  rotate_row<D>(v, sg);
+  PackOp<D> op{v, codes + row * (b * D / 8), scales + row * (D / G)};
+  dispatch_gb<D>(G, b, op);
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) k_decode_rows(const uint8_t* __restrict__ codes,
+                                                     const float* __restrict__ scales, int64_t rows,
+                                                     int b, int G, uint64_t seed, float* e) {
+  __shared__ float sg[D];
+  for (int d = threadIdx.x; d < D; d += blockDim.x) sg[d] = hadamard_sign(seed, d);
+  __syncthreads();
+  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= rows) return;
+  float v[D];
+  UnpackOp<D> op{v, codes + row * (b * D / 8), scales + row * (D / G)};
+  dispatch_gb<D>(G, b, op);
+  unrotate_row<D>(v, sg);
+#pragma unroll
+  for (int d = 0; d < D; d += 4)
+    *reinterpret_cast<float4*>(e + row * D + d) = make_float4(v[d], v[d + 1], v[d + 2], v[d + 3]);
+}
+
+jolt_status launch_encode_rows(const float* e, int64_t rows, int D, int b, int G, uint64_t seed,
+                               uint8_t* codes, float* scales, cudaStream_t s) {
+  if (rows <= 0) return JOLT_OK;
+  int64_t nb = (rows + 127) / 128;
+  if (D == 128) k_encode_rows<128><<<(unsigned)nb, 128, 0, s>>>(e, rows, b, G, seed, codes, scales);
+  else k_encode_rows<64><<<(unsigned)nb, 128, 0, s>>>(e, rows, b, G, seed, codes, scales);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+jolt_status launch_decode_rows(const uint8_t* codes, const float* scales, int64_t rows, int D,
+                               int b, int G, uint64_t seed, float* e, cudaStream_t s) {
+  if (rows <= 0) return JOLT_OK;
+  int64_t nb = (rows + 127) / 128;
+  if (D == 128) k_decode_rows<128><<<(unsigned)nb, 128, 0, s>>>(codes, scales, rows, b, G, seed, e);
+  else k_decode_rows<64><<<(unsigned)nb, 128, 0, s>>>(codes, scales, rows, b, G, seed, e);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// ------------------------------------------------------------ RoPE table ---
+__global__ void k_rope_table(int T, int D, double theta, float2* cs) {
+  const int half = D / 2;
+  const int64_t n = (int64_t)T * half;
+  for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < n; k += (int64_t)gridDim.x * blockDim.x) {
+    int t = (int)(k / half), i = (int)(k % half);
+    double inv = pow(theta, -2.0 * (double)i / (double)D);
+    double ang = (double)t * inv;
+    cs[k] = make_float2((float)cos(ang), (float)sin(ang));
+  }
+}
+
+jolt_status launch_rope_table(int T, int D, double theta, float2* cs, cudaStream_t s) {
+  int64_t n = (int64_t)T * (D / 2);
+  int nb = (int)std::min<int64_t>((n + 255) / 256, 4096);
+  k_rope_table<<<nb, 256, 0, s>>>(T, D, theta, cs);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+}  // namespace jolt
