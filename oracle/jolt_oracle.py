@@ -47,6 +47,8 @@ library as well):
   R7 sign of every singular/eigen vector: its largest-magnitude entry is
      positive (first such entry on ties).
   R8 budget C: B = floor(dense bf16 bytes of K and V / C).
+  R9 an option with r_d > |g| n_h r_T is excluded (multilinear rank of the
+     core; see CellTable.valid).
 """
 from __future__ import annotations
 
@@ -386,15 +388,27 @@ class CellTable:
         for bi, b in enumerate(self.bits):
             for rT in self.rt_grid:
                 for rd in self.rd_grid:
+                    if not self.valid(rT, rd):
+                        continue
                     e = float(self.eps2[bi]) * (float(self.tT[rT]) + float(self.tD[rd]))
                     s = cost_bytes(self.Lg, self.H, self.T, self.D, int(rT), int(rd), int(b), self.g)
                     yield int(b), int(rT), int(rd), e, s
 
+    def valid(self, rT, rd):
+        """Reading R9: the core G in R^{|g| x n_h x r_T x r_d} comes from the
+        token-projected tensor, whose feature unfolding has rank at most
+        |g| n_h r_T, so an option with r_d > |g| n_h r_T is not a partial Tucker
+        decomposition of that rank (its extra feature columns would be an
+        arbitrary null-space basis); such options are excluded."""
+        return rd <= self.Lg * self.H * rT
+
     def arrays(self):
-        """All options as arrays (same enumeration order)."""
+        """All options as arrays (same enumeration order); excluded options
+        carry e = +inf so that no multiplier selects them."""
         bb, tt, dd = np.meshgrid(self.bits, self.rt_grid, self.rd_grid, indexing="ij")
         ei = np.broadcast_to(self.eps2[:, None, None], bb.shape)
         e = ei * (self.tT[tt] + self.tD[dd])
+        e = np.where(self.valid(tt, dd), e, np.inf)
         rb = np.array([residual_row_bytes(int(x), self.D, self.g) for x in self.bits], dtype=np.int64)
         rbb = np.broadcast_to(rb[:, None, None], bb.shape)
         s = (self.Lg * self.H * tt * dd + self.T * tt + self.D * dd) * 2 + rbb * (self.Lg * self.H * self.T)
@@ -478,7 +492,7 @@ def greedy_cell(tab: CellTable, lam: float) -> Tuple[int, int, int, float]:
                 v1, e1, s1 = val(rT + 1, rd)
                 if v1 < v0:
                     cands.append(((e0 - e1) / (s1 - s0), 0))
-            if rd < rmaxD:
+            if rd < rmaxD and tab.valid(rT, rd + 1):
                 v2, e2, s2 = val(rT, rd + 1)
                 if v2 < v0:
                     cands.append(((e0 - e2) / (s2 - s0), 1))

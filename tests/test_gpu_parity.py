@@ -202,7 +202,10 @@ def _compare(K, V, gs, B, rope=0.0, **kw):
     got = [(c.r_t, c.r_d, c.bits) for c in cells]
     assert got == comp.alloc.choice
     assert nbytes == sum(comp.alloc.bytes) and nbytes <= B
-    assert lam == comp.alloc.lam and it == comp.alloc.iters
+    # the spectra come from another eigensolver (agreement ~1e-13), so lambda,
+    # resolved by 50 halvings of its log-bracket, agrees to that level only;
+    # with identical tables it is bit-exact (test_allocation_* above)
+    assert abs(lam - comp.alloc.lam) <= 1e-9 * comp.alloc.lam and it == comp.alloc.iters
     assert rel(Kh, Ko) <= RTOL_RECON, rel(Kh, Ko)
     assert rel(Vh, Vo) <= RTOL_RECON, rel(Vh, Vo)
     eK, eV = o.rel_frobenius(Kn, Kh), o.rel_frobenius(Vn, Vh)

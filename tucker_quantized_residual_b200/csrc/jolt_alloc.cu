@@ -165,7 +165,11 @@ __device__ __forceinline__ int64_t opt_bytes(const AllocArgs& a, const CellRD& c
   return 2 * (LH * rt * rd + (int64_t)c.T * rt + (int64_t)c.D * rd) + a.rowbytes[bi] * LH * c.T;
 }
 
+// Eq. (2). An option whose feature rank exceeds |g| n_h r_T is excluded
+// (+inf): the token-projected tensor has feature rank at most |g| n_h r_T, so
+// extra feature columns would be an arbitrary null-space basis.
 __device__ __forceinline__ double opt_err(const AllocArgs& a, const CellRD& c, int bi, int rt, int rd) {
+  if (rd > c.Lg * c.H * rt) return INFINITY;
   return __dmul_rn(a.eps2[bi], __dadd_rn(c.tT[rt], c.tD[rd]));
 }
 

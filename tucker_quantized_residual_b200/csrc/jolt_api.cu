@@ -274,13 +274,21 @@ jolt_status jolt_plan(const jolt_layout* L, int64_t byte_budget, const jolt_opti
     for (int r : p->rt_grid) if (r <= c.rmax) ++c.n_rt;
     if (c.n_rt == 0) { delete p; set_error("rt grid has no value within the token-rank bound"); return JOLT_ERR_INVALID_ARG; }
     c.rmax = p->rt_grid[c.n_rt - 1];
-    // cheapest option
+    // cheapest admissible option (r_d <= L_g*H*r_T)
     int64_t best = INT64_MAX;
-    for (size_t bi = 0; bi < p->bits.size(); ++bi) {
-      int64_t LH = (int64_t)c.Lg * p->H;
-      int rt = p->rt_grid[0], rd = p->rd_grid[0];
-      int64_t s = 2 * (LH * rt * rd + (int64_t)p->T * rt + (int64_t)p->D * rd) + p->rowbytes[bi] * LH * p->T;
-      best = std::min(best, s);
+    const int64_t LH = (int64_t)c.Lg * p->H;
+    for (size_t bi = 0; bi < p->bits.size(); ++bi)
+      for (int ti = 0; ti < c.n_rt; ++ti) {
+        const int rt = p->rt_grid[ti];
+        const int rd = p->rd_grid[0];
+        if (rd > LH * rt) continue;
+        int64_t s = 2 * (LH * rt * rd + (int64_t)p->T * rt + (int64_t)p->D * rd) + p->rowbytes[bi] * LH * p->T;
+        best = std::min(best, s);
+      }
+    if (best == INT64_MAX) {
+      delete p;
+      set_error("no admissible (r_t, r_d) pair: every r_d exceeds L_g*H*r_t");
+      return JOLT_ERR_INVALID_ARG;
     }
     c.min_bytes = best;
     p->nmin_max = std::max(p->nmin_max, c.nmin);

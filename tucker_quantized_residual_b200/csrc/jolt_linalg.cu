@@ -318,6 +318,13 @@ __global__ void __launch_bounds__(EIG_THREADS) k_eigh(const EighJob* __restrict_
   __syncthreads();
 
   // ---- 2. implicit QL
+  // A sub-diagonal entry is negligible when it is tiny next to its two
+  // diagonal neighbours or next to the whole matrix (norm bound anorm); the
+  // second test deflates clusters of (numerically) zero eigenvalues, which a
+  // purely relative test would iterate on forever.
+  double anorm = 0.0;
+  if (tid == 0)
+    for (int i = 0; i < n; ++i) anorm = fmax(anorm, fabs(dd[i]) + fabs(ee[i]));
   for (int l = 0; l < n; ++l) {
     int iter = 0;
     while (true) {
@@ -325,7 +332,7 @@ __global__ void __launch_bounds__(EIG_THREADS) k_eigh(const EighJob* __restrict_
         int m = l;
         for (; m < n - 1; ++m) {
           double s2 = fabs(dd[m]) + fabs(dd[m + 1]);
-          if (fabs(ee[m]) <= 2.220446049250313e-16 * s2) break;
+          if (fabs(ee[m]) <= 2.220446049250313e-16 * s2 || fabs(ee[m]) <= 2.220446049250313e-16 * anorm) break;
         }
         if (m == l) {
           ctl[0] = 1;
