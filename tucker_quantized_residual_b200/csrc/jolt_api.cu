@@ -10,6 +10,7 @@
 
 #include "jolt_internal.cuh"
 #include "jolt_kernels.cuh"
+#include "jolt_umma.cuh"
 
 namespace jolt {
 
@@ -79,7 +80,7 @@ struct jolt_plan_s {
   int64_t budget = 0;
   int G = 0, D = 0, T = 0, H = 0;
   double C = 0.0;
-  int qcap = 0, k = 0;
+  int qcap = 0;
   int ncells = 0, nmin_max = 0, rmax_all = 0, lh_max = 0, nt_max = 0;
   std::vector<HostCell> hc;
   std::vector<CellDesc> cdesc;
@@ -119,6 +120,20 @@ struct jolt_plan_s {
   std::vector<double*> h_tT, h_tD, h_wT, h_wD, h_nsq;
   std::vector<uint16_t*> h_M;
   void* ws_alloc = nullptr;
+  // randomized mode (Section 3.1): sketch width k = q + p rounded up to 16,
+  // GEMM tile width BN, padded extents, working buffers
+  int k = 0, BN = 0, nt_k = 0, kpad = 0, rpad = 0, tp = 0, Ncmax = 0, fg_chunks = 0, fg_spc = 0, q_used = 0;
+  bool copy_k = false, copy_v = false;
+  uint16_t* Xk = nullptr;  uint16_t* Xv = nullptr;
+  uint16_t* Wt = nullptr;  uint16_t* Yt = nullptr;  uint16_t* Pt = nullptr;
+  float* Z = nullptr;      float* GW32 = nullptr;   float* fgpart = nullptr;
+  double* Gz = nullptr;    double* Rm = nullptr;    double* P0 = nullptr;   double* X1 = nullptr;
+  double* MB = nullptr;    double* eZ = nullptr;    double* eVt = nullptr;  double* ew = nullptr;
+  double* ework = nullptr; double* trs = nullptr;   double* P64 = nullptr;
+  int* d_cl0 = nullptr; int* d_cb = nullptr; int* d_cLg = nullptr; int* d_ckind = nullptr;
+  int* d_Nc = nullptr; int* d_cis = nullptr;
+  uint16_t** d_utp = nullptr;
+  EighJob* d_jobs_rand = nullptr;
 };
 
 struct jolt_handle_s {
@@ -301,6 +316,32 @@ jolt_status jolt_plan(const jolt_layout* L, int64_t byte_budget, const jolt_opti
     set_error("exact mode needs min(T, L_g*H*D) <= 2048 (got %d); use JOLT_RANDOMIZED", p->nmin_max);
     return JOLT_ERR_UNSUPPORTED_SHAPE;
   }
+  if (rnd) {
+    int q = 0, nmin_all = INT32_MAX;
+    for (auto& c : p->hc) { q = std::max(q, c.nt - 1); nmin_all = std::min(nmin_all, c.nmin); p->Ncmax = std::max(p->Ncmax, c.N); }
+    p->q_used = q;
+    p->k = ((q + std::max(opt->oversample_p, 0) + 15) / 16) * 16;
+    if (p->k > nmin_all) {
+      delete p;
+      set_error("sketch width k=%d exceeds min(T, L_g*H*D)=%d; use JOLT_EXACT", q + opt->oversample_p, nmin_all);
+      return JOLT_ERR_UNSUPPORTED_SHAPE;
+    }
+    if (opt->power_iters < 0 || opt->power_iters > 8) { delete p; set_error("power_iters must be 0..8"); return JOLT_ERR_INVALID_ARG; }
+    const int ntile = (p->k + 255) / 256;
+    p->BN = (((p->k + ntile - 1) / ntile) + 15) / 16 * 16;
+    p->nt_k = (p->k + p->BN - 1) / p->BN;
+    p->kpad = (p->k + 63) / 64 * 64;
+    p->rpad = (p->rmax_all + 127) / 128 * 128;
+    p->tp = (p->T + 7) / 8 * 8;
+    const int steps = ((p->Ncmax + 127) / 128) * ((p->T + 63) / 64);
+    p->fg_spc = std::max(64, (steps + 31) / 32);
+    p->fg_chunks = (steps + p->fg_spc - 1) / p->fg_spc;
+    auto aligned = [&](int64_t st) { return st % 8 == 0; };
+    const bool tma_ok = L->dtype == JOLT_BF16 && aligned(L->stride_t) && aligned(L->stride_h) &&
+                        aligned(L->stride_l) && aligned(L->stride_b);
+    p->copy_k = !tma_ok || L->rope_theta_k > 0;
+    p->copy_v = !tma_ok;
+  }
   int64_t minsum = 0;
   for (auto& c : p->hc) minsum += c.min_bytes;
   if (byte_budget < minsum) {
@@ -356,6 +397,30 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
     p->d_api = A.take<int>((size_t)nc * p->achunk);
     p->d_cur = A.take<int>(nc);
     p->d_keep = A.take<int>(nc);
+    if (p->opt.mode == JOLT_RANDOMIZED) {
+      const int k = p->k;
+      const size_t kk = (size_t)k * k;
+      const jolt_layout& L = p->lay;
+      const size_t full = (size_t)L.batch * L.n_layers * p->H * T * D;
+      p->Xk = p->copy_k ? A.take<uint16_t>(full) : nullptr;
+      p->Xv = p->copy_v ? A.take<uint16_t>(full) : nullptr;
+      p->Wt = A.take<uint16_t>((size_t)nc * k * p->Ncmax);
+      p->Yt = A.take<uint16_t>((size_t)nc * k * p->tp);
+      p->Pt = A.take<uint16_t>((size_t)nc * p->rpad * p->kpad);
+      p->Z = A.take<float>((size_t)nc * p->Ncmax * k);
+      p->GW32 = A.take<float>((size_t)nc * kk);
+      p->fgpart = A.take<float>((size_t)nc * p->fg_chunks * 128 * 128);
+      p->Gz = A.take<double>(nc * kk); p->Rm = A.take<double>(nc * kk); p->P0 = A.take<double>(nc * kk);
+      p->X1 = A.take<double>(nc * kk); p->MB = A.take<double>(nc * kk); p->eZ = A.take<double>(nc * kk);
+      p->eVt = A.take<double>(nc * kk); p->ew = A.take<double>((size_t)nc * k);
+      p->ework = A.take<double>((size_t)nc * k);
+      p->trs = A.take<double>((size_t)nc * p->Ncmax * k);
+      p->P64 = A.take<double>((size_t)nc * k * p->rmax_all);
+      p->d_cl0 = A.take<int>(nc); p->d_cb = A.take<int>(nc); p->d_cLg = A.take<int>(nc);
+      p->d_ckind = A.take<int>(nc); p->d_Nc = A.take<int>(nc); p->d_cis = A.take<int>(nc);
+      p->d_utp = A.take<uint16_t*>(nc);
+      p->d_jobs_rand = A.take<EighJob>(2 * nc);
+    }
     // per-cell buffers
     std::vector<double*> GT(nc), ZT(nc), VtT(nc), wT(nc), Cd(nc), wD(nc), nsq(nc), tT(nc), tD(nc),
         Y(nc), CY(nc), VtY(nc), wY(nc), ZY(nc), Uf(nc), workT(nc), workD(nc), workY(nc);
@@ -428,12 +493,35 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
     JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_jobs_spec, js.data(), js.size() * sizeof(EighJob), cudaMemcpyHostToDevice, s));
     JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_jobs_fit, jf.data(), jf.size() * sizeof(EighJob), cudaMemcpyHostToDevice, s));
 #define UP(dst, v) JOLT_CUDA_TRY(cudaMemcpyAsync(dst, v.data(), nc * sizeof(v[0]), cudaMemcpyHostToDevice, s))
+#define UPI(dst, v) JOLT_CUDA_TRY(cudaMemcpyAsync(dst, v.data(), v.size() * sizeof(int), cudaMemcpyHostToDevice, s))
     UP(p->d_GT, GT); UP(p->d_ZT, ZT); UP(p->d_VtT, VtT); UP(p->d_wT, wT); UP(p->d_Cd, Cd);
     UP(p->d_wD, wD); UP(p->d_nsq, nsq); UP(p->d_tT, tT); UP(p->d_tD, tD); UP(p->d_Y, Y);
     UP(p->d_CY, CY); UP(p->d_VtY, VtY); UP(p->d_wY, wY); UP(p->d_ZY, ZY); UP(p->d_Uf, Uf);
     UP(p->d_M, M);
 #undef UP
     p->h_tT = tT; p->h_tD = tD; p->h_wT = wT; p->h_wD = wD; p->h_nsq = nsq; p->h_M = M;
+    if (rnd) {
+      const int k = p->k;
+      const size_t kk = (size_t)k * k;
+      std::vector<int> l0v(nc), bv(nc), lgv(nc), kindv(nc), ncv(nc), cisv(nc);
+      std::vector<EighJob> jr(2 * nc);
+      for (int i = 0; i < nc; ++i) {
+        const HostCell& c = p->hc[i];
+        l0v[i] = c.l0; bv[i] = c.seq; lgv[i] = c.Lg; kindv[i] = c.kind; ncv[i] = c.N;
+        cisv[i] = 2 * c.group + c.kind;
+        jr[i] = EighJob{k, 1, p->MB + i * kk, p->ew + (size_t)i * k, p->eVt + i * kk, p->eZ + i * kk,
+                        p->ework + (size_t)i * k};
+        jr[nc + i] = EighJob{D, 0, Cd[i], wD[i], nullptr, nullptr, workD[i]};
+      }
+      UPI(p->d_cl0, l0v); UPI(p->d_cb, bv); UPI(p->d_cLg, lgv); UPI(p->d_ckind, kindv);
+      UPI(p->d_Nc, ncv); UPI(p->d_cis, cisv);
+      JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_jobs_rand, jr.data(), jr.size() * sizeof(EighJob), cudaMemcpyHostToDevice, s));
+      // bf16 operand buffers start at zero: padding rows/columns are read by the
+      // tensor cores and must not hold NaN bit patterns
+      JOLT_CUDA_TRY(cudaMemsetAsync(p->Wt, 0, (size_t)nc * k * p->Ncmax * 2, s));
+      JOLT_CUDA_TRY(cudaMemsetAsync(p->Yt, 0, (size_t)nc * k * p->tp * 2, s));
+      JOLT_CUDA_TRY(cudaMemsetAsync(p->Pt, 0, (size_t)nc * p->rpad * p->kpad * 2, s));
+    }
     if (p->d_cs) JOLT_TRY(launch_rope_table(T, D, (double)p->lay.rope_theta_k, p->d_cs, s));
     JOLT_TRY(launch_eps2(p->bits.data(), (int)p->bits.size(), p->G, p->d_eps2, p->d_fpart, s));
     JOLT_CUDA_TRY(cudaStreamSynchronize(s));
@@ -467,16 +555,136 @@ static jolt_status upload_cells(jolt_plan_s* p, const void* k, const void* v, cu
 }
 
 // Spectra of every cell: ||X||^2, feature Gram eigenvalues, token spectrum.
-static jolt_status run_spectra(jolt_plan_s* p, int* status, cudaStream_t s) {
+// Tensor maps of the bf16 compression targets (working copies or inputs).
+static jolt_status x_maps(jolt_plan_s* p, const void* k_in, const void* v_in, umma::Maps& m) {
+  const jolt_layout& L = p->lay;
+  const int B = L.batch, Ln = L.n_layers, H = p->H, T = p->T, D = p->D;
+  const int64_t ch = (int64_t)T * D, cl = ch * H, cb = cl * Ln;
+  if (p->copy_k) JOLT_TRY(map_x5(&m.xk, p->Xk, B, Ln, H, T, D, cb, cl, ch, D));
+  else JOLT_TRY(map_x5(&m.xk, k_in, B, Ln, H, T, D, L.stride_b, L.stride_l, L.stride_h, L.stride_t));
+  if (p->copy_v) JOLT_TRY(map_x5(&m.xv, p->Xv, B, Ln, H, T, D, cb, cl, ch, D));
+  else JOLT_TRY(map_x5(&m.xv, v_in, B, Ln, H, T, D, L.stride_b, L.stride_l, L.stride_h, L.stride_t));
+  return JOLT_OK;
+}
+
+static umma::Problem gemm_problem(jolt_plan_s* p, int mode, int* status) {
+  umma::Problem q{};
+  q.mode = mode;
+  q.ncells = p->ncells;
+  q.H = p->H; q.D = p->D; q.T = p->T; q.t_pitch = p->tp; q.nbatch = p->lay.batch;
+  q.cell_l0 = p->d_cl0; q.cell_b = p->d_cb; q.cell_Lg = p->d_cLg; q.cell_kind = p->d_ckind;
+  q.status = status;
+  return q;
+}
+
+// Section 3.1: sketch + power iterations on the feature side, then the
+// spectrum of B B^T with the synthetic tail entry; also the feature Gram.
+static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void* v_in, uint64_t seed,
+                                    int* status, cudaStream_t s) {
+  const jolt_layout& L = p->lay;
+  const int nc = p->ncells, D = p->D, T = p->T, k = p->k;
+  const int64_t kk = (int64_t)k * k;
+  if (p->copy_k)
+    JOLT_TRY(launch_make_xb(k_in, L.dtype == JOLT_F32, L.rope_theta_k > 0, p->d_cs, L.batch, L.n_layers, p->H, T, D,
+                            L.stride_b, L.stride_l, L.stride_h, L.stride_t, p->Xk, s));
+  if (p->copy_v)
+    JOLT_TRY(launch_make_xb(v_in, L.dtype == JOLT_F32, 0, p->d_cs, L.batch, L.n_layers, p->H, T, D,
+                            L.stride_b, L.stride_l, L.stride_h, L.stride_t, p->Xv, s));
+  umma::Maps m{};
+  JOLT_TRY(x_maps(p, k_in, v_in, m));
+  m.at = m.xk;
+  m.bt = m.xk;
+  // feature Gram (tensor cores, fp32 partials per row chunk, fp64 reduction)
+  {
+    umma::Problem q = gemm_problem(p, umma::FG, status);
+    q.BN = 128; q.N = 128; q.mt = p->fg_chunks; q.nt = 1;
+    q.fg_chunks = p->fg_chunks; q.fg_spc = p->fg_spc;
+    q.out_f32 = p->fgpart;
+    JOLT_TRY(launch_umma(m, q, s));
+    JOLT_TRY(launch_fgram_reduce(p->fgpart, p->fg_chunks, D, p->d_Cd, p->d_nsq, nc, s));
+  }
+  // W_0^T = Omega^T
+  JOLT_TRY(launch_omega(p->Wt, nc, k, p->Ncmax, p->d_Nc, p->d_cb, p->d_cis, seed, s));
+  auto xw = [&]() -> jolt_status {
+    umma::Maps mm = m;
+    JOLT_TRY(map_3d(&mm.bt, p->Wt, nc, k, p->Ncmax, p->Ncmax, p->BN));
+    umma::Problem q = gemm_problem(p, umma::XW, status);
+    q.M = T; q.N = k; q.BN = p->BN; q.mt = (T + 127) / 128; q.nt = p->nt_k;
+    q.out_bf16 = p->Yt; q.out_cell_stride = (int64_t)k * p->tp;
+    return launch_umma(mm, q, s);
+  };
+  auto xty = [&]() -> jolt_status {
+    umma::Maps mm = m;
+    JOLT_TRY(map_3d(&mm.bt, p->Yt, nc, k, T, p->tp, p->BN));
+    umma::Problem q = gemm_problem(p, umma::XTY, status);
+    q.M = p->Ncmax; q.N = k; q.Kdim = T; q.BN = p->BN; q.mt = (p->Ncmax + 127) / 128; q.nt = p->nt_k;
+    q.out_f32 = p->Z; q.out_cell_stride = (int64_t)p->Ncmax * k;
+    return launch_umma(mm, q, s);
+  };
+  JOLT_TRY(xw());
+  for (int it = 0; it < p->opt.power_iters; ++it) {
+    JOLT_TRY(xty());
+    // V = Z R^{-1} with Z^T Z = R^T R (fp64), stored as the next W^T
+    JOLT_TRY(launch_gram_cols(p->Z, (int64_t)p->Ncmax * k, p->d_Nc, k, p->Gz, kk, nc, s));
+    JOLT_TRY(launch_cholesky(p->Gz, kk, nullptr, 0, k, nc, status, s));
+    JOLT_TRY(launch_trsm_rows(p->Z, (int64_t)p->Ncmax * k, p->Gz, kk, k, p->d_Nc, p->Ncmax, p->Wt,
+                              (int64_t)k * p->Ncmax, p->Ncmax, p->trs, (int64_t)p->Ncmax * k, nc, s));
+    JOLT_TRY(xw());
+  }
+  JOLT_TRY(xty());
+  // G_W = W^T W (tensor cores) = R^T R
+  {
+    umma::Maps mm = m;
+    JOLT_TRY(map_3d(&mm.at, p->Yt, nc, k, T, p->tp, 128));
+    JOLT_TRY(map_3d(&mm.bt, p->Yt, nc, k, T, p->tp, p->BN));
+    umma::Problem q = gemm_problem(p, umma::GRAM, status);
+    q.M = k; q.N = k; q.Kdim = T; q.BN = p->BN; q.mt = (k + 127) / 128; q.nt = p->nt_k;
+    q.out_f32 = p->GW32; q.out_cell_stride = kk;
+    JOLT_TRY(launch_umma(mm, q, s));
+  }
+  JOLT_TRY(launch_cholesky(p->Rm, kk, p->GW32, kk, k, nc, status, s));
+  // B B^T = R^{-T} (Z^T Z) R^{-1}, then its eigenpairs (and the feature spectrum)
+  JOLT_TRY(launch_gram_cols(p->Z, (int64_t)p->Ncmax * k, p->d_Nc, k, p->P0, kk, nc, s));
+  JOLT_TRY(launch_bbt(p->Rm, p->P0, p->X1, p->MB, kk, k, nc, s));
+  JOLT_TRY(launch_eigh(p->d_jobs_rand, 2 * nc, std::max(k, D), status, s));
+  JOLT_TRY(launch_rand_spectrum(p->ew, k, p->q_used, p->d_nsq, p->d_wT, nc, s));
+  return JOLT_OK;
+}
+
+// U_T^ = bf16(W_q R^{-1} U_B[:, :r_T]) into the payload (tensor cores), and
+// Y = (Z R^{-1} U_B[:, :r_T])^T for the feature factor.
+static jolt_status run_random_fit(jolt_plan_s* p, const void* k_in, const void* v_in, CellOut* d_out, int* status,
+                                  cudaStream_t s) {
+  const int nc = p->ncells, T = p->T, k = p->k;
+  const int64_t kk = (int64_t)k * k;
+  JOLT_TRY(launch_make_p(p->Rm, p->eVt, kk, k, d_out, p->P64, (int64_t)k * p->rmax_all, p->rmax_all, p->Pt,
+                         (int64_t)p->rpad * p->kpad, p->kpad, nc, s));
+  JOLT_TRY(launch_copy_out(d_out, p->d_rT_used, p->d_utp, nc, s));
+  umma::Maps m{};
+  JOLT_TRY(x_maps(p, k_in, v_in, m));
+  JOLT_TRY(map_3d(&m.at, p->Yt, nc, k, T, p->tp, 64));
+  JOLT_TRY(map_3d(&m.bt, p->Pt, nc, p->rpad, p->kpad, p->kpad, 128));
+  umma::Problem q = gemm_problem(p, umma::WP, status);
+  q.M = T; q.N = p->rpad; q.Kdim = k; q.BN = 128; q.mt = (T + 127) / 128; q.nt = p->rpad / 128;
+  q.wp_rows = p->d_rT_used; q.wp_dst = p->d_utp;
+  JOLT_TRY(launch_umma(m, q, s));
+  JOLT_TRY(launch_yproj(p->Z, (int64_t)p->Ncmax * k, p->P64, (int64_t)k * p->rmax_all, k, p->rmax_all, d_out,
+                        p->d_nlh, p->d_Y, p->lh_max, p->D, nc, s));
+  return JOLT_OK;
+}
+
+static jolt_status run_spectra(jolt_plan_s* p, const void* k_in, const void* v_in, uint64_t seed, int* status,
+                               cudaStream_t s) {
   const int nc = p->ncells, D = p->D;
-  JOLT_TRY(launch_fgram_x(p->d_cells, nc, D, p->d_cs, p->fchunk, p->d_fpart, s));
-  JOLT_TRY(launch_sum_chunks(p->d_fpart, p->fchunk, D * D + 1, nc, p->d_Cd, p->d_nsq, s));
+  if (p->opt.mode == JOLT_EXACT) {
+    JOLT_TRY(launch_fgram_x(p->d_cells, nc, D, p->d_cs, p->fchunk, p->d_fpart, s));
+    JOLT_TRY(launch_sum_chunks(p->d_fpart, p->fchunk, D * D + 1, nc, p->d_Cd, p->d_nsq, s));
+  }
   if (p->opt.mode == JOLT_EXACT) {
     JOLT_TRY(launch_token_gram(p->d_cells, nc, p->nmin_max, p->d_cs, p->d_GT, s));
     JOLT_TRY(launch_eigh(p->d_jobs_spec, 2 * nc, std::max(p->nmin_max, D), status, s));
   } else {
-    set_error("randomized mode is not built yet");
-    return JOLT_ERR_UNSUPPORTED_SHAPE;
+    JOLT_TRY(run_range_finder(p, k_in, v_in, seed, status, s));
   }
   JOLT_TRY(launch_rd_tables(p->d_rd_cells, nc, p->d_wT, p->d_wD, nullptr, p->d_tT, p->d_tD, p->d_nt,
                             p->d_nsq, status, s));
@@ -544,7 +752,7 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   if (cudaMemsetAsync(h->d_status, 0, 4 * sizeof(int), s) != cudaSuccess) return fail(JOLT_ERR_CUDA);
   jolt_status st;
   if ((st = upload_cells(p, k, v, s)) != JOLT_OK) return fail(st);
-  if ((st = run_spectra(p, h->d_status, s)) != JOLT_OK) return fail(st);
+  if ((st = run_spectra(p, k, v, seed, h->d_status, s)) != JOLT_OK) return fail(st);
   if ((st = run_allocation(p, B, p->d_eps2, h->d_state, h->d_choice, h->d_status, s)) != JOLT_OK) return fail(st);
   if ((st = launch_payload_layout(p->d_cells, h->d_choice, nc, p->G, h->payload, h->capacity, h->d_out,
                                   h->d_status, s)) != JOLT_OK) return fail(st);
@@ -555,6 +763,8 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   if (p->opt.mode == JOLT_EXACT) {
     if ((st = launch_ut_exact(fa, p->T, p->rmax_all, s)) != JOLT_OK) return fail(st);
     if ((st = launch_project_y(fa, p->T, p->rmax_all, p->lh_max, s)) != JOLT_OK) return fail(st);
+  } else {
+    if ((st = run_random_fit(p, k, v, h->d_out, h->d_status, s)) != JOLT_OK) return fail(st);
   }
   // feature Gram of Y (rows r < r_T), then its eigenvectors
   if ((st = launch_copy_rt(h->d_out, p->d_rT_used, nc, s)) != JOLT_OK) return fail(st);
@@ -659,7 +869,7 @@ jolt_status jolt_rd_table(jolt_plan_t* p, const void* k, const void* v, double* 
   if (max_t < p->nt_max) { set_error("max_t must be >= %d", p->nt_max); return JOLT_ERR_INVALID_ARG; }
   JOLT_CUDA_TRY(cudaMemsetAsync(p->d_status, 0, sizeof(int), s));
   JOLT_TRY(upload_cells(p, k, v, s));
-  JOLT_TRY(run_spectra(p, p->d_status, s));
+  JOLT_TRY(run_spectra(p, k, v, 0, p->d_status, s));
   JOLT_CUDA_TRY(cudaStreamSynchronize(s));
   int st = 0;
   JOLT_CUDA_TRY(cudaMemcpy(&st, p->d_status, sizeof(int), cudaMemcpyDeviceToHost));

@@ -255,6 +255,17 @@ __global__ void k_copy_rt(const CellOut* out, int* rt, int ncells) {
   if (c < ncells) rt[c] = out[c].rT;
 }
 
+__global__ void k_copy_out(const CellOut* out, int* rt, uint16_t** ut, int ncells) {
+  int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c < ncells) { rt[c] = out[c].rT; ut[c] = out[c].ut; }
+}
+
+jolt_status launch_copy_out(const CellOut* out, int* rt, uint16_t** ut, int ncells, cudaStream_t s) {
+  k_copy_out<<<(ncells + 127) / 128, 128, 0, s>>>(out, rt, ut, ncells);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
 jolt_status launch_copy_rt(const CellOut* out, int* rt, int ncells, cudaStream_t s) {
   k_copy_rt<<<(ncells + 127) / 128, 128, 0, s>>>(out, rt, ncells);
   JOLT_LAUNCHED();

@@ -1,5 +1,6 @@
 // Kernel-side structures and host launchers shared across translation units.
 #pragma once
+#include <cuda.h>
 #include "jolt_internal.cuh"
 
 namespace jolt {
@@ -149,5 +150,34 @@ jolt_status launch_encode_rows(const float* e, int64_t rows, int D, int b, int G
 jolt_status launch_decode_rows(const uint8_t* codes, const float* scales, int64_t rows, int D,
                                int b, int G, uint64_t seed, float* e, cudaStream_t s);
 jolt_status launch_rope_table(int T, int D, double theta, float2* cs, cudaStream_t s);
+jolt_status launch_copy_out(const CellOut* out, int* rt, uint16_t** ut, int ncells, cudaStream_t s);
+
+// ------------------------------------------------------- randomized mode ---
+jolt_status map_x5(CUtensorMap* m, const void* base, int B, int L, int H, int T, int D, int64_t sb, int64_t sl,
+                   int64_t sh, int64_t st);
+jolt_status map_3d(CUtensorMap* m, const void* base, int cells, int rows, int cols, int64_t pitch, int box_rows);
+jolt_status launch_make_xb(const void* src, int f32, int rope, const float2* cs, int B, int L, int H, int T,
+                           int D, int64_t sb, int64_t sl, int64_t sh, int64_t st, uint16_t* dst, cudaStream_t s);
+jolt_status launch_omega(uint16_t* wt, int ncells, int k, int ld, const int* Nc, const int* seq, const int* cis,
+                         uint64_t seed, cudaStream_t s);
+jolt_status launch_gram_cols(const float* A, int64_t a_cell, const int* rows_of, int k, double* C, int64_t c_cell,
+                             int ncells, cudaStream_t s);
+jolt_status launch_cholesky(double* A, int64_t a_cell, const float* src32, int64_t s_cell, int k, int ncells,
+                            int* status, cudaStream_t s);
+jolt_status launch_trsm_rows(const float* Z, int64_t z_cell, const double* R, int64_t r_cell, int k, const int* Nc,
+                             int Ncmax, uint16_t* Wt, int64_t w_cell, int ldw, double* scratch, int64_t s_cell,
+                             int ncells, cudaStream_t s);
+jolt_status launch_bbt(const double* R, const double* P, double* X1, double* M, int64_t cs, int k, int ncells,
+                       cudaStream_t s);
+jolt_status launch_rand_spectrum(const double* w_eig, int64_t cs, int q, const double* const* normsq,
+                                 double* const* wT, int ncells, cudaStream_t s);
+jolt_status launch_make_p(const double* R, const double* Vt, int64_t cs, int k, const CellOut* outs, double* P64,
+                          int64_t p_cell, int rmax, uint16_t* Pt, int64_t pt_cell, int ldp, int ncells,
+                          cudaStream_t s);
+jolt_status launch_yproj(const float* Z, int64_t z_cell, const double* P64, int64_t p_cell, int k, int rmax,
+                         const CellOut* outs, const int* nlh, double* const* Y, int lh_max, int D, int ncells,
+                         cudaStream_t s);
+jolt_status launch_fgram_reduce(const float* part, int nchunk, int D, double* const* C, double* const* normsq,
+                                int ncells, cudaStream_t s);
 
 }  // namespace jolt

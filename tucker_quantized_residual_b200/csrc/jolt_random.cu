@@ -1,0 +1,536 @@
+// Randomized token-mode range finder ("A JoLT for the KV Cache", Section 3.1,
+// "FlashJoLT"): a Gaussian sketch plus power iterations give the leading q_cap
+// token-mode singular values and vectors; the energy they miss is appended as
+// one synthetic tail entry (||X||^2 minus the computed energy).
+//
+// The subspace iteration is carried on the feature side, where matrices are
+// N x k (N = L_g H D, small) instead of T x k:
+//   W_0 = X Omega;  for i: Z_i = X^T W_{i-1}, V_i = Z_i R_i^{-1} (CholeskyQR
+//   in fp64), W_i = X V_i;  Z = X^T W_q.
+// range(W_q) = range((X X^T)^q X Omega), the subspace of the usual
+// power-iterated sketch. With G_W = W_q^T W_q = R^T R, Q = W_q R^{-1} is
+// orthonormal, B = Q^T X = R^{-T} Z^T and B B^T = R^{-T} (Z^T Z) R^{-1}; its
+// eigenpairs (sigma~^2, U_B) give U_T = Q U_B = W_q (R^{-1} U_B). The
+// projection Y = U_T^T X used by the fit is (Z R^{-1} U_B)^T, no extra pass
+// over X.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "jolt_internal.cuh"
+#include "jolt_kernels.cuh"
+#define JOLT_UMMA_IMPL
+#include "jolt_umma.cuh"
+
+namespace jolt {
+
+// ------------------------------------------------------------- tensor maps --
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+static jolt_status make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                            const uint64_t* strides_bytes, const uint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) { set_error("cuTensorMapEncodeTiled unavailable"); return JOLT_ERR_CUDA; }
+  uint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides_bytes,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) { set_error("cuTensorMapEncodeTiled failed (%d)", (int)r); return JOLT_ERR_CUDA; }
+  return JOLT_OK;
+}
+
+jolt_status map_x5(CUtensorMap* m, const void* base, int B, int L, int H, int T, int D, int64_t sb, int64_t sl,
+                   int64_t sh, int64_t st) {
+  uint64_t dims[5] = {(uint64_t)D, (uint64_t)T, (uint64_t)H, (uint64_t)L, (uint64_t)B};
+  uint64_t str[4] = {(uint64_t)st * 2, (uint64_t)sh * 2, (uint64_t)sl * 2, (uint64_t)sb * 2};
+  uint32_t box[5] = {64, 64, 1, 1, 1};
+  return make_map(m, base, 5, dims, str, box);
+}
+
+// [cells][rows][cols] bf16 with row pitch `pitch` elements; box {64, box_rows}
+jolt_status map_3d(CUtensorMap* m, const void* base, int cells, int rows, int cols, int64_t pitch,
+                   int box_rows) {
+  uint64_t dims[3] = {(uint64_t)cols, (uint64_t)rows, (uint64_t)cells};
+  uint64_t str[2] = {(uint64_t)pitch * 2, (uint64_t)pitch * 2 * rows};
+  uint32_t box[3] = {64, (uint32_t)box_rows, 1};
+  return make_map(m, base, 3, dims, str, box);
+}
+
+static int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+jolt_status launch_umma(const umma::Maps& maps, const umma::Problem& p, cudaStream_t s) {
+  const int ntiles = p.ncells * p.mt * p.nt;
+  if (ntiles == 0) return JOLT_OK;
+  if (p.BN % 16 || p.BN < 16 || p.BN > umma::BN_MAX) { set_error("bad GEMM tile width %d", p.BN); return JOLT_ERR_INVALID_ARG; }
+  static bool attr = false;
+  if (!attr) {
+    JOLT_CUDA_TRY(cudaFuncSetAttribute(umma::k_umma_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       umma::SMEM_BYTES));
+    attr = true;
+  }
+  const int grid = std::min(ntiles, num_sms());
+  umma::k_umma_gemm<<<grid, umma::THREADS, umma::SMEM_BYTES, s>>>(maps, p);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// --------------------------------------------------- bf16 working copies ---
+// dst (contiguous [B][L][H][T][D] bf16) = bf16_rne(x), x the compression
+// target: un-RoPE'd keys in fp32 (rope != 0) or the stored values.
+__global__ void k_make_xb(const void* __restrict__ src, int f32, int rope, const float2* __restrict__ cs,
+                          int B, int L, int H, int T, int D, int64_t sb, int64_t sl, int64_t sh, int64_t st,
+                          uint16_t* __restrict__ dst) {
+  const int half = D / 2;
+  const int64_t rows = (int64_t)B * L * H * T;
+  const int per_row = half / 8;              // 8-pair blocks per row
+  const int64_t n = rows * per_row;
+  for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < n; k += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = k / per_row;
+    const int i0 = (int)(k % per_row) * 8;
+    int64_t r = row;
+    const int t = (int)(r % T); r /= T;
+    const int h = (int)(r % H); r /= H;
+    const int l = (int)(r % L); r /= L;
+    const int b = (int)r;
+    const int64_t off = (int64_t)b * sb + (int64_t)l * sl + (int64_t)h * sh + (int64_t)t * st;
+    float y0[8], y1[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (f32) {
+        y0[j] = reinterpret_cast<const float*>(src)[off + i0 + j];
+        y1[j] = reinterpret_cast<const float*>(src)[off + half + i0 + j];
+      } else {
+        y0[j] = bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(src)[off + i0 + j]);
+        y1[j] = bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(src)[off + half + i0 + j]);
+      }
+    }
+    uint16_t o0[8], o1[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float a = y0[j], c = y1[j];
+      if (rope) {
+        const float2 q = cs[(int64_t)t * half + i0 + j];
+        a = __fadd_rn(__fmul_rn(y0[j], q.x), __fmul_rn(y1[j], q.y));
+        c = __fsub_rn(__fmul_rn(y1[j], q.x), __fmul_rn(y0[j], q.y));
+      }
+      o0[j] = bf16_bits_from_f32(a);
+      o1[j] = bf16_bits_from_f32(c);
+    }
+    uint16_t* d = dst + row * D;
+    *reinterpret_cast<uint4*>(d + i0) = *reinterpret_cast<uint4*>(o0);
+    *reinterpret_cast<uint4*>(d + half + i0) = *reinterpret_cast<uint4*>(o1);
+  }
+}
+
+jolt_status launch_make_xb(const void* src, int f32, int rope, const float2* cs, int B, int L, int H, int T,
+                           int D, int64_t sb, int64_t sl, int64_t sh, int64_t st, uint16_t* dst,
+                           cudaStream_t s) {
+  const int64_t n = (int64_t)B * L * H * T * (D / 16);
+  const int grid = (int)std::min<int64_t>((n + 255) / 256, 148 * 16);
+  k_make_xb<<<grid, 256, 0, s>>>(src, f32, rope, cs, B, L, H, T, D, sb, sl, sh, st, dst);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// ------------------------------------------------------- Gaussian sketch ---
+// W^T[cell][j][n] = bf16(N(0,1)) for n < N_c(cell), 0 beyond. Four normals per
+// Philox4x32-10 call (Box-Muller on (w0, w1) and (w2, w3), fp64), counter
+// (e/4, cell_in_sequence, STREAM_SKETCH, 0) with e = j * ld + n, key = seed + b.
+__global__ void k_omega(uint16_t* __restrict__ wt, int ncells, int k, int ld, const int* __restrict__ Nc,
+                        const int* __restrict__ seq, const int* __restrict__ cis, uint64_t seed) {
+  const int cell = blockIdx.y;
+  const int64_t n4 = (int64_t)k * ld / 4;
+  uint16_t* w = wt + (int64_t)cell * k * ld;
+  const int nc = Nc[cell];
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    const u4 r = philox_at(seed + (uint64_t)seq[cell], STREAM_SKETCH, (uint32_t)i, (uint32_t)cis[cell]);
+    const double u0 = ((double)r.x + 0.5) * 0x1p-32, u1 = ((double)r.y + 0.5) * 0x1p-32;
+    const double u2 = ((double)r.z + 0.5) * 0x1p-32, u3 = ((double)r.w + 0.5) * 0x1p-32;
+    const double r0 = sqrt(-2.0 * log(u0)), r1 = sqrt(-2.0 * log(u2));
+    const double t0 = 6.283185307179586 * u1, t1 = 6.283185307179586 * u3;
+    const double z[4] = {r0 * cos(t0), r0 * sin(t0), r1 * cos(t1), r1 * sin(t1)};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int64_t e = 4 * i + c;
+      const int n = (int)(e % ld);
+      w[e] = (n < nc) ? bf16_bits_from_f64(z[c]) : (uint16_t)0;
+    }
+  }
+}
+
+jolt_status launch_omega(uint16_t* wt, int ncells, int k, int ld, const int* Nc, const int* seq, const int* cis,
+                         uint64_t seed, cudaStream_t s) {
+  const int64_t n4 = (int64_t)k * ld / 4;
+  dim3 g((unsigned)std::min<int64_t>((n4 + 255) / 256, 1024), ncells);
+  k_omega<<<g, 256, 0, s>>>(wt, ncells, k, ld, Nc, seq, cis, seed);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// -------------------------------------------------- fp64 Gram of columns ---
+// C[cell][i][j] = sum_n A[cell][n][i] A[cell][n][j], A fp32 row-major [rows][k]
+__global__ void __launch_bounds__(256) k_gram_cols(const float* __restrict__ A, int64_t a_cell, const int* __restrict__ rows_of,
+                                                   int k, double* __restrict__ C, int64_t c_cell) {
+  constexpr int TB = 64, KB = 16;
+  __shared__ double As[KB][TB + 1];
+  __shared__ double Bs[KB][TB + 1];
+  const int cell = blockIdx.y;
+  const int nrows = rows_of[cell];
+  const float* a = A + (int64_t)cell * a_cell;
+  const int nt = (k + TB - 1) / TB;
+  int b = blockIdx.x, ti = 0;
+  while (ti < nt && b >= nt - ti) { b -= nt - ti; ++ti; }
+  if (ti >= nt) return;
+  const int tj = ti + b;
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  double acc[4][4] = {};
+  for (int r0 = 0; r0 < nrows; r0 += KB) {
+    for (int e = threadIdx.x; e < KB * TB; e += blockDim.x) {
+      const int kk = e / TB, ii = e % TB;
+      const int r = r0 + kk, ia = ti * TB + ii, ib = tj * TB + ii;
+      As[kk][ii] = (r < nrows && ia < k) ? (double)a[(int64_t)r * k + ia] : 0.0;
+      Bs[kk][ii] = (r < nrows && ib < k) ? (double)a[(int64_t)r * k + ib] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < KB; ++kk) {
+      double x[4], y[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { x[i] = As[kk][ty * 4 + i]; y[i] = Bs[kk][tx * 4 + i]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fma(x[i], y[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  double* c = C + (int64_t)cell * c_cell;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = ti * TB + ty * 4 + i, q = tj * TB + tx * 4 + j;
+      if (r < k && q < k) { c[(int64_t)r * k + q] = acc[i][j]; c[(int64_t)q * k + r] = acc[i][j]; }
+    }
+}
+
+jolt_status launch_gram_cols(const float* A, int64_t a_cell, const int* rows_of, int k, double* C, int64_t c_cell,
+                             int ncells, cudaStream_t s) {
+  const int nt = (k + 63) / 64;
+  dim3 g(nt * (nt + 1) / 2, ncells);
+  k_gram_cols<<<g, 256, 0, s>>>(A, a_cell, rows_of, k, C, c_cell);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// ----------------------------------------------------------- Cholesky ------
+// In place: A (k x k fp64 symmetric, or fp32 source copied in) becomes R
+// (upper triangular, A = R^T R). A relative diagonal shift of 1e-13 trace/k
+// keeps a numerically rank-deficient sketch factorizable (shifted
+// CholeskyQR); a non-positive pivot is still reported.
+__global__ void __launch_bounds__(512) k_cholesky(double* __restrict__ A, int64_t a_cell, const float* __restrict__ src32,
+                                                  int64_t s_cell, int k, int* status) {
+  double* a = A + (int64_t)blockIdx.x * a_cell;
+  __shared__ double inv_piv;
+  __shared__ double red[32];
+  if (src32) {
+    const float* s32 = src32 + (int64_t)blockIdx.x * s_cell;
+    for (int64_t e = threadIdx.x; e < (int64_t)k * k; e += blockDim.x) a[e] = (double)s32[e];
+    __syncthreads();
+  }
+  double tr = 0.0;
+  for (int i = threadIdx.x; i < k; i += blockDim.x) tr += a[(int64_t)i * k + i];
+  // block sum
+  for (int o = 16; o > 0; o >>= 1) tr += __shfl_xor_sync(0xffffffffu, tr, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = tr;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+    red[0] = t;
+  }
+  __syncthreads();
+  // an all-zero Gram (an all-zero cell) factors as the identity: any R works
+  // because the columns it orthonormalizes are zero
+  const double shift = (red[0] > 0.0) ? 1e-13 * red[0] / k : 1.0;
+  for (int i = threadIdx.x; i < k; i += blockDim.x) a[(int64_t)i * k + i] += shift;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int j = 0; j < k; ++j) {
+    if (threadIdx.x == 0) {
+      double piv = a[(int64_t)j * k + j];
+      if (!(piv > 0.0)) { atomicOr(status, DEV_ERR_CHOL); piv = fmax(shift, 1e-300); }
+      const double r = sqrt(piv);
+      a[(int64_t)j * k + j] = r;
+      inv_piv = 1.0 / r;
+    }
+    __syncthreads();
+    for (int i = j + 1 + threadIdx.x; i < k; i += blockDim.x) a[(int64_t)j * k + i] *= inv_piv;
+    __syncthreads();
+    for (int i = j + 1 + warp; i < k; i += nw) {
+      const double rji = a[(int64_t)j * k + i];
+      double* row = a + (int64_t)i * k;
+      const double* rj = a + (int64_t)j * k;
+      for (int l = i + lane; l < k; l += 32) row[l] -= rji * rj[l];
+    }
+    __syncthreads();
+  }
+  for (int64_t e = threadIdx.x; e < (int64_t)k * k; e += blockDim.x)
+    if (e / k > e % k) a[e] = 0.0;
+}
+
+jolt_status launch_cholesky(double* A, int64_t a_cell, const float* src32, int64_t s_cell, int k, int ncells,
+                            int* status, cudaStream_t s) {
+  k_cholesky<<<ncells, 512, 0, s>>>(A, a_cell, src32, s_cell, k, status);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// ------------------------------------------------------ triangular solves --
+// V = Z R^{-1} row by row (forward substitution on R^T), stored transposed in
+// bf16: Wt[cell][j][n] for n < N_c. Z fp32 [cell][Ncmax][k].
+__global__ void k_trsm_rows(const float* __restrict__ Z, int64_t z_cell, const double* __restrict__ R, int64_t r_cell,
+                            int k, const int* __restrict__ Nc, uint16_t* __restrict__ Wt, int64_t w_cell, int ldw,
+                            double* __restrict__ scratch, int64_t s_cell) {
+  const int cell = blockIdx.y;
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= Nc[cell]) return;
+  const float* z = Z + (int64_t)cell * z_cell + (int64_t)n * k;
+  const double* r = R + (int64_t)cell * r_cell;
+  double* v = scratch + (int64_t)cell * s_cell + (int64_t)n * k;
+  uint16_t* w = Wt + (int64_t)cell * w_cell + n;
+  for (int j = 0; j < k; ++j) {
+    double acc = (double)z[j];
+    for (int i = 0; i < j; ++i) acc -= v[i] * r[(int64_t)i * k + j];
+    const double x = acc / r[(int64_t)j * k + j];
+    v[j] = x;
+    w[(int64_t)j * ldw] = bf16_bits_from_f64(x);
+  }
+}
+
+jolt_status launch_trsm_rows(const float* Z, int64_t z_cell, const double* R, int64_t r_cell, int k, const int* Nc,
+                             int Ncmax, uint16_t* Wt, int64_t w_cell, int ldw, double* scratch, int64_t s_cell,
+                             int ncells, cudaStream_t s) {
+  dim3 g((Ncmax + 127) / 128, ncells);
+  k_trsm_rows<<<g, 128, 0, s>>>(Z, z_cell, R, r_cell, k, Nc, Wt, w_cell, ldw, scratch, s_cell);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// X1 = R^{-T} P (column c per thread, forward substitution), then
+// M = X1 R^{-1} (row per thread), symmetrized into M.
+__global__ void k_solve_left_t(const double* __restrict__ R, const double* __restrict__ P, double* __restrict__ X1,
+                               int64_t cs, int k) {
+  const int cell = blockIdx.y, c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= k) return;
+  const double* r = R + (int64_t)cell * cs;
+  const double* p = P + (int64_t)cell * cs;
+  double* x = X1 + (int64_t)cell * cs;
+  for (int i = 0; i < k; ++i) {
+    double acc = p[(int64_t)i * k + c];
+    for (int l = 0; l < i; ++l) acc -= r[(int64_t)l * k + i] * x[(int64_t)l * k + c];
+    x[(int64_t)i * k + c] = acc / r[(int64_t)i * k + i];
+  }
+}
+
+__global__ void k_solve_right(const double* __restrict__ R, const double* __restrict__ X1, double* __restrict__ M,
+                              int64_t cs, int k) {
+  const int cell = blockIdx.y, row = blockIdx.x * blockDim.x + threadIdx.x;
+  if (row >= k) return;
+  const double* r = R + (int64_t)cell * cs;
+  const double* x = X1 + (int64_t)cell * cs + (int64_t)row * k;
+  double* m = M + (int64_t)cell * cs + (int64_t)row * k;
+  for (int j = 0; j < k; ++j) {
+    double acc = x[j];
+    for (int i = 0; i < j; ++i) acc -= m[i] * r[(int64_t)i * k + j];
+    m[j] = acc / r[(int64_t)j * k + j];
+  }
+}
+
+__global__ void k_symmetrize(double* __restrict__ M, int64_t cs, int k) {
+  const int cell = blockIdx.y;
+  double* m = M + (int64_t)cell * cs;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < (int64_t)k * k; e += (int64_t)gridDim.x * blockDim.x) {
+    const int i = (int)(e / k), j = (int)(e % k);
+    if (i < j) {
+      const double a = 0.5 * (m[(int64_t)i * k + j] + m[(int64_t)j * k + i]);
+      m[(int64_t)i * k + j] = a;
+      m[(int64_t)j * k + i] = a;
+    }
+  }
+}
+
+jolt_status launch_bbt(const double* R, const double* P, double* X1, double* M, int64_t cs, int k, int ncells,
+                       cudaStream_t s) {
+  dim3 g((k + 127) / 128, ncells);
+  k_solve_left_t<<<g, 128, 0, s>>>(R, P, X1, cs, k);
+  JOLT_LAUNCHED();
+  k_solve_right<<<g, 128, 0, s>>>(R, X1, M, cs, k);
+  JOLT_LAUNCHED();
+  dim3 g2(64, ncells);
+  k_symmetrize<<<g2, 256, 0, s>>>(M, cs, k);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// Token spectrum for the allocator: the q leading eigenvalues of B B^T and the
+// synthetic tail max(0, ||X||^2 - sum of them) (Section 3.1).
+__global__ void k_rand_spectrum(const double* __restrict__ w_eig, int64_t cs, int q, const double* const* __restrict__ normsq,
+                                double* const* __restrict__ wT) {
+  const int cell = blockIdx.x;
+  if (threadIdx.x != 0) return;
+  const double* w = w_eig + (int64_t)cell * cs;
+  double s = 0.0;
+  double* o = wT[cell];
+  for (int i = 0; i < q; ++i) {
+    const double x = fmax(w[i], 0.0);
+    o[i] = x;
+    s += x;
+  }
+  o[q] = fmax(*normsq[cell] - s, 0.0);
+}
+
+jolt_status launch_rand_spectrum(const double* w_eig, int64_t cs, int q, const double* const* normsq,
+                                 double* const* wT, int ncells, cudaStream_t s) {
+  k_rand_spectrum<<<ncells, 32, 0, s>>>(w_eig, cs, q, normsq, wT);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// P = R^{-1} U_B[:, :r_T] by back substitution, one column per thread:
+// P64[cell][i][r] (fp64) and Pt[cell][r][i] (bf16, row pitch ldp).
+__global__ void k_make_p(const double* __restrict__ R, const double* __restrict__ Vt, int64_t cs, int k,
+                         const CellOut* __restrict__ outs, double* __restrict__ P64, int64_t p_cell, int rmax,
+                         uint16_t* __restrict__ Pt, int64_t pt_cell, int ldp) {
+  const int cell = blockIdx.y, c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= outs[cell].rT) return;
+  const double* r = R + (int64_t)cell * cs;
+  const double* u = Vt + (int64_t)cell * cs + (int64_t)c * k;    // eigenvector c
+  double* p = P64 + (int64_t)cell * p_cell;
+  uint16_t* pt = Pt + (int64_t)cell * pt_cell + (int64_t)c * ldp;
+  for (int i = k - 1; i >= 0; --i) {
+    double acc = u[i];
+    for (int l = i + 1; l < k; ++l) acc -= r[(int64_t)i * k + l] * p[(int64_t)l * rmax + c];
+    const double x = acc / r[(int64_t)i * k + i];
+    p[(int64_t)i * rmax + c] = x;
+    pt[i] = bf16_bits_from_f64(x);
+  }
+}
+
+jolt_status launch_make_p(const double* R, const double* Vt, int64_t cs, int k, const CellOut* outs, double* P64,
+                          int64_t p_cell, int rmax, uint16_t* Pt, int64_t pt_cell, int ldp, int ncells,
+                          cudaStream_t s) {
+  dim3 g((rmax + 127) / 128, ncells);
+  k_make_p<<<g, 128, 0, s>>>(R, Vt, cs, k, outs, P64, p_cell, rmax, Pt, pt_cell, ldp);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// Y[lh][r][d] = sum_j Z[(lh*D + d)][j] P[j][r]   (fp64)
+template <int D>
+__global__ void __launch_bounds__(256) k_yproj(const float* __restrict__ Z, int64_t z_cell, const double* __restrict__ P64,
+                                               int64_t p_cell, int k, int rmax, const CellOut* __restrict__ outs,
+                                               const int* __restrict__ nlh, double* const* __restrict__ Y) {
+  constexpr int RB = 16, JB = 32, PD = D / 16;
+  __shared__ double zs[JB][D + 1];
+  __shared__ double ps[JB][RB];
+  const int cell = blockIdx.z, lh = blockIdx.x, r0 = blockIdx.y * RB;
+  const int rT = outs[cell].rT;
+  if (lh >= nlh[cell] || r0 >= rT) return;
+  const float* z = Z + (int64_t)cell * z_cell + (int64_t)lh * D * k;
+  const double* p = P64 + (int64_t)cell * p_cell;
+  const int ri = threadIdx.x / 16, dj = threadIdx.x % 16;
+  double acc[PD] = {};
+  for (int j0 = 0; j0 < k; j0 += JB) {
+    for (int e = threadIdx.x; e < JB * D; e += blockDim.x) {
+      const int jj = e % JB, d = e / JB;
+      zs[jj][d] = (j0 + jj < k) ? (double)z[(int64_t)d * k + j0 + jj] : 0.0;
+    }
+    for (int e = threadIdx.x; e < JB * RB; e += blockDim.x) {
+      const int jj = e / RB, rr = e % RB;
+      ps[jj][rr] = (j0 + jj < k && r0 + rr < rT) ? p[(int64_t)(j0 + jj) * rmax + r0 + rr] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int jj = 0; jj < JB; ++jj) {
+      const double pv = ps[jj][ri];
+#pragma unroll
+      for (int q = 0; q < PD; ++q) acc[q] = fma(zs[jj][dj * PD + q], pv, acc[q]);
+    }
+    __syncthreads();
+  }
+  const int r = r0 + ri;
+  if (r < rT) {
+    double* y = Y[cell] + ((int64_t)lh * rmax + r) * D;
+#pragma unroll
+    for (int q = 0; q < PD; ++q) y[dj * PD + q] = acc[q];
+  }
+}
+
+jolt_status launch_yproj(const float* Z, int64_t z_cell, const double* P64, int64_t p_cell, int k, int rmax,
+                         const CellOut* outs, const int* nlh, double* const* Y, int lh_max, int D, int ncells,
+                         cudaStream_t s) {
+  dim3 g(lh_max, (rmax + 15) / 16, ncells);
+  if (D == 128) k_yproj<128><<<g, 256, 0, s>>>(Z, z_cell, P64, p_cell, k, rmax, outs, nlh, Y);
+  else k_yproj<64><<<g, 256, 0, s>>>(Z, z_cell, P64, p_cell, k, rmax, outs, nlh, Y);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// Feature Gram from the fp32 tensor-core partials: C[cell][i][j] =
+// sum over chunks (fixed order) of the D x D diagonal blocks of the 128 x 128
+// partial tiles; ||X||^2 = trace(C).
+__global__ void k_fgram_reduce(const float* __restrict__ part, int nchunk, int D, double* const* __restrict__ C,
+                               double* const* __restrict__ normsq) {
+  const int cell = blockIdx.y;
+  const int nblk = 128 / D;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < D * D; e += gridDim.x * blockDim.x) {
+    const int i = e / D, j = e % D;
+    double s = 0.0;
+    for (int c = 0; c < nchunk; ++c) {
+      const float* t = part + ((int64_t)cell * nchunk + c) * 128 * 128;
+      for (int b = 0; b < nblk; ++b) s += (double)t[(b * D + i) * 128 + b * D + j];
+    }
+    C[cell][e] = s;
+  }
+}
+
+__global__ void k_trace(double* const* __restrict__ C, int D, double* const* __restrict__ normsq) {
+  const int cell = blockIdx.x;
+  if (threadIdx.x != 0) return;
+  double s = 0.0;
+  for (int i = 0; i < D; ++i) s += C[cell][i * D + i];
+  *normsq[cell] = s;
+}
+
+jolt_status launch_fgram_reduce(const float* part, int nchunk, int D, double* const* C, double* const* normsq,
+                                int ncells, cudaStream_t s) {
+  dim3 g((D * D + 255) / 256, ncells);
+  k_fgram_reduce<<<g, 256, 0, s>>>(part, nchunk, D, C, normsq);
+  JOLT_LAUNCHED();
+  k_trace<<<ncells, 32, 0, s>>>(C, D, normsq);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+}  // namespace jolt
