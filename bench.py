@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the JoLT compress -> decompress path on B200.
+
+Metric: GB/s of dense bf16 KV cache (K and V) compressed and decompressed,
+at a global byte budget of dense / ratio. One step = jolt_compress (spectra,
+allocation, fit, residual) + jolt_decompress of the whole cache; inputs are
+resident in HBM and larger than L2. Default workload: the LLaMA-3.1-8B-shaped
+64K-token cache (32 layers in groups of 4, 8 KV heads, D = 128), randomized
+token-mode SVD (q_cap = Eq. (5), p = 8, 2 power iterations), 2x budget.
+
+Under torchrun every rank compresses its own independent cache (its own
+seed): the path has no cross-rank exchange, so scaling is weak and the value
+is the total over ranks divided by the slowest rank's time.
+
+--impl reference runs the CPU oracle (exact JoLT, fp64) on a bounded sample of
+the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="jolt", choices=["jolt", "reference"])
+    ap.add_argument("--config", default="llama31_8b_64k")
+    ap.add_argument("--ratio", type=float, default=2.0)
+    ap.add_argument("--mode", default="randomized", choices=["randomized", "exact"])
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stages", action="store_true", help="print the per-stage table to stderr")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.f = None
+
+    def start(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------ workload
+def gemm_flops(spec, k, ncells_per_kind):
+    """Algorithmic FLOPs of one launch of each tensor-core GEMM stage."""
+    Lg = spec.group_size
+    N = Lg * spec.n_heads * spec.head_dim
+    T = spec.seq_len
+    cells = 2 * ncells_per_kind
+    return {"gemm_xw": 2.0 * T * N * k * cells, "gemm_xty": 2.0 * N * T * k * cells,
+            "gemm_gram": 2.0 * k * k * T * cells,
+            "fgram": 2.0 * spec.head_dim ** 2 * Lg * spec.n_heads * T * cells}
+
+
+def residual_bytes(spec, cells):
+    """Algorithmic HBM bytes of one residual launch and one decompress launch,
+    from the chosen (r_T, r_d, b) of every cell."""
+    D, T, H = spec.head_dim, spec.seq_len, spec.n_heads
+    res = dec = 0.0
+    for c in cells:
+        n = c.bits
+        rows = spec.group_size * H * T
+        dense = rows * D * 2
+        payload = c.bytes
+        resid = rows * (n * D // 8 + 4 * (D // D)) if n else 0     # codes + one scale per row
+        res += (dense + resid) if n else 0.0
+        dec += payload + dense
+    return res, dec
+
+
+def run_jolt(args):
+    import torch
+    import torch.distributed as dist
+    from tucker_quantized_residual_b200 import jolt, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    spec = synth.SPECS[args.config]
+    gs = synth.group_starts(spec)
+    K, V = synth.make_cache(spec, seed=1000 * rank, device="cuda")
+    torch.cuda.synchronize()
+    dense = synth.dense_bf16_bytes(spec)
+    B = int(math.floor(dense / args.ratio))
+    mode = jolt.JOLT_RANDOMIZED if args.mode == "randomized" else jolt.JOLT_EXACT
+    lay, keep = jolt.make_layout(K, gs, spec.rope_theta_k)
+    opt, keep2 = jolt.make_options(mode=mode)
+    plan = jolt.jolt_plan(lay, B, opt)
+    ncell = jolt.jolt_num_cells(plan)
+    Ko = torch.empty_like(K)
+    Vo = torch.empty_like(V)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        h = jolt.jolt_compress(plan, K, V, B, 1234 + rank, stream)
+        jolt.jolt_decompress(h, Ko, Vo, None, stream)
+        return h
+
+    for _ in range(args.warmup):
+        jolt.jolt_free_handle(step())
+    torch.cuda.synchronize()
+    # one synchronised step for the allocation report
+    h = step()
+    cells, lam, iters = jolt.jolt_handle_info(h, ncell)
+    nbytes = jolt.jolt_bytes(h)
+    jolt.jolt_free_handle(h)
+
+    # ---- timed region (device time, CUDA events on the launching stream)
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    jolt.jolt_profile_enable(True)
+    l0 = jolt.jolt_launch_count()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        jolt.jolt_free_handle(step())
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    launches = jolt.jolt_launch_count() - l0
+    prof = jolt.jolt_profile_read()
+    jolt.jolt_profile_enable(False)
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    value = world * dense * args.steps / (ms / 1e3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Kh = torch.empty(K.shape, dtype=K.dtype, pin_memory=True)
+        Vh = torch.empty(V.shape, dtype=V.dtype, pin_memory=True)
+        Kh.copy_(K)
+        Vh.copy_(V)
+        Koh = torch.empty_like(Kh, pin_memory=True)
+        Voh = torch.empty_like(Vh, pin_memory=True)
+        Kd = torch.empty_like(K)
+        Vd = torch.empty_like(V)
+        lay2, keep3 = jolt.make_layout(Kd, gs, spec.rope_theta_k)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.e2e_steps):
+            Kd.copy_(Kh, non_blocking=True)
+            Vd.copy_(Vh, non_blocking=True)
+            hh = jolt.jolt_compress(plan, Kd, Vd, B, 1234 + rank, stream)
+            jolt.jolt_decompress(hh, Ko, Vo, None, stream)
+            Koh.copy_(Ko, non_blocking=True)
+            Voh.copy_(Vo, non_blocking=True)
+            jolt.jolt_free_handle(hh)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        ems = f0.elapsed_time(f1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": round(world * dense * args.e2e_steps / (ems / 1e3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": 2 * K.numel() * K.element_size(),
+               "d2h_bytes_per_step": 2 * Ko.numel() * Ko.element_size()}
+        del Kh, Vh, Koh, Voh, Kd, Vd
+
+    # ---- roofline of the dominant stage
+    pk, src = peaks()
+    k_sk = ((min(max(32 if args.ratio <= 4 else 64, -(-spec.seq_len // 32)), 512) + 8 + 15) // 16) * 16
+    flops = gemm_flops(spec, k_sk, ncell // 2)
+    res_b, dec_b = residual_bytes(spec, cells)
+    per_step = {s: prof[s][0] / args.steps for s in prof}
+    dom = max(per_step, key=per_step.get)
+    roof = None
+    if dom in flops and prof[dom][1] > 0:
+        per_launch_ms = prof[dom][0] / prof[dom][1]
+        ach = flops[dom] / (per_launch_ms / 1e3) / 1e12
+        peak = pk["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(ach / peak, 3), "peak_source": f"{src} (sustained bf16)", "traffic": None}
+    elif dom in ("residual", "decompress") and prof[dom][1] > 0:
+        per_launch_ms = prof[dom][0] / prof[dom][1]
+        byt = res_b if dom == "residual" else dec_b
+        ach = byt / (per_launch_ms / 1e3) / 1e9
+        peak = pk["hbm_gbs"]
+        roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 3), "peak_source": f"{src} (copy bandwidth)", "traffic": None}
+    else:
+        roof = {"bound": "latency", "kernel": dom, "achieved": None, "peak": None, "unit": None, "frac": None,
+                "traffic": None}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(spec, K, V, args.ratio)
+
+    if args.stages and rank == 0:
+        for s in jolt.STAGES:
+            msx, calls, ln = prof[s]
+            if calls:
+                sys.stderr.write(f"{s:12s} {msx / args.steps:9.3f} ms/step  calls {calls / args.steps:5.1f}  "
+                                 f"launches {ln / args.steps:6.1f}\n")
+        sys.stderr.write(f"alloc: lambda {lam:.3e} iters {iters} bytes {nbytes} budget {B}\n")
+        for c in cells[:6]:
+            sys.stderr.write(f"  cell g{c.group} {'KV'[c.kind]}: r_T {c.r_t} r_d {c.r_d} b {c.bits}\n")
+
+    # errors of this run (for the record; not part of the timed region)
+    errK = errV = None
+    if rank == 0:
+        errK = rel_err(K, Ko)
+        errV = rel_err(V, Vo)
+
+    if rank == 0:
+        line = {
+            "metric": "GB/s of bf16 KV cache compressed+decompressed at 2x/3x budget; rel. Frobenius err",
+            "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{args.config} ({spec.n_layers} layers / groups of {spec.group_size}, "
+                                   f"{spec.n_heads} KV heads, D={spec.head_dim}, T={spec.seq_len}, "
+                                   f"batch {spec.batch}), {args.ratio:g}x budget, {args.mode} token SVD",
+                       "global_batch": spec.batch * world, "seq_len": spec.seq_len,
+                       "parallelism": f"independent caches per GPU (dp{world})",
+                       "l2": "inputs 8.6 GB per GPU, larger than L2; no flush"},
+            "rel_frobenius_err": {"K": errK, "V": errV}, "bytes": nbytes, "budget": B,
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+            "clocks": clk,
+            "stages_ms_per_step": {s: round(v, 3) for s, v in per_step.items() if v > 0},
+        }
+        print(json.dumps(line), flush=True)
+    jolt.jolt_free_plan(plan)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def rel_err(X, Xh):
+    import torch
+    num = 0.0
+    den = 0.0
+    for l in range(X.shape[1]):
+        a = X[:, l].float()
+        b = Xh[:, l].float()
+        num += float(((a - b) ** 2).sum())
+        den += float((a * a).sum())
+    return round(math.sqrt(num / den), 6)
+
+
+# ---------------------------------------------------------- CPU baseline
+def cpu_sample(spec, K, V, T_sample):
+    """The first T_sample tokens of layer group 0 (its K and V cells)."""
+    import torch
+    g1 = spec.group_size
+    Ks = K[:1, :g1, :, :T_sample].float().cpu().numpy()
+    Vs = V[:1, :g1, :, :T_sample].float().cpu().numpy()
+    return Ks, Vs
+
+
+def run_oracle_sample(Ks, Vs, spec, ratio):
+    from oracle import jolt_oracle as o
+    n = Ks.size + Vs.size
+    B = o.budget_for_ratio(n, ratio)
+    q = o.q_cap(Ks.shape[3], ratio)
+    opt = o.Options(rt_max=q)
+    t0 = time.perf_counter()
+    comp = o.compress(Ks, Vs, [0, spec.group_size], B, 0, opt, spec.rope_theta_k)
+    o.decompress(comp)
+    return time.perf_counter() - t0, 2 * n
+
+
+def cpu_baseline(spec, K, V, ratio, T_sample=2048):
+    Ks, Vs = cpu_sample(spec, K, V, T_sample)
+    sec, nbytes = run_oracle_sample(Ks, Vs, spec, ratio)
+    return {"value": round(nbytes / sec / 1e9, 6), "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"layer group 0 (K and V cells) of the {spec.name} cache, first {T_sample} tokens, "
+                      f"exact JoLT in fp64 (numpy/OpenBLAS) with the token rank capped at q_cap, "
+                      f"{nbytes / 1e6:.1f} MB dense bf16 in {sec:.2f} s"}
+
+
+def run_reference(args):
+    """The oracle arm: bounded samples of the same workload on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+    from tucker_quantized_residual_b200 import synth
+    spec = synth.SPECS[args.config]
+    # the sample's cells come from the same generator (CPU, group 0 only)
+    T_sample = 1024
+    spec_s = spec.replace(seq_len=T_sample, n_layers=spec.group_size, batch=1)
+    K, V = synth.make_cache(spec_s, seed=0)
+    Ks, Vs = K.float().numpy(), V.float().numpy()
+    for _ in range(args.warmup):
+        run_oracle_sample(Ks, Vs, spec, args.ratio)
+    total = 0.0
+    nb = 0
+    for _ in range(args.steps):
+        sec, nbytes = run_oracle_sample(Ks, Vs, spec, args.ratio)
+        total += sec
+        nb += nbytes
+    value = nb / total / 1e9
+    sample = (f"layer group 0 (K and V cells) of a {spec.name}-shaped cache, first {T_sample} tokens; exact "
+              f"JoLT in fp64 with the token rank capped at q_cap")
+    line = {"impl": "reference",
+            "metric": "GB/s of bf16 KV cache compressed+decompressed at 2x/3x budget; rel. Frobenius err",
+            "value": round(value, 6), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{args.config} sample, {args.ratio:g}x budget"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_jolt(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -232,6 +232,34 @@ JOLT_API const char* jolt_last_error(void);
  * launch-count reporting). */
 JOLT_API uint64_t jolt_launch_count(void);
 
+/* Stage timing. While enabled, every stage of compress/decompress records a
+ * CUDA event before and after itself on the call's stream (no extra host
+ * synchronisation); jolt_profile_read waits for the recorded events and
+ * returns, per stage, the summed device time and the kernel launches.
+ * Enabling (or disabling) clears the counters. Not thread-safe. */
+enum {
+  JOLT_STAGE_COPY = 0,        /* bf16 working copies (un-RoPE keys)          */
+  JOLT_STAGE_FGRAM = 1,       /* feature Gram X_(d) X_(d)^T and ||X||^2      */
+  JOLT_STAGE_TOKEN_GRAM = 2,  /* exact mode: token Gram                      */
+  JOLT_STAGE_GEMM_XW = 3,     /* randomized: X * W (sketch, power steps)     */
+  JOLT_STAGE_GEMM_XTY = 4,    /* randomized: X^T * Y                         */
+  JOLT_STAGE_ORTH = 5,        /* randomized: fp64 CholeskyQR of Z            */
+  JOLT_STAGE_GEMM_GRAM = 6,   /* randomized: W^T W                           */
+  JOLT_STAGE_EIG = 7,         /* eigensolvers (+ the small k x k solves)     */
+  JOLT_STAGE_ALLOC = 8,       /* rate-distortion tables + lambda bisection   */
+  JOLT_STAGE_FIT = 9,         /* factors, projection, core                   */
+  JOLT_STAGE_RESIDUAL = 10,   /* residual, rotation, quantization, packing   */
+  JOLT_STAGE_DECOMPRESS = 11, /* decoder                                     */
+  JOLT_NUM_STAGES = 12
+};
+typedef struct {
+  double ms;
+  int64_t calls;
+  int64_t launches;
+} jolt_stage_stats;
+JOLT_API void jolt_profile_enable(int32_t on);
+JOLT_API jolt_status jolt_profile_read(jolt_stage_stats* out, int32_t n);
+
 #ifdef __cplusplus
 }
 #endif

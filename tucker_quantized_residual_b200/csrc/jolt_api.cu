@@ -46,6 +46,52 @@ void dev_free(void* p, cudaStream_t s) {
   cudaFreeAsync(p, s);
 }
 
+// ------------------------------------------------------------- profiling ---
+struct ProfRec {
+  int stage;
+  cudaEvent_t a, b;
+  int64_t launches;
+};
+static bool g_prof_on = false;
+static std::vector<ProfRec> g_prof;
+static std::vector<cudaEvent_t> g_prof_pool;
+
+static cudaEvent_t prof_event() {
+  if (!g_prof_pool.empty()) {
+    cudaEvent_t e = g_prof_pool.back();
+    g_prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+static void prof_clear() {
+  for (auto& r : g_prof) {
+    if (r.a) g_prof_pool.push_back(r.a);
+    if (r.b) g_prof_pool.push_back(r.b);
+  }
+  g_prof.clear();
+}
+
+ProfScope::ProfScope(int st, cudaStream_t s) : stage(st), stream(s), launches0(g_launches), slot(-1) {
+  if (!g_prof_on) return;
+  ProfRec r{st, prof_event(), prof_event(), 0};
+  cudaEventRecord(r.a, s);
+  slot = (int)g_prof.size();
+  g_prof.push_back(r);
+}
+
+void ProfScope::end() {
+  if (slot < 0) return;
+  cudaEventRecord(g_prof[slot].b, stream);
+  g_prof[slot].launches = (int64_t)(g_launches - launches0);
+  slot = -1;
+}
+
+ProfScope::~ProfScope() { end(); }
+
 // A bump region carved out of one device allocation.
 struct Arena {
   uint8_t* base = nullptr;
@@ -84,6 +130,10 @@ struct jolt_plan_s {
   int ncells = 0, nmin_max = 0, rmax_all = 0, lh_max = 0, nt_max = 0;
   std::vector<HostCell> hc;
   std::vector<CellDesc> cdesc;
+  CellDesc* cdesc_pinned = nullptr;
+  bool cdesc_valid = false;
+  const void* cdesc_k = nullptr;
+  const void* cdesc_v = nullptr;
   // device
   cudaStream_t init_stream = 0;
   Arena ws;
@@ -185,6 +235,26 @@ void jolt_default_options(jolt_options* o) {
 
 const char* jolt_last_error(void) { return g_err; }
 uint64_t jolt_launch_count(void) { return g_launches; }
+
+void jolt_profile_enable(int32_t on) {
+  prof_clear();
+  g_prof_on = on != 0;
+}
+
+jolt_status jolt_profile_read(jolt_stage_stats* out, int32_t n) {
+  if (!out || n < 1) { set_error("null output"); return JOLT_ERR_INVALID_ARG; }
+  for (int i = 0; i < n; ++i) out[i] = jolt_stage_stats{0.0, 0, 0};
+  for (auto& r : g_prof) {
+    if (r.stage < 0 || r.stage >= n) continue;
+    JOLT_CUDA_TRY(cudaEventSynchronize(r.b));
+    float ms = 0.0f;
+    JOLT_CUDA_TRY(cudaEventElapsedTime(&ms, r.a, r.b));
+    out[r.stage].ms += ms;
+    out[r.stage].calls += 1;
+    out[r.stage].launches += r.launches;
+  }
+  return JOLT_OK;
+}
 
 jolt_status jolt_set_allocator(jolt_alloc_fn a, jolt_free_fn f, void* ctx) {
   if ((a == nullptr) != (f == nullptr)) { set_error("alloc and free must both be set or both NULL"); return JOLT_ERR_INVALID_ARG; }
@@ -532,6 +602,16 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
 // Device descriptors of the cells for given K/V base pointers.
 static jolt_status upload_cells(jolt_plan_s* p, const void* k, const void* v, cudaStream_t s) {
   const jolt_layout& L = p->lay;
+  // descriptors depend only on the two base pointers: skip the copy when they
+  // are those of the previous call (the copy comes from pinned memory, so it
+  // never blocks the host on the stream)
+  if (p->cdesc_valid && p->cdesc_k == k && p->cdesc_v == v) return JOLT_OK;
+  if (!p->cdesc_pinned) {
+    JOLT_CUDA_TRY(cudaMallocHost(&p->cdesc_pinned, p->ncells * sizeof(CellDesc)));
+  } else {
+    // the previous upload may still be in flight
+    JOLT_CUDA_TRY(cudaStreamSynchronize(s));
+  }
   p->cdesc.resize(p->ncells);
   const size_t esz = L.dtype == JOLT_F32 ? 4 : 2;
   for (int i = 0; i < p->ncells; ++i) {
@@ -550,7 +630,11 @@ static jolt_status upload_cells(jolt_plan_s* p, const void* k, const void* v, cu
     d.rtmax = c.rmax;
     p->cdesc[i] = d;
   }
-  JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_cells, p->cdesc.data(), p->ncells * sizeof(CellDesc), cudaMemcpyHostToDevice, s));
+  memcpy(p->cdesc_pinned, p->cdesc.data(), p->ncells * sizeof(CellDesc));
+  JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_cells, p->cdesc_pinned, p->ncells * sizeof(CellDesc), cudaMemcpyHostToDevice, s));
+  p->cdesc_valid = true;
+  p->cdesc_k = k;
+  p->cdesc_v = v;
   return JOLT_OK;
 }
 
@@ -584,18 +668,21 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
   const jolt_layout& L = p->lay;
   const int nc = p->ncells, D = p->D, T = p->T, k = p->k;
   const int64_t kk = (int64_t)k * k;
+  ProfScope ps_copy(JOLT_STAGE_COPY, s);
   if (p->copy_k)
     JOLT_TRY(launch_make_xb(k_in, L.dtype == JOLT_F32, L.rope_theta_k > 0, p->d_cs, L.batch, L.n_layers, p->H, T, D,
                             L.stride_b, L.stride_l, L.stride_h, L.stride_t, p->Xk, s));
   if (p->copy_v)
     JOLT_TRY(launch_make_xb(v_in, L.dtype == JOLT_F32, 0, p->d_cs, L.batch, L.n_layers, p->H, T, D,
                             L.stride_b, L.stride_l, L.stride_h, L.stride_t, p->Xv, s));
+  ps_copy.end();
   umma::Maps m{};
   JOLT_TRY(x_maps(p, k_in, v_in, m));
   m.at = m.xk;
   m.bt = m.xk;
   // feature Gram (tensor cores, fp32 partials per row chunk, fp64 reduction)
   {
+    ProfScope ps(JOLT_STAGE_FGRAM, s);
     umma::Problem q = gemm_problem(p, umma::FG, status);
     q.BN = 128; q.N = 128; q.mt = p->fg_chunks; q.nt = 1;
     q.fg_chunks = p->fg_chunks; q.fg_spc = p->fg_spc;
@@ -606,6 +693,7 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
   // W_0^T = Omega^T
   JOLT_TRY(launch_omega(p->Wt, nc, k, p->Ncmax, p->d_Nc, p->d_cb, p->d_cis, seed, s));
   auto xw = [&]() -> jolt_status {
+    ProfScope ps(JOLT_STAGE_GEMM_XW, s);
     umma::Maps mm = m;
     JOLT_TRY(map_3d(&mm.bt, p->Wt, nc, k, p->Ncmax, p->Ncmax, p->BN));
     umma::Problem q = gemm_problem(p, umma::XW, status);
@@ -614,6 +702,7 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
     return launch_umma(mm, q, s);
   };
   auto xty = [&]() -> jolt_status {
+    ProfScope ps(JOLT_STAGE_GEMM_XTY, s);
     umma::Maps mm = m;
     JOLT_TRY(map_3d(&mm.bt, p->Yt, nc, k, T, p->tp, p->BN));
     umma::Problem q = gemm_problem(p, umma::XTY, status);
@@ -625,6 +714,7 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
   for (int it = 0; it < p->opt.power_iters; ++it) {
     JOLT_TRY(xty());
     // V = Z R^{-1} with Z^T Z = R^T R (fp64), stored as the next W^T
+    ProfScope ps(JOLT_STAGE_ORTH, s);
     JOLT_TRY(launch_gram_cols(p->Z, (int64_t)p->Ncmax * k, p->d_Nc, k, p->Gz, kk, nc, s));
     JOLT_TRY(launch_cholesky(p->Gz, kk, nullptr, 0, k, nc, status, s));
     JOLT_TRY(launch_trsm_rows(p->Z, (int64_t)p->Ncmax * k, p->Gz, kk, k, p->d_Nc, p->Ncmax, p->Wt,
@@ -637,11 +727,13 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
     umma::Maps mm = m;
     JOLT_TRY(map_3d(&mm.at, p->Yt, nc, k, T, p->tp, 128));
     JOLT_TRY(map_3d(&mm.bt, p->Yt, nc, k, T, p->tp, p->BN));
+    ProfScope ps(JOLT_STAGE_GEMM_GRAM, s);
     umma::Problem q = gemm_problem(p, umma::GRAM, status);
     q.M = k; q.N = k; q.Kdim = T; q.BN = p->BN; q.mt = (k + 127) / 128; q.nt = p->nt_k;
     q.out_f32 = p->GW32; q.out_cell_stride = kk;
     JOLT_TRY(launch_umma(mm, q, s));
   }
+  ProfScope ps_eig(JOLT_STAGE_EIG, s);
   JOLT_TRY(launch_cholesky(p->Rm, kk, p->GW32, kk, k, nc, status, s));
   // B B^T = R^{-T} (Z^T Z) R^{-1}, then its eigenpairs (and the feature spectrum)
   JOLT_TRY(launch_gram_cols(p->Z, (int64_t)p->Ncmax * k, p->d_Nc, k, p->P0, kk, nc, s));
@@ -657,6 +749,7 @@ static jolt_status run_random_fit(jolt_plan_s* p, const void* k_in, const void* 
                                   cudaStream_t s) {
   const int nc = p->ncells, T = p->T, k = p->k;
   const int64_t kk = (int64_t)k * k;
+  ProfScope ps(JOLT_STAGE_FIT, s);
   JOLT_TRY(launch_make_p(p->Rm, p->eVt, kk, k, d_out, p->P64, (int64_t)k * p->rmax_all, p->rmax_all, p->Pt,
                          (int64_t)p->rpad * p->kpad, p->kpad, nc, s));
   JOLT_TRY(launch_copy_out(d_out, p->d_rT_used, p->d_utp, nc, s));
@@ -677,15 +770,21 @@ static jolt_status run_spectra(jolt_plan_s* p, const void* k_in, const void* v_i
                                cudaStream_t s) {
   const int nc = p->ncells, D = p->D;
   if (p->opt.mode == JOLT_EXACT) {
+    ProfScope ps(JOLT_STAGE_FGRAM, s);
     JOLT_TRY(launch_fgram_x(p->d_cells, nc, D, p->d_cs, p->fchunk, p->d_fpart, s));
     JOLT_TRY(launch_sum_chunks(p->d_fpart, p->fchunk, D * D + 1, nc, p->d_Cd, p->d_nsq, s));
   }
   if (p->opt.mode == JOLT_EXACT) {
-    JOLT_TRY(launch_token_gram(p->d_cells, nc, p->nmin_max, p->d_cs, p->d_GT, s));
+    {
+      ProfScope ps(JOLT_STAGE_TOKEN_GRAM, s);
+      JOLT_TRY(launch_token_gram(p->d_cells, nc, p->nmin_max, p->d_cs, p->d_GT, s));
+    }
+    ProfScope ps(JOLT_STAGE_EIG, s);
     JOLT_TRY(launch_eigh(p->d_jobs_spec, 2 * nc, std::max(p->nmin_max, D), status, s));
   } else {
     JOLT_TRY(run_range_finder(p, k_in, v_in, seed, status, s));
   }
+  ProfScope ps_rd(JOLT_STAGE_ALLOC, s);
   JOLT_TRY(launch_rd_tables(p->d_rd_cells, nc, p->d_wT, p->d_wD, nullptr, p->d_tT, p->d_tD, p->d_nt,
                             p->d_nsq, status, s));
   return JOLT_OK;
@@ -712,6 +811,7 @@ extern "C" {
 
 void jolt_free_plan(jolt_plan_t* p) {
   if (!p) return;
+  if (p->cdesc_pinned) cudaFreeHost(p->cdesc_pinned);
   if (p->ws_alloc) dev_free(p->ws_alloc, p->init_stream);
   delete p;
 }
@@ -753,7 +853,11 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   jolt_status st;
   if ((st = upload_cells(p, k, v, s)) != JOLT_OK) return fail(st);
   if ((st = run_spectra(p, k, v, seed, h->d_status, s)) != JOLT_OK) return fail(st);
-  if ((st = run_allocation(p, B, p->d_eps2, h->d_state, h->d_choice, h->d_status, s)) != JOLT_OK) return fail(st);
+  {
+    ProfScope ps(JOLT_STAGE_ALLOC, s);
+    if ((st = run_allocation(p, B, p->d_eps2, h->d_state, h->d_choice, h->d_status, s)) != JOLT_OK) return fail(st);
+  }
+  ProfScope ps_fit(JOLT_STAGE_FIT, s);
   if ((st = launch_payload_layout(p->d_cells, h->d_choice, nc, p->G, h->payload, h->capacity, h->d_out,
                                   h->d_status, s)) != JOLT_OK) return fail(st);
   FitArgs fa{};
@@ -775,6 +879,8 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   ResidArgs ra{};
   ra.cells = p->d_cells; ra.cs = p->d_cs; ra.out = h->d_out; ra.M = p->d_M; ra.rmax_of = p->d_rmax;
   ra.G = p->G; ra.seed = seed;
+  ps_fit.end();
+  ProfScope ps_res(JOLT_STAGE_RESIDUAL, s);
   if ((st = launch_residual_simt(ra, nc, p->D, p->T, p->lh_max, s)) != JOLT_OK) return fail(st);
   *out = h;
   return JOLT_OK;
@@ -792,6 +898,7 @@ jolt_status jolt_decompress(const jolt_handle_t* h, void* k_out, void* v_out, co
     set_error("output strides must be even and stride_t >= head_dim"); return JOLT_ERR_UNSUPPORTED_SHAPE;
   }
   const int nc = p->ncells;
+  ProfScope ps(JOLT_STAGE_DECOMPRESS, s);
   JOLT_TRY(launch_core_m(h->d_out, p->d_cells, p->d_M, p->d_rmax, nc, p->D, p->rmax_all, p->lh_max, s));
   ResidArgs ra{};
   ra.cells = p->d_cells; ra.cs = p->d_cs; ra.out = h->d_out; ra.M = p->d_M; ra.rmax_of = p->d_rmax;

@@ -52,6 +52,18 @@ enum : int {
   DEV_ERR_INFEASIBLE = 16,
 };
 
+// ------------------------------------------------------------- profiling ---
+// Records a CUDA event pair around a stage when profiling is enabled.
+struct ProfScope {
+  ProfScope(int stage, cudaStream_t s);
+  ~ProfScope();
+  void end();
+  int stage;
+  cudaStream_t stream;
+  uint64_t launches0;
+  int slot;
+};
+
 // ------------------------------------------------------------- allocator ---
 void* dev_alloc(size_t bytes, cudaStream_t s);
 void dev_free(void* p, cudaStream_t s);

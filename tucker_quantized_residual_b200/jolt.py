@@ -83,7 +83,16 @@ _SIGS = {
     "jolt_set_allocator": (C.c_int, [_VP, _VP, _VP]),
     "jolt_last_error": (C.c_char_p, []),
     "jolt_launch_count": (_U64, []),
+    "jolt_profile_enable": (None, [_I32]),
+    "jolt_profile_read": (C.c_int, [C.c_void_p, _I32]),
 }
+
+STAGES = ["copy", "fgram", "token_gram", "gemm_xw", "gemm_xty", "orth", "gemm_gram", "eig", "alloc", "fit",
+          "residual", "decompress"]
+
+
+class jolt_stage_stats(C.Structure):
+    _fields_ = [("ms", C.c_double), ("calls", C.c_int64), ("launches", C.c_int64)]
 
 
 def load_library():
@@ -270,6 +279,17 @@ def jolt_residual_decode(codes, scales, rows: int, D: int, bits: int, group: int
                          stream=None) -> None:
     _check(load_library().jolt_residual_decode(_ptr(codes), _ptr(scales), rows, D, bits, group, int(seed),
                                                _ptr(e_hat), _stream(stream)))
+
+
+def jolt_profile_enable(on: bool) -> None:
+    load_library().jolt_profile_enable(1 if on else 0)
+
+
+def jolt_profile_read() -> dict:
+    """{stage: (ms, calls, launches)} summed since the last enable."""
+    arr = (jolt_stage_stats * len(STAGES))()
+    _check(load_library().jolt_profile_read(C.cast(arr, C.c_void_p), len(STAGES)))
+    return {name: (arr[i].ms, arr[i].calls, arr[i].launches) for i, name in enumerate(STAGES)}
 
 
 def jolt_last_error() -> str:
