@@ -203,6 +203,25 @@ JOLT_API jolt_status jolt_allocate(jolt_plan_t* plan, const double* t_t, int32_t
 JOLT_API jolt_status jolt_eps2(const int32_t* bits, int32_t n, int32_t group,
                       double* eps2, jolt_stream_t stream);
 
+/* jolt_eps2 without any device allocation, for callers that cannot allocate
+ * GPU memory while they run (an engine that reserved HBM for its KV pool up
+ * front and gives libraries no allocator, or a loop where an allocation is not
+ * allowed). The paper has no counterpart to this entry point; it computes the
+ * same values as jolt_eps2 with the same kernels.
+ *   bits: HOST, n entries (1 <= n <= 8) from {0,2,3,4,8}; group: 32, 64 or 128.
+ *   eps2_dev: DEVICE output of n doubles, owned by the caller.
+ * Asynchronous on `stream`; the caller synchronises before reading eps2_dev.
+ * Partial sums live in a static 9 KB device array that every GPU loading the
+ * library holds until exit (limit: 128 partial blocks x 9 slots, i.e. up to 8
+ * bit widths and any supported group). The first call on each device looks up
+ * that array's address (cudaGetSymbolAddress, with that device current); make
+ * this first call before any stream capture. All calls share the array and it
+ * keeps the last call's contents: calls whose work overlaps on the GPU race,
+ * so issue them on one stream or order them. Arguments beyond the limits
+ * return JOLT_ERR_INVALID_ARG with a message naming the limit. */
+JOLT_API jolt_status jolt_eps2_noalloc(const int32_t* bits, int32_t n, int32_t group,
+                                       double* eps2_dev, jolt_stream_t stream);
+
 /* The residual stage alone (Section 3, "Rotated low-bit residual"), for
  * rows of D fp32 values: r = D^-1/2 H_D diag(s) e with s from `seed`, then
  * absmax quantization to `bits` with one fp32 scale per `group` values and

@@ -78,6 +78,7 @@ _SIGS = {
     "jolt_allocate": (C.c_int, [_VP, C.POINTER(_D), _I32, C.POINTER(_D), _I32, C.POINTER(_D), _I64,
                                 C.POINTER(_I32), C.POINTER(_I64), C.POINTER(_D), C.POINTER(_I32), _VP]),
     "jolt_eps2": (C.c_int, [C.POINTER(_I32), _I32, _I32, C.POINTER(_D), _VP]),
+    "jolt_eps2_noalloc": (C.c_int, [C.POINTER(_I32), _I32, _I32, _VP, _VP]),
     "jolt_residual_encode": (C.c_int, [_VP, _I64, _I32, _I32, _I32, _U64, _VP, _VP, _VP]),
     "jolt_residual_decode": (C.c_int, [_VP, _VP, _I64, _I32, _I32, _I32, _U64, _VP, _VP]),
     "jolt_set_allocator": (C.c_int, [_VP, _VP, _VP]),
@@ -267,6 +268,13 @@ def jolt_eps2(bits: Sequence[int], group: int, stream=None) -> List[float]:
     out = (C.c_double * len(bits))()
     _check(load_library().jolt_eps2(b, len(bits), group, out, _stream(stream)))
     return list(out)
+
+
+def jolt_eps2_noalloc(bits: Sequence[int], group: int, out, stream=None) -> None:
+    """Same values as jolt_eps2, written to the device tensor `out` (float64,
+    len(bits) entries) without any device allocation inside the library."""
+    b = (C.c_int32 * len(bits))(*bits)
+    _check(load_library().jolt_eps2_noalloc(b, len(bits), group, _ptr(out), _stream(stream)))
 
 
 def jolt_residual_encode(e, D: int, bits: int, group: int, seed: int, codes, scales, stream=None) -> None:
