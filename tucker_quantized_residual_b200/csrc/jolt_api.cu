@@ -173,6 +173,11 @@ struct jolt_plan_s {
   // randomized mode (Section 3.1): sketch width k = q + p rounded up to 16,
   // GEMM tile width BN, padded extents, working buffers
   int k = 0, BN = 0, nt_k = 0, kpad = 0, rpad = 0, tp = 0, Ncmax = 0, fg_chunks = 0, fg_spc = 0, q_used = 0;
+  // tensor-core residual/decode streams: U_T^ rows and M^T, padded to 64 ranks
+  bool tc_in = false;
+  int rows_u = 0, rpad_m = 0;
+  uint16_t* Ut_ws = nullptr;
+  uint16_t* Mt_ws = nullptr;
   bool copy_k = false, copy_v = false;
   uint16_t* Xk = nullptr;  uint16_t* Xv = nullptr;
   uint16_t* Wt = nullptr;  uint16_t* Yt = nullptr;  uint16_t* Pt = nullptr;
@@ -419,6 +424,13 @@ jolt_status jolt_plan(const jolt_layout* L, int64_t byte_budget, const jolt_opti
     set_error("budget %lld below the cheapest allocation %lld", (long long)byte_budget, (long long)minsum);
     return JOLT_ERR_BUDGET_INFEASIBLE;
   }
+  p->tp = (p->T + 7) / 8 * 8;
+  p->rows_u = (p->rmax_all + 63) / 64 * 64;
+  p->rpad_m = p->rows_u;
+  // bf16 input whose strides TMA can address (16-byte multiples) takes the
+  // tensor-core residual stream; fp32 input uses the per-row kernel
+  p->tc_in = L->dtype == JOLT_BF16 && L->stride_t % 8 == 0 && L->stride_h % 8 == 0 && L->stride_l % 8 == 0 &&
+             L->stride_b % 8 == 0;
   jolt_status st = plan_build_workspace(p);
   if (st != JOLT_OK) { jolt_free_plan(p); return st; }
   *out = p;
@@ -467,6 +479,8 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
     p->d_api = A.take<int>((size_t)nc * p->achunk);
     p->d_cur = A.take<int>(nc);
     p->d_keep = A.take<int>(nc);
+    p->Ut_ws = A.take<uint16_t>((size_t)nc * p->rows_u * p->tp);
+    p->Mt_ws = A.take<uint16_t>((size_t)nc * p->lh_max * D * p->rpad_m);
     if (p->opt.mode == JOLT_RANDOMIZED) {
       const int k = p->k;
       const size_t kk = (size_t)k * k;
@@ -766,6 +780,39 @@ static jolt_status run_random_fit(jolt_plan_s* p, const void* k_in, const void* 
   return JOLT_OK;
 }
 
+// Residual (k_in != NULL) or decoding pass on tensor cores: the backbone
+// U_T^ M^_lh comes from the payload through two small re-layout kernels.
+static jolt_status run_stream(jolt_plan_s* p, const jolt_handle_s* h, const void* k_in, const void* v_in,
+                              void* k_out, void* v_out, const jolt_layout* ol, cudaStream_t s) {
+  const bool compress = k_in != nullptr;
+  const int nc = p->ncells, D = p->D;
+  const jolt_layout& L = p->lay;
+  JOLT_TRY(launch_m_transpose(h->d_out, p->d_cells, p->d_M, p->d_rmax, p->Mt_ws, p->lh_max, D, p->rpad_m, nc, s));
+  JOLT_TRY(launch_ut_to_ws(h->d_out, p->Ut_ws, p->rows_u, p->tp, nc, s));
+  StreamMaps m{};
+  JOLT_TRY(map_3d_box(&m.ut, p->Ut_ws, nc, p->rows_u, p->tp, p->tp, 64, 64));
+  JOLT_TRY(map_3d_box(&m.mt, p->Mt_ws, nc * p->lh_max, D, p->rpad_m, p->rpad_m, 64, D));
+  if (compress) {
+    JOLT_TRY(map_x5_box(&m.xk, k_in, L.batch, L.n_layers, p->H, p->T, D, L.stride_b, L.stride_l, L.stride_h,
+                        L.stride_t, 128));
+    JOLT_TRY(map_x5_box(&m.xv, v_in, L.batch, L.n_layers, p->H, p->T, D, L.stride_b, L.stride_l, L.stride_h,
+                        L.stride_t, 128));
+  } else {
+    m.xk = m.ut;
+    m.xv = m.ut;
+  }
+  StreamArgs a{};
+  a.ncells = nc; a.T = p->T; a.H = p->H; a.lhmax = p->lh_max; a.rpad_m = p->rpad_m; a.G = p->G;
+  a.cells = p->d_cells; a.outs = h->d_out; a.cs = p->d_cs; a.seed = h->seed;
+  if (!compress) {
+    a.out_k = reinterpret_cast<uint16_t*>(k_out);
+    a.out_v = reinterpret_cast<uint16_t*>(v_out);
+    a.osb = ol->stride_b; a.osl = ol->stride_l; a.osh = ol->stride_h; a.ost = ol->stride_t;
+  }
+  a.status = h->d_status;
+  return launch_stream(compress, D, m, a, s);
+}
+
 static jolt_status run_spectra(jolt_plan_s* p, const void* k_in, const void* v_in, uint64_t seed, int* status,
                                cudaStream_t s) {
   const int nc = p->ncells, D = p->D;
@@ -881,7 +928,11 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   ra.G = p->G; ra.seed = seed;
   ps_fit.end();
   ProfScope ps_res(JOLT_STAGE_RESIDUAL, s);
-  if ((st = launch_residual_simt(ra, nc, p->D, p->T, p->lh_max, s)) != JOLT_OK) return fail(st);
+  if (p->tc_in && reinterpret_cast<uintptr_t>(k) % 16 == 0 && reinterpret_cast<uintptr_t>(v) % 16 == 0) {
+    if ((st = run_stream(p, h, k, v, nullptr, nullptr, nullptr, s)) != JOLT_OK) return fail(st);
+  } else {
+    if ((st = launch_residual_simt(ra, nc, p->D, p->T, p->lh_max, s)) != JOLT_OK) return fail(st);
+  }
   *out = h;
   return JOLT_OK;
 }
@@ -905,7 +956,10 @@ jolt_status jolt_decompress(const jolt_handle_t* h, void* k_out, void* v_out, co
   ra.G = p->G; ra.seed = h->seed;
   ra.out_k = reinterpret_cast<uint16_t*>(k_out); ra.out_v = reinterpret_cast<uint16_t*>(v_out);
   ra.osb = L.stride_b; ra.osl = L.stride_l; ra.osh = L.stride_h; ra.ost = L.stride_t;
-  JOLT_TRY(launch_decompress_simt(ra, nc, p->D, p->T, p->lh_max, s));
+  const bool tc_out = L.stride_t % 8 == 0 && L.stride_h % 8 == 0 && L.stride_l % 8 == 0 && L.stride_b % 8 == 0 &&
+                      (reinterpret_cast<uintptr_t>(k_out) % 16) == 0 && (reinterpret_cast<uintptr_t>(v_out) % 16) == 0;
+  if (tc_out) JOLT_TRY(run_stream(p, h, nullptr, nullptr, k_out, v_out, &L, s));
+  else JOLT_TRY(launch_decompress_simt(ra, nc, p->D, p->T, p->lh_max, s));
   return JOLT_OK;
 }
 

@@ -181,3 +181,32 @@ jolt_status launch_fgram_reduce(const float* part, int nchunk, int D, double* co
                                 int ncells, cudaStream_t s);
 
 }  // namespace jolt
+
+namespace jolt {
+// ------------------------------------------- tensor-core residual streams --
+struct StreamMaps {
+  CUtensorMap ut;   // U_T^ workspace [cells][rows][tp], box {64 t, 64 r}
+  CUtensorMap mt;   // M^T workspace [cells*lhmax][D][rpad_m], box {64 r, D}
+  CUtensorMap xk;   // key input, box {64 d, 128 t, 1, 1, 1}
+  CUtensorMap xv;   // value input
+};
+struct StreamArgs {
+  int ncells, T, H, lhmax, rpad_m, G;
+  const CellDesc* cells;
+  const CellOut* outs;
+  const float2* cs;
+  uint64_t seed;
+  uint16_t* out_k;
+  uint16_t* out_v;
+  int64_t osb, osl, osh, ost;
+  int* status;
+};
+jolt_status launch_stream(bool compress, int D, const StreamMaps& m, const StreamArgs& a, cudaStream_t s);
+jolt_status launch_ut_to_ws(const CellOut* outs, uint16_t* ws, int rows, int tp, int ncells, cudaStream_t s);
+jolt_status launch_m_transpose(const CellOut* outs, const CellDesc* cells, uint16_t* const* M, const int* rmax_of,
+                               uint16_t* Mt, int lhmax, int D, int rpad, int ncells, cudaStream_t s);
+jolt_status map_x5_box(CUtensorMap* m, const void* base, int B, int L, int H, int T, int D, int64_t sb,
+                       int64_t sl, int64_t sh, int64_t st, int box_t);
+jolt_status map_3d_box(CUtensorMap* m, const void* base, int cells, int rows, int cols, int64_t pitch,
+                       int box_cols, int box_rows);
+}  // namespace jolt

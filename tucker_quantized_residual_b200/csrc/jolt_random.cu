@@ -58,6 +58,22 @@ jolt_status map_x5(CUtensorMap* m, const void* base, int B, int L, int H, int T,
   return make_map(m, base, 5, dims, str, box);
 }
 
+jolt_status map_x5_box(CUtensorMap* m, const void* base, int B, int L, int H, int T, int D, int64_t sb,
+                       int64_t sl, int64_t sh, int64_t st, int box_t) {
+  uint64_t dims[5] = {(uint64_t)D, (uint64_t)T, (uint64_t)H, (uint64_t)L, (uint64_t)B};
+  uint64_t str[4] = {(uint64_t)st * 2, (uint64_t)sh * 2, (uint64_t)sl * 2, (uint64_t)sb * 2};
+  uint32_t box[5] = {64, (uint32_t)box_t, 1, 1, 1};
+  return make_map(m, base, 5, dims, str, box);
+}
+
+jolt_status map_3d_box(CUtensorMap* m, const void* base, int cells, int rows, int cols, int64_t pitch,
+                       int box_cols, int box_rows) {
+  uint64_t dims[3] = {(uint64_t)cols, (uint64_t)rows, (uint64_t)cells};
+  uint64_t str[2] = {(uint64_t)pitch * 2, (uint64_t)pitch * 2 * rows};
+  uint32_t box[3] = {(uint32_t)box_cols, (uint32_t)box_rows, 1};
+  return make_map(m, base, 3, dims, str, box);
+}
+
 // [cells][rows][cols] bf16 with row pitch `pitch` elements; box {64, box_rows}
 jolt_status map_3d(CUtensorMap* m, const void* base, int cells, int rows, int cols, int64_t pitch,
                    int box_rows) {

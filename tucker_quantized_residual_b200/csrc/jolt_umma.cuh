@@ -79,7 +79,9 @@ jolt_status launch_umma(const umma::Maps& maps, const umma::Problem& p, cudaStre
 
 }  // namespace jolt
 
-#ifdef JOLT_UMMA_IMPL
+#if defined(JOLT_UMMA_IMPL) || defined(JOLT_PTX_HELPERS)
+#ifndef JOLT_PTX_HELPERS_DONE
+#define JOLT_PTX_HELPERS_DONE
 namespace jolt {
 namespace umma {
 
@@ -189,6 +191,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
 }
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+}  // namespace umma
+}  // namespace jolt
+#endif  // JOLT_PTX_HELPERS_DONE
+#endif  // helpers
+
+#ifdef JOLT_UMMA_IMPL
+namespace jolt {
+namespace umma {
 
 // Tile -> (cell, m0, n0)
 __device__ __forceinline__ void tile_coords(const Problem& p, int tile, int& cell, int& m0, int& n0) {
