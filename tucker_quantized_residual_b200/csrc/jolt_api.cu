@@ -150,6 +150,7 @@ struct jolt_plan_s {
   int* d_rmax = nullptr;
   int* d_nlh = nullptr;
   int* d_rT_used = nullptr;      // r_T per cell (device copy for Y gram)
+  int* d_Dn = nullptr;           // D per cell (eigenvector count of the D x D solves)
   // per-cell arrays of pointers (device)
   double** d_GT = nullptr;  double** d_ZT = nullptr;  double** d_VtT = nullptr;
   double** d_wT = nullptr;  double** d_Cd = nullptr;  double** d_wD = nullptr;
@@ -185,6 +186,8 @@ struct jolt_plan_s {
   double* Gz = nullptr;    double* Rm = nullptr;    double* P0 = nullptr;   double* X1 = nullptr;
   double* MB = nullptr;    double* eZ = nullptr;    double* eVt = nullptr;  double* ew = nullptr;
   double* ework = nullptr; double* trs = nullptr;   double* P64 = nullptr;
+  double* eF = nullptr;    float* Ri32 = nullptr;   double* RTk = nullptr;
+  std::vector<double*> h_FT;     // exact mode: inverse-iteration scratch per cell
   int* d_cl0 = nullptr; int* d_cb = nullptr; int* d_cLg = nullptr; int* d_ckind = nullptr;
   int* d_Nc = nullptr; int* d_cis = nullptr;
   uint16_t** d_utp = nullptr;
@@ -431,6 +434,19 @@ jolt_status jolt_plan(const jolt_layout* L, int64_t byte_budget, const jolt_opti
   // tensor-core residual stream; fp32 input uses the per-row kernel
   p->tc_in = L->dtype == JOLT_BF16 && L->stride_t % 8 == 0 && L->stride_h % 8 == 0 && L->stride_l % 8 == 0 &&
              L->stride_b % 8 == 0;
+  if (!g_alloc) {
+    // With the default allocator, keep freed blocks in the device's default
+    // pool instead of returning them at every synchronisation: a handle's
+    // payload (gigabytes for long contexts) is then reused by the next call
+    // rather than mapped again.
+    int dev = 0;
+    cudaMemPool_t pool;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+      uint64_t thr = UINT64_MAX;
+      cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr);
+    }
+    cudaGetLastError();
+  }
   jolt_status st = plan_build_workspace(p);
   if (st != JOLT_OK) { jolt_free_plan(p); return st; }
   *out = p;
@@ -466,6 +482,7 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
     p->d_rmax = A.take<int>(nc);
     p->d_nlh = A.take<int>(nc);
     p->d_rT_used = A.take<int>(nc);
+    p->d_Dn = A.take<int>(nc);
     p->d_GT = A.take<double*>(nc); p->d_ZT = A.take<double*>(nc); p->d_VtT = A.take<double*>(nc);
     p->d_wT = A.take<double*>(nc); p->d_Cd = A.take<double*>(nc); p->d_wD = A.take<double*>(nc);
     p->d_nsq = A.take<double*>(nc); p->d_tT = A.take<double*>(nc); p->d_tD = A.take<double*>(nc);
@@ -497,8 +514,11 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
       p->Gz = A.take<double>(nc * kk); p->Rm = A.take<double>(nc * kk); p->P0 = A.take<double>(nc * kk);
       p->X1 = A.take<double>(nc * kk); p->MB = A.take<double>(nc * kk); p->eZ = A.take<double>(nc * kk);
       p->eVt = A.take<double>(nc * kk); p->ew = A.take<double>((size_t)nc * k);
-      p->ework = A.take<double>((size_t)nc * k);
-      p->trs = A.take<double>((size_t)nc * p->Ncmax * k);
+      p->ework = A.take<double>((size_t)nc * 3 * k);
+      p->eF = A.take<double>((size_t)nc * p->rmax_all * 5 * k);
+      p->Ri32 = A.take<float>((size_t)nc * kk);
+      p->RTk = A.take<double>((size_t)nc * kk);
+      p->trs = nullptr;
       p->P64 = A.take<double>((size_t)nc * k * p->rmax_all);
       p->d_cl0 = A.take<int>(nc); p->d_cb = A.take<int>(nc); p->d_cLg = A.take<int>(nc);
       p->d_ckind = A.take<int>(nc); p->d_Nc = A.take<int>(nc); p->d_cis = A.take<int>(nc);
@@ -507,7 +527,7 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
     }
     // per-cell buffers
     std::vector<double*> GT(nc), ZT(nc), VtT(nc), wT(nc), Cd(nc), wD(nc), nsq(nc), tT(nc), tD(nc),
-        Y(nc), CY(nc), VtY(nc), wY(nc), ZY(nc), Uf(nc), workT(nc), workD(nc), workY(nc);
+        Y(nc), CY(nc), VtY(nc), wY(nc), ZY(nc), Uf(nc), workT(nc), workD(nc), workY(nc), FT(nc), FY(nc);
     std::vector<uint16_t*> M(nc);
     const bool rnd = p->opt.mode == JOLT_RANDOMIZED;
     for (int i = 0; i < nc; ++i) {
@@ -519,15 +539,16 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
         ZT[i] = A.take<double>((size_t)n * n);
         VtT[i] = A.take<double>((size_t)n * n);
         wT[i] = A.take<double>(n);
-        workT[i] = A.take<double>(n);
+        workT[i] = A.take<double>(3 * n);
+        FT[i] = A.take<double>((size_t)c.rmax * 5 * n);
         Uf[i] = (T > c.N) ? A.take<double>((size_t)c.rmax * T) : nullptr;
       } else {
-        GT[i] = ZT[i] = VtT[i] = Uf[i] = workT[i] = nullptr;
+        GT[i] = ZT[i] = VtT[i] = Uf[i] = workT[i] = FT[i] = nullptr;
         wT[i] = A.take<double>(c.nt);
       }
       Cd[i] = A.take<double>((size_t)D * D);
       wD[i] = A.take<double>(D);
-      workD[i] = A.take<double>(D);
+      workD[i] = A.take<double>(3 * D);
       nsq[i] = A.take<double>(1);
       tT[i] = A.take<double>(c.nt + 1);
       tD[i] = A.take<double>(D + 1);
@@ -536,7 +557,8 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
       VtY[i] = A.take<double>((size_t)D * D);
       wY[i] = A.take<double>(D);
       ZY[i] = A.take<double>((size_t)D * D);
-      workY[i] = A.take<double>(D);
+      workY[i] = A.take<double>(3 * D);
+      FY[i] = A.take<double>((size_t)5 * D * D);
       M[i] = A.take<uint16_t>((size_t)LH * c.rmax * D);
     }
     if (pass == 0) {
@@ -566,14 +588,19 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
       ntv[i] = c.nt;
       rmaxv[i] = c.rmax;
       nlhv[i] = c.Lg * p->H;
-      js[i] = EighJob{rnd ? 0 : c.nmin, 1, GT[i], wT[i], VtT[i], ZT[i], workT[i]};
-      js[nc + i] = EighJob{D, 0, Cd[i], wD[i], nullptr, nullptr, workD[i]};
-      jf[i] = EighJob{D, 1, CY[i], wY[i], VtY[i], ZY[i], workY[i]};
+      js[i] = EighJob{rnd ? 0 : c.nmin, 1, GT[i], wT[i], VtT[i], ZT[i], workT[i], FT[i]};
+      js[nc + i] = EighJob{D, 0, Cd[i], wD[i], nullptr, nullptr, workD[i], nullptr};
+      jf[i] = EighJob{D, 1, CY[i], wY[i], VtY[i], ZY[i], workY[i], FY[i]};
     }
     JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_rd_cells, rdc.data(), nc * sizeof(CellRD), cudaMemcpyHostToDevice, s));
     JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_nt, ntv.data(), nc * sizeof(int), cudaMemcpyHostToDevice, s));
     JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_rmax, rmaxv.data(), nc * sizeof(int), cudaMemcpyHostToDevice, s));
     JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_nlh, nlhv.data(), nc * sizeof(int), cudaMemcpyHostToDevice, s));
+    {
+      std::vector<int> dv(nc, D);
+      JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_Dn, dv.data(), nc * sizeof(int), cudaMemcpyHostToDevice, s));
+      JOLT_CUDA_TRY(cudaStreamSynchronize(s));
+    }
     JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_jobs_spec, js.data(), js.size() * sizeof(EighJob), cudaMemcpyHostToDevice, s));
     JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_jobs_fit, jf.data(), jf.size() * sizeof(EighJob), cudaMemcpyHostToDevice, s));
 #define UP(dst, v) JOLT_CUDA_TRY(cudaMemcpyAsync(dst, v.data(), nc * sizeof(v[0]), cudaMemcpyHostToDevice, s))
@@ -594,8 +621,8 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
         l0v[i] = c.l0; bv[i] = c.seq; lgv[i] = c.Lg; kindv[i] = c.kind; ncv[i] = c.N;
         cisv[i] = 2 * c.group + c.kind;
         jr[i] = EighJob{k, 1, p->MB + i * kk, p->ew + (size_t)i * k, p->eVt + i * kk, p->eZ + i * kk,
-                        p->ework + (size_t)i * k};
-        jr[nc + i] = EighJob{D, 0, Cd[i], wD[i], nullptr, nullptr, workD[i]};
+                        p->ework + (size_t)i * 3 * k, p->eF + (size_t)i * p->rmax_all * 5 * k};
+        jr[nc + i] = EighJob{D, 0, Cd[i], wD[i], nullptr, nullptr, workD[i], nullptr};
       }
       UPI(p->d_cl0, l0v); UPI(p->d_cb, bv); UPI(p->d_cLg, lgv); UPI(p->d_ckind, kindv);
       UPI(p->d_Nc, ncv); UPI(p->d_cis, cisv);
@@ -730,9 +757,13 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
     // V = Z R^{-1} with Z^T Z = R^T R (fp64), stored as the next W^T
     ProfScope ps(JOLT_STAGE_ORTH, s);
     JOLT_TRY(launch_gram_cols(p->Z, (int64_t)p->Ncmax * k, p->d_Nc, k, p->Gz, kk, nc, s));
-    JOLT_TRY(launch_cholesky(p->Gz, kk, nullptr, 0, k, nc, status, s));
-    JOLT_TRY(launch_trsm_rows(p->Z, (int64_t)p->Ncmax * k, p->Gz, kk, k, p->d_Nc, p->Ncmax, p->Wt,
-                              (int64_t)k * p->Ncmax, p->Ncmax, p->trs, (int64_t)p->Ncmax * k, nc, s));
+    JOLT_TRY(launch_chol_blocked(p->Gz, p->RTk, kk, nullptr, k, nc, status, s));
+    TrsmArgs ta{};
+    ta.R = p->Gz; ta.RT = p->RTk; ta.r_cell = kk; ta.k = k; ta.backward = 0;
+    ta.B = p->Z; ta.b64 = 0; ta.b_cell = (int64_t)p->Ncmax * k; ta.ldb_r = k; ta.ldb_c = 1;
+    ta.rows_of = p->d_Nc;
+    ta.X16 = p->Wt; ta.x16_cell = (int64_t)k * p->Ncmax; ta.ld16_r = 1; ta.ld16_c = p->Ncmax;
+    JOLT_TRY(launch_trsm_rows2(ta, p->Ncmax, nc, s));
     JOLT_TRY(xw());
   }
   JOLT_TRY(xty());
@@ -748,11 +779,23 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
     JOLT_TRY(launch_umma(mm, q, s));
   }
   ProfScope ps_eig(JOLT_STAGE_EIG, s);
-  JOLT_TRY(launch_cholesky(p->Rm, kk, p->GW32, kk, k, nc, status, s));
-  // B B^T = R^{-T} (Z^T Z) R^{-1}, then its eigenpairs (and the feature spectrum)
+  JOLT_TRY(launch_chol_blocked(p->Rm, p->RTk, kk, p->GW32, k, nc, status, s));
+  // B B^T = R^{-T} (Z^T Z) R^{-1}: Y1 = P0 R^{-1}, then (Y1^T) R^{-1}
   JOLT_TRY(launch_gram_cols(p->Z, (int64_t)p->Ncmax * k, p->d_Nc, k, p->P0, kk, nc, s));
-  JOLT_TRY(launch_bbt(p->Rm, p->P0, p->X1, p->MB, kk, k, nc, s));
-  JOLT_TRY(launch_eigh(p->d_jobs_rand, 2 * nc, std::max(k, D), status, s));
+  {
+    TrsmArgs ta{};
+    ta.R = p->Rm; ta.RT = p->RTk; ta.r_cell = kk; ta.k = k; ta.backward = 0;
+    ta.B = p->P0; ta.b64 = 1; ta.b_cell = kk; ta.ldb_r = k; ta.ldb_c = 1; ta.rows_fixed = k;
+    ta.X64 = p->X1; ta.x64_cell = kk; ta.ld64_r = k; ta.ld64_c = 1;
+    JOLT_TRY(launch_trsm_rows2(ta, k, nc, s));
+    ta.B = p->X1; ta.ldb_r = 1; ta.ldb_c = k;
+    ta.X64 = p->MB;
+    JOLT_TRY(launch_trsm_rows2(ta, k, nc, s));
+    JOLT_TRY(launch_symmetrize(p->MB, kk, k, nc, s));
+  }
+  // spectra only here: eigenvectors follow the allocation (top r_T only)
+  JOLT_TRY(launch_tridiag(p->d_jobs_rand, 2 * nc, std::max(k, D), s));
+  JOLT_TRY(launch_bisect(p->d_jobs_rand, 2 * nc, std::max(k, D), s));
   JOLT_TRY(launch_rand_spectrum(p->ew, k, p->q_used, p->d_nsq, p->d_wT, nc, s));
   return JOLT_OK;
 }
@@ -764,9 +807,21 @@ static jolt_status run_random_fit(jolt_plan_s* p, const void* k_in, const void* 
   const int nc = p->ncells, T = p->T, k = p->k;
   const int64_t kk = (int64_t)k * k;
   ProfScope ps(JOLT_STAGE_FIT, s);
-  JOLT_TRY(launch_make_p(p->Rm, p->eVt, kk, k, d_out, p->P64, (int64_t)k * p->rmax_all, p->rmax_all, p->Pt,
-                         (int64_t)p->rpad * p->kpad, p->kpad, nc, s));
   JOLT_TRY(launch_copy_out(d_out, p->d_rT_used, p->d_utp, nc, s));
+  {
+    ProfScope pe(JOLT_STAGE_EIG, s);
+    JOLT_TRY(launch_eigvecs(p->d_jobs_rand, nc, p->rmax_all, p->d_rT_used, s));
+  }
+  {
+    // P = R^{-1} U_B[:, :r_T]: rows of P^T solve x R^T = u (backward)
+    TrsmArgs ta{};
+    ta.R = p->Rm; ta.RT = p->RTk; ta.r_cell = kk; ta.k = k; ta.backward = 1;
+    ta.B = p->eVt; ta.b64 = 1; ta.b_cell = kk; ta.ldb_r = k; ta.ldb_c = 1;
+    ta.rows_of = p->d_rT_used;
+    ta.X64 = p->P64; ta.x64_cell = (int64_t)k * p->rmax_all; ta.ld64_r = 1; ta.ld64_c = p->rmax_all;
+    ta.X16 = p->Pt; ta.x16_cell = (int64_t)p->rpad * p->kpad; ta.ld16_r = p->kpad; ta.ld16_c = 1;
+    JOLT_TRY(launch_trsm_rows2(ta, p->rmax_all, nc, s));
+  }
   umma::Maps m{};
   JOLT_TRY(x_maps(p, k_in, v_in, m));
   JOLT_TRY(map_3d(&m.at, p->Yt, nc, k, T, p->tp, 64));
@@ -826,8 +881,10 @@ static jolt_status run_spectra(jolt_plan_s* p, const void* k_in, const void* v_i
       ProfScope ps(JOLT_STAGE_TOKEN_GRAM, s);
       JOLT_TRY(launch_token_gram(p->d_cells, nc, p->nmin_max, p->d_cs, p->d_GT, s));
     }
+    // spectra only: the token eigenvectors follow the allocation (top r_T)
     ProfScope ps(JOLT_STAGE_EIG, s);
-    JOLT_TRY(launch_eigh(p->d_jobs_spec, 2 * nc, std::max(p->nmin_max, D), status, s));
+    JOLT_TRY(launch_tridiag(p->d_jobs_spec, 2 * nc, std::max(p->nmin_max, D), s));
+    JOLT_TRY(launch_bisect(p->d_jobs_spec, 2 * nc, std::max(p->nmin_max, D), s));
   } else {
     JOLT_TRY(run_range_finder(p, k_in, v_in, seed, status, s));
   }
@@ -912,6 +969,11 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   fa.VtT = p->d_VtT; fa.wT = p->d_wT; fa.Uf = p->d_Uf; fa.Y = p->d_Y; fa.rmax_of = p->d_rmax;
   fa.VtY = p->d_VtY; fa.M = p->d_M;
   if (p->opt.mode == JOLT_EXACT) {
+    if ((st = launch_copy_rt(h->d_out, p->d_rT_used, nc, s)) != JOLT_OK) return fail(st);
+    {
+      ProfScope pe(JOLT_STAGE_EIG, s);
+      if ((st = launch_eigvecs(p->d_jobs_spec, nc, p->rmax_all, p->d_rT_used, s)) != JOLT_OK) return fail(st);
+    }
     if ((st = launch_ut_exact(fa, p->T, p->rmax_all, s)) != JOLT_OK) return fail(st);
     if ((st = launch_project_y(fa, p->T, p->rmax_all, p->lh_max, s)) != JOLT_OK) return fail(st);
   } else {
@@ -921,7 +983,9 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   if ((st = launch_copy_rt(h->d_out, p->d_rT_used, nc, s)) != JOLT_OK) return fail(st);
   if ((st = launch_fgram_rows(p->d_Y, p->d_rT_used, p->d_rmax, p->d_nlh, nc, p->D, p->fchunk, p->d_fpart, s)) != JOLT_OK) return fail(st);
   if ((st = launch_sum_chunks(p->d_fpart, p->fchunk, p->D * p->D + 1, nc, p->d_CY, nullptr, s)) != JOLT_OK) return fail(st);
-  if ((st = launch_eigh(p->d_jobs_fit, nc, p->D, h->d_status, s)) != JOLT_OK) return fail(st);
+  if ((st = launch_tridiag(p->d_jobs_fit, nc, p->D, s)) != JOLT_OK) return fail(st);
+  if ((st = launch_bisect(p->d_jobs_fit, nc, p->D, s)) != JOLT_OK) return fail(st);
+  if ((st = launch_eigvecs(p->d_jobs_fit, nc, p->D, p->d_Dn, s)) != JOLT_OK) return fail(st);
   if ((st = launch_core(fa, p->rmax_all, p->lh_max, s)) != JOLT_OK) return fail(st);
   ResidArgs ra{};
   ra.cells = p->d_cells; ra.cs = p->d_cs; ra.out = h->d_out; ra.M = p->d_M; ra.rmax_of = p->d_rmax;

@@ -13,11 +13,15 @@ struct EighJob {
   double* w;      // n, descending
   double* Vt;     // n*n, row j = eigenvector j (if want_vec)
   double* Z;      // n*n scratch (if want_vec)
-  double* work;   // n scratch
+  double* work;   // n scratch (3n for the split solver: d, e, beta)
+  double* F;      // split solver: 5n doubles per requested eigenvector
 };
 
 jolt_status launch_eigh(const EighJob* jobs_dev, int njobs, int nmax, int* status, cudaStream_t s);
 size_t eigh_smem_bytes(int nmax);
+jolt_status launch_tridiag(const EighJob* jobs, int njobs, int nmax, cudaStream_t s);
+jolt_status launch_bisect(const EighJob* jobs, int njobs, int nmax, cudaStream_t s);
+jolt_status launch_eigvecs(const EighJob* jobs, int njobs, int nvec_max, const int* nvec, cudaStream_t s);
 jolt_status launch_fgram_x(const CellDesc* cells, int ncells, int D, const float2* cs, int nchunk,
                            double* partial, cudaStream_t s);
 jolt_status launch_fgram_rows(const double* const* Y, const int* nrow_used, const int* rmax_of,
@@ -167,6 +171,9 @@ jolt_status launch_cholesky(double* A, int64_t a_cell, const float* src32, int64
 jolt_status launch_trsm_rows(const float* Z, int64_t z_cell, const double* R, int64_t r_cell, int k, const int* Nc,
                              int Ncmax, uint16_t* Wt, int64_t w_cell, int ldw, double* scratch, int64_t s_cell,
                              int ncells, cudaStream_t s);
+jolt_status launch_orth_apply(const double* R, int64_t r_cell, int k, float* Ri, double* X, int64_t x_cell,
+                              const float* Z, int64_t z_cell, const int* Nc, int Ncmax, uint16_t* Wt, int64_t w_cell,
+                              int ldw, int ncells, cudaStream_t s);
 jolt_status launch_bbt(const double* R, const double* P, double* X1, double* M, int64_t cs, int k, int ncells,
                        cudaStream_t s);
 jolt_status launch_rand_spectrum(const double* w_eig, int64_t cs, int q, const double* const* normsq,
@@ -209,4 +216,28 @@ jolt_status map_x5_box(CUtensorMap* m, const void* base, int B, int L, int H, in
                        int64_t sl, int64_t sh, int64_t st, int box_t);
 jolt_status map_3d_box(CUtensorMap* m, const void* base, int cells, int rows, int cols, int64_t pitch,
                        int box_cols, int box_rows);
+}  // namespace jolt
+
+namespace jolt {
+// ------------------------------------------ batched dense fp64 (k x k) -----
+struct TrsmArgs {
+  const double* R;      // upper R (k x k, row-major), read by the backward solve
+  const double* RT;     // R^T (k x k, row-major), read by the forward solve
+  int64_t r_cell;
+  int k;
+  int backward;         // 0: X R = B, 1: X R^T = B
+  const void* B;        // element (r, j) at B[cell*b_cell + r*ldb_r + j*ldb_c]
+  int b64;              // 1: fp64, 0: fp32
+  int64_t b_cell, ldb_r, ldb_c;
+  const int* rows_of;   // rows per cell (null: rows_fixed)
+  int rows_fixed;
+  double* X64;          // optional fp64 output at X64[cell*x64_cell + r*ld64_r + j*ld64_c]
+  int64_t x64_cell, ld64_r, ld64_c;
+  uint16_t* X16;        // optional bf16 output at X16[cell*x16_cell + r*ld16_r + j*ld16_c]
+  int64_t x16_cell, ld16_r, ld16_c;
+};
+jolt_status launch_chol_blocked(double* G, double* RT, int64_t cs, const float* src32, int k, int ncells, int* status,
+                                cudaStream_t s);
+jolt_status launch_trsm_rows2(const TrsmArgs& a, int rows_max, int ncells, cudaStream_t s);
+jolt_status launch_symmetrize(double* M, int64_t cs, int k, int ncells, cudaStream_t s);
 }  // namespace jolt

@@ -441,9 +441,260 @@ __global__ void __launch_bounds__(EIG_THREADS) k_eigh(const EighJob* __restrict_
 
 size_t eigh_smem_bytes(int nmax) { return (size_t)(6 * nmax + 32) * sizeof(double); }
 
+// ------------------------------------------- split eigensolver (big n) -----
+// For the token-mode matrices only the spectrum is needed before the
+// allocation and only the leading r_T eigenvectors after it, so the solver is
+// split: (1) Householder tridiagonalization, one block per matrix, leaving
+// the reflectors in A's columns and d, e, beta in work[0..3n); (2) every
+// eigenvalue by bisection on Sturm counts, one thread per eigenvalue;
+// (3) after the allocation, eigenvectors of the leading r eigenvalues by
+// inverse iteration on the tridiagonal matrix, back-transformed by the
+// reflectors, one warp per vector over many blocks.
+
+__global__ void __launch_bounds__(EIG_THREADS) k_tridiag(const EighJob* __restrict__ jobs) {
+  const EighJob J = jobs[blockIdx.x];
+  const int n = J.n;
+  if (n <= 0) return;
+  extern __shared__ double sh[];
+  double* v = sh;            // n
+  double* p = v + n;         // n
+  double* red = p + n;       // 32
+  double* A = J.A;
+  double* dd = J.work;
+  double* ee = dd + n;
+  double* tau = ee + n;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5, nwarp = nt >> 5;
+  for (int k = 0; k + 2 < n; ++k) {
+    const int m = n - k - 1;
+    for (int i = tid; i < m; i += nt) v[i] = A[(int64_t)(k + 1 + i) * n + k];
+    __syncthreads();
+    double s = 0.0;
+    for (int i = 1 + tid; i < m; i += nt) s += v[i] * v[i];
+    s = block_sum(s, red);
+    const double x0 = v[0];
+    if (s == 0.0) {
+      if (tid == 0) { dd[k] = A[(int64_t)k * n + k]; ee[k] = x0; tau[k] = 0.0; }
+      __syncthreads();
+      continue;
+    }
+    const double nrm = sqrt(x0 * x0 + s);
+    const double alpha = (x0 <= 0.0) ? nrm : -nrm;
+    const double v0 = x0 - alpha;
+    const double beta = 2.0 / (s + v0 * v0);
+    __syncthreads();
+    if (tid == 0) v[0] = v0;
+    __syncthreads();
+    for (int i = warp; i < m; i += nwarp) {
+      const double* row = A + (int64_t)(k + 1 + i) * n + (k + 1);
+      double acc = 0.0;
+      for (int j = lane; j < m; j += 32) acc += row[j] * v[j];
+      acc = warp_sum(acc);
+      if (lane == 0) p[i] = beta * acc;
+    }
+    __syncthreads();
+    double pv = 0.0;
+    for (int i = tid; i < m; i += nt) pv += p[i] * v[i];
+    const double Kc = 0.5 * beta * block_sum(pv, red);
+    for (int i = tid; i < m; i += nt) p[i] -= Kc * v[i];
+    __syncthreads();
+    for (int i = warp; i < m; i += nwarp) {
+      double* row = A + (int64_t)(k + 1 + i) * n + (k + 1);
+      const double vi = v[i], wi = p[i];
+      for (int j = lane; j < m; j += 32) row[j] -= vi * p[j] + wi * v[j];
+    }
+    if (tid == 0) { dd[k] = A[(int64_t)k * n + k]; ee[k] = alpha; tau[k] = beta; }
+    for (int i = tid; i < m; i += nt) A[(int64_t)(k + 1 + i) * n + k] = v[i];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    if (n >= 2) {
+      dd[n - 2] = A[(int64_t)(n - 2) * n + (n - 2)];
+      ee[n - 2] = A[(int64_t)(n - 1) * n + (n - 2)];
+      tau[n - 2] = 0.0;
+    }
+    dd[n - 1] = A[(int64_t)(n - 1) * n + (n - 1)];
+    ee[n - 1] = 0.0;
+    tau[n - 1] = 0.0;
+  }
+}
+
+// Number of eigenvalues of the tridiagonal (d, e) smaller than x.
+__device__ __forceinline__ int sturm_count(const double* d, const double* e, int n, double x, double pivmin) {
+  int c = 0;
+  double q = d[0] - x;
+  if (fabs(q) < pivmin) q = -pivmin;
+  c += q < 0.0;
+  for (int i = 1; i < n; ++i) {
+    q = (d[i] - x) - e[i - 1] * e[i - 1] / q;
+    if (fabs(q) < pivmin) q = -pivmin;
+    c += q < 0.0;
+  }
+  return c;
+}
+
+// w[j] = j-th largest eigenvalue, one thread per j (the Sturm count is
+// monotone in x, so bisection converges to the eigenvalue of that rank).
+__global__ void __launch_bounds__(256) k_bisect(const EighJob* __restrict__ jobs) {
+  const EighJob J = jobs[blockIdx.y];
+  const int n = J.n;
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n <= 0) return;
+  extern __shared__ double sh[];
+  double* d = sh;
+  double* e = sh + n;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) { d[i] = J.work[i]; e[i] = J.work[n + i]; }
+  __syncthreads();
+  if (j >= n) return;
+  double lo = d[0], hi = d[0], emax = 0.0;
+  for (int i = 0; i < n; ++i) {
+    const double r = (i > 0 ? fabs(e[i - 1]) : 0.0) + (i + 1 < n ? fabs(e[i]) : 0.0);
+    lo = fmin(lo, d[i] - r);
+    hi = fmax(hi, d[i] + r);
+    emax = fmax(emax, fabs(e[i]));
+  }
+  const double nrm = fmax(fabs(lo), fabs(hi));
+  const double pivmin = fmax(1e-300, 2.2250738585072014e-308 * fmax(1.0, emax * emax));
+  lo -= 4.0 * 2.220446049250313e-16 * nrm + pivmin;
+  hi += 4.0 * 2.220446049250313e-16 * nrm + pivmin;
+  const int m = n - 1 - j;          // rank among the ascending eigenvalues
+  for (int it = 0; it < 128; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (mid <= lo || mid >= hi) break;
+    if (sturm_count(d, e, n, mid, pivmin) > m) hi = mid;
+    else lo = mid;
+  }
+  J.w[j] = 0.5 * (lo + hi);
+}
+
+// Eigenvectors of the leading nvec[job] eigenvalues: inverse iteration on the
+// tridiagonal matrix (T - lam I factored once by Gaussian elimination with
+// partial pivoting, three solves from a fixed start vector), then the
+// back-transformation by the reflectors and the sign convention (largest
+// |entry| positive, first on ties). One warp per vector; lane 0 runs the
+// O(n) factorization and solves. Scratch per vector: z = Z[j*n ..] and
+// 5n doubles of J.F for the factors.
+__global__ void __launch_bounds__(256) k_eigvecs(const EighJob* __restrict__ jobs, const int* __restrict__ nvec) {
+  const EighJob J = jobs[blockIdx.y];
+  const int n = J.n;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (n <= 0 || j >= min(nvec[blockIdx.y], n)) return;
+  const double* d = J.work;
+  const double* e = d + n;
+  const double* tau = e + n;
+  double* z = J.Z + (int64_t)j * n;
+  if (lane == 0) {
+    double* dg = J.F + (int64_t)j * 5 * n;   // diagonal of U
+    double* u1 = dg + n;                     // first superdiagonal of U
+    double* u2 = u1 + n;                     // second superdiagonal of U
+    double* ml = u2 + n;                     // multipliers
+    double* sw = ml + n;                     // 1.0 where rows i, i+1 were swapped
+    double nrm = 0.0;
+    for (int i = 0; i < n; ++i) nrm = fmax(nrm, fabs(d[i]) + fabs(e[i]) + (i ? fabs(e[i - 1]) : 0.0));
+    const double lam = J.w[j];
+    const double tiny = fmax(nrm, 1e-300) * 2.220446049250313e-16;
+    for (int i = 0; i < n; ++i) {
+      dg[i] = d[i] - lam;
+      u1[i] = (i + 1 < n) ? e[i] : 0.0;
+      u2[i] = 0.0;
+    }
+    for (int i = 0; i + 1 < n; ++i) {
+      const double sub = e[i];              // row i+1, column i
+      if (fabs(dg[i]) >= fabs(sub)) {
+        const double f = (dg[i] != 0.0) ? sub / dg[i] : 0.0;
+        ml[i] = f;
+        sw[i] = 0.0;
+        dg[i + 1] -= f * u1[i];
+      } else {
+        const double f = dg[i] / sub;
+        dg[i] = sub;
+        ml[i] = f;
+        sw[i] = 1.0;
+        const double t = u1[i];
+        u1[i] = dg[i + 1];
+        dg[i + 1] = t - f * dg[i + 1];
+        if (i + 2 < n) {
+          u2[i] = u1[i + 1];
+          u1[i + 1] = -f * u1[i + 1];
+        }
+      }
+    }
+    for (int i = 0; i < n; ++i)
+      if (fabs(dg[i]) < tiny) dg[i] = (dg[i] < 0.0) ? -tiny : tiny;
+    for (int i = 0; i < n; ++i) z[i] = 1.0 + 0.5 * sin(0.7 * (double)i + 0.3 * (double)j);
+    for (int iter = 0; iter < 3; ++iter) {
+      for (int i = 0; i + 1 < n; ++i) {
+        if (sw[i] != 0.0) { const double t = z[i]; z[i] = z[i + 1]; z[i + 1] = t; }
+        z[i + 1] -= ml[i] * z[i];
+      }
+      z[n - 1] /= dg[n - 1];
+      if (n >= 2) z[n - 2] = (z[n - 2] - u1[n - 2] * z[n - 1]) / dg[n - 2];
+      for (int i = n - 3; i >= 0; --i) z[i] = (z[i] - u1[i] * z[i + 1] - u2[i] * z[i + 2]) / dg[i];
+      double s = 0.0;
+      for (int i = 0; i < n; ++i) s += z[i] * z[i];
+      s = 1.0 / sqrt(s);
+      for (int i = 0; i < n; ++i) z[i] *= s;
+    }
+  }
+  __syncwarp();
+  // back-transformation z <- H_k z, k = n-3 .. 0; reflector k is column k of A
+  for (int k = n - 3; k >= 0; --k) {
+    const double beta = tau[k];
+    if (beta == 0.0) continue;
+    const int m = n - k - 1;
+    const double* vk = J.A + (int64_t)(k + 1) * n + k;
+    double acc = 0.0;
+    for (int i = lane; i < m; i += 32) acc += vk[(int64_t)i * n] * z[k + 1 + i];
+    acc = beta * warp_sum(acc);
+    for (int i = lane; i < m; i += 32) z[k + 1 + i] -= acc * vk[(int64_t)i * n];
+    __syncwarp();
+  }
+  double best = -1.0;
+  int bi = 0x7fffffff;
+  for (int i = lane; i < n; i += 32) {
+    const double a = fabs(z[i]);
+    if (a > best) { best = a; bi = i; }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+  }
+  const double sg = (z[bi] < 0.0) ? -1.0 : 1.0;
+  double* dst = J.Vt + (int64_t)j * n;
+  for (int i = lane; i < n; i += 32) dst[i] = sg * z[i];
+}
+
+jolt_status launch_tridiag(const EighJob* jobs, int njobs, int nmax, cudaStream_t s) {
+  const size_t smem = (size_t)(2 * nmax + 32) * sizeof(double);
+  { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_tridiag, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
+  k_tridiag<<<njobs, EIG_THREADS, smem, s>>>(jobs);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+jolt_status launch_bisect(const EighJob* jobs, int njobs, int nmax, cudaStream_t s) {
+  const size_t smem = (size_t)(2 * nmax) * sizeof(double);
+  { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_bisect, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
+  dim3 g((nmax + 255) / 256, njobs);
+  k_bisect<<<g, 256, smem, s>>>(jobs);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+jolt_status launch_eigvecs(const EighJob* jobs, int njobs, int nvec_max, const int* nvec, cudaStream_t s) {
+  if (nvec_max <= 0) return JOLT_OK;
+  dim3 g((nvec_max + 7) / 8, njobs);
+  k_eigvecs<<<g, 256, 0, s>>>(jobs, nvec);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
 jolt_status launch_eigh(const EighJob* jobs_dev, int njobs, int nmax, int* status, cudaStream_t s) {
   size_t smem = eigh_smem_bytes(nmax);
-  JOLT_CUDA_TRY(cudaFuncSetAttribute(k_eigh, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_eigh, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
   k_eigh<<<njobs, EIG_THREADS, smem, s>>>(jobs_dev, status);
   JOLT_LAUNCHED();
   return JOLT_OK;

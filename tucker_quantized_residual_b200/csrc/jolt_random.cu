@@ -353,6 +353,89 @@ jolt_status launch_trsm_rows(const float* Z, int64_t z_cell, const double* R, in
   return JOLT_OK;
 }
 
+// R^{-1} of the upper triangular R (fp64), one column per thread by back
+// substitution, stored as fp32 [k][k] for the product below.
+__global__ void k_tri_inv(const double* __restrict__ R, int64_t r_cell, int k, float* __restrict__ Ri,
+                          double* __restrict__ X, int64_t x_cell) {
+  const int cell = blockIdx.y, c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= k) return;
+  const double* r = R + (int64_t)cell * r_cell;
+  double* x = X + (int64_t)cell * x_cell;
+  float* ri = Ri + (int64_t)cell * k * k;
+  for (int i = k - 1; i >= 0; --i) {
+    double acc = (i == c) ? 1.0 : 0.0;
+    if (i <= c) {
+      for (int l = i + 1; l <= c; ++l) acc -= r[(int64_t)i * k + l] * x[(int64_t)l * k + c];
+      acc /= r[(int64_t)i * k + i];
+    } else {
+      acc = 0.0;
+    }
+    x[(int64_t)i * k + c] = acc;
+    ri[(int64_t)i * k + c] = (float)acc;
+  }
+}
+
+// W^T[cell][j][n] = bf16( sum_i Z[cell][n][i] Ri[cell][i][j] ), fp32 tiles of
+// 64 (n) x 64 (j), 4 x 4 outputs per thread.
+__global__ void __launch_bounds__(256) k_z_rinv(const float* __restrict__ Z, int64_t z_cell, const float* __restrict__ Ri,
+                                                int k, const int* __restrict__ Nc, uint16_t* __restrict__ Wt,
+                                                int64_t w_cell, int ldw) {
+  constexpr int TB = 64, KB = 16;
+  __shared__ float As[KB][TB + 4];
+  __shared__ float Bs[KB][TB + 4];
+  const int cell = blockIdx.z;
+  const int n0 = blockIdx.x * TB, j0 = blockIdx.y * TB;
+  const int nc = Nc[cell];
+  if (n0 >= nc || j0 >= k) return;
+  const float* z = Z + (int64_t)cell * z_cell;
+  const float* ri = Ri + (int64_t)cell * k * k;
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  float acc[4][4] = {};
+  const int iend = min(k, j0 + TB);          // Ri is upper triangular: i <= j
+  for (int i0 = 0; i0 < iend; i0 += KB) {
+    for (int e = threadIdx.x; e < KB * TB; e += blockDim.x) {
+      const int kk = e % KB, nn = e / KB;
+      const int n = n0 + nn, i = i0 + kk;
+      As[kk][nn] = (n < nc && i < k) ? z[(int64_t)n * k + i] : 0.0f;
+      const int jj = e % TB, k2 = e / TB;
+      const int j = j0 + jj, i2 = i0 + k2;
+      Bs[k2][jj] = (j < k && i2 < k) ? ri[(int64_t)i2 * k + j] : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < KB; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) { a[q] = As[kk][ty * 4 + q]; b[q] = Bs[kk][tx * 4 + q]; }
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(a[p], b[q], acc[p][q]);
+    }
+    __syncthreads();
+  }
+  uint16_t* w = Wt + (int64_t)cell * w_cell;
+#pragma unroll
+  for (int p = 0; p < 4; ++p)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int n = n0 + ty * 4 + p, j = j0 + tx * 4 + q;
+      if (n < nc && j < k) w[(int64_t)j * ldw + n] = bf16_bits_from_f32(acc[p][q]);
+    }
+}
+
+jolt_status launch_orth_apply(const double* R, int64_t r_cell, int k, float* Ri, double* X, int64_t x_cell,
+                              const float* Z, int64_t z_cell, const int* Nc, int Ncmax, uint16_t* Wt, int64_t w_cell,
+                              int ldw, int ncells, cudaStream_t s) {
+  dim3 g1((k + 127) / 128, ncells);
+  k_tri_inv<<<g1, 128, 0, s>>>(R, r_cell, k, Ri, X, x_cell);
+  JOLT_LAUNCHED();
+  dim3 g2((Ncmax + 63) / 64, (k + 63) / 64, ncells);
+  k_z_rinv<<<g2, 256, 0, s>>>(Z, z_cell, Ri, k, Nc, Wt, w_cell, ldw);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
 // X1 = R^{-T} P (column c per thread, forward substitution), then
 // M = X1 R^{-1} (row per thread), symmetrized into M.
 __global__ void k_solve_left_t(const double* __restrict__ R, const double* __restrict__ P, double* __restrict__ X1,
@@ -394,6 +477,13 @@ __global__ void k_symmetrize(double* __restrict__ M, int64_t cs, int k) {
       m[(int64_t)j * k + i] = a;
     }
   }
+}
+
+jolt_status launch_symmetrize(double* M, int64_t cs, int k, int ncells, cudaStream_t s) {
+  dim3 g2(64, ncells);
+  k_symmetrize<<<g2, 256, 0, s>>>(M, cs, k);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
 }
 
 jolt_status launch_bbt(const double* R, const double* P, double* X1, double* M, int64_t cs, int k, int ncells,
