@@ -186,7 +186,7 @@ struct jolt_plan_s {
   double* Gz = nullptr;    double* Rm = nullptr;    double* P0 = nullptr;   double* X1 = nullptr;
   double* MB = nullptr;    double* eZ = nullptr;    double* eVt = nullptr;  double* ew = nullptr;
   double* ework = nullptr; double* trs = nullptr;   double* P64 = nullptr;
-  double* eF = nullptr;    float* Ri32 = nullptr;   double* RTk = nullptr;
+  double* eF = nullptr;    double* Rinv = nullptr;  double* RTk = nullptr;
   std::vector<double*> h_FT;     // exact mode: inverse-iteration scratch per cell
   int* d_cl0 = nullptr; int* d_cb = nullptr; int* d_cLg = nullptr; int* d_ckind = nullptr;
   int* d_Nc = nullptr; int* d_cis = nullptr;
@@ -516,7 +516,7 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
       p->eVt = A.take<double>(nc * kk); p->ew = A.take<double>((size_t)nc * k);
       p->ework = A.take<double>((size_t)nc * 3 * k);
       p->eF = A.take<double>((size_t)nc * p->rmax_all * 5 * k);
-      p->Ri32 = A.take<float>((size_t)nc * kk);
+      p->Rinv = A.take<double>((size_t)nc * kk);
       p->RTk = A.take<double>((size_t)nc * kk);
       p->trs = nullptr;
       p->P64 = A.take<double>((size_t)nc * k * p->rmax_all);
@@ -758,12 +758,13 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
     ProfScope ps(JOLT_STAGE_ORTH, s);
     JOLT_TRY(launch_gram_cols(p->Z, (int64_t)p->Ncmax * k, p->d_Nc, k, p->Gz, kk, nc, s));
     JOLT_TRY(launch_chol_blocked(p->Gz, p->RTk, kk, nullptr, k, nc, status, s));
+    JOLT_TRY(launch_tri_inverse(p->Gz, p->Rinv, p->RTk, kk, k, nc, s));
     TrsmArgs ta{};
-    ta.R = p->Gz; ta.RT = p->RTk; ta.r_cell = kk; ta.k = k; ta.backward = 0;
+    ta.Rinv = p->Rinv; ta.RinvT = p->RTk; ta.r_cell = kk; ta.k = k; ta.backward = 0;
     ta.B = p->Z; ta.b64 = 0; ta.b_cell = (int64_t)p->Ncmax * k; ta.ldb_r = k; ta.ldb_c = 1;
     ta.rows_of = p->d_Nc;
     ta.X16 = p->Wt; ta.x16_cell = (int64_t)k * p->Ncmax; ta.ld16_r = 1; ta.ld16_c = p->Ncmax;
-    JOLT_TRY(launch_trsm_rows2(ta, p->Ncmax, nc, s));
+    JOLT_TRY(launch_tri_apply(ta, p->Ncmax, nc, s));
     JOLT_TRY(xw());
   }
   JOLT_TRY(xty());
@@ -780,17 +781,18 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
   }
   ProfScope ps_eig(JOLT_STAGE_EIG, s);
   JOLT_TRY(launch_chol_blocked(p->Rm, p->RTk, kk, p->GW32, k, nc, status, s));
+  JOLT_TRY(launch_tri_inverse(p->Rm, p->Rinv, p->RTk, kk, k, nc, s));
   // B B^T = R^{-T} (Z^T Z) R^{-1}: Y1 = P0 R^{-1}, then (Y1^T) R^{-1}
   JOLT_TRY(launch_gram_cols(p->Z, (int64_t)p->Ncmax * k, p->d_Nc, k, p->P0, kk, nc, s));
   {
     TrsmArgs ta{};
-    ta.R = p->Rm; ta.RT = p->RTk; ta.r_cell = kk; ta.k = k; ta.backward = 0;
+    ta.Rinv = p->Rinv; ta.RinvT = p->RTk; ta.r_cell = kk; ta.k = k; ta.backward = 0;
     ta.B = p->P0; ta.b64 = 1; ta.b_cell = kk; ta.ldb_r = k; ta.ldb_c = 1; ta.rows_fixed = k;
     ta.X64 = p->X1; ta.x64_cell = kk; ta.ld64_r = k; ta.ld64_c = 1;
-    JOLT_TRY(launch_trsm_rows2(ta, k, nc, s));
+    JOLT_TRY(launch_tri_apply(ta, k, nc, s));
     ta.B = p->X1; ta.ldb_r = 1; ta.ldb_c = k;
     ta.X64 = p->MB;
-    JOLT_TRY(launch_trsm_rows2(ta, k, nc, s));
+    JOLT_TRY(launch_tri_apply(ta, k, nc, s));
     JOLT_TRY(launch_symmetrize(p->MB, kk, k, nc, s));
   }
   // spectra only here: eigenvectors follow the allocation (top r_T only)
@@ -815,12 +817,12 @@ static jolt_status run_random_fit(jolt_plan_s* p, const void* k_in, const void* 
   {
     // P = R^{-1} U_B[:, :r_T]: rows of P^T solve x R^T = u (backward)
     TrsmArgs ta{};
-    ta.R = p->Rm; ta.RT = p->RTk; ta.r_cell = kk; ta.k = k; ta.backward = 1;
+    ta.Rinv = p->Rinv; ta.RinvT = p->RTk; ta.r_cell = kk; ta.k = k; ta.backward = 1;
     ta.B = p->eVt; ta.b64 = 1; ta.b_cell = kk; ta.ldb_r = k; ta.ldb_c = 1;
     ta.rows_of = p->d_rT_used;
     ta.X64 = p->P64; ta.x64_cell = (int64_t)k * p->rmax_all; ta.ld64_r = 1; ta.ld64_c = p->rmax_all;
     ta.X16 = p->Pt; ta.x16_cell = (int64_t)p->rpad * p->kpad; ta.ld16_r = p->kpad; ta.ld16_c = 1;
-    JOLT_TRY(launch_trsm_rows2(ta, p->rmax_all, nc, s));
+    JOLT_TRY(launch_tri_apply(ta, p->rmax_all, nc, s));
   }
   umma::Maps m{};
   JOLT_TRY(x_maps(p, k_in, v_in, m));

@@ -221,8 +221,8 @@ jolt_status map_3d_box(CUtensorMap* m, const void* base, int cells, int rows, in
 namespace jolt {
 // ------------------------------------------ batched dense fp64 (k x k) -----
 struct TrsmArgs {
-  const double* R;      // upper R (k x k, row-major), read by the backward solve
-  const double* RT;     // R^T (k x k, row-major), read by the forward solve
+  const double* Rinv;   // R^{-1} (k x k, row-major, upper), read by the forward product
+  const double* RinvT;  // R^{-T} (k x k, row-major, lower), read by the backward product
   int64_t r_cell;
   int k;
   int backward;         // 0: X R = B, 1: X R^T = B
@@ -238,6 +238,8 @@ struct TrsmArgs {
 };
 jolt_status launch_chol_blocked(double* G, double* RT, int64_t cs, const float* src32, int k, int ncells, int* status,
                                 cudaStream_t s);
-jolt_status launch_trsm_rows2(const TrsmArgs& a, int rows_max, int ncells, cudaStream_t s);
+jolt_status launch_tri_inverse(const double* R, double* Ri, double* RiT, int64_t cs, int k, int ncells,
+                               cudaStream_t s);
+jolt_status launch_tri_apply(const TrsmArgs& a, int rows_max, int ncells, cudaStream_t s);
 jolt_status launch_symmetrize(double* M, int64_t cs, int k, int ncells, cudaStream_t s);
 }  // namespace jolt
