@@ -765,6 +765,7 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
     ta.rows_of = p->d_Nc;
     ta.X16 = p->Wt; ta.x16_cell = (int64_t)k * p->Ncmax; ta.ld16_r = 1; ta.ld16_c = p->Ncmax;
     JOLT_TRY(launch_tri_apply(ta, p->Ncmax, nc, s));
+    ps.end();
     JOLT_TRY(xw());
   }
   JOLT_TRY(xty());

@@ -6,13 +6,20 @@
 //
 // One persistent CTA per SM walks tiles (cell, 128 tokens, layer-head) with
 // the layer-head index fastest, so consecutive tiles share U_T^ rows and the
-// RoPE table rows in L2. Warp 0 loads U_T^ / M^ slices (and, when
-// compressing, the 128 x D input tile) with TMA; warp 1 issues tcgen05.mma
-// (backbone tile 128 x D in TMEM, K = r_T rounded up to 64, fp32 accumulate);
-// warps 2..5 each own 32 rows: they read the backbone row from TMEM, the input
-// row from the 128-byte-swizzled tile, and run the rotation and the quantizer
-// in registers. Packed codes, scales and decoded rows go through padded
-// shared staging so that global loads and stores are coalesced.
+// RoPE table rows in L2. Warp 0 loads U_T^ / M^ slices and, when compressing,
+// the 128 x D input tile with TMA, or, when decoding, the tile's packed codes
+// and scales with bulk copies; warp 1 issues tcgen05.mma (backbone tile
+// 128 x D in TMEM, K = r_T rounded up to 64, fp32 accumulate).
+//
+// Warps 2..9 form the epilogue: two threads per row, from two warps on the
+// same TMEM lane quarter. Thread half h of a row owns the columns
+// [hC, hC + C) and [D/2 + hC, D/2 + hC + C), C = D/4, so each RoPE pair
+// (i, i + D/2) stays in one thread. The Walsh-Hadamard stages of span < C and
+// the stage of span D/2 run in registers; the stage of span C pairs the two
+// halves and goes through a swizzled shared-memory exchange. Every stage
+// performs the same fp32 additions as the one-row transform, so the result
+// is identical to it. Codes, scales and decoded rows are stored straight
+// from registers.
 #define JOLT_PTX_HELPERS
 #include "jolt_internal.cuh"
 #include "jolt_kernels.cuh"
@@ -28,11 +35,13 @@ constexpr int SSTAGES = 3;
 constexpr int S_A = 128 * 64 * 2;          // U_T^ slice: 128 tokens x 64 ranks
 constexpr int S_B = 128 * 64 * 2;          // M^T slice: D rows x 64 ranks (D <= 128)
 constexpr int S_X = 128 * 128 * 2;         // input tile: 128 tokens x D
-constexpr int ROWPITCH_OUT = 128 * 2 + 16; // decoded bf16 row + pad
-constexpr int CODE_PITCH_MAX = 128 + 8;    // packed row (<= 8 bits x 128 / 8) + pad
-constexpr int SMEM_STREAM = SSTAGES * (S_A + S_B) + 2 * S_X + 128 * ROWPITCH_OUT + 128 * CODE_PITCH_MAX +
-                            128 * 4 * 4 + 1024 + 512;
-constexpr int STHREADS = 192;
+constexpr int S_CODE = 128 * 128;          // packed codes of a tile (<= 8 bits x 128 per row)
+constexpr int S_SCALE = 128 * 4 * 4;       // scales of a tile (<= 4 groups per row)
+constexpr int S_XCH = 128 * 256;           // pair exchange: 128 rows x 2 halves x 128 bytes
+constexpr int S_R1 = (2 * S_X > 2 * (S_CODE + S_SCALE)) ? 2 * S_X : 2 * (S_CODE + S_SCALE);
+constexpr int SMEM_STREAM = SSTAGES * (S_A + S_B) + S_R1 + S_XCH + 128 * 16 + 128 * 4 + 1024 + 512;
+constexpr int EPI_WARPS = 8;
+constexpr int STHREADS = 64 + 32 * EPI_WARPS;
 
 struct Args {
   int ncells, T, H, lhmax, rpad_m, G, ntile_t;
@@ -53,7 +62,12 @@ struct SMaps {
   CUtensorMap xv;
 };
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float* v);
+template <>
+__device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, float* v) { tmem_ld16(taddr, v); }
+template <>
+__device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, float* v) {
   uint32_t r[32];
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
@@ -68,18 +82,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-// AND of `ok` over the 128 epilogue threads: every one of them takes the same
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * EPI_WARPS) : "memory"); }
+// Barrier of the two warps that share a TMEM lane quarter (64 threads).
+__device__ __forceinline__ void pair_sync(int q) { asm volatile("bar.sync %0, 64;" ::"r"(2 + q) : "memory"); }
+// AND of `ok` over the epilogue threads: every one of them takes the same
 // branch after a bounded wait, so none is left at a named barrier alone.
 __device__ __forceinline__ bool epi_all(bool ok) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)ok)
+      : "r"((uint32_t)ok), "n"(32 * EPI_WARPS)
       : "memory");
   return r != 0;
 }
@@ -98,34 +120,223 @@ __device__ __forceinline__ bool tile_of(const Args& a, int tile, int& cell, int&
   return o.rT > 0;
 }
 
-template <int D>
-struct RowPack {
-  float* e;
-  uint8_t* dst;
-  float* sc;
-  template <int G, int B>
-  __device__ __forceinline__ void run() { quantize_pack_row<D, G, B>(e, dst, sc); }
+// Byte extents of a decoded tile's codes and scales, and whether each can be
+// fetched by one bulk copy (16-byte aligned start and length).
+struct CodeTile {
+  const uint8_t* codes;
+  const float* scales;
+  uint32_t cbytes, sbytes;
+  bool cbulk, sbulk;
 };
+__device__ __forceinline__ CodeTile code_tile(const CellOut& o, int64_t row0, int nrows, int D, int G) {
+  CodeTile ct;
+  const int rowbytes = o.b * D / 8, ng = D / G;
+  ct.codes = o.codes + row0 * rowbytes;
+  ct.scales = o.scales + row0 * ng;
+  ct.cbytes = (uint32_t)(nrows * rowbytes);
+  ct.sbytes = (uint32_t)(nrows * ng * 4);
+  ct.cbulk = ((reinterpret_cast<uintptr_t>(ct.codes) | ct.cbytes) & 15u) == 0;
+  ct.sbulk = ((reinterpret_cast<uintptr_t>(ct.scales) | ct.sbytes) & 15u) == 0;
+  return ct;
+}
+
+// 8 bf16 of row r starting at column col (multiple of 8) of the
+// 128-byte-swizzled input tile (64-column boxes of 128 rows).
+__device__ __forceinline__ void ld_x8(const uint8_t* xs, int r, int col, float* o) {
+  const int box = col >> 6, ch = (col & 63) >> 3;
+  const uint4 w = *reinterpret_cast<const uint4*>(xs + box * 16384 + r * 128 + ((ch ^ (r & 7)) << 4));
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    o[2 * j] = __uint_as_float(u[j] << 16);
+    o[2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+  }
+}
+
+// Walsh-Hadamard stages of span 1 .. C/2 on one chunk of C values.
+template <int C>
+__device__ __forceinline__ void fwht_chunk(float* v) {
+#pragma unroll
+  for (int h = 1; h < C; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < C; i += 2 * h) {
+#pragma unroll
+      for (int j = i; j < i + h; ++j) {
+        const float a = v[j], b = v[j + h];
+        v[j] = __fadd_rn(a, b);
+        v[j + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+}
+
+// Exchange slot of (row r, half hf), 16-byte unit u < 8, swizzled by row.
+__device__ __forceinline__ float4* xch_at(uint8_t* xch, int r, int hf, int u) {
+  return reinterpret_cast<float4*>(xch + r * 256 + hf * 128 + ((u ^ (r & 7)) << 4));
+}
+
+// Full transform of the thread's 2C values: in-chunk stages, the span-C stage
+// with the partner half, then the span-D/2 stage between the two chunks.
+template <int C>
+__device__ __forceinline__ void fwht_pair(float* e, uint8_t* xch, int r, int hf, int q) {
+  fwht_chunk<C>(e);
+  fwht_chunk<C>(e + C);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    float* v = e + k * C;
+#pragma unroll
+    for (int u = 0; u < C / 4; ++u) *xch_at(xch, r, hf, u) = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+    pair_sync(q);
+#pragma unroll
+    for (int u = 0; u < C / 4; ++u) {
+      const float4 p = *xch_at(xch, r, hf ^ 1, u);
+      const float pv[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        // half 0 holds the lower index of each pair (a + b), half 1 the upper (a - b)
+        const float mine = v[4 * u + j];
+        v[4 * u + j] = hf == 0 ? __fadd_rn(mine, pv[j]) : __fsub_rn(pv[j], mine);
+      }
+    }
+    pair_sync(q);
+  }
+#pragma unroll
+  for (int j = 0; j < C; ++j) {
+    const float a = e[j], b = e[j + C];
+    e[j] = __fadd_rn(a, b);
+    e[j + C] = __fsub_rn(a, b);
+  }
+}
+
+// b-bit codes of one chunk of C values with one scale: code =
+// clamp(rint(fl32(r / sc))). The quotient is taken as r * fl32(1/sc) and
+// replaced by the correctly rounded one wherever the product lies within
+// 1e-4 of a rounding boundary (it differs from the quotient by at most
+// 128 * 2^-23 < 2e-5 there), so the codes equal the divided ones.
+template <int C, int B>
+__device__ __forceinline__ void quant_chunk(const float* r, float sc, uint32_t* w) {
+  constexpr int NW = (C * B + 31) / 32;
+  const float qm = (float)((1 << (B - 1)) - 1);
+#pragma unroll
+  for (int i = 0; i < NW; ++i) w[i] = 0u;
+  uint32_t need = 0u;
+  if (sc > 0.0f) {
+    const float inv = __frcp_rn(sc);
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      const float y = __fmul_rn(r[i], inv);
+      float qf = rintf(y);
+      if (!(0.5f - fabsf(y - qf) >= 1e-4f)) need |= 1u << i;
+      qf = fminf(fmaxf(qf, -qm), qm);
+      const uint32_t u = (uint32_t)((int)qf + (1 << (B - 1)));
+      const int bit = i * B, wi = bit >> 5, sh = bit & 31;
+      w[wi] |= u << sh;
+      if (sh + B > 32) w[wi + 1] |= u >> (32 - sh);
+    }
+    if (need) {
+      constexpr uint32_t mask = (1u << B) - 1u;
+#pragma unroll
+      for (int i = 0; i < C; ++i) {
+        if (!((need >> i) & 1u)) continue;
+        const float qf = fminf(fmaxf(rintf(__fdiv_rn(r[i], sc)), -qm), qm);
+        const uint32_t u = (uint32_t)((int)qf + (1 << (B - 1)));
+        const int bit = i * B, wi = bit >> 5, sh = bit & 31;
+        w[wi] = (w[wi] & ~(mask << sh)) | (u << sh);
+        if (sh + B > 32) w[wi + 1] = (w[wi + 1] & ~(mask >> (32 - sh))) | (u >> (32 - sh));
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      const uint32_t u = 1u << (B - 1);
+      const int bit = i * B, wi = bit >> 5, sh = bit & 31;
+      w[wi] |= u << sh;
+      if (sh + B > 32) w[wi + 1] |= u >> (32 - sh);
+    }
+  }
+}
+
+template <int C, int B>
+__device__ __forceinline__ void dequant_chunk(const uint32_t* w, float sc, float* v) {
+  constexpr uint32_t mask = (1u << B) - 1u;
+#pragma unroll
+  for (int i = 0; i < C; ++i) {
+    const int bit = i * B, wi = bit >> 5, sh = bit & 31;
+    uint32_t u = w[wi] >> sh;
+    if (sh + B > 32) u |= w[wi + 1] << (32 - sh);
+    const int q = (int)(u & mask) - (1 << (B - 1));
+    v[i] = __fmul_rn((float)q, sc);
+  }
+}
+
+// Chunk bits (C * B of them, a multiple of 16) to / from memory: 32-bit
+// units when C = 32 (4-byte aligned offsets), 16-bit units otherwise.
+template <int C, int B>
+__device__ __forceinline__ void store_bits(uint8_t* p, const uint32_t* w) {
+  if constexpr (C == 32) {
+    uint32_t* d = reinterpret_cast<uint32_t*>(p);
+#pragma unroll
+    for (int i = 0; i < B; ++i) d[i] = w[i];
+  } else {
+    uint16_t* d = reinterpret_cast<uint16_t*>(p);
+#pragma unroll
+    for (int i = 0; i < C * B / 16; ++i) d[i] = (uint16_t)(w[i >> 1] >> (16 * (i & 1)));
+  }
+}
+template <int C, int B>
+__device__ __forceinline__ void load_bits(const uint8_t* p, uint32_t* w) {
+  if constexpr (C == 32) {
+    const uint32_t* s = reinterpret_cast<const uint32_t*>(p);
+#pragma unroll
+    for (int i = 0; i < B; ++i) w[i] = s[i];
+  } else {
+    const uint16_t* s = reinterpret_cast<const uint16_t*>(p);
+#pragma unroll
+    for (int i = 0; i < (C * B + 31) / 32; ++i) w[i] = 0u;
+#pragma unroll
+    for (int i = 0; i < C * B / 16; ++i) w[i >> 1] |= (uint32_t)s[i] << (16 * (i & 1));
+  }
+}
+
+// Chunk maxima of both halves -> scale of each of this thread's chunks;
+// the thread whose chunk opens a group stores the group's scale.
 template <int D>
-struct RowUnpack {
-  float* v;
-  const uint8_t* src;
-  const float* sc;
-  template <int G, int B>
-  __device__ __forceinline__ void run() { unpack_dequant_row<D, G, B>(src, sc, v); }
-};
+__device__ __forceinline__ void chunk_scales(const float* am, float* pm, int r, int hf, int q, int G, float qm,
+                                             float* sc, float* srow) {
+  constexpr int C = D / 4;
+  pm[(r * 2 + hf) * 2 + 0] = am[0];
+  pm[(r * 2 + hf) * 2 + 1] = am[1];
+  pair_sync(q);
+  float part[2];
+  part[0] = pm[(r * 2 + (hf ^ 1)) * 2 + 0];
+  part[1] = pm[(r * 2 + (hf ^ 1)) * 2 + 1];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int s0 = k * (D / 2) + hf * C, g = s0 / G;
+    float a = 0.0f;
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int s1 = kk * (D / 2) + hh * C;
+        if (s1 / G == g) a = fmaxf(a, hh == hf ? am[kk] : part[kk]);
+      }
+    sc[k] = __fdiv_rn(a, qm);
+    if (s0 % G == 0) srow[g] = sc[k];
+  }
+}
 
 template <int D, bool COMPRESS>
 __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ SMaps maps, Args a) {
+  constexpr int C = D / 4;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem;                                   // SSTAGES x S_A
   uint8_t* sB = sA + SSTAGES * S_A;                     // SSTAGES x S_B
-  uint8_t* sX = sB + SSTAGES * S_B;                     // 2 x S_X
-  uint8_t* sOut = sX + 2 * S_X;                         // 128 x ROWPITCH_OUT
-  uint8_t* sCode = sOut + 128 * ROWPITCH_OUT;           // 128 x CODE_PITCH_MAX
-  float* sScale = reinterpret_cast<float*>(sCode + 128 * CODE_PITCH_MAX);   // 128 x 4
-  float* sSign = sScale + 128 * 4;                      // D
+  uint8_t* sR1 = sB + SSTAGES * S_B;                    // 2 x S_X (compress) | 2 x (codes + scales)
+  uint8_t* sXch = sR1 + S_R1;                           // S_XCH
+  float* sPm = reinterpret_cast<float*>(sXch + S_XCH);  // 128 rows x 2 halves x 2 chunk maxima
+  float* sSign = sPm + 128 * 4;                         // D (<= 128)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sSign + 128);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * SSTAGES + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -137,17 +348,19 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
   auto empty_bar = [&](int s) { return bar0 + 8u * (SSTAGES + s); };
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * SSTAGES + b); };
   auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * SSTAGES + 2 + b); };
+  // second input buffer: the X tile (compress) or the codes + scales (decode)
   auto xfull_bar = [&](int b) { return bar0 + 8u * (2 * SSTAGES + 4 + b); };
   auto xempty_bar = [&](int b) { return bar0 + 8u * (2 * SSTAGES + 6 + b); };
+  auto in_buf = [&](int b) { return sR1 + b * (COMPRESS ? S_X : S_CODE + S_SCALE); };
   constexpr int NCOLS = (2 * D <= 128) ? 128 : 256;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SSTAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 4);
+      mbar_init(tempty_bar(b), EPI_WARPS);
       mbar_init(xfull_bar(b), 1);
-      mbar_init(xempty_bar(b), 4);
+      mbar_init(xempty_bar(b), EPI_WARPS);
     }
     *abort_flag = 0;
     *sign_seq = -1;
@@ -193,19 +406,25 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
           if (++stage == SSTAGES) { stage = 0; ph ^= 1; }
         }
         if (!ok) break;
+        if (!COMPRESS && o.b == 0) continue;
+        if (!mbar_wait(xempty_bar(xb), xph[xb] ^ 1, abort_flag, a.status)) break;
+        const uint32_t sx = smem_u32(in_buf(xb));
         if (COMPRESS) {
-          if (!mbar_wait(xempty_bar(xb), xph[xb] ^ 1, abort_flag, a.status)) break;
-          const uint32_t sx = smem_u32(sX + xb * S_X);
           mbar_expect_tx(xfull_bar(xb), D * 128 * 2);
           const CUtensorMap* xm = (c.kind == 0) ? &maps.xk : &maps.xv;
           const int l = c.l0 + lh / c.H, h = lh % c.H;
           for (int hh = 0; hh < D / 64; ++hh)
             tma_load_5d(sx + hh * 16384, xm, xfull_bar(xb), hh * 64, t0, h, l, c.seq);
-          xissued[xb] = true;
-          xissued_phase[xb] = xph[xb];
-          xph[xb] ^= 1;
-          xb ^= 1;
+        } else {
+          const CodeTile ct = code_tile(o, (int64_t)lh * c.T + t0, min(SBM, c.T - t0), D, a.G);
+          mbar_expect_tx(xfull_bar(xb), (ct.cbulk ? ct.cbytes : 0u) + (ct.sbulk ? ct.sbytes : 0u));
+          if (ct.cbulk) bulk_load(sx, ct.codes, ct.cbytes, xfull_bar(xb));
+          if (ct.sbulk) bulk_load(sx + S_CODE, ct.scales, ct.sbytes, xfull_bar(xb));
         }
+        xissued[xb] = true;
+        xissued_phase[xb] = xph[xb];
+        xph[xb] ^= 1;
+        xb ^= 1;
       }
       for (int s = 0; s < SSTAGES; ++s)
         if (issued[s]) {
@@ -252,9 +471,11 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
     }
   } else {
     // --------------------------------------------------------- epilogue rows
-    const int q = warp & 3;
-    const int rl = q * 32 + lane;            // row within the tile (TMEM lane)
-    const int et = threadIdx.x - 64;         // 0..127 among the epilogue threads
+    const int q = warp & 3;                   // TMEM lane quarter
+    const int hf = (warp - 2) >> 2;           // column half of the row
+    const int rl = q * 32 + lane;             // row within the tile (TMEM lane)
+    const int et = threadIdx.x - 64;          // 0..255 among the epilogue threads
+    const float rs = (float)(1.0 / sqrt((double)D));
     int acc = 0, xb = 0;
     uint32_t aph[2] = {0, 0}, xph[2] = {0, 0};
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -276,137 +497,182 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
       const int l = lh / c.H, h = lh % c.H;
       const int b = o.b;
       const int rowbytes = b * D / 8;
-      const int cpitch = rowbytes + 8;
       const int ng = D / a.G;
-      if (!epi_all(mbar_wait(tfull_bar(acc), aph[acc], abort_flag, a.status))) break;
-      fence_after();
-      float v[D];
-      const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * D);
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) tmem_ld32(tb + c0, v + c0);
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar(acc));
-      aph[acc] ^= 1;
-      acc ^= 1;
       const int64_t row0 = (int64_t)lh * c.T + t0;   // first residual row of the tile
+      const int64_t row = row0 + rl;
+      float e[2 * C];
       if (COMPRESS) {
+        // backbone
+        if (!epi_all(mbar_wait(tfull_bar(acc), aph[acc], abort_flag, a.status))) break;
+        fence_after();
+        const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * D);
+        tmem_ld<C>(tb + hf * C, e);
+        tmem_ld<C>(tb + D / 2 + hf * C, e + C);
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(acc));
+        aph[acc] ^= 1;
+        acc ^= 1;
+        // E = [un-RoPE](X) - backbone
         if (!epi_all(mbar_wait(xfull_bar(xb), xph[xb], abort_flag, a.status))) break;
-        float x[D];
-        const uint8_t* xs = sX + xb * S_X;
+        const uint8_t* xs = in_buf(xb);
+        const float4* cs4 = reinterpret_cast<const float4*>(a.cs + (int64_t)(valid ? t : 0) * (D / 2) + hf * C);
 #pragma unroll
-        for (int hh = 0; hh < D / 64; ++hh)
+        for (int u = 0; u < C / 8; ++u) {
+          float x0[8], x1[8];
+          ld_x8(xs, rl, hf * C + 8 * u, x0);
+          ld_x8(xs, rl, D / 2 + hf * C + 8 * u, x1);
+          if (c.rope) {
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const uint4 w = *reinterpret_cast<const uint4*>(xs + hh * 16384 + rl * 128 + ((ch ^ (rl & 7)) << 4));
-            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+            for (int p = 0; p < 4; ++p) {
+              const float4 q2 = cs4[4 * u + p];
+              const float cc[2] = {q2.x, q2.z}, ss[2] = {q2.y, q2.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              x[hh * 64 + ch * 8 + 2 * j] = __uint_as_float(u[j] << 16);
-              x[hh * 64 + ch * 8 + 2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+              for (int j = 0; j < 2; ++j) {
+                const float yi = x0[2 * p + j], yj = x1[2 * p + j];
+                x0[2 * p + j] = __fadd_rn(__fmul_rn(yi, cc[j]), __fmul_rn(yj, ss[j]));
+                x1[2 * p + j] = __fsub_rn(__fmul_rn(yj, cc[j]), __fmul_rn(yi, ss[j]));
+              }
             }
           }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            e[8 * u + j] = __fsub_rn(x0[j], e[8 * u + j]);
+            e[C + 8 * u + j] = __fsub_rn(x1[j], e[C + 8 * u + j]);
+          }
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(xempty_bar(xb));
         xph[xb] ^= 1;
         xb ^= 1;
-        if (c.rope && valid) {
-          const float4* cs4 = reinterpret_cast<const float4*>(a.cs + (int64_t)t * (D / 2));
-#pragma unroll
-          for (int i = 0; i < D / 2; i += 2) {
-            const float4 q2 = cs4[i / 2];
-            const float cc[2] = {q2.x, q2.z}, ss[2] = {q2.y, q2.w};
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const float yi = x[i + j], yj = x[i + j + D / 2];
-              x[i + j] = __fadd_rn(__fmul_rn(yi, cc[j]), __fmul_rn(yj, ss[j]));
-              x[i + j + D / 2] = __fsub_rn(__fmul_rn(yj, cc[j]), __fmul_rn(yi, ss[j]));
-            }
-          }
-        }
-#pragma unroll
-        for (int d = 0; d < D; ++d) x[d] = __fsub_rn(x[d], v[d]);
         // rotation
 #pragma unroll
-        for (int d = 0; d < D; ++d) x[d] = __fmul_rn(x[d], sSign[d]);
-        fwht_row<D>(x);
-        const float rs = (float)(1.0 / sqrt((double)D));
+        for (int k = 0; k < 2; ++k)
 #pragma unroll
-        for (int d = 0; d < D; ++d) x[d] = __fmul_rn(x[d], rs);
-        RowPack<D> op{x, sCode + rl * cpitch, sScale + rl * 4};
-        dispatch_gb<D>(a.G, b, op);
-        epi_sync();
-        // coalesced copy of the tile's packed rows and scales to global
-        {
-          const int wpr = rowbytes / 8;
-          uint64_t* gdst = reinterpret_cast<uint64_t*>(o.codes + row0 * rowbytes);
-          for (int u = et; u < nrows * wpr; u += 128) {
-            const int rr = u / wpr, w = u - rr * wpr;
-            gdst[u] = *reinterpret_cast<const uint64_t*>(sCode + rr * cpitch + w * 8);
+          for (int u = 0; u < C / 4; ++u) {
+            const float4 s4 = reinterpret_cast<const float4*>(sSign + k * (D / 2) + hf * C)[u];
+            e[k * C + 4 * u + 0] = __fmul_rn(e[k * C + 4 * u + 0], s4.x);
+            e[k * C + 4 * u + 1] = __fmul_rn(e[k * C + 4 * u + 1], s4.y);
+            e[k * C + 4 * u + 2] = __fmul_rn(e[k * C + 4 * u + 2], s4.z);
+            e[k * C + 4 * u + 3] = __fmul_rn(e[k * C + 4 * u + 3], s4.w);
           }
-          float* sdst = o.scales + row0 * ng;
-          for (int u = et; u < nrows * ng; u += 128) sdst[u] = sScale[(u / ng) * 4 + (u % ng)];
-        }
-        epi_sync();
-      } else {
-        if (b > 0) {
-          // coalesced load of the tile's codes and scales into staging
-          const int wpr = rowbytes / 8;
-          const uint64_t* gsrc = reinterpret_cast<const uint64_t*>(o.codes + row0 * rowbytes);
-          for (int u = et; u < nrows * wpr; u += 128) {
-            const int rr = u / wpr, w = u - rr * wpr;
-            *reinterpret_cast<uint64_t*>(sCode + rr * cpitch + w * 8) = gsrc[u];
+        fwht_pair<C>(e, sXch, rl, hf, q);
+        float am[2] = {0.0f, 0.0f};
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+          for (int j = 0; j < C; ++j) {
+            e[k * C + j] = __fmul_rn(e[k * C + j], rs);
+            am[k] = fmaxf(am[k], fabsf(e[k * C + j]));
           }
-          const float* ssrc = o.scales + row0 * ng;
-          for (int u = et; u < nrows * ng; u += 128) sScale[(u / ng) * 4 + (u % ng)] = ssrc[u];
-          epi_sync();
-          if (valid) {
-            float e[D];
-            RowUnpack<D> op{e, sCode + rl * cpitch, sScale + rl * 4};
-            dispatch_gb<D>(a.G, b, op);
-            fwht_row<D>(e);
-            const float rs = (float)(1.0 / sqrt((double)D));
+        float sc[2];
+        float* srow = o.scales + row * ng;
+        float dummy[4];
+        chunk_scales<D>(am, sPm, rl, hf, q, a.G, (float)qmax_of(b), sc, valid ? srow : dummy);
+        if (valid) {
+          uint8_t* crow = o.codes + row * rowbytes;
 #pragma unroll
-            for (int d = 0; d < D; ++d) v[d] = __fadd_rn(v[d], __fmul_rn(__fmul_rn(e[d], rs), sSign[d]));
-          }
-        }
-        if (c.rope && valid) {
-          const float4* cs4 = reinterpret_cast<const float4*>(a.cs + (int64_t)t * (D / 2));
-#pragma unroll
-          for (int i = 0; i < D / 2; i += 2) {
-            const float4 q2 = cs4[i / 2];
-            const float cc[2] = {q2.x, q2.z}, ss[2] = {q2.y, q2.w};
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const float x0 = v[i + j], x1 = v[i + j + D / 2];
-              v[i + j] = __fsub_rn(__fmul_rn(x0, cc[j]), __fmul_rn(x1, ss[j]));
-              v[i + j + D / 2] = __fadd_rn(__fmul_rn(x1, cc[j]), __fmul_rn(x0, ss[j]));
+          for (int k = 0; k < 2; ++k) {
+            uint8_t* dst = crow + (k * (D / 2) + hf * C) * b / 8;
+            uint32_t w[C * 8 / 32];
+            switch (b) {
+              case 2: quant_chunk<C, 2>(e + k * C, sc[k], w); store_bits<C, 2>(dst, w); break;
+              case 3: quant_chunk<C, 3>(e + k * C, sc[k], w); store_bits<C, 3>(dst, w); break;
+              case 4: quant_chunk<C, 4>(e + k * C, sc[k], w); store_bits<C, 4>(dst, w); break;
+              default: quant_chunk<C, 8>(e + k * C, sc[k], w); store_bits<C, 8>(dst, w); break;
             }
           }
         }
-        // decoded row -> staging (bf16), then coalesced 16-byte stores
-        uint8_t* srow = sOut + rl * ROWPITCH_OUT;
+      } else {
+        if (b > 0) {
+          if (!epi_all(mbar_wait(xfull_bar(xb), xph[xb], abort_flag, a.status))) break;
+          const CodeTile ct = code_tile(o, row0, nrows, D, a.G);
+          const uint8_t* cbase = ct.cbulk ? in_buf(xb) : ct.codes;
+          const float* sbase = ct.sbulk ? reinterpret_cast<const float*>(in_buf(xb) + S_CODE) : ct.scales;
 #pragma unroll
-        for (int d = 0; d < D; d += 8) {
-          uint4 w;
-          w.x = (uint32_t)bf16_bits_from_f32(v[d]) | ((uint32_t)bf16_bits_from_f32(v[d + 1]) << 16);
-          w.y = (uint32_t)bf16_bits_from_f32(v[d + 2]) | ((uint32_t)bf16_bits_from_f32(v[d + 3]) << 16);
-          w.z = (uint32_t)bf16_bits_from_f32(v[d + 4]) | ((uint32_t)bf16_bits_from_f32(v[d + 5]) << 16);
-          w.w = (uint32_t)bf16_bits_from_f32(v[d + 6]) | ((uint32_t)bf16_bits_from_f32(v[d + 7]) << 16);
-          *reinterpret_cast<uint4*>(srow + d * 2) = w;
+          for (int k = 0; k < 2; ++k) {
+            const int s0 = k * (D / 2) + hf * C;
+            const float sc = valid ? sbase[rl * ng + s0 / a.G] : 0.0f;
+            uint32_t w[C * 8 / 32];
+            const uint8_t* src = cbase + (int64_t)rl * rowbytes + s0 * b / 8;
+            if (!valid) {
+#pragma unroll
+              for (int j = 0; j < C; ++j) e[k * C + j] = 0.0f;
+              continue;
+            }
+            switch (b) {
+              case 2: load_bits<C, 2>(src, w); dequant_chunk<C, 2>(w, sc, e + k * C); break;
+              case 3: load_bits<C, 3>(src, w); dequant_chunk<C, 3>(w, sc, e + k * C); break;
+              case 4: load_bits<C, 4>(src, w); dequant_chunk<C, 4>(w, sc, e + k * C); break;
+              default: load_bits<C, 8>(src, w); dequant_chunk<C, 8>(w, sc, e + k * C); break;
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xempty_bar(xb));
+          xph[xb] ^= 1;
+          xb ^= 1;
+          fwht_pair<C>(e, sXch, rl, hf, q);
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (int u = 0; u < C / 4; ++u) {
+              const float4 s4 = reinterpret_cast<const float4*>(sSign + k * (D / 2) + hf * C)[u];
+              const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) e[k * C + 4 * u + j] = __fmul_rn(__fmul_rn(e[k * C + 4 * u + j], rs), sv[j]);
+            }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 2 * C; ++j) e[j] = 0.0f;
         }
-        epi_sync();
+        // + backbone
+        if (!epi_all(mbar_wait(tfull_bar(acc), aph[acc], abort_flag, a.status))) break;
+        fence_after();
         {
-          uint16_t* base = (c.kind == 0 ? a.out_k : a.out_v) + (int64_t)c.seq * a.osb + (int64_t)(c.l0 + l) * a.osl +
-                           (int64_t)h * a.osh;
-          constexpr int UPR = D * 2 / 16;    // 16-byte units per row
-          for (int u = et; u < nrows * UPR; u += 128) {
-            const int rr = u / UPR, w = u - rr * UPR;
-            *reinterpret_cast<uint4*>(base + (int64_t)(t0 + rr) * a.ost + w * 8) =
-                *reinterpret_cast<const uint4*>(sOut + rr * ROWPITCH_OUT + w * 16);
+          const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * D);
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            float v[C];
+            tmem_ld<C>(tb + k * (D / 2) + hf * C, v);
+#pragma unroll
+            for (int j = 0; j < C; ++j) e[k * C + j] = __fadd_rn(v[j], e[k * C + j]);
           }
         }
-        epi_sync();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(acc));
+        aph[acc] ^= 1;
+        acc ^= 1;
+        if (valid) {
+          if (c.rope) {
+            const float4* cs4 = reinterpret_cast<const float4*>(a.cs + (int64_t)t * (D / 2) + hf * C);
+#pragma unroll
+            for (int p = 0; p < C / 2; ++p) {
+              const float4 q2 = cs4[p];
+              const float cc[2] = {q2.x, q2.z}, ss[2] = {q2.y, q2.w};
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                const float x0 = e[2 * p + j], x1 = e[C + 2 * p + j];
+                e[2 * p + j] = __fsub_rn(__fmul_rn(x0, cc[j]), __fmul_rn(x1, ss[j]));
+                e[C + 2 * p + j] = __fadd_rn(__fmul_rn(x1, cc[j]), __fmul_rn(x0, ss[j]));
+              }
+            }
+          }
+          uint16_t* base = (c.kind == 0 ? a.out_k : a.out_v) + (int64_t)c.seq * a.osb + (int64_t)(c.l0 + l) * a.osl +
+                           (int64_t)h * a.osh + (int64_t)t * a.ost;
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (int u = 0; u < C / 8; ++u) {
+              const float* s = e + k * C + 8 * u;
+              uint4 w;
+              w.x = (uint32_t)bf16_bits_from_f32(s[0]) | ((uint32_t)bf16_bits_from_f32(s[1]) << 16);
+              w.y = (uint32_t)bf16_bits_from_f32(s[2]) | ((uint32_t)bf16_bits_from_f32(s[3]) << 16);
+              w.z = (uint32_t)bf16_bits_from_f32(s[4]) | ((uint32_t)bf16_bits_from_f32(s[5]) << 16);
+              w.w = (uint32_t)bf16_bits_from_f32(s[6]) | ((uint32_t)bf16_bits_from_f32(s[7]) << 16);
+              *reinterpret_cast<uint4*>(base + k * (D / 2) + hf * C + 8 * u) = w;
+            }
+        }
       }
     }
   }
