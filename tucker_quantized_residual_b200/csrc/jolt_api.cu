@@ -192,6 +192,7 @@ struct jolt_plan_s {
   int* d_Nc = nullptr; int* d_cis = nullptr;
   uint16_t** d_utp = nullptr;
   EighJob* d_jobs_rand = nullptr;
+  double* eig_scr = nullptr;   unsigned int* eig_cnt = nullptr;   int eig_nmax = 0;
 };
 
 struct jolt_handle_s {
@@ -498,6 +499,9 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
     p->d_keep = A.take<int>(nc);
     p->Ut_ws = A.take<uint16_t>((size_t)nc * p->rows_u * p->tp);
     p->Mt_ws = A.take<uint16_t>((size_t)nc * p->lh_max * D * p->rpad_m);
+    p->eig_nmax = std::max(p->opt.mode == JOLT_RANDOMIZED ? p->k : p->nmin_max, D);
+    p->eig_scr = A.take<double>((size_t)nc * (p->eig_nmax + 64));
+    p->eig_cnt = A.take<unsigned int>(nc + 1);
     if (p->opt.mode == JOLT_RANDOMIZED) {
       const int k = p->k;
       const size_t kk = (size_t)k * k;
@@ -797,7 +801,8 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
     JOLT_TRY(launch_symmetrize(p->MB, kk, k, nc, s));
   }
   // spectra only here: eigenvectors follow the allocation (top r_T only)
-  JOLT_TRY(launch_tridiag(p->d_jobs_rand, 2 * nc, std::max(k, D), s));
+  JOLT_TRY(launch_tridiag_multi(p->d_jobs_rand, nc, k, p->eig_scr, p->eig_cnt, status, s));
+  JOLT_TRY(launch_tridiag(p->d_jobs_rand + nc, nc, D, s));
   JOLT_TRY(launch_bisect(p->d_jobs_rand, 2 * nc, std::max(k, D), s));
   JOLT_TRY(launch_rand_spectrum(p->ew, k, p->q_used, p->d_nsq, p->d_wT, nc, s));
   return JOLT_OK;
@@ -886,7 +891,8 @@ static jolt_status run_spectra(jolt_plan_s* p, const void* k_in, const void* v_i
     }
     // spectra only: the token eigenvectors follow the allocation (top r_T)
     ProfScope ps(JOLT_STAGE_EIG, s);
-    JOLT_TRY(launch_tridiag(p->d_jobs_spec, 2 * nc, std::max(p->nmin_max, D), s));
+    JOLT_TRY(launch_tridiag_multi(p->d_jobs_spec, nc, p->nmin_max, p->eig_scr, p->eig_cnt, status, s));
+    JOLT_TRY(launch_tridiag(p->d_jobs_spec + nc, nc, D, s));
     JOLT_TRY(launch_bisect(p->d_jobs_spec, 2 * nc, std::max(p->nmin_max, D), s));
   } else {
     JOLT_TRY(run_range_finder(p, k_in, v_in, seed, status, s));

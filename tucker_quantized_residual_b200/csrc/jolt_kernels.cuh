@@ -20,6 +20,10 @@ struct EighJob {
 jolt_status launch_eigh(const EighJob* jobs_dev, int njobs, int nmax, int* status, cudaStream_t s);
 size_t eigh_smem_bytes(int nmax);
 jolt_status launch_tridiag(const EighJob* jobs, int njobs, int nmax, cudaStream_t s);
+// Multi-block reduction of jobs[0..njobs) (all of size <= nmax); scratch holds
+// njobs * (nmax + 64) doubles, counters njobs + 1 words.
+jolt_status launch_tridiag_multi(const EighJob* jobs, int njobs, int nmax, double* scratch, unsigned int* counters,
+                                 int* status, cudaStream_t s);
 jolt_status launch_bisect(const EighJob* jobs, int njobs, int nmax, cudaStream_t s);
 jolt_status launch_eigvecs(const EighJob* jobs, int njobs, int nvec_max, const int* nvec, cudaStream_t s);
 jolt_status launch_fgram_x(const CellDesc* cells, int ncells, int D, const float2* cs, int nchunk,

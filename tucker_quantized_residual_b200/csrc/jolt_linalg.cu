@@ -519,6 +519,137 @@ __global__ void __launch_bounds__(EIG_THREADS) k_tridiag(const EighJob* __restri
   }
 }
 
+// The same reduction with G thread blocks per matrix (one cooperative launch
+// over all jobs). Every block of a job computes the reflector of column k
+// itself from row k (A is kept exactly symmetric, so row k equals column k),
+// forms p = beta A v for its share of the rows, and publishes it; after a
+// job-wide barrier each block rebuilds w = p - (beta/2)(p.v) v from all
+// shares (partial sums added in block order, so every block gets the same
+// bits) and applies the rank-2 update to its own rows; a second barrier
+// precedes the next column. A is read through L2 only (other blocks write
+// it). Barriers are counters in global memory with bounded waits: on expiry
+// the block raises the job's abort flag and the timeout status and returns,
+// and the others follow at their next wait.
+__device__ __forceinline__ unsigned long long gtimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ bool job_barrier(unsigned int* cnt, unsigned int target, volatile int* abort_flag, int* status) {
+  __shared__ int ok_s;
+  __threadfence();          // this thread's writes of A, p and the partial sums
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    atomicAdd(cnt, 1u);
+    int ok = 1;
+    const unsigned long long t0 = gtimer_ns();
+    while (true) {
+      unsigned int c;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(cnt) : "memory");
+      if (c >= target) break;
+      if (*abort_flag) { ok = 0; break; }
+      if (gtimer_ns() - t0 > 2000000000ull) {
+        *abort_flag = 1;
+        atomicOr(status, DEV_ERR_TIMEOUT);
+        ok = 0;
+        break;
+      }
+    }
+    __threadfence();
+    ok_s = ok;
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
+__global__ void __launch_bounds__(EIG_THREADS) k_tridiag_multi(const EighJob* __restrict__ jobs, int G, int nmax,
+                                                               double* __restrict__ scratch,
+                                                               unsigned int* __restrict__ counters, int* status) {
+  const int job = blockIdx.x / G, c = blockIdx.x % G;
+  const EighJob J = jobs[job];
+  const int n = J.n;
+  if (n <= 0) return;
+  extern __shared__ double sh[];
+  double* v = sh;            // n
+  double* w = v + n;         // n
+  double* red = w + n;       // 32
+  double* A = J.A;
+  double* dd = J.work;
+  double* ee = dd + n;
+  double* tau = ee + n;
+  double* P = scratch + (size_t)job * (nmax + 64);   // p (n) then per-block partial sums (G <= 64)
+  double* part = P + nmax;
+  unsigned int* cnt = counters + job;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(counters + gridDim.x / G);
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5, nwarp = nt >> 5;
+  const int gw = c * nwarp + warp, GW = G * nwarp;
+  unsigned int nbar = 0;
+  for (int k = 0; k + 2 < n; ++k) {
+    const int m = n - k - 1;
+    const double* rowk = A + (int64_t)k * n + (k + 1);
+    for (int i = tid; i < m; i += nt) v[i] = __ldcg(rowk + i);
+    __syncthreads();
+    double s = 0.0;
+    for (int i = 1 + tid; i < m; i += nt) s += v[i] * v[i];
+    s = block_sum(s, red);
+    const double x0 = v[0];
+    if (s == 0.0) {
+      if (c == 0 && tid == 0) { dd[k] = __ldcg(A + (int64_t)k * n + k); ee[k] = x0; tau[k] = 0.0; }
+      __syncthreads();
+      continue;
+    }
+    const double nrm = sqrt(x0 * x0 + s);
+    const double alpha = (x0 <= 0.0) ? nrm : -nrm;
+    const double v0 = x0 - alpha;
+    const double beta = 2.0 / (s + v0 * v0);
+    __syncthreads();
+    if (tid == 0) v[0] = v0;
+    __syncthreads();
+    double pv = 0.0;
+    for (int i = gw; i < m; i += GW) {
+      const double* row = A + (int64_t)(k + 1 + i) * n + (k + 1);
+      double acc = 0.0;
+      for (int j = lane; j < m; j += 32) acc += __ldcg(row + j) * v[j];
+      acc = warp_sum(acc);
+      if (lane == 0) {
+        const double pi = beta * acc;
+        P[i] = pi;
+        pv += pi * v[i];
+      }
+    }
+    pv = block_sum(pv, red);
+    if (tid == 0) part[c] = pv;
+    if (!job_barrier(cnt, (++nbar) * (unsigned)G, abort_flag, status)) return;
+    double tot = 0.0;
+    for (int b = 0; b < G; ++b) tot += __ldcg(part + b);
+    const double Kc = 0.5 * beta * tot;
+    for (int i = tid; i < m; i += nt) w[i] = __ldcg(P + i) - Kc * v[i];
+    __syncthreads();
+    for (int i = gw; i < m; i += GW) {
+      double* row = A + (int64_t)(k + 1 + i) * n + (k + 1);
+      const double vi = v[i], wi = w[i];
+      // no contraction: entry (i, j) and (j, i) get the same two products
+      for (int j = lane; j < m; j += 32)
+        row[j] = __dsub_rn(__ldcg(row + j), __dadd_rn(__dmul_rn(vi, w[j]), __dmul_rn(wi, v[j])));
+      if (lane == 0) A[(int64_t)(k + 1 + i) * n + k] = v[i];
+    }
+    if (c == 0 && tid == 0) { dd[k] = __ldcg(A + (int64_t)k * n + k); ee[k] = alpha; tau[k] = beta; }
+    if (!job_barrier(cnt, (++nbar) * (unsigned)G, abort_flag, status)) return;
+  }
+  if (c == 0 && tid == 0) {
+    if (n >= 2) {
+      dd[n - 2] = __ldcg(A + (int64_t)(n - 2) * n + (n - 2));
+      ee[n - 2] = __ldcg(A + (int64_t)(n - 1) * n + (n - 2));
+      tau[n - 2] = 0.0;
+    }
+    dd[n - 1] = __ldcg(A + (int64_t)(n - 1) * n + (n - 1));
+    ee[n - 1] = 0.0;
+    tau[n - 1] = 0.0;
+  }
+}
+
 // Number of eigenvalues of the tridiagonal (d, e) smaller than x.
 __device__ __forceinline__ int sturm_count(const double* d, const double* e, int n, double x, double pivmin) {
   int c = 0;
@@ -671,6 +802,44 @@ jolt_status launch_tridiag(const EighJob* jobs, int njobs, int nmax, cudaStream_
   const size_t smem = (size_t)(2 * nmax + 32) * sizeof(double);
   { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_tridiag, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
   k_tridiag<<<njobs, EIG_THREADS, smem, s>>>(jobs);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+// Blocks per job for the multi-block reduction: as many as fit on the device
+// at once (cooperative launch), at least two matrix rows per warp.
+static int tridiag_blocks_per_job(int njobs, int nmax, size_t smem) {
+  static int sms = 0, per_sm = -1;
+  static size_t smem_at = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  if (per_sm < 0 || smem_at != smem) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_tridiag_multi, EIG_THREADS, smem) != cudaSuccess)
+      per_sm = 0;
+    cudaGetLastError();
+    smem_at = smem;
+  }
+  const int cap = sms * per_sm;
+  int G = njobs > 0 ? cap / njobs : 0;
+  G = std::min(G, std::max(1, nmax / (2 * (EIG_THREADS / 32))));
+  return std::min(G, 64);
+}
+
+jolt_status launch_tridiag_multi(const EighJob* jobs, int njobs, int nmax, double* scratch, unsigned int* counters,
+                                 int* status, cudaStream_t s) {
+  if (njobs <= 0) return JOLT_OK;
+  const size_t smem = (size_t)(2 * nmax + 32) * sizeof(double);
+  { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_tridiag_multi, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
+  const int G = tridiag_blocks_per_job(njobs, nmax, smem);
+  if (G < 2) return launch_tridiag(jobs, njobs, nmax, s);
+  JOLT_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)(njobs + 1) * sizeof(unsigned int), s));
+  int Gv = G, nm = nmax;
+  void* args[] = {(void*)&jobs, (void*)&Gv, (void*)&nm, (void*)&scratch, (void*)&counters, (void*)&status};
+  JOLT_CUDA_TRY(cudaLaunchCooperativeKernel((const void*)k_tridiag_multi, dim3(njobs * G), dim3(EIG_THREADS), args,
+                                            smem, s));
   JOLT_LAUNCHED();
   return JOLT_OK;
 }
