@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--groups", type=int, default=0,
+                    help="only the first N layer groups of the config (small profiling cases)")
+    ap.add_argument("--cpu-tokens", type=int, default=4096, help="tokens in the CPU baseline sample")
     ap.add_argument("--stages", action="store_true", help="print the per-stage table to stderr")
     return ap.parse_args()
 
@@ -107,31 +110,48 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ workload
-def gemm_flops(spec, k, ncells_per_kind):
-    """Algorithmic FLOPs of one launch of each tensor-core GEMM stage."""
-    Lg = spec.group_size
-    N = Lg * spec.n_heads * spec.head_dim
-    T = spec.seq_len
-    cells = 2 * ncells_per_kind
-    return {"gemm_xw": 2.0 * T * N * k * cells, "gemm_xty": 2.0 * N * T * k * cells,
-            "gemm_gram": 2.0 * k * k * T * cells,
-            "fgram": 2.0 * spec.head_dim ** 2 * Lg * spec.n_heads * T * cells}
+# DRAM bytes per launch of the dominant kernel from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), scaled to the full launch
+# by the cells it processes; None once the kernel has changed since.
+GEMM_TRAFFIC = None
 
 
-def residual_bytes(spec, cells):
-    """Algorithmic HBM bytes of one residual launch and one decompress launch,
-    from the chosen (r_T, r_d, b) of every cell."""
-    D, T, H = spec.head_dim, spec.seq_len, spec.n_heads
-    res = dec = 0.0
+def sketch_width(spec, ratio, p=8):
+    """k = q_cap (Eq. 5) + p, rounded up to a multiple of 16."""
+    q = min(max(32 if ratio <= 4 else 64, -(-spec.seq_len // 32)), 512)
+    return ((q + p + 15) // 16) * 16
+
+
+def stage_work(spec, cells, k, power_iters=2):
+    """Algorithmic work of one step, per stage: (flops, HBM bytes, launches).
+
+    Tensor-core GEMM passes over X (2k flops and one 2-byte read per element
+    each): the sketch X W0, then per power iteration X^T Y and X W, then the
+    final X^T Y; the Gram Y^T Y of the last sketch. Residual pass: read X
+    (2 B/elem), write codes + scales, 2 r_T flops/elem for the backbone.
+    Decode: read the payload, write 2 B/elem, 2 r_T flops/elem."""
+    Lg, H, D, T = spec.group_size, spec.n_heads, spec.head_dim, spec.seq_len
+    ncell = len(cells)
+    elems = Lg * H * T * D                     # per cell
+    N = Lg * H * D
+    w = {}
+    w["gemm_xw"] = (2.0 * T * N * k * ncell * (power_iters + 1),
+                    (2.0 * elems + 2.0 * (N + T) * k) * ncell * (power_iters + 1), power_iters + 1)
+    w["gemm_xty"] = (2.0 * T * N * k * ncell * (power_iters + 1),
+                     (2.0 * elems + 2.0 * T * k + 4.0 * N * k) * ncell * (power_iters + 1), power_iters + 1)
+    w["gemm_gram"] = (2.0 * k * k * T * ncell, 2.0 * T * k * ncell, 1)
+    res_f = res_b = dec_f = dec_b = 0.0
+    rows = Lg * H * T
     for c in cells:
-        n = c.bits
-        rows = spec.group_size * H * T
-        dense = rows * D * 2
-        payload = c.bytes
-        resid = rows * (n * D // 8 + 4 * (D // D)) if n else 0     # codes + one scale per row
-        res += (dense + resid) if n else 0.0
-        dec += payload + dense
-    return res, dec
+        back = 2.0 * c.r_t * elems
+        dec_f += back
+        dec_b += c.bytes + 2.0 * elems
+        if c.bits:
+            res_f += back
+            res_b += 2.0 * elems + rows * (c.bits * D // 8 + 4)
+    w["residual"] = (res_f, res_b, 1)
+    w["decompress"] = (dec_f, dec_b, 1)
+    return w
 
 
 def run_jolt(args):
@@ -148,6 +168,8 @@ def run_jolt(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     spec = synth.SPECS[args.config]
+    if args.groups:
+        spec = spec.replace(n_layers=min(spec.n_layers, args.groups * spec.group_size))
     gs = synth.group_starts(spec)
     K, V = synth.make_cache(spec, seed=1000 * rank, device="cuda")
     torch.cuda.synchronize()
@@ -239,34 +261,50 @@ def run_jolt(args):
                "d2h_bytes_per_step": 2 * Ko.numel() * Ko.element_size()}
         del Kh, Vh, Koh, Voh, Kd, Vd
 
-    # ---- roofline of the dominant stage
+    # ---- roofline: the dominant kernel, and the whole path per stage
     pk, src = peaks()
-    k_sk = ((min(max(32 if args.ratio <= 4 else 64, -(-spec.seq_len // 32)), 512) + 8 + 15) // 16) * 16
-    flops = gemm_flops(spec, k_sk, ncell // 2)
-    res_b, dec_b = residual_bytes(spec, cells)
-    per_step = {s: prof[s][0] / args.steps for s in prof}
-    dom = max(per_step, key=per_step.get)
-    roof = None
-    if dom in flops and prof[dom][1] > 0:
-        per_launch_ms = prof[dom][0] / prof[dom][1]
-        ach = flops[dom] / (per_launch_ms / 1e3) / 1e12
-        peak = pk["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(ach / peak, 3), "peak_source": f"{src} (sustained bf16)", "traffic": None}
-    elif dom in ("residual", "decompress") and prof[dom][1] > 0:
-        per_launch_ms = prof[dom][0] / prof[dom][1]
-        byt = res_b if dom == "residual" else dec_b
-        ach = byt / (per_launch_ms / 1e3) / 1e9
-        peak = pk["hbm_gbs"]
-        roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(ach / peak, 3), "peak_source": f"{src} (copy bandwidth)", "traffic": None}
+    work = stage_work(spec, cells, sketch_width(spec, args.ratio))
+    per_step = {s_: prof[s_][0] / args.steps for s_ in prof}
+    tc = pk["bf16_tflops_sustained"] * 1e12
+    bw = pk["hbm_gbs"] * 1e9
+    # the tcgen05 GEMM kernel (its X W and X^T Y launches) against the stream passes
+    gemm_ms = per_step.get("gemm_xw", 0.0) + per_step.get("gemm_xty", 0.0)
+    cand = {"gemm": gemm_ms, "residual": per_step.get("residual", 0.0),
+            "decompress": per_step.get("decompress", 0.0)}
+    dom = max(cand, key=cand.get)
+    if dom == "gemm":
+        fl = work["gemm_xw"][0] + work["gemm_xty"][0]
+        nl = work["gemm_xw"][2] + work["gemm_xty"][2]
+        per_launch_s = gemm_ms / 1e3 / nl
+        ach = fl / nl / per_launch_s / 1e12
+        roof = {"bound": "tensor", "kernel": "k_umma_gemm (X W and X^T Y launches)", "achieved": round(ach, 1),
+                "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops_sustained"], 3),
+                "peak_source": f"{src} bf16 sustained", "flops_per_launch": fl / nl,
+                "traffic": GEMM_TRAFFIC}
     else:
-        roof = {"bound": "latency", "kernel": dom, "achieved": None, "peak": None, "unit": None, "frac": None,
-                "traffic": None}
+        fl, by, nl = work[dom]
+        per_launch_s = cand[dom] / 1e3 / nl
+        if fl / tc > by / bw:
+            ach = fl / nl / per_launch_s / 1e12
+            roof = {"bound": "tensor", "kernel": f"k_stream ({dom})", "achieved": round(ach, 1),
+                    "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                    "frac": round(ach / pk["bf16_tflops_sustained"], 3), "peak_source": f"{src} bf16 sustained",
+                    "traffic": None}
+        else:
+            ach = by / nl / per_launch_s / 1e9
+            roof = {"bound": "hbm", "kernel": f"k_stream ({dom})", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 3), "peak_source": f"{src} copy bandwidth",
+                    "traffic": None}
+    bound_ms = 0.0
+    for st_, (fl, by, nl) in work.items():
+        bound_ms += 1e3 * max(fl / tc, by / bw)
+    path_roof = {"bound_ms": round(bound_ms, 3), "ms_per_step": round(ms / args.steps, 3),
+                 "frac": round(bound_ms / (ms / args.steps), 3),
+                 "rule": "sum over GEMM passes, residual and decode of max(flops / sustained bf16, bytes / HBM)"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(spec, K, V, args.ratio)
+        cpu = cpu_baseline(spec, K, V, args.ratio, args.cpu_tokens)
 
     if args.stages and rank == 0:
         for s in jolt.STAGES:
@@ -295,9 +333,10 @@ def run_jolt(args):
                                    f"batch {spec.batch}), {args.ratio:g}x budget, {args.mode} token SVD",
                        "global_batch": spec.batch * world, "seq_len": spec.seq_len,
                        "parallelism": f"independent caches per GPU (dp{world})",
-                       "l2": "inputs 8.6 GB per GPU, larger than L2; no flush"},
+                       "l2": f"inputs {dense / 1e9:.2f} GB per GPU" + (
+                           ", larger than L2; no flush" if dense > 126e6 else ", smaller than L2")},
             "rel_frobenius_err": {"K": errK, "V": errV}, "bytes": nbytes, "budget": B,
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+            "roofline": roof, "path_roofline": path_roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clk,
             "stages_ms_per_step": {s: round(v, 3) for s, v in per_step.items() if v > 0},
         }
@@ -342,7 +381,7 @@ def run_oracle_sample(Ks, Vs, spec, ratio):
     return time.perf_counter() - t0, 2 * n
 
 
-def cpu_baseline(spec, K, V, ratio, T_sample=2048):
+def cpu_baseline(spec, K, V, ratio, T_sample=4096):
     Ks, Vs = cpu_sample(spec, K, V, T_sample)
     sec, nbytes = run_oracle_sample(Ks, Vs, spec, ratio)
     return {"value": round(nbytes / sec / 1e9, 6), "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",

@@ -101,11 +101,11 @@ jolt_status launch_umma(const umma::Maps& maps, const umma::Problem& p, cudaStre
   static bool attr = false;
   if (!attr) {
     JOLT_CUDA_TRY(cudaFuncSetAttribute(umma::k_umma_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       umma::SMEM_BYTES));
+                                       umma::SMEM_DATA_MAX + 1024 + 256));
     attr = true;
   }
   const int grid = std::min(ntiles, num_sms());
-  umma::k_umma_gemm<<<grid, umma::THREADS, umma::SMEM_BYTES, s>>>(maps, p);
+  umma::k_umma_gemm<<<grid, umma::THREADS, umma::smem_bytes(p.BN), s>>>(maps, p);
   JOLT_LAUNCHED();
   return JOLT_OK;
 }

@@ -393,6 +393,28 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
         CellDesc c;
         CellOut o;
         if (!tile_of(a, tile, cell, t0, lh, c, o, COMPRESS)) continue;
+        // the tile's second input (X, or codes + scales) first: it then loads
+        // while the tensor cores work on the backbone
+        if (COMPRESS || o.b > 0) {
+          if (!mbar_wait(xempty_bar(xb), xph[xb] ^ 1, abort_flag, a.status)) break;
+          const uint32_t sx = smem_u32(in_buf(xb));
+          if (COMPRESS) {
+            mbar_expect_tx(xfull_bar(xb), D * 128 * 2);
+            const CUtensorMap* xm = (c.kind == 0) ? &maps.xk : &maps.xv;
+            const int l = c.l0 + lh / c.H, h = lh % c.H;
+            for (int hh = 0; hh < D / 64; ++hh)
+              tma_load_5d(sx + hh * 16384, xm, xfull_bar(xb), hh * 64, t0, h, l, c.seq);
+          } else {
+            const CodeTile ct = code_tile(o, (int64_t)lh * c.T + t0, min(SBM, c.T - t0), D, a.G);
+            mbar_expect_tx(xfull_bar(xb), (ct.cbulk ? ct.cbytes : 0u) + (ct.sbulk ? ct.sbytes : 0u));
+            if (ct.cbulk) bulk_load(sx, ct.codes, ct.cbytes, xfull_bar(xb));
+            if (ct.sbulk) bulk_load(sx + S_CODE, ct.scales, ct.sbytes, xfull_bar(xb));
+          }
+          xissued[xb] = true;
+          xissued_phase[xb] = xph[xb];
+          xph[xb] ^= 1;
+          xb ^= 1;
+        }
         const int nk = (o.rT + 63) / 64;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(empty_bar(stage), ph ^ 1, abort_flag, a.status)) { ok = false; break; }
@@ -406,25 +428,6 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
           if (++stage == SSTAGES) { stage = 0; ph ^= 1; }
         }
         if (!ok) break;
-        if (!COMPRESS && o.b == 0) continue;
-        if (!mbar_wait(xempty_bar(xb), xph[xb] ^ 1, abort_flag, a.status)) break;
-        const uint32_t sx = smem_u32(in_buf(xb));
-        if (COMPRESS) {
-          mbar_expect_tx(xfull_bar(xb), D * 128 * 2);
-          const CUtensorMap* xm = (c.kind == 0) ? &maps.xk : &maps.xv;
-          const int l = c.l0 + lh / c.H, h = lh % c.H;
-          for (int hh = 0; hh < D / 64; ++hh)
-            tma_load_5d(sx + hh * 16384, xm, xfull_bar(xb), hh * 64, t0, h, l, c.seq);
-        } else {
-          const CodeTile ct = code_tile(o, (int64_t)lh * c.T + t0, min(SBM, c.T - t0), D, a.G);
-          mbar_expect_tx(xfull_bar(xb), (ct.cbulk ? ct.cbytes : 0u) + (ct.sbulk ? ct.sbytes : 0u));
-          if (ct.cbulk) bulk_load(sx, ct.codes, ct.cbytes, xfull_bar(xb));
-          if (ct.sbulk) bulk_load(sx + S_CODE, ct.scales, ct.sbytes, xfull_bar(xb));
-        }
-        xissued[xb] = true;
-        xissued_phase[xb] = xph[xb];
-        xph[xb] ^= 1;
-        xb ^= 1;
       }
       for (int s = 0; s < SSTAGES; ++s)
         if (issued[s]) {

@@ -35,11 +35,17 @@ enum Mode : int { XW = 0, XTY = 1, GRAM = 2, WP = 3, FG = 4 };
 constexpr int BM = 128;          // rows of an output tile (TMEM lanes)
 constexpr int BK = 64;           // K per pipeline stage (128 bytes of bf16)
 constexpr int BN_MAX = 256;
-constexpr int STAGES = 4;
+constexpr int MAX_STAGES = 8;
 constexpr int A_BYTES = BM * BK * 2;          // 16 KB
-constexpr int B_BYTES = BN_MAX * BK * 2;      // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int SMEM_DATA_MAX = 224 * 1024;     // pipeline stages (plus 1 KB alignment and barriers)
+// Bytes of one pipeline stage for an output tile BN wide (A tile + B tile,
+// each a whole number of 1 KB swizzle atoms), and the stages that fit.
+__host__ __device__ inline int stage_bytes(int BN) { return A_BYTES + (BN * BK * 2 + 1023) / 1024 * 1024; }
+__host__ __device__ inline int num_stages(int BN) {
+  const int n = SMEM_DATA_MAX / stage_bytes(BN);
+  return n < MAX_STAGES ? n : MAX_STAGES;
+}
+__host__ __device__ inline int smem_bytes(int BN) { return num_stages(BN) * stage_bytes(BN) + 1024 + 256; }
 constexpr int THREADS = 192;
 constexpr unsigned long long WAIT_NS = 2000000000ull;   // 2 s per wait
 
@@ -239,6 +245,7 @@ __device__ __forceinline__ void k_range(const Problem& p, int cell, int m0, int&
 __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm(const __grid_constant__ Maps maps, Problem p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int STAGES = num_stages(p.BN), STAGE_BYTES = stage_bytes(p.BN);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
   // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
@@ -276,9 +283,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm(const __grid_constant_
     if (lane == 0) {
       int stage = 0;
       uint32_t ph = 0;
-      uint32_t issued_phase[STAGES];
-      bool issued[STAGES];
-      for (int s = 0; s < STAGES; ++s) issued[s] = false;
+      uint32_t issued_phase[MAX_STAGES];
+      bool issued[MAX_STAGES];
+      for (int s = 0; s < MAX_STAGES; ++s) issued[s] = false;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         int cell, m0, n0;
