@@ -154,6 +154,21 @@ def stage_work(spec, cells, k, power_iters=2):
     return w
 
 
+def max_over_ranks(x, world, dist=None, device=None):
+    """The largest value of x over all ranks (each rank's own device time)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput_gbs(world, dense_bytes, steps, ms):
+    """Whole-job GB/s: every rank's dense bytes over the slowest rank's time."""
+    return world * dense_bytes * steps / (ms / 1e3) / 1e9
+
+
 def run_jolt(args):
     import torch
     import torch.distributed as dist
@@ -216,13 +231,10 @@ def run_jolt(args):
     launches = jolt.jolt_launch_count() - l0
     prof = jolt.jolt_profile_read()
     jolt.jolt_profile_enable(False)
-    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
-    value = world * dense * args.steps / (ms / 1e3) / 1e9
+    value = throughput_gbs(world, dense, args.steps, ms)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -251,12 +263,8 @@ def run_jolt(args):
             jolt.jolt_free_handle(hh)
         f1.record(stream)
         torch.cuda.synchronize()
-        ems = f0.elapsed_time(f1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": round(world * dense * args.e2e_steps / (ems / 1e3) / 1e9, 3), "unit": "GB/s",
+        ems = max_over_ranks(f0.elapsed_time(f1), world, dist, dev)
+        e2e = {"value": round(throughput_gbs(world, dense, args.e2e_steps, ems), 3), "unit": "GB/s",
                "h2d_bytes_per_step": 2 * K.numel() * K.element_size(),
                "d2h_bytes_per_step": 2 * Ko.numel() * Ko.element_size()}
         del Kh, Vh, Koh, Voh, Kd, Vd

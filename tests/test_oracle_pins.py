@@ -33,6 +33,15 @@ def test_philox_words_are_uniform_and_distinct():
     assert np.mean(o.philox_block(1024, 7, 4) == o.philox_block(1024, 7, 3)) < 0.01
 
 
+def test_philox_known_answer_vectors():
+    kat = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "philox4x32_10_kat.json")))
+    for v in kat["vectors"]:
+        ctr = np.array([int(x, 16) for x in v["ctr"]], dtype=np.uint32)
+        key = tuple(int(x, 16) for x in v["key"])
+        out = o.philox4x32_10(ctr, key)
+        assert [int(x) for x in out] == [int(x, 16) for x in v["out"]]
+
+
 def test_gaussian_moments_and_tails():
     z = o.gaussian_f64(1 << 18, seed=0, stream=o.STREAM_CALIB)
     assert abs(z.mean()) < 0.01 and abs(z.var() - 1) < 0.01
