@@ -37,9 +37,8 @@ constexpr int S_B = 128 * 64 * 2;          // M^T slice: D rows x 64 ranks (D <=
 constexpr int S_X = 128 * 128 * 2;         // input tile: 128 tokens x D
 constexpr int S_CODE = 128 * 128;          // packed codes of a tile (<= 8 bits x 128 per row)
 constexpr int S_SCALE = 128 * 4 * 4;       // scales of a tile (<= 4 groups per row)
-constexpr int S_XCH = 128 * 256;           // pair exchange: 128 rows x 2 halves x 128 bytes
 constexpr int S_R1 = (2 * S_X > 2 * (S_CODE + S_SCALE)) ? 2 * S_X : 2 * (S_CODE + S_SCALE);
-constexpr int SMEM_STREAM = SSTAGES * (S_A + S_B) + S_R1 + S_XCH + 128 * 16 + 128 * 4 + 1024 + 512;
+constexpr int SMEM_STREAM = SSTAGES * (S_A + S_B) + S_R1 + 128 * 16 + 128 * 4 + 1024 + 512;
 constexpr int EPI_WARPS = 8;
 constexpr int STHREADS = 64 + 32 * EPI_WARPS;
 
@@ -170,35 +169,53 @@ __device__ __forceinline__ void fwht_chunk(float* v) {
   }
 }
 
-// Exchange slot of (row r, half hf), 16-byte unit u < 8, swizzled by row.
-__device__ __forceinline__ float4* xch_at(uint8_t* xch, int r, int hf, int u) {
-  return reinterpret_cast<float4*>(xch + r * 256 + hf * 128 + ((u ^ (r & 7)) << 4));
+template <int N>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const float* v);
+template <>
+__device__ __forceinline__ void tmem_st<16>(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+      : "memory");
 }
+template <>
+__device__ __forceinline__ void tmem_st<32>(uint32_t taddr, const float* v) {
+  tmem_st<16>(taddr, v);
+  tmem_st<16>(taddr + 16, v + 16);
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Full transform of the thread's 2C values: in-chunk stages, the span-C stage
 // with the partner half, then the span-D/2 stage between the two chunks.
+// The partner's values come through tensor memory: each thread stores its
+// 2C values in its own TMEM lane at columns xcol + hf * 2C (xcol alternates
+// between two regions from tile to tile, so a region is rewritten only after
+// the partner has passed the next pair barrier), and reads the partner's
+// columns after the barrier.
 template <int C>
-__device__ __forceinline__ void fwht_pair(float* e, uint8_t* xch, int r, int hf, int q) {
+__device__ __forceinline__ void fwht_pair(float* e, uint32_t lane_base, uint32_t xcol, int hf, int q) {
   fwht_chunk<C>(e);
   fwht_chunk<C>(e + C);
+  const uint32_t mine = lane_base + xcol + (uint32_t)(hf * 2 * C);
+  const uint32_t theirs = lane_base + xcol + (uint32_t)((hf ^ 1) * 2 * C);
+  tmem_st<C>(mine, e);
+  tmem_st<C>(mine + C, e + C);
+  tmem_wait_st();
+  fence_before();
+  pair_sync(q);
+  fence_after();
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
+    float p[C];
+    tmem_ld<C>(theirs + k * C, p);
     float* v = e + k * C;
 #pragma unroll
-    for (int u = 0; u < C / 4; ++u) *xch_at(xch, r, hf, u) = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-    pair_sync(q);
-#pragma unroll
-    for (int u = 0; u < C / 4; ++u) {
-      const float4 p = *xch_at(xch, r, hf ^ 1, u);
-      const float pv[4] = {p.x, p.y, p.z, p.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        // half 0 holds the lower index of each pair (a + b), half 1 the upper (a - b)
-        const float mine = v[4 * u + j];
-        v[4 * u + j] = hf == 0 ? __fadd_rn(mine, pv[j]) : __fsub_rn(pv[j], mine);
-      }
-    }
-    pair_sync(q);
+    for (int j = 0; j < C; ++j)   // half 0 holds the lower index of each pair (a + b), half 1 the upper (a - b)
+      v[j] = hf == 0 ? __fadd_rn(v[j], p[j]) : __fsub_rn(p[j], v[j]);
   }
 #pragma unroll
   for (int j = 0; j < C; ++j) {
@@ -334,8 +351,7 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
   uint8_t* sA = smem;                                   // SSTAGES x S_A
   uint8_t* sB = sA + SSTAGES * S_A;                     // SSTAGES x S_B
   uint8_t* sR1 = sB + SSTAGES * S_B;                    // 2 x S_X (compress) | 2 x (codes + scales)
-  uint8_t* sXch = sR1 + S_R1;                           // S_XCH
-  float* sPm = reinterpret_cast<float*>(sXch + S_XCH);  // 128 rows x 2 halves x 2 chunk maxima
+  float* sPm = reinterpret_cast<float*>(sR1 + S_R1);   // 128 rows x 2 halves x 2 chunk maxima
   float* sSign = sPm + 128 * 4;                         // D (<= 128)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sSign + 128);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * SSTAGES + 8);
@@ -352,7 +368,8 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
   auto xfull_bar = [&](int b) { return bar0 + 8u * (2 * SSTAGES + 4 + b); };
   auto xempty_bar = [&](int b) { return bar0 + 8u * (2 * SSTAGES + 6 + b); };
   auto in_buf = [&](int b) { return sR1 + b * (COMPRESS ? S_X : S_CODE + S_SCALE); };
-  constexpr int NCOLS = (2 * D <= 128) ? 128 : 256;
+  // two accumulators (2D columns) and two exchange regions of 2 x D/2 columns
+  constexpr int NCOLS = (4 * D <= 256) ? 256 : 512;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SSTAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
@@ -479,8 +496,9 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
     const int rl = q * 32 + lane;             // row within the tile (TMEM lane)
     const int et = threadIdx.x - 64;          // 0..255 among the epilogue threads
     const float rs = (float)(1.0 / sqrt((double)D));
-    int acc = 0, xb = 0;
+    int acc = 0, xb = 0, xpar = 0;
     uint32_t aph[2] = {0, 0}, xph[2] = {0, 0};
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
       int cell, t0, lh;
       CellDesc c;
@@ -505,6 +523,13 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
       const int64_t row = row0 + rl;
       float e[2 * C];
       if (COMPRESS) {
+        // the first half of this row's RoPE table entries, fetched before the waits
+        const float4* cs4 = reinterpret_cast<const float4*>(a.cs + (int64_t)(valid ? t : 0) * (D / 2) + hf * C);
+        float4 csr[C / 4];
+        if (c.rope) {
+#pragma unroll
+          for (int p = 0; p < C / 4; ++p) csr[p] = cs4[p];
+        }
         // backbone
         if (!epi_all(mbar_wait(tfull_bar(acc), aph[acc], abort_flag, a.status))) break;
         fence_after();
@@ -519,7 +544,6 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
         // E = [un-RoPE](X) - backbone
         if (!epi_all(mbar_wait(xfull_bar(xb), xph[xb], abort_flag, a.status))) break;
         const uint8_t* xs = in_buf(xb);
-        const float4* cs4 = reinterpret_cast<const float4*>(a.cs + (int64_t)(valid ? t : 0) * (D / 2) + hf * C);
 #pragma unroll
         for (int u = 0; u < C / 8; ++u) {
           float x0[8], x1[8];
@@ -528,7 +552,7 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
           if (c.rope) {
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
-              const float4 q2 = cs4[4 * u + p];
+              const float4 q2 = (4 * u + p < C / 4) ? csr[4 * u + p] : cs4[4 * u + p];
               const float cc[2] = {q2.x, q2.z}, ss[2] = {q2.y, q2.w};
 #pragma unroll
               for (int j = 0; j < 2; ++j) {
@@ -559,7 +583,8 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
             e[k * C + 4 * u + 2] = __fmul_rn(e[k * C + 4 * u + 2], s4.z);
             e[k * C + 4 * u + 3] = __fmul_rn(e[k * C + 4 * u + 3], s4.w);
           }
-        fwht_pair<C>(e, sXch, rl, hf, q);
+        fwht_pair<C>(e, lane_base, (uint32_t)(2 * D + xpar * D), hf, q);
+        xpar ^= 1;
         float am[2] = {0.0f, 0.0f};
 #pragma unroll
         for (int k = 0; k < 2; ++k)
@@ -590,31 +615,37 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
         if (b > 0) {
           if (!epi_all(mbar_wait(xfull_bar(xb), xph[xb], abort_flag, a.status))) break;
           const CodeTile ct = code_tile(o, row0, nrows, D, a.G);
-          const uint8_t* cbase = ct.cbulk ? in_buf(xb) : ct.codes;
-          const float* sbase = ct.sbulk ? reinterpret_cast<const float*>(in_buf(xb) + S_CODE) : ct.scales;
+          const uint8_t* stage_in = in_buf(xb);
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
             const int s0 = k * (D / 2) + hf * C;
-            const float sc = valid ? sbase[rl * ng + s0 / a.G] : 0.0f;
-            uint32_t w[C * 8 / 32];
-            const uint8_t* src = cbase + (int64_t)rl * rowbytes + s0 * b / 8;
             if (!valid) {
 #pragma unroll
               for (int j = 0; j < C; ++j) e[k * C + j] = 0.0f;
               continue;
             }
+            // staged copies are read as shared memory, the fallback from global memory
+            const float sc = ct.sbulk ? reinterpret_cast<const float*>(stage_in + S_CODE)[rl * ng + s0 / a.G]
+                                      : ct.scales[rl * ng + s0 / a.G];
+            const int64_t off = (int64_t)rl * rowbytes + s0 * b / 8;
+            uint32_t w[C * 8 / 32];
             switch (b) {
-              case 2: load_bits<C, 2>(src, w); dequant_chunk<C, 2>(w, sc, e + k * C); break;
-              case 3: load_bits<C, 3>(src, w); dequant_chunk<C, 3>(w, sc, e + k * C); break;
-              case 4: load_bits<C, 4>(src, w); dequant_chunk<C, 4>(w, sc, e + k * C); break;
-              default: load_bits<C, 8>(src, w); dequant_chunk<C, 8>(w, sc, e + k * C); break;
+              case 2: if (ct.cbulk) load_bits<C, 2>(stage_in + off, w); else load_bits<C, 2>(ct.codes + off, w);
+                      dequant_chunk<C, 2>(w, sc, e + k * C); break;
+              case 3: if (ct.cbulk) load_bits<C, 3>(stage_in + off, w); else load_bits<C, 3>(ct.codes + off, w);
+                      dequant_chunk<C, 3>(w, sc, e + k * C); break;
+              case 4: if (ct.cbulk) load_bits<C, 4>(stage_in + off, w); else load_bits<C, 4>(ct.codes + off, w);
+                      dequant_chunk<C, 4>(w, sc, e + k * C); break;
+              default: if (ct.cbulk) load_bits<C, 8>(stage_in + off, w); else load_bits<C, 8>(ct.codes + off, w);
+                       dequant_chunk<C, 8>(w, sc, e + k * C); break;
             }
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(xempty_bar(xb));
           xph[xb] ^= 1;
           xb ^= 1;
-          fwht_pair<C>(e, sXch, rl, hf, q);
+          fwht_pair<C>(e, lane_base, (uint32_t)(2 * D + xpar * D), hf, q);
+        xpar ^= 1;
 #pragma unroll
           for (int k = 0; k < 2; ++k)
 #pragma unroll
