@@ -818,7 +818,7 @@ static jolt_status run_random_fit(jolt_plan_s* p, const void* k_in, const void* 
   JOLT_TRY(launch_copy_out(d_out, p->d_rT_used, p->d_utp, nc, s));
   {
     ProfScope pe(JOLT_STAGE_EIG, s);
-    JOLT_TRY(launch_eigvecs(p->d_jobs_rand, nc, p->rmax_all, p->d_rT_used, s));
+    JOLT_TRY(launch_eigvecs_n(p->d_jobs_rand, nc, p->rmax_all, k, p->d_rT_used, s));
   }
   {
     // P = R^{-1} U_B[:, :r_T]: rows of P^T solve x R^T = u (backward)
@@ -981,7 +981,7 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
     if ((st = launch_copy_rt(h->d_out, p->d_rT_used, nc, s)) != JOLT_OK) return fail(st);
     {
       ProfScope pe(JOLT_STAGE_EIG, s);
-      if ((st = launch_eigvecs(p->d_jobs_spec, nc, p->rmax_all, p->d_rT_used, s)) != JOLT_OK) return fail(st);
+      if ((st = launch_eigvecs_n(p->d_jobs_spec, nc, p->rmax_all, p->nmin_max, p->d_rT_used, s)) != JOLT_OK) return fail(st);
     }
     if ((st = launch_ut_exact(fa, p->T, p->rmax_all, s)) != JOLT_OK) return fail(st);
     if ((st = launch_project_y(fa, p->T, p->rmax_all, p->lh_max, s)) != JOLT_OK) return fail(st);
@@ -994,7 +994,7 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   if ((st = launch_sum_chunks(p->d_fpart, p->fchunk, p->D * p->D + 1, nc, p->d_CY, nullptr, s)) != JOLT_OK) return fail(st);
   if ((st = launch_tridiag(p->d_jobs_fit, nc, p->D, s)) != JOLT_OK) return fail(st);
   if ((st = launch_bisect(p->d_jobs_fit, nc, p->D, s)) != JOLT_OK) return fail(st);
-  if ((st = launch_eigvecs(p->d_jobs_fit, nc, p->D, p->d_Dn, s)) != JOLT_OK) return fail(st);
+  if ((st = launch_eigvecs_n(p->d_jobs_fit, nc, p->D, p->D, p->d_Dn, s)) != JOLT_OK) return fail(st);
   if ((st = launch_core(fa, p->rmax_all, p->lh_max, s)) != JOLT_OK) return fail(st);
   ResidArgs ra{};
   ra.cells = p->d_cells; ra.cs = p->d_cs; ra.out = h->d_out; ra.M = p->d_M; ra.rmax_of = p->d_rmax;

@@ -26,6 +26,8 @@ jolt_status launch_tridiag_multi(const EighJob* jobs, int njobs, int nmax, doubl
                                  int* status, cudaStream_t s);
 jolt_status launch_bisect(const EighJob* jobs, int njobs, int nmax, cudaStream_t s);
 jolt_status launch_eigvecs(const EighJob* jobs, int njobs, int nvec_max, const int* nvec, cudaStream_t s);
+// Same, for matrices of size <= nmax (sizes the back-transformation blocks).
+jolt_status launch_eigvecs_n(const EighJob* jobs, int njobs, int nvec_max, int nmax, const int* nvec, cudaStream_t s);
 jolt_status launch_fgram_x(const CellDesc* cells, int ncells, int D, const float2* cs, int nchunk,
                            double* partial, cudaStream_t s);
 jolt_status launch_fgram_rows(const double* const* Y, const int* nrow_used, const int* rmax_of,

@@ -444,12 +444,12 @@ size_t eigh_smem_bytes(int nmax) { return (size_t)(6 * nmax + 32) * sizeof(doubl
 // ------------------------------------------- split eigensolver (big n) -----
 // For the token-mode matrices only the spectrum is needed before the
 // allocation and only the leading r_T eigenvectors after it, so the solver is
-// split: (1) Householder tridiagonalization, one block per matrix, leaving
-// the reflectors in A's columns and d, e, beta in work[0..3n); (2) every
-// eigenvalue by bisection on Sturm counts, one thread per eigenvalue;
-// (3) after the allocation, eigenvectors of the leading r eigenvalues by
-// inverse iteration on the tridiagonal matrix, back-transformed by the
-// reflectors, one warp per vector over many blocks.
+// split: (1) Householder tridiagonalization, leaving reflector k in row k of
+// A (entries k+1 .. n-1) and d, e, beta in work[0..3n); (2) every eigenvalue
+// by bisection on Sturm counts, one thread per eigenvalue; (3) after the
+// allocation, eigenvectors of the leading r eigenvalues by inverse iteration
+// on the tridiagonal matrix (one thread per vector), then the
+// back-transformation by the reflectors (a block per group of vectors).
 
 __global__ void __launch_bounds__(EIG_THREADS) k_tridiag(const EighJob* __restrict__ jobs) {
   const EighJob J = jobs[blockIdx.x];
@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(EIG_THREADS) k_tridiag(const EighJob* __restri
   const int lane = tid & 31, warp = tid >> 5, nwarp = nt >> 5;
   for (int k = 0; k + 2 < n; ++k) {
     const int m = n - k - 1;
-    for (int i = tid; i < m; i += nt) v[i] = A[(int64_t)(k + 1 + i) * n + k];
+    for (int i = tid; i < m; i += nt) v[i] = A[(int64_t)k * n + (k + 1 + i)];   // row k = column k
     __syncthreads();
     double s = 0.0;
     for (int i = 1 + tid; i < m; i += nt) s += v[i] * v[i];
@@ -501,10 +501,10 @@ __global__ void __launch_bounds__(EIG_THREADS) k_tridiag(const EighJob* __restri
     for (int i = warp; i < m; i += nwarp) {
       double* row = A + (int64_t)(k + 1 + i) * n + (k + 1);
       const double vi = v[i], wi = p[i];
-      for (int j = lane; j < m; j += 32) row[j] -= vi * p[j] + wi * v[j];
+      for (int j = lane; j < m; j += 32) row[j] = __dsub_rn(row[j], __dadd_rn(__dmul_rn(vi, p[j]), __dmul_rn(wi, v[j])));   // exactly symmetric
     }
     if (tid == 0) { dd[k] = A[(int64_t)k * n + k]; ee[k] = alpha; tau[k] = beta; }
-    for (int i = tid; i < m; i += nt) A[(int64_t)(k + 1 + i) * n + k] = v[i];
+    for (int i = tid; i < m; i += nt) A[(int64_t)k * n + (k + 1 + i)] = v[i];   // reflector k in row k
     __syncthreads();
   }
   if (tid == 0) {
@@ -633,7 +633,7 @@ __global__ void __launch_bounds__(EIG_THREADS) k_tridiag_multi(const EighJob* __
       // no contraction: entry (i, j) and (j, i) get the same two products
       for (int j = lane; j < m; j += 32)
         row[j] = __dsub_rn(__ldcg(row + j), __dadd_rn(__dmul_rn(vi, w[j]), __dmul_rn(wi, v[j])));
-      if (lane == 0) A[(int64_t)(k + 1 + i) * n + k] = v[i];
+      if (lane == 0) A[(int64_t)k * n + (k + 1 + i)] = v[i];   // reflector k in row k
     }
     if (c == 0 && tid == 0) { dd[k] = __ldcg(A + (int64_t)k * n + k); ee[k] = alpha; tau[k] = beta; }
     if (!job_barrier(cnt, (++nbar) * (unsigned)G, abort_flag, status)) return;
@@ -664,138 +664,240 @@ __device__ __forceinline__ int sturm_count(const double* d, const double* e, int
   return c;
 }
 
-// w[j] = j-th largest eigenvalue, one thread per j (the Sturm count is
-// monotone in x, so bisection converges to the eigenvalue of that rank).
+// w[j] = j-th largest eigenvalue by multisection on Sturm counts: one warp
+// per eigenvalue, its 32 lanes count at 32 interior points of the current
+// interval, and the interval shrinks to the sub-interval where the count
+// passes the eigenvalue's rank (the count is monotone in x), 33x per round
+// until no interior point is left.
 __global__ void __launch_bounds__(256) k_bisect(const EighJob* __restrict__ jobs) {
   const EighJob J = jobs[blockIdx.y];
   const int n = J.n;
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (n <= 0) return;
   extern __shared__ double sh[];
   double* d = sh;
   double* e = sh + n;
   for (int i = threadIdx.x; i < n; i += blockDim.x) { d[i] = J.work[i]; e[i] = J.work[n + i]; }
   __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (j >= n) return;
-  double lo = d[0], hi = d[0], emax = 0.0;
-  for (int i = 0; i < n; ++i) {
+  double lo = 1e300, hi = -1e300, emax = 0.0;
+  for (int i = lane; i < n; i += 32) {
     const double r = (i > 0 ? fabs(e[i - 1]) : 0.0) + (i + 1 < n ? fabs(e[i]) : 0.0);
     lo = fmin(lo, d[i] - r);
     hi = fmax(hi, d[i] + r);
     emax = fmax(emax, fabs(e[i]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fmin(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmax(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    emax = fmax(emax, __shfl_xor_sync(0xffffffffu, emax, o));
   }
   const double nrm = fmax(fabs(lo), fabs(hi));
   const double pivmin = fmax(1e-300, 2.2250738585072014e-308 * fmax(1.0, emax * emax));
   lo -= 4.0 * 2.220446049250313e-16 * nrm + pivmin;
   hi += 4.0 * 2.220446049250313e-16 * nrm + pivmin;
   const int m = n - 1 - j;          // rank among the ascending eigenvalues
-  for (int it = 0; it < 128; ++it) {
+  for (int round = 0; round < 64; ++round) {
     const double mid = 0.5 * (lo + hi);
     if (mid <= lo || mid >= hi) break;
-    if (sturm_count(d, e, n, mid, pivmin) > m) hi = mid;
-    else lo = mid;
+    const double x = lo + (hi - lo) * ((double)(lane + 1) / 33.0);
+    const bool above = (x > lo && x < hi) ? (sturm_count(d, e, n, x, pivmin) > m) : (x >= hi);
+    const unsigned bal = __ballot_sync(0xffffffffu, above);
+    const int f = bal ? (__ffs(bal) - 1) : 32;   // first point past the eigenvalue
+    const double xl = __shfl_sync(0xffffffffu, x, f > 0 ? f - 1 : 0);
+    const double xh = __shfl_sync(0xffffffffu, x, f < 32 ? f : 31);
+    const double nlo = (f > 0) ? fmax(lo, xl) : lo;
+    const double nhi = (f < 32) ? fmin(hi, xh) : hi;
+    if (nlo == lo && nhi == hi) break;           // no interior point moved the interval
+    lo = nlo;
+    hi = nhi;
   }
-  J.w[j] = 0.5 * (lo + hi);
+  if (lane == 0) J.w[j] = 0.5 * (lo + hi);
 }
 
-// Eigenvectors of the leading nvec[job] eigenvalues: inverse iteration on the
-// tridiagonal matrix (T - lam I factored once by Gaussian elimination with
-// partial pivoting, three solves from a fixed start vector), then the
-// back-transformation by the reflectors and the sign convention (largest
-// |entry| positive, first on ties). One warp per vector; lane 0 runs the
-// O(n) factorization and solves. Scratch per vector: z = Z[j*n ..] and
-// 5n doubles of J.F for the factors.
-__global__ void __launch_bounds__(256) k_eigvecs(const EighJob* __restrict__ jobs, const int* __restrict__ nvec) {
+// Eigenvectors of the leading nvec[job] eigenvalues, step 1: inverse
+// iteration on the tridiagonal matrix. T - lam I is factored once by Gaussian
+// elimination with partial pivoting (U with two superdiagonals, multipliers
+// and swap flags), then three solves from a fixed start vector, each followed
+// by normalization. One thread per vector, INV_W vectors per block; a block's
+// factors and iterate are interleaved by vector ([array][i][vector] in J.F,
+// [i][vector] in J.Z from the block's first vector on), so a warp's accesses
+// are contiguous. The recurrences carry their running values in registers;
+// the back substitution multiplies by the stored reciprocal pivots.
+constexpr int INV_W = 64;
+
+__global__ void __launch_bounds__(INV_W) k_invit(const EighJob* __restrict__ jobs, const int* __restrict__ nvec) {
   const EighJob J = jobs[blockIdx.y];
   const int n = J.n;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (n <= 0 || j >= min(nvec[blockIdx.y], n)) return;
+  if (n <= 0) return;
+  const int nv = min(nvec[blockIdx.y], n);
+  const int j0 = blockIdx.x * INV_W;
+  if (j0 >= nv) return;
+  const int W = min(INV_W, nv - j0), lane = threadIdx.x;
+  if (lane >= W) return;
+  const int j = j0 + lane;
   const double* d = J.work;
   const double* e = d + n;
-  const double* tau = e + n;
-  double* z = J.Z + (int64_t)j * n;
-  if (lane == 0) {
-    double* dg = J.F + (int64_t)j * 5 * n;   // diagonal of U
-    double* u1 = dg + n;                     // first superdiagonal of U
-    double* u2 = u1 + n;                     // second superdiagonal of U
-    double* ml = u2 + n;                     // multipliers
-    double* sw = ml + n;                     // 1.0 where rows i, i+1 were swapped
-    double nrm = 0.0;
-    for (int i = 0; i < n; ++i) nrm = fmax(nrm, fabs(d[i]) + fabs(e[i]) + (i ? fabs(e[i - 1]) : 0.0));
-    const double lam = J.w[j];
-    const double tiny = fmax(nrm, 1e-300) * 2.220446049250313e-16;
-    for (int i = 0; i < n; ++i) {
-      dg[i] = d[i] - lam;
-      u1[i] = (i + 1 < n) ? e[i] : 0.0;
-      u2[i] = 0.0;
+  double* F = J.F + (int64_t)j0 * 5 * n;
+  double* rdg = F;                          // 1 / pivot of U
+  double* u1 = F + (int64_t)n * W;          // first superdiagonal of U
+  double* u2 = F + (int64_t)2 * n * W;      // second superdiagonal of U
+  double* ml = F + (int64_t)3 * n * W;      // multipliers
+  double* sw = F + (int64_t)4 * n * W;      // 1.0 where rows i, i+1 were swapped
+  double* z = J.Z + (int64_t)j0 * n;
+  auto at = [&](int i) { return (int64_t)i * W + lane; };
+  double nrm = 0.0;
+  for (int i = 0; i < n; ++i) nrm = fmax(nrm, fabs(__ldg(d + i)) + fabs(__ldg(e + i)) + (i ? fabs(__ldg(e + i - 1)) : 0.0));
+  const double lam = J.w[j];
+  const double tiny = fmax(nrm, 1e-300) * 2.220446049250313e-16;
+  auto guard = [&](double g) { return (fabs(g) < tiny) ? ((g < 0.0) ? -tiny : tiny) : g; };
+  // factorization: row i is final after step i
+  double dg = __ldg(d) - lam, ui = (n > 1) ? __ldg(e) : 0.0;
+  double dn = (n > 1) ? __ldg(d + 1) - lam : 0.0, un = (n > 2) ? __ldg(e + 1) : 0.0;
+  for (int i = 0; i + 1 < n; ++i) {
+    const double sub = __ldg(e + i);      // row i+1, column i
+    double f, u2i = 0.0, swi;
+    if (fabs(dg) >= fabs(sub)) {
+      f = (dg != 0.0) ? sub / dg : 0.0;
+      swi = 0.0;
+      dn -= f * ui;
+    } else {
+      f = dg / sub;
+      swi = 1.0;
+      const double t = ui;
+      ui = dn;
+      dn = t - f * dn;
+      dg = sub;
+      if (i + 2 < n) {
+        u2i = un;
+        un = -f * un;
+      }
     }
+    rdg[at(i)] = 1.0 / guard(dg);
+    u1[at(i)] = ui;
+    u2[at(i)] = u2i;
+    ml[at(i)] = f;
+    sw[at(i)] = swi;
+    dg = dn;
+    ui = un;
+    dn = (i + 2 < n) ? __ldg(d + i + 2) - lam : 0.0;
+    un = (i + 3 < n) ? __ldg(e + i + 2) : 0.0;
+  }
+  rdg[at(n - 1)] = 1.0 / guard(dg);
+  u1[at(n - 1)] = 0.0;
+  u2[at(n - 1)] = 0.0;
+  double scale = 1.0;
+  for (int i = 0; i < n; ++i) z[at(i)] = 1.0 + 0.5 * sin(0.7 * (double)i + 0.3 * (double)j);
+  for (int iter = 0; iter < 3; ++iter) {
+    // forward: apply the row swaps and multipliers (and the last normalization)
+    double zc = scale * z[at(0)];
     for (int i = 0; i + 1 < n; ++i) {
-      const double sub = e[i];              // row i+1, column i
-      if (fabs(dg[i]) >= fabs(sub)) {
-        const double f = (dg[i] != 0.0) ? sub / dg[i] : 0.0;
-        ml[i] = f;
-        sw[i] = 0.0;
-        dg[i + 1] -= f * u1[i];
-      } else {
-        const double f = dg[i] / sub;
-        dg[i] = sub;
-        ml[i] = f;
-        sw[i] = 1.0;
-        const double t = u1[i];
-        u1[i] = dg[i + 1];
-        dg[i + 1] = t - f * dg[i + 1];
-        if (i + 2 < n) {
-          u2[i] = u1[i + 1];
-          u1[i + 1] = -f * u1[i + 1];
-        }
-      }
+      double zn = scale * z[at(i + 1)];
+      if (sw[at(i)] != 0.0) { const double t = zc; zc = zn; zn = t; }
+      zn -= ml[at(i)] * zc;
+      z[at(i)] = zc;
+      zc = zn;
     }
-    for (int i = 0; i < n; ++i)
-      if (fabs(dg[i]) < tiny) dg[i] = (dg[i] < 0.0) ? -tiny : tiny;
-    for (int i = 0; i < n; ++i) z[i] = 1.0 + 0.5 * sin(0.7 * (double)i + 0.3 * (double)j);
-    for (int iter = 0; iter < 3; ++iter) {
-      for (int i = 0; i + 1 < n; ++i) {
-        if (sw[i] != 0.0) { const double t = z[i]; z[i] = z[i + 1]; z[i + 1] = t; }
-        z[i + 1] -= ml[i] * z[i];
-      }
-      z[n - 1] /= dg[n - 1];
-      if (n >= 2) z[n - 2] = (z[n - 2] - u1[n - 2] * z[n - 1]) / dg[n - 2];
-      for (int i = n - 3; i >= 0; --i) z[i] = (z[i] - u1[i] * z[i + 1] - u2[i] * z[i + 2]) / dg[i];
-      double s = 0.0;
-      for (int i = 0; i < n; ++i) s += z[i] * z[i];
-      s = 1.0 / sqrt(s);
-      for (int i = 0; i < n; ++i) z[i] *= s;
+    // back substitution with U
+    double z1 = zc * rdg[at(n - 1)], z2 = 0.0;
+    z[at(n - 1)] = z1;
+    double ss = z1 * z1;
+    for (int i = n - 2; i >= 0; --i) {
+      const double zi = (z[at(i)] - u1[at(i)] * z1 - u2[at(i)] * z2) * rdg[at(i)];
+      z[at(i)] = zi;
+      ss += zi * zi;
+      z2 = z1;
+      z1 = zi;
     }
+    scale = 1.0 / sqrt(ss);
   }
-  __syncwarp();
-  // back-transformation z <- H_k z, k = n-3 .. 0; reflector k is column k of A
-  for (int k = n - 3; k >= 0; --k) {
-    const double beta = tau[k];
-    if (beta == 0.0) continue;
-    const int m = n - k - 1;
-    const double* vk = J.A + (int64_t)(k + 1) * n + k;
-    double acc = 0.0;
-    for (int i = lane; i < m; i += 32) acc += vk[(int64_t)i * n] * z[k + 1 + i];
-    acc = beta * warp_sum(acc);
-    for (int i = lane; i < m; i += 32) z[k + 1 + i] -= acc * vk[(int64_t)i * n];
-    __syncwarp();
+  for (int i = 0; i < n; ++i) z[at(i)] *= scale;
+}
+
+// Step 2: z <- H_0 H_1 ... H_{n-3} z for a block of up to vb vectors held in
+// shared memory; reflector k (row k of A) is read once per block, the next
+// one is fetched while the current one is applied. Then the sign convention
+// (largest |entry| positive, first on ties) and the rows of Vt.
+constexpr int BT_PRE = 8;     // reflector entries a thread prefetches (n <= 256 * 8)
+
+__global__ void __launch_bounds__(256) k_backtr(const EighJob* __restrict__ jobs, const int* __restrict__ nvec,
+                                              int vb) {
+  const EighJob J = jobs[blockIdx.y];
+  const int n = J.n;
+  if (n <= 0) return;
+  const int nv = min(nvec[blockIdx.y], n);
+  const int v0 = blockIdx.x * vb;
+  if (v0 >= nv) return;
+  const int nb = min(vb, nv - v0);
+  extern __shared__ double sh[];
+  double* Zs = sh;                        // nb x n
+  double* vbuf = sh + (int64_t)vb * n;    // 2 x n
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const double* tau = J.work + 2 * n;
+  // gather the block's vectors from the interleaved layout of k_invit
+  for (int vv = 0; vv < nb; ++vv) {
+    const int jj = v0 + vv, b0 = (jj / INV_W) * INV_W, W = min(INV_W, nv - b0), ln = jj - b0;
+    const double* z = J.Z + (int64_t)b0 * n;
+    for (int i = tid; i < n; i += 256) Zs[(int64_t)vv * n + i] = z[(int64_t)i * W + ln];
   }
-  double best = -1.0;
-  int bi = 0x7fffffff;
-  for (int i = lane; i < n; i += 32) {
-    const double a = fabs(z[i]);
-    if (a > best) { best = a; bi = i; }
-  }
+  auto load_v = [&](int k, double* r) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const double ob = __shfl_xor_sync(0xffffffffu, best, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-    if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+    for (int u = 0; u < BT_PRE; ++u) {
+      const int i = tid + 256 * u;
+      r[u] = (k >= 0 && i < n - k - 1) ? __ldg(J.A + (int64_t)k * n + k + 1 + i) : 0.0;
+    }
+  };
+  auto store_v = [&](int k, const double* r) {
+    double* dst = vbuf + (k & 1) * n;
+#pragma unroll
+    for (int u = 0; u < BT_PRE; ++u) {
+      const int i = tid + 256 * u;
+      if (k >= 0 && i < n - k - 1) dst[i] = r[u];
+    }
+  };
+  double pre[BT_PRE];
+  if (n >= 3) {
+    load_v(n - 3, pre);
+    store_v(n - 3, pre);
   }
-  const double sg = (z[bi] < 0.0) ? -1.0 : 1.0;
-  double* dst = J.Vt + (int64_t)j * n;
-  for (int i = lane; i < n; i += 32) dst[i] = sg * z[i];
+  __syncthreads();
+  for (int k = n - 3; k >= 0; --k) {
+    load_v(k - 1, pre);                   // next reflector, in flight during this one
+    const double beta = __ldg(tau + k);
+    const int m = n - k - 1;
+    if (beta != 0.0) {
+      const double* v = vbuf + (k & 1) * n;
+      for (int vv = warp; vv < nb; vv += 8) {
+        double* z = Zs + (int64_t)vv * n + (k + 1);
+        double acc = 0.0;
+        for (int i = lane; i < m; i += 32) acc += v[i] * z[i];
+        acc = beta * warp_sum(acc);
+        for (int i = lane; i < m; i += 32) z[i] -= acc * v[i];
+      }
+    }
+    store_v(k - 1, pre);
+    __syncthreads();
+  }
+  for (int vv = warp; vv < nb; vv += 8) {
+    const double* z = Zs + (int64_t)vv * n;
+    double best = -1.0;
+    int bi = 0x7fffffff;
+    for (int i = lane; i < n; i += 32) {
+      const double a = fabs(z[i]);
+      if (a > best) { best = a; bi = i; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+    }
+    const double sg = (z[bi] < 0.0) ? -1.0 : 1.0;
+    double* dst = J.Vt + (int64_t)(v0 + vv) * n;
+    for (int i = lane; i < n; i += 32) dst[i] = sg * z[i];
+  }
 }
 
 jolt_status launch_tridiag(const EighJob* jobs, int njobs, int nmax, cudaStream_t s) {
@@ -847,16 +949,26 @@ jolt_status launch_tridiag_multi(const EighJob* jobs, int njobs, int nmax, doubl
 jolt_status launch_bisect(const EighJob* jobs, int njobs, int nmax, cudaStream_t s) {
   const size_t smem = (size_t)(2 * nmax) * sizeof(double);
   { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_bisect, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
-  dim3 g((nmax + 255) / 256, njobs);
+  dim3 g((nmax + 7) / 8, njobs);          // a warp per eigenvalue, 8 per block
   k_bisect<<<g, 256, smem, s>>>(jobs);
   JOLT_LAUNCHED();
   return JOLT_OK;
 }
 
 jolt_status launch_eigvecs(const EighJob* jobs, int njobs, int nvec_max, const int* nvec, cudaStream_t s) {
-  if (nvec_max <= 0) return JOLT_OK;
-  dim3 g((nvec_max + 7) / 8, njobs);
-  k_eigvecs<<<g, 256, 0, s>>>(jobs, nvec);
+  return launch_eigvecs_n(jobs, njobs, nvec_max, 2048, nvec, s);
+}
+
+jolt_status launch_eigvecs_n(const EighJob* jobs, int njobs, int nvec_max, int nmax, const int* nvec, cudaStream_t s) {
+  if (nvec_max <= 0 || njobs <= 0) return JOLT_OK;
+  if (nmax > 256 * BT_PRE) { set_error("eigenvectors need n <= %d (n=%d)", 256 * BT_PRE, nmax); return JOLT_ERR_UNSUPPORTED_SHAPE; }
+  k_invit<<<dim3((nvec_max + INV_W - 1) / INV_W, njobs), INV_W, 0, s>>>(jobs, nvec);
+  JOLT_LAUNCHED();
+  // vectors per block: as many as 200 KB of shared memory hold, at most 32
+  const int vb = std::max(1, std::min(32, (int)((200 * 1024) / ((size_t)nmax * sizeof(double))) - 2));
+  const size_t smem = (size_t)(vb + 2) * nmax * sizeof(double);
+  { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_backtr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
+  k_backtr<<<dim3((nvec_max + vb - 1) / vb, njobs), 256, smem, s>>>(jobs, nvec, vb);
   JOLT_LAUNCHED();
   return JOLT_OK;
 }
