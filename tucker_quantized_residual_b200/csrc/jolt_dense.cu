@@ -306,91 +306,195 @@ jolt_status launch_tri_inverse(const double* R, double* Ri, double* RiT, int64_t
   return JOLT_OK;
 }
 
-// ------------------------------------------------- triangular products ------
+// ------------------------------------------------ fp64 tensor-core GEMM ----
+// C[m][n] = sum_k A[m][k] B[k][n] per cell (blockIdx.z) on the fp64 tensor
+// cores (mma.sync m8n8k4, fp64 in and out). Operands are strided views
+// (fp32 or fp64): A[m][k] = a[cell*a_cell + m*a_lm + k*a_lk], likewise B.
+// 64 x 64 output tiles, 4 warps of 32 x 32 (4 x 4 fragments), K in steps of
+// 16 through two shared-memory stages (row pitch 68 doubles: the fragment
+// loads of a warp hit distinct banks), the next stage fetched into registers
+// while the current one is multiplied. K range per tile: all of K (kmode 0),
+// k < n0 + 64 (kmode 1: C = B R^{-1} with R^{-1} upper), k >= n0 (kmode 2:
+// C = B R^{-T}). sym: only tiles with n0 >= m0, each written to (m, n) and
+// (n, m). The tile is staged through shared memory so the stores run along
+// whichever output index is contiguous.
+struct DgemmArgs {
+  const void* A; int a64; int64_t a_cell, a_lm, a_lk;
+  const void* B; int b64; int64_t b_cell, b_lk, b_ln;
+  const int* M_of; int M_fixed;
+  const int* K_of; int K_fixed;
+  int N, kmode, sym;
+  double* C64; int64_t c_cell, c_lm, c_ln;
+  uint16_t* C16; int64_t h_cell, h_lm, h_ln;
+};
+
+constexpr int DG_T = 64, DG_K = 16, DG_P = 68;
+
+__device__ __forceinline__ void dmma(double& c0, double& c1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(c0), "+d"(c1)
+               : "d"(a), "d"(b));
+}
+
+__device__ __forceinline__ double ld_op(const void* p, int is64, int64_t off) {
+  return is64 ? reinterpret_cast<const double*>(p)[off] : (double)reinterpret_cast<const float*>(p)[off];
+}
+
+__global__ void __launch_bounds__(128) k_dgemm(DgemmArgs g) {
+  __shared__ __align__(16) double sm[2 * 2 * DG_K * DG_P];   // [stage][A|B][k][m|n]; reused for the tile
+  const int cell = blockIdx.z;
+  int m0, n0;
+  if (g.sym) {
+    int b = blockIdx.x, ti = 0;
+    const int nt = (g.N + DG_T - 1) / DG_T;
+    while (ti < nt && b >= nt - ti) { b -= nt - ti; ++ti; }
+    if (ti >= nt) return;
+    m0 = ti * DG_T;
+    n0 = (ti + b) * DG_T;
+  } else {
+    m0 = blockIdx.x * DG_T;
+    n0 = blockIdx.y * DG_T;
+  }
+  const int M = g.M_of ? g.M_of[cell] : g.M_fixed;
+  const int K = g.K_of ? g.K_of[cell] : g.K_fixed;
+  if (m0 >= M || n0 >= g.N) return;
+  int k_lo = 0, k_hi = K;
+  if (g.kmode == 1) k_hi = min(K, n0 + DG_T);
+  if (g.kmode == 2) k_lo = (n0 / DG_K) * DG_K;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
+  const int gq = lane >> 2, tq = lane & 3;          // fragment row / column group
+  const void* A = g.A;
+  const void* B = g.B;
+  const int64_t aoff = (int64_t)cell * g.a_cell, boff = (int64_t)cell * g.b_cell;
+  const bool a_m_fast = g.a_lm == 1, b_n_fast = g.b_ln == 1;
+  double ra[8], rb[8];
+  auto fetch = [&](int kb) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = tid + 128 * u;
+      int mm, kk;
+      if (a_m_fast) { mm = e % DG_T; kk = e / DG_T; } else { kk = e % DG_K; mm = e / DG_K; }
+      const int gm = m0 + mm, gk = kb + kk;
+      ra[u] = (gm < M && gk < k_hi) ? ld_op(A, g.a64, aoff + (int64_t)gm * g.a_lm + (int64_t)gk * g.a_lk) : 0.0;
+      int nn, k2;
+      if (b_n_fast) { nn = e % DG_T; k2 = e / DG_T; } else { k2 = e % DG_K; nn = e / DG_K; }
+      const int gn = n0 + nn, gk2 = kb + k2;
+      rb[u] = (gn < g.N && gk2 < k_hi) ? ld_op(B, g.b64, boff + (int64_t)gk2 * g.b_lk + (int64_t)gn * g.b_ln) : 0.0;
+    }
+  };
+  auto stash = [&](int st) {
+    double* As = sm + st * 2 * DG_K * DG_P;
+    double* Bs = As + DG_K * DG_P;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = tid + 128 * u;
+      int mm, kk;
+      if (a_m_fast) { mm = e % DG_T; kk = e / DG_T; } else { kk = e % DG_K; mm = e / DG_K; }
+      As[kk * DG_P + mm] = ra[u];
+      int nn, k2;
+      if (b_n_fast) { nn = e % DG_T; k2 = e / DG_T; } else { k2 = e % DG_K; nn = e / DG_K; }
+      Bs[k2 * DG_P + nn] = rb[u];
+    }
+  };
+  double c[4][4][2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) c[i][j][0] = c[i][j][1] = 0.0;
+  int st = 0;
+  if (k_lo < k_hi) {
+    fetch(k_lo);
+    stash(0);
+  }
+  __syncthreads();
+  for (int kb = k_lo; kb < k_hi; kb += DG_K) {
+    const bool more = kb + DG_K < k_hi;
+    if (more) fetch(kb + DG_K);
+    const double* As = sm + st * 2 * DG_K * DG_P;
+    const double* Bs = As + DG_K * DG_P;
+#pragma unroll
+    for (int ks = 0; ks < DG_K / 4; ++ks) {
+      double a[4], b[4];
+#pragma unroll
+      for (int f = 0; f < 4; ++f) {
+        a[f] = As[(ks * 4 + tq) * DG_P + wm + f * 8 + gq];
+        b[f] = Bs[(ks * 4 + tq) * DG_P + wn + f * 8 + gq];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dmma(c[i][j][0], c[i][j][1], a[i], b[j]);
+    }
+    if (more) stash(st ^ 1);
+    __syncthreads();
+    st ^= 1;
+  }
+  // tile -> shared memory [m][n] (pitch 65), then strided stores
+  double* Ts = sm;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int v = 0; v < 2; ++v) Ts[(wm + i * 8 + gq) * (DG_T + 1) + wn + j * 8 + 2 * tq + v] = c[i][j][v];
+  __syncthreads();
+  auto store = [&](int r, int q, double v) {
+    if (g.C64) g.C64[(int64_t)cell * g.c_cell + (int64_t)r * g.c_lm + (int64_t)q * g.c_ln] = v;
+    if (g.C16) g.C16[(int64_t)cell * g.h_cell + (int64_t)r * g.h_lm + (int64_t)q * g.h_ln] = bf16_bits_from_f64(v);
+  };
+  const bool m_fast = (g.C64 ? g.c_lm : g.h_lm) == 1;
+  for (int e = tid; e < DG_T * DG_T; e += 128) {
+    int mm, nn;
+    if (m_fast) { nn = e / DG_T; mm = e % DG_T; } else { mm = e / DG_T; nn = e % DG_T; }
+    const int r = m0 + mm, q = n0 + nn;
+    if (r >= M || q >= g.N) continue;
+    const double v = Ts[mm * (DG_T + 1) + nn];
+    store(r, q, v);
+    if (g.sym && r != q) store(q, r, v);
+  }
+}
+
+static jolt_status launch_dgemm(const DgemmArgs& g, int M_max, int ncells, cudaStream_t s) {
+  if (M_max <= 0 || g.N <= 0 || ncells <= 0) return JOLT_OK;
+  const int mt = (M_max + DG_T - 1) / DG_T, nt = (g.N + DG_T - 1) / DG_T;
+  dim3 grid = g.sym ? dim3(nt * (nt + 1) / 2, 1, ncells) : dim3(mt, nt, ncells);
+  k_dgemm<<<grid, 128, 0, s>>>(g);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
 // Rows x of X (one cell per blockIdx.z) as products with the inverse:
 //   forward  (X R = B):    x_j = sum_{i <= j} b_i R^{-1}[i][j]
 //   backward (X R^T = B):  x_j = sum_{i >= j} b_i R^{-T}[i][j]
 // B: element (r, i) at B[r*ldb_r + i*ldb_c], fp32 or fp64 (b64 != 0).
 // Outputs (either may be null): X64[r*ld64_r + j*ld64_c] fp64 and
-// X16[r*ld16_r + j*ld16_c] bf16. 64 x 64 output tiles, 4 x 4 per thread on a
-// stride-16 lattice; the tile is staged through shared memory so the stores
-// run along whichever index is contiguous.
-
-constexpr int AP_T = 64, AP_K = 16;
-
-__global__ void __launch_bounds__(256) k_tri_apply(TrsmArgs a) {
-  __shared__ double sm[AP_T * (AP_T + 1)];
-  double* Bs = sm;                          // [AP_K][AP_T]   (i, r)
-  double* Qs = sm + AP_K * AP_T;            // [AP_K][AP_T]   (i, j)
-  const int cell = blockIdx.z;
-  const int rows = a.rows_of ? a.rows_of[cell] : a.rows_fixed;
-  const int r0 = blockIdx.x * AP_T, j0 = blockIdx.y * AP_T;
-  if (r0 >= rows) return;
-  const int k = a.k;
-  if (j0 >= k) return;
-  const double* Q = (a.backward ? a.RinvT : a.Rinv) + (int64_t)cell * a.r_cell;
-  const int i_lo = a.backward ? (j0 / AP_K) * AP_K : 0;
-  const int i_hi = a.backward ? k : min(k, j0 + AP_T);
-  const int t = threadIdx.x, ty = t / 16, tx = t % 16;
-  const bool b_rowmajor = a.ldb_c == 1;
-  const int64_t boff = (int64_t)cell * a.b_cell;
-  double acc[4][4] = {};
-  for (int ib = i_lo; ib < i_hi; ib += AP_K) {
-    __syncthreads();
-#pragma unroll
-    for (int u = 0; u < (AP_K * AP_T) / 256; ++u) {
-      const int e = t + 256 * u;
-      int ii, rr;
-      if (b_rowmajor) { rr = e / AP_K; ii = e % AP_K; }
-      else { ii = e / AP_T; rr = e % AP_T; }
-      const int i = ib + ii, r = r0 + rr;
-      double v = 0.0;
-      if (i < k && r < rows) {
-        const int64_t off = boff + (int64_t)r * a.ldb_r + (int64_t)i * a.ldb_c;
-        v = a.b64 ? reinterpret_cast<const double*>(a.B)[off] : (double)reinterpret_cast<const float*>(a.B)[off];
-      }
-      Bs[ii * AP_T + rr] = v;
-      const int qi = e / AP_T, qj = e % AP_T;
-      const int iq = ib + qi, jq = j0 + qj;
-      Qs[qi * AP_T + qj] = (iq < k && jq < k) ? Q[(int64_t)iq * k + jq] : 0.0;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int ii = 0; ii < AP_K; ++ii) {
-      double x[4], y[4];
-#pragma unroll
-      for (int p = 0; p < 4; ++p) { x[p] = Bs[ii * AP_T + ty + 16 * p]; y[p] = Qs[ii * AP_T + tx + 16 * p]; }
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[p][q] = fma(x[p], y[q], acc[p][q]);
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int p = 0; p < 4; ++p)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) sm[(ty + 16 * p) * (AP_T + 1) + tx + 16 * q] = acc[p][q];
-  __syncthreads();
-  const bool trans = (a.X16 && a.ld16_r == 1) || (a.X64 && a.ld64_r == 1);
-  for (int e = t; e < AP_T * AP_T; e += 256) {
-    int rr, jj;
-    if (trans) { jj = e / AP_T; rr = e % AP_T; }
-    else { rr = e / AP_T; jj = e % AP_T; }
-    const int r = r0 + rr, j = j0 + jj;
-    if (r >= rows || j >= k) continue;
-    const double v = sm[rr * (AP_T + 1) + jj];
-    if (a.X64) a.X64[(int64_t)cell * a.x64_cell + (int64_t)r * a.ld64_r + (int64_t)j * a.ld64_c] = v;
-    if (a.X16) a.X16[(int64_t)cell * a.x16_cell + (int64_t)r * a.ld16_r + (int64_t)j * a.ld16_c] = bf16_bits_from_f64(v);
-  }
+// X16[r*ld16_r + j*ld16_c] bf16.
+jolt_status launch_tri_apply(const TrsmArgs& a, int rows_max, int ncells, cudaStream_t s) {
+  DgemmArgs g{};
+  g.A = a.B; g.a64 = a.b64; g.a_cell = a.b_cell; g.a_lm = a.ldb_r; g.a_lk = a.ldb_c;
+  g.B = a.backward ? a.RinvT : a.Rinv; g.b64 = 1; g.b_cell = a.r_cell; g.b_lk = a.k; g.b_ln = 1;
+  g.M_of = a.rows_of; g.M_fixed = a.rows_fixed;
+  g.K_of = nullptr; g.K_fixed = a.k;
+  g.N = a.k; g.kmode = a.backward ? 2 : 1; g.sym = 0;
+  g.C64 = a.X64; g.c_cell = a.x64_cell; g.c_lm = a.ld64_r; g.c_ln = a.ld64_c;
+  g.C16 = a.X16; g.h_cell = a.x16_cell; g.h_lm = a.ld16_r; g.h_ln = a.ld16_c;
+  return launch_dgemm(g, rows_max, ncells, s);
 }
 
-jolt_status launch_tri_apply(const TrsmArgs& a, int rows_max, int ncells, cudaStream_t s) {
-  if (rows_max <= 0 || a.k <= 0) return JOLT_OK;
-  dim3 g((rows_max + AP_T - 1) / AP_T, (a.k + AP_T - 1) / AP_T, ncells);
-  k_tri_apply<<<g, 256, 0, s>>>(a);
-  JOLT_LAUNCHED();
-  return JOLT_OK;
+// C = A^T A for A = [rows_of[cell]] x k fp32 (row-major, cell stride a_cell),
+// C k x k fp64 (cell stride c_cell), exactly symmetric.
+jolt_status launch_gram_cols(const float* A, int64_t a_cell, const int* rows_of, int k, double* C, int64_t c_cell,
+                             int ncells, cudaStream_t s) {
+  DgemmArgs g{};
+  g.A = A; g.a64 = 0; g.a_cell = a_cell; g.a_lm = 1; g.a_lk = k;
+  g.B = A; g.b64 = 0; g.b_cell = a_cell; g.b_lk = k; g.b_ln = 1;
+  g.M_of = nullptr; g.M_fixed = k;
+  g.K_of = rows_of; g.K_fixed = 0;
+  g.N = k; g.kmode = 0; g.sym = 1;
+  g.C64 = C; g.c_cell = c_cell; g.c_lm = k; g.c_ln = 1;
+  g.C16 = nullptr;
+  return launch_dgemm(g, k, ncells, s);
 }
 
 }  // namespace jolt

@@ -664,11 +664,13 @@ __device__ __forceinline__ int sturm_count(const double* d, const double* e, int
   return c;
 }
 
-// w[j] = j-th largest eigenvalue by multisection on Sturm counts: one warp
-// per eigenvalue, its 32 lanes count at 32 interior points of the current
+// w[j] = j-th largest eigenvalue by multisection on Sturm counts: BIS_L
+// lanes per eigenvalue count at BIS_L interior points of the current
 // interval, and the interval shrinks to the sub-interval where the count
-// passes the eigenvalue's rank (the count is monotone in x), 33x per round
-// until no interior point is left.
+// passes the eigenvalue's rank (the count is monotone in x), (BIS_L + 1)x per
+// round until no interior point is left.
+constexpr int BIS_L = 8;
+
 __global__ void __launch_bounds__(256) k_bisect(const EighJob* __restrict__ jobs) {
   const EighJob J = jobs[blockIdx.y];
   const int n = J.n;
@@ -678,9 +680,10 @@ __global__ void __launch_bounds__(256) k_bisect(const EighJob* __restrict__ jobs
   double* e = sh + n;
   for (int i = threadIdx.x; i < n; i += blockDim.x) { d[i] = J.work[i]; e[i] = J.work[n + i]; }
   __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (j >= n) return;
+  const int lane = threadIdx.x & 31, sub = lane & (BIS_L - 1), base = lane & ~(BIS_L - 1);
+  const int j = blockIdx.x * (blockDim.x / BIS_L) + threadIdx.x / BIS_L;
+  const bool act = j < n;
+  // Gershgorin bounds (every lane of the warp takes part)
   double lo = 1e300, hi = -1e300, emax = 0.0;
   for (int i = lane; i < n; i += 32) {
     const double r = (i > 0 ? fabs(e[i - 1]) : 0.0) + (i + 1 < n ? fabs(e[i]) : 0.0);
@@ -698,23 +701,27 @@ __global__ void __launch_bounds__(256) k_bisect(const EighJob* __restrict__ jobs
   const double pivmin = fmax(1e-300, 2.2250738585072014e-308 * fmax(1.0, emax * emax));
   lo -= 4.0 * 2.220446049250313e-16 * nrm + pivmin;
   hi += 4.0 * 2.220446049250313e-16 * nrm + pivmin;
-  const int m = n - 1 - j;          // rank among the ascending eigenvalues
-  for (int round = 0; round < 64; ++round) {
+  const int m = n - 1 - (act ? j : 0);    // rank among the ascending eigenvalues
+  bool done = !act;
+  for (int round = 0; round < 96; ++round) {
     const double mid = 0.5 * (lo + hi);
-    if (mid <= lo || mid >= hi) break;
-    const double x = lo + (hi - lo) * ((double)(lane + 1) / 33.0);
-    const bool above = (x > lo && x < hi) ? (sturm_count(d, e, n, x, pivmin) > m) : (x >= hi);
-    const unsigned bal = __ballot_sync(0xffffffffu, above);
-    const int f = bal ? (__ffs(bal) - 1) : 32;   // first point past the eigenvalue
-    const double xl = __shfl_sync(0xffffffffu, x, f > 0 ? f - 1 : 0);
-    const double xh = __shfl_sync(0xffffffffu, x, f < 32 ? f : 31);
-    const double nlo = (f > 0) ? fmax(lo, xl) : lo;
-    const double nhi = (f < 32) ? fmin(hi, xh) : hi;
-    if (nlo == lo && nhi == hi) break;           // no interior point moved the interval
-    lo = nlo;
-    hi = nhi;
+    if (mid <= lo || mid >= hi) done = true;
+    if (__all_sync(0xffffffffu, done)) break;
+    const double x = lo + (hi - lo) * ((double)(sub + 1) / (double)(BIS_L + 1));
+    const bool above = (!done && x > lo && x < hi) ? (sturm_count(d, e, n, x, pivmin) > m) : (x >= hi);
+    const unsigned bal = (__ballot_sync(0xffffffffu, above) >> base) & ((1u << BIS_L) - 1u);
+    const int f = bal ? (__ffs(bal) - 1) : BIS_L;   // first point past the eigenvalue
+    const double xl = __shfl_sync(0xffffffffu, x, base + (f > 0 ? f - 1 : 0));
+    const double xh = __shfl_sync(0xffffffffu, x, base + (f < BIS_L ? f : BIS_L - 1));
+    if (!done) {
+      const double nlo = (f > 0) ? fmax(lo, xl) : lo;
+      const double nhi = (f < BIS_L) ? fmin(hi, xh) : hi;
+      if (nlo == lo && nhi == hi) done = true;     // no interior point moved the interval
+      lo = nlo;
+      hi = nhi;
+    }
   }
-  if (lane == 0) J.w[j] = 0.5 * (lo + hi);
+  if (act && sub == 0) J.w[j] = 0.5 * (lo + hi);
 }
 
 // Eigenvectors of the leading nvec[job] eigenvalues, step 1: inverse
@@ -949,7 +956,7 @@ jolt_status launch_tridiag_multi(const EighJob* jobs, int njobs, int nmax, doubl
 jolt_status launch_bisect(const EighJob* jobs, int njobs, int nmax, cudaStream_t s) {
   const size_t smem = (size_t)(2 * nmax) * sizeof(double);
   { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_bisect, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
-  dim3 g((nmax + 7) / 8, njobs);          // a warp per eigenvalue, 8 per block
+  dim3 g((nmax + 256 / BIS_L - 1) / (256 / BIS_L), njobs);   // BIS_L lanes per eigenvalue
   k_bisect<<<g, 256, smem, s>>>(jobs);
   JOLT_LAUNCHED();
   return JOLT_OK;

@@ -113,23 +113,35 @@ jolt_status launch_umma(const umma::Maps& maps, const umma::Problem& p, cudaStre
 // --------------------------------------------------- bf16 working copies ---
 // dst (contiguous [B][L][H][T][D] bf16) = bf16_rne(x), x the compression
 // target: un-RoPE'd keys in fp32 (rope != 0) or the stored values.
-__global__ void k_make_xb(const void* __restrict__ src, int f32, int rope, const float2* __restrict__ cs,
-                          int B, int L, int H, int T, int D, int64_t sb, int64_t sl, int64_t sh, int64_t st,
-                          uint16_t* __restrict__ dst) {
+// One thread per (token, 8 rotation pairs) of one (b, l, h) row block
+// (blockIdx.y); vec != 0: bf16 input with 16-byte aligned rows, read as
+// 8-element vectors, and the cos/sin pairs as float4.
+__global__ void __launch_bounds__(256) k_make_xb(const void* __restrict__ src, int f32, int rope, int vec,
+                                                 const float2* __restrict__ cs, int L, int H, int T, int D,
+                                                 int64_t sb, int64_t sl, int64_t sh, int64_t st,
+                                                 uint16_t* __restrict__ dst) {
   const int half = D / 2;
-  const int64_t rows = (int64_t)B * L * H * T;
   const int per_row = half / 8;              // 8-pair blocks per row
-  const int64_t n = rows * per_row;
-  for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < n; k += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = k / per_row;
-    const int i0 = (int)(k % per_row) * 8;
-    int64_t r = row;
-    const int t = (int)(r % T); r /= T;
-    const int h = (int)(r % H); r /= H;
-    const int l = (int)(r % L); r /= L;
-    const int b = (int)r;
-    const int64_t off = (int64_t)b * sb + (int64_t)l * sl + (int64_t)h * sh + (int64_t)t * st;
-    float y0[8], y1[8];
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= T * per_row) return;
+  const int t = e / per_row, i0 = (e - t * per_row) * 8;
+  const int blh = blockIdx.y;
+  const int h = blh % H, l = (blh / H) % L, b = blh / (H * L);
+  const int64_t off = (int64_t)b * sb + (int64_t)l * sl + (int64_t)h * sh + (int64_t)t * st;
+  float y0[8], y1[8];
+  if (vec) {
+    const uint16_t* p = reinterpret_cast<const uint16_t*>(src) + off;
+    const uint4 w0 = *reinterpret_cast<const uint4*>(p + i0);
+    const uint4 w1 = *reinterpret_cast<const uint4*>(p + half + i0);
+    const uint32_t a0[4] = {w0.x, w0.y, w0.z, w0.w}, a1[4] = {w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      y0[2 * j] = __uint_as_float(a0[j] << 16);
+      y0[2 * j + 1] = __uint_as_float(a0[j] & 0xFFFF0000u);
+      y1[2 * j] = __uint_as_float(a1[j] << 16);
+      y1[2 * j + 1] = __uint_as_float(a1[j] & 0xFFFF0000u);
+    }
+  } else {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (f32) {
@@ -140,30 +152,36 @@ __global__ void k_make_xb(const void* __restrict__ src, int f32, int rope, const
         y1[j] = bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(src)[off + half + i0 + j]);
       }
     }
-    uint16_t o0[8], o1[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float a = y0[j], c = y1[j];
-      if (rope) {
-        const float2 q = cs[(int64_t)t * half + i0 + j];
-        a = __fadd_rn(__fmul_rn(y0[j], q.x), __fmul_rn(y1[j], q.y));
-        c = __fsub_rn(__fmul_rn(y1[j], q.x), __fmul_rn(y0[j], q.y));
-      }
-      o0[j] = bf16_bits_from_f32(a);
-      o1[j] = bf16_bits_from_f32(c);
-    }
-    uint16_t* d = dst + row * D;
-    *reinterpret_cast<uint4*>(d + i0) = *reinterpret_cast<uint4*>(o0);
-    *reinterpret_cast<uint4*>(d + half + i0) = *reinterpret_cast<uint4*>(o1);
   }
+  uint32_t o0[4], o1[4];
+  const float4* cs4 = rope ? reinterpret_cast<const float4*>(cs + (int64_t)t * half + i0) : nullptr;
+#pragma unroll
+  for (int j = 0; j < 8; j += 2) {
+    float a[2] = {y0[j], y0[j + 1]}, c[2] = {y1[j], y1[j + 1]};
+    if (rope) {
+      const float4 q = cs4[j / 2];
+      const float cc[2] = {q.x, q.z}, ss[2] = {q.y, q.w};
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        a[u] = __fadd_rn(__fmul_rn(y0[j + u], cc[u]), __fmul_rn(y1[j + u], ss[u]));
+        c[u] = __fsub_rn(__fmul_rn(y1[j + u], cc[u]), __fmul_rn(y0[j + u], ss[u]));
+      }
+    }
+    o0[j / 2] = (uint32_t)bf16_bits_from_f32(a[0]) | ((uint32_t)bf16_bits_from_f32(a[1]) << 16);
+    o1[j / 2] = (uint32_t)bf16_bits_from_f32(c[0]) | ((uint32_t)bf16_bits_from_f32(c[1]) << 16);
+  }
+  uint16_t* d = dst + ((int64_t)blh * T + t) * D;
+  *reinterpret_cast<uint4*>(d + i0) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+  *reinterpret_cast<uint4*>(d + half + i0) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
 }
 
 jolt_status launch_make_xb(const void* src, int f32, int rope, const float2* cs, int B, int L, int H, int T,
                            int D, int64_t sb, int64_t sl, int64_t sh, int64_t st, uint16_t* dst,
                            cudaStream_t s) {
-  const int64_t n = (int64_t)B * L * H * T * (D / 16);
-  const int grid = (int)std::min<int64_t>((n + 255) / 256, 148 * 16);
-  k_make_xb<<<grid, 256, 0, s>>>(src, f32, rope, cs, B, L, H, T, D, sb, sl, sh, st, dst);
+  if ((int64_t)B * L * H > 65535) { set_error("too many (b, l, h) rows for the copy kernel"); return JOLT_ERR_UNSUPPORTED_SHAPE; }
+  const int vec = !f32 && ((sb | sl | sh | st) % 8 == 0) && (reinterpret_cast<uintptr_t>(src) % 16 == 0);
+  dim3 g((T * (D / 16) + 255) / 256, B * L * H);
+  k_make_xb<<<g, 256, 0, s>>>(src, f32, rope, vec, cs, L, H, T, D, sb, sl, sh, st, dst);
   JOLT_LAUNCHED();
   return JOLT_OK;
 }
@@ -199,62 +217,6 @@ jolt_status launch_omega(uint16_t* wt, int ncells, int k, int ld, const int* Nc,
   const int64_t n4 = (int64_t)k * ld / 4;
   dim3 g((unsigned)std::min<int64_t>((n4 + 255) / 256, 1024), ncells);
   k_omega<<<g, 256, 0, s>>>(wt, ncells, k, ld, Nc, seq, cis, seed);
-  JOLT_LAUNCHED();
-  return JOLT_OK;
-}
-
-// -------------------------------------------------- fp64 Gram of columns ---
-// C[cell][i][j] = sum_n A[cell][n][i] A[cell][n][j], A fp32 row-major [rows][k]
-__global__ void __launch_bounds__(256) k_gram_cols(const float* __restrict__ A, int64_t a_cell, const int* __restrict__ rows_of,
-                                                   int k, double* __restrict__ C, int64_t c_cell) {
-  constexpr int TB = 64, KB = 16;
-  __shared__ double As[KB][TB + 1];
-  __shared__ double Bs[KB][TB + 1];
-  const int cell = blockIdx.y;
-  const int nrows = rows_of[cell];
-  const float* a = A + (int64_t)cell * a_cell;
-  const int nt = (k + TB - 1) / TB;
-  int b = blockIdx.x, ti = 0;
-  while (ti < nt && b >= nt - ti) { b -= nt - ti; ++ti; }
-  if (ti >= nt) return;
-  const int tj = ti + b;
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
-  double acc[4][4] = {};
-  for (int r0 = 0; r0 < nrows; r0 += KB) {
-    for (int e = threadIdx.x; e < KB * TB; e += blockDim.x) {
-      const int kk = e / TB, ii = e % TB;
-      const int r = r0 + kk, ia = ti * TB + ii, ib = tj * TB + ii;
-      As[kk][ii] = (r < nrows && ia < k) ? (double)a[(int64_t)r * k + ia] : 0.0;
-      Bs[kk][ii] = (r < nrows && ib < k) ? (double)a[(int64_t)r * k + ib] : 0.0;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < KB; ++kk) {
-      double x[4], y[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) { x[i] = As[kk][ty * 4 + i]; y[i] = Bs[kk][tx * 4 + i]; }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fma(x[i], y[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-  double* c = C + (int64_t)cell * c_cell;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int r = ti * TB + ty * 4 + i, q = tj * TB + tx * 4 + j;
-      if (r < k && q < k) { c[(int64_t)r * k + q] = acc[i][j]; c[(int64_t)q * k + r] = acc[i][j]; }
-    }
-}
-
-jolt_status launch_gram_cols(const float* A, int64_t a_cell, const int* rows_of, int k, double* C, int64_t c_cell,
-                             int ncells, cudaStream_t s) {
-  const int nt = (k + 63) / 64;
-  dim3 g(nt * (nt + 1) / 2, ncells);
-  k_gram_cols<<<g, 256, 0, s>>>(A, a_cell, rows_of, k, C, c_cell);
   JOLT_LAUNCHED();
   return JOLT_OK;
 }
