@@ -81,6 +81,12 @@ __device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Two fp32 values rounded to bf16 (nearest, ties to even), lo in the low half.
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(bar)
@@ -229,29 +235,33 @@ __device__ __forceinline__ void fwht_pair(float* e, uint32_t lane_base, uint32_t
 // clamp(rint(fl32(r / sc))). The quotient is taken as r * fl32(1/sc) and
 // replaced by the correctly rounded one wherever the product lies within
 // 1e-4 of a rounding boundary (it differs from the quotient by at most
-// 128 * 2^-23 < 2e-5 there), so the codes equal the divided ones.
+// 128 * 2^-23 < 2e-5 there), so the codes equal the divided ones. Rounding
+// to the nearest integer (ties to even) is the fp32 addition of
+// 1.5 * 2^23 + 2^(b-1), whose low b mantissa bits then hold u = code + 2^(b-1),
+// packed LSB first.
 template <int C, int B>
 __device__ __forceinline__ void quant_chunk(const float* r, float sc, uint32_t* w) {
   constexpr int NW = (C * B + 31) / 32;
+  constexpr uint32_t mask = (1u << B) - 1u;
+  // 1.5 * 2^23 + 2^(b-1): the sum's low b bits are u = rint(y) + 2^(b-1)
+  constexpr float magic = 12582912.0f + (float)(1 << (B - 1));
   const float qm = (float)((1 << (B - 1)) - 1);
 #pragma unroll
   for (int i = 0; i < NW; ++i) w[i] = 0u;
-  uint32_t need = 0u;
   if (sc > 0.0f) {
     const float inv = __frcp_rn(sc);
+    uint32_t need = 0u;
 #pragma unroll
     for (int i = 0; i < C; ++i) {
-      const float y = __fmul_rn(r[i], inv);
-      float qf = rintf(y);
-      if (!(0.5f - fabsf(y - qf) >= 1e-4f)) need |= 1u << i;
-      qf = fminf(fmaxf(qf, -qm), qm);
-      const uint32_t u = (uint32_t)((int)qf + (1 << (B - 1)));
+      const float y = fminf(fmaxf(__fmul_rn(r[i], inv), -qm), qm);
+      const float t = __fadd_rn(y, magic);
+      if (!(0.5f - fabsf(__fsub_rn(y, __fsub_rn(t, magic))) >= 1e-4f)) need |= 1u << i;
+      const uint32_t u = __float_as_uint(t) & mask;
       const int bit = i * B, wi = bit >> 5, sh = bit & 31;
       w[wi] |= u << sh;
       if (sh + B > 32) w[wi + 1] |= u >> (32 - sh);
     }
     if (need) {
-      constexpr uint32_t mask = (1u << B) - 1u;
 #pragma unroll
       for (int i = 0; i < C; ++i) {
         if (!((need >> i) & 1u)) continue;
@@ -275,14 +285,18 @@ __device__ __forceinline__ void quant_chunk(const float* r, float sc, uint32_t* 
 
 template <int C, int B>
 __device__ __forceinline__ void dequant_chunk(const uint32_t* w, float sc, float* v) {
+  // u in the low mantissa bits of 2^23 gives 2^23 + u exactly; subtracting
+  // 2^23 + 2^(b-1) leaves the code as a float
   constexpr uint32_t mask = (1u << B) - 1u;
+  constexpr float off = 8388608.0f + (float)(1 << (B - 1));
 #pragma unroll
   for (int i = 0; i < C; ++i) {
     const int bit = i * B, wi = bit >> 5, sh = bit & 31;
-    uint32_t u = w[wi] >> sh;
-    if (sh + B > 32) u |= w[wi + 1] << (32 - sh);
-    const int q = (int)(u & mask) - (1 << (B - 1));
-    v[i] = __fmul_rn((float)q, sc);
+    uint32_t u;
+    if (sh + B <= 32) u = (w[wi] >> sh) & mask;
+    else u = __funnelshift_r(w[wi], w[wi + 1], sh) & mask;
+    const float q = __fsub_rn(__uint_as_float(0x4B000000u | u), off);
+    v[i] = __fmul_rn(q, sc);
   }
 }
 
@@ -290,7 +304,12 @@ __device__ __forceinline__ void dequant_chunk(const uint32_t* w, float sc, float
 // units when C = 32 (4-byte aligned offsets), 16-bit units otherwise.
 template <int C, int B>
 __device__ __forceinline__ void store_bits(uint8_t* p, const uint32_t* w) {
-  if constexpr (C == 32) {
+  if constexpr (C == 32 && B == 2) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+  } else if constexpr (C == 32 && (B == 4 || B == 8)) {
+#pragma unroll
+    for (int i = 0; i < B; i += 4) *reinterpret_cast<uint4*>(p + 4 * i) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
+  } else if constexpr (C == 32) {
     uint32_t* d = reinterpret_cast<uint32_t*>(p);
 #pragma unroll
     for (int i = 0; i < B; ++i) d[i] = w[i];
@@ -302,7 +321,16 @@ __device__ __forceinline__ void store_bits(uint8_t* p, const uint32_t* w) {
 }
 template <int C, int B>
 __device__ __forceinline__ void load_bits(const uint8_t* p, uint32_t* w) {
-  if constexpr (C == 32) {
+  if constexpr (C == 32 && B == 2) {
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    w[0] = x.x; w[1] = x.y;
+  } else if constexpr (C == 32 && (B == 4 || B == 8)) {
+#pragma unroll
+    for (int i = 0; i < B; i += 4) {
+      const uint4 x = *reinterpret_cast<const uint4*>(p + 4 * i);
+      w[i] = x.x; w[i + 1] = x.y; w[i + 2] = x.z; w[i + 3] = x.w;
+    }
+  } else if constexpr (C == 32) {
     const uint32_t* s = reinterpret_cast<const uint32_t*>(p);
 #pragma unroll
     for (int i = 0; i < B; ++i) w[i] = s[i];
@@ -394,6 +422,12 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
   fence_after();
   const uint32_t tmem = *tmem_slot;
   const int ntiles = a.ncells * a.ntile_t * a.lhmax;
+  // Work is dealt out by token tile: a CTA takes every layer-head tile of one
+  // 128-token tile in a row (so U_T^ slices and RoPE rows are reused from the
+  // caches), and token tiles go round-robin over the CTAs (so cells without a
+  // residual, skipped when compressing, do not unbalance the CTAs).
+  const int ngroups = a.ncells * a.ntile_t;
+  (void)ntiles;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -405,7 +439,8 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
       bool xissued[2] = {false, false};
       for (int s = 0; s < SSTAGES; ++s) issued[s] = false;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int tile = blockIdx.x * a.lhmax; tile < ngroups * a.lhmax && ok;
+           tile += (tile % a.lhmax == a.lhmax - 1) ? 1 + (gridDim.x - 1) * a.lhmax : 1) {
         int cell, t0, lh;
         CellDesc c;
         CellOut o;
@@ -463,7 +498,8 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
       uint32_t ph = 0, aph[2] = {0, 0};
       const uint32_t idesc = idesc_bf16(D, 1, 0);
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int tile = blockIdx.x * a.lhmax; tile < ngroups * a.lhmax && ok;
+           tile += (tile % a.lhmax == a.lhmax - 1) ? 1 + (gridDim.x - 1) * a.lhmax : 1) {
         int cell, t0, lh;
         CellDesc c;
         CellOut o;
@@ -499,7 +535,8 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
     int acc = 0, xb = 0, xpar = 0;
     uint32_t aph[2] = {0, 0}, xph[2] = {0, 0};
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    for (int tile = blockIdx.x * a.lhmax; tile < ngroups * a.lhmax;
+         tile += (tile % a.lhmax == a.lhmax - 1) ? 1 + (gridDim.x - 1) * a.lhmax : 1) {
       int cell, t0, lh;
       CellDesc c;
       CellOut o;
@@ -700,10 +737,10 @@ __global__ void __launch_bounds__(STHREADS, 1) k_stream(const __grid_constant__ 
             for (int u = 0; u < C / 8; ++u) {
               const float* s = e + k * C + 8 * u;
               uint4 w;
-              w.x = (uint32_t)bf16_bits_from_f32(s[0]) | ((uint32_t)bf16_bits_from_f32(s[1]) << 16);
-              w.y = (uint32_t)bf16_bits_from_f32(s[2]) | ((uint32_t)bf16_bits_from_f32(s[3]) << 16);
-              w.z = (uint32_t)bf16_bits_from_f32(s[4]) | ((uint32_t)bf16_bits_from_f32(s[5]) << 16);
-              w.w = (uint32_t)bf16_bits_from_f32(s[6]) | ((uint32_t)bf16_bits_from_f32(s[7]) << 16);
+              w.x = bf16x2_bits(s[0], s[1]);
+              w.y = bf16x2_bits(s[2], s[3]);
+              w.z = bf16x2_bits(s[4], s[5]);
+              w.w = bf16x2_bits(s[6], s[7]);
               *reinterpret_cast<uint4*>(base + k * (D / 2) + hf * C + 8 * u) = w;
             }
         }
