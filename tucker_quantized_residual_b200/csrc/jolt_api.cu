@@ -174,6 +174,7 @@ struct jolt_plan_s {
   // randomized mode (Section 3.1): sketch width k = q + p rounded up to 16,
   // GEMM tile width BN, padded extents, working buffers
   int k = 0, BN = 0, nt_k = 0, kpad = 0, rpad = 0, tp = 0, Ncmax = 0, fg_chunks = 0, fg_spc = 0, q_used = 0;
+  int gemm_pair = 0;        // X W / X^T Y on CTA pairs (tcgen05 cta_group::2)
   // tensor-core residual/decode streams: U_T^ rows and M^T, padded to 64 ranks
   bool tc_in = false;
   int rows_u = 0, rpad_m = 0;
@@ -410,6 +411,7 @@ jolt_status jolt_plan(const jolt_layout* L, int64_t byte_budget, const jolt_opti
     p->BN = (((p->k + ntile - 1) / ntile) + 15) / 16 * 16;
     p->nt_k = (p->k + p->BN - 1) / p->BN;
     p->kpad = (p->k + 63) / 64 * 64;
+    p->gemm_pair = (p->BN / 2) % 8 == 0;   // BN is a multiple of 16, so always
     p->rpad = (p->rmax_all + 127) / 128 * 128;
     p->tp = (p->T + 7) / 8 * 8;
     const int steps = ((p->Ncmax + 127) / 128) * ((p->T + 63) / 64);
@@ -740,18 +742,19 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
   auto xw = [&]() -> jolt_status {
     ProfScope ps(JOLT_STAGE_GEMM_XW, s);
     umma::Maps mm = m;
-    JOLT_TRY(map_3d(&mm.bt, p->Wt, nc, k, p->Ncmax, p->Ncmax, p->BN));
+    JOLT_TRY(map_3d(&mm.bt, p->Wt, nc, k, p->Ncmax, p->Ncmax, p->gemm_pair ? p->BN / 2 : p->BN));
     umma::Problem q = gemm_problem(p, umma::XW, status);
-    q.M = T; q.N = k; q.BN = p->BN; q.mt = (T + 127) / 128; q.nt = p->nt_k;
+    q.M = T; q.N = k; q.BN = p->BN; q.mt = (T + 127) / 128; q.nt = p->nt_k; q.pair = p->gemm_pair;
     q.out_bf16 = p->Yt; q.out_cell_stride = (int64_t)k * p->tp;
     return launch_umma(mm, q, s);
   };
   auto xty = [&]() -> jolt_status {
     ProfScope ps(JOLT_STAGE_GEMM_XTY, s);
     umma::Maps mm = m;
-    JOLT_TRY(map_3d(&mm.bt, p->Yt, nc, k, T, p->tp, p->BN));
+    JOLT_TRY(map_3d(&mm.bt, p->Yt, nc, k, T, p->tp, p->gemm_pair ? p->BN / 2 : p->BN));
     umma::Problem q = gemm_problem(p, umma::XTY, status);
     q.M = p->Ncmax; q.N = k; q.Kdim = T; q.BN = p->BN; q.mt = (p->Ncmax + 127) / 128; q.nt = p->nt_k;
+    q.pair = p->gemm_pair;
     q.out_f32 = p->Z; q.out_cell_stride = (int64_t)p->Ncmax * k;
     return launch_umma(mm, q, s);
   };

@@ -538,9 +538,9 @@ __device__ __forceinline__ unsigned long long gtimer_ns() {
 
 __device__ bool job_barrier(unsigned int* cnt, unsigned int target, volatile int* abort_flag, int* status) {
   __shared__ int ok_s;
-  __threadfence();          // this thread's writes of A, p and the partial sums
-  __syncthreads();
+  __syncthreads();          // the block's writes of A, p and the partial sums ...
   if (threadIdx.x == 0) {
+    __threadfence();        // ... are ordered before the arrival by this fence (cumulative)
     atomicAdd(cnt, 1u);
     int ok = 1;
     const unsigned long long t0 = gtimer_ns();

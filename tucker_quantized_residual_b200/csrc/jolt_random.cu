@@ -104,6 +104,36 @@ jolt_status launch_umma(const umma::Maps& maps, const umma::Problem& p, cudaStre
                                        umma::SMEM_DATA_MAX + 1024 + 256));
     attr = true;
   }
+  if (p.pair) {
+    if ((p.mode != umma::XW && p.mode != umma::XTY) || (p.BN / 2) % 8) {
+      set_error("CTA-pair GEMM: X W / X^T Y only, BN/2 a multiple of 8 (BN=%d)", p.BN);
+      return JOLT_ERR_INVALID_ARG;
+    }
+    static bool attr2 = false;
+    if (!attr2) {
+      JOLT_CUDA_TRY(cudaFuncSetAttribute(umma::k_umma_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         umma::SMEM_DATA_MAX + 1024 + 256));
+      attr2 = true;
+    }
+    const int mt2 = (p.M + 2 * umma::BM - 1) / (2 * umma::BM);
+    const int tiles2 = p.ncells * mt2 * p.nt;
+    const int pairs = std::max(1, std::min(tiles2, num_sms() / 2));
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(umma::THREADS);
+    cfg.dynamicSmemBytes = umma::pair_smem_bytes(p.BN);
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    JOLT_CUDA_TRY(cudaLaunchKernelEx(&cfg, umma::k_umma_gemm_pair, maps, p));
+    JOLT_LAUNCHED();
+    return JOLT_OK;
+  }
   const int grid = std::min(ntiles, num_sms());
   umma::k_umma_gemm<<<grid, umma::THREADS, umma::smem_bytes(p.BN), s>>>(maps, p);
   JOLT_LAUNCHED();

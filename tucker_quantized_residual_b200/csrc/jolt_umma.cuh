@@ -70,6 +70,7 @@ struct Problem {
   const int* wp_rows;    // WP: r_T per cell (columns >= r_T not stored)
   uint16_t* const* wp_dst;   // WP: per-cell U^T base, row pitch t_pitch
   int* status;
+  int pair;              // 1: CTA pairs (tcgen05 cta_group::2), M = 256 per pair; XW and XTY only
 };
 
 struct Maps {
@@ -77,6 +78,7 @@ struct Maps {
   CUtensorMap xv;     // X of values
   CUtensorMap bt;     // XW: W^T [cells][k][N_c]; XTY/GRAM: Y^T [cells][k][T]; WP: P^T [cells][r][k]; box {64, BN}
   CUtensorMap at;     // GRAM: Y^T, box {64, 128}; WP: Y^T read along t, box {64, 64}
+  // pair mode: bt's box is {64, BN/2}, each CTA of a pair loads its half of the N columns
 };
 
 }  // namespace umma
@@ -456,6 +458,253 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm(const __grid_constant_
   if (warp == 1) {
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols));
+  }
+}
+
+// ------------------------------------------------------------------------
+// CTA-pair variant of the X W and X^T Y passes (tcgen05 cta_group::2): a
+// cluster of two CTAs computes a 256 x BN tile. Each CTA loads its own 128
+// rows of A and half of the BN columns of B into the same shared-memory
+// offsets; the leader CTA (rank 0) issues the 256-row MMA, which reads both
+// CTAs' operands and leaves each CTA's 128 rows of the result in that CTA's
+// TMEM. Per CTA a stage is 16 KB of A and BN/2 x 128 bytes of B, half the B
+// traffic of the single-CTA tile. Barriers: the leader's full[s] counts the
+// bytes of both CTAs' loads (the leader's producer arms it); the leader's
+// commit arrives on empty[s] and tfull[b] of both CTAs; both CTAs' epilogue
+// warps arrive on the leader's tempty[b]. No load is multicast.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(addr), "r"(rank));
+  return d;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+__device__ __forceinline__ void tma2_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
+                                             int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(map), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tma2_load_5d(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
+                                             int c1, int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(map), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
+__device__ __forceinline__ void mma2_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void mma2_commit_both(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
+__host__ __device__ inline int pair_stage_bytes(int BN) { return A_BYTES + ((BN / 2) * BK * 2 + 1023) / 1024 * 1024; }
+__host__ __device__ inline int pair_num_stages(int BN) {
+  const int n = SMEM_DATA_MAX / pair_stage_bytes(BN);
+  return n < MAX_STAGES ? n : MAX_STAGES;
+}
+__host__ __device__ inline int pair_smem_bytes(int BN) { return pair_num_stages(BN) * pair_stage_bytes(BN) + 1024 + 256; }
+
+__global__ void __launch_bounds__(THREADS, 1) k_umma_gemm_pair(const __grid_constant__ Maps maps, Problem p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int STAGES = pair_num_stages(p.BN), STAGE_BYTES = pair_stage_bytes(p.BN);
+  const int BNH = p.BN / 2;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  // bars: full[STAGES] (leader), empty[STAGES], tfull[2], tempty[2] (leader)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
+  const int ncols = (2 * p.BN <= 64) ? 64 : (2 * p.BN <= 128) ? 128 : (2 * p.BN <= 256) ? 256 : 512;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(tfull_bar(b), 1); mbar_init(tempty_bar(b), 8); }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(ncols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  fence_before();
+  __syncthreads();
+  cluster_sync_all();          // both CTAs' barriers exist before any remote arrival
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int mt2 = (p.M + 2 * BM - 1) / (2 * BM);
+  const int ntiles = p.ncells * mt2 * p.nt;
+  const int pair_id = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      uint32_t issued_phase[MAX_STAGES];
+      bool issued[MAX_STAGES];
+      for (int s = 0; s < MAX_STAGES; ++s) issued[s] = false;
+      bool ok = true;
+      const uint32_t stage_tx = 2u * (uint32_t)(A_BYTES + BNH * BK * 2);
+      for (int tile = pair_id; tile < ntiles && ok; tile += npairs) {
+        const int cell = tile / (mt2 * p.nt);
+        const int r = tile - cell * (mt2 * p.nt);
+        const int m0 = (r / p.nt) * (2 * BM) + (int)rank * BM;
+        const int n0 = (r % p.nt) * p.BN + (int)rank * BNH;
+        const int Kc = (p.mode == XW) ? p.cell_Lg[cell] * p.H * p.D : p.Kdim;
+        const int nkb = (Kc + BK - 1) / BK;
+        const CUtensorMap* xm = (p.cell_kind[cell] == 0) ? &maps.xk : &maps.xv;
+        const int l0 = p.cell_l0[cell], b = p.cell_b[cell];
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(empty_bar(stage), ph ^ 1, abort_flag, p.status)) { ok = false; break; }
+          const uint32_t sa = sbase + stage * STAGE_BYTES, sb = sa + A_BYTES;
+          const uint32_t fb = map_to_rank(full_bar(stage), 0);
+          if (rank == 0) mbar_expect_tx(full_bar(stage), stage_tx);
+          const int k0 = kb * BK;
+          if (p.mode == XW) {
+            const int lh = k0 / p.D, d0 = k0 % p.D;
+            const int l = l0 + lh / p.H, h = lh % p.H;
+            tma2_load_5d(sa, xm, fb, d0, m0, h, l, b);
+            tma2_load_5d(sa + 8192, xm, fb, d0, m0 + 64, h, l, b);
+          } else {
+            for (int half = 0; half < 2; ++half) {
+              const int m = m0 + 64 * half;
+              const int lh = m / p.D, d0 = m % p.D;
+              tma2_load_5d(sa + 8192 * half, xm, fb, d0, k0, lh % p.H, l0 + lh / p.H, b);
+            }
+          }
+          tma2_load_3d(sb, &maps.bt, fb, k0, n0, cell);
+          issued[stage] = true;
+          issued_phase[stage] = ph;
+          if (++stage == STAGES) { stage = 0; ph ^= 1; }
+        }
+      }
+      // drain: the leader's full barriers count both CTAs' loads, so the
+      // leader waits (bounded) for every stage it armed before the final sync
+      if (rank == 0)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued[s]) {
+            const unsigned long long t0 = now_ns();
+            while (!mbar_try(full_bar(s), issued_phase[s]) && now_ns() - t0 < WAIT_NS) {}
+          }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t aph[2] = {0, 0};
+      const int a_mn = (p.mode == XTY) ? 1 : 0;
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) |
+                             ((uint32_t)(p.BN >> 3) << 17) | ((uint32_t)((2 * BM) >> 4) << 24);
+      bool ok = true;
+      for (int tile = pair_id; tile < ntiles && ok; tile += npairs) {
+        const int cell = tile / (mt2 * p.nt);
+        const int Kc = (p.mode == XW) ? p.cell_Lg[cell] * p.H * p.D : p.Kdim;
+        const int nkb = (Kc + BK - 1) / BK;
+        if (!mbar_wait(tempty_bar(acc), aph[acc] ^ 1, abort_flag, p.status)) break;
+        fence_after();
+        const uint32_t dcol = tmem + (uint32_t)(acc * p.BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(full_bar(stage), ph, abort_flag, p.status)) { ok = false; break; }
+          fence_after();
+          const uint32_t sa = sbase + stage * STAGE_BYTES, sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t da = a_mn ? sdesc(sa + kk * 2048, 8192, 1024) : sdesc(sa + kk * 32, 16, 1024);
+            const uint64_t db = sdesc(sb + kk * 32, 16, 1024);
+            mma2_bf16(dcol, da, db, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma2_commit_both(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+        mma2_commit_both(tfull_bar(acc));
+        aph[acc] ^= 1;
+        acc ^= 1;
+      }
+      if (!ok) *abort_flag = 1;
+    }
+  } else {
+    // ------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t aph[2] = {0, 0};
+    for (int tile = pair_id; tile < ntiles; tile += npairs) {
+      const int cell = tile / (mt2 * p.nt);
+      const int r = tile - cell * (mt2 * p.nt);
+      const int m0 = (r / p.nt) * (2 * BM) + (int)rank * BM;
+      const int n0 = (r % p.nt) * p.BN;
+      const int Mc = (p.mode == XTY) ? p.cell_Lg[cell] * p.H * p.D : p.M;
+      if (!mbar_wait(tfull_bar(acc), aph[acc], abort_flag, p.status)) break;
+      fence_after();
+      const int row = m0 + q * 32 + lane;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.BN);
+      for (int c0 = 0; c0 < p.BN; c0 += 16) {
+        float v[16];
+        tmem_ld16(tbase + c0, v);
+        const int n = n0 + c0;
+        if (p.mode == XW) {
+          if (row < p.T) {
+            uint16_t* dst = p.out_bf16 + (int64_t)cell * p.out_cell_stride + row;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (n + i < p.N) dst[(int64_t)(n + i) * p.t_pitch] = bf16_bits_from_f32(v[i]);
+          }
+        } else {
+          if (row < Mc) {
+            float* dst = p.out_f32 + (int64_t)cell * p.out_cell_stride + (int64_t)row * p.N;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (n + i < p.N) dst[n + i] = v[i];
+          }
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(tempty_bar(acc), 0));
+      aph[acc] ^= 1;
+      acc ^= 1;
+    }
+  }
+  fence_before();
+  __syncthreads();
+  cluster_sync_all();          // no remote arrival or MMA is outstanding on either CTA
+  if (warp == 1) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols));
   }
 }
 
