@@ -194,6 +194,7 @@ struct jolt_plan_s {
   uint16_t** d_utp = nullptr;
   EighJob* d_jobs_rand = nullptr;
   double* eig_scr = nullptr;   unsigned int* eig_cnt = nullptr;   int eig_nmax = 0;
+  double* gram_part = nullptr;  // GRAM_SPLIT partial Grams (randomized)
 };
 
 struct jolt_handle_s {
@@ -523,6 +524,7 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
       p->ework = A.take<double>((size_t)nc * 3 * k);
       p->eF = A.take<double>((size_t)nc * p->rmax_all * 5 * k);
       p->Rinv = A.take<double>((size_t)nc * kk);
+      p->gram_part = A.take<double>((size_t)GRAM_SPLIT * nc * kk);
       p->RTk = A.take<double>((size_t)nc * kk);
       p->trs = nullptr;
       p->P64 = A.take<double>((size_t)nc * k * p->rmax_all);
@@ -763,7 +765,7 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
     JOLT_TRY(xty());
     // V = Z R^{-1} with Z^T Z = R^T R (fp64), stored as the next W^T
     ProfScope ps(JOLT_STAGE_ORTH, s);
-    JOLT_TRY(launch_gram_cols(p->Z, (int64_t)p->Ncmax * k, p->d_Nc, k, p->Gz, kk, nc, s));
+    JOLT_TRY(launch_gram_cols(p->Z, (int64_t)p->Ncmax * k, p->d_Nc, k, p->Gz, kk, nc, p->gram_part, s));
     JOLT_TRY(launch_chol_blocked(p->Gz, p->RTk, kk, nullptr, k, nc, status, s));
     JOLT_TRY(launch_tri_inverse(p->Gz, p->Rinv, p->RTk, kk, k, nc, s));
     TrsmArgs ta{};
@@ -791,7 +793,7 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
   JOLT_TRY(launch_chol_blocked(p->Rm, p->RTk, kk, p->GW32, k, nc, status, s));
   JOLT_TRY(launch_tri_inverse(p->Rm, p->Rinv, p->RTk, kk, k, nc, s));
   // B B^T = R^{-T} (Z^T Z) R^{-1}: Y1 = P0 R^{-1}, then (Y1^T) R^{-1}
-  JOLT_TRY(launch_gram_cols(p->Z, (int64_t)p->Ncmax * k, p->d_Nc, k, p->P0, kk, nc, s));
+  JOLT_TRY(launch_gram_cols(p->Z, (int64_t)p->Ncmax * k, p->d_Nc, k, p->P0, kk, nc, p->gram_part, s));
   {
     TrsmArgs ta{};
     ta.Rinv = p->Rinv; ta.RinvT = p->RTk; ta.r_cell = kk; ta.k = k; ta.backward = 0;

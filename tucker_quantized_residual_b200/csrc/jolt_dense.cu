@@ -326,6 +326,8 @@ struct DgemmArgs {
   int N, kmode, sym;
   double* C64; int64_t c_cell, c_lm, c_ln;
   uint16_t* C16; int64_t h_cell, h_lm, h_ln;
+  int ksplit, ncells;   // ksplit > 1: blockIdx.z = cell + ncells * slice, C64 holds one partial per slice
+  int64_t part_stride;  // elements between slices' partials
 };
 
 constexpr int DG_T = 64, DG_K = 16, DG_P = 68;
@@ -342,7 +344,7 @@ __device__ __forceinline__ double ld_op(const void* p, int is64, int64_t off) {
 
 __global__ void __launch_bounds__(128) k_dgemm(DgemmArgs g) {
   __shared__ __align__(16) double sm[2 * 2 * DG_K * DG_P];   // [stage][A|B][k][m|n]; reused for the tile
-  const int cell = blockIdx.z;
+  const int cell = (int)(blockIdx.z % g.ncells), slice = (int)(blockIdx.z / g.ncells);
   int m0, n0;
   if (g.sym) {
     int b = blockIdx.x, ti = 0;
@@ -361,6 +363,13 @@ __global__ void __launch_bounds__(128) k_dgemm(DgemmArgs g) {
   int k_lo = 0, k_hi = K;
   if (g.kmode == 1) k_hi = min(K, n0 + DG_T);
   if (g.kmode == 2) k_lo = (n0 / DG_K) * DG_K;
+  if (g.ksplit > 1) {        // this block's slice of K, in whole steps of DG_K
+    const int steps = (k_hi - k_lo + DG_K - 1) / DG_K;
+    const int per = (steps + g.ksplit - 1) / g.ksplit;
+    const int s0 = k_lo + slice * per * DG_K;
+    k_hi = min(k_hi, s0 + per * DG_K);
+    k_lo = s0;
+  }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
   const int gq = lane >> 2, tq = lane & 3;          // fragment row / column group
@@ -439,8 +448,9 @@ __global__ void __launch_bounds__(128) k_dgemm(DgemmArgs g) {
 #pragma unroll
       for (int v = 0; v < 2; ++v) Ts[(wm + i * 8 + gq) * (DG_T + 1) + wn + j * 8 + 2 * tq + v] = c[i][j][v];
   __syncthreads();
+  double* c64 = g.C64 ? g.C64 + (int64_t)slice * g.part_stride : nullptr;
   auto store = [&](int r, int q, double v) {
-    if (g.C64) g.C64[(int64_t)cell * g.c_cell + (int64_t)r * g.c_lm + (int64_t)q * g.c_ln] = v;
+    if (c64) c64[(int64_t)cell * g.c_cell + (int64_t)r * g.c_lm + (int64_t)q * g.c_ln] = v;
     if (g.C16) g.C16[(int64_t)cell * g.h_cell + (int64_t)r * g.h_lm + (int64_t)q * g.h_ln] = bf16_bits_from_f64(v);
   };
   const bool m_fast = (g.C64 ? g.c_lm : g.h_lm) == 1;
@@ -455,13 +465,25 @@ __global__ void __launch_bounds__(128) k_dgemm(DgemmArgs g) {
   }
 }
 
-static jolt_status launch_dgemm(const DgemmArgs& g, int M_max, int ncells, cudaStream_t s) {
+static jolt_status launch_dgemm(DgemmArgs g, int M_max, int ncells, cudaStream_t s) {
   if (M_max <= 0 || g.N <= 0 || ncells <= 0) return JOLT_OK;
+  if (g.ksplit < 1) g.ksplit = 1;
+  g.ncells = ncells;
   const int mt = (M_max + DG_T - 1) / DG_T, nt = (g.N + DG_T - 1) / DG_T;
-  dim3 grid = g.sym ? dim3(nt * (nt + 1) / 2, 1, ncells) : dim3(mt, nt, ncells);
+  dim3 grid = g.sym ? dim3(nt * (nt + 1) / 2, 1, ncells * g.ksplit) : dim3(mt, nt, ncells * g.ksplit);
   k_dgemm<<<grid, 128, 0, s>>>(g);
   JOLT_LAUNCHED();
   return JOLT_OK;
+}
+
+// C[e] = sum over slices of part[slice][e], slices in order (deterministic).
+__global__ void k_sum_slices(const double* __restrict__ part, int64_t stride, int nslices, int64_t n,
+                             double* __restrict__ C) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    double acc = part[e];
+    for (int sl = 1; sl < nslices; ++sl) acc += part[(int64_t)sl * stride + e];
+    C[e] = acc;
+  }
 }
 
 // Rows x of X (one cell per blockIdx.z) as products with the inverse:
@@ -483,18 +505,29 @@ jolt_status launch_tri_apply(const TrsmArgs& a, int rows_max, int ncells, cudaSt
 }
 
 // C = A^T A for A = [rows_of[cell]] x k fp32 (row-major, cell stride a_cell),
-// C k x k fp64 (cell stride c_cell), exactly symmetric.
+// C k x k fp64 (cell stride c_cell), exactly symmetric. The long K (rows) is
+// split into GRAM_SPLIT slices whose partial Grams go to `part`
+// (GRAM_SPLIT * ncells * c_cell doubles) and are then added in order.
 jolt_status launch_gram_cols(const float* A, int64_t a_cell, const int* rows_of, int k, double* C, int64_t c_cell,
-                             int ncells, cudaStream_t s) {
+                             int ncells, double* part, cudaStream_t s) {
   DgemmArgs g{};
   g.A = A; g.a64 = 0; g.a_cell = a_cell; g.a_lm = 1; g.a_lk = k;
   g.B = A; g.b64 = 0; g.b_cell = a_cell; g.b_lk = k; g.b_ln = 1;
   g.M_of = nullptr; g.M_fixed = k;
   g.K_of = rows_of; g.K_fixed = 0;
   g.N = k; g.kmode = 0; g.sym = 1;
-  g.C64 = C; g.c_cell = c_cell; g.c_lm = k; g.c_ln = 1;
+  g.c_cell = c_cell; g.c_lm = k; g.c_ln = 1;
   g.C16 = nullptr;
-  return launch_dgemm(g, k, ncells, s);
+  if (!part) {
+    g.C64 = C;
+    return launch_dgemm(g, k, ncells, s);
+  }
+  g.C64 = part; g.ksplit = GRAM_SPLIT; g.part_stride = (int64_t)ncells * c_cell;
+  JOLT_TRY(launch_dgemm(g, k, ncells, s));
+  const int64_t n = (int64_t)ncells * c_cell;
+  k_sum_slices<<<(int)std::min<int64_t>((n + 255) / 256, 148 * 8), 256, 0, s>>>(part, g.part_stride, GRAM_SPLIT, n, C);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
 }
 
 }  // namespace jolt

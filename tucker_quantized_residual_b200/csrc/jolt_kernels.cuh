@@ -170,8 +170,9 @@ jolt_status launch_make_xb(const void* src, int f32, int rope, const float2* cs,
                            int D, int64_t sb, int64_t sl, int64_t sh, int64_t st, uint16_t* dst, cudaStream_t s);
 jolt_status launch_omega(uint16_t* wt, int ncells, int k, int ld, const int* Nc, const int* seq, const int* cis,
                          uint64_t seed, cudaStream_t s);
+constexpr int GRAM_SPLIT = 4;   // K slices of the fp64 Gram (partials in a scratch buffer)
 jolt_status launch_gram_cols(const float* A, int64_t a_cell, const int* rows_of, int k, double* C, int64_t c_cell,
-                             int ncells, cudaStream_t s);
+                             int ncells, double* part, cudaStream_t s);
 jolt_status launch_cholesky(double* A, int64_t a_cell, const float* src32, int64_t s_cell, int k, int ncells,
                             int* status, cudaStream_t s);
 jolt_status launch_trsm_rows(const float* Z, int64_t z_cell, const double* R, int64_t r_cell, int k, const int* Nc,
