@@ -202,6 +202,21 @@ __device__ __forceinline__ void fwht_row(float* v) {
 
 __host__ __device__ inline int qmax_of(int b) { return (1 << (b - 1)) - 1; }
 
+// fl32(a / b) without a divide instruction, by residual corrections
+// (P. Markstein, "IA-64 and Elementary Functions", 2000). With rb = RN(1/b),
+// q0 = RN(a * rb) is within 1.5 ulp of a / b; one correction
+// q1 = RN(q0 + (a - q0 b) rb), the residual exact in one fused multiply-add,
+// brings it within one ulp, and by Markstein's theorem a second correction
+// from such an estimate returns the correctly rounded quotient. Valid while b
+// and 1/b are normal numbers (quot_ok); callers bring b into that range by an
+// exact power-of-two scaling of both operands otherwise.
+__device__ __forceinline__ bool quot_ok(float b) { return b >= 1e-30f && b <= 1e30f; }
+__device__ __forceinline__ float quot_rn(float a, float b, float rb) {
+  const float q0 = __fmul_rn(a, rb);
+  const float q1 = __fmaf_rn(__fmaf_rn(-q0, b, a), rb, q0);
+  return __fmaf_rn(__fmaf_rn(-q1, b, a), rb, q1);
+}
+
 // Quantize + pack one rotated row r[D] (fp32) with groups of G values and B
 // bits: scale = fl32(absmax / q_max), code = clamp(rint(fl32(r / scale))),
 // u = code + 2^(B-1) stored LSB first. codes: B*D/8 bytes (8-byte aligned);
@@ -221,10 +236,17 @@ __device__ __forceinline__ void quantize_pack_row(const float* r, uint8_t* __res
     for (int j = 0; j < G; ++j) a = fmaxf(a, fabsf(r[g0 + j]));
     const float sc = __fdiv_rn(a, qm);
     scales[g0 / G] = sc;
+    // quotients by quot_rn; a scale outside its range is first brought into
+    // it by an exact power-of-two factor applied to both operands
+    const float m = quot_ok(sc) ? 1.0f : (sc < 1.0f ? 18446744073709551616.0f : 5.421010862427522e-20f);
+    const float sm = __fmul_rn(sc, m), rsm = (sc > 0.0f) ? __frcp_rn(sm) : 0.0f;
 #pragma unroll
     for (int j = 0; j < G; ++j) {
       int q = 0;
-      if (sc > 0.0f) q = (int)fminf(fmaxf(rintf(__fdiv_rn(r[g0 + j], sc)), -qm), qm);
+      if (sc > 0.0f) {
+        const float y = quot_rn(__fmul_rn(r[g0 + j], m), sm, rsm);
+        q = (int)fminf(fmaxf(rintf(y), -qm), qm);
+      }
       const uint64_t u = (uint64_t)(uint32_t)(q + (1 << (B - 1)));
       const int bit = (g0 + j) * B;
       const int wi = bit >> 6, sh = bit & 63;
