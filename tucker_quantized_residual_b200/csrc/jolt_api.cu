@@ -503,8 +503,8 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
     p->Ut_ws = A.take<uint16_t>((size_t)nc * p->rows_u * p->tp);
     p->Mt_ws = A.take<uint16_t>((size_t)nc * p->lh_max * D * p->rpad_m);
     p->eig_nmax = std::max(p->opt.mode == JOLT_RANDOMIZED ? p->k : p->nmin_max, D);
-    p->eig_scr = A.take<double>((size_t)nc * (p->eig_nmax + 64));
-    p->eig_cnt = A.take<unsigned int>(nc + 1);
+    p->eig_scr = A.take<double>((size_t)nc * (2 * p->eig_nmax + 128));
+    p->eig_cnt = A.take<unsigned int>(2 * nc + 1);
     if (p->opt.mode == JOLT_RANDOMIZED) {
       const int k = p->k;
       const size_t kk = (size_t)k * k;

@@ -21,7 +21,7 @@ jolt_status launch_eigh(const EighJob* jobs_dev, int njobs, int nmax, int* statu
 size_t eigh_smem_bytes(int nmax);
 jolt_status launch_tridiag(const EighJob* jobs, int njobs, int nmax, cudaStream_t s);
 // Multi-block reduction of jobs[0..njobs) (all of size <= nmax); scratch holds
-// njobs * (nmax + 64) doubles, counters njobs + 1 words.
+// njobs * (2 nmax + 128) doubles, counters 2 njobs + 1 words.
 jolt_status launch_tridiag_multi(const EighJob* jobs, int njobs, int nmax, double* scratch, unsigned int* counters,
                                  int* status, cudaStream_t s);
 jolt_status launch_bisect(const EighJob* jobs, int njobs, int nmax, cudaStream_t s);

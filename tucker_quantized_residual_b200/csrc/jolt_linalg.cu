@@ -520,16 +520,19 @@ __global__ void __launch_bounds__(EIG_THREADS) k_tridiag(const EighJob* __restri
 }
 
 // The same reduction with G thread blocks per matrix (one cooperative launch
-// over all jobs). Every block of a job computes the reflector of column k
-// itself from row k (A is kept exactly symmetric, so row k equals column k),
-// forms p = beta A v for its share of the rows, and publishes it; after a
-// job-wide barrier each block rebuilds w = p - (beta/2)(p.v) v from all
-// shares (partial sums added in block order, so every block gets the same
-// bits) and applies the rank-2 update to its own rows; a second barrier
-// precedes the next column. A is read through L2 only (other blocks write
-// it). Barriers are counters in global memory with bounded waits: on expiry
-// the block raises the job's abort flag and the timeout status and returns,
-// and the others follow at their next wait.
+// over all jobs). Row r of the trailing matrix belongs to warp r mod (G x
+// warps per block) for the whole reduction. At column k every block computes
+// the reflector itself from row k (A is kept exactly symmetric, so row k
+// equals column k), forms p = beta A v for its own rows and publishes them;
+// after a job-wide barrier each block rebuilds w = p - (beta/2)(p.v) v from
+// all shares (partial sums added in block order, so every block gets the
+// same bits) and applies the rank-2 update to its own rows. The owner of row
+// k+1 updates it first and publishes it with a per-job flag; the next column
+// waits for that flag only, not for every block (its other reads are the
+// block's own rows). p and the partial sums alternate between two buffers by
+// column parity. A is read through L2 only. Barriers and flags are bounded
+// waits: on expiry the block raises the job's abort flag and the timeout
+// status and returns, and the others follow at their next wait.
 __device__ __forceinline__ unsigned long long gtimer_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -563,9 +566,39 @@ __device__ bool job_barrier(unsigned int* cnt, unsigned int target, volatile int
   return ok_s != 0;
 }
 
+// Bounded wait until the job's published-row flag reaches `target`.
+__device__ bool wait_flag(volatile unsigned int* flag, unsigned int target, volatile int* abort_flag, int* status) {
+  __shared__ int ok_f;
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const unsigned long long t0 = gtimer_ns();
+    while (true) {
+      unsigned int f;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(f) : "l"(flag) : "memory");
+      if (f >= target) break;
+      if (*abort_flag) { ok = 0; break; }
+      if (gtimer_ns() - t0 > 2000000000ull) {
+        *abort_flag = 1;
+        atomicOr(status, DEV_ERR_TIMEOUT);
+        ok = 0;
+        break;
+      }
+    }
+    ok_f = ok;
+  }
+  __syncthreads();
+  return ok_f != 0;
+}
+
+__device__ __forceinline__ void publish_flag(unsigned int* flag, unsigned int value) {
+  __threadfence();
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(value) : "memory");
+}
+
 __global__ void __launch_bounds__(EIG_THREADS) k_tridiag_multi(const EighJob* __restrict__ jobs, int G, int nmax,
                                                                double* __restrict__ scratch,
                                                                unsigned int* __restrict__ counters, int* status) {
+  const int njobs = gridDim.x / G;
   const int job = blockIdx.x / G, c = blockIdx.x % G;
   const EighJob J = jobs[job];
   const int n = J.n;
@@ -578,16 +611,19 @@ __global__ void __launch_bounds__(EIG_THREADS) k_tridiag_multi(const EighJob* __
   double* dd = J.work;
   double* ee = dd + n;
   double* tau = ee + n;
-  double* P = scratch + (size_t)job * (nmax + 64);   // p (n) then per-block partial sums (G <= 64)
-  double* part = P + nmax;
+  double* Pb = scratch + (size_t)job * (2 * nmax + 128);   // p[2][nmax], then partial sums [2][64]
   unsigned int* cnt = counters + job;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(counters + gridDim.x / G);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(counters + njobs);
+  unsigned int* flag = counters + njobs + 1 + job;          // rows published: row k is final when flag >= k
   const int tid = threadIdx.x, nt = blockDim.x;
   const int lane = tid & 31, warp = tid >> 5, nwarp = nt >> 5;
   const int gw = c * nwarp + warp, GW = G * nwarp;
   unsigned int nbar = 0;
   for (int k = 0; k + 2 < n; ++k) {
-    const int m = n - k - 1;
+    const int m = n - k - 1, buf = k & 1;
+    double* P = Pb + buf * nmax;
+    double* part = Pb + 2 * nmax + buf * 64;
+    if (k > 0 && !wait_flag(flag, (unsigned)k, abort_flag, status)) return;
     const double* rowk = A + (int64_t)k * n + (k + 1);
     for (int i = tid; i < m; i += nt) v[i] = __ldcg(rowk + i);
     __syncthreads();
@@ -595,9 +631,14 @@ __global__ void __launch_bounds__(EIG_THREADS) k_tridiag_multi(const EighJob* __
     for (int i = 1 + tid; i < m; i += nt) s += v[i] * v[i];
     s = block_sum(s, red);
     const double x0 = v[0];
+    // this warp's first row past k (rows r with r mod GW == gw)
+    const int r0 = k + 1 + (((gw - (k + 1)) % GW) + GW) % GW;
     if (s == 0.0) {
       if (c == 0 && tid == 0) { dd[k] = __ldcg(A + (int64_t)k * n + k); ee[k] = x0; tau[k] = 0.0; }
-      __syncthreads();
+      if (r0 == k + 1 && lane == 0) publish_flag(flag, (unsigned)(k + 1));   // row k+1 is unchanged
+      // one barrier per column in every case, so the two p buffers are never
+      // rewritten while a slower block still reads them
+      if (!job_barrier(cnt, (++nbar) * (unsigned)G, abort_flag, status)) return;
       continue;
     }
     const double nrm = sqrt(x0 * x0 + s);
@@ -608,8 +649,9 @@ __global__ void __launch_bounds__(EIG_THREADS) k_tridiag_multi(const EighJob* __
     if (tid == 0) v[0] = v0;
     __syncthreads();
     double pv = 0.0;
-    for (int i = gw; i < m; i += GW) {
-      const double* row = A + (int64_t)(k + 1 + i) * n + (k + 1);
+    for (int r = r0; r < n; r += GW) {
+      const int i = r - k - 1;
+      const double* row = A + (int64_t)r * n + (k + 1);
       double acc = 0.0;
       for (int j = lane; j < m; j += 32) acc += __ldcg(row + j) * v[j];
       acc = warp_sum(acc);
@@ -627,17 +669,23 @@ __global__ void __launch_bounds__(EIG_THREADS) k_tridiag_multi(const EighJob* __
     const double Kc = 0.5 * beta * tot;
     for (int i = tid; i < m; i += nt) w[i] = __ldcg(P + i) - Kc * v[i];
     __syncthreads();
-    for (int i = gw; i < m; i += GW) {
-      double* row = A + (int64_t)(k + 1 + i) * n + (k + 1);
+    for (int r = r0; r < n; r += GW) {
+      const int i = r - k - 1;
+      double* row = A + (int64_t)r * n + (k + 1);
       const double vi = v[i], wi = w[i];
       // no contraction: entry (i, j) and (j, i) get the same two products
       for (int j = lane; j < m; j += 32)
         row[j] = __dsub_rn(__ldcg(row + j), __dadd_rn(__dmul_rn(vi, w[j]), __dmul_rn(wi, v[j])));
-      if (lane == 0) A[(int64_t)k * n + (k + 1 + i)] = v[i];   // reflector k in row k
+      __syncwarp();
+      if (lane == 0) {
+        A[(int64_t)k * n + r] = v[i];                       // reflector k in row k
+        if (r == k + 1) publish_flag(flag, (unsigned)(k + 1));
+      }
     }
     if (c == 0 && tid == 0) { dd[k] = __ldcg(A + (int64_t)k * n + k); ee[k] = alpha; tau[k] = beta; }
-    if (!job_barrier(cnt, (++nbar) * (unsigned)G, abort_flag, status)) return;
   }
+  // every row's last update is in before the last diagonal entries are read
+  if (!job_barrier(cnt, (++nbar) * (unsigned)G, abort_flag, status)) return;
   if (c == 0 && tid == 0) {
     if (n >= 2) {
       dd[n - 2] = __ldcg(A + (int64_t)(n - 2) * n + (n - 2));
@@ -944,7 +992,7 @@ jolt_status launch_tridiag_multi(const EighJob* jobs, int njobs, int nmax, doubl
   { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_tridiag_multi, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
   const int G = tridiag_blocks_per_job(njobs, nmax, smem);
   if (G < 2) return launch_tridiag(jobs, njobs, nmax, s);
-  JOLT_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)(njobs + 1) * sizeof(unsigned int), s));
+  JOLT_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)(2 * njobs + 1) * sizeof(unsigned int), s));
   int Gv = G, nm = nmax;
   void* args[] = {(void*)&jobs, (void*)&Gv, (void*)&nm, (void*)&scratch, (void*)&counters, (void*)&status};
   JOLT_CUDA_TRY(cudaLaunchCooperativeKernel((const void*)k_tridiag_multi, dim3(njobs * G), dim3(EIG_THREADS), args,
