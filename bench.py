@@ -111,9 +111,11 @@ class ClockSampler:
 
 # ------------------------------------------------------------ workload
 # DRAM bytes per launch of the dominant kernel from an ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum), scaled to the full launch
-# by the cells it processes; None once the kernel has changed since.
-GEMM_TRAFFIC = None
+# (dram__bytes_read.sum + dram__bytes_write.sum) of the first layer group of
+# the 64K-token cache (profiles/k_umma_gemm_pair_llama31_64k_1group.md),
+# scaled to the full 16-cell launch by the cells it processes (mean of the
+# X W and X^T Y launches); None once the kernel has changed since.
+GEMM_TRAFFIC = {"llama31_8b_64k": 10.38e9}
 
 
 def sketch_width(spec, ratio, p=8):
@@ -285,10 +287,11 @@ def run_jolt(args):
         nl = work["gemm_xw"][2] + work["gemm_xty"][2]
         per_launch_s = gemm_ms / 1e3 / nl
         ach = fl / nl / per_launch_s / 1e12
-        roof = {"bound": "tensor", "kernel": "k_umma_gemm (X W and X^T Y launches)", "achieved": round(ach, 1),
+        traffic = GEMM_TRAFFIC.get(args.config) if (GEMM_TRAFFIC and not args.groups and args.ratio == 2.0) else None
+        roof = {"bound": "tensor", "kernel": "k_umma_gemm_pair (X W and X^T Y launches)", "achieved": round(ach, 1),
                 "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops_sustained"], 3),
                 "peak_source": f"{src} bf16 sustained", "flops_per_launch": fl / nl,
-                "traffic": GEMM_TRAFFIC}
+                "traffic": traffic}
     else:
         fl, by, nl = work[dom]
         per_launch_s = cand[dom] / 1e3 / nl
