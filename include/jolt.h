@@ -58,6 +58,7 @@ typedef enum {
 enum { JOLT_BF16 = 0, JOLT_F32 = 1 };             /* jolt_layout.dtype        */
 enum { JOLT_EXACT = 0, JOLT_RANDOMIZED = 1 };      /* jolt_options.mode        */
 enum { JOLT_ROT_HADAMARD = 0 };                    /* jolt_options.rotation    */
+enum { JOLT_MIN_ENUMERATE = 0, JOLT_MIN_GREEDY = 1 }; /* jolt_options.minimizer */
 
 /*
  * Where the cache lives. Element (b, l, h, t, d) of K (and of V, same layout)
@@ -86,7 +87,12 @@ typedef struct {
  *   oversample_p 8, power_iters 2 (randomized range finder);
  *   scale_group 0 (= D: one fp32 scale per row, Eq. 1's 32/d_h term);
  *   budget_tol 0.005 and max_iters 50 (Section 3: "stopping within 0.5% of
- *   the target budget or after 50 iterations").
+ *   the target budget or after 50 iterations");
+ *   minimizer JOLT_MIN_ENUMERATE: the per-cell argmin of e + lambda s over
+ *   every option. JOLT_MIN_GREEDY is the page's per-cell search ("Solving the
+ *   allocation"): for each b, start at the smallest ranks and take whichever
+ *   single grid step of r_T or r_d lowers the error most per added byte, while
+ *   it lowers e + lambda s; keep the best b.
  * Grids are HOST arrays of strictly increasing values >= 1, copied at plan
  * time; NULL/0 means "every integer 1..max".
  */
@@ -104,6 +110,7 @@ typedef struct {
   int32_t rotation;              /* JOLT_ROT_HADAMARD                          */
   double budget_tol;
   int32_t max_iters;
+  int32_t minimizer;             /* JOLT_MIN_ENUMERATE | JOLT_MIN_GREEDY       */
 } jolt_options;
 
 typedef struct jolt_plan_s jolt_plan_t;

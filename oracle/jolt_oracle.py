@@ -433,12 +433,18 @@ class Allocation:
 
 
 def allocate(tables: List[CellTable], budget: int, tol: float = 0.005,
-             max_iters: int = 50, lam_lo: float = 1e-30, lam_hi: float = 1.0) -> Allocation:
-    """Geometric bisection on the shared multiplier lambda (reading R4)."""
+             max_iters: int = 50, lam_lo: float = 1e-30, lam_hi: float = 1.0,
+             minimizer: str = "enumerate") -> Allocation:
+    """Geometric bisection on the shared multiplier lambda (reading R4). The
+    per-cell minimizer is exact enumeration (reading R3) or the page's greedy
+    search (minimizer="greedy")."""
     arrs = [t.arrays() for t in tables]
 
     def at(lam):
-        idx = [argmin_cell(t, lam, a) for t, a in zip(tables, arrs)]
+        if minimizer == "greedy":
+            idx = [greedy_index(t, lam) for t in tables]
+        else:
+            idx = [argmin_cell(t, lam, a) for t, a in zip(tables, arrs)]
         S = int(sum(int(a[4][i]) for a, i in zip(arrs, idx)))
         return idx, S
 
@@ -468,45 +474,56 @@ def allocate(tables: List[CellTable], budget: int, tol: float = 0.005,
 
 
 def greedy_cell(tab: CellTable, lam: float) -> Tuple[int, int, int, float]:
-    """The page's per-cell search under integer rank grids: for every b, start
-    at r_T = r_d = 1 and repeatedly take whichever single-step rank increment
-    has the steeper error decrease per byte, as long as that step lowers
-    e + lam*s; keep the b with the smallest e + lam*s. Returns
+    """The page's per-cell search ("Solving the allocation"): for every b,
+    start at the smallest ranks of the grids and repeatedly take whichever
+    single grid step (r_T or r_d to its next grid value; with the default
+    integer grids, rank + 1) has the steeper error decrease per byte, as long
+    as that step lowers e + lam*s; keep the b with the smallest e + lam*s
+    (first on ties). Ties between the two steps go to r_T. Returns
     (r_T, r_d, b, value)."""
     best = None
-    rmaxT = len(tab.tT) - 1
-    rmaxD = len(tab.tD) - 1
+    nT, nD = len(tab.rt_grid), len(tab.rd_grid)
     for bi, b in enumerate(tab.bits):
         eps = float(tab.eps2[bi])
-        rT, rd = 1, 1
+        ti, di = 0, 0
 
         def val(a, c):
-            e = eps * (float(tab.tT[a]) + float(tab.tD[c]))
-            s = cost_bytes(tab.Lg, tab.H, tab.T, tab.D, a, c, int(b), tab.g)
+            rT, rd = int(tab.rt_grid[a]), int(tab.rd_grid[c])
+            e = eps * (float(tab.tT[rT]) + float(tab.tD[rd])) if tab.valid(rT, rd) else math.inf
+            s = cost_bytes(tab.Lg, tab.H, tab.T, tab.D, rT, rd, int(b), tab.g)
             return e + lam * s, e, s
 
         while True:
-            v0, e0, s0 = val(rT, rd)
+            v0, e0, s0 = val(ti, di)
             cands = []
-            if rT < rmaxT:
-                v1, e1, s1 = val(rT + 1, rd)
+            if ti + 1 < nT:
+                v1, e1, s1 = val(ti + 1, di)
                 if v1 < v0:
                     cands.append(((e0 - e1) / (s1 - s0), 0))
-            if rd < rmaxD and tab.valid(rT, rd + 1):
-                v2, e2, s2 = val(rT, rd + 1)
+            if di + 1 < nD:
+                v2, e2, s2 = val(ti, di + 1)
                 if v2 < v0:
                     cands.append(((e0 - e2) / (s2 - s0), 1))
             if not cands:
                 break
             cands.sort(key=lambda z: (-z[0], z[1]))
             if cands[0][1] == 0:
-                rT += 1
+                ti += 1
             else:
-                rd += 1
-        v, _, _ = val(rT, rd)
+                di += 1
+        v, _, _ = val(ti, di)
         if best is None or v < best[3]:
-            best = (rT, rd, int(b), v)
+            best = (int(tab.rt_grid[ti]), int(tab.rd_grid[di]), int(b), v)
     return best
+
+
+def greedy_index(tab: CellTable, lam: float) -> int:
+    """greedy_cell's choice as an index in the enumeration order of arrays()."""
+    rT, rd, b, _ = greedy_cell(tab, lam)
+    bi = int(np.searchsorted(tab.bits, b))
+    ti = int(np.searchsorted(tab.rt_grid, rT))
+    di = int(np.searchsorted(tab.rd_grid, rd))
+    return (bi * len(tab.rt_grid) + ti) * len(tab.rd_grid) + di
 
 
 # --------------------------------------------------------------------------
@@ -582,6 +599,7 @@ class Options:
     scale_group: int = 0                          # 0: D (one scale per row)
     tol: float = 0.005
     max_iters: int = 50
+    minimizer: str = "enumerate"                  # or "greedy" (the page's per-cell search)
 
 
 @dataclasses.dataclass
@@ -668,7 +686,7 @@ def compress(cache_k: np.ndarray, cache_v: np.ndarray, group_starts: Sequence[in
         tabs.append(tab)
         Us.append(U)
         Xs.append(X)
-    al = allocate(tabs, budget, opt.tol, opt.max_iters)
+    al = allocate(tabs, budget, opt.tol, opt.max_iters, minimizer=opt.minimizer)
     out = []
     for c, X, U, (rT, rd, b), nb in zip(refs, Xs, Us, al.choice, al.bytes):
         f = fit(X, U, rT, rd)

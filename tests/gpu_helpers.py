@@ -15,7 +15,10 @@ def gpu_compress(K: torch.Tensor, V: torch.Tensor, group_starts, budget: int, se
     iters, bytes, plan, handle) with K_hat/V_hat as float64 numpy arrays."""
     Kd, Vd = K.cuda().contiguous(), V.cuda().contiguous()
     lay, keep = jolt.make_layout(Kd, group_starts, rope_theta_k)
-    opt, keep2 = jolt.make_options(**opt_kw)
+    kw = dict(opt_kw)
+    if isinstance(kw.get("minimizer"), str):
+        kw["minimizer"] = jolt.JOLT_MIN_GREEDY if kw["minimizer"] == "greedy" else jolt.JOLT_MIN_ENUMERATE
+    opt, keep2 = jolt.make_options(**kw)
     plan = jolt.jolt_plan(lay, budget, opt)
     try:
         h = jolt.jolt_compress(plan, Kd, Vd, budget, seed)
@@ -44,7 +47,8 @@ def oracle_compress(K: torch.Tensor, V: torch.Tensor, group_starts, budget: int,
                     rt_grid=tuple(kw["rt_grid"]) if kw.get("rt_grid") else None,
                     rd_grid=tuple(kw["rd_grid"]) if kw.get("rd_grid") else None,
                     rt_max=kw.get("rt_max", 0), scale_group=kw["scale_group"],
-                    tol=kw.get("budget_tol", 0.005), max_iters=kw.get("max_iters", 50))
+                    tol=kw.get("budget_tol", 0.005), max_iters=kw.get("max_iters", 50),
+                    minimizer=kw.get("minimizer", "enumerate"))
     comp = o.compress(Kn, Vn, group_starts, budget, seed, opt, rope_theta_k)
     Kh, Vh = o.decompress(comp)
     return Kn, Vn, Kh, Vh, comp

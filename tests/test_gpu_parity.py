@@ -169,6 +169,54 @@ def test_allocation_tiny_grid_bit_exact():
             jolt.jolt_free_plan(plan)
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("C_ratio", [2.0, 3.0])
+def test_greedy_allocation_bit_exact_on_oracle_tables(C_ratio):
+    """The page's greedy per-cell search inside the same bisection."""
+    T, D, Lg, H, ng = 1024, 128, 4, 8, 8
+    raw = _synthetic_tables(2 * ng, T, D, Lg, H, seed=int(C_ratio * 10) + 1)
+    dense = 2 * 2 * ng * Lg * H * T * D
+    B = int(dense // C_ratio)
+    plan, keep = _plan_for(T, D, Lg, H, ng, B, minimizer=jolt.JOLT_MIN_GREEDY)
+    try:
+        eps = o.eps2_table((0, 2, 4, 8), D)
+        tabs = []
+        for ns, sT, sD in raw:
+            tabs.append(o.CellTable(Lg, H, T, D, D, ns, o.tail_fractions(sT, ns), o.tail_fractions(sD, ns),
+                                    np.arange(1, min(T, Lg * H * D) + 1), np.arange(1, D + 1),
+                                    np.array([0, 2, 4, 8]), np.array([eps[b] for b in (0, 2, 4, 8)])))
+        ref = o.allocate(tabs, B, minimizer="greedy")
+        ch, by, lam, it = jolt.jolt_allocate(plan, [t.tT for t in tabs], [t.tD for t in tabs],
+                                             [eps[b] for b in (0, 2, 4, 8)], B)
+        assert ch == ref.choice
+        assert by == ref.bytes
+        assert lam == ref.lam and it == ref.iters
+    finally:
+        jolt.jolt_free_plan(plan)
+
+
+@pytest.mark.gpu
+def test_greedy_tiny_end_to_end():
+    spec = synth.SPECS["tiny"]
+    K, V = synth.make_cache(spec, 0)
+    B = o.budget_for_ratio(K.numel() * 2, 2.0)
+    eK, eV = _compare(K, V, synth.group_starts(spec), B, 0.0, bits=(0, 2, 3, 4, 8),
+                      rt_grid=(8, 16, 32, 64), rd_grid=(16, 32, 48), minimizer="greedy")
+    assert eK < 0.2 and eV < 0.2
+
+
+@pytest.mark.gpu
+def test_mistral_exact_token_rank_capped_at_qcap():
+    """Exact mode with the token rank capped at q_cap (Eq. 5), as the pages do
+    for long contexts."""
+    spec = synth.SPECS["mistral"]
+    K, V = synth.make_cache(spec, 0)
+    B = o.budget_for_ratio(K.numel() * 2, 2.0)
+    q = o.q_cap(spec.seq_len, 2.0)
+    eK, eV = _compare(K, V, synth.group_starts(spec), B, spec.rope_theta_k, rt_max=q)
+    assert eK < 0.05 and eV < 0.05
+
+
 # ----------------------------------------------------------------- spectra
 @pytest.mark.parametrize("name", ["tiny", "mistral"])
 def test_rd_spectra_match_oracle(name):

@@ -383,6 +383,50 @@ def test_greedy_never_beats_enumeration_on_integer_grids():
         assert v_g >= v_enum - 1e-15
 
 
+def test_greedy_ends_at_a_local_minimum_of_its_grid():
+    """No single grid step from the greedy choice lowers e + lam*s, and at a
+    prohibitive price it stays at the smallest ranks."""
+    X = _noisy_cell(2, 2, 40, 16)
+    opt = o.Options(bits=(0, 2, 4, 8))
+    eps = o.eps2_table(opt.bits, 16)
+    tab = o.build_table(X, opt, eps)[0]
+
+    def value(bi, ti, di):
+        rT, rd = int(tab.rt_grid[ti]), int(tab.rd_grid[di])
+        if not tab.valid(rT, rd):
+            return math.inf
+        e = float(tab.eps2[bi]) * (float(tab.tT[rT]) + float(tab.tD[rd]))
+        return e + lam * o.cost_bytes(tab.Lg, tab.H, tab.T, tab.D, rT, rd, int(tab.bits[bi]), tab.g)
+
+    for lam in (1e-9, 1e-7, 1e-5, 1e-4):
+        rT, rd, b, v = o.greedy_cell(tab, lam)
+        bi = list(tab.bits).index(b)
+        ti, di = list(tab.rt_grid).index(rT), list(tab.rd_grid).index(rd)
+        assert v == value(bi, ti, di)
+        if ti + 1 < len(tab.rt_grid):
+            assert value(bi, ti + 1, di) >= v
+        if di + 1 < len(tab.rd_grid):
+            assert value(bi, ti, di + 1) >= v
+    lam = 1e3
+    rT, rd, b, v = o.greedy_cell(tab, lam)
+    assert (rT, rd, b) == (int(tab.rt_grid[0]), int(tab.rd_grid[0]), int(tab.bits[0]))
+
+
+def test_greedy_allocation_respects_the_budget():
+    tabs = _tiny_tables()
+    dense = 2 * 2 * 2 * 256 * 64 * 2
+    for C in (2.0, 3.0):
+        B = o.budget_for_ratio(dense // 2, C)
+        g = o.allocate(tabs, B, minimizer="greedy")
+        e = o.allocate(tabs, B)
+        assert sum(g.bytes) <= B
+        assert all(ch[0] in tabs[0].rt_grid and ch[1] in tabs[0].rd_grid for ch in g.choice)
+        # enumeration is the exact per-cell minimizer: at its own attained budget
+        # it is at least as good as any allocation that fits in that budget
+        if sum(g.bytes) <= sum(e.bytes):
+            assert sum(e.errors) <= sum(g.errors) * (1 + 1e-12)
+
+
 # --------------------------------------------------------------- full path
 def test_full_ranks_no_residual_is_bf16_storage_exact_level():
     from tucker_quantized_residual_b200 import synth

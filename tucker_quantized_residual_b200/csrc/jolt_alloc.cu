@@ -208,6 +208,63 @@ __global__ void __launch_bounds__(256) k_alloc_eval(AllocArgs a) {
   }
 }
 
+// The page's greedy per-cell search ("Solving the allocation"): for each b
+// (one lane per bit width) start at the first grid entries and repeatedly
+// take whichever single grid step of r_T or r_d lowers the error most per
+// added byte, while that step lowers e + lambda s (ties: the r_T step); then
+// the best b, first on ties. The result goes to chunk 0 of the partial
+// argmins in enumeration-index form, the other chunks get +inf.
+__global__ void __launch_bounds__(32) k_alloc_greedy(AllocArgs a) {
+  if (a.st->phase == 3) return;
+  const int cell = blockIdx.x, lane = threadIdx.x;
+  const CellRD c = a.cells[cell];
+  const double lam = a.st->lam;
+  double best = INFINITY;
+  int bidx = 0x7fffffff;
+  if (lane < a.n_bits) {
+    const int bi = lane;
+    int ti = 0, di = 0;
+    auto eval = [&](int t, int d, double& e, int64_t& s) {
+      const int rt = a.rt_grid[t], rd = a.rd_grid[d];
+      e = opt_err(a, c, bi, rt, rd);
+      s = opt_bytes(a, c, bi, rt, rd);
+      return __dadd_rn(e, __dmul_rn(lam, (double)s));
+    };
+    for (int guard = 0; guard < c.n_rt + a.n_rd; ++guard) {
+      double e0, e1, e2;
+      int64_t s0, s1, s2;
+      const double v0 = eval(ti, di, e0, s0);
+      bool c1 = false, c2 = false;
+      double r1 = 0.0, r2 = 0.0;
+      if (ti + 1 < c.n_rt) {
+        const double v1 = eval(ti + 1, di, e1, s1);
+        if (v1 < v0) { c1 = true; r1 = __ddiv_rn(__dsub_rn(e0, e1), (double)(s1 - s0)); }
+      }
+      if (di + 1 < a.n_rd) {
+        const double v2 = eval(ti, di + 1, e2, s2);
+        if (v2 < v0) { c2 = true; r2 = __ddiv_rn(__dsub_rn(e0, e2), (double)(s2 - s0)); }
+      }
+      if (!c1 && !c2) break;
+      if (c1 && (!c2 || r1 >= r2)) ++ti;
+      else ++di;
+    }
+    double e;
+    int64_t sb;
+    best = eval(ti, di, e, sb);
+    bidx = (bi * c.n_rt + ti) * a.n_rd + di;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+    if (ob < best || (ob == best && oi < bidx)) { best = ob; bidx = oi; }
+  }
+  for (int k = lane; k < a.nchunk; k += 32) {
+    a.pv[cell * a.nchunk + k] = (k == 0) ? best : INFINITY;
+    a.pi[cell * a.nchunk + k] = (k == 0) ? bidx : 0x7fffffff;
+  }
+}
+
 // One block: per-cell argmin over chunks, total bytes, one bisection step.
 __global__ void __launch_bounds__(512) k_alloc_decide(AllocArgs a) {
   AllocState* st = a.st;
@@ -290,7 +347,8 @@ jolt_status launch_alloc(const AllocArgs& a, const AllocState& init, cudaStream_
   JOLT_LAUNCHED();
   dim3 grid(a.nchunk, a.ncells);
   for (int it = 0; it < init.max_iters + 2; ++it) {
-    k_alloc_eval<<<grid, 256, 0, s>>>(a);
+    if (a.greedy) k_alloc_greedy<<<a.ncells, 32, 0, s>>>(a);
+    else k_alloc_eval<<<grid, 256, 0, s>>>(a);
     JOLT_LAUNCHED();
     k_alloc_decide<<<1, 512, 0, s>>>(a);
     JOLT_LAUNCHED();

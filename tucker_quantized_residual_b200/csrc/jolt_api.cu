@@ -241,6 +241,7 @@ void jolt_default_options(jolt_options* o) {
   o->scale_group = 0;
   o->rotation = JOLT_ROT_HADAMARD;
   o->budget_tol = 0.005;
+  o->minimizer = JOLT_MIN_ENUMERATE;
   o->max_iters = 50;
 }
 
@@ -298,6 +299,7 @@ static jolt_status validate(const jolt_layout* L, const jolt_options* o) {
   int G = o->scale_group ? o->scale_group : L->head_dim;
   if (!(G == 32 || G == 64 || G == 128) || L->head_dim % G) { set_error("scale_group must be 32/64/128 and divide D"); return JOLT_ERR_INVALID_ARG; }
   if (o->budget_tol < 0 || o->budget_tol >= 1 || o->max_iters < 1) { set_error("bad tolerance/max_iters"); return JOLT_ERR_INVALID_ARG; }
+  if (o->minimizer != JOLT_MIN_ENUMERATE && o->minimizer != JOLT_MIN_GREEDY) { set_error("minimizer must be JOLT_MIN_ENUMERATE or JOLT_MIN_GREEDY"); return JOLT_ERR_INVALID_ARG; }
   auto chk = [](int n, const int32_t* g) {
     if (n < 0 || (n > 0 && !g)) return false;
     for (int i = 0; i < n; ++i) if (g[i] < 1 || (i && g[i] <= g[i - 1])) return false;
@@ -917,6 +919,7 @@ static jolt_status run_allocation(jolt_plan_s* p, int64_t budget, const double* 
   st.max_iters = p->opt.max_iters;
   st.phase = 0;
   AllocArgs a{};
+  a.greedy = p->opt.minimizer == JOLT_MIN_GREEDY;
   a.cells = p->d_rd_cells; a.ncells = p->ncells;
   a.rt_grid = p->d_rt; a.rd_grid = p->d_rd; a.n_rd = (int)p->rd_grid.size();
   a.bits = p->d_bits; a.eps2 = eps2; a.rowbytes = p->d_rowbytes; a.n_bits = (int)p->bits.size();

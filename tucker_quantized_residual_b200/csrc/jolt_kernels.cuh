@@ -86,6 +86,7 @@ struct AllocArgs {
   AllocState* st;
   Choice* out;              // [ncells]
   int* status;
+  int greedy;               // 1: the page's greedy per-cell search instead of enumeration
 };
 
 jolt_status launch_alloc(const AllocArgs& a, const AllocState& init, cudaStream_t s);
