@@ -295,6 +295,15 @@ def test_ragged_and_small_shapes(dtype, D, T, rope):
     _compare(K, V, gs, B, rope, bits=(0, 2, 3, 4, 8), scale_group=32)
 
 
+def test_batch_of_sequences_exact():
+    """batch > 1: each sequence has its own cells and seed (seed + sequence
+    index) and all cells share one byte budget."""
+    spec = synth.CacheSpec("batch3", 3, 4, 2, 256, 64, 2, 16, 1.0, 0.02, rope_theta_k=1e4, dtype="bf16")
+    K, V = synth.make_cache(spec, 7)
+    B = o.budget_for_ratio(K.numel() * 2, 2.0)
+    _compare(K, V, synth.group_starts(spec), B, spec.rope_theta_k)
+
+
 def test_all_zero_bits_and_generous_budget():
     spec = synth.SPECS["tiny"]
     K, V = synth.make_cache(spec, 1)

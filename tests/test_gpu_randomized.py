@@ -21,8 +21,8 @@ from gpu_helpers import gpu_compress, oracle_compress
 pytestmark = pytest.mark.gpu
 
 
-def _gate(name, C_ratio, **kw):
-    spec = synth.SPECS[name]
+def _gate(name, C_ratio, spec=None, **kw):
+    spec = spec or synth.SPECS[name]
     K, V = synth.make_cache(spec, 0)
     gs = synth.group_starts(spec)
     B = o.budget_for_ratio(K.numel() * 2, C_ratio)
@@ -54,6 +54,14 @@ def test_mistral_randomized_gate(C_ratio):
     B = o.budget_for_ratio(K.numel() * 2, C_ratio)
     Kn, Vn, Ko, Vo, comp = oracle_compress(K, V, synth.group_starts(spec), B, 0, spec.rope_theta_k)
     print(f"mistral {C_ratio}x uncapped exact K/V {o.rel_frobenius(Kn, Ko):.5f}/{o.rel_frobenius(Vn, Vo):.5f}")
+
+
+def test_moe_batch_randomized_gate():
+    """The MoE/GQA batch shape (groups of 6 layers, 4 KV heads, D = 128,
+    T = 1024), reduced to 2 sequences of 2 groups: every sequence gets its own
+    cells, seeds and allocation under one shared 3x budget in one call."""
+    spec = synth.SPECS["moe_t1024"].replace(batch=2, n_layers=12)
+    _gate("moe_t1024", 3.0, spec=spec)
 
 
 def test_randomized_spectrum_tracks_exact():
