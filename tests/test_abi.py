@@ -22,6 +22,7 @@ def test_default_options_are_the_papers():
     assert list(o.bits[: o.n_bits]) == [0, 2, 4, 8]
     assert o.budget_tol == 0.005 and o.max_iters == 50
     assert o.oversample_p == 8 and o.power_iters == 2 and o.scale_group == 0
+    assert o.minimizer == jolt.JOLT_MIN_ENUMERATE
 
 
 def _layout(D=64, theta=0.0, groups=(0, 2)):
@@ -31,7 +32,7 @@ def _layout(D=64, theta=0.0, groups=(0, 2)):
     return L, gs
 
 
-@pytest.mark.parametrize("bad", ["D", "bits", "group", "grid", "groups"])
+@pytest.mark.parametrize("bad", ["D", "bits", "group", "grid", "groups", "minimizer"])
 def test_plan_rejects_bad_arguments_before_touching_the_device(bad):
     L, keep = _layout()
     o, k2 = jolt.make_options()
@@ -46,6 +47,8 @@ def test_plan_rejects_bad_arguments_before_touching_the_device(bad):
     elif bad == "groups":
         L, keep = _layout(groups=(0, 1))
         L.n_layers = 2
+    elif bad == "minimizer":
+        o.minimizer = 7
     with pytest.raises(jolt.JoltError) as ei:
         jolt.jolt_plan(L, 10 ** 6, o)
     assert ei.value.status in (1, 2)

@@ -13,20 +13,18 @@ struct EighJob {
   double* w;      // n, descending
   double* Vt;     // n*n, row j = eigenvector j (if want_vec)
   double* Z;      // n*n scratch (if want_vec)
-  double* work;   // n scratch (3n for the split solver: d, e, beta)
-  double* F;      // split solver: 5n doubles per requested eigenvector
+  double* work;   // 3n scratch: d, e, beta of the tridiagonal reduction
+  double* F;      // 5n doubles per requested eigenvector (inverse iteration)
 };
 
-jolt_status launch_eigh(const EighJob* jobs_dev, int njobs, int nmax, int* status, cudaStream_t s);
-size_t eigh_smem_bytes(int nmax);
 jolt_status launch_tridiag(const EighJob* jobs, int njobs, int nmax, cudaStream_t s);
 // Multi-block reduction of jobs[0..njobs) (all of size <= nmax); scratch holds
 // njobs * (2 nmax + 128) doubles, counters 2 njobs + 1 words.
 jolt_status launch_tridiag_multi(const EighJob* jobs, int njobs, int nmax, double* scratch, unsigned int* counters,
                                  int* status, cudaStream_t s);
 jolt_status launch_bisect(const EighJob* jobs, int njobs, int nmax, cudaStream_t s);
-jolt_status launch_eigvecs(const EighJob* jobs, int njobs, int nvec_max, const int* nvec, cudaStream_t s);
-// Same, for matrices of size <= nmax (sizes the back-transformation blocks).
+// Eigenvectors of the leading nvec[job] eigenvalues of jobs of size <= nmax
+// (nmax sizes the back-transformation blocks).
 jolt_status launch_eigvecs_n(const EighJob* jobs, int njobs, int nvec_max, int nmax, const int* nvec, cudaStream_t s);
 jolt_status launch_fgram_x(const CellDesc* cells, int ncells, int D, const float2* cs, int nchunk,
                            double* partial, cudaStream_t s);
@@ -174,21 +172,8 @@ jolt_status launch_omega(uint16_t* wt, int ncells, int k, int ld, const int* Nc,
 constexpr int GRAM_SPLIT = 4;   // K slices of the fp64 Gram (partials in a scratch buffer)
 jolt_status launch_gram_cols(const float* A, int64_t a_cell, const int* rows_of, int k, double* C, int64_t c_cell,
                              int ncells, double* part, cudaStream_t s);
-jolt_status launch_cholesky(double* A, int64_t a_cell, const float* src32, int64_t s_cell, int k, int ncells,
-                            int* status, cudaStream_t s);
-jolt_status launch_trsm_rows(const float* Z, int64_t z_cell, const double* R, int64_t r_cell, int k, const int* Nc,
-                             int Ncmax, uint16_t* Wt, int64_t w_cell, int ldw, double* scratch, int64_t s_cell,
-                             int ncells, cudaStream_t s);
-jolt_status launch_orth_apply(const double* R, int64_t r_cell, int k, float* Ri, double* X, int64_t x_cell,
-                              const float* Z, int64_t z_cell, const int* Nc, int Ncmax, uint16_t* Wt, int64_t w_cell,
-                              int ldw, int ncells, cudaStream_t s);
-jolt_status launch_bbt(const double* R, const double* P, double* X1, double* M, int64_t cs, int k, int ncells,
-                       cudaStream_t s);
 jolt_status launch_rand_spectrum(const double* w_eig, int64_t cs, int q, const double* const* normsq,
                                  double* const* wT, int ncells, cudaStream_t s);
-jolt_status launch_make_p(const double* R, const double* Vt, int64_t cs, int k, const CellOut* outs, double* P64,
-                          int64_t p_cell, int rmax, uint16_t* Pt, int64_t pt_cell, int ldp, int ncells,
-                          cudaStream_t s);
 jolt_status launch_yproj(const float* Z, int64_t z_cell, const double* P64, int64_t p_cell, int k, int rmax,
                          const CellOut* outs, const int* nlh, double* const* Y, int lh_max, int D, int ncells,
                          cudaStream_t s);

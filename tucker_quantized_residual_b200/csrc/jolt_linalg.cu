@@ -241,206 +241,6 @@ __global__ void __launch_bounds__(256) k_token_gram(const CellDesc* __restrict__
 // Outputs: w[n]; Vt[j*n + i] = component i of eigenvector j (if want_vec).
 constexpr int EIG_THREADS = 512;
 
-__global__ void __launch_bounds__(EIG_THREADS) k_eigh(const EighJob* __restrict__ jobs, int* status) {
-  const EighJob J = jobs[blockIdx.x];
-  const int n = J.n;
-  if (n <= 0) return;
-  extern __shared__ double sh[];
-  double* v = sh;            // n
-  double* p = v + n;         // n
-  double* dd = p + n;        // n   diagonal
-  double* ee = dd + n;       // n   off-diagonal
-  double* rc = ee + n;       // n   rotation cosines of the current sweep
-  double* rs = rc + n;       // n   rotation sines
-  double* red = rs + n;      // 32
-  __shared__ int ctl[4];
-  double* A = J.A;
-  double* tau = J.work;      // n
-  double* Z = J.Z;           // Z[j*n + i] = component i of vector j
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const int lane = tid & 31, warp = tid >> 5, nwarp = nt >> 5;
-
-  // ---- 1. tridiagonalization
-  for (int k = 0; k + 2 < n; ++k) {
-    const int m = n - k - 1;
-    for (int i = tid; i < m; i += nt) v[i] = A[(int64_t)(k + 1 + i) * n + k];
-    __syncthreads();
-    double s = 0.0;
-    for (int i = 1 + tid; i < m; i += nt) s += v[i] * v[i];
-    s = block_sum(s, red);
-    const double x0 = v[0];
-    if (s == 0.0) {
-      if (tid == 0) { dd[k] = A[(int64_t)k * n + k]; ee[k] = x0; tau[k] = 0.0; }
-      __syncthreads();
-      continue;
-    }
-    const double nrm = sqrt(x0 * x0 + s);
-    const double alpha = (x0 <= 0.0) ? nrm : -nrm;
-    const double v0 = x0 - alpha;
-    const double beta = 2.0 / (s + v0 * v0);
-    __syncthreads();
-    if (tid == 0) v[0] = v0;
-    __syncthreads();
-    // p = beta A22 v
-    for (int i = warp; i < m; i += nwarp) {
-      const double* row = A + (int64_t)(k + 1 + i) * n + (k + 1);
-      double acc = 0.0;
-      for (int j = lane; j < m; j += 32) acc += row[j] * v[j];
-      acc = warp_sum(acc);
-      if (lane == 0) p[i] = beta * acc;
-    }
-    __syncthreads();
-    double pv = 0.0;
-    for (int i = tid; i < m; i += nt) pv += p[i] * v[i];
-    const double Kc = 0.5 * beta * block_sum(pv, red);
-    for (int i = tid; i < m; i += nt) p[i] -= Kc * v[i];
-    __syncthreads();
-    // A22 -= v w^T + w v^T
-    for (int i = warp; i < m; i += nwarp) {
-      double* row = A + (int64_t)(k + 1 + i) * n + (k + 1);
-      const double vi = v[i], wi = p[i];
-      for (int j = lane; j < m; j += 32) row[j] -= vi * p[j] + wi * v[j];
-    }
-    if (tid == 0) { dd[k] = A[(int64_t)k * n + k]; ee[k] = alpha; tau[k] = beta; }
-    for (int i = tid; i < m; i += nt) A[(int64_t)(k + 1 + i) * n + k] = v[i];
-    __syncthreads();
-  }
-  if (tid == 0) {
-    if (n >= 2) {
-      dd[n - 2] = A[(int64_t)(n - 2) * n + (n - 2)];
-      ee[n - 2] = A[(int64_t)(n - 1) * n + (n - 2)];
-    }
-    dd[n - 1] = A[(int64_t)(n - 1) * n + (n - 1)];
-    ee[n - 1] = 0.0;
-  }
-  if (J.want_vec)
-    for (int64_t e = tid; e < (int64_t)n * n; e += nt) Z[e] = ((e / n) == (e % n)) ? 1.0 : 0.0;
-  __syncthreads();
-
-  // ---- 2. implicit QL
-  // A sub-diagonal entry is negligible when it is tiny next to its two
-  // diagonal neighbours or next to the whole matrix (norm bound anorm); the
-  // second test deflates clusters of (numerically) zero eigenvalues, which a
-  // purely relative test would iterate on forever.
-  double anorm = 0.0;
-  if (tid == 0)
-    for (int i = 0; i < n; ++i) anorm = fmax(anorm, fabs(dd[i]) + fabs(ee[i]));
-  for (int l = 0; l < n; ++l) {
-    int iter = 0;
-    while (true) {
-      if (tid == 0) {
-        int m = l;
-        for (; m < n - 1; ++m) {
-          double s2 = fabs(dd[m]) + fabs(dd[m + 1]);
-          if (fabs(ee[m]) <= 2.220446049250313e-16 * s2 || fabs(ee[m]) <= 2.220446049250313e-16 * anorm) break;
-        }
-        if (m == l) {
-          ctl[0] = 1;
-        } else if (++iter > 90) {
-          atomicOr(status, DEV_ERR_EIG_NOCONV);
-          ctl[0] = 1;
-        } else {
-          double g = (dd[l + 1] - dd[l]) / (2.0 * ee[l]);
-          double r = hypot(g, 1.0);
-          g = dd[m] - dd[l] + ee[l] / (g + copysign(r, g));
-          double s = 1.0, cc = 1.0, pp = 0.0;
-          int i = m - 1;
-          bool early = false;
-          for (; i >= l; --i) {
-            double f = s * ee[i], b = cc * ee[i];
-            r = hypot(f, g);
-            ee[i + 1] = r;
-            if (r == 0.0) { dd[i + 1] -= pp; ee[m] = 0.0; early = true; break; }
-            s = f / r;
-            cc = g / r;
-            g = dd[i + 1] - pp;
-            r = (dd[i] - g) * s + 2.0 * cc * b;
-            pp = s * r;
-            dd[i + 1] = g + pp;
-            g = cc * r - b;
-            rc[i] = cc;
-            rs[i] = s;
-          }
-          if (!early) { dd[l] -= pp; ee[l] = g; ee[m] = 0.0; ctl[2] = l; }
-          else ctl[2] = i + 1;
-          ctl[0] = 0;
-          ctl[1] = m - 1;
-        }
-      }
-      __syncthreads();
-      if (ctl[0]) { __syncthreads(); break; }
-      if (J.want_vec) {
-        const int hi = ctl[1], lo = ctl[2];
-        for (int r = tid; r < n; r += nt) {
-          double z1 = Z[(int64_t)(hi + 1) * n + r];
-          for (int i = hi; i >= lo; --i) {
-            double zi = Z[(int64_t)i * n + r];
-            Z[(int64_t)(i + 1) * n + r] = rs[i] * zi + rc[i] * z1;
-            z1 = rc[i] * zi - rs[i] * z1;
-          }
-          if (hi >= lo) Z[(int64_t)lo * n + r] = z1;
-        }
-      }
-      __syncthreads();
-    }
-  }
-
-  // ---- 3. back-transformation
-  if (J.want_vec) {
-    for (int k = n - 3; k >= 0; --k) {
-      const double beta = tau[k];
-      if (beta == 0.0) continue;
-      const int m = n - k - 1;
-      for (int i = tid; i < m; i += nt) v[i] = A[(int64_t)(k + 1 + i) * n + k];
-      __syncthreads();
-      for (int j = warp; j < n; j += nwarp) {
-        double* z = Z + (int64_t)j * n + (k + 1);
-        double acc = 0.0;
-        for (int i = lane; i < m; i += 32) acc += v[i] * z[i];
-        acc = beta * warp_sum(acc);
-        for (int i = lane; i < m; i += 32) z[i] -= acc * v[i];
-      }
-      __syncthreads();
-    }
-  }
-
-  // ---- 4. sort descending, fix signs, write out
-  for (int i = tid; i < n; i += nt) {
-    const double di = dd[i];
-    int rank = 0;
-    for (int j = 0; j < n; ++j) {
-      const double dj = dd[j];
-      rank += (dj > di) || (dj == di && j < i);
-    }
-    J.w[rank] = di;
-    p[i] = (double)rank;
-  }
-  __syncthreads();
-  if (J.want_vec) {
-    for (int j = warp; j < n; j += nwarp) {
-      const double* z = Z + (int64_t)j * n;
-      double best = -1.0;
-      int bi = 0x7fffffff;
-      for (int i = lane; i < n; i += 32) {
-        double a = fabs(z[i]);
-        if (a > best) { best = a; bi = i; }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        double ob = __shfl_xor_sync(0xffffffffu, best, o);
-        int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
-      }
-      const double sg = (z[bi] < 0.0) ? -1.0 : 1.0;
-      const int rank = (int)p[j];
-      double* dst = J.Vt + (int64_t)rank * n;
-      for (int i = lane; i < n; i += 32) dst[i] = sg * z[i];
-    }
-  }
-}
-
-size_t eigh_smem_bytes(int nmax) { return (size_t)(6 * nmax + 32) * sizeof(double); }
-
 // ------------------------------------------- split eigensolver (big n) -----
 // For the token-mode matrices only the spectrum is needed before the
 // allocation and only the leading r_T eigenvectors after it, so the solver is
@@ -1010,10 +810,6 @@ jolt_status launch_bisect(const EighJob* jobs, int njobs, int nmax, cudaStream_t
   return JOLT_OK;
 }
 
-jolt_status launch_eigvecs(const EighJob* jobs, int njobs, int nvec_max, const int* nvec, cudaStream_t s) {
-  return launch_eigvecs_n(jobs, njobs, nvec_max, 2048, nvec, s);
-}
-
 jolt_status launch_eigvecs_n(const EighJob* jobs, int njobs, int nvec_max, int nmax, const int* nvec, cudaStream_t s) {
   if (nvec_max <= 0 || njobs <= 0) return JOLT_OK;
   if (nmax > 256 * BT_PRE) { set_error("eigenvectors need n <= %d (n=%d)", 256 * BT_PRE, nmax); return JOLT_ERR_UNSUPPORTED_SHAPE; }
@@ -1024,14 +820,6 @@ jolt_status launch_eigvecs_n(const EighJob* jobs, int njobs, int nvec_max, int n
   const size_t smem = (size_t)(vb + 2) * nmax * sizeof(double);
   { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_backtr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
   k_backtr<<<dim3((nvec_max + vb - 1) / vb, njobs), 256, smem, s>>>(jobs, nvec, vb);
-  JOLT_LAUNCHED();
-  return JOLT_OK;
-}
-
-jolt_status launch_eigh(const EighJob* jobs_dev, int njobs, int nmax, int* status, cudaStream_t s) {
-  size_t smem = eigh_smem_bytes(nmax);
-  { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_eigh, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
-  k_eigh<<<njobs, EIG_THREADS, smem, s>>>(jobs_dev, status);
   JOLT_LAUNCHED();
   return JOLT_OK;
 }

@@ -251,213 +251,6 @@ jolt_status launch_omega(uint16_t* wt, int ncells, int k, int ld, const int* Nc,
   return JOLT_OK;
 }
 
-// ----------------------------------------------------------- Cholesky ------
-// In place: A (k x k fp64 symmetric, or fp32 source copied in) becomes R
-// (upper triangular, A = R^T R). A relative diagonal shift of 1e-13 trace/k
-// keeps a numerically rank-deficient sketch factorizable (shifted
-// CholeskyQR); a non-positive pivot is still reported.
-__global__ void __launch_bounds__(512) k_cholesky(double* __restrict__ A, int64_t a_cell, const float* __restrict__ src32,
-                                                  int64_t s_cell, int k, int* status) {
-  double* a = A + (int64_t)blockIdx.x * a_cell;
-  __shared__ double inv_piv;
-  __shared__ double red[32];
-  if (src32) {
-    const float* s32 = src32 + (int64_t)blockIdx.x * s_cell;
-    for (int64_t e = threadIdx.x; e < (int64_t)k * k; e += blockDim.x) a[e] = (double)s32[e];
-    __syncthreads();
-  }
-  double tr = 0.0;
-  for (int i = threadIdx.x; i < k; i += blockDim.x) tr += a[(int64_t)i * k + i];
-  // block sum
-  for (int o = 16; o > 0; o >>= 1) tr += __shfl_xor_sync(0xffffffffu, tr, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = tr;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double t = 0.0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
-    red[0] = t;
-  }
-  __syncthreads();
-  // an all-zero Gram (an all-zero cell) factors as the identity: any R works
-  // because the columns it orthonormalizes are zero
-  const double shift = (red[0] > 0.0) ? 1e-13 * red[0] / k : 1.0;
-  for (int i = threadIdx.x; i < k; i += blockDim.x) a[(int64_t)i * k + i] += shift;
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int j = 0; j < k; ++j) {
-    if (threadIdx.x == 0) {
-      double piv = a[(int64_t)j * k + j];
-      if (!(piv > 0.0)) { atomicOr(status, DEV_ERR_CHOL); piv = fmax(shift, 1e-300); }
-      const double r = sqrt(piv);
-      a[(int64_t)j * k + j] = r;
-      inv_piv = 1.0 / r;
-    }
-    __syncthreads();
-    for (int i = j + 1 + threadIdx.x; i < k; i += blockDim.x) a[(int64_t)j * k + i] *= inv_piv;
-    __syncthreads();
-    for (int i = j + 1 + warp; i < k; i += nw) {
-      const double rji = a[(int64_t)j * k + i];
-      double* row = a + (int64_t)i * k;
-      const double* rj = a + (int64_t)j * k;
-      for (int l = i + lane; l < k; l += 32) row[l] -= rji * rj[l];
-    }
-    __syncthreads();
-  }
-  for (int64_t e = threadIdx.x; e < (int64_t)k * k; e += blockDim.x)
-    if (e / k > e % k) a[e] = 0.0;
-}
-
-jolt_status launch_cholesky(double* A, int64_t a_cell, const float* src32, int64_t s_cell, int k, int ncells,
-                            int* status, cudaStream_t s) {
-  k_cholesky<<<ncells, 512, 0, s>>>(A, a_cell, src32, s_cell, k, status);
-  JOLT_LAUNCHED();
-  return JOLT_OK;
-}
-
-// ------------------------------------------------------ triangular solves --
-// V = Z R^{-1} row by row (forward substitution on R^T), stored transposed in
-// bf16: Wt[cell][j][n] for n < N_c. Z fp32 [cell][Ncmax][k].
-__global__ void k_trsm_rows(const float* __restrict__ Z, int64_t z_cell, const double* __restrict__ R, int64_t r_cell,
-                            int k, const int* __restrict__ Nc, uint16_t* __restrict__ Wt, int64_t w_cell, int ldw,
-                            double* __restrict__ scratch, int64_t s_cell) {
-  const int cell = blockIdx.y;
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= Nc[cell]) return;
-  const float* z = Z + (int64_t)cell * z_cell + (int64_t)n * k;
-  const double* r = R + (int64_t)cell * r_cell;
-  double* v = scratch + (int64_t)cell * s_cell + (int64_t)n * k;
-  uint16_t* w = Wt + (int64_t)cell * w_cell + n;
-  for (int j = 0; j < k; ++j) {
-    double acc = (double)z[j];
-    for (int i = 0; i < j; ++i) acc -= v[i] * r[(int64_t)i * k + j];
-    const double x = acc / r[(int64_t)j * k + j];
-    v[j] = x;
-    w[(int64_t)j * ldw] = bf16_bits_from_f64(x);
-  }
-}
-
-jolt_status launch_trsm_rows(const float* Z, int64_t z_cell, const double* R, int64_t r_cell, int k, const int* Nc,
-                             int Ncmax, uint16_t* Wt, int64_t w_cell, int ldw, double* scratch, int64_t s_cell,
-                             int ncells, cudaStream_t s) {
-  dim3 g((Ncmax + 127) / 128, ncells);
-  k_trsm_rows<<<g, 128, 0, s>>>(Z, z_cell, R, r_cell, k, Nc, Wt, w_cell, ldw, scratch, s_cell);
-  JOLT_LAUNCHED();
-  return JOLT_OK;
-}
-
-// R^{-1} of the upper triangular R (fp64), one column per thread by back
-// substitution, stored as fp32 [k][k] for the product below.
-__global__ void k_tri_inv(const double* __restrict__ R, int64_t r_cell, int k, float* __restrict__ Ri,
-                          double* __restrict__ X, int64_t x_cell) {
-  const int cell = blockIdx.y, c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= k) return;
-  const double* r = R + (int64_t)cell * r_cell;
-  double* x = X + (int64_t)cell * x_cell;
-  float* ri = Ri + (int64_t)cell * k * k;
-  for (int i = k - 1; i >= 0; --i) {
-    double acc = (i == c) ? 1.0 : 0.0;
-    if (i <= c) {
-      for (int l = i + 1; l <= c; ++l) acc -= r[(int64_t)i * k + l] * x[(int64_t)l * k + c];
-      acc /= r[(int64_t)i * k + i];
-    } else {
-      acc = 0.0;
-    }
-    x[(int64_t)i * k + c] = acc;
-    ri[(int64_t)i * k + c] = (float)acc;
-  }
-}
-
-// W^T[cell][j][n] = bf16( sum_i Z[cell][n][i] Ri[cell][i][j] ), fp32 tiles of
-// 64 (n) x 64 (j), 4 x 4 outputs per thread.
-__global__ void __launch_bounds__(256) k_z_rinv(const float* __restrict__ Z, int64_t z_cell, const float* __restrict__ Ri,
-                                                int k, const int* __restrict__ Nc, uint16_t* __restrict__ Wt,
-                                                int64_t w_cell, int ldw) {
-  constexpr int TB = 64, KB = 16;
-  __shared__ float As[KB][TB + 4];
-  __shared__ float Bs[KB][TB + 4];
-  const int cell = blockIdx.z;
-  const int n0 = blockIdx.x * TB, j0 = blockIdx.y * TB;
-  const int nc = Nc[cell];
-  if (n0 >= nc || j0 >= k) return;
-  const float* z = Z + (int64_t)cell * z_cell;
-  const float* ri = Ri + (int64_t)cell * k * k;
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
-  float acc[4][4] = {};
-  const int iend = min(k, j0 + TB);          // Ri is upper triangular: i <= j
-  for (int i0 = 0; i0 < iend; i0 += KB) {
-    for (int e = threadIdx.x; e < KB * TB; e += blockDim.x) {
-      const int kk = e % KB, nn = e / KB;
-      const int n = n0 + nn, i = i0 + kk;
-      As[kk][nn] = (n < nc && i < k) ? z[(int64_t)n * k + i] : 0.0f;
-      const int jj = e % TB, k2 = e / TB;
-      const int j = j0 + jj, i2 = i0 + k2;
-      Bs[k2][jj] = (j < k && i2 < k) ? ri[(int64_t)i2 * k + j] : 0.0f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < KB; ++kk) {
-      float a[4], b[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) { a[q] = As[kk][ty * 4 + q]; b[q] = Bs[kk][tx * 4 + q]; }
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(a[p], b[q], acc[p][q]);
-    }
-    __syncthreads();
-  }
-  uint16_t* w = Wt + (int64_t)cell * w_cell;
-#pragma unroll
-  for (int p = 0; p < 4; ++p)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int n = n0 + ty * 4 + p, j = j0 + tx * 4 + q;
-      if (n < nc && j < k) w[(int64_t)j * ldw + n] = bf16_bits_from_f32(acc[p][q]);
-    }
-}
-
-jolt_status launch_orth_apply(const double* R, int64_t r_cell, int k, float* Ri, double* X, int64_t x_cell,
-                              const float* Z, int64_t z_cell, const int* Nc, int Ncmax, uint16_t* Wt, int64_t w_cell,
-                              int ldw, int ncells, cudaStream_t s) {
-  dim3 g1((k + 127) / 128, ncells);
-  k_tri_inv<<<g1, 128, 0, s>>>(R, r_cell, k, Ri, X, x_cell);
-  JOLT_LAUNCHED();
-  dim3 g2((Ncmax + 63) / 64, (k + 63) / 64, ncells);
-  k_z_rinv<<<g2, 256, 0, s>>>(Z, z_cell, Ri, k, Nc, Wt, w_cell, ldw);
-  JOLT_LAUNCHED();
-  return JOLT_OK;
-}
-
-// X1 = R^{-T} P (column c per thread, forward substitution), then
-// M = X1 R^{-1} (row per thread), symmetrized into M.
-__global__ void k_solve_left_t(const double* __restrict__ R, const double* __restrict__ P, double* __restrict__ X1,
-                               int64_t cs, int k) {
-  const int cell = blockIdx.y, c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= k) return;
-  const double* r = R + (int64_t)cell * cs;
-  const double* p = P + (int64_t)cell * cs;
-  double* x = X1 + (int64_t)cell * cs;
-  for (int i = 0; i < k; ++i) {
-    double acc = p[(int64_t)i * k + c];
-    for (int l = 0; l < i; ++l) acc -= r[(int64_t)l * k + i] * x[(int64_t)l * k + c];
-    x[(int64_t)i * k + c] = acc / r[(int64_t)i * k + i];
-  }
-}
-
-__global__ void k_solve_right(const double* __restrict__ R, const double* __restrict__ X1, double* __restrict__ M,
-                              int64_t cs, int k) {
-  const int cell = blockIdx.y, row = blockIdx.x * blockDim.x + threadIdx.x;
-  if (row >= k) return;
-  const double* r = R + (int64_t)cell * cs;
-  const double* x = X1 + (int64_t)cell * cs + (int64_t)row * k;
-  double* m = M + (int64_t)cell * cs + (int64_t)row * k;
-  for (int j = 0; j < k; ++j) {
-    double acc = x[j];
-    for (int i = 0; i < j; ++i) acc -= m[i] * r[(int64_t)i * k + j];
-    m[j] = acc / r[(int64_t)j * k + j];
-  }
-}
-
 __global__ void k_symmetrize(double* __restrict__ M, int64_t cs, int k) {
   const int cell = blockIdx.y;
   double* m = M + (int64_t)cell * cs;
@@ -472,19 +265,6 @@ __global__ void k_symmetrize(double* __restrict__ M, int64_t cs, int k) {
 }
 
 jolt_status launch_symmetrize(double* M, int64_t cs, int k, int ncells, cudaStream_t s) {
-  dim3 g2(64, ncells);
-  k_symmetrize<<<g2, 256, 0, s>>>(M, cs, k);
-  JOLT_LAUNCHED();
-  return JOLT_OK;
-}
-
-jolt_status launch_bbt(const double* R, const double* P, double* X1, double* M, int64_t cs, int k, int ncells,
-                       cudaStream_t s) {
-  dim3 g((k + 127) / 128, ncells);
-  k_solve_left_t<<<g, 128, 0, s>>>(R, P, X1, cs, k);
-  JOLT_LAUNCHED();
-  k_solve_right<<<g, 128, 0, s>>>(R, X1, M, cs, k);
-  JOLT_LAUNCHED();
   dim3 g2(64, ncells);
   k_symmetrize<<<g2, 256, 0, s>>>(M, cs, k);
   JOLT_LAUNCHED();
@@ -511,35 +291,6 @@ __global__ void k_rand_spectrum(const double* __restrict__ w_eig, int64_t cs, in
 jolt_status launch_rand_spectrum(const double* w_eig, int64_t cs, int q, const double* const* normsq,
                                  double* const* wT, int ncells, cudaStream_t s) {
   k_rand_spectrum<<<ncells, 32, 0, s>>>(w_eig, cs, q, normsq, wT);
-  JOLT_LAUNCHED();
-  return JOLT_OK;
-}
-
-// P = R^{-1} U_B[:, :r_T] by back substitution, one column per thread:
-// P64[cell][i][r] (fp64) and Pt[cell][r][i] (bf16, row pitch ldp).
-__global__ void k_make_p(const double* __restrict__ R, const double* __restrict__ Vt, int64_t cs, int k,
-                         const CellOut* __restrict__ outs, double* __restrict__ P64, int64_t p_cell, int rmax,
-                         uint16_t* __restrict__ Pt, int64_t pt_cell, int ldp) {
-  const int cell = blockIdx.y, c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= outs[cell].rT) return;
-  const double* r = R + (int64_t)cell * cs;
-  const double* u = Vt + (int64_t)cell * cs + (int64_t)c * k;    // eigenvector c
-  double* p = P64 + (int64_t)cell * p_cell;
-  uint16_t* pt = Pt + (int64_t)cell * pt_cell + (int64_t)c * ldp;
-  for (int i = k - 1; i >= 0; --i) {
-    double acc = u[i];
-    for (int l = i + 1; l < k; ++l) acc -= r[(int64_t)i * k + l] * p[(int64_t)l * rmax + c];
-    const double x = acc / r[(int64_t)i * k + i];
-    p[(int64_t)i * rmax + c] = x;
-    pt[i] = bf16_bits_from_f64(x);
-  }
-}
-
-jolt_status launch_make_p(const double* R, const double* Vt, int64_t cs, int k, const CellOut* outs, double* P64,
-                          int64_t p_cell, int rmax, uint16_t* Pt, int64_t pt_cell, int ldp, int ncells,
-                          cudaStream_t s) {
-  dim3 g((rmax + 127) / 128, ncells);
-  k_make_p<<<g, 128, 0, s>>>(R, Vt, cs, k, outs, P64, p_cell, rmax, Pt, pt_cell, ldp);
   JOLT_LAUNCHED();
   return JOLT_OK;
 }
