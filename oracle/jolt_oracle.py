@@ -14,6 +14,8 @@ via Joint Rank-bit Allocation" (Krishnan & Schulz), Section 3:
                                        greedy_cell (the page's own heuristic)
   * Section 3.1 "FlashJoLT", Eq. (5) -> q_cap (the randomized mode itself is
                                        not in the oracle: the oracle is exact)
+  * Section 3, layer grouping        -> layer_token_basis, basis_score,
+                                       layer_scores, group_layers
 and, for keys, the pre-RoPE handling of Section 3 (keys decomposed before the
 rotary embedding; the rotation re-applied to the reconstruction).
 
@@ -49,6 +51,12 @@ library as well):
   R8 budget C: B = floor(dense bf16 bytes of K and V / C).
   R9 an option with r_d > |g| n_h r_T is excluded (multilinear rank of the
      core; see CellTable.valid).
+  R12 layer score: "mean squared cosine between their bases" is the mean of
+     cos^2 over the 8 principal angles, ||U_l^T U_(l+1)||_F^2 / 8.
+  R13 a layer whose keys are all zero has the zero basis (score 0 with both
+     neighbours); below rank 8 the trailing basis vectors are arbitrary.
+  R14 with a batch, the score of (l, l+1) is the mean over sequences.
+  R15 median of the L-1 scores as numpy computes it; "falls below" is strict.
 """
 from __future__ import annotations
 
@@ -727,3 +735,86 @@ def rel_frobenius(X: np.ndarray, Xh: np.ndarray) -> float:
 def budget_for_ratio(n_elems_kv: int, C: float) -> int:
     """Reading R8: B = floor(2 bytes * (elements of K and V) / C)."""
     return int(math.floor(2.0 * n_elems_kv / C))
+
+
+# --------------------------------------------------------------------------
+# data-driven layer grouping, Section 3 (the paragraph before "Partial Tucker
+# backbone" and its footnote on the size bounds); readings R12-R15
+# --------------------------------------------------------------------------
+GROUP_VECTORS = 8        # "the top eight token-mode singular vectors"
+GROUP_MIN = 2            # a new group opens only once the current one has >= 2 layers
+GROUP_MAX = 8            # a group is closed at eight layers
+
+
+def layer_keys(cache_k: np.ndarray, b: int, l: int, rope_theta_k: float) -> np.ndarray:
+    """Layer l's key cache of sequence b as [1, H, T, D] fp64: the keys the
+    method decomposes, i.e. before RoPE (the inverse rotation of reading R6
+    when the cache holds post-RoPE keys)."""
+    X = f32(cache_k[b, l:l + 1])
+    if rope_theta_k > 0:
+        cs, sn = rope_table(X.shape[2], X.shape[3], rope_theta_k)
+        X = unrope_f32(X, cs, sn)
+    return X.astype(np.float64)
+
+
+def layer_token_basis(X: np.ndarray, r: int = GROUP_VECTORS) -> np.ndarray:
+    """T x r: the top-r left singular vectors of the token unfolding X_(T)
+    (exact, via token_spectrum). Reading R13: a layer whose keys are all zero
+    has no singular vectors; its basis is the zero matrix."""
+    if not np.any(X):
+        return np.zeros((X.shape[2], r))
+    _, U = token_spectrum(X, r_needed=r)
+    return U[:, :r]
+
+
+def basis_score(Ua: np.ndarray, Ub: np.ndarray) -> float:
+    """Reading R12: the mean squared cosine between two r-column orthonormal
+    bases is the mean of cos^2 over the r principal angles between the
+    spanned subspaces, (1/r) ||Ua^T Ub||_F^2 (independent of the choice of
+    basis inside each subspace)."""
+    M = Ua.T @ Ub
+    return float(np.sum(M * M)) / Ua.shape[1]
+
+
+def layer_scores(cache_k: np.ndarray, rope_theta_k: float = 0.0) -> np.ndarray:
+    """Score of consecutive layers (l, l+1), l = 0..L-2. Reading R14: with a
+    batch of sequences the score is the mean of the per-sequence scores
+    (the groups are shared by every sequence of the batch)."""
+    B, L = cache_k.shape[0], cache_k.shape[1]
+    s = np.zeros(max(L - 1, 0))
+    for b in range(B):
+        U = [layer_token_basis(layer_keys(cache_k, b, l, rope_theta_k)) for l in range(L)]
+        for l in range(L - 1):
+            s[l] += basis_score(U[l], U[l + 1])
+    return s / B
+
+
+def group_layers(scores: Sequence[float]) -> List[int]:
+    """Group starts (0 first, L last) from the L-1 consecutive scores.
+    A new group starts at layer l when score(l-1, l) falls strictly below the
+    median of all scores (numpy's median: the mean of the two middle values
+    for an even count; reading R15), but only once the current group holds
+    GROUP_MIN layers; a group that reached GROUP_MAX layers is closed
+    whatever the score; a trailing group of one layer joins its predecessor."""
+    L = len(scores) + 1
+    if L == 1:
+        return [0, 1]
+    med = float(np.median(np.asarray(scores, np.float64)))
+    starts = [0]
+    size = 1
+    for l in range(1, L):
+        s = float(scores[l - 1])
+        if size >= GROUP_MAX or (size >= GROUP_MIN and s < med):
+            starts.append(l)
+            size = 1
+        else:
+            size += 1
+    if len(starts) > 1 and L - starts[-1] == 1:
+        starts.pop()
+    return starts + [L]
+
+
+def layer_groups(cache_k: np.ndarray, rope_theta_k: float = 0.0) -> Tuple[List[int], np.ndarray]:
+    """(group starts, scores) for a key cache [B, L, H, T, D]."""
+    s = layer_scores(cache_k, rope_theta_k)
+    return group_layers(s), s

@@ -124,3 +124,73 @@ def test_backbone_without_feature_factor(monkeypatch):
         return f
     monkeypatch.setattr(o, "fit", bad)
     _fails(pins.test_factors_orthonormal)
+
+
+# ----------------------------------------------------- layer grouping plants
+import test_oracle_grouping as gpins
+
+
+def test_feature_mode_basis(monkeypatch):
+    def bad(X, r=o.GROUP_VECTORS):
+        # right singular vectors (feature mode) instead of token mode
+        _, _, vt = np.linalg.svd(o.token_unfolding(X), full_matrices=False)
+        return vt[:r].T
+    monkeypatch.setattr(o, "layer_token_basis", bad)
+    _fails(gpins.test_layer_scores_recover_planted_overlaps)
+
+
+def test_score_summed_not_averaged(monkeypatch):
+    monkeypatch.setattr(o, "basis_score", lambda a, b: float(np.sum((a.T @ b) ** 2)))
+    _fails(gpins.test_score_of_bases_sharing_m_columns, 3)
+
+
+def test_rope_not_undone(monkeypatch):
+    monkeypatch.setattr(o, "layer_keys", lambda K, b, l, th: np.asarray(K[b, l:l + 1], np.float64))
+    _fails(gpins.test_rope_keys_scored_before_rope)
+
+
+def _rule(lower_median=False, le=False, merge=True, min_size=2, max_size=8):
+    def rule(scores):
+        L = len(scores) + 1
+        if L == 1:
+            return [0, 1]
+        srt = sorted(scores)
+        med = srt[(len(srt) - 1) // 2] if lower_median else float(np.median(scores))
+        starts, size = [0], 1
+        for l in range(1, L):
+            s = scores[l - 1]
+            below = s <= med if le else s < med
+            if size >= max_size or (size >= min_size and below):
+                starts.append(l)
+                size = 1
+            else:
+                size += 1
+        if merge and len(starts) > 1 and L - starts[-1] == 1:
+            starts.pop()
+        return starts + [L]
+    return rule
+
+
+def test_rule_lower_median(monkeypatch):
+    monkeypatch.setattr(o, "group_layers", _rule(lower_median=True))
+    _fails(gpins.test_even_count_median_is_mean_of_middle_pair)
+
+
+def test_rule_not_strict(monkeypatch):
+    monkeypatch.setattr(o, "group_layers", _rule(le=True))
+    _fails(gpins.test_equal_to_median_does_not_split)
+
+
+def test_rule_no_trailing_merge(monkeypatch):
+    monkeypatch.setattr(o, "group_layers", _rule(merge=False))
+    _fails(gpins.test_trailing_single_layer_joins_predecessor)
+
+
+def test_rule_no_minimum_size(monkeypatch):
+    monkeypatch.setattr(o, "group_layers", _rule(min_size=1))
+    _fails(gpins.test_low_score_ignored_until_group_holds_two_layers)
+
+
+def test_rule_size_cap_off_by_one(monkeypatch):
+    monkeypatch.setattr(o, "group_layers", _rule(max_size=9))
+    _fails(gpins.test_equal_scores_close_groups_at_eight)
