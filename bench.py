@@ -57,6 +57,7 @@ def parse():
                     help="only the first N layer groups of the config (small profiling cases)")
     ap.add_argument("--cpu-tokens", type=int, default=4096, help="tokens in the CPU baseline sample")
     ap.add_argument("--stages", action="store_true", help="print the per-stage table to stderr")
+    ap.add_argument("--no-grouping", action="store_true", help="skip the layer-grouping measurement")
     return ap.parse_args()
 
 
@@ -171,6 +172,40 @@ def throughput_gbs(world, dense_bytes, steps, ms):
     return world * dense_bytes * steps / (ms / 1e3) / 1e9
 
 
+# fp32 lanes per SM (4 partitions x 32) on B200; with 148 SMs and the 1965 MHz
+# boost clock this is the fp32 FMA ceiling of the grouping's sketch passes
+FP32_LANES_PER_SM = 128
+
+
+def time_grouping(jolt, K, spec, stream, power_iters=4, reps=3):
+    """jolt_layer_groups on the resident key cache: device time per call
+    (CUDA events on the launching stream, one warm-up call). Each call makes
+    2 * power_iters + 2 passes over the keys (X Z and X^T Q, 16 columns, fp32
+    FMAs); the roofline is that FMA work against the fp32 ALU peak."""
+    import torch
+    jolt.jolt_layer_groups(K, spec.rope_theta_k, power_iters, 0, stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        starts, _s = jolt.jolt_layer_groups(K, spec.rope_theta_k, power_iters, 0, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    passes = 2 * power_iters + 2
+    flops = passes * 2.0 * K.numel() * 16
+    key_bytes = K.numel() * K.element_size()
+    sm = torch.cuda.get_device_properties(K.device).multi_processor_count
+    peak = sm * FP32_LANES_PER_SM * 2 * 1.965e9 / 1e12
+    ach = flops / (ms / 1e3) / 1e12
+    return {"ms_per_call": round(ms, 3), "power_iters": power_iters, "passes_over_keys": passes,
+            "n_groups": len(starts) - 1,
+            "roofline": {"bound": "alu", "achieved": round(ach, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                         "frac": round(ach / peak, 3),
+                         "peak_source": f"derived: {sm} SMs x {FP32_LANES_PER_SM} fp32 lanes x 2 x 1965 MHz",
+                         "key_gb_read": round(passes * key_bytes / 1e9, 2)}}
+
+
 def run_jolt(args):
     import torch
     import torch.distributed as dist
@@ -271,6 +306,12 @@ def run_jolt(args):
                "d2h_bytes_per_step": 2 * Ko.numel() * Ko.element_size()}
         del Kh, Vh, Koh, Voh, Kd, Vd
 
+    # ---- data-driven layer grouping of the same key cache (the step before
+    # the compression path; rank 0, outside the timed region above)
+    grouping = None
+    if rank == 0 and not args.no_grouping:
+        grouping = time_grouping(jolt, K, spec, stream)
+
     # ---- roofline: the dominant kernel, and the whole path per stage
     pk, src = peaks()
     work = stage_work(spec, cells, sketch_width(spec, args.ratio))
@@ -348,7 +389,7 @@ def run_jolt(args):
                            ", larger than L2; no flush" if dense > 126e6 else ", smaller than L2")},
             "rel_frobenius_err": {"K": errK, "V": errV}, "bytes": nbytes, "budget": B,
             "roofline": roof, "path_roofline": path_roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
-            "clocks": clk,
+            "clocks": clk, "layer_grouping": grouping,
             "stages_ms_per_step": {s: round(v, 3) for s, v in per_step.items() if v > 0},
         }
         print(json.dumps(line), flush=True)

@@ -244,6 +244,41 @@ JOLT_API jolt_status jolt_residual_decode(const uint8_t* codes, const float* sca
                                  int32_t group, uint64_t seed, float* e_hat,
                                  jolt_stream_t stream);
 
+/* Data-driven layer grouping (Section 3, the paragraph that partitions the L
+ * layers into G contiguous groups, and its footnote on size bounds): for each
+ * sequence b and layer l, an 8-dimensional basis U of the top token-mode
+ * singular vectors of the keys K[b, l] unfolded as [T, H*D] (the keys before
+ * RoPE when rope_theta_k > 0, undone as for jolt_compress); the score of
+ * layers (l, l+1) is the mean squared cosine of the principal angles between
+ * the two bases, ||U_l^T U_(l+1)||_F^2 / 8, averaged over the sequences of
+ * the batch. A new group starts at layer l when score(l-1, l) is strictly
+ * below the median of the n_layers-1 scores (the mean of the two middle ones
+ * for an even count), but only once the current group holds 2 layers; a
+ * group that holds 8 layers is closed whatever the score; a trailing group of
+ * one layer joins its predecessor (so the last group can hold 9).
+ * The basis comes from a randomized subspace iteration of width 16 (8
+ * vectors + 8 oversampling) with `power_iters` power iterations and a
+ * Rayleigh-Ritz step; the sketch is seeded by `seed` (Philox4x32-10). The
+ * subspace error falls like (sigma_17 / sigma_8)^(2 power_iters + 1); 4 is a
+ * good default. A layer whose keys are all zero has the zero basis (score 0).
+ *   layout: as for jolt_plan; n_groups and group_start are not read.
+ *     seq_len >= 16, n_layers <= 1024, batch * n_layers <= 65535; strides
+ *     even and `k` 8-byte aligned.
+ *   k: DEVICE keys in that layout.
+ *   power_iters: 0..32.
+ *   scores: HOST output of n_layers-1 doubles, or NULL.
+ *   group_start: HOST output, room for n_layers+1 entries: 0, the starts,
+ *     n_layers. n_groups: HOST output.
+ * Allocates its workspace through the library allocator (64 bytes per
+ * (sequence, layer, token) plus 4 bytes per key element rounded up to
+ * 2048-token chunks, i.e. about twice the bf16 keys over 16) and
+ * synchronises `stream`. A non-finite Gram or score (Inf/NaN
+ * keys) returns JOLT_ERR_NONFINITE. */
+JOLT_API jolt_status jolt_layer_groups(const jolt_layout* layout, const void* k,
+                                       int32_t power_iters, uint64_t seed,
+                                       double* scores, int32_t* group_start,
+                                       int32_t* n_groups, jolt_stream_t stream);
+
 /* Device allocator used for handles and workspace. alloc returns NULL on
  * failure (-> JOLT_ERR_OOM). Passing NULLs restores the default. */
 typedef void* (*jolt_alloc_fn)(size_t bytes, jolt_stream_t stream, void* ctx);

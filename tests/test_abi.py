@@ -60,3 +60,43 @@ def test_plan_rejects_infeasible_budget():
     with pytest.raises(jolt.JoltError) as ei:
         jolt.jolt_plan(L, 100, o)
     assert ei.value.status == 3
+
+
+def _groups_call(L, k=0x10000, iters=4):
+    lib = jolt.load_library()
+    n = max(L.n_layers + 1, 2)
+    starts = (C.c_int32 * n)()
+    ng = C.c_int32(-1)
+    st = lib.jolt_layer_groups(C.byref(L), k, iters, 0, None, starts, C.byref(ng), None)
+    return st, list(starts), ng.value
+
+
+@pytest.mark.parametrize("bad", ["null", "short", "odd_stride", "iters", "layers", "D", "align", "theta"])
+def test_layer_groups_rejects_bad_arguments_before_touching_the_device(bad):
+    L, keep = _layout(groups=(0, 4))
+    k, iters = 0x10000, 4
+    if bad == "null":
+        k = None
+    elif bad == "short":
+        L.seq_len = 15
+    elif bad == "odd_stride":
+        L.stride_t = 65
+    elif bad == "iters":
+        iters = 33
+    elif bad == "layers":
+        L.n_layers = 1025
+    elif bad == "D":
+        L.head_dim = 96
+    elif bad == "align":
+        k = 0x10004
+    elif bad == "theta":
+        L.rope_theta_k = -1.0
+    st, _, _ = _groups_call(L, k, iters)
+    assert st in (1, 2), bad             # JOLT_ERR_INVALID_ARG, JOLT_ERR_UNSUPPORTED_SHAPE
+    assert jolt.jolt_last_error()
+
+
+def test_layer_groups_single_layer_needs_no_device():
+    L, keep = _layout(groups=(0, 1))
+    st, starts, ng = _groups_call(L)
+    assert st == 0 and ng == 1 and starts[:2] == [0, 1]

@@ -82,6 +82,8 @@ _SIGS = {
     "jolt_eps2_noalloc": (C.c_int, [C.POINTER(_I32), _I32, _I32, _VP, _VP]),
     "jolt_residual_encode": (C.c_int, [_VP, _I64, _I32, _I32, _I32, _U64, _VP, _VP, _VP]),
     "jolt_residual_decode": (C.c_int, [_VP, _VP, _I64, _I32, _I32, _I32, _U64, _VP, _VP]),
+    "jolt_layer_groups": (C.c_int, [C.POINTER(jolt_layout), _VP, _I32, _U64, C.POINTER(C.c_double),
+                                    C.POINTER(C.c_int32), C.POINTER(C.c_int32), _VP]),
     "jolt_set_allocator": (C.c_int, [_VP, _VP, _VP]),
     "jolt_last_error": (C.c_char_p, []),
     "jolt_launch_count": (_U64, []),
@@ -289,6 +291,21 @@ def jolt_residual_decode(codes, scales, rows: int, D: int, bits: int, group: int
                          stream=None) -> None:
     _check(load_library().jolt_residual_decode(_ptr(codes), _ptr(scales), rows, D, bits, group, int(seed),
                                                _ptr(e_hat), _stream(stream)))
+
+
+def jolt_layer_groups(k, rope_theta_k: float = 0.0, power_iters: int = 4, seed: int = 0,
+                      stream=None) -> Tuple[List[int], List[float]]:
+    """Data-driven layer grouping of a [B, L, H, T, D] device key tensor:
+    (group starts including 0 and L, the L-1 consecutive-layer scores)."""
+    L = k.shape[1]
+    lay, keep = make_layout(k, [0, L], rope_theta_k)
+    starts = (C.c_int32 * (L + 1))()
+    scores = (C.c_double * max(L - 1, 1))()
+    ng = C.c_int32(0)
+    _check(load_library().jolt_layer_groups(C.byref(lay), _ptr(k), int(power_iters), int(seed), scores, starts,
+                                            C.byref(ng), _stream(stream)))
+    del keep
+    return list(starts[:ng.value + 1]), list(scores[:L - 1])
 
 
 def jolt_profile_enable(on: bool) -> None:
