@@ -62,43 +62,59 @@ __device__ __forceinline__ int64_t job_base(const KeySrc& s, int job) {
 // Stage rows [t0, t0 + TM) of head h into xs[row * pitch + d] as fp32, the
 // RoPE rotation undone when a table is given (x_i = y_i c + y_j s,
 // x_j = y_j c - y_i s, j = i + D/2, no fused multiply-add). Rows past T are
-// zero. Each thread moves "quads": elements (2q, 2q+1) and their partners
-// (D/2 + 2q, D/2 + 2q + 1).
-template <int D>
+// zero. Each of the NT threads moves TM * D / 4 / NT "quads": elements
+// (2q, 2q+1) and their partners (D/2 + 2q, D/2 + 2q + 1), in batches of
+// STAGE_BATCH whose loads are all issued before any is used.
+constexpr int STAGE_BATCH = 8;
+template <int D, int NT>
 __device__ __forceinline__ void stage_x(const KeySrc& s, int job, int h, int t0, float* xs, int pitch) {
-  constexpr int half = D / 2, QPR = D / 4;
+  constexpr int half = D / 2, QPR = D / 4, NQ = TM * QPR / NT;
+  static_assert(NQ % STAGE_BATCH == 0, "quads per thread must be a multiple of the batch");
   const int64_t base = job_base(s, job) + (int64_t)h * s.sh;
-  for (int qi = threadIdx.x; qi < TM * QPR; qi += blockDim.x) {
-    const int r = qi / QPR, q = qi % QPR, t = t0 + r;
-    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-    if (t < s.T) {
-      const int64_t off = base + (int64_t)t * s.st + 2 * q;
-      if (s.f32) {
-        const float* p = reinterpret_cast<const float*>(s.k);
-        const float2 va = *reinterpret_cast<const float2*>(p + off);
-        const float2 vb = *reinterpret_cast<const float2*>(p + off + half);
-        a0 = va.x; a1 = va.y; b0 = vb.x; b1 = vb.y;
-      } else {
-        const uint16_t* p = reinterpret_cast<const uint16_t*>(s.k);
-        const uint32_t wa = *reinterpret_cast<const uint32_t*>(p + off);
-        const uint32_t wb = *reinterpret_cast<const uint32_t*>(p + off + half);
-        a0 = bf16_bits_to_f32((uint16_t)(wa & 0xFFFFu)); a1 = bf16_bits_to_f32((uint16_t)(wa >> 16));
-        b0 = bf16_bits_to_f32((uint16_t)(wb & 0xFFFFu)); b1 = bf16_bits_to_f32((uint16_t)(wb >> 16));
-      }
-      if (s.cs) {
-        const float4 c = *reinterpret_cast<const float4*>(s.cs + (int64_t)t * half + 2 * q);
-        const float x0 = __fadd_rn(__fmul_rn(a0, c.x), __fmul_rn(b0, c.y));
-        const float y0 = __fsub_rn(__fmul_rn(b0, c.x), __fmul_rn(a0, c.y));
-        const float x1 = __fadd_rn(__fmul_rn(a1, c.z), __fmul_rn(b1, c.w));
-        const float y1 = __fsub_rn(__fmul_rn(b1, c.z), __fmul_rn(a1, c.w));
-        a0 = x0; b0 = y0; a1 = x1; b1 = y1;
+#pragma unroll 1
+  for (int u0 = 0; u0 < NQ; u0 += STAGE_BATCH) {
+    float a0[STAGE_BATCH], a1[STAGE_BATCH], b0[STAGE_BATCH], b1[STAGE_BATCH];
+    float4 c[STAGE_BATCH];
+#pragma unroll
+    for (int u = 0; u < STAGE_BATCH; ++u) {
+      const int qi = threadIdx.x + NT * (u0 + u);
+      const int r = qi / QPR, q = qi % QPR, t = t0 + r;
+      a0[u] = a1[u] = b0[u] = b1[u] = 0.f;
+      c[u] = make_float4(1.f, 0.f, 1.f, 0.f);
+      if (t < s.T) {
+        const int64_t off = base + (int64_t)t * s.st + 2 * q;
+        if (s.f32) {
+          const float* p = reinterpret_cast<const float*>(s.k);
+          const float2 va = *reinterpret_cast<const float2*>(p + off);
+          const float2 vb = *reinterpret_cast<const float2*>(p + off + half);
+          a0[u] = va.x; a1[u] = va.y; b0[u] = vb.x; b1[u] = vb.y;
+        } else {
+          const uint16_t* p = reinterpret_cast<const uint16_t*>(s.k);
+          const uint32_t wa = *reinterpret_cast<const uint32_t*>(p + off);
+          const uint32_t wb = *reinterpret_cast<const uint32_t*>(p + off + half);
+          a0[u] = __uint_as_float(wa << 16); a1[u] = __uint_as_float(wa & 0xFFFF0000u);
+          b0[u] = __uint_as_float(wb << 16); b1[u] = __uint_as_float(wb & 0xFFFF0000u);
+        }
+        if (s.cs) c[u] = *reinterpret_cast<const float4*>(s.cs + (int64_t)t * half + 2 * q);
       }
     }
-    float* row = xs + r * pitch;
-    row[2 * q] = a0;
-    row[2 * q + 1] = a1;
-    row[half + 2 * q] = b0;
-    row[half + 2 * q + 1] = b1;
+#pragma unroll
+    for (int u = 0; u < STAGE_BATCH; ++u) {
+      const int qi = threadIdx.x + NT * (u0 + u);
+      const int r = qi / QPR, q = qi % QPR;
+      float x0 = a0[u], x1 = a1[u], y0 = b0[u], y1 = b1[u];
+      if (s.cs) {
+        x0 = __fadd_rn(__fmul_rn(a0[u], c[u].x), __fmul_rn(b0[u], c[u].y));
+        y0 = __fsub_rn(__fmul_rn(b0[u], c[u].x), __fmul_rn(a0[u], c[u].y));
+        x1 = __fadd_rn(__fmul_rn(a1[u], c[u].z), __fmul_rn(b1[u], c[u].w));
+        y1 = __fsub_rn(__fmul_rn(b1[u], c[u].z), __fmul_rn(a1[u], c[u].w));
+      }
+      float* row = xs + r * pitch;
+      row[2 * q] = x0;
+      row[2 * q + 1] = x1;
+      row[half + 2 * q] = y0;
+      row[half + 2 * q + 1] = y1;
+    }
   }
 }
 
@@ -141,8 +157,15 @@ __global__ void __launch_bounds__(128) k_grp_xz(KeySrc s, const double* __restri
     for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
   for (int h = 0; h < s.H; ++h) {
     __syncthreads();
-    stage_x<D>(s, job, h, t0, xs, XP);
-    for (int e = tid; e < D * S; e += blockDim.x) zs[e] = (float)z[(int64_t)h * D * S + e];
+    stage_x<D, 128>(s, job, h, t0, xs, XP);
+    {
+      constexpr int NZ = D * S / 128;    // 16 (D = 128) or 8 (D = 64) values per thread
+      double zv[NZ];
+#pragma unroll
+      for (int u = 0; u < NZ; ++u) zv[u] = z[(int64_t)h * D * S + tid + 128 * u];
+#pragma unroll
+      for (int u = 0; u < NZ; ++u) zs[tid + 128 * u] = (float)zv[u];
+    }
     __syncthreads();
 #pragma unroll 4
     for (int d = 0; d < D; ++d) {
@@ -190,12 +213,21 @@ __global__ void __launch_bounds__(D) k_grp_xtq(KeySrc s, const float* __restrict
     const int t0 = (chunk * XTQ_TILES + tile) * TM;
     if (t0 >= s.T) break;
     __syncthreads();
-    stage_x<D>(s, job, h, t0, xs, XP);
-    for (int e = tid; e < TM * S / 4; e += blockDim.x) {
-      const int r = e / (S / 4), c4 = e % (S / 4), t = t0 + r;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (t < s.T) v = *reinterpret_cast<const float4*>(q + (int64_t)t * S + 4 * c4);
-      *reinterpret_cast<float4*>(qs + r * S + 4 * c4) = v;
+    {
+      constexpr int NV4 = TM * S / 4 / D;   // float4 of Q per thread: 4 (D = 128) or 8 (D = 64)
+      float4 v[NV4];
+#pragma unroll
+      for (int u = 0; u < NV4; ++u) {
+        const int e = tid + D * u, r = e / (S / 4), c4 = e % (S / 4), t = t0 + r;
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t < s.T) v[u] = *reinterpret_cast<const float4*>(q + (int64_t)t * S + 4 * c4);
+      }
+      stage_x<D, D>(s, job, h, t0, xs, XP);
+#pragma unroll
+      for (int u = 0; u < NV4; ++u) {
+        const int e = tid + D * u, r = e / (S / 4), c4 = e % (S / 4);
+        *reinterpret_cast<float4*>(qs + r * S + 4 * c4) = v[u];
+      }
     }
     __syncthreads();
     float acc[4][4];
@@ -244,8 +276,8 @@ __global__ void k_grp_zsum(const double* __restrict__ P, int nchunk, int64_t n, 
 // memory.
 __global__ void __launch_bounds__(256) k_grp_gram(const float* __restrict__ Q, int T, int L, int cross,
                                                   int ngram, double* __restrict__ G) {
-  __shared__ __align__(16) float as[TM * S];
-  __shared__ __align__(16) float bs[TM * S];
+  __shared__ __align__(16) double as[TM * S];
+  __shared__ __align__(16) double bs[TM * S];
   const int chunk = blockIdx.x, g = blockIdx.y;
   int ja = g, jb = g;
   if (cross) {
@@ -267,12 +299,14 @@ __global__ void __launch_bounds__(256) k_grp_gram(const float* __restrict__ Q, i
         va = *reinterpret_cast<const float4*>(qa + (int64_t)t * S + 4 * c4);
         vb = *reinterpret_cast<const float4*>(qb + (int64_t)t * S + 4 * c4);
       }
-      *reinterpret_cast<float4*>(as + r * S + 4 * c4) = va;
-      *reinterpret_cast<float4*>(bs + r * S + 4 * c4) = vb;
+      double* pa = as + r * S + 4 * c4;
+      double* pb = bs + r * S + 4 * c4;
+      pa[0] = va.x; pa[1] = va.y; pa[2] = va.z; pa[3] = va.w;
+      pb[0] = vb.x; pb[1] = vb.y; pb[2] = vb.z; pb[3] = vb.w;
     }
     __syncthreads();
 #pragma unroll 8
-    for (int r = 0; r < TM; ++r) acc = fma((double)as[r * S + a], (double)bs[r * S + c], acc);
+    for (int r = 0; r < TM; ++r) acc = fma(as[r * S + a], bs[r * S + c], acc);
   }
   G[((int64_t)chunk * ngram + g) * (S * S) + tid] = acc;
 }
