@@ -22,7 +22,7 @@
 //
 // Precision: the T-sized passes (X Z, X^T Q) multiply in fp32 with fp32
 // accumulators over one 128-row tile (X^T Q) or one row (X Z) and fp64
-// across tiles; Grams, Cholesky factors, the Jacobi solve and the scores are
+// across tiles (X^T Q); Grams, Cholesky factors, the Jacobi solve and the scores are
 // fp64. Q is kept in fp32.
 #include <cuda_runtime.h>
 
@@ -65,7 +65,7 @@ __device__ __forceinline__ int64_t job_base(const KeySrc& s, int job) {
 // zero. Each of the NT threads moves TM * D / 4 / NT "quads": elements
 // (2q, 2q+1) and their partners (D/2 + 2q, D/2 + 2q + 1), in batches of
 // STAGE_BATCH whose loads are all issued before any is used.
-constexpr int STAGE_BATCH = 8;
+constexpr int STAGE_BATCH = 4;
 template <int D, int NT>
 __device__ __forceinline__ void stage_x(const KeySrc& s, int job, int h, int t0, float* xs, int pitch) {
   constexpr int half = D / 2, QPR = D / 4, NQ = TM * QPR / NT;
@@ -137,42 +137,44 @@ __global__ void k_grp_omega(double* __restrict__ om, int F, uint64_t seed) {
 
 // W[job][t][c] = sum_f X[t][f] Z[job][f][c] for one tile of TM rows; the
 // Z block of a job starts at Z + job * zstride (zstride 0: one Omega for
-// all jobs). 128 threads, each 4 rows x 4 columns; heads staged one at a
-// time (X tile [TM][D+1] and Z rows [D][S], both fp32).
+// all jobs). 256 threads, each 2 rows x 4 columns; heads staged one at a
+// time (X tile [TM][D+1] and Z rows [D][S], both fp32). Three blocks fit an
+// SM (shared memory), 24 warps, enough to cover the staging loads' latency.
+constexpr int XZ_THREADS = 256;
 template <int D>
-__global__ void __launch_bounds__(128) k_grp_xz(KeySrc s, const double* __restrict__ Z, int64_t zstride,
-                                                float* __restrict__ W) {
+__global__ void __launch_bounds__(XZ_THREADS, 3) k_grp_xz(KeySrc s, const double* __restrict__ Z, int64_t zstride,
+                                                       float* __restrict__ W) {
   extern __shared__ __align__(16) float sm[];
   constexpr int XP = D + 1;
   static_assert((TM * XP) % 4 == 0, "zs must start on a 16-byte boundary");
   float* xs = sm;
   float* zs = sm + TM * XP;       // TM * XP is a multiple of 4: zs stays 16-byte aligned
   const int job = blockIdx.y, t0 = blockIdx.x * TM;
-  const int tid = threadIdx.x, cg = tid & 3, rg = tid >> 2;
+  const int tid = threadIdx.x, cg = tid & 3, rg = tid >> 2;   // rows 2rg, 2rg+1; columns 4cg..4cg+3
   const double* z = Z + (int64_t)job * zstride;
-  float acc[4][4];
+  float acc[2][4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
+  for (int j = 0; j < 2; ++j)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[j][c] = 0.f;
   for (int h = 0; h < s.H; ++h) {
     __syncthreads();
-    stage_x<D, 128>(s, job, h, t0, xs, XP);
+    stage_x<D, XZ_THREADS>(s, job, h, t0, xs, XP);
     {
-      constexpr int NZ = D * S / 128;    // 16 (D = 128) or 8 (D = 64) values per thread
+      constexpr int NZ = D * S / XZ_THREADS;    // 8 (D = 128) or 4 (D = 64) values per thread
       double zv[NZ];
 #pragma unroll
-      for (int u = 0; u < NZ; ++u) zv[u] = z[(int64_t)h * D * S + tid + 128 * u];
+      for (int u = 0; u < NZ; ++u) zv[u] = z[(int64_t)h * D * S + tid + XZ_THREADS * u];
 #pragma unroll
-      for (int u = 0; u < NZ; ++u) zs[tid + 128 * u] = (float)zv[u];
+      for (int u = 0; u < NZ; ++u) zs[tid + XZ_THREADS * u] = (float)zv[u];
     }
     __syncthreads();
-#pragma unroll 4
+#pragma unroll 8
     for (int d = 0; d < D; ++d) {
       const float4 zv = *reinterpret_cast<const float4*>(zs + d * S + 4 * cg);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float x = xs[(4 * rg + j) * XP + d];
+      for (int j = 0; j < 2; ++j) {
+        const float x = xs[(2 * rg + j) * XP + d];
         acc[j][0] = fmaf(x, zv.x, acc[j][0]);
         acc[j][1] = fmaf(x, zv.y, acc[j][1]);
         acc[j][2] = fmaf(x, zv.z, acc[j][2]);
@@ -181,8 +183,8 @@ __global__ void __launch_bounds__(128) k_grp_xz(KeySrc s, const double* __restri
     }
   }
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int t = t0 + 4 * rg + j;
+  for (int j = 0; j < 2; ++j) {
+    const int t = t0 + 2 * rg + j;
     if (t < s.T)
       *reinterpret_cast<float4*>(W + ((int64_t)job * s.T + t) * S + 4 * cg) =
           make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
@@ -190,22 +192,23 @@ __global__ void __launch_bounds__(128) k_grp_xz(KeySrc s, const double* __restri
 }
 
 // P[chunk][job][f][c] = sum over the chunk's rows t of X[t][f] Q[job][t][c],
-// f in head blockIdx.y. D threads, each 4 features x 4 columns; fp32 sums
+// f in head blockIdx.y. 2D threads, each 2 features x 4 columns; fp32 sums
 // over one tile of TM rows, fp64 across the chunk's tiles.
 template <int D>
-__global__ void __launch_bounds__(D) k_grp_xtq(KeySrc s, const float* __restrict__ Q, double* __restrict__ P,
-                                               int njobs) {
+__global__ void __launch_bounds__(2 * D, 3) k_grp_xtq(KeySrc s, const float* __restrict__ Q, double* __restrict__ P,
+                                                   int njobs) {
   extern __shared__ __align__(16) float sm[];
+  constexpr int NT = 2 * D;
   constexpr int XP = D + 4;
-  static_assert(XP % 4 == 0 && (TM * XP) % 4 == 0, "float4 rows of xs and qs");
+  static_assert(XP % 4 == 0 && (TM * XP) % 4 == 0, "float2 rows of xs, float4 rows of qs");
   float* xs = sm;                  // [TM][XP]
   float* qs = sm + TM * XP;        // [TM][S]
   const int chunk = blockIdx.x, h = blockIdx.y, job = blockIdx.z;
-  const int tid = threadIdx.x, cg = tid & 3, fg = tid >> 2;
+  const int tid = threadIdx.x, cg = tid & 3, fg = tid >> 2;   // features 2fg, 2fg+1; columns 4cg..4cg+3
   const int F = s.H * D;
-  double acc64[4][4];
+  double acc64[2][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 2; ++i)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc64[i][c] = 0.0;
   const float* q = Q + (int64_t)job * s.T * S;
@@ -214,34 +217,34 @@ __global__ void __launch_bounds__(D) k_grp_xtq(KeySrc s, const float* __restrict
     if (t0 >= s.T) break;
     __syncthreads();
     {
-      constexpr int NV4 = TM * S / 4 / D;   // float4 of Q per thread: 4 (D = 128) or 8 (D = 64)
+      constexpr int NV4 = TM * S / 4 / NT;   // float4 of Q per thread: 2
       float4 v[NV4];
 #pragma unroll
       for (int u = 0; u < NV4; ++u) {
-        const int e = tid + D * u, r = e / (S / 4), c4 = e % (S / 4), t = t0 + r;
+        const int e = tid + NT * u, r = e / (S / 4), c4 = e % (S / 4), t = t0 + r;
         v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (t < s.T) v[u] = *reinterpret_cast<const float4*>(q + (int64_t)t * S + 4 * c4);
       }
-      stage_x<D, D>(s, job, h, t0, xs, XP);
+      stage_x<D, NT>(s, job, h, t0, xs, XP);
 #pragma unroll
       for (int u = 0; u < NV4; ++u) {
-        const int e = tid + D * u, r = e / (S / 4), c4 = e % (S / 4);
+        const int e = tid + NT * u, r = e / (S / 4), c4 = e % (S / 4);
         *reinterpret_cast<float4*>(qs + r * S + 4 * c4) = v[u];
       }
     }
     __syncthreads();
-    float acc[4][4];
+    float acc[2][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
-#pragma unroll 4
+#pragma unroll 8
     for (int r = 0; r < TM; ++r) {
-      const float4 xv = *reinterpret_cast<const float4*>(xs + r * XP + 4 * fg);
+      const float2 xv = *reinterpret_cast<const float2*>(xs + r * XP + 2 * fg);
       const float4 qv = *reinterpret_cast<const float4*>(qs + r * S + 4 * cg);
-      const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+      const float xa[2] = {xv.x, xv.y};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 2; ++i) {
         acc[i][0] = fmaf(xa[i], qv.x, acc[i][0]);
         acc[i][1] = fmaf(xa[i], qv.y, acc[i][1]);
         acc[i][2] = fmaf(xa[i], qv.z, acc[i][2]);
@@ -249,13 +252,13 @@ __global__ void __launch_bounds__(D) k_grp_xtq(KeySrc s, const float* __restrict
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc64[i][c] += (double)acc[i][c];
   }
-  double* p = P + (((int64_t)chunk * njobs + job) * F + (int64_t)h * D + 4 * fg) * S + 4 * cg;
+  double* p = P + (((int64_t)chunk * njobs + job) * F + (int64_t)h * D + 2 * fg) * S + 4 * cg;
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 2; ++i)
 #pragma unroll
     for (int c = 0; c < 4; ++c) p[(int64_t)i * S + c] = acc64[i][c];
 }
@@ -564,7 +567,7 @@ template <int D>
 static jolt_status launch_xz(const KeySrc& ks, const double* Z, int64_t zstride, float* W, int J, cudaStream_t st) {
   constexpr size_t smem = (size_t)(TM * (D + 1) + D * S) * sizeof(float);
   JOLT_CUDA_TRY(cudaFuncSetAttribute(k_grp_xz<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  k_grp_xz<D><<<dim3((ks.T + TM - 1) / TM, J), 128, smem, st>>>(ks, Z, zstride, W);
+  k_grp_xz<D><<<dim3((ks.T + TM - 1) / TM, J), XZ_THREADS, smem, st>>>(ks, Z, zstride, W);
   JOLT_LAUNCHED();
   return JOLT_OK;
 }
@@ -574,7 +577,7 @@ static jolt_status launch_xtq(const KeySrc& ks, const float* Q, double* P, doubl
                               cudaStream_t st) {
   constexpr size_t smem = (size_t)(TM * (D + 4) + TM * S) * sizeof(float);
   JOLT_CUDA_TRY(cudaFuncSetAttribute(k_grp_xtq<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  k_grp_xtq<D><<<dim3(nchunk, ks.H, J), D, smem, st>>>(ks, Q, P, J);
+  k_grp_xtq<D><<<dim3(nchunk, ks.H, J), 2 * D, smem, st>>>(ks, Q, P, J);
   JOLT_LAUNCHED();
   const int64_t n = (int64_t)J * ks.H * D * S;
   k_grp_zsum<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(P, nchunk, n, Z);
