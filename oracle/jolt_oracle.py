@@ -7,7 +7,8 @@ with the CUDA library, and the library never calls it.
 What it follows: "A JoLT for the KV Cache: Near-Lossless KV Cache Compression
 via Joint Rank-bit Allocation" (Krishnan & Schulz), Section 3:
   * "Partial Tucker backbone"       -> token_spectrum, feature_spectrum, fit
-  * "Rotated low-bit residual"      -> rotate / quantize / pack, residual_*
+  * "Rotated low-bit residual"      -> rotate / quantize / pack, residual_*,
+                                       qr_rotation (the page's own rotation)
   * "Joint Lagrangian allocation"   -> Eq. (1) cost_bytes, Eq. (2) error model,
                                        eps2_table
   * "Solving the allocation"        -> Eqs. (3)-(4): argmin_cell, allocate,
@@ -57,6 +58,9 @@ library as well):
      neighbours); below rank 8 the trailing basis vectors are arbitrary.
   R14 with a batch, the score of (l, l+1) is the mean over sequences.
   R15 median of the L-1 scores as numpy computes it; "falls below" is strict.
+  R17 QR-Gaussian rotation (option rotation="qr"): R = Q of G = QR, G a D x D
+     matrix of Philox/Box-Muller normals (row-major), R's diagonal made
+     positive; r = Q e and e = Q^T r summed in fp64, rounded once to fp32.
 """
 from __future__ import annotations
 
@@ -213,6 +217,48 @@ def rotate(E: np.ndarray, signs: np.ndarray) -> np.ndarray:
 def unrotate(r: np.ndarray, signs: np.ndarray) -> np.ndarray:
     """R^T r = s * fl32( FWHT(r) * fl32(1/sqrt(D)) ) (fp32)."""
     return f32(f32(fwht_f32(r) * rot_scale(r.shape[-1])) * signs)
+
+
+def qr_rotation(D: int, seed: int) -> np.ndarray:
+    """The page's rotation (Section 3, "Rotated low-bit residual"): the
+    orthogonal factor Q of the QR factorization of a D x D matrix G of
+    standard normals (gaussian_f64 on stream STREAM_QRGAUSS, row-major), made
+    unique by a positive diagonal of the triangular factor (reading R17). fp64."""
+    G = gaussian_f64(D * D, seed, STREAM_QRGAUSS).reshape(D, D)
+    Q, R = np.linalg.qr(G)
+    s = np.sign(np.diag(R))
+    s[s == 0] = 1.0
+    return Q * s[None, :]
+
+
+def rotate_qr(E: np.ndarray, Q: np.ndarray) -> np.ndarray:
+    """r = Q e for every row e (r_i = sum_j Q_ij e_j), the products summed in
+    fp64 and rounded once to fp32 (reading R17)."""
+    return f32(np.asarray(E, np.float64) @ Q.T)
+
+
+def unrotate_qr(r: np.ndarray, Q: np.ndarray) -> np.ndarray:
+    """e = Q^T r for every row, fp64 sums, one rounding to fp32."""
+    return f32(np.asarray(r, np.float64) @ Q)
+
+
+def rotation_for(D: int, seed: int, kind: str = "hadamard") -> np.ndarray:
+    """The rotation of one sequence: Hadamard signs (a vector, reading R2) or
+    the QR-Gaussian matrix (reading R17). The residual functions tell them
+    apart by their rank."""
+    if kind == "hadamard":
+        return hadamard_signs(D, seed)
+    if kind == "qr":
+        return qr_rotation(D, seed)
+    raise ValueError(kind)
+
+
+def apply_rotation(E: np.ndarray, rot: np.ndarray) -> np.ndarray:
+    return rotate(E, rot) if rot.ndim == 1 else rotate_qr(E, rot)
+
+
+def undo_rotation(r: np.ndarray, rot: np.ndarray) -> np.ndarray:
+    return unrotate(r, rot) if rot.ndim == 1 else unrotate_qr(r, rot)
 
 
 def qmax(b: int) -> int:
@@ -581,9 +627,10 @@ def residual_from(X: np.ndarray, Xt: np.ndarray) -> np.ndarray:
 
 
 def encode_residual(E: np.ndarray, b: int, g: int, signs: np.ndarray) -> Residual:
+    """signs: the rotation of rotation_for (Hadamard signs or a QR matrix)."""
     if b == 0:
         return Residual(0, None, None, None)
-    r = rotate(E, signs)
+    r = apply_rotation(E, signs)
     codes, scales = quantize(r, b, g)
     return Residual(b, codes, pack_bits(codes, b), scales)
 
@@ -592,7 +639,7 @@ def decode_residual(res: Residual, g: int, signs: np.ndarray, D: int) -> Optiona
     if res.b == 0:
         return None
     codes = unpack_bits(res.packed, res.b, D)
-    return unrotate(dequantize(codes, res.scales, g), signs)
+    return undo_rotation(dequantize(codes, res.scales, g), signs)
 
 
 # --------------------------------------------------------------------------
@@ -608,6 +655,7 @@ class Options:
     tol: float = 0.005
     max_iters: int = 50
     minimizer: str = "enumerate"                  # or "greedy" (the page's per-cell search)
+    rotation: str = "hadamard"                    # or "qr" (the page's QR of a Gaussian)
 
 
 @dataclasses.dataclass
@@ -677,6 +725,7 @@ class Compressed:
     rope_theta_k: float
     seed: int
     g_of_D: int
+    rotation: str = "hadamard"
 
 
 def compress(cache_k: np.ndarray, cache_v: np.ndarray, group_starts: Sequence[int],
@@ -698,16 +747,17 @@ def compress(cache_k: np.ndarray, cache_v: np.ndarray, group_starts: Sequence[in
     out = []
     for c, X, U, (rT, rd, b), nb in zip(refs, Xs, Us, al.choice, al.bytes):
         f = fit(X, U, rT, rd)
-        sg = hadamard_signs(D, seed + c.b)
+        sg = rotation_for(D, seed + c.b, opt.rotation)
         res = encode_residual(residual_from(X, backbone(f)), b, g, sg)
         out.append(CompressedCell(c, rT, rd, b, f, res, nb))
-    return Compressed(out, al, (B, L, H, T, D), rope_theta_k, seed, g)
+    return Compressed(out, al, (B, L, H, T, D), rope_theta_k, seed, g, opt.rotation)
 
 
-def decompress_cell(cc: CompressedCell, D: int, g: int, seed: int, rope_theta_k: float) -> np.ndarray:
+def decompress_cell(cc: CompressedCell, D: int, g: int, seed: int, rope_theta_k: float,
+                    rotation: str = "hadamard") -> np.ndarray:
     """X^ = bf16( [RoPE]( X~ + R^T dequant(codes) ) ), fp32 sum and RoPE."""
     Xt = backbone(cc.fit)
-    sg = hadamard_signs(D, seed + cc.ref.b)
+    sg = rotation_for(D, seed + cc.ref.b, rotation)
     e = decode_residual(cc.res, g, sg, D)
     x = f32(Xt) if e is None else f32(f32(Xt) + e)
     if cc.ref.kind == 0 and rope_theta_k > 0:
@@ -722,7 +772,8 @@ def decompress(comp: Compressed) -> Tuple[np.ndarray, np.ndarray]:
     V = np.zeros(comp.shape, np.float64)
     for cc in comp.cells:
         dst = K if cc.ref.kind == 0 else V
-        dst[cc.ref.b, cc.ref.l0:cc.ref.l1] = decompress_cell(cc, D, comp.g_of_D, comp.seed, comp.rope_theta_k)
+        dst[cc.ref.b, cc.ref.l0:cc.ref.l1] = decompress_cell(cc, D, comp.g_of_D, comp.seed, comp.rope_theta_k,
+                                                             comp.rotation)
     return K, V
 
 

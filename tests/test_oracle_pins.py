@@ -458,3 +458,50 @@ def test_residual_bits_lower_the_error():
     for b, e in zip((2, 4, 8), errs[1:]):
         ratio = (e ** 2 - floor2) / (errs[0] ** 2 - floor2)
         assert 0.5 * eps[b] < ratio < 2.0 * eps[b]
+
+
+# ------------------------------------------------------- QR-Gaussian rotation
+# ("Rotated low-bit residual": the page rotates by the Q of a seeded
+# Gaussian's QR factorization; reading R17 fixes the sign convention)
+@pytest.mark.parametrize("D", [64, 128])
+def test_qr_rotation_is_the_positive_diagonal_factor_of_its_gaussian(D):
+    Q = o.qr_rotation(D, 11)
+    assert np.abs(Q.T @ Q - np.eye(D)).max() < 1e-13
+    # uniqueness: with R upper triangular and R_ii > 0, R^T R = G^T G, so R is
+    # the transposed Cholesky factor of G^T G and Q = G R^-1
+    G = o.gaussian_f64(D * D, 11, o.STREAM_QRGAUSS).reshape(D, D)
+    R = np.linalg.cholesky(G.T @ G).T
+    assert np.abs(Q - G @ np.linalg.inv(R)).max() < 1e-9
+    assert np.abs(o.qr_rotation(D, 12) - Q).max() > 0.1
+
+
+def test_qr_rotation_orientation_and_round_trip():
+    D = 64
+    Q = o.qr_rotation(D, 5)
+    # rotating a unit vector e_j gives column j of Q (r = Q e)
+    E = np.eye(D, dtype=np.float32)[:3]
+    r = o.rotate_qr(E, Q)
+    for j in range(3):
+        assert np.abs(r[j] - Q[:, j].astype(np.float32)).max() < 1e-7
+    x = np.random.default_rng(0).standard_normal((50, D)).astype(np.float32)
+    y = o.rotate_qr(x, Q)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-6)
+    back = o.unrotate_qr(y, Q)
+    # each r_i carries one fp32 rounding (|d r_i| <= 2^-24 |r_i|); Q^T spreads
+    # them by at most ||r||_2 = ||x||_2 per element (unit columns), plus the
+    # final rounding of e_j
+    bound = 2.0 ** -24 * (np.linalg.norm(x, axis=1)[:, None] + np.abs(x)) * 1.01
+    assert np.all(np.abs(back - x) <= bound)
+
+
+def test_qr_rotation_residual_round_trip_error_bound():
+    # encode/decode through the rotation: the error is the quantizer's,
+    # rotated back, so its norm is bounded by the per-row bound sqrt(D) s/2
+    D, b = 64, 8
+    Q = o.rotation_for(D, 3, "qr")
+    E = np.random.default_rng(1).standard_normal((40, D)).astype(np.float32)
+    res = o.encode_residual(E, b, D, Q)
+    back = o.decode_residual(res, D, Q, D)
+    err = np.linalg.norm(back - E, axis=1)
+    bound = np.sqrt(D) * res.scales[:, 0] / 2 * 1.001 + 1e-5
+    assert np.all(err <= bound)

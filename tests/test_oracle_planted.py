@@ -194,3 +194,22 @@ def test_rule_no_minimum_size(monkeypatch):
 def test_rule_size_cap_off_by_one(monkeypatch):
     monkeypatch.setattr(o, "group_layers", _rule(max_size=9))
     _fails(gpins.test_equal_scores_close_groups_at_eight)
+
+
+# ------------------------------------------------- QR rotation plants
+def test_qr_without_sign_fix(monkeypatch):
+    def bad(D, seed):
+        G = o.gaussian_f64(D * D, seed, o.STREAM_QRGAUSS).reshape(D, D)
+        return np.linalg.qr(G)[0]
+    monkeypatch.setattr(o, "qr_rotation", bad)
+    _fails(pins.test_qr_rotation_is_the_positive_diagonal_factor_of_its_gaussian, 64)
+
+
+def test_qr_rotation_transposed(monkeypatch):
+    monkeypatch.setattr(o, "rotate_qr", lambda E, Q: o.f32(np.asarray(E, np.float64) @ Q))
+    _fails(pins.test_qr_rotation_orientation_and_round_trip)
+
+
+def test_qr_unrotation_transposed(monkeypatch):
+    monkeypatch.setattr(o, "unrotate_qr", lambda r, Q: o.f32(np.asarray(r, np.float64) @ Q.T))
+    _fails(pins.test_qr_rotation_residual_round_trip_error_bound)
