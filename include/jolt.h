@@ -57,7 +57,7 @@ typedef enum {
 
 enum { JOLT_BF16 = 0, JOLT_F32 = 1 };             /* jolt_layout.dtype        */
 enum { JOLT_EXACT = 0, JOLT_RANDOMIZED = 1 };      /* jolt_options.mode        */
-enum { JOLT_ROT_HADAMARD = 0 };                    /* jolt_options.rotation    */
+enum { JOLT_ROT_HADAMARD = 0, JOLT_ROT_QR_GAUSS = 1 }; /* jolt_options.rotation */
 enum { JOLT_MIN_ENUMERATE = 0, JOLT_MIN_GREEDY = 1 }; /* jolt_options.minimizer */
 
 /*
@@ -93,6 +93,14 @@ typedef struct {
  *   allocation"): for each b, start at the smallest ranks and take whichever
  *   single grid step of r_T or r_d lowers the error most per added byte, while
  *   it lowers e + lambda s; keep the best b.
+ *   rotation JOLT_ROT_HADAMARD: R = D^-1/2 H_D diag(s), s seeded per
+ *   sequence (the fast path: the tensor-core stream kernels). JOLT_ROT_QR_GAUSS
+ *   is the page's own rotation ("Rotated low-bit residual"): R = the Q of the
+ *   QR factorization of a seeded D x D standard Gaussian (Philox4x32-10 +
+ *   Box-Muller, one matrix per sequence, R's triangular factor with a
+ *   positive diagonal), r = R e and e = R^T r summed in fp64 and rounded once
+ *   to fp32. It runs on the row-per-thread kernels (a dense D x D product per
+ *   row) and is much slower; the handle keeps the matrices (batch*D*D*8 bytes).
  * Grids are HOST arrays of strictly increasing values >= 1, copied at plan
  * time; NULL/0 means "every integer 1..max".
  */
@@ -107,7 +115,7 @@ typedef struct {
   int32_t rt_max;
   int32_t oversample_p, power_iters;
   int32_t scale_group;           /* 0 (= D), 32, 64 or 128; must divide D      */
-  int32_t rotation;              /* JOLT_ROT_HADAMARD                          */
+  int32_t rotation;              /* JOLT_ROT_HADAMARD | JOLT_ROT_QR_GAUSS      */
   double budget_tol;
   int32_t max_iters;
   int32_t minimizer;             /* JOLT_MIN_ENUMERATE | JOLT_MIN_GREEDY       */

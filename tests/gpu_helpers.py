@@ -18,6 +18,8 @@ def gpu_compress(K: torch.Tensor, V: torch.Tensor, group_starts, budget: int, se
     kw = dict(opt_kw)
     if isinstance(kw.get("minimizer"), str):
         kw["minimizer"] = jolt.JOLT_MIN_GREEDY if kw["minimizer"] == "greedy" else jolt.JOLT_MIN_ENUMERATE
+    if isinstance(kw.get("rotation"), str):
+        kw["rotation"] = jolt.JOLT_ROT_QR_GAUSS if kw["rotation"] == "qr" else jolt.JOLT_ROT_HADAMARD
     opt, keep2 = jolt.make_options(**kw)
     plan = jolt.jolt_plan(lay, budget, opt)
     try:
@@ -48,7 +50,8 @@ def oracle_compress(K: torch.Tensor, V: torch.Tensor, group_starts, budget: int,
                     rd_grid=tuple(kw["rd_grid"]) if kw.get("rd_grid") else None,
                     rt_max=kw.get("rt_max", 0), scale_group=kw["scale_group"],
                     tol=kw.get("budget_tol", 0.005), max_iters=kw.get("max_iters", 50),
-                    minimizer=kw.get("minimizer", "enumerate"))
+                    minimizer=kw.get("minimizer", "enumerate"),
+                    rotation=kw.get("rotation", "hadamard"))
     comp = o.compress(Kn, Vn, group_starts, budget, seed, opt, rope_theta_k)
     Kh, Vh = o.decompress(comp)
     return Kn, Vn, Kh, Vh, comp

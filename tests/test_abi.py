@@ -32,7 +32,7 @@ def _layout(D=64, theta=0.0, groups=(0, 2)):
     return L, gs
 
 
-@pytest.mark.parametrize("bad", ["D", "bits", "group", "grid", "groups", "minimizer"])
+@pytest.mark.parametrize("bad", ["D", "bits", "group", "grid", "groups", "minimizer", "rotation"])
 def test_plan_rejects_bad_arguments_before_touching_the_device(bad):
     L, keep = _layout()
     o, k2 = jolt.make_options()
@@ -49,6 +49,8 @@ def test_plan_rejects_bad_arguments_before_touching_the_device(bad):
         L.n_layers = 2
     elif bad == "minimizer":
         o.minimizer = 7
+    elif bad == "rotation":
+        o.rotation = 2
     with pytest.raises(jolt.JoltError) as ei:
         jolt.jolt_plan(L, 10 ** 6, o)
     assert ei.value.status in (1, 2)

@@ -308,3 +308,27 @@ def test_all_zero_bits_and_generous_budget():
     spec = synth.SPECS["tiny"]
     K, V = synth.make_cache(spec, 1)
     _compare(K, V, [0, 2], 10 ** 9, bits=(0,), rt_grid=(8, 64), rd_grid=(16, 64))
+
+
+# ------------------------------------------------ QR-Gaussian rotation option
+@pytest.mark.parametrize("case", ["tiny", "batch2_rope_d64", "mistral_4layers"])
+def test_qr_gaussian_rotation_end_to_end(case):
+    """The page's rotation (Q of a seeded Gaussian's QR, one per sequence) on
+    the row-per-thread kernels, against the oracle with the same rotation; the
+    result must also differ from the Hadamard run (the option takes effect)."""
+    if case == "tiny":
+        spec = synth.SPECS["tiny"]
+        kw = dict(bits=(0, 2, 3, 4, 8), rt_grid=(8, 16, 32, 64), rd_grid=(16, 32, 48))
+    elif case == "batch2_rope_d64":
+        spec = synth.CacheSpec("qrb", 2, 2, 2, 200, 64, 2, 16, 1.0, 0.02, rope_theta_k=1e4, dtype="bf16")
+        kw = dict(bits=(0, 2, 3, 4, 8), scale_group=32)
+    else:
+        spec = synth.SPECS["mistral"].replace(n_layers=4)
+        kw = {}
+    K, V = synth.make_cache(spec, 5)
+    gs = synth.group_starts(spec)
+    B = o.budget_for_ratio(K.numel() * 2, 2.5)
+    _compare(K, V, gs, B, spec.rope_theta_k, rotation="qr", **kw)
+    Kq, Vq = gpu_compress(K, V, gs, B, 0, spec.rope_theta_k, rotation="qr", **kw)[:2]
+    Kh, Vh = gpu_compress(K, V, gs, B, 0, spec.rope_theta_k, **kw)[:2]
+    assert rel(Kq, Kh) > 10 * RTOL_RECON or rel(Vq, Vh) > 10 * RTOL_RECON

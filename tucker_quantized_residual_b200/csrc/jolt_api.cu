@@ -208,6 +208,8 @@ struct jolt_handle_s {
   AllocState* d_state = nullptr;
   int* d_status = nullptr;
   void* block = nullptr;
+  void* qblock = nullptr;        // QR-Gaussian rotation: scratch + Q per sequence
+  double* d_qrot = nullptr;      // [batch][D][D], NULL for the Hadamard rotation
 };
 
 static jolt_status status_from_dev(int st) {
@@ -289,7 +291,7 @@ static jolt_status validate(const jolt_layout* L, const jolt_options* o) {
   if (L->stride_t < L->head_dim || L->stride_h < 1 || L->stride_l < 1 || L->stride_b < 1) { set_error("bad strides"); return JOLT_ERR_INVALID_ARG; }
   if (L->rope_theta_k < 0.0f) { set_error("rope_theta_k must be >= 0"); return JOLT_ERR_INVALID_ARG; }
   if (o->mode != JOLT_EXACT && o->mode != JOLT_RANDOMIZED) { set_error("bad mode"); return JOLT_ERR_INVALID_ARG; }
-  if (o->rotation != JOLT_ROT_HADAMARD) { set_error("only the Hadamard rotation is implemented"); return JOLT_ERR_INVALID_ARG; }
+  if (o->rotation != JOLT_ROT_HADAMARD && o->rotation != JOLT_ROT_QR_GAUSS) { set_error("rotation must be JOLT_ROT_HADAMARD or JOLT_ROT_QR_GAUSS"); return JOLT_ERR_INVALID_ARG; }
   if (o->n_bits < 1 || o->n_bits > 8) { set_error("n_bits must be 1..8"); return JOLT_ERR_INVALID_ARG; }
   for (int i = 0; i < o->n_bits; ++i) {
     int b = o->bits[i];
@@ -972,6 +974,15 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   auto fail = [&](jolt_status st) { jolt_free_handle(h); return st; };
   if (cudaMemsetAsync(h->d_status, 0, 4 * sizeof(int), s) != cudaSuccess) return fail(JOLT_ERR_CUDA);
   jolt_status st;
+  if (p->opt.rotation == JOLT_ROT_QR_GAUSS) {
+    const size_t qn = (size_t)p->lay.batch * p->D * p->D;
+    h->qblock = dev_alloc(2 * qn * sizeof(double), s);
+    if (!h->qblock) { set_error("rotation allocation failed"); return fail(JOLT_ERR_OOM); }
+    h->d_qrot = reinterpret_cast<double*>(h->qblock) + qn;
+    if ((st = launch_qr_rotation(p->D, p->lay.batch, seed, reinterpret_cast<double*>(h->qblock), h->d_qrot, s)) !=
+        JOLT_OK)
+      return fail(st);
+  }
   if ((st = upload_cells(p, k, v, s)) != JOLT_OK) return fail(st);
   if ((st = run_spectra(p, k, v, seed, h->d_status, s)) != JOLT_OK) return fail(st);
   {
@@ -1006,10 +1017,11 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   if ((st = launch_core(fa, p->rmax_all, p->lh_max, s)) != JOLT_OK) return fail(st);
   ResidArgs ra{};
   ra.cells = p->d_cells; ra.cs = p->d_cs; ra.out = h->d_out; ra.M = p->d_M; ra.rmax_of = p->d_rmax;
-  ra.G = p->G; ra.seed = seed;
+  ra.G = p->G; ra.seed = seed; ra.qrot = h->d_qrot;
   ps_fit.end();
   ProfScope ps_res(JOLT_STAGE_RESIDUAL, s);
-  if (p->tc_in && reinterpret_cast<uintptr_t>(k) % 16 == 0 && reinterpret_cast<uintptr_t>(v) % 16 == 0) {
+  // the tensor-core stream kernel implements the Hadamard rotation only
+  if (p->tc_in && !h->d_qrot && reinterpret_cast<uintptr_t>(k) % 16 == 0 && reinterpret_cast<uintptr_t>(v) % 16 == 0) {
     if ((st = run_stream(p, h, k, v, nullptr, nullptr, nullptr, s)) != JOLT_OK) return fail(st);
   } else {
     if ((st = launch_residual_simt(ra, nc, p->D, p->T, p->lh_max, s)) != JOLT_OK) return fail(st);
@@ -1034,12 +1046,12 @@ jolt_status jolt_decompress(const jolt_handle_t* h, void* k_out, void* v_out, co
   JOLT_TRY(launch_core_m(h->d_out, p->d_cells, p->d_M, p->d_rmax, nc, p->D, p->rmax_all, p->lh_max, s));
   ResidArgs ra{};
   ra.cells = p->d_cells; ra.cs = p->d_cs; ra.out = h->d_out; ra.M = p->d_M; ra.rmax_of = p->d_rmax;
-  ra.G = p->G; ra.seed = h->seed;
+  ra.G = p->G; ra.seed = h->seed; ra.qrot = h->d_qrot;
   ra.out_k = reinterpret_cast<uint16_t*>(k_out); ra.out_v = reinterpret_cast<uint16_t*>(v_out);
   ra.osb = L.stride_b; ra.osl = L.stride_l; ra.osh = L.stride_h; ra.ost = L.stride_t;
   const bool tc_out = L.stride_t % 8 == 0 && L.stride_h % 8 == 0 && L.stride_l % 8 == 0 && L.stride_b % 8 == 0 &&
                       (reinterpret_cast<uintptr_t>(k_out) % 16) == 0 && (reinterpret_cast<uintptr_t>(v_out) % 16) == 0;
-  if (tc_out) JOLT_TRY(run_stream(p, h, nullptr, nullptr, k_out, v_out, &L, s));
+  if (tc_out && !h->d_qrot) JOLT_TRY(run_stream(p, h, nullptr, nullptr, k_out, v_out, &L, s));
   else JOLT_TRY(launch_decompress_simt(ra, nc, p->D, p->T, p->lh_max, s));
   return JOLT_OK;
 }
@@ -1101,6 +1113,7 @@ jolt_status jolt_handle_cell(const jolt_handle_t* h, int32_t cell, jolt_cell_vie
 void jolt_free_handle(jolt_handle_t* h) {
   if (!h) return;
   if (h->block) dev_free(h->block, h->stream);
+  if (h->qblock) dev_free(h->qblock, h->stream);
   delete h;
 }
 

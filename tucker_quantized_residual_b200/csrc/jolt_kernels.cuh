@@ -144,6 +144,7 @@ struct ResidArgs {
   const int* rmax_of;
   int G;
   uint64_t seed;
+  const double* qrot;           // [batch][D][D] QR-Gaussian rotation; NULL: Hadamard
   // decompress outputs (bf16)
   uint16_t* out_k;              // decompress outputs (bf16), NULL when encoding
   uint16_t* out_v;
@@ -159,6 +160,9 @@ jolt_status launch_encode_rows(const float* e, int64_t rows, int D, int b, int G
 jolt_status launch_decode_rows(const uint8_t* codes, const float* scales, int64_t rows, int D,
                                int b, int G, uint64_t seed, float* e, cudaStream_t s);
 jolt_status launch_rope_table(int T, int D, double theta, float2* cs, cudaStream_t s);
+// The QR-Gaussian rotation of each sequence b (seed + b): q[b][D][D], fp64;
+// work holds batch * D * D doubles of scratch.
+jolt_status launch_qr_rotation(int D, int batch, uint64_t seed, double* work, double* q, cudaStream_t s);
 jolt_status launch_copy_out(const CellOut* out, int* rt, uint16_t** ut, int ncells, cudaStream_t s);
 
 // ------------------------------------------------------- randomized mode ---

@@ -6,7 +6,10 @@
 // X~ = U_T^ M^_lh. Keys get RoPE re-applied after decoding.
 //
 // This file holds the row-per-thread (SIMT) forms: the backbone product is
-// accumulated in fp32 registers, the transform runs inside the thread.
+// accumulated in fp32 registers, the transform runs inside the thread. It
+// also holds the page's own rotation, R = the Q of a seeded Gaussian's QR
+// factorization, as an option: r = Q e and e = Q^T r are dense row products
+// summed in fp64 and rounded once to fp32.
 #include "jolt_internal.cuh"
 #include "jolt_kernels.cuh"
 
@@ -32,6 +35,36 @@ __device__ __forceinline__ void unrotate_row(float* v, const float* sgn) {
   const float rs = rot_scale_f(D);
 #pragma unroll
   for (int d = 0; d < D; ++d) v[d] = __fmul_rn(__fmul_rn(v[d], rs), sgn[d]);
+}
+
+// r_i = fl32(sum_j Q[i][j] e_j), j ascending, fp64 fused multiply-adds. buf is
+// this thread's D floats of shared memory.
+template <int D>
+__device__ __forceinline__ void qr_rotate_row(float* v, const double* __restrict__ Q, float* buf) {
+#pragma unroll
+  for (int j = 0; j < D; ++j) buf[j] = v[j];
+#pragma unroll
+  for (int i = 0; i < D; ++i) {
+    const double* q = Q + i * D;
+    double s = 0.0;
+#pragma unroll 8
+    for (int j = 0; j < D; ++j) s = fma(q[j], (double)buf[j], s);
+    v[i] = (float)s;
+  }
+}
+
+// e_j = fl32(sum_i Q[i][j] r_i), i ascending, fp64 fused multiply-adds.
+template <int D>
+__device__ __forceinline__ void qr_unrotate_row(float* v, const double* __restrict__ Q, float* buf) {
+#pragma unroll
+  for (int j = 0; j < D; ++j) buf[j] = v[j];
+#pragma unroll
+  for (int j = 0; j < D; ++j) {
+    double s = 0.0;
+#pragma unroll 8
+    for (int i = 0; i < D; ++i) s = fma(Q[i * D + j], (double)buf[i], s);
+    v[j] = (float)s;
+  }
 }
 
 template <int D>
@@ -80,8 +113,9 @@ __device__ __forceinline__ void backbone_rows(const ResidArgs& a, int cell, cons
   }
 }
 
-template <int D>
+template <int D, bool QR>
 __global__ void __launch_bounds__(128) k_residual_simt(ResidArgs a) {
+  extern __shared__ float rowbuf[];   // QR: [128][D + 1], one row per thread
   const int cell = blockIdx.z, lh = blockIdx.y, t0 = blockIdx.x * 128;
   const CellDesc c = a.cells[cell];
   const CellOut o = a.out[cell];
@@ -98,14 +132,16 @@ __global__ void __launch_bounds__(128) k_residual_simt(ResidArgs a) {
   const int l = lh / c.H, h = lh % c.H;
 #pragma unroll
   for (int d = 0; d < D; ++d) acc[d] = __fsub_rn(x_elem(c, a.cs, l, h, t, d), acc[d]);
-  rotate_row<D>(acc, sg);
+  if constexpr (QR) qr_rotate_row<D>(acc, a.qrot + (int64_t)c.seq * D * D, rowbuf + threadIdx.x * (D + 1));
+  else rotate_row<D>(acc, sg);
   const int64_t row = (int64_t)lh * c.T + t;
   PackOp<D> op{acc, o.codes + row * (o.b * D / 8), o.scales + row * (D / a.G)};
   dispatch_gb<D>(a.G, o.b, op);
 }
 
-template <int D>
+template <int D, bool QR>
 __global__ void __launch_bounds__(128) k_decompress_simt(ResidArgs a) {
+  extern __shared__ float rowbuf[];   // QR: [128][D + 1], one row per thread
   const int cell = blockIdx.z, lh = blockIdx.y, t0 = blockIdx.x * 128;
   const CellDesc c = a.cells[cell];
   const CellOut o = a.out[cell];
@@ -125,7 +161,8 @@ __global__ void __launch_bounds__(128) k_decompress_simt(ResidArgs a) {
     const int64_t row = (int64_t)lh * c.T + t;
     UnpackOp<D> op{v, o.codes + row * (o.b * D / 8), o.scales + row * (D / a.G)};
     dispatch_gb<D>(a.G, o.b, op);
-    unrotate_row<D>(v, sg);
+    if constexpr (QR) qr_unrotate_row<D>(v, a.qrot + (int64_t)c.seq * D * D, rowbuf + threadIdx.x * (D + 1));
+    else unrotate_row<D>(v, sg);
 #pragma unroll
     for (int d = 0; d < D; ++d) acc[d] = __fadd_rn(acc[d], v[d]);
   }
@@ -149,20 +186,113 @@ __global__ void __launch_bounds__(128) k_decompress_simt(ResidArgs a) {
   }
 }
 
+template <class K>
+static jolt_status launch_rows(K kern, dim3 g, size_t smem, const ResidArgs& a, cudaStream_t s) {
+  if (smem) JOLT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  kern<<<g, 128, smem, s>>>(a);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
 jolt_status launch_residual_simt(const ResidArgs& a, int ncells, int D, int Tmax, int lh_max,
                                  cudaStream_t s) {
   dim3 g((Tmax + 127) / 128, lh_max, ncells);
-  if (D == 128) k_residual_simt<128><<<g, 128, 0, s>>>(a);
-  else k_residual_simt<64><<<g, 128, 0, s>>>(a);
-  JOLT_LAUNCHED();
-  return JOLT_OK;
+  const size_t qs = (size_t)128 * (D + 1) * sizeof(float);
+  if (a.qrot) return D == 128 ? launch_rows(k_residual_simt<128, true>, g, qs, a, s)
+                              : launch_rows(k_residual_simt<64, true>, g, qs, a, s);
+  return D == 128 ? launch_rows(k_residual_simt<128, false>, g, 0, a, s)
+                  : launch_rows(k_residual_simt<64, false>, g, 0, a, s);
 }
 
 jolt_status launch_decompress_simt(const ResidArgs& a, int ncells, int D, int Tmax, int lh_max,
                                    cudaStream_t s) {
   dim3 g((Tmax + 127) / 128, lh_max, ncells);
-  if (D == 128) k_decompress_simt<128><<<g, 128, 0, s>>>(a);
-  else k_decompress_simt<64><<<g, 128, 0, s>>>(a);
+  const size_t qs = (size_t)128 * (D + 1) * sizeof(float);
+  if (a.qrot) return D == 128 ? launch_rows(k_decompress_simt<128, true>, g, qs, a, s)
+                              : launch_rows(k_decompress_simt<64, true>, g, qs, a, s);
+  return D == 128 ? launch_rows(k_decompress_simt<128, false>, g, 0, a, s)
+                  : launch_rows(k_decompress_simt<64, false>, g, 0, a, s);
+}
+
+// ---------------------------------------------------- QR-Gaussian rotation --
+// Q of G = Q R for G a D x D matrix of standard normals (Philox4x32-10 words
+// of counter (i, 0, STREAM_QRGAUSS, 0) with key seed + b, u = (w + 0.5) 2^-32,
+// Box-Muller on (u0, u1) and (u2, u3); G[i][j] = z[i * D + j]). Householder
+// reflections H_k = I - beta_k v_k v_k^T with v_k = x - alpha e_1,
+// alpha = -sign(x_0) ||x|| (Golub & Van Loan, "Matrix Computations",
+// Section 5.1-5.2), Q = H_0 ... H_(D-1) accumulated backwards from I, then
+// column k negated where R_kk = alpha_k < 0 so that R's diagonal is positive.
+// One block per sequence; A (overwritten by the reflectors) and Q live in
+// global memory; reductions in a fixed order.
+__global__ void __launch_bounds__(256) k_qr_rotation(int D, uint64_t seed, double* __restrict__ work,
+                                                     double* __restrict__ qout) {
+  __shared__ double red[256];
+  __shared__ double alpha_s[128], beta_s[128];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  double* A = work + (int64_t)b * D * D;
+  double* Q = qout + (int64_t)b * D * D;
+  for (int i4 = tid; i4 < D * D / 4; i4 += blockDim.x) {
+    const u4 r = philox_at(seed + (uint64_t)b, STREAM_QRGAUSS, (uint32_t)i4);
+    const double u0 = ((double)r.x + 0.5) * 0x1p-32, u1 = ((double)r.y + 0.5) * 0x1p-32;
+    const double u2 = ((double)r.z + 0.5) * 0x1p-32, u3 = ((double)r.w + 0.5) * 0x1p-32;
+    const double r0 = sqrt(-2.0 * log(u0)), r1 = sqrt(-2.0 * log(u2));
+    const double t0 = 6.283185307179586 * u1, t1 = 6.283185307179586 * u3;
+    A[4 * i4 + 0] = r0 * cos(t0);
+    A[4 * i4 + 1] = r0 * sin(t0);
+    A[4 * i4 + 2] = r1 * cos(t1);
+    A[4 * i4 + 3] = r1 * sin(t1);
+  }
+  __syncthreads();
+  for (int k = 0; k < D; ++k) {
+    double part = 0.0;
+    for (int i = k + 1 + tid; i < D; i += blockDim.x) part += A[i * D + k] * A[i * D + k];
+    red[tid] = part;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+      if (tid < w) red[tid] += red[tid + w];
+      __syncthreads();
+    }
+    const double tail = red[0];           // sum of squares below the diagonal
+    const double x0 = A[k * D + k];
+    const double nrm = sqrt(tail + x0 * x0);
+    const double alpha = (x0 >= 0.0) ? -nrm : nrm;
+    const double vk = x0 - alpha;
+    const double vtv = vk * vk + tail;
+    const double beta = vtv > 0.0 ? 2.0 / vtv : 0.0;
+    __syncthreads();                      // every thread has read red[0] and A[k][k]
+    if (tid == 0) {
+      A[k * D + k] = vk;
+      alpha_s[k] = alpha;
+      beta_s[k] = beta;
+    }
+    __syncthreads();
+    for (int j = k + 1 + tid; j < D; j += blockDim.x) {
+      double w = 0.0;
+      for (int i = k; i < D; ++i) w = fma(A[i * D + k], A[i * D + j], w);
+      w *= beta;
+      for (int i = k; i < D; ++i) A[i * D + j] = fma(-w, A[i * D + k], A[i * D + j]);
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < D * D; e += blockDim.x) Q[e] = (e / D == e % D) ? 1.0 : 0.0;
+  __syncthreads();
+  for (int k = D - 1; k >= 0; --k) {
+    const double beta = beta_s[k];
+    for (int j = tid; j < D; j += blockDim.x) {
+      double w = 0.0;
+      for (int i = k; i < D; ++i) w = fma(A[i * D + k], Q[i * D + j], w);
+      w *= beta;
+      for (int i = k; i < D; ++i) Q[i * D + j] = fma(-w, A[i * D + k], Q[i * D + j]);
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < D * D; e += blockDim.x)
+    if (alpha_s[e % D] < 0.0) Q[e] = -Q[e];
+}
+
+jolt_status launch_qr_rotation(int D, int batch, uint64_t seed, double* work, double* q, cudaStream_t s) {
+  if (D > 128 || D % 4) { set_error("QR rotation supports D <= 128, D % 4 == 0"); return JOLT_ERR_UNSUPPORTED_SHAPE; }
+  k_qr_rotation<<<batch, 256, 0, s>>>(D, seed, work, q);
   JOLT_LAUNCHED();
   return JOLT_OK;
 }

@@ -18,7 +18,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "jolt.h")
 JOLT_BF16, JOLT_F32 = 0, 1
 JOLT_EXACT, JOLT_RANDOMIZED = 0, 1
 JOLT_MIN_ENUMERATE, JOLT_MIN_GREEDY = 0, 1
-JOLT_ROT_HADAMARD = 0
+JOLT_ROT_HADAMARD, JOLT_ROT_QR_GAUSS = 0, 1
 STATUS = {0: "JOLT_OK", 1: "JOLT_ERR_INVALID_ARG", 2: "JOLT_ERR_UNSUPPORTED_SHAPE",
           3: "JOLT_ERR_BUDGET_INFEASIBLE", 4: "JOLT_ERR_OOM", 5: "JOLT_ERR_CUDA",
           6: "JOLT_ERR_TIMEOUT", 7: "JOLT_ERR_NONFINITE"}
@@ -156,7 +156,8 @@ def make_options(mode: int = JOLT_EXACT, bits: Sequence[int] = (0, 2, 4, 8),
                  rt_grid: Optional[Sequence[int]] = None, rd_grid: Optional[Sequence[int]] = None,
                  rt_max: int = 0, oversample_p: int = 8, power_iters: int = 2,
                  scale_group: int = 0, budget_tol: float = 0.005,
-                 max_iters: int = 50, minimizer: int = 0) -> Tuple[jolt_options, list]:
+                 max_iters: int = 50, minimizer: int = 0,
+                 rotation: int = JOLT_ROT_HADAMARD) -> Tuple[jolt_options, list]:
     lib = load_library()
     o = jolt_options()
     lib.jolt_default_options(C.byref(o))
@@ -176,6 +177,7 @@ def make_options(mode: int = JOLT_EXACT, bits: Sequence[int] = (0, 2, 4, 8),
     o.rt_max, o.oversample_p, o.power_iters = rt_max, oversample_p, power_iters
     o.scale_group, o.budget_tol, o.max_iters = scale_group, budget_tol, max_iters
     o.minimizer = minimizer
+    o.rotation = rotation
     return o, keep
 
 
