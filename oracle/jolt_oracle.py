@@ -17,6 +17,7 @@ via Joint Rank-bit Allocation" (Krishnan & Schulz), Section 3:
                                        not in the oracle: the oracle is exact)
   * Section 3, layer grouping        -> layer_token_basis, basis_score,
                                        layer_scores, group_layers
+  * Section 3.1, decode kernel       -> reconstruct_f32, decode_attention
 and, for keys, the pre-RoPE handling of Section 3 (keys decomposed before the
 rotary embedding; the rotation re-applied to the reconstruction).
 
@@ -58,6 +59,9 @@ library as well):
      neighbours); below rank 8 the trailing basis vectors are arbitrary.
   R14 with a batch, the score of (l, l+1) is the mean over sequences.
   R15 median of the L-1 scores as numpy computes it; "falls below" is strict.
+  R18 decode attention: scores use the fp32 reconstruction (no bf16 storage
+     rounding: the fused kernel never stores the dense cache), scale
+     1/sqrt(D), one softmax over prefix and dense tail, fp64 arithmetic.
   R17 QR-Gaussian rotation (option rotation="qr"): R = Q of G = QR, G a D x D
      matrix of Philox/Box-Muller normals (row-major), R's diagonal made
      positive; r = Q e and e = Q^T r summed in fp64, rounded once to fp32.
@@ -753,9 +757,10 @@ def compress(cache_k: np.ndarray, cache_v: np.ndarray, group_starts: Sequence[in
     return Compressed(out, al, (B, L, H, T, D), rope_theta_k, seed, g, opt.rotation)
 
 
-def decompress_cell(cc: CompressedCell, D: int, g: int, seed: int, rope_theta_k: float,
+def reconstruct_f32(cc: CompressedCell, D: int, g: int, seed: int, rope_theta_k: float,
                     rotation: str = "hadamard") -> np.ndarray:
-    """X^ = bf16( [RoPE]( X~ + R^T dequant(codes) ) ), fp32 sum and RoPE."""
+    """[RoPE]( X~ + R^T dequant(codes) ) of one cell in fp32, before any
+    storage rounding: fp32 sum, RoPE (keys only) in fp32."""
     Xt = backbone(cc.fit)
     sg = rotation_for(D, seed + cc.ref.b, rotation)
     e = decode_residual(cc.res, g, sg, D)
@@ -763,7 +768,13 @@ def decompress_cell(cc: CompressedCell, D: int, g: int, seed: int, rope_theta_k:
     if cc.ref.kind == 0 and rope_theta_k > 0:
         cs, sn = rope_table(x.shape[2], D, rope_theta_k)
         x = rope_f32(x, cs, sn)
-    return bf16_rne(x)
+    return x
+
+
+def decompress_cell(cc: CompressedCell, D: int, g: int, seed: int, rope_theta_k: float,
+                    rotation: str = "hadamard") -> np.ndarray:
+    """X^ = bf16( [RoPE]( X~ + R^T dequant(codes) ) ), fp32 sum and RoPE."""
+    return bf16_rne(reconstruct_f32(cc, D, g, seed, rope_theta_k, rotation))
 
 
 def decompress(comp: Compressed) -> Tuple[np.ndarray, np.ndarray]:
@@ -869,3 +880,49 @@ def layer_groups(cache_k: np.ndarray, rope_theta_k: float = 0.0) -> Tuple[List[i
     """(group starts, scores) for a key cache [B, L, H, T, D]."""
     s = layer_scores(cache_k, rope_theta_k)
     return group_layers(s), s
+
+
+# --------------------------------------------------------------------------
+# decode attention over the compressed cache, Section 3.1 ("the FlashJoLT
+# decode kernel evaluates attention directly over the stored factors and
+# packed residual"); reading R18
+# --------------------------------------------------------------------------
+def layer_kv_f32(comp: Compressed, b: int, l: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Reconstructed keys (RoPE re-applied) and values of layer l, sequence b,
+    as fp32 [H, T, D], before the bf16 rounding of decompress."""
+    D = comp.shape[4]
+    K = V = None
+    for cc in comp.cells:
+        if cc.ref.b == b and cc.ref.l0 <= l < cc.ref.l1:
+            X = reconstruct_f32(cc, D, comp.g_of_D, comp.seed, comp.rope_theta_k, comp.rotation)[l - cc.ref.l0]
+            if cc.ref.kind == 0:
+                K = X
+            else:
+                V = X
+    return K, V
+
+
+def decode_attention(comp: Compressed, b: int, l: int, q: np.ndarray,
+                     tail_k: Optional[np.ndarray] = None, tail_v: Optional[np.ndarray] = None) -> np.ndarray:
+    """One decode step of layer l, sequence b: for query head j (q [Hq, D],
+    already rotated for its position), out_j = sum_t softmax_t(q_j . k_t /
+    sqrt(D)) v_t over the T reconstructed tokens followed by the dense tail
+    (tail_k, tail_v [H, n, D], keys already rotated), all in fp64. Query head j
+    reads KV head j // (Hq / H) (grouped-query attention)."""
+    K, V = layer_kv_f32(comp, b, l)
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    if tail_k is not None and tail_k.shape[1] > 0:
+        K = np.concatenate([K, np.asarray(tail_k, np.float64)], axis=1)
+        V = np.concatenate([V, np.asarray(tail_v, np.float64)], axis=1)
+    H, _, D = K.shape
+    q = np.asarray(q, np.float64)
+    Hq = q.shape[0]
+    per = Hq // H
+    out = np.zeros((Hq, D))
+    for j in range(Hq):
+        h = j // per
+        s = K[h] @ q[j] / math.sqrt(D)
+        p = np.exp(s - s.max())
+        out[j] = (p / p.sum()) @ V[h]
+    return out

@@ -213,3 +213,42 @@ def test_qr_rotation_transposed(monkeypatch):
 def test_qr_unrotation_transposed(monkeypatch):
     monkeypatch.setattr(o, "unrotate_qr", lambda r, Q: o.f32(np.asarray(r, np.float64) @ Q.T))
     _fails(pins.test_qr_rotation_residual_round_trip_error_bound)
+
+
+# ------------------------------------------------- decode attention plants
+import math as _math
+
+import test_oracle_decode as dpins
+
+
+def _bad_decode(head_of, scale):
+    def bad(comp, b, l, q, tail_k=None, tail_v=None):
+        K, V = o.layer_kv_f32(comp, b, l)
+        K, V = np.asarray(K, np.float64), np.asarray(V, np.float64)
+        if tail_k is not None and tail_k.shape[1] > 0:
+            K = np.concatenate([K, tail_k], axis=1)
+            V = np.concatenate([V, tail_v], axis=1)
+        H, _, D = K.shape
+        out = np.zeros((q.shape[0], D))
+        for j in range(q.shape[0]):
+            h = head_of(j, q.shape[0], H)
+            s = K[h] @ q[j] * scale(D)
+            p = np.exp(s - s.max())
+            out[j] = (p / p.sum()) @ V[h]
+        return out
+    return bad
+
+
+def test_decode_head_mapping_modulo(monkeypatch, comp):
+    monkeypatch.setattr(o, "decode_attention", _bad_decode(lambda j, Hq, H: j % H, lambda D: 1 / _math.sqrt(D)))
+    _fails(dpins.test_grouped_query_heads_read_their_kv_head, comp)
+
+
+def test_decode_without_scale(monkeypatch, comp):
+    monkeypatch.setattr(o, "decode_attention", _bad_decode(lambda j, Hq, H: j // (Hq // H), lambda D: 1.0))
+    _fails(dpins.test_matches_library_attention_with_tail, comp, 2)
+
+
+@pytest.fixture(scope="module")
+def comp():
+    return dpins.make_comp()
