@@ -5,8 +5,8 @@ prefix and a dense tail of new tokens).
 
 Expected values come from an independent library routine (torch's
 scaled_dot_product_attention in fp64 on the same tensors), from closed forms
-(a zero query averages the values; constant values pass through; a key far
-more aligned with the query than any other selects its value), and from the
+(a zero query averages the values, tail tokens included; a key far more
+aligned with the query than any other selects its value), and from the
 decompression path the other pins cover (the fp32 reconstruction rounds to
 decompress's bf16 output)."""
 import numpy as np
@@ -68,7 +68,7 @@ def test_matches_library_attention_with_tail(comp, Hq):
     assert np.abs(out0 - _sdpa(q, K.astype(np.float64), V.astype(np.float64))).max() < 1e-12
 
 
-def test_zero_query_averages_values_and_constant_values_pass(comp):
+def test_zero_query_averages_values_tail_included(comp):
     D = comp.shape[4]
     K, V = o.layer_kv_f32(comp, 0, 0)
     out = o.decode_attention(comp, 0, 0, np.zeros((2, D)))
