@@ -13,8 +13,10 @@ via Joint Rank-bit Allocation" (Krishnan & Schulz), Section 3:
                                        eps2_table
   * "Solving the allocation"        -> Eqs. (3)-(4): argmin_cell, allocate,
                                        greedy_cell (the page's own heuristic)
-  * Section 3.1 "FlashJoLT", Eq. (5) -> q_cap (the randomized mode itself is
-                                       not in the oracle: the oracle is exact)
+  * Section 3.1 "FlashJoLT", Eq. (5) -> q_cap, randomized_token_spectrum (the
+                                       randomized SVD the page cites, with the
+                                       sketch passed in; the end-to-end oracle
+                                       path is exact)
   * Section 3, layer grouping        -> layer_token_basis, basis_score,
                                        layer_scores, group_layers
   * Section 3.1, decode kernel       -> reconstruct_f32, decode_attention
@@ -404,6 +406,31 @@ def token_spectrum(X: np.ndarray, r_needed: Optional[int] = None):
     sv = np.sqrt(w[:r])
     U = (XT @ V[:, :r]) / np.where(sv > 0, sv, 1.0)[None, :]
     return w, fix_signs(U)
+
+
+def randomized_token_spectrum(X: np.ndarray, Omega: np.ndarray, n_iter: int, q_cap: int):
+    """Section 3.1 (FlashJoLT): the leading q_cap token-mode singular values
+    from the randomized SVD the page cites (Halko, Martinsson, Tropp, "Finding
+    structure with randomness", SIAM Review 2011: randomized subspace
+    iteration, then the SVD of B = Q^T A), all in fp64:
+      A = X_(T) (T x N); Q = orth(A Omega);
+      n_iter times: Q = orth(A^T Q), then Q = orth(A Q);
+      B = Q^T A; sigma~^2 = squared singular values of B, descending.
+    Omega (N x k, k >= q_cap) is an input: the random draw of the method.
+    Returns (spectrum, U): the q_cap leading sigma~^2 followed by the synthetic
+    tail entry max(0, ||X||^2 - their sum) (the page's single tail entry), and
+    the q_cap leading left vectors U = Q U_B (signs fixed)."""
+    A = token_unfolding(X)
+    Q = np.linalg.qr(A @ Omega)[0]
+    for _ in range(n_iter):
+        Q = np.linalg.qr(A.T @ Q)[0]
+        Q = np.linalg.qr(A @ Q)[0]
+    Bm = Q.T @ A
+    Ub, sv, _ = np.linalg.svd(Bm, full_matrices=False)
+    w = sv[:q_cap] ** 2
+    tail = max(0.0, float(np.sum(A * A)) - float(np.sum(w)))
+    U = fix_signs(Q @ Ub[:, :q_cap])
+    return np.concatenate([w, [tail]]), U
 
 
 def feature_spectrum(X: np.ndarray) -> np.ndarray:

@@ -252,3 +252,34 @@ def test_decode_without_scale(monkeypatch, comp):
 @pytest.fixture(scope="module")
 def comp():
     return dpins.make_comp()
+
+
+# --------------------------------------------- randomized spectrum plants
+import test_oracle_randomized as rpins
+
+_rand_orig = o.randomized_token_spectrum
+
+
+def test_randomized_without_tail(monkeypatch):
+    def bad(X, Om, n_iter, q):
+        w, U = _rand_orig(X, Om, n_iter, q)
+        w = w.copy()
+        w[-1] = 0.0
+        return w, U
+    monkeypatch.setattr(o, "randomized_token_spectrum", bad)
+    _fails(rpins.test_ritz_values_interlace_and_tail_bounds_discarded_energy, 1)
+
+
+def test_randomized_values_not_squared(monkeypatch):
+    def bad(X, Om, n_iter, q):
+        w, U = _rand_orig(X, Om, n_iter, q)
+        head = np.sqrt(w[:q])
+        A = o.token_unfolding(X)
+        return np.concatenate([head, [max(0.0, float(np.sum(A * A)) - float(np.sum(head)))]]), U
+    monkeypatch.setattr(o, "randomized_token_spectrum", bad)
+    _fails(rpins.test_low_rank_input_is_recovered_exactly)
+
+
+def test_randomized_power_iterations_skipped(monkeypatch):
+    monkeypatch.setattr(o, "randomized_token_spectrum", lambda X, Om, n_iter, q: _rand_orig(X, Om, 0, q))
+    _fails(rpins.test_power_iterations_approach_the_exact_values)
