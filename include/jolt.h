@@ -13,6 +13,9 @@
  *      Lagrange multiplier under a single byte budget (Section 3, Eqs. 1-4),
  *   4. optionally a randomized token-mode SVD (Section 3.1, "FlashJoLT",
  *      Eq. 5 for the rank cap).
+ * It also provides the data-driven layer grouping that precedes compression
+ * (Section 3; jolt_layer_groups) and, as an option, the page's own
+ * QR-Gaussian residual rotation (jolt_options.rotation).
  *
  * Conventions for every entry point:
  *   * Device pointers are CUDA device (or managed) memory of the current
