@@ -59,3 +59,15 @@ def test_reference_arm_other_ranks_exit_without_work():
                        env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_grouping_roofline_arithmetic():
+    import bench
+    # LLaMA-3.1-8B-shaped 64K key cache: 2^32 bf16 keys; 4 power iterations = 10 passes
+    n = 32 * 8 * 65536 * 128
+    r = bench.grouping_roofline(43.8, n, 2, 4, 148)
+    assert r["peak"] == 74.4                       # 148 x 128 x 2 x 1.965 GHz
+    flops = 10 * 2 * 16 * n
+    assert abs(r["achieved"] - flops / 43.8e-3 / 1e12) < 0.01
+    assert r["key_gb_read"] == round(10 * n * 2 / 1e9, 2)
+    assert r["bound"] == "alu" and 0 < r["frac"] < 1
