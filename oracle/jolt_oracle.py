@@ -119,11 +119,12 @@ def philox_block(n_ctr: int, seed: int, stream: int, hi: int = 0) -> np.ndarray:
     return philox4x32_10(ctr, (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF))
 
 
-def gaussian_f64(n: int, seed: int, stream: int) -> np.ndarray:
+def gaussian_f64(n: int, seed: int, stream: int, hi: int = 0) -> np.ndarray:
     """n standard normals: each Philox call gives 4 words, u = (w + 0.5) 2^-32,
-    and Box-Muller turns (u0, u1) and (u2, u3) into two pairs (fp64)."""
+    and Box-Muller turns (u0, u1) and (u2, u3) into two pairs (fp64). hi is
+    the counter's second word."""
     nc = (n + 3) // 4
-    w = philox_block(nc, seed, stream).astype(np.float64)
+    w = philox_block(nc, seed, stream, hi).astype(np.float64)
     u = (w + 0.5) * (2.0 ** -32)
     r0 = np.sqrt(-2.0 * np.log(u[:, 0]))
     r1 = np.sqrt(-2.0 * np.log(u[:, 2]))
@@ -406,6 +407,16 @@ def token_spectrum(X: np.ndarray, r_needed: Optional[int] = None):
     sv = np.sqrt(w[:r])
     U = (XT @ V[:, :r]) / np.where(sv > 0, sv, 1.0)[None, :]
     return w, fix_signs(U)
+
+
+def library_sketch(N: int, k: int, ld: int, seed: int, hi: int) -> np.ndarray:
+    """The sketch Omega (N x k) that the CUDA library draws for one cell, from
+    the same counter-based generator (reading R10): column j, row n is
+    bf16(z[j * ld + n]) with z = gaussian_f64 on stream STREAM_SKETCH, key
+    seed = run seed + sequence, counter word hi = 2 * group + kind, and ld the
+    largest N over the cache's cells (the library's row pitch)."""
+    z = gaussian_f64(k * ld, seed, STREAM_SKETCH, hi)
+    return bf16_rne(z).reshape(k, ld)[:, :N].T
 
 
 def randomized_token_spectrum(X: np.ndarray, Omega: np.ndarray, n_iter: int, q_cap: int):

@@ -59,3 +59,19 @@ def test_power_iterations_approach_the_exact_values():
         err.append(np.abs(w[:8] - s[:8] ** 2).max() / s[0] ** 2)
     assert err[2] < err[1] < err[0]
     assert err[2] < 1e-4
+
+
+def test_library_sketch_layout_and_rounding():
+    N, k = 40, 16
+    a = o.library_sketch(N, k, N, 7, 0)
+    z = o.gaussian_f64(k * N, 7, o.STREAM_SKETCH)
+    assert np.array_equal(a, o.bf16_rne(z).reshape(k, N).T)
+    # values are bf16: 8 significant bits
+    m, _ = np.frexp(a[a != 0])
+    assert np.all(np.rint(m * 256) == m * 256)
+    # a wider pitch takes the first N of each row of length ld
+    b = o.library_sketch(N, k, 48, 7, 0)
+    z48 = o.bf16_rne(o.gaussian_f64(k * 48, 7, o.STREAM_SKETCH)).reshape(k, 48)
+    assert np.array_equal(b, z48[:, :N].T)
+    # the counter word separates cells
+    assert not np.array_equal(o.library_sketch(N, k, N, 7, 1), a)
