@@ -95,3 +95,38 @@ def test_randomized_spectrum_tracks_exact():
             assert np.max(np.abs(np.array(sd[i]) - wD)) <= 2e-3 * wD[0]
     finally:
         jolt.jolt_free_plan(plan)
+
+
+@pytest.mark.parametrize("name,C_ratio", [("tiny", 2.0), ("mistral", 3.0)])
+def test_randomized_spectrum_matches_oracle_on_the_same_sketch(name, C_ratio):
+    """Spectrum-level parity of the randomized range finder: jolt_rd_table
+    (randomized, seed 0) against oracle.randomized_token_spectrum fed the
+    library's own draw of Omega (library_sketch). In exact arithmetic both
+    span the same subspace; the GPU rounds its GEMM operands (X, Omega, the
+    iterates W and Z) to bf16 (relative 2^-9), which moves the Ritz values by
+    a small multiple of that relative to sigma_1^2; the bound 1e-2 sigma_1^2
+    leaves a margin of five."""
+    spec = synth.SPECS[name]
+    K, V = synth.make_cache(spec, 0)
+    gs = synth.group_starts(spec)
+    B = o.budget_for_ratio(K.numel() * 2, C_ratio)
+    Kd, Vd = K.cuda(), V.cuda()
+    lay, keep = jolt.make_layout(Kd, gs, spec.rope_theta_k)
+    opt, k2 = jolt.make_options(mode=jolt.JOLT_RANDOMIZED)
+    plan = jolt.jolt_plan(lay, B, opt)
+    try:
+        n = jolt.jolt_num_cells(plan)
+        qc = o.q_cap(spec.seq_len, C_ratio)
+        ns, st, nt, sd = jolt.jolt_rd_table(plan, Kd, Vd, n, qc + 1, spec.head_dim)
+    finally:
+        jolt.jolt_free_plan(plan)
+    k = ((qc + 8 + 15) // 16) * 16                 # q_cap + p rounded up to 16
+    refs = o.cells_of(1, gs)
+    ld = max((c.l1 - c.l0) * spec.n_heads * spec.head_dim for c in refs)
+    for i, c in enumerate(refs):
+        X = o.cell_tensor(K.float().numpy(), V.float().numpy(), c, spec.rope_theta_k)
+        N = (c.l1 - c.l0) * spec.n_heads * spec.head_dim
+        Om = o.library_sketch(N, k, ld, 0 + c.b, 2 * c.g + c.kind)
+        w, _ = o.randomized_token_spectrum(X, Om, 2, qc)
+        rel = np.abs(np.array(st[i][:qc]) - w[:qc]) / w[0]
+        assert rel.max() < 1e-2, (i, rel.max())
