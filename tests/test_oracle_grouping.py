@@ -175,3 +175,17 @@ def test_groups_of_planted_cache():
     starts, s = o.layer_groups(X)
     assert np.allclose(s, np.array(ov) / 8, atol=1e-9)
     assert starts == [0, 2, 4, 6, 8, 11]
+
+
+def test_score_against_library_principal_angles():
+    # scipy computes principal angles by its own (SVD-based, sine/cosine
+    # switching) method; the score is the mean squared cosine over them
+    from scipy.linalg import subspace_angles
+    rng = np.random.default_rng(21)
+    for _ in range(5):
+        Ua = _orthonormal(120, 8, rng)
+        Ub = _orthonormal(120, 8, rng)
+        mix = 0.3 * Ua + Ub                          # partial alignment
+        Ub = np.linalg.qr(mix)[0]
+        th = subspace_angles(Ua, Ub)
+        assert o.basis_score(Ua, Ub) == pytest.approx(float(np.mean(np.cos(th) ** 2)), abs=1e-12)
