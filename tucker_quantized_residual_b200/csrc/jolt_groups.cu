@@ -20,10 +20,10 @@
 // averaged over the batch's sequences. One thread then takes the median and
 // applies the rule.
 //
-// Precision: the T-sized passes (X Z, X^T Q) multiply in fp32 with fp32
-// accumulators over one 128-row tile (X^T Q) or one row (X Z) and fp64
-// across tiles (X^T Q); Grams, Cholesky factors, the Jacobi solve and the scores are
-// fp64. Q is kept in fp32.
+// Precision: the T-sized passes (X Z, X^T Q) multiply in fp32. X Z sums a
+// whole row in fp32; X^T Q sums one 128-row tile in fp32 and the tiles in
+// fp64. Grams, Cholesky factors, the Jacobi solve and the scores are fp64;
+// Q is kept in fp32.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -43,9 +43,9 @@ constexpr int TM = 128;           // rows per tile in X Z and X^T Q
 constexpr int XTQ_TILES = 16;     // tiles per X^T Q block (2048 rows)
 constexpr int GRAM_ROWS = 4096;   // rows per Gram partial
 constexpr int MAX_LAYERS = 1024;
-constexpr uint32_t STREAM_GROUPING = 5;
 
-// Where one job's keys are: element (t, h, d) at x + h*sh + t*st + d.
+// Where one job's keys are: for job = b * L + l, element (t, h, d) at
+// k + b*sb + l*sl + h*sh + t*st + d (strides in elements).
 struct KeySrc {
   const void* k;
   int f32;

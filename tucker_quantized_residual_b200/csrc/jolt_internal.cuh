@@ -86,7 +86,13 @@ __host__ __device__ inline u4 philox4x32_10(u4 c, uint32_t k0, uint32_t k1) {
 }
 
 // stream tags in the third counter word
-enum : uint32_t { STREAM_HADAMARD = 1, STREAM_CALIB = 2, STREAM_SKETCH = 3, STREAM_QRGAUSS = 4 };
+enum : uint32_t {
+  STREAM_HADAMARD = 1,    // residual rotation signs
+  STREAM_CALIB = 2,       // eps^2 calibration samples
+  STREAM_SKETCH = 3,      // range-finder sketch Omega
+  STREAM_QRGAUSS = 4,     // QR-Gaussian rotation matrix
+  STREAM_GROUPING = 5     // layer-grouping sketch
+};
 
 __host__ __device__ inline u4 philox_at(uint64_t seed, uint32_t stream, uint32_t i, uint32_t hi = 0) {
   return philox4x32_10(u4{i, hi, stream, 0u}, (uint32_t)seed, (uint32_t)(seed >> 32));
