@@ -231,9 +231,12 @@ JOLT_API jolt_status jolt_eps2(const int32_t* bits, int32_t n, int32_t group,
  * Asynchronous on `stream`; the caller synchronises before reading eps2_dev.
  * Partial sums live in a static 9 KB device array that every GPU loading the
  * library holds until exit (limit: 128 partial blocks x 9 slots, i.e. up to 8
- * bit widths and any supported group). The first call on each device looks up
- * that array's address (cudaGetSymbolAddress, with that device current); make
- * this first call before any stream capture. All calls share the array and it
+ * bit widths and any supported group). The first call in each CUDA context
+ * (the primary context of each device, or any other context made current)
+ * looks up that array's address there (cudaGetSymbolAddress, with that device
+ * current) and caches it; make this first call before any stream capture. A
+ * device reset unloads the array: after cudaDeviceReset, do not call this
+ * entry point again in the same process. All calls share the array and it
  * keeps the last call's contents: calls whose work overlaps on the GPU race,
  * so issue them on one stream or order them. Arguments beyond the limits
  * return JOLT_ERR_INVALID_ARG with a message naming the limit. */
@@ -254,6 +257,37 @@ JOLT_API jolt_status jolt_residual_decode(const uint8_t* codes, const float* sca
                                  int64_t rows, int32_t D, int32_t bits,
                                  int32_t group, uint64_t seed, float* e_hat,
                                  jolt_stream_t stream);
+
+/* The residual stage exactly as jolt_compress runs it (the tensor-core
+ * stream kernel of Section 3, "Rotated low-bit residual": E = X - U_T^ M^_lh
+ * per (layer, head), keys un-RoPE'd first, the seeded Hadamard rotation,
+ * absmax quantization, LSB-first packing), on caller-given factors instead of
+ * fitted ones, so that its codes and scales can be checked bit for bit.
+ *   x: DEVICE bf16 [LH][T][D], 16-byte aligned (LH = layer-head pairs).
+ *   ut_t: DEVICE bf16 [r][T], U_T^ transposed (1 <= r <= 512).
+ *   m: DEVICE bf16 [LH][r][D], the per-(layer, head) products M^.
+ *   rope_theta > 0: x holds keys after a rotate-half RoPE of that base over
+ *     positions 0..T-1, undone in fp32 before the residual (as jolt_compress
+ *     does for keys).
+ *   codes: DEVICE [LH][T][bits*D/8]; scales: DEVICE fp32 [LH][T][D/group]
+ *     (both 16-byte aligned). bits in {2,3,4,8}; group 32, 64 or D.
+ * Allocates scratch through the library allocator and synchronises the
+ * stream; a device status (timeout) is returned as for jolt_compress. */
+JOLT_API jolt_status jolt_residual_stream_encode(const void* x, int32_t LH, int32_t T, int32_t D,
+                                                 const uint16_t* ut_t, int32_t r, const uint16_t* m,
+                                                 int32_t bits, int32_t group, uint64_t seed, float rope_theta,
+                                                 uint8_t* codes, float* scales, jolt_stream_t stream);
+
+/* The Gaussian sketch Omega of Section 3.1 (the randomized range finder's
+ * test matrix) that jolt_compress and jolt_rd_table draw for every cell of a
+ * JOLT_RANDOMIZED plan with this seed: column j of cell c's Omega is row j of
+ * omega_t[c] (DEVICE, bf16 bit patterns, [n_cells][k][ld]); entries n >= N_c
+ * (N_c = L_g*H*D of the cell) are zero. k (the sketch width, q_cap + p
+ * rounded up to 16) and ld (the largest N_c) are written to *k_out / *ld_out
+ * (HOST, either may be NULL). omega_t NULL returns only k and ld.
+ * JOLT_ERR_INVALID_ARG for an exact-mode plan. Asynchronous. */
+JOLT_API jolt_status jolt_sketch(jolt_plan_t* plan, uint64_t seed, uint16_t* omega_t, int32_t* k_out,
+                                 int32_t* ld_out, jolt_stream_t stream);
 
 /* Data-driven layer grouping (Section 3, the paragraph that partitions the L
  * layers into G contiguous groups, and its footnote on size bounds): for each

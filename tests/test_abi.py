@@ -102,3 +102,48 @@ def test_layer_groups_single_layer_needs_no_device():
     L, keep = _layout(groups=(0, 1))
     st, starts, ng = _groups_call(L)
     assert st == 0 and ng == 1 and starts[:2] == [0, 1]
+
+
+@pytest.mark.parametrize("bad", ["not_tensor", "dtype", "strided", "short", "cpu"])
+def test_noalloc_wrapper_rejects_outputs_the_library_cannot_write(bad):
+    """The C entry point only sees a raw pointer and writes len(bits) doubles
+    there from a kernel; the binding refuses anything else before the call."""
+    import torch
+    bits = (0, 2, 4, 8)
+    out = {"not_tensor": [0.0] * 4,
+           "dtype": torch.zeros(4, dtype=torch.float32),
+           "strided": torch.zeros(8, dtype=torch.float64)[::2],
+           "short": torch.zeros(3, dtype=torch.float64),
+           "cpu": torch.zeros(4, dtype=torch.float64)}[bad]
+    with pytest.raises((TypeError, ValueError)):
+        jolt.jolt_eps2_noalloc(bits, 128, out)
+
+
+def test_plan_reports_oom_from_a_failing_allocator_without_touching_the_device():
+    """jolt_plan asks the registered allocator for its workspace before any
+    CUDA call; a NULL answer is JOLT_ERR_OOM and nothing is freed."""
+    lib = jolt.load_library()
+    calls = {"alloc": 0, "free": 0}
+    AF = C.CFUNCTYPE(C.c_void_p, C.c_size_t, C.c_void_p, C.c_void_p)
+    FF = C.CFUNCTYPE(None, C.c_void_p, C.c_void_p, C.c_void_p)
+
+    def a(n, s, ctx):
+        calls["alloc"] += 1
+        return None
+
+    def f(p, s, ctx):
+        calls["free"] += 1
+
+    af, ff = AF(a), FF(f)
+    assert lib.jolt_set_allocator(C.cast(af, C.c_void_p), C.cast(ff, C.c_void_p), None) == 0
+    try:
+        L, keep = _layout()
+        o, k2 = jolt.make_options()
+        with pytest.raises(jolt.JoltError) as ei:
+            jolt.jolt_plan(L, 10 ** 6, o)
+        assert ei.value.status == 4
+        assert calls == {"alloc": 1, "free": 0}
+    finally:
+        assert lib.jolt_set_allocator(None, None, None) == 0
+    # only one of the two callbacks is an error
+    assert lib.jolt_set_allocator(C.cast(af, C.c_void_p), None, None) == 1

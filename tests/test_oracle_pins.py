@@ -505,3 +505,45 @@ def test_qr_rotation_residual_round_trip_error_bound():
     err = np.linalg.norm(back - E, axis=1)
     bound = np.sqrt(D) * res.scales[:, 0] / 2 * 1.001 + 1e-5
     assert np.all(err <= bound)
+
+
+# --------------------------------------------------------------------------
+# Reading R9: which (r_T, r_d) pairs are admissible options
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("rT", [2, 3, 5])
+def test_admissible_feature_ranks_end_where_the_projected_gram_runs_out_of_rank(rT):
+    """The token-projected tensor Y = X x_T U_T^T has a feature unfolding of
+    D rows and L_g*H*r_T columns, so its feature Gram has rank at most
+    L_g*H*r_T: feature ranks beyond that add null-space columns and cannot
+    lower the backbone error (Section 3, "Partial Tucker backbone"). With fp64
+    storage, fit() shows the error falling strictly up to that rank and flat
+    after it; CellTable.valid must admit exactly the ranks up to the first
+    r_d at which the error reaches its floor."""
+    rng = np.random.default_rng(rT)
+    Lg, H, T, D = 1, 2, 40, 16
+    X = rng.standard_normal((Lg, H, T, D))
+    _, U = o.token_spectrum(X)
+    errs = []
+    for rd in range(1, D + 1):
+        f = o.fit(X, U, rT, rd, store_f64=True)
+        errs.append(float(np.sum((X - o.backbone(f)) ** 2)))
+    floor = errs[-1]
+    r_floor = next(rd for rd in range(1, D + 1) if errs[rd - 1] <= floor * (1 + 1e-10))
+    assert all(errs[i + 1] < errs[i] * (1 - 1e-8) for i in range(r_floor - 1))
+    assert r_floor == Lg * H * rT          # the boundary the algebra fixes
+    tab = o.CellTable(Lg, H, T, D, D, 1.0, np.zeros(T + 1), np.zeros(D + 1), np.arange(1, 9),
+                      np.arange(1, D + 1), np.array([0]), np.array([1.0]))
+    assert [bool(tab.valid(rT, rd)) for rd in range(1, D + 1)] == [rd <= r_floor for rd in range(1, D + 1)]
+
+
+def test_tiny_grid_excludes_exactly_one_pair_per_bit_width():
+    """On the tiny grid (L_g = H = 2: r_d <= 4 r_T), only (r_T, r_d) = (8, 48)
+    is ruled out, for each of the 5 bit widths: 5 of the 60 options carry
+    e = +inf and the enumeration skips exactly them."""
+    tab = _tiny_tables()[0]
+    full = {(int(b), int(t), int(d)) for b in tab.bits for t in tab.rt_grid for d in tab.rd_grid}
+    listed = {(b, t, d) for b, t, d, _, _ in tab.options()}
+    assert full - listed == {(int(b), 8, 48) for b in tab.bits}
+    b, t, d, e, s = tab.arrays()
+    assert sorted(zip(b[np.isinf(e)].tolist(), t[np.isinf(e)].tolist(), d[np.isinf(e)].tolist())) == \
+        sorted((int(x), 8, 48) for x in tab.bits)

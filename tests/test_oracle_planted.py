@@ -283,3 +283,15 @@ def test_randomized_values_not_squared(monkeypatch):
 def test_randomized_power_iterations_skipped(monkeypatch):
     monkeypatch.setattr(o, "randomized_token_spectrum", lambda X, Om, n_iter, q: _rand_orig(X, Om, 0, q))
     _fails(rpins.test_power_iterations_approach_the_exact_values)
+
+
+def test_admissible_pairs_strict(monkeypatch):
+    monkeypatch.setattr(o.CellTable, "valid", lambda self, rT, rd: rd < self.Lg * self.H * rT)
+    _fails(pins.test_tiny_grid_excludes_exactly_one_pair_per_bit_width)
+    _fails(pins.test_admissible_feature_ranks_end_where_the_projected_gram_runs_out_of_rank, 3)
+
+
+def test_admissible_pairs_without_heads(monkeypatch):
+    monkeypatch.setattr(o.CellTable, "valid", lambda self, rT, rd: rd <= self.Lg * rT)
+    _fails(pins.test_tiny_grid_excludes_exactly_one_pair_per_bit_width)
+    _fails(pins.test_admissible_feature_ranks_end_where_the_projected_gram_runs_out_of_rank, 3)

@@ -131,11 +131,18 @@ __global__ void k_rd_tables(const CellRD* __restrict__ cells, int ncells,
   else { w = wT[c]; t = tT[c]; n = nt_used[c]; }
   double acc = 0.0;
   t[n] = 0.0;
+  bool finite = true;
   for (int i = n - 1; i >= 0; --i) {
-    acc += fmax(w[i], 0.0);
+    // a non-finite spectrum entry (from Inf/NaN in the cache) is reported and
+    // counted as zero, so the table, and every option the allocator decodes
+    // from it, stays finite
+    double wi = w[i];
+    if (!isfinite(wi)) { finite = false; wi = 0.0; }
+    acc += fmax(wi, 0.0);
     t[i] = acc / ns;
   }
   t[n] = 0.0;
+  if (!finite) atomicOr(status, DEV_ERR_NONFINITE);
 }
 
 jolt_status launch_rd_tables(const CellRD* cells, int ncells, const double* const* wT,
@@ -279,6 +286,12 @@ __global__ void __launch_bounds__(512) k_alloc_decide(AllocArgs a) {
       double v = a.pv[c * a.nchunk + k];
       int i = a.pi[c * a.nchunk + k];
       if (v < best || (v == best && i < bidx)) { best = v; bidx = i; }
+    }
+    // no finite e + lambda s in any chunk (non-finite inputs): fall back to the
+    // first option, whose grid indices are valid, and report the cell
+    if (bidx < 0 || bidx >= a.n_bits * a.cells[c].n_rt * a.n_rd) {
+      bidx = 0;
+      atomicOr(a.status, DEV_ERR_NONFINITE);
     }
     a.cur[c] = bidx;
     int bi, rt, rd;

@@ -930,6 +930,20 @@ static jolt_status run_allocation(jolt_plan_s* p, int64_t budget, const double* 
   return launch_alloc(a, st, s);
 }
 
+// Randomized mode reads K and V through TMA unless the plan makes working
+// copies; a TMA tensor map needs a 16-byte-aligned base address.
+static jolt_status check_tma_inputs(const jolt_plan_s* p, const void* k, const void* v) {
+  if (p->opt.mode != JOLT_RANDOMIZED) return JOLT_OK;
+  const bool bad_k = !p->copy_k && reinterpret_cast<uintptr_t>(k) % 16;
+  const bool bad_v = !p->copy_v && reinterpret_cast<uintptr_t>(v) % 16;
+  if (bad_k || bad_v) {
+    set_error("randomized mode reads %s through TMA: its base pointer must be 16-byte aligned",
+              bad_k ? "K" : "V");
+    return JOLT_ERR_UNSUPPORTED_SHAPE;
+  }
+  return JOLT_OK;
+}
+
 extern "C" {
 
 void jolt_free_plan(jolt_plan_t* p) {
@@ -944,6 +958,7 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   cudaStream_t s = (cudaStream_t)stream_;
   if (!p || !k || !v || !out) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
   *out = nullptr;
+  JOLT_TRY(check_tma_inputs(p, k, v));
   const int64_t B = byte_budget > 0 ? byte_budget : p->budget;
   int64_t minsum = 0, extra = 0;
   for (auto& c : p->hc) {
@@ -1122,6 +1137,7 @@ jolt_status jolt_rd_table(jolt_plan_t* p, const void* k, const void* v, double* 
   cudaStream_t s = (cudaStream_t)stream_;
   if (!p || !k || !v || !norm_sq || !sig_t || !n_t || !sig_d) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
   if (max_t < p->nt_max) { set_error("max_t must be >= %d", p->nt_max); return JOLT_ERR_INVALID_ARG; }
+  JOLT_TRY(check_tma_inputs(p, k, v));
   JOLT_CUDA_TRY(cudaMemsetAsync(p->d_status, 0, sizeof(int), s));
   JOLT_TRY(upload_cells(p, k, v, s));
   JOLT_TRY(run_spectra(p, k, v, 0, p->d_status, s));
@@ -1211,6 +1227,95 @@ jolt_status jolt_residual_decode(const uint8_t* codes, const float* scales, int6
   JOLT_TRY(check_rows(D, bits, group));
   if (rows < 0 || (rows > 0 && (!e_hat || !codes || !scales))) { set_error("bad arguments"); return JOLT_ERR_INVALID_ARG; }
   return launch_decode_rows(codes, scales, rows, D, bits, group, seed, e_hat, (cudaStream_t)stream_);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------ single-stage hooks --
+extern "C" {
+
+jolt_status jolt_sketch(jolt_plan_t* p, uint64_t seed, uint16_t* omega_t, int32_t* k_out, int32_t* ld_out,
+                        jolt_stream_t stream_) {
+  if (!p) { set_error("null plan"); return JOLT_ERR_INVALID_ARG; }
+  if (p->opt.mode != JOLT_RANDOMIZED) { set_error("the plan is not in JOLT_RANDOMIZED mode: it draws no sketch"); return JOLT_ERR_INVALID_ARG; }
+  if (k_out) *k_out = p->k;
+  if (ld_out) *ld_out = p->Ncmax;
+  if (!omega_t) return JOLT_OK;
+  if (reinterpret_cast<uintptr_t>(omega_t) % 8) { set_error("omega_t must be 8-byte aligned"); return JOLT_ERR_INVALID_ARG; }
+  return launch_omega(omega_t, p->ncells, p->k, p->Ncmax, p->d_Nc, p->d_cb, p->d_cis, seed, (cudaStream_t)stream_);
+}
+
+jolt_status jolt_residual_stream_encode(const void* x, int32_t LH, int32_t T, int32_t D, const uint16_t* ut_t,
+                                        int32_t r, const uint16_t* m, int32_t bits, int32_t group, uint64_t seed,
+                                        float rope_theta, uint8_t* codes, float* scales, jolt_stream_t stream_) {
+  cudaStream_t s = (cudaStream_t)stream_;
+  JOLT_TRY(check_rows(D, bits, group));
+  if (!x || !ut_t || !m || !codes || !scales) { set_error("null pointer"); return JOLT_ERR_INVALID_ARG; }
+  if (LH < 1 || T < 1 || r < 1 || r > 512 || !(rope_theta >= 0.0f)) {
+    set_error("need LH >= 1, T >= 1, 1 <= r <= 512 and rope_theta >= 0"); return JOLT_ERR_INVALID_ARG;
+  }
+  if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(codes) % 16 ||
+      reinterpret_cast<uintptr_t>(scales) % 16) {
+    set_error("x, codes and scales must be 16-byte aligned"); return JOLT_ERR_UNSUPPORTED_SHAPE;
+  }
+  const int tp = (T + 7) / 8 * 8, rows = (r + 63) / 64 * 64;
+  Arena A;
+  CellDesc* d_cell = nullptr; CellOut* d_out = nullptr; uint16_t** d_M = nullptr; int* d_rmax = nullptr;
+  int* d_status = nullptr; uint16_t* ut_ws = nullptr; uint16_t* mt_ws = nullptr; float2* cs = nullptr;
+  void* block = nullptr;
+  for (int pass = 0; pass < 2; ++pass) {
+    A.used = 0;
+    d_cell = A.take<CellDesc>(1);
+    d_out = A.take<CellOut>(1);
+    d_M = A.take<uint16_t*>(1);
+    d_rmax = A.take<int>(1);
+    d_status = A.take<int>(4);
+    ut_ws = A.take<uint16_t>((size_t)rows * tp);
+    mt_ws = A.take<uint16_t>((size_t)LH * D * rows);
+    cs = rope_theta > 0.0f ? A.take<float2>((size_t)T * (D / 2)) : nullptr;
+    if (pass == 0) {
+      block = dev_alloc(A.used + 256, s);
+      if (!block) { set_error("scratch allocation failed"); return JOLT_ERR_OOM; }
+      A.base = reinterpret_cast<uint8_t*>(block);
+    }
+  }
+  jolt_status st = JOLT_OK;
+  auto run = [&]() -> jolt_status {
+    CellDesc c{};
+    c.src = x; c.sl = (int64_t)LH * T * D; c.sh = (int64_t)T * D; c.st = D;
+    c.Lg = 1; c.H = LH; c.T = T; c.D = D; c.kind = 0; c.rope = rope_theta > 0.0f; c.f32 = 0;
+    c.seq = 0; c.l0 = 0; c.nt = 0; c.rtmax = r;
+    CellOut o{};
+    o.ut = const_cast<uint16_t*>(ut_t); o.codes = codes; o.scales = scales;
+    o.rT = r; o.rd = D; o.b = bits; o.t_pitch = T;
+    uint16_t* mp = const_cast<uint16_t*>(m);
+    JOLT_CUDA_TRY(cudaMemcpyAsync(d_cell, &c, sizeof(c), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemcpyAsync(d_out, &o, sizeof(o), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemcpyAsync(d_M, &mp, sizeof(mp), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemcpyAsync(d_rmax, &r, sizeof(int), cudaMemcpyHostToDevice, s));
+    JOLT_CUDA_TRY(cudaMemsetAsync(d_status, 0, 4 * sizeof(int), s));
+    if (cs) JOLT_TRY(launch_rope_table(T, D, (double)rope_theta, cs, s));
+    JOLT_TRY(launch_m_transpose(d_out, d_cell, d_M, d_rmax, mt_ws, LH, D, rows, 1, s));
+    JOLT_TRY(launch_ut_to_ws(d_out, ut_ws, rows, tp, 1, s));
+    StreamMaps mp4{};
+    JOLT_TRY(map_3d_box(&mp4.ut, ut_ws, 1, rows, tp, tp, 64, 64));
+    JOLT_TRY(map_3d_box(&mp4.mt, mt_ws, LH, D, rows, rows, 64, D));
+    JOLT_TRY(map_x5_box(&mp4.xk, x, 1, 1, LH, T, D, c.sl, c.sl, c.sh, c.st, 128));
+    mp4.xv = mp4.xk;
+    StreamArgs a{};
+    a.ncells = 1; a.T = T; a.H = LH; a.lhmax = LH; a.rpad_m = rows; a.G = group;
+    a.cells = d_cell; a.outs = d_out; a.cs = cs; a.seed = seed; a.status = d_status;
+    JOLT_TRY(launch_stream(true, D, mp4, a, s));
+    // the host structures above are read by copies still in flight: wait
+    JOLT_CUDA_TRY(cudaStreamSynchronize(s));
+    int dst = 0;
+    JOLT_CUDA_TRY(cudaMemcpy(&dst, d_status, sizeof(int), cudaMemcpyDeviceToHost));
+    return status_from_dev(dst);
+  };
+  st = run();
+  cudaStreamSynchronize(s);
+  dev_free(block, s);
+  return st;
 }
 
 }  // extern "C"

@@ -9,6 +9,7 @@
 // allocates nothing. The caller passes the bit widths (host) and a device
 // buffer for the result.
 #include <mutex>
+#include <vector>
 
 #include "jolt_internal.cuh"
 #include "jolt_kernels.cuh"
@@ -27,21 +28,57 @@ constexpr int NOALLOC_SLOTS = 9;
 static __device__ __align__(256) double g_eps2_scratch[NOALLOC_MAX_BLOCKS * NOALLOC_SLOTS];
 
 static std::mutex g_noalloc_mu;
-static double* g_noalloc_ptr[64] = {nullptr};
 
-// Device address of the scratch on the current device, looked up once per
-// device (with that device current) and cached.
+// One cached address per CUDA context that has called in: the array lives in
+// the library's module, and every context (the primary context of each
+// device, or any other context a caller makes current) loads its own copy.
+struct ScratchEntry {
+  void* ctx;
+  int dev;
+  double* ptr;
+};
+static std::vector<ScratchEntry> g_noalloc_cache;
+
+// The driver's cuCtxGetCurrent, reached through the runtime (the library
+// does not link the driver API directly).
+typedef int (*CtxGetCurrentFn)(void**);
+static CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    cudaGetLastError();
+  }
+  return fn;
+}
+
+// Device address of the scratch in the current context, looked up once per
+// (device, context) with that device current, and cached.
+static void* current_ctx() {
+  void* ctx = nullptr;
+  if (CtxGetCurrentFn f = ctx_get_current())
+    if (f(&ctx) != 0) ctx = nullptr;
+  return ctx;
+}
+
 static jolt_status scratch_address(double** out) {
   int dev = 0;
   JOLT_CUDA_TRY(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) { set_error("device index %d out of range", dev); return JOLT_ERR_INVALID_ARG; }
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    JOLT_CUDA_TRY(cudaGetSymbolAddress(&p, g_eps2_scratch));
-    g_noalloc_ptr[dev] = reinterpret_cast<double*>(p);
-  }
-  *out = g_noalloc_ptr[dev];
+  const void* ctx = current_ctx();
+  for (const ScratchEntry& e : g_noalloc_cache)
+    if (e.dev == dev && e.ctx == ctx) { *out = e.ptr; return JOLT_OK; }
+  void* p = nullptr;
+  JOLT_CUDA_TRY(cudaGetSymbolAddress(&p, g_eps2_scratch));
+  // the lookup makes the device's context current if none was: key the entry
+  // on the context that holds the array
+  g_noalloc_cache.push_back(ScratchEntry{current_ctx(), dev, reinterpret_cast<double*>(p)});
+  *out = reinterpret_cast<double*>(p);
   return JOLT_OK;
 }
 

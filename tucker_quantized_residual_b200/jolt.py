@@ -82,6 +82,9 @@ _SIGS = {
     "jolt_eps2_noalloc": (C.c_int, [C.POINTER(_I32), _I32, _I32, _VP, _VP]),
     "jolt_residual_encode": (C.c_int, [_VP, _I64, _I32, _I32, _I32, _U64, _VP, _VP, _VP]),
     "jolt_residual_decode": (C.c_int, [_VP, _VP, _I64, _I32, _I32, _I32, _U64, _VP, _VP]),
+    "jolt_residual_stream_encode": (C.c_int, [_VP, _I32, _I32, _I32, _VP, _I32, _VP, _I32, _I32, _U64,
+                                              C.c_float, _VP, _VP, _VP]),
+    "jolt_sketch": (C.c_int, [_VP, _U64, _VP, C.POINTER(_I32), C.POINTER(_I32), _VP]),
     "jolt_layer_groups": (C.c_int, [C.POINTER(jolt_layout), _VP, _I32, _U64, C.POINTER(C.c_double),
                                     C.POINTER(C.c_int32), C.POINTER(C.c_int32), _VP]),
     "jolt_set_allocator": (C.c_int, [_VP, _VP, _VP]),
@@ -278,9 +281,54 @@ def jolt_eps2(bits: Sequence[int], group: int, stream=None) -> List[float]:
 
 def jolt_eps2_noalloc(bits: Sequence[int], group: int, out, stream=None) -> None:
     """Same values as jolt_eps2, written to the device tensor `out` (float64,
-    len(bits) entries) without any device allocation inside the library."""
+    len(bits) entries) without any device allocation inside the library.
+
+    The library only sees a raw pointer and writes len(bits) doubles there,
+    so the tensor is checked here: a CUDA float64 tensor, contiguous, with
+    room for every bit width."""
+    import torch
+    if not isinstance(out, torch.Tensor):
+        raise TypeError("out must be a torch.Tensor")
+    if out.dtype != torch.float64:
+        raise ValueError(f"out must be float64, not {out.dtype}")
+    if not out.is_contiguous():
+        raise ValueError("out must be contiguous")
+    if out.numel() < len(bits):
+        raise ValueError(f"out holds {out.numel()} values, {len(bits)} needed")
+    if not out.is_cuda:
+        raise ValueError("out must be a CUDA tensor (the library writes it from a kernel)")
     b = (C.c_int32 * len(bits))(*bits)
     _check(load_library().jolt_eps2_noalloc(b, len(bits), group, _ptr(out), _stream(stream)))
+
+
+def jolt_residual_stream_encode(x, ut_t, m, bits: int, group: int, seed: int, rope_theta: float,
+                                codes, scales, stream=None) -> None:
+    """The compress path's residual kernel on given factors. x: bf16 [LH, T, D];
+    ut_t: bf16 [r, T]; m: bf16 [LH, r, D]; codes: uint8 [LH, T, bits*D/8];
+    scales: float32 [LH, T, D/group] (all CUDA, contiguous)."""
+    import torch
+    LH, T, D = x.shape
+    r = ut_t.shape[0]
+    for t, dt, shape in ((x, torch.bfloat16, (LH, T, D)), (ut_t, torch.bfloat16, (r, T)),
+                         (m, torch.bfloat16, (LH, r, D)), (codes, torch.uint8, (LH, T, bits * D // 8)),
+                         (scales, torch.float32, (LH, T, D // group))):
+        if not (t.is_cuda and t.dtype == dt and t.is_contiguous() and tuple(t.shape) == shape):
+            raise ValueError(f"expected a contiguous CUDA {dt} tensor of shape {shape}")
+    _check(load_library().jolt_residual_stream_encode(_ptr(x), LH, T, D, _ptr(ut_t), r, _ptr(m), bits, group,
+                                                      int(seed), float(rope_theta), _ptr(codes), _ptr(scales),
+                                                      _stream(stream)))
+
+
+def jolt_sketch(plan: int, seed: int, n_cells: int, stream=None):
+    """The randomized plan's sketch: a CUDA int16 tensor [n_cells, k, ld] of
+    bf16 bit patterns (row j of cell c = column j of that cell's Omega)."""
+    import torch
+    lib = load_library()
+    k, ld = C.c_int32(), C.c_int32()
+    _check(lib.jolt_sketch(plan, int(seed), None, C.byref(k), C.byref(ld), _stream(stream)))
+    out = torch.zeros((n_cells, k.value, ld.value), dtype=torch.int16, device="cuda")
+    _check(lib.jolt_sketch(plan, int(seed), _ptr(out), None, None, _stream(stream)))
+    return out
 
 
 def jolt_residual_encode(e, D: int, bits: int, group: int, seed: int, codes, scales, stream=None) -> None:
