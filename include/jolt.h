@@ -122,6 +122,18 @@ typedef struct {
   double budget_tol;
   int32_t max_iters;
   int32_t minimizer;             /* JOLT_MIN_ENUMERATE | JOLT_MIN_GREEDY       */
+  /* Where this plan's cache sits in a larger one that several processes
+   * compress under one budget (jolt_compress_begin): its sequence b and
+   * group g are sequence seq_base + b and group group_base + g of the whole
+   * cache. They only enter the random draws (the rotation of sequence s uses
+   * seed + s; the sketch of group g uses group g's counter words) and the
+   * identities in jolt_cell_info, so a shard draws exactly what a single
+   * process would for the same cells. Default 0. */
+  int32_t seq_base, group_base;
+  /* The compression ratio C of Eq. (5) (q_cap = 32 or 64 by C <= 4, Section
+   * 3.1). 0: this plan's dense bf16 bytes / byte_budget. A shard of a
+   * shared-budget compression passes the whole cache's ratio. */
+  double cap_ratio;
 } jolt_options;
 
 typedef struct jolt_plan_s jolt_plan_t;
@@ -171,6 +183,37 @@ JOLT_API void jolt_free_plan(jolt_plan_t* plan);
 JOLT_API jolt_status jolt_compress(jolt_plan_t* plan, const void* k, const void* v,
                           int64_t byte_budget, uint64_t seed,
                           jolt_stream_t stream, jolt_handle_t** out);
+
+/* One byte budget shared by several processes (one per GPU), each holding
+ * part of the cells (Section 3, "Solving the allocation": the allocation
+ * separates across cells once the multiplier is fixed, so only per-cell
+ * rate-distortion summaries need to travel). Protocol:
+ *   1. every rank: jolt_compress_begin on its plan (its own sequences or
+ *      layer groups, with seq_base / group_base set), which computes the
+ *      spectra and the rate-distortion table of its cells (the steps before
+ *      the allocation) and writes one summary record per cell into
+ *      summary_dev (DEVICE, n_cells * jolt_summary_bytes(plan) bytes, 16-byte
+ *      aligned, owned by the caller);
+ *   2. the caller all-gathers the records of every rank into one DEVICE
+ *      buffer (NCCL or any transport; the records are plain bytes);
+ *   3. every rank: jolt_compress_end with the gathered buffer, which runs the
+ *      same multiplier bisection over all n_total cells (deterministic, so
+ *      every rank reaches the same allocation bit for bit) and then fits and
+ *      encodes its own cells, records [first_cell, first_cell + n_cells).
+ * Every rank must pass the same byte_budget and options (grids, bits, scale
+ * group, tolerances); records carry a fingerprint of those settings and a
+ * mismatch, or a local slice that holds other cells, is reported as
+ * JOLT_ERR_INVALID_ARG by the next synchronising call on the handle.
+ * Between begin and end the plan holds the cells' spectral state: run no
+ * other jolt_compress / jolt_rd_table on that plan in between. The handle
+ * from begin is the compressed cache once end has run; before that only
+ * jolt_free_handle may be called on it. Both calls are asynchronous. */
+JOLT_API int64_t jolt_summary_bytes(const jolt_plan_t* plan);
+JOLT_API jolt_status jolt_compress_begin(jolt_plan_t* plan, const void* k, const void* v, int64_t byte_budget,
+                                         uint64_t seed, void* summary_dev, jolt_stream_t stream,
+                                         jolt_handle_t** out);
+JOLT_API jolt_status jolt_compress_end(jolt_handle_t* h, const void* all_summaries_dev, int32_t n_total,
+                                       int32_t first_cell, jolt_stream_t stream);
 
 /* Decompress into k_out / v_out (DEVICE, bf16, layout out_layout; NULL means
  * the plan's layout with dtype bf16). Section 3: "Decoding inverts the

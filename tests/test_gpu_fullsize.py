@@ -78,7 +78,10 @@ def _same_sketch(spec, C_ratio):
         Om = o.library_sketch(N, k, ld, c.b, 2 * c.g + c.kind)
         w, _ = o.randomized_token_spectrum(X, Om, 2, qc)
         nsq = float(np.sum(X * X))
-        assert abs(ns[i] - nsq) <= 1e-5 * nsq
+        # the feature Gram (and its trace) is summed by the tensor cores 256 rows
+        # at a time, then in fp32 with round-to-nearest; inside the tensor cores
+        # each row's product can lose up to one ulp toward zero
+        assert abs(ns[i] - nsq) <= 256 * 2.0 ** -23 * nsq
         rel = np.abs(np.array(st[i][:qc]) - w[:qc]) / w[0]
         worst = max(worst, float(rel.max()))
         assert rel.max() < 1e-2, (i, rel.max())

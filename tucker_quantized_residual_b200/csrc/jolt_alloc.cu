@@ -370,3 +370,72 @@ jolt_status launch_alloc(const AllocArgs& a, const AllocState& init, cudaStream_
 }
 
 }  // namespace jolt
+
+namespace jolt {
+
+// ---------------------------------------------- sharded allocation records --
+__global__ void k_write_records(const CellRD* __restrict__ cells, const double* const* __restrict__ normsq,
+                                const int4* __restrict__ ids, uint64_t fp, int ntp, int rec_bytes,
+                                uint8_t* __restrict__ out) {
+  const int c = blockIdx.x;
+  const CellRD cd = cells[c];
+  uint8_t* rec = out + (int64_t)c * rec_bytes;
+  double* tT = reinterpret_cast<double*>(rec + sizeof(RDRecordHdr));
+  double* tD = tT + ntp;
+  for (int i = threadIdx.x; i < ntp; i += blockDim.x) tT[i] = (i <= cd.nt) ? cd.tT[i] : 0.0;
+  for (int i = threadIdx.x; i <= cd.D; i += blockDim.x) tD[i] = cd.tD[i];
+  if (threadIdx.x == 0) {
+    RDRecordHdr h;
+    h.magic = RD_MAGIC;
+    h.Lg = cd.Lg; h.H = cd.H; h.T = cd.T; h.D = cd.D; h.n_rt = cd.n_rt; h.nt = cd.nt; h.ntp = ntp;
+    h.fingerprint = fp;
+    h.norm_sq = *normsq[c];
+    const int4 id = ids[c];
+    h.seq = id.x; h.group = id.y; h.kind = id.z; h.rec_bytes = rec_bytes;
+    *reinterpret_cast<RDRecordHdr*>(rec) = h;
+  }
+}
+
+jolt_status launch_write_records(const CellRD* cells, int ncells, const double* const* normsq, const int4* ids,
+                                 uint64_t fingerprint, int ntp, int rec_bytes, uint8_t* out, cudaStream_t s) {
+  if (ncells <= 0) return JOLT_OK;
+  k_write_records<<<ncells, 128, 0, s>>>(cells, normsq, ids, fingerprint, ntp, rec_bytes, out);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+__global__ void k_records_to_rd(const uint8_t* __restrict__ recs, int n_total, int rec_bytes, int ntp, int D,
+                                uint64_t fp, int n_rt_max, int first, int nlocal, const int4* __restrict__ ids,
+                                CellRD* __restrict__ out, int* status) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_total) return;
+  const uint8_t* rec = recs + (int64_t)i * rec_bytes;
+  const RDRecordHdr h = *reinterpret_cast<const RDRecordHdr*>(rec);
+  const double* tT = reinterpret_cast<const double*>(rec + sizeof(RDRecordHdr));
+  bool ok = h.magic == RD_MAGIC && h.fingerprint == fp && h.rec_bytes == rec_bytes && h.ntp == ntp && h.D == D &&
+            h.n_rt >= 1 && h.n_rt <= n_rt_max && h.nt >= 1 && h.nt < ntp && h.Lg >= 1 && h.H >= 1 && h.T >= 1;
+  if (i >= first && i < first + nlocal) {
+    const int4 id = ids[i - first];
+    ok = ok && h.seq == id.x && h.group == id.y && h.kind == id.z;
+  }
+  CellRD c;
+  c.Lg = ok ? h.Lg : 1; c.H = ok ? h.H : 1; c.T = ok ? h.T : 1; c.D = D;
+  c.n_rt = ok ? h.n_rt : 1;
+  c.nt = ok ? h.nt : 1;
+  c.tT = tT;
+  c.tD = tT + ntp;
+  out[i] = c;
+  if (!ok) atomicOr(status, DEV_ERR_MISMATCH);
+}
+
+jolt_status launch_records_to_rd(const uint8_t* recs, int n_total, int rec_bytes, int ntp, int D, uint64_t fingerprint,
+                                 int n_rt_max, int first, int nlocal, const int4* ids, CellRD* out, int* status,
+                                 cudaStream_t s) {
+  if (n_total <= 0) return JOLT_OK;
+  k_records_to_rd<<<(n_total + 127) / 128, 128, 0, s>>>(recs, n_total, rec_bytes, ntp, D, fingerprint, n_rt_max, first,
+                                                        nlocal, ids, out, status);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
+}  // namespace jolt

@@ -114,7 +114,7 @@ struct HostCell {
   int N, nmin;     // N = Lg*H*D, nmin = min(T, N)
   int nt;          // token spectrum length fed to the allocator
   int n_rt, rmax;  // usable rank-grid entries and the largest of them
-  int64_t min_bytes;
+  int64_t min_bytes, max_bytes;   // cheapest and dearest admissible option (Eq. 1)
 };
 
 struct jolt_plan_s {
@@ -195,6 +195,10 @@ struct jolt_plan_s {
   EighJob* d_jobs_rand = nullptr;
   double* eig_scr = nullptr;   unsigned int* eig_cnt = nullptr;   int eig_nmax = 0;
   double* gram_part = nullptr;  // GRAM_SPLIT partial Grams (randomized)
+  // shared-budget protocol: summary record layout and the settings' fingerprint
+  int ntp = 0, rec_bytes = 0;
+  uint64_t fingerprint = 0;
+  int4* d_ids = nullptr;        // (global sequence, global group, kind) per cell
 };
 
 struct jolt_handle_s {
@@ -210,6 +214,10 @@ struct jolt_handle_s {
   void* block = nullptr;
   void* qblock = nullptr;        // QR-Gaussian rotation: scratch + Q per sequence
   double* d_qrot = nullptr;      // [batch][D][D], NULL for the Hadamard rotation
+  int64_t budget = 0;
+  int phase = 0;                 // 1: spectra done (begin), 2: compressed (end)
+  const void* k_in = nullptr;    // inputs of a begun two-phase compression
+  const void* v_in = nullptr;
 };
 
 static jolt_status status_from_dev(int st) {
@@ -219,6 +227,11 @@ static jolt_status status_from_dev(int st) {
   if (st & DEV_ERR_TIMEOUT) { set_error("a bounded device wait expired"); return JOLT_ERR_TIMEOUT; }
   if (st & DEV_ERR_EIG_NOCONV) { set_error("eigensolver did not converge"); return JOLT_ERR_CUDA; }
   if (st & DEV_ERR_CHOL) { set_error("Cholesky factorization failed (rank-deficient sketch)"); return JOLT_ERR_CUDA; }
+  if (st & DEV_ERR_MISMATCH) {
+    set_error("gathered rate-distortion records do not match this plan (other settings, sizes, or another cell "
+              "in this plan's slice)");
+    return JOLT_ERR_INVALID_ARG;
+  }
   set_error("device status 0x%x", st);
   return JOLT_ERR_CUDA;
 }
@@ -301,6 +314,8 @@ static jolt_status validate(const jolt_layout* L, const jolt_options* o) {
   int G = o->scale_group ? o->scale_group : L->head_dim;
   if (!(G == 32 || G == 64 || G == 128) || L->head_dim % G) { set_error("scale_group must be 32/64/128 and divide D"); return JOLT_ERR_INVALID_ARG; }
   if (o->budget_tol < 0 || o->budget_tol >= 1 || o->max_iters < 1) { set_error("bad tolerance/max_iters"); return JOLT_ERR_INVALID_ARG; }
+  if (o->seq_base < 0 || o->group_base < 0) { set_error("seq_base and group_base must be >= 0"); return JOLT_ERR_INVALID_ARG; }
+  if (!(o->cap_ratio >= 0.0)) { set_error("cap_ratio must be >= 0"); return JOLT_ERR_INVALID_ARG; }
   if (o->minimizer != JOLT_MIN_ENUMERATE && o->minimizer != JOLT_MIN_GREEDY) { set_error("minimizer must be JOLT_MIN_ENUMERATE or JOLT_MIN_GREEDY"); return JOLT_ERR_INVALID_ARG; }
   auto chk = [](int n, const int32_t* g) {
     if (n < 0 || (n > 0 && !g)) return false;
@@ -338,7 +353,7 @@ jolt_status jolt_plan(const jolt_layout* L, int64_t byte_budget, const jolt_opti
   p->G = opt->scale_group ? opt->scale_group : p->D;
   for (int b : p->bits) p->rowbytes.push_back(residual_row_bytes(b, p->D, p->G));
   const double dense = 2.0 * 2.0 * (double)L->batch * L->n_layers * L->n_heads * (double)L->seq_len * p->D;
-  p->C = dense / (double)byte_budget;
+  p->C = opt->cap_ratio > 0.0 ? opt->cap_ratio : dense / (double)byte_budget;
   p->qcap = qcap_eq5(p->T, p->C);
   const bool rnd = opt->mode == JOLT_RANDOMIZED;
   // rd grid: default every integer 1..D
@@ -391,6 +406,14 @@ jolt_status jolt_plan(const jolt_layout* L, int64_t byte_budget, const jolt_opti
       return JOLT_ERR_INVALID_ARG;
     }
     c.min_bytes = best;
+    {
+      // Eq. (1) grows with each of r_T, r_d and b: the dearest admissible
+      // option takes the largest of each (r_d capped at L_g*H*r_T)
+      const int rt = c.rmax;
+      int rd = 0;
+      for (int x : p->rd_grid) if (x <= LH * rt) rd = x;
+      c.max_bytes = 2 * (LH * rt * rd + (int64_t)p->T * rt + (int64_t)p->D * rd) + p->rowbytes.back() * LH * p->T;
+    }
     p->nmin_max = std::max(p->nmin_max, c.nmin);
     p->rmax_all = std::max(p->rmax_all, c.rmax);
     p->lh_max = std::max(p->lh_max, c.Lg * p->H);
@@ -455,6 +478,27 @@ jolt_status jolt_plan(const jolt_layout* L, int64_t byte_budget, const jolt_opti
     }
     cudaGetLastError();
   }
+  // settings every process of a shared-budget allocation must agree on
+  {
+    uint64_t h = 1469598103934665603ull;
+    auto mix = [&](uint64_t x) { for (int i = 0; i < 8; ++i) { h ^= (x >> (8 * i)) & 0xFF; h *= 1099511628211ull; } };
+    mix((uint64_t)p->D); mix((uint64_t)p->G); mix((uint64_t)opt->mode); mix((uint64_t)opt->minimizer);
+    mix((uint64_t)opt->max_iters);
+    uint64_t tb;
+    memcpy(&tb, &opt->budget_tol, 8);
+    mix(tb);
+    mix(p->bits.size());
+    for (int b : p->bits) mix((uint64_t)b);
+    mix(p->rd_grid.size());
+    for (int r : p->rd_grid) mix((uint64_t)r);
+    // an explicit token-rank grid must match; the default one is the
+    // integers from 1 and agrees on every prefix
+    mix(opt->rt_grid ? (uint64_t)opt->n_rt : 0xFFFFFFFFull);
+    if (opt->rt_grid) for (int i = 0; i < opt->n_rt; ++i) mix((uint64_t)opt->rt_grid[i]);
+    p->fingerprint = h;
+  }
+  p->ntp = p->nt_max + 1;
+  p->rec_bytes = (int)((sizeof(RDRecordHdr) + 8 * (size_t)p->ntp + 8 * (size_t)(p->D + 1) + 255) / 256 * 256);
   jolt_status st = plan_build_workspace(p);
   if (st != JOLT_OK) { jolt_free_plan(p); return st; }
   *out = p;
@@ -504,6 +548,7 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
     p->d_api = A.take<int>((size_t)nc * p->achunk);
     p->d_cur = A.take<int>(nc);
     p->d_keep = A.take<int>(nc);
+    p->d_ids = A.take<int4>(nc);
     p->Ut_ws = A.take<uint16_t>((size_t)nc * p->rows_u * p->tp);
     p->Mt_ws = A.take<uint16_t>((size_t)nc * p->lh_max * D * p->rpad_m);
     p->eig_nmax = std::max(p->opt.mode == JOLT_RANDOMIZED ? p->k : p->nmin_max, D);
@@ -605,6 +650,13 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
       jf[i] = EighJob{D, 1, CY[i], wY[i], VtY[i], ZY[i], workY[i], FY[i]};
     }
     JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_rd_cells, rdc.data(), nc * sizeof(CellRD), cudaMemcpyHostToDevice, s));
+    {
+      std::vector<int4> ids(nc);
+      for (int i = 0; i < nc; ++i)
+        ids[i] = make_int4(p->hc[i].seq + p->opt.seq_base, p->hc[i].group + p->opt.group_base, p->hc[i].kind, 0);
+      JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_ids, ids.data(), nc * sizeof(int4), cudaMemcpyHostToDevice, s));
+      JOLT_CUDA_TRY(cudaStreamSynchronize(s));
+    }
     JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_nt, ntv.data(), nc * sizeof(int), cudaMemcpyHostToDevice, s));
     JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_rmax, rmaxv.data(), nc * sizeof(int), cudaMemcpyHostToDevice, s));
     JOLT_CUDA_TRY(cudaMemcpyAsync(p->d_nlh, nlhv.data(), nc * sizeof(int), cudaMemcpyHostToDevice, s));
@@ -631,7 +683,7 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
       for (int i = 0; i < nc; ++i) {
         const HostCell& c = p->hc[i];
         l0v[i] = c.l0; bv[i] = c.seq; lgv[i] = c.Lg; kindv[i] = c.kind; ncv[i] = c.N;
-        cisv[i] = 2 * c.group + c.kind;
+        cisv[i] = 2 * (c.group + p->opt.group_base) + c.kind;
         jr[i] = EighJob{k, 1, p->MB + i * kk, p->ew + (size_t)i * k, p->eVt + i * kk, p->eZ + i * kk,
                         p->ework + (size_t)i * 3 * k, p->eF + (size_t)i * p->rmax_all * 5 * k};
         jr[nc + i] = EighJob{D, 0, Cd[i], wD[i], nullptr, nullptr, workD[i], nullptr};
@@ -953,16 +1005,14 @@ void jolt_free_plan(jolt_plan_t* p) {
   delete p;
 }
 
-jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t byte_budget,
-                          uint64_t seed, jolt_stream_t stream_, jolt_handle_t** out) {
-  cudaStream_t s = (cudaStream_t)stream_;
-  if (!p || !k || !v || !out) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
-  *out = nullptr;
-  JOLT_TRY(check_tma_inputs(p, k, v));
-  const int64_t B = byte_budget > 0 ? byte_budget : p->budget;
-  int64_t minsum = 0, extra = 0;
+// Phase 1 of a compression: a handle for this plan's cells, then the spectra
+// and rate-distortion tables (the steps before the allocation).
+static jolt_status compress_begin(jolt_plan_s* p, const void* k, const void* v, int64_t B, uint64_t seed,
+                                  cudaStream_t s, jolt_handle_s** out) {
+  int64_t minsum = 0, maxsum = 0, extra = 0;
   for (auto& c : p->hc) {
     minsum += c.min_bytes;
+    maxsum += c.max_bytes;
     extra += 5 * 256 + (int64_t)c.rmax * 16;
   }
   if (B < minsum) { set_error("budget %lld below the cheapest allocation %lld", (long long)B, (long long)minsum); return JOLT_ERR_BUDGET_INFEASIBLE; }
@@ -970,8 +1020,12 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   auto* h = new jolt_handle_s();
   h->plan = p;
   h->stream = s;
-  h->seed = seed;
-  h->capacity = B + extra + 4096;
+  // sequence b of this plan is sequence seq_base + b of the whole cache: its
+  // rotation (and sketch) are drawn from seed + seq_base + b
+  h->seed = seed + (uint64_t)p->opt.seq_base;
+  h->budget = B;
+  // the cells' bytes never exceed the budget, nor their dearest options
+  h->capacity = std::min(B, maxsum) + extra + 4096;
   Arena A;
   for (int pass = 0; pass < 2; ++pass) {
     A.used = 0;
@@ -994,42 +1048,102 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
     h->qblock = dev_alloc(2 * qn * sizeof(double), s);
     if (!h->qblock) { set_error("rotation allocation failed"); return fail(JOLT_ERR_OOM); }
     h->d_qrot = reinterpret_cast<double*>(h->qblock) + qn;
-    if ((st = launch_qr_rotation(p->D, p->lay.batch, seed, reinterpret_cast<double*>(h->qblock), h->d_qrot, s)) !=
+    if ((st = launch_qr_rotation(p->D, p->lay.batch, h->seed, reinterpret_cast<double*>(h->qblock), h->d_qrot, s)) !=
         JOLT_OK)
       return fail(st);
   }
   if ((st = upload_cells(p, k, v, s)) != JOLT_OK) return fail(st);
-  if ((st = run_spectra(p, k, v, seed, h->d_status, s)) != JOLT_OK) return fail(st);
+  if ((st = run_spectra(p, k, v, h->seed, h->d_status, s)) != JOLT_OK) return fail(st);
+  h->phase = 1;
+  *out = h;
+  return JOLT_OK;
+}
+
+// Phase 2: the allocation (over this plan's cells, or over gathered records
+// of every process sharing the budget), then fit and residual of this plan's
+// cells.
+static jolt_status compress_end(jolt_handle_s* h, const void* k, const void* v, const uint8_t* recs, int n_total,
+                                int first, cudaStream_t s) {
+  jolt_plan_s* p = h->plan;
+  const int nc = p->ncells;
+  const uint64_t seed = h->seed;
+  jolt_status st;
   {
     ProfScope ps(JOLT_STAGE_ALLOC, s);
-    if ((st = run_allocation(p, B, p->d_eps2, h->d_state, h->d_choice, h->d_status, s)) != JOLT_OK) return fail(st);
+    if (!recs) {
+      JOLT_TRY(run_allocation(p, h->budget, p->d_eps2, h->d_state, h->d_choice, h->d_status, s));
+    } else {
+      // every cell's record: CellRD views, then the same bisection as above
+      Arena A;
+      CellRD* rd = nullptr; double* pv = nullptr; int* pi = nullptr; int* cur = nullptr; int* keep = nullptr;
+      Choice* ch = nullptr; AllocState* ast = nullptr;
+      void* blk = nullptr;
+      for (int pass = 0; pass < 2; ++pass) {
+        A.used = 0;
+        rd = A.take<CellRD>(n_total);
+        pv = A.take<double>((size_t)n_total * p->achunk);
+        pi = A.take<int>((size_t)n_total * p->achunk);
+        cur = A.take<int>(n_total);
+        keep = A.take<int>(n_total);
+        ch = A.take<Choice>(n_total);
+        ast = A.take<AllocState>(1);
+        if (pass == 0) {
+          blk = dev_alloc(A.used + 256, s);
+          if (!blk) { set_error("allocation scratch for %d cells failed", n_total); return JOLT_ERR_OOM; }
+          A.base = reinterpret_cast<uint8_t*>(blk);
+        }
+      }
+      auto run = [&]() -> jolt_status {
+        JOLT_TRY(launch_records_to_rd(recs, n_total, p->rec_bytes, p->ntp, p->D, p->fingerprint,
+                                      (int)p->rt_grid.size(), first, nc, p->d_ids, rd, h->d_status, s));
+        AllocState st0{};
+        st0.lo = 1e-30; st0.hi = 1.0; st0.lam = st0.lo;
+        st0.tol = p->opt.budget_tol;
+        st0.budget = h->budget;
+        st0.max_iters = p->opt.max_iters;
+        st0.phase = 0;
+        AllocArgs a{};
+        a.greedy = p->opt.minimizer == JOLT_MIN_GREEDY;
+        a.cells = rd; a.ncells = n_total;
+        a.rt_grid = p->d_rt; a.rd_grid = p->d_rd; a.n_rd = (int)p->rd_grid.size();
+        a.bits = p->d_bits; a.eps2 = p->d_eps2; a.rowbytes = p->d_rowbytes; a.n_bits = (int)p->bits.size();
+        a.nchunk = p->achunk; a.pv = pv; a.pi = pi; a.cur = cur; a.keep = keep;
+        a.st = ast; a.out = ch; a.status = h->d_status;
+        JOLT_TRY(launch_alloc(a, st0, s));
+        JOLT_CUDA_TRY(cudaMemcpyAsync(h->d_choice, ch + first, nc * sizeof(Choice), cudaMemcpyDeviceToDevice, s));
+        JOLT_CUDA_TRY(cudaMemcpyAsync(h->d_state, ast, sizeof(AllocState), cudaMemcpyDeviceToDevice, s));
+        return JOLT_OK;
+      };
+      st = run();
+      dev_free(blk, s);
+      if (st != JOLT_OK) return st;
+    }
   }
   ProfScope ps_fit(JOLT_STAGE_FIT, s);
-  if ((st = launch_payload_layout(p->d_cells, h->d_choice, nc, p->G, h->payload, h->capacity, h->d_out,
-                                  h->d_status, s)) != JOLT_OK) return fail(st);
+  JOLT_TRY(launch_payload_layout(p->d_cells, h->d_choice, nc, p->G, h->payload, h->capacity, h->d_out, h->d_status, s));
   FitArgs fa{};
   fa.cells = p->d_cells; fa.cs = p->d_cs; fa.out = h->d_out; fa.ncells = nc; fa.D = p->D;
   fa.VtT = p->d_VtT; fa.wT = p->d_wT; fa.Uf = p->d_Uf; fa.Y = p->d_Y; fa.rmax_of = p->d_rmax;
   fa.VtY = p->d_VtY; fa.M = p->d_M;
   if (p->opt.mode == JOLT_EXACT) {
-    if ((st = launch_copy_rt(h->d_out, p->d_rT_used, nc, s)) != JOLT_OK) return fail(st);
+    JOLT_TRY(launch_copy_rt(h->d_out, p->d_rT_used, nc, s));
     {
       ProfScope pe(JOLT_STAGE_EIG, s);
-      if ((st = launch_eigvecs_n(p->d_jobs_spec, nc, p->rmax_all, p->nmin_max, p->d_rT_used, s)) != JOLT_OK) return fail(st);
+      JOLT_TRY(launch_eigvecs_n(p->d_jobs_spec, nc, p->rmax_all, p->nmin_max, p->d_rT_used, s));
     }
-    if ((st = launch_ut_exact(fa, p->T, p->rmax_all, s)) != JOLT_OK) return fail(st);
-    if ((st = launch_project_y(fa, p->T, p->rmax_all, p->lh_max, s)) != JOLT_OK) return fail(st);
+    JOLT_TRY(launch_ut_exact(fa, p->T, p->rmax_all, s));
+    JOLT_TRY(launch_project_y(fa, p->T, p->rmax_all, p->lh_max, s));
   } else {
-    if ((st = run_random_fit(p, k, v, h->d_out, h->d_status, s)) != JOLT_OK) return fail(st);
+    JOLT_TRY(run_random_fit(p, k, v, h->d_out, h->d_status, s));
   }
   // feature Gram of Y (rows r < r_T), then its eigenvectors
-  if ((st = launch_copy_rt(h->d_out, p->d_rT_used, nc, s)) != JOLT_OK) return fail(st);
-  if ((st = launch_fgram_rows(p->d_Y, p->d_rT_used, p->d_rmax, p->d_nlh, nc, p->D, p->fchunk, p->d_fpart, s)) != JOLT_OK) return fail(st);
-  if ((st = launch_sum_chunks(p->d_fpart, p->fchunk, p->D * p->D + 1, nc, p->d_CY, nullptr, s)) != JOLT_OK) return fail(st);
-  if ((st = launch_tridiag(p->d_jobs_fit, nc, p->D, s)) != JOLT_OK) return fail(st);
-  if ((st = launch_bisect(p->d_jobs_fit, nc, p->D, s)) != JOLT_OK) return fail(st);
-  if ((st = launch_eigvecs_n(p->d_jobs_fit, nc, p->D, p->D, p->d_Dn, s)) != JOLT_OK) return fail(st);
-  if ((st = launch_core(fa, p->rmax_all, p->lh_max, s)) != JOLT_OK) return fail(st);
+  JOLT_TRY(launch_copy_rt(h->d_out, p->d_rT_used, nc, s));
+  JOLT_TRY(launch_fgram_rows(p->d_Y, p->d_rT_used, p->d_rmax, p->d_nlh, nc, p->D, p->fchunk, p->d_fpart, s));
+  JOLT_TRY(launch_sum_chunks(p->d_fpart, p->fchunk, p->D * p->D + 1, nc, p->d_CY, nullptr, s));
+  JOLT_TRY(launch_tridiag(p->d_jobs_fit, nc, p->D, s));
+  JOLT_TRY(launch_bisect(p->d_jobs_fit, nc, p->D, s));
+  JOLT_TRY(launch_eigvecs_n(p->d_jobs_fit, nc, p->D, p->D, p->d_Dn, s));
+  JOLT_TRY(launch_core(fa, p->rmax_all, p->lh_max, s));
   ResidArgs ra{};
   ra.cells = p->d_cells; ra.cs = p->d_cs; ra.out = h->d_out; ra.M = p->d_M; ra.rmax_of = p->d_rmax;
   ra.G = p->G; ra.seed = seed; ra.qrot = h->d_qrot;
@@ -1037,18 +1151,68 @@ jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t 
   ProfScope ps_res(JOLT_STAGE_RESIDUAL, s);
   // the tensor-core stream kernel implements the Hadamard rotation only
   if (p->tc_in && !h->d_qrot && reinterpret_cast<uintptr_t>(k) % 16 == 0 && reinterpret_cast<uintptr_t>(v) % 16 == 0) {
-    if ((st = run_stream(p, h, k, v, nullptr, nullptr, nullptr, s)) != JOLT_OK) return fail(st);
+    JOLT_TRY(run_stream(p, h, k, v, nullptr, nullptr, nullptr, s));
   } else {
-    if ((st = launch_residual_simt(ra, nc, p->D, p->T, p->lh_max, s)) != JOLT_OK) return fail(st);
+    JOLT_TRY(launch_residual_simt(ra, nc, p->D, p->T, p->lh_max, s));
   }
+  h->phase = 2;
+  return JOLT_OK;
+}
+
+jolt_status jolt_compress(jolt_plan_t* p, const void* k, const void* v, int64_t byte_budget,
+                          uint64_t seed, jolt_stream_t stream_, jolt_handle_t** out) {
+  cudaStream_t s = (cudaStream_t)stream_;
+  if (!p || !k || !v || !out) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
+  *out = nullptr;
+  JOLT_TRY(check_tma_inputs(p, k, v));
+  jolt_handle_s* h = nullptr;
+  JOLT_TRY(compress_begin(p, k, v, byte_budget > 0 ? byte_budget : p->budget, seed, s, &h));
+  jolt_status st = compress_end(h, k, v, nullptr, p->ncells, 0, s);
+  if (st != JOLT_OK) { jolt_free_handle(h); return st; }
   *out = h;
   return JOLT_OK;
+}
+
+int64_t jolt_summary_bytes(const jolt_plan_t* p) { return p ? (int64_t)p->rec_bytes : 0; }
+
+jolt_status jolt_compress_begin(jolt_plan_t* p, const void* k, const void* v, int64_t byte_budget, uint64_t seed,
+                                void* summary_dev, jolt_stream_t stream_, jolt_handle_t** out) {
+  cudaStream_t s = (cudaStream_t)stream_;
+  if (!p || !k || !v || !out || !summary_dev) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
+  *out = nullptr;
+  if (reinterpret_cast<uintptr_t>(summary_dev) % 16) { set_error("summary_dev must be 16-byte aligned"); return JOLT_ERR_INVALID_ARG; }
+  JOLT_TRY(check_tma_inputs(p, k, v));
+  jolt_handle_s* h = nullptr;
+  JOLT_TRY(compress_begin(p, k, v, byte_budget > 0 ? byte_budget : p->budget, seed, s, &h));
+  h->k_in = k;
+  h->v_in = v;
+  jolt_status st = launch_write_records(p->d_rd_cells, p->ncells, p->d_nsq, p->d_ids, p->fingerprint, p->ntp,
+                                        p->rec_bytes, reinterpret_cast<uint8_t*>(summary_dev), s);
+  if (st != JOLT_OK) { jolt_free_handle(h); return st; }
+  *out = h;
+  return JOLT_OK;
+}
+
+jolt_status jolt_compress_end(jolt_handle_t* h, const void* all_dev, int32_t n_total, int32_t first_cell,
+                              jolt_stream_t stream_) {
+  cudaStream_t s = (cudaStream_t)stream_;
+  if (!h || !all_dev) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
+  if (h->phase != 1) { set_error("jolt_compress_end needs a handle from jolt_compress_begin that has not ended"); return JOLT_ERR_INVALID_ARG; }
+  const int nc = h->plan->ncells;
+  if (n_total < nc || first_cell < 0 || first_cell > n_total - nc) {
+    set_error("this plan's %d cells must lie inside the %d gathered records (first_cell %d)", nc, n_total, first_cell);
+    return JOLT_ERR_INVALID_ARG;
+  }
+  if (reinterpret_cast<uintptr_t>(all_dev) % 16) { set_error("all_summaries_dev must be 16-byte aligned"); return JOLT_ERR_INVALID_ARG; }
+  h->stream = s;
+  return compress_end(h, h->k_in, h->v_in, reinterpret_cast<const uint8_t*>(all_dev), n_total, first_cell, s);
 }
 
 jolt_status jolt_decompress(const jolt_handle_t* h, void* k_out, void* v_out, const jolt_layout* ol,
                             jolt_stream_t stream_) {
   cudaStream_t s = (cudaStream_t)stream_;
   if (!h || !k_out || !v_out) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
+  if (h->phase != 2) { set_error("the handle's compression has not ended (jolt_compress_end)"); return JOLT_ERR_INVALID_ARG; }
   jolt_plan_s* p = h->plan;
   const jolt_layout& L = ol ? *ol : p->lay;
   if (L.batch != p->lay.batch || L.n_layers != p->lay.n_layers || L.n_heads != p->H || L.seq_len != p->T ||
@@ -1072,6 +1236,7 @@ jolt_status jolt_decompress(const jolt_handle_t* h, void* k_out, void* v_out, co
 }
 
 static jolt_status handle_sync(const jolt_handle_t* h) {
+  if (h->phase != 2) { set_error("the handle's compression has not ended (jolt_compress_end)"); return JOLT_ERR_INVALID_ARG; }
   JOLT_CUDA_TRY(cudaStreamSynchronize(h->stream));
   int st = 0;
   JOLT_CUDA_TRY(cudaMemcpy(&st, h->d_status, sizeof(int), cudaMemcpyDeviceToHost));
@@ -1104,7 +1269,8 @@ jolt_status jolt_handle_info(const jolt_handle_t* h, jolt_cell_info* cells, int3
       const HostCell& c = p->hc[i];
       double nsq = 0.0;
       JOLT_CUDA_TRY(cudaMemcpy(&nsq, p->h_nsq[i], sizeof(double), cudaMemcpyDeviceToHost));
-      cells[i] = jolt_cell_info{c.seq, c.group, c.kind, ch[i].rT, ch[i].rd, ch[i].b, ch[i].bytes, ch[i].err, nsq};
+      cells[i] = jolt_cell_info{c.seq + p->opt.seq_base, c.group + p->opt.group_base, c.kind, ch[i].rT, ch[i].rd,
+                                ch[i].b, ch[i].bytes, ch[i].err, nsq};
     }
   }
   if (lambda) *lambda = st.lam_final;
@@ -1140,7 +1306,7 @@ jolt_status jolt_rd_table(jolt_plan_t* p, const void* k, const void* v, double* 
   JOLT_TRY(check_tma_inputs(p, k, v));
   JOLT_CUDA_TRY(cudaMemsetAsync(p->d_status, 0, sizeof(int), s));
   JOLT_TRY(upload_cells(p, k, v, s));
-  JOLT_TRY(run_spectra(p, k, v, 0, p->d_status, s));
+  JOLT_TRY(run_spectra(p, k, v, (uint64_t)p->opt.seq_base, p->d_status, s));
   JOLT_CUDA_TRY(cudaStreamSynchronize(s));
   int st = 0;
   JOLT_CUDA_TRY(cudaMemcpy(&st, p->d_status, sizeof(int), cudaMemcpyDeviceToHost));
@@ -1242,7 +1408,8 @@ jolt_status jolt_sketch(jolt_plan_t* p, uint64_t seed, uint16_t* omega_t, int32_
   if (ld_out) *ld_out = p->Ncmax;
   if (!omega_t) return JOLT_OK;
   if (reinterpret_cast<uintptr_t>(omega_t) % 8) { set_error("omega_t must be 8-byte aligned"); return JOLT_ERR_INVALID_ARG; }
-  return launch_omega(omega_t, p->ncells, p->k, p->Ncmax, p->d_Nc, p->d_cb, p->d_cis, seed, (cudaStream_t)stream_);
+  return launch_omega(omega_t, p->ncells, p->k, p->Ncmax, p->d_Nc, p->d_cb, p->d_cis, seed + (uint64_t)p->opt.seq_base,
+                      (cudaStream_t)stream_);
 }
 
 jolt_status jolt_residual_stream_encode(const void* x, int32_t LH, int32_t T, int32_t D, const uint16_t* ut_t,

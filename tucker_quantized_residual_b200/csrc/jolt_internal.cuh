@@ -50,6 +50,7 @@ enum : int {
   DEV_ERR_TIMEOUT = 4,
   DEV_ERR_NONFINITE = 8,
   DEV_ERR_INFEASIBLE = 16,
+  DEV_ERR_MISMATCH = 32,   // gathered rate-distortion records do not fit this plan
 };
 
 // ------------------------------------------------------------- profiling ---

@@ -88,6 +88,32 @@ struct AllocArgs {
 };
 
 jolt_status launch_alloc(const AllocArgs& a, const AllocState& init, cudaStream_t s);
+
+// One cell's rate-distortion summary as exchanged between processes that
+// share one byte budget: this 64-byte header, then t_T[ntp] and t_D[D + 1]
+// (doubles), the record padded to rec_bytes. The header carries the cell's
+// shape and grid length, its global (sequence, group, kind), and a
+// fingerprint of the allocation settings (grids, bits, scale group,
+// tolerance), which every record of one allocation must share.
+struct RDRecordHdr {
+  uint32_t magic;
+  int32_t Lg, H, T, D, n_rt, nt, ntp;
+  uint64_t fingerprint;
+  double norm_sq;
+  int32_t seq, group, kind, rec_bytes;
+};
+static_assert(sizeof(RDRecordHdr) == 64, "record header is 64 bytes");
+constexpr uint32_t RD_MAGIC = 0x3144524Au;
+jolt_status launch_write_records(const CellRD* cells, int ncells, const double* const* normsq, const int4* ids,
+                                 uint64_t fingerprint, int ntp, int rec_bytes, uint8_t* out, cudaStream_t s);
+// CellRD views of n_total gathered records (pointers into the record
+// buffer, laid out by this plan's ntp and D, never by a record's own header);
+// a record whose header disagrees with this plan (magic, fingerprint, sizes,
+// a grid longer than this plan's, or, for the local slice, another cell's
+// identity) raises DEV_ERR_MISMATCH and is read as a one-option cell.
+jolt_status launch_records_to_rd(const uint8_t* recs, int n_total, int rec_bytes, int ntp, int D, uint64_t fingerprint,
+                                 int n_rt_max, int first, int nlocal, const int4* ids, CellRD* out, int* status,
+                                 cudaStream_t s);
 jolt_status launch_rd_tables(const CellRD* cells, int ncells, const double* const* wT,
                              const double* const* wD, const double* normsq,
                              double* const* tT, double* const* tD, const int* nt_used,

@@ -6,7 +6,8 @@
 // X~ = U_T^ M^_lh. Keys get RoPE re-applied after decoding.
 //
 // This file holds the row-per-thread (SIMT) forms: the backbone product is
-// accumulated in fp32 registers, the transform runs inside the thread. It
+// summed in fp64 registers (so the residual is the one of the fp64
+// reconstruction), the transform runs inside the thread. It
 // also holds the page's own rotation, R = the Q of a seeded Gaussian's QR
 // factorization, as an option: r = Q e and e = Q^T r are dense row products
 // summed in fp64 and rounded once to fp32.
@@ -85,17 +86,22 @@ struct UnpackOp {
   __device__ __forceinline__ void run() { unpack_dequant_row<D, G, B>(codes, scales, v); }
 };
 
-// X~ row t of (cell, lh) accumulated in fp32: acc[d] = sum_r U_T^[t][r] M^[r][d]
-template <int D>
-__device__ __forceinline__ void backbone_rows(const ResidArgs& a, int cell, const CellOut& o, int lh,
-                                              int t0, float* acc, float (*ms)[D], float (*us)[128]) {
+// Columns [c0, c0 + W) of X~ row t of (cell, lh), summed in fp64:
+// acc[j] = sum_r U_T^[t][r] M^[r][c0 + j]. Each product of two bf16 values is
+// exact in fp64 and the sums keep 53 bits, so the result is the fp64 sum the
+// reading of the residual (X - U_T^ M^ formed before any rounding to fp32)
+// calls for. The U_T^ and M^ tiles are staged in shared memory 32 ranks at a
+// time; every thread of the block takes part in the staging.
+template <int D, int W>
+__device__ __forceinline__ void backbone_cols(const ResidArgs& a, int cell, const CellOut& o, int lh, int t0,
+                                              int c0, double* acc, float (*ms)[D], float (*us)[128]) {
   const int rmax = a.rmax_of[cell];
   const uint16_t* M = a.M[cell] + (int64_t)lh * rmax * D;
 #pragma unroll
-  for (int d = 0; d < D; ++d) acc[d] = 0.0f;
+  for (int j = 0; j < W; ++j) acc[j] = 0.0;
   for (int r0 = 0; r0 < o.rT; r0 += 32) {
-    for (int e = threadIdx.x; e < 32 * D; e += blockDim.x) {
-      int rr = e / D, d = e % D;
+    for (int e = threadIdx.x; e < 32 * W; e += blockDim.x) {
+      int rr = e / W, d = c0 + e % W;
       ms[rr][d] = (r0 + rr < o.rT) ? bf16_bits_to_f32(M[(int64_t)(r0 + rr) * D + d]) : 0.0f;
     }
     for (int e = threadIdx.x; e < 32 * 128; e += blockDim.x) {
@@ -105,11 +111,34 @@ __device__ __forceinline__ void backbone_rows(const ResidArgs& a, int cell, cons
     }
     __syncthreads();
     for (int rr = 0; rr < 32; ++rr) {
-      const float u = us[rr][threadIdx.x];
+      const double u = (double)us[rr][threadIdx.x];
 #pragma unroll
-      for (int d = 0; d < D; ++d) acc[d] = fmaf(u, ms[rr][d], acc[d]);
+      for (int j = 0; j < W; ++j) acc[j] = fma(u, (double)ms[rr][c0 + j], acc[j]);
     }
     __syncthreads();
+  }
+}
+
+// Row t's backbone, four column quarters in turn (32 fp64 partial sums live
+// at a time). Encoding (ENC): out = fl32(x - X~) from the fp64 sum, one
+// rounding; decoding: out = fl32(X~).
+template <int D, bool ENC>
+__device__ __forceinline__ void backbone_row(const ResidArgs& a, const CellDesc& c, int cell, const CellOut& o,
+                                             int lh, int t0, float* out, float (*ms)[D], float (*us)[128]) {
+  constexpr int W = D / 4;
+  const int t = t0 + threadIdx.x;
+  const int l = lh / c.H, h = lh % c.H;
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq) {
+    double acc[W];
+    backbone_cols<D, W>(a, cell, o, lh, t0, qq * W, acc, ms, us);
+    if (t < c.T) {
+#pragma unroll
+      for (int j = 0; j < W; ++j) {
+        if constexpr (ENC) out[qq * W + j] = (float)((double)x_elem(c, a.cs, l, h, t, qq * W + j) - acc[j]);
+        else out[qq * W + j] = (float)acc[j];
+      }
+    }
   }
 }
 
@@ -126,12 +155,9 @@ __global__ void __launch_bounds__(128) k_residual_simt(ResidArgs a) {
   for (int d = threadIdx.x; d < D; d += blockDim.x) sg[d] = hadamard_sign(a.seed + c.seq, d);
   __syncthreads();
   float acc[D];
-  backbone_rows<D>(a, cell, o, lh, t0, acc, ms, us);
+  backbone_row<D, true>(a, c, cell, o, lh, t0, acc, ms, us);   // E = X - X~
   const int t = t0 + threadIdx.x;
   if (t >= c.T) return;
-  const int l = lh / c.H, h = lh % c.H;
-#pragma unroll
-  for (int d = 0; d < D; ++d) acc[d] = __fsub_rn(x_elem(c, a.cs, l, h, t, d), acc[d]);
   if constexpr (QR) qr_rotate_row<D>(acc, a.qrot + (int64_t)c.seq * D * D, rowbuf + threadIdx.x * (D + 1));
   else rotate_row<D>(acc, sg);
   const int64_t row = (int64_t)lh * c.T + t;
@@ -152,7 +178,7 @@ __global__ void __launch_bounds__(128) k_decompress_simt(ResidArgs a) {
   for (int d = threadIdx.x; d < D; d += blockDim.x) sg[d] = hadamard_sign(a.seed + c.seq, d);
   __syncthreads();
   float acc[D];
-  backbone_rows<D>(a, cell, o, lh, t0, acc, ms, us);
+  backbone_row<D, false>(a, c, cell, o, lh, t0, acc, ms, us);
   const int t = t0 + threadIdx.x;
   if (t >= c.T) return;
   const int l = lh / c.H, h = lh % c.H;

@@ -31,6 +31,9 @@ namespace jolt {
 namespace umma {
 
 enum Mode : int { XW = 0, XTY = 1, GRAM = 2, WP = 3, FG = 4 };
+// FG: k-steps (64 rows each) the tensor cores accumulate before the epilogue
+// adds the partial into its fp32 sums
+constexpr int FG_PROMOTE = 4;
 
 constexpr int BM = 128;          // rows of an output tile (TMEM lanes)
 constexpr int BK = 64;           // K per pipeline stage (128 bytes of bf16)
@@ -371,10 +374,18 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm(const __grid_constant_
         int kb0, kb1;
         k_range(p, cell, m0, kb0, kb1);
         if (kb0 >= kb1) continue;
-        if (!mbar_wait(tempty_bar(acc), aph[acc] ^ 1, abort_flag, p.status)) break;
-        fence_after();
-        const uint32_t dcol = tmem + (uint32_t)(acc * p.BN);
+        // FG sums squares: its tile is cut into sub-tiles of FG_PROMOTE
+        // k-steps, each accumulated afresh and added up by the epilogue in
+        // fp32 with round-to-nearest (see the epilogue)
+        const int sub = (p.mode == FG) ? FG_PROMOTE : (kb1 - kb0);
+        uint32_t dcol = 0;
         for (int kb = kb0; kb < kb1; ++kb) {
+          const int ks = (kb - kb0) % sub;
+          if (ks == 0) {
+            if (!mbar_wait(tempty_bar(acc), aph[acc] ^ 1, abort_flag, p.status)) { ok = false; break; }
+            fence_after();
+            dcol = tmem + (uint32_t)(acc * p.BN);
+          }
           if (!mbar_wait(full_bar(stage), ph, abort_flag, p.status)) { ok = false; break; }
           fence_after();
           const uint32_t sa = sbase + stage * STAGE_BYTES, sb = sa + A_BYTES;
@@ -383,15 +394,17 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm(const __grid_constant_
             // K-major: +32 bytes per 16 K; MN-major: +2 groups of 8 K-rows (2048 bytes)
             const uint64_t da = a_mn ? sdesc(sa + kk * 2048, 8192, 1024) : sdesc(sa + kk * 32, 16, 1024);
             const uint64_t db = (p.mode == FG) ? da : sdesc(sb + kk * 32, 16, 1024);
-            mma_bf16(dcol, da, db, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            mma_bf16(dcol, da, db, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; ph ^= 1; }
+          if (ks == sub - 1 || kb == kb1 - 1) {
+            mma_commit(tfull_bar(acc));
+            aph[acc] ^= 1;
+            acc ^= 1;
+          }
         }
         if (!ok) break;
-        mma_commit(tfull_bar(acc));
-        aph[acc] ^= 1;
-        acc ^= 1;
       }
     }
   } else {
@@ -405,10 +418,42 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm(const __grid_constant_
       const int Mc = cell_M(p, cell);
       if (m0 >= Mc) continue;
       if (p.mode == WP && n0 >= p.wp_rows[cell]) continue;
-      {
-        int kb0, kb1;
-        k_range(p, cell, m0, kb0, kb1);
-        if (kb0 >= kb1) continue;
+      int kb0, kb1;
+      k_range(p, cell, m0, kb0, kb1);
+      if (kb0 >= kb1) continue;
+      if (p.mode == FG) {
+        // the tile's sub-tiles (FG_PROMOTE k-steps each, accumulated by the
+        // tensor cores) summed here in fp32, round-to-nearest: the tensor
+        // cores' own fp32 accumulation loses a fraction of an ulp per step
+        // toward zero, a bias that grows with the number of steps over a sum
+        // of squares, so it is kept to FG_PROMOTE steps at a time
+        const int nsub = (kb1 - kb0 + FG_PROMOTE - 1) / FG_PROMOTE;
+        float sum[128];
+#pragma unroll
+        for (int i = 0; i < 128; ++i) sum[i] = 0.0f;
+        bool ok = true;
+        for (int sidx = 0; sidx < nsub; ++sidx) {
+          if (!mbar_wait(tfull_bar(acc), aph[acc], abort_flag, p.status)) { ok = false; break; }
+          fence_after();
+          const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.BN);
+#pragma unroll
+          for (int c0 = 0; c0 < 128; c0 += 16) {
+            float v[16];
+            tmem_ld16(tb + c0, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sum[c0 + i] = __fadd_rn(sum[c0 + i], v[i]);
+          }
+          fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar(acc));
+          aph[acc] ^= 1;
+          acc ^= 1;
+        }
+        if (!ok) break;
+        float* dst = p.out_f32 + ((int64_t)cell * p.fg_chunks + m0 / BM) * (BM * 128) + (int64_t)(q * 32 + lane) * 128;
+#pragma unroll
+        for (int i = 0; i < 128; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(sum[i], sum[i + 1], sum[i + 2], sum[i + 3]);
+        continue;
       }
       if (!mbar_wait(tfull_bar(acc), aph[acc], abort_flag, p.status)) break;
       fence_after();
@@ -425,10 +470,6 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm(const __grid_constant_
             for (int i = 0; i < 16; ++i)
               if (n + i < p.N) dst[(int64_t)(n + i) * p.t_pitch] = bf16_bits_from_f32(v[i]);
           }
-        } else if (p.mode == FG) {
-          float* dst = p.out_f32 + ((int64_t)cell * p.fg_chunks + m0 / BM) * (BM * 128) + (int64_t)(q * 32 + lane) * 128;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) dst[n + i] = v[i];
         } else if (p.mode == XTY || p.mode == GRAM) {
           if (row < Mc) {
             float* dst = p.out_f32 + (int64_t)cell * p.out_cell_stride + (int64_t)row * p.N;

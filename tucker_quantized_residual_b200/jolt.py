@@ -44,7 +44,8 @@ class jolt_options(C.Structure):
                 ("n_rd", C.c_int32), ("rd_grid", C.POINTER(C.c_int32)),
                 ("rt_max", C.c_int32), ("oversample_p", C.c_int32), ("power_iters", C.c_int32),
                 ("scale_group", C.c_int32), ("rotation", C.c_int32),
-                ("budget_tol", C.c_double), ("max_iters", C.c_int32), ("minimizer", C.c_int32)]
+                ("budget_tol", C.c_double), ("max_iters", C.c_int32), ("minimizer", C.c_int32),
+                ("seq_base", C.c_int32), ("group_base", C.c_int32), ("cap_ratio", C.c_double)]
 
 
 class jolt_cell_info(C.Structure):
@@ -68,6 +69,9 @@ _SIGS = {
     "jolt_plan": (C.c_int, [C.POINTER(jolt_layout), _I64, C.POINTER(jolt_options), C.POINTER(_VP)]),
     "jolt_free_plan": (None, [_VP]),
     "jolt_compress": (C.c_int, [_VP, _VP, _VP, _I64, _U64, _VP, C.POINTER(_VP)]),
+    "jolt_summary_bytes": (_I64, [_VP]),
+    "jolt_compress_begin": (C.c_int, [_VP, _VP, _VP, _I64, _U64, _VP, _VP, C.POINTER(_VP)]),
+    "jolt_compress_end": (C.c_int, [_VP, _VP, _I32, _I32, _VP]),
     "jolt_decompress": (C.c_int, [_VP, _VP, _VP, C.POINTER(jolt_layout), _VP]),
     "jolt_bytes": (C.c_int, [_VP, C.POINTER(_I64)]),
     "jolt_handle_info": (C.c_int, [_VP, C.POINTER(jolt_cell_info), _I32, C.POINTER(_D), C.POINTER(_I32)]),
@@ -160,7 +164,8 @@ def make_options(mode: int = JOLT_EXACT, bits: Sequence[int] = (0, 2, 4, 8),
                  rt_max: int = 0, oversample_p: int = 8, power_iters: int = 2,
                  scale_group: int = 0, budget_tol: float = 0.005,
                  max_iters: int = 50, minimizer: int = 0,
-                 rotation: int = JOLT_ROT_HADAMARD) -> Tuple[jolt_options, list]:
+                 rotation: int = JOLT_ROT_HADAMARD, seq_base: int = 0,
+                 group_base: int = 0, cap_ratio: float = 0.0) -> Tuple[jolt_options, list]:
     lib = load_library()
     o = jolt_options()
     lib.jolt_default_options(C.byref(o))
@@ -181,6 +186,7 @@ def make_options(mode: int = JOLT_EXACT, bits: Sequence[int] = (0, 2, 4, 8),
     o.scale_group, o.budget_tol, o.max_iters = scale_group, budget_tol, max_iters
     o.minimizer = minimizer
     o.rotation = rotation
+    o.seq_base, o.group_base, o.cap_ratio = seq_base, group_base, cap_ratio
     return o, keep
 
 
@@ -206,6 +212,31 @@ def jolt_compress(plan: int, k, v, byte_budget: int = 0, seed: int = 0, stream=N
     _check(lib.jolt_compress(plan, _ptr(k), _ptr(v), int(byte_budget), int(seed), _stream(stream),
                              C.byref(out)))
     return out.value
+
+
+def jolt_summary_bytes(plan: int) -> int:
+    return load_library().jolt_summary_bytes(plan)
+
+
+def jolt_compress_begin(plan: int, k, v, byte_budget: int, seed: int, summary, stream=None) -> int:
+    """Phase 1 of a shared-budget compression; `summary` is a CUDA uint8
+    tensor of jolt_num_cells(plan) * jolt_summary_bytes(plan) bytes."""
+    need = jolt_num_cells(plan) * jolt_summary_bytes(plan)
+    if not (summary.is_cuda and summary.is_contiguous() and summary.numel() * summary.element_size() >= need):
+        raise ValueError(f"summary must be a contiguous CUDA buffer of at least {need} bytes")
+    out = C.c_void_p()
+    _check(load_library().jolt_compress_begin(plan, _ptr(k), _ptr(v), int(byte_budget), int(seed), _ptr(summary),
+                                              _stream(stream), C.byref(out)))
+    return out.value
+
+
+def jolt_compress_end(handle: int, all_summaries, n_total: int, first_cell: int, stream=None) -> None:
+    """Phase 2: the allocation over the gathered records of every process,
+    then this plan's fit and residual."""
+    if not (all_summaries.is_cuda and all_summaries.is_contiguous()):
+        raise ValueError("all_summaries must be a contiguous CUDA buffer")
+    _check(load_library().jolt_compress_end(handle, _ptr(all_summaries), int(n_total), int(first_cell),
+                                            _stream(stream)))
 
 
 def jolt_decompress(handle: int, k_out, v_out, out_layout: Optional[jolt_layout] = None, stream=None) -> None:
