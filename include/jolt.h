@@ -222,6 +222,31 @@ JOLT_API jolt_status jolt_compress_end(jolt_handle_t* h, const void* all_summari
 JOLT_API jolt_status jolt_decompress(const jolt_handle_t* h, void* k_out, void* v_out,
                             const jolt_layout* out_layout, jolt_stream_t stream);
 
+/* Fused decode attention over the compressed cache (Section 3.1, the decode
+ * kernel that evaluates attention directly over the stored factors and the
+ * packed residual): one decode step of layer `layer` for every sequence of
+ * the handle. For sequence b and query head j (KV head j / G, G = n_q_heads /
+ * n_heads <= 8):
+ *   out[b][j] = sum_t softmax_t(q[b][j] . k_t / sqrt(D)) v_t,
+ * over the T compressed tokens, whose keys and values are the fp32
+ * reconstruction decompression would round to bf16 (keys with RoPE
+ * re-applied), followed by n_tail dense tokens (tail_k / tail_v), with one
+ * softmax over both. Keys are rebuilt tile by tile on chip; values stay in
+ * rank space and the rotated residual domain until one final product per
+ * query head.
+ *   q: DEVICE fp32 [batch][n_q_heads][D], 16-byte aligned, already rotated
+ *     for the decode position (RoPE) as the model's queries are.
+ *   tail_k, tail_v: DEVICE bf16 [batch][n_heads][n_tail][D] (keys already
+ *     rotated), NULL when n_tail == 0; n_tail <= 1024.
+ *   out: DEVICE fp32 [batch][n_q_heads][D].
+ * The handle must use the Hadamard rotation (JOLT_ERR_UNSUPPORTED_SHAPE for
+ * JOLT_ROT_QR_GAUSS). The first call on a handle reads the cells' layout to
+ * the host (synchronises the handle's stream once); later calls are
+ * asynchronous. Workspace comes from the library allocator. */
+JOLT_API jolt_status jolt_decode_attention(const jolt_handle_t* h, int32_t layer, const float* q,
+                                           int32_t n_q_heads, const uint16_t* tail_k, const uint16_t* tail_v,
+                                           int32_t n_tail, float* out, jolt_stream_t stream);
+
 /* Sum over cells of Eq. (1) at the chosen (r_T, r_d, b): the compressed size
  * in bytes. Synchronises the handle's stream. */
 JOLT_API jolt_status jolt_bytes(const jolt_handle_t* h, int64_t* payload_bytes);

@@ -1,0 +1,139 @@
+"""Fused decode attention over the compressed cache (jolt_decode_attention,
+Section 3.1's decode kernel) against the oracle's decode_attention.
+
+The oracle compresses the same seeded cache itself (exact mode, where the
+library's allocation is bit-identical to the oracle's and its reconstruction
+within 1e-4 relative Frobenius) and evaluates attention in fp64 on its fp32
+reconstruction with one softmax over the compressed prefix and the dense tail.
+Bound: a key or value that moves by delta moves a score by at most
+|q| |delta k| / sqrt(D) and the output by at most |delta v| plus the spread of
+the values times twice the score change; with reconstructions that agree to
+about 1e-4 of their size and |q| of order sqrt(D), the outputs agree to a few
+1e-4 of max|out|: 1e-3 is the stated tolerance. A second check compares with
+torch's scaled_dot_product_attention on the library's own bf16 decompressed
+cache, whose bf16 rounding (2^-9 relative) sets a 1e-2 tolerance."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import jolt_oracle as o
+from tucker_quantized_residual_b200 import jolt, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(spec, C_ratio, seed=0, **opt):
+    K, V = synth.make_cache(spec, seed)
+    gs = synth.group_starts(spec)
+    B = o.budget_for_ratio(K.numel() * 2, C_ratio)
+    Kd, Vd = K.cuda(), V.cuda()
+    lay, keep = jolt.make_layout(Kd, gs, spec.rope_theta_k)
+    op, k2 = jolt.make_options(**opt)
+    plan = jolt.jolt_plan(lay, B, op)
+    h = jolt.jolt_compress(plan, Kd, Vd, B, 0)
+    cells, lam, it = jolt.jolt_handle_info(h, jolt.jolt_num_cells(plan))
+    oo = o.Options(**{k: v for k, v in opt.items() if k in ("bits", "rt_grid", "rd_grid")})
+    comp = o.compress(K.float().numpy(), V.float().numpy(), gs, B, 0, oo, spec.rope_theta_k)
+    assert [(c.r_t, c.r_d, c.bits) for c in cells] == comp.alloc.choice
+    return K, V, plan, h, comp
+
+
+def _run(h, layer, q, tail_k=None, tail_v=None):
+    out = torch.empty_like(q)
+    jolt.jolt_decode_attention(h, layer, q, out, tail_k, tail_v)
+    torch.cuda.synchronize()
+    return out.double().cpu().numpy()
+
+
+def _check(comp, h, spec, layer, Hq, n_tail, rng):
+    Bsz, H, D = spec.batch, spec.n_heads, spec.head_dim
+    q = torch.from_numpy(rng.standard_normal((Bsz, Hq, D)).astype(np.float32))
+    tk = tv = None
+    if n_tail:
+        tk = torch.from_numpy(rng.standard_normal((Bsz, H, n_tail, D)).astype(np.float32)).to(torch.bfloat16)
+        tv = torch.from_numpy(rng.standard_normal((Bsz, H, n_tail, D)).astype(np.float32)).to(torch.bfloat16)
+    got = _run(h, layer, q.cuda(), tk.cuda() if n_tail else None, tv.cuda() if n_tail else None)
+    worst = 0.0
+    for b in range(Bsz):
+        ref = o.decode_attention(comp, b, layer, q[b].double().numpy(),
+                                 tk[b].double().numpy() if n_tail else None,
+                                 tv[b].double().numpy() if n_tail else None)
+        err = np.abs(got[b] - ref).max() / np.abs(ref).max()
+        worst = max(worst, err)
+        assert err <= 1e-3, (b, err)
+    return got, q, tk, tv, worst
+
+
+@pytest.mark.parametrize("Hq_per,n_tail,layer", [(1, 0, 0), (4, 5, 3), (2, 17, 5)])
+def test_decode_matches_oracle_mistral_shape(Hq_per, n_tail, layer):
+    """Mistral-shaped groups of 4 layers x 8 KV heads, D = 128, keys with RoPE,
+    T = 1000 (a ragged last tile), 3x budget."""
+    spec = synth.SPECS["mistral"].replace(n_layers=8, seq_len=1000)
+    K, V, plan, h, comp = _case(spec, 3.0)
+    try:
+        rng = np.random.default_rng(7 + layer)
+        got, q, tk, tv, worst = _check(comp, h, spec, layer, spec.n_heads * Hq_per, n_tail, rng)
+        print(f"decode layer {layer} G={Hq_per} tail={n_tail}: max rel err vs oracle {worst:.2e}")
+        # the same step through reconstruct-then-attend on the library's own cache
+        Ko = torch.empty(K.shape, dtype=torch.bfloat16, device="cuda")
+        Vo = torch.empty_like(Ko)
+        jolt.jolt_decompress(h, Ko, Vo)
+        Kl, Vl = Ko[0, layer].float(), Vo[0, layer].float()
+        if n_tail:
+            Kl = torch.cat([Kl, tk[0].cuda().float()], dim=1)
+            Vl = torch.cat([Vl, tv[0].cuda().float()], dim=1)
+        Kr = Kl.repeat_interleave(Hq_per, 0)[None]
+        Vr = Vl.repeat_interleave(Hq_per, 0)[None]
+        sd = torch.nn.functional.scaled_dot_product_attention(q[0].cuda()[None, :, None, :], Kr, Vr)[0, :, 0, :]
+        sd = sd.double().cpu().numpy()
+        assert np.abs(got[0] - sd).max() / np.abs(sd).max() <= 1e-2
+    finally:
+        torch.cuda.synchronize()
+        jolt.jolt_free_handle(h)
+        jolt.jolt_free_plan(plan)
+
+
+def test_decode_batch_and_d64_and_zero_bit_values():
+    """A batch of two sequences (each with its own rotation seed and
+    allocation), D = 64 heads with RoPE, a budget loose enough that some cells
+    drop the residual, and the tiny grid."""
+    spec = synth.CacheSpec("dec64", 2, 4, 4, 700, 64, 2, 24, 0.9, 0.02, rope_theta_k=1e4)
+    K, V, plan, h, comp = _case(spec, 2.5, seed=3, bits=(0, 2, 4), rt_grid=(4, 8, 16, 32, 64),
+                                rd_grid=(8, 16, 32, 64))
+    try:
+        rng = np.random.default_rng(11)
+        for layer in (0, 3):
+            _check(comp, h, spec, layer, 8, 3, rng)
+    finally:
+        torch.cuda.synchronize()
+        jolt.jolt_free_handle(h)
+        jolt.jolt_free_plan(plan)
+
+
+def test_decode_without_residual_bits():
+    spec = synth.SPECS["mistral"].replace(n_layers=4, seq_len=384)
+    K, V, plan, h, comp = _case(spec, 2.0, bits=(0,))
+    try:
+        assert all(c.bits == 0 for c in comp.cells)
+        _check(comp, h, spec, 2, 16, 4, np.random.default_rng(5))
+    finally:
+        torch.cuda.synchronize()
+        jolt.jolt_free_handle(h)
+        jolt.jolt_free_plan(plan)
+
+
+def test_decode_rejects_bad_arguments():
+    spec = synth.SPECS["mistral"].replace(n_layers=4, seq_len=256)
+    K, V, plan, h, comp = _case(spec, 3.0)
+    try:
+        q = torch.zeros((1, 8, 128), device="cuda")
+        out = torch.zeros_like(q)
+        with pytest.raises(jolt.JoltError):
+            jolt.jolt_decode_attention(h, 4, q, out)                 # layer out of range
+        q12 = torch.zeros((1, 12, 128), device="cuda")
+        with pytest.raises(jolt.JoltError):
+            jolt.jolt_decode_attention(h, 0, q12, torch.zeros_like(q12))   # 12 query heads over 8 KV heads
+    finally:
+        torch.cuda.synchronize()
+        jolt.jolt_free_handle(h)
+        jolt.jolt_free_plan(plan)

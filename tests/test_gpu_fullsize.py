@@ -77,7 +77,10 @@ def _same_sketch(spec, C_ratio):
         N = (c.l1 - c.l0) * spec.n_heads * spec.head_dim
         Om = o.library_sketch(N, k, ld, c.b, 2 * c.g + c.kind)
         w, _ = o.randomized_token_spectrum(X, Om, 2, qc)
-        nsq = float(np.sum(X * X))
+        # randomized mode reads keys with a RoPE base as the un-RoPE'd values
+        # rounded to bf16 (the tensor-core operand); values are read as stored
+        Xop = o.bf16_rne(X) if (c.kind == 0 and spec.rope_theta_k > 0) else X
+        nsq = float(np.sum(Xop * Xop))
         # the feature Gram (and its trace) is summed by the tensor cores 256 rows
         # at a time, then in fp32 with round-to-nearest; inside the tensor cores
         # each row's product can lose up to one ulp toward zero

@@ -218,6 +218,7 @@ struct jolt_handle_s {
   int phase = 0;                 // 1: spectra done (begin), 2: compressed (end)
   const void* k_in = nullptr;    // inputs of a begun two-phase compression
   const void* v_in = nullptr;
+  std::vector<CellOut> h_out;    // host copy of the cells' layout (decode attention)
 };
 
 static jolt_status status_from_dev(int st) {
@@ -1486,3 +1487,87 @@ jolt_status jolt_residual_stream_encode(const void* x, int32_t LH, int32_t T, in
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------- decode attention ----
+extern "C" jolt_status jolt_decode_attention(const jolt_handle_t* hc, int32_t layer, const float* q,
+                                             int32_t n_q_heads, const uint16_t* tail_k, const uint16_t* tail_v,
+                                             int32_t n_tail, float* out, jolt_stream_t stream_) {
+  cudaStream_t s = (cudaStream_t)stream_;
+  if (!hc || !q || !out) { set_error("null argument"); return JOLT_ERR_INVALID_ARG; }
+  jolt_handle_s* h = const_cast<jolt_handle_s*>(hc);
+  if (h->phase != 2) { set_error("the handle's compression has not ended (jolt_compress_end)"); return JOLT_ERR_INVALID_ARG; }
+  jolt_plan_s* p = h->plan;
+  const jolt_layout& L = p->lay;
+  if (layer < 0 || layer >= L.n_layers) { set_error("layer %d out of range", layer); return JOLT_ERR_INVALID_ARG; }
+  if (n_q_heads < p->H || n_q_heads % p->H || n_q_heads / p->H > 8) {
+    set_error("n_q_heads must be 1..8 times the %d KV heads", p->H); return JOLT_ERR_INVALID_ARG;
+  }
+  if (n_tail < 0 || n_tail > 1024 || (n_tail > 0 && (!tail_k || !tail_v))) {
+    set_error("n_tail must be 0..1024, with both tail tensors when positive"); return JOLT_ERR_INVALID_ARG;
+  }
+  if (h->d_qrot) { set_error("fused decode attention implements the Hadamard rotation only"); return JOLT_ERR_UNSUPPORTED_SHAPE; }
+  if (reinterpret_cast<uintptr_t>(q) % 16) { set_error("q must be 16-byte aligned"); return JOLT_ERR_INVALID_ARG; }
+  // the cells' layout on the host, read once per handle
+  if (h->h_out.empty()) {
+    JOLT_CUDA_TRY(cudaStreamSynchronize(h->stream));
+    h->h_out.resize(p->ncells);
+    JOLT_CUDA_TRY(cudaMemcpy(h->h_out.data(), h->d_out, p->ncells * sizeof(CellOut), cudaMemcpyDeviceToHost));
+  }
+  int g = 0;
+  while (g + 1 < L.n_groups && p->gstart[g + 1] <= layer) ++g;
+  const int li = layer - p->gstart[g];
+  const int H = p->H, D = p->D, G = n_q_heads / H;
+  for (int b0 = 0; b0 < L.batch; b0 += DEC_BMAX) {
+    const int Bc = std::min(DEC_BMAX, L.batch - b0);
+    std::vector<CellOut> ko(Bc), vo(Bc);
+    int rk = 1, rv = 1;
+    DecodeCall c{};
+    for (int b = 0; b < Bc; ++b) {
+      ko[b] = h->h_out[((b0 + b) * L.n_groups + g) * 2 + 0];
+      vo[b] = h->h_out[((b0 + b) * L.n_groups + g) * 2 + 1];
+      rk = std::max(rk, ko[b].rT);
+      rv = std::max(rv, vo[b].rT);
+      c.ut[b] = ko[b].ut;
+      c.rt_k[b] = ko[b].rT;
+      c.tpitch[b] = ko[b].t_pitch;
+    }
+    const int rpk = (rk + 63) / 64 * 64, rpv = (rv + 63) / 64 * 64;
+    const int64_t part_len = (int64_t)Bc * H * 64 * G * (2 + rpv + D);
+    Arena A;
+    CellOut* dko = nullptr; CellOut* dvo = nullptr; uint16_t* mtk = nullptr; float* mv = nullptr; float* part = nullptr;
+    void* blk = nullptr;
+    for (int pass = 0; pass < 2; ++pass) {
+      A.used = 0;
+      dko = A.take<CellOut>(Bc);
+      dvo = A.take<CellOut>(Bc);
+      mtk = A.take<uint16_t>((size_t)Bc * H * D * rpk);
+      mv = A.take<float>((size_t)Bc * H * rpv * D);
+      part = A.take<float>((size_t)part_len);
+      if (pass == 0) {
+        blk = dev_alloc(A.used + 256, s);
+        if (!blk) { set_error("decode attention workspace allocation failed"); return JOLT_ERR_OOM; }
+        A.base = reinterpret_cast<uint8_t*>(blk);
+      }
+    }
+    auto run = [&]() -> jolt_status {
+      JOLT_CUDA_TRY(cudaMemcpyAsync(dko, ko.data(), Bc * sizeof(CellOut), cudaMemcpyHostToDevice, s));
+      JOLT_CUDA_TRY(cudaMemcpyAsync(dvo, vo.data(), Bc * sizeof(CellOut), cudaMemcpyHostToDevice, s));
+      c.B = Bc; c.H = H; c.D = D; c.T = p->T; c.G = G; c.gq = p->G; c.li = li;
+      c.kout = dko; c.vout = dvo;
+      c.cs = (L.rope_theta_k > 0) ? p->d_cs : nullptr;
+      c.seed = h->seed + (uint64_t)b0;
+      c.q = q + (int64_t)b0 * n_q_heads * D;
+      c.out = out + (int64_t)b0 * n_q_heads * D;
+      c.tail_k = n_tail ? tail_k + (int64_t)b0 * H * n_tail * D : nullptr;
+      c.tail_v = n_tail ? tail_v + (int64_t)b0 * H * n_tail * D : nullptr;
+      c.ntail = n_tail;
+      c.mtk = mtk; c.rpk = rpk; c.mv = mv; c.rpv = rpv; c.part = part; c.part_len = part_len;
+      c.status = h->d_status;
+      return launch_decode_attention(c, s);
+    };
+    jolt_status st = run();
+    dev_free(blk, s);
+    if (st != JOLT_OK) return st;
+  }
+  return JOLT_OK;
+}

@@ -232,6 +232,28 @@ struct StreamArgs {
   int* status;
 };
 jolt_status launch_stream(bool compress, int D, const StreamMaps& m, const StreamArgs& a, cudaStream_t s);
+
+// ------------------------------------------------- fused decode attention --
+constexpr int DEC_BMAX = 16;      // sequences per launch
+struct DecodeCall {
+  int B, H, D, T, G, gq, li;      // G query heads per KV head, li = layer within its group
+  const CellOut* kout;            // [B] key cells (device)
+  const CellOut* vout;            // [B] value cells (device)
+  const float2* cs;               // RoPE table of the keys, or null
+  uint64_t seed;                  // rotation seed of sequence 0
+  const float* q;                 // [B][H*G][D]
+  float* out;                     // [B][H*G][D]
+  const uint16_t* tail_k;         // [B][H][ntail][D] bf16, or null
+  const uint16_t* tail_v;
+  int ntail;
+  uint16_t* mtk; int rpk;         // workspace: M^_K^T [B*H][D][rpk]
+  float* mv; int rpv;             // workspace: M^_V [B*H][rpv][D]
+  float* part; int64_t part_len;  // workspace: split states
+  const uint16_t* ut[DEC_BMAX];   // U_T^ of each sequence's key cell and its shape
+  int rt_k[DEC_BMAX], tpitch[DEC_BMAX];
+  int* status;
+};
+jolt_status launch_decode_attention(const DecodeCall& c, cudaStream_t s);
 jolt_status launch_ut_to_ws(const CellOut* outs, uint16_t* ws, int rows, int tp, int ncells, cudaStream_t s);
 jolt_status launch_m_transpose(const CellOut* outs, const CellDesc* cells, uint16_t* const* M, const int* rmax_of,
                                uint16_t* Mt, int lhmax, int D, int rpad, int ncells, cudaStream_t s);

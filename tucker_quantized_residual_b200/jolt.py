@@ -73,6 +73,7 @@ _SIGS = {
     "jolt_compress_begin": (C.c_int, [_VP, _VP, _VP, _I64, _U64, _VP, _VP, C.POINTER(_VP)]),
     "jolt_compress_end": (C.c_int, [_VP, _VP, _I32, _I32, _VP]),
     "jolt_decompress": (C.c_int, [_VP, _VP, _VP, C.POINTER(jolt_layout), _VP]),
+    "jolt_decode_attention": (C.c_int, [_VP, _I32, _VP, _I32, _VP, _VP, _I32, _VP, _VP]),
     "jolt_bytes": (C.c_int, [_VP, C.POINTER(_I64)]),
     "jolt_handle_info": (C.c_int, [_VP, C.POINTER(jolt_cell_info), _I32, C.POINTER(_D), C.POINTER(_I32)]),
     "jolt_handle_cell": (C.c_int, [_VP, _I32, C.POINTER(jolt_cell_view)]),
@@ -243,6 +244,23 @@ def jolt_decompress(handle: int, k_out, v_out, out_layout: Optional[jolt_layout]
     lib = load_library()
     _check(lib.jolt_decompress(handle, _ptr(k_out), _ptr(v_out),
                                C.byref(out_layout) if out_layout is not None else None, _stream(stream)))
+
+
+def jolt_decode_attention(handle: int, layer: int, q, out, tail_k=None, tail_v=None, stream=None) -> None:
+    """One fused decode step of `layer`: q fp32 [B, Hq, D] -> out fp32 [B, Hq, D];
+    optional dense tail bf16 [B, H, n_tail, D] (CUDA, contiguous)."""
+    import torch
+    for t, dt in ((q, torch.float32), (out, torch.float32)):
+        if not (t.is_cuda and t.dtype == dt and t.is_contiguous() and t.dim() == 3):
+            raise ValueError("q and out must be contiguous CUDA float32 tensors [B, Hq, D]")
+    n_tail = 0
+    if tail_k is not None:
+        for t in (tail_k, tail_v):
+            if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
+                raise ValueError("tail_k and tail_v must be contiguous CUDA bfloat16 tensors [B, H, n, D]")
+        n_tail = tail_k.shape[2]
+    _check(load_library().jolt_decode_attention(handle, int(layer), _ptr(q), q.shape[1], _ptr(tail_k),
+                                                _ptr(tail_v), n_tail, _ptr(out), _stream(stream)))
 
 
 def jolt_bytes(handle: int) -> int:

@@ -48,20 +48,26 @@ def first_cells(counts: Sequence[int]) -> List[int]:
     return out
 
 
-def gather_records(local, n_local: int, rec_bytes: int, group=None):
+def gather_records(local, n_local: int, rec_bytes: int, group=None, counts=None):
     """All-gather every rank's records into one contiguous buffer in rank
     order, for any mix of per-rank counts. `local` is a uint8 tensor holding
     n_local records of rec_bytes each (on the device for NCCL, on the host for
-    gloo). Returns (all_records, counts): all_records holds sum(counts)
-    records, rank r's at first_cells(counts)[r]."""
+    gloo). `counts` (every rank's record count) may be given when known, which
+    saves an exchange and a host synchronisation. Returns (all_records,
+    counts): all_records holds sum(counts) records, rank r's at
+    first_cells(counts)[r]."""
     import torch
     import torch.distributed as dist
     world = dist.get_world_size(group)
     dev = local.device
-    cnt = torch.tensor([n_local], dtype=torch.int64, device=dev)
-    counts_t = torch.zeros(world, dtype=torch.int64, device=dev)
-    dist.all_gather_into_tensor(counts_t, cnt, group=group)
-    counts = [int(c) for c in counts_t.cpu().tolist()]
+    if counts is None:
+        cnt = torch.tensor([n_local], dtype=torch.int64, device=dev)
+        counts_t = torch.zeros(world, dtype=torch.int64, device=dev)
+        dist.all_gather_into_tensor(counts_t, cnt, group=group)
+        counts = [int(c) for c in counts_t.cpu().tolist()]
+    counts = list(counts)
+    if len(counts) != world or counts[dist.get_rank(group)] != n_local:
+        raise ValueError("counts must list every rank's record count, this rank's included")
     cmax = max(counts)
     # equal-size contributions for the collective: pad to the largest count
     send = torch.zeros(cmax * rec_bytes, dtype=torch.uint8, device=dev)
@@ -102,10 +108,11 @@ def encode_record(rec: Dict, rec_bytes: int) -> bytes:
     return bytes(body)
 
 
-def compress_sharded(plan: int, k, v, byte_budget: int, seed: int, group=None, stream=None):
+def compress_sharded(plan: int, k, v, byte_budget: int, seed: int, group=None, stream=None, counts=None):
     """The whole protocol on this rank: begin (local spectra and records),
     all-gather of the records, end (shared allocation, local fit and
-    residual). Returns (handle, counts, first_cell)."""
+    residual). `counts`: every rank's cell count, when known. Returns
+    (handle, counts, first_cell)."""
     import torch
     import torch.distributed as dist
     from . import jolt
@@ -117,7 +124,7 @@ def compress_sharded(plan: int, k, v, byte_budget: int, seed: int, group=None, s
         # the collective runs on the current stream: order it after begin's kernels
         if stream is not None and stream != torch.cuda.current_stream():
             torch.cuda.current_stream().wait_stream(stream)
-        allrec, counts = gather_records(local, n, rb, group)
+        allrec, counts = gather_records(local, n, rb, group, counts)
         first = first_cells(counts)[dist.get_rank(group)]
         if stream is not None and stream != torch.cuda.current_stream():
             stream.wait_stream(torch.cuda.current_stream())
