@@ -114,7 +114,7 @@ def test_decode_without_residual_bits():
     spec = synth.SPECS["mistral"].replace(n_layers=4, seq_len=384)
     K, V, plan, h, comp = _case(spec, 2.0, bits=(0,))
     try:
-        assert all(c.bits == 0 for c in comp.cells)
+        assert all(c.b == 0 for c in comp.cells)
         _check(comp, h, spec, 2, 16, 4, np.random.default_rng(5))
     finally:
         torch.cuda.synchronize()
