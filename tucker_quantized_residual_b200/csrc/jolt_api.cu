@@ -144,6 +144,7 @@ struct jolt_plan_s {
   int* d_rt = nullptr;
   int* d_rd = nullptr;
   float2* d_cs = nullptr;
+  float4* d_csq = nullptr;       // the RoPE table tiled for the stream kernels
   CellDesc* d_cells = nullptr;
   CellRD* d_rd_cells = nullptr;
   int* d_nt = nullptr;
@@ -529,6 +530,7 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
     p->d_rt = A.take<int>(p->rt_grid.size());
     p->d_rd = A.take<int>(p->rd_grid.size());
     p->d_cs = p->lay.rope_theta_k > 0 ? A.take<float2>((size_t)T * (D / 2)) : nullptr;
+    p->d_csq = p->lay.rope_theta_k > 0 ? A.take<float4>((size_t)((T + 127) / 128) * 128 * (D / 4)) : nullptr;
     p->d_cells = A.take<CellDesc>(nc);
     p->d_rd_cells = A.take<CellRD>(nc);
     p->d_nt = A.take<int>(nc);
@@ -698,7 +700,10 @@ static jolt_status plan_build_workspace(jolt_plan_s* p) {
       JOLT_CUDA_TRY(cudaMemsetAsync(p->Yt, 0, (size_t)nc * k * p->tp * 2, s));
       JOLT_CUDA_TRY(cudaMemsetAsync(p->Pt, 0, (size_t)nc * p->rpad * p->kpad * 2, s));
     }
-    if (p->d_cs) JOLT_TRY(launch_rope_table(T, D, (double)p->lay.rope_theta_k, p->d_cs, s));
+    if (p->d_cs) {
+      JOLT_TRY(launch_rope_table(T, D, (double)p->lay.rope_theta_k, p->d_cs, s));
+      JOLT_TRY(launch_rope_tiled(p->d_cs, T, D, p->d_csq, s));
+    }
     JOLT_TRY(launch_eps2(p->bits.data(), (int)p->bits.size(), p->G, p->d_eps2, p->d_fpart, s));
     JOLT_CUDA_TRY(cudaStreamSynchronize(s));
   }
@@ -928,7 +933,7 @@ static jolt_status run_stream(jolt_plan_s* p, const jolt_handle_s* h, const void
   }
   StreamArgs a{};
   a.ncells = nc; a.T = p->T; a.H = p->H; a.lhmax = p->lh_max; a.rpad_m = p->rpad_m; a.G = p->G;
-  a.cells = p->d_cells; a.outs = h->d_out; a.cs = p->d_cs; a.seed = h->seed;
+  a.cells = p->d_cells; a.outs = h->d_out; a.cs = p->d_cs; a.csq = p->d_csq; a.seed = h->seed;
   if (!compress) {
     a.out_k = reinterpret_cast<uint16_t*>(k_out);
     a.out_v = reinterpret_cast<uint16_t*>(v_out);
@@ -1430,6 +1435,7 @@ jolt_status jolt_residual_stream_encode(const void* x, int32_t LH, int32_t T, in
   Arena A;
   CellDesc* d_cell = nullptr; CellOut* d_out = nullptr; uint16_t** d_M = nullptr; int* d_rmax = nullptr;
   int* d_status = nullptr; uint16_t* ut_ws = nullptr; uint16_t* mt_ws = nullptr; float2* cs = nullptr;
+  float4* csq = nullptr;
   void* block = nullptr;
   for (int pass = 0; pass < 2; ++pass) {
     A.used = 0;
@@ -1441,6 +1447,7 @@ jolt_status jolt_residual_stream_encode(const void* x, int32_t LH, int32_t T, in
     ut_ws = A.take<uint16_t>((size_t)rows * tp);
     mt_ws = A.take<uint16_t>((size_t)LH * D * rows);
     cs = rope_theta > 0.0f ? A.take<float2>((size_t)T * (D / 2)) : nullptr;
+    csq = rope_theta > 0.0f ? A.take<float4>((size_t)((T + 127) / 128) * 128 * (D / 4)) : nullptr;
     if (pass == 0) {
       block = dev_alloc(A.used + 256, s);
       if (!block) { set_error("scratch allocation failed"); return JOLT_ERR_OOM; }
@@ -1462,7 +1469,10 @@ jolt_status jolt_residual_stream_encode(const void* x, int32_t LH, int32_t T, in
     JOLT_CUDA_TRY(cudaMemcpyAsync(d_M, &mp, sizeof(mp), cudaMemcpyHostToDevice, s));
     JOLT_CUDA_TRY(cudaMemcpyAsync(d_rmax, &r, sizeof(int), cudaMemcpyHostToDevice, s));
     JOLT_CUDA_TRY(cudaMemsetAsync(d_status, 0, 4 * sizeof(int), s));
-    if (cs) JOLT_TRY(launch_rope_table(T, D, (double)rope_theta, cs, s));
+    if (cs) {
+      JOLT_TRY(launch_rope_table(T, D, (double)rope_theta, cs, s));
+      JOLT_TRY(launch_rope_tiled(cs, T, D, csq, s));
+    }
     JOLT_TRY(launch_m_transpose(d_out, d_cell, d_M, d_rmax, mt_ws, LH, D, rows, 1, s));
     JOLT_TRY(launch_ut_to_ws(d_out, ut_ws, rows, tp, 1, s));
     StreamMaps mp4{};
@@ -1472,7 +1482,7 @@ jolt_status jolt_residual_stream_encode(const void* x, int32_t LH, int32_t T, in
     mp4.xv = mp4.xk;
     StreamArgs a{};
     a.ncells = 1; a.T = T; a.H = LH; a.lhmax = LH; a.rpad_m = rows; a.G = group;
-    a.cells = d_cell; a.outs = d_out; a.cs = cs; a.seed = seed; a.status = d_status;
+    a.cells = d_cell; a.outs = d_out; a.cs = cs; a.csq = csq; a.seed = seed; a.status = d_status;
     JOLT_TRY(launch_stream(true, D, mp4, a, s));
     // the host structures above are read by copies still in flight: wait
     JOLT_CUDA_TRY(cudaStreamSynchronize(s));

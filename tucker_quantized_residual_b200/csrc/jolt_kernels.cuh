@@ -225,6 +225,7 @@ struct StreamArgs {
   const CellDesc* cells;
   const CellOut* outs;
   const float2* cs;
+  const float4* csq;     // the RoPE table tiled for the stream kernel (launch_rope_tiled), or null
   uint64_t seed;
   uint16_t* out_k;
   uint16_t* out_v;
@@ -232,6 +233,12 @@ struct StreamArgs {
   int* status;
 };
 jolt_status launch_stream(bool compress, int D, const StreamMaps& m, const StreamArgs& a, cudaStream_t s);
+// The RoPE table rearranged so that the stream kernel's warps read it with
+// coalesced 16-byte loads: for token tile tau (128 tokens), column quarter j
+// and pair unit u (pairs 2u, 2u + 1 of the quarter's D/8 pairs), the 128 rows'
+// float4 (cos, sin, cos, sin) are contiguous: csq[((tau*4 + j)*(D/16) + u)*128 + row].
+// Rows past T hold zeros. ceil(T/128)*128*D/2 float2 entries.
+jolt_status launch_rope_tiled(const float2* cs, int T, int D, float4* csq, cudaStream_t s);
 
 // ------------------------------------------------- fused decode attention --
 constexpr int DEC_BMAX = 16;      // sequences per launch

@@ -23,6 +23,11 @@ constexpr int S_CODE = 128 * 128;          // packed codes of a tile (<= 8 bits 
 constexpr int S_SCALE = 128 * 4 * 4;       // scales of a tile (<= 4 groups per row)
 constexpr int S_R1 = (2 * S_X > 2 * (S_CODE + S_SCALE)) ? 2 * S_X : 2 * (S_CODE + S_SCALE);
 constexpr int SMEM_STREAM = SSTAGES * (S_A + S_B) + S_R1 + 128 * 16 + 128 * 4 + 1024 + 512;
+// the four-threads-per-row stream kernel: code rows staged with a 16-byte pad
+constexpr int S_CODEP = 128 * (128 + 16);
+constexpr int S_R1Q = (2 * S_X > 2 * (S_CODEP + S_SCALE)) ? 2 * S_X : 2 * (S_CODEP + S_SCALE);
+static_assert(S_R1Q <= S_R1 + 8192, "stream staging");
+constexpr int SMEM_STREAM4 = SSTAGES * (S_A + S_B) + S_R1Q + 128 * 8 * 4 + 128 * 4 + 1024 + 512;
 constexpr int EPI_WARPS = 8;
 constexpr int STHREADS = 64 + 32 * EPI_WARPS;
 
@@ -31,6 +36,7 @@ struct Args {
   const CellDesc* cells;
   const CellOut* outs;
   const float2* cs;
+  const float4* csq;
   uint64_t seed;
   uint16_t* out_k;
   uint16_t* out_v;
@@ -223,6 +229,14 @@ __device__ __forceinline__ void fwht_pair(float* e, uint32_t lane_base, uint32_t
 // to the nearest integer (ties to even) is the fp32 addition of
 // 1.5 * 2^23 + 2^(b-1), whose low b mantissa bits then hold u = code + 2^(b-1),
 // packed LSB first.
+// Bit-field insert: the low `len` bits of a into b at bit `pos` (constant
+// pos and len after unrolling).
+__device__ __forceinline__ uint32_t bfi(uint32_t a, uint32_t b, int pos, int len) {
+  uint32_t d;
+  asm("bfi.b32 %0, %1, %2, %3, %4;" : "=r"(d) : "r"(a), "r"(b), "r"(pos), "r"(len));
+  return d;
+}
+
 template <int C, int B>
 __device__ __forceinline__ void quant_chunk(const float* r, float sc, uint32_t* w) {
   constexpr int NW = (C * B + 31) / 32;
@@ -240,10 +254,15 @@ __device__ __forceinline__ void quant_chunk(const float* r, float sc, uint32_t* 
       const float y = fminf(fmaxf(__fmul_rn(r[i], inv), -qm), qm);
       const float t = __fadd_rn(y, magic);
       if (!(0.5f - fabsf(__fsub_rn(y, __fsub_rn(t, magic))) >= 1e-4f)) need |= 1u << i;
-      const uint32_t u = __float_as_uint(t) & mask;
+      const uint32_t u = __float_as_uint(t);
       const int bit = i * B, wi = bit >> 5, sh = bit & 31;
-      w[wi] |= u << sh;
-      if (sh + B > 32) w[wi + 1] |= u >> (32 - sh);
+      // insert the low bits of u (one bit-field insert masks them)
+      if (sh + B <= 32) {
+        w[wi] = bfi(u, w[wi], sh, B);
+      } else {
+        w[wi] |= (u & mask) << sh;
+        w[wi + 1] |= (u & mask) >> (32 - sh);
+      }
     }
     if (need) {
 #pragma unroll
