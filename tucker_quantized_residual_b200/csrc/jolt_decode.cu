@@ -34,21 +34,24 @@ using namespace strm;
 constexpr int GMAX = 8;          // query heads per KV head
 constexpr int RVMAX = 512;       // value token rank (rank-space accumulators)
 constexpr int BMAX = DEC_BMAX;   // sequences per launch (one U_T^ tensor map each)
-constexpr int RCH = 64;          // ranks per staged chunk of U_T^V
 
 // shared-memory layout (bytes, from the 1 KB-aligned base)
 constexpr int OFF_RING = 0;
 constexpr int OFF_KCODE = SSTAGES * (S_A + S_B);                    // 2 x (codes + scales) of keys
-constexpr int OFF_U = OFF_KCODE + 2 * (S_CODE + S_SCALE);            // [128 t][RCH r] bf16
-constexpr int OFF_VCODE = OFF_U + 128 * RCH * 2;                     // [128][<= 128 bytes]
+constexpr int TSUB = 32;         // tokens per staged U_T^V slice
+constexpr int UP = TSUB + 2;     // its row pitch in bf16 (17 words: rank rows on distinct banks)
+constexpr int OFF_U = OFF_KCODE + 2 * (S_CODE + S_SCALE);            // [RVMAX r][UP] bf16
+constexpr int OFF_VCODE = OFF_U + RVMAX * UP * 2;                    // [128][<= 128 bytes]
 constexpr int OFF_VSCALE = OFF_VCODE + S_CODE;                       // [128][<= 4] fp32
 constexpr int OFF_Q = OFF_VSCALE + S_SCALE;                          // [GMAX][128] fp32
-constexpr int OFF_P = OFF_Q + GMAX * 128 * 4;                        // [GMAX][128] fp32
+constexpr int OFF_P = OFF_Q + GMAX * 128 * 4;                        // [128 t][GMAX] fp32
 constexpr int OFF_PART = OFF_P + GMAX * 128 * 4;                     // [GMAX][128][2] fp32
 constexpr int OFF_RED = OFF_PART + GMAX * 128 * 2 * 4;               // [2][GMAX][4] fp32
 constexpr int OFF_SIGN = OFF_RED + 2 * GMAX * 4 * 4;                 // [128] fp32
-constexpr int OFF_BAR = OFF_SIGN + 128 * 4;
+constexpr int OFF_ERED = OFF_SIGN + 128 * 4;                         // [4][GMAX][128] fp32 (item end)
+constexpr int OFF_BAR = OFF_ERED + 4 * GMAX * 128 * 4;
 constexpr int SMEM_DEC = OFF_BAR + 256 + 1024;
+static_assert(SMEM_DEC <= 227 * 1024, "decode attention shared memory");
 
 struct Maps {
   CUtensorMap mt;          // M^_K^T workspace [B*H][D][rpk] bf16, box {64 r, D}
@@ -94,6 +97,7 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
   float* sPart = reinterpret_cast<float*>(smem + OFF_PART);
   float* sRed = reinterpret_cast<float*>(smem + OFF_RED);
   float* sSign = reinterpret_cast<float*>(smem + OFF_SIGN);
+  float* sEred = reinterpret_cast<float*>(smem + OFF_ERED);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * SSTAGES + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -237,7 +241,6 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
       item_of(a, it, b, h, s);
       const CellOut ko = a.kout[b], vo = a.vout[b];
       const int tb = s * a.per, te = min(a.T, tb + a.per);
-      const int nchunk = (vo.rT + RCH - 1) / RCH;
       // queries of this KV head and the sequence's rotation signs
       epi_sync();
       for (int e = et; e < G * D; e += 32 * EPI_WARPS)
@@ -247,12 +250,14 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
       float m_run[GMAX], l_run[GMAX];
 #pragma unroll
       for (int g = 0; g < GMAX; ++g) { m_run[g] = -INFINITY; l_run[g] = 0.0f; }
-      float ar[RVMAX / RCH][2];        // rank-space state: pairs (g, r) = et + 256 i of each chunk
-      float ae[4];                     // rotated residual state: pairs (g, d) = et + 256 i
+      // rank-space state: ranks r = et and et + 256, every query head
+      float ar[2][GMAX];
+      // rotated residual state: column d = et % D, the token part et / D, every query head
+      float ae[GMAX];
 #pragma unroll
-      for (int c = 0; c < RVMAX / RCH; ++c) { ar[c][0] = 0.0f; ar[c][1] = 0.0f; }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) ae[i] = 0.0f;
+      for (int g = 0; g < GMAX; ++g) { ar[0][g] = 0.0f; ar[1][g] = 0.0f; ae[g] = 0.0f; }
+      constexpr int TPARTS = 256 / D;          // token parts of the residual accumulation
+      const int dcol = et % D, tpart = et / D;
 
       for (int t0 = tb; t0 < te; t0 += SBM) {
         const int t = t0 + rl;
@@ -373,7 +378,7 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
           mnew[g] = fmaxf(m_run[g], mt);
           alpha[g] = (g < G) ? expf(m_run[g] - mnew[g]) : 0.0f;
           const float p = (g < G && valid) ? expf(sc[g] - mnew[g]) : 0.0f;
-          if (hf == 0) sP[g * 128 + rl] = p;
+          if (hf == 0) sP[rl * GMAX + g] = p;
           float ssum = p;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
@@ -399,80 +404,70 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
           l_run[g] = fmaf(l_run[g], alpha[g], tsum);
           m_run[g] = mnew[g];
         }
-        // ---- rotated value residual: pairs (g, d) = et + 256 i
+        // every value state takes the tile's rescale
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) {
+          ar[0][g] = __fmul_rn(ar[0][g], alpha[g]);
+          ar[1][g] = __fmul_rn(ar[1][g], alpha[g]);
+          ae[g] = __fmul_rn(ae[g], alpha[g]);
+        }
+        // ---- rotated value residual: this thread's column over its token part
         if (vo.b > 0) {
           const int ng = D / a.gq;
+          const int bit = dcol * vo.b, wi = bit >> 5, sh = bit & 31;
+          const uint32_t mask = (1u << vo.b) - 1u;
+          const int vrow4 = vo.b * D / 32;      // 32-bit words per row
+          const float off = (float)(1 << (vo.b - 1));
+          const int t_lo = tpart * (128 / TPARTS), t_hi = min(nrows, t_lo + 128 / TPARTS);
+          for (int tt = t_lo; tt < t_hi; ++tt) {
+            const uint32_t* wr = reinterpret_cast<const uint32_t*>(sVC) + tt * vrow4;
+            uint32_t u = wr[wi] >> sh;
+            if (sh + vo.b > 32) u |= wr[wi + 1] << (32 - sh);
+            const float dq = __fmul_rn(__fsub_rn((float)(u & mask), off), sVS[tt * ng + dcol / a.gq]);
+            const float4 p0 = reinterpret_cast<const float4*>(sP + tt * GMAX)[0];
+            const float4 p1 = reinterpret_cast<const float4*>(sP + tt * GMAX)[1];
+            const float pv[GMAX] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int pr = et + 256 * i, g = pr / D, d = pr % D;
-            if (g >= G) continue;
-            float acc_e = __fmul_rn(ae[i], alpha[g]);
-            const int bit = d * vo.b, wi = bit >> 5, sh = bit & 31;
-            const uint32_t mask = (1u << vo.b) - 1u;
-            const int vrow4 = vo.b * D / 32;      // 32-bit words per row
-            const float off = (float)(1 << (vo.b - 1));
-            for (int tt = 0; tt < nrows; ++tt) {
-              const uint32_t* wr = reinterpret_cast<const uint32_t*>(sVC) + tt * vrow4;
-              uint32_t u = wr[wi] >> sh;
-              if (sh + vo.b > 32) u |= wr[wi + 1] << (32 - sh);
-              const float code = __fsub_rn((float)(u & mask), off);
-              acc_e = fmaf(sP[g * 128 + tt], __fmul_rn(code, sVS[tt * ng + d / a.gq]), acc_e);
-            }
-            ae[i] = acc_e;
+            for (int g = 0; g < GMAX; ++g) ae[g] = fmaf(pv[g], dq, ae[g]);
           }
         }
-        // ---- rank-space values, RCH ranks at a time: pairs (g, r) = et + 256 i
-#pragma unroll
-        for (int c = 0; c < RVMAX / RCH; ++c) {
-          if (c >= nchunk) break;
-          epi_sync();   // the previous chunk's readers are done with sU
-          for (int w = et; w < RCH * 128 / 8; w += 32 * EPI_WARPS) {
-            const int r = w % RCH, tq = (w / RCH) * 8;   // 8 tokens of rank row r
-            const int rr = c * RCH + r;
+        // ---- rank-space values: TSUB tokens of U_T^V at a time, all ranks
+        for (int ts = 0; ts < nrows; ts += TSUB) {
+          epi_sync();   // the previous slice's readers are done with sU
+          const int nt = min(TSUB, nrows - ts);
+          for (int w = et; w < vo.rT * (TSUB / 8); w += 32 * EPI_WARPS) {
+            const int r = w / (TSUB / 8), tq = (w % (TSUB / 8)) * 8;
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (rr < vo.rT && t0 + tq < te) {
-              const uint16_t* src = vo.ut + (int64_t)rr * vo.t_pitch + t0 + tq;
-              if (t0 + tq + 8 <= te && ((reinterpret_cast<uintptr_t>(src) & 15u) == 0)) {
+            if (tq < nt) {
+              const uint16_t* src = vo.ut + (int64_t)r * vo.t_pitch + t0 + ts + tq;
+              if (tq + 8 <= nt && ((reinterpret_cast<uintptr_t>(src) & 15u) == 0)) {
                 v = *reinterpret_cast<const uint4*>(src);
               } else {
                 uint16_t tmp[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) tmp[j] = (t0 + tq + j < te) ? src[j] : (uint16_t)0;
+                for (int j2 = 0; j2 < 8; ++j2) tmp[j2] = (tq + j2 < nt) ? src[j2] : (uint16_t)0;
                 v = make_uint4(tmp[0] | (uint32_t)tmp[1] << 16, tmp[2] | (uint32_t)tmp[3] << 16,
                                tmp[4] | (uint32_t)tmp[5] << 16, tmp[6] | (uint32_t)tmp[7] << 16);
               }
             }
-            const uint16_t vals[8] = {(uint16_t)(v.x & 0xFFFF), (uint16_t)(v.x >> 16), (uint16_t)(v.y & 0xFFFF),
-                                      (uint16_t)(v.y >> 16), (uint16_t)(v.z & 0xFFFF), (uint16_t)(v.z >> 16),
-                                      (uint16_t)(v.w & 0xFFFF), (uint16_t)(v.w >> 16)};
-#pragma unroll
-            for (int j = 0; j < 8; ++j) sU[(tq + j) * RCH + r] = vals[j];
+            uint32_t* dst = reinterpret_cast<uint32_t*>(sU + r * UP + tq);
+            dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
           }
           epi_sync();
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
-            const int pr = et + 256 * i, g = pr / RCH, r = pr % RCH;
-            if (g >= G) continue;
-            float v = __fmul_rn(ar[c][i], alpha[g]);
-            for (int tt = 0; tt < nrows; ++tt) v = fmaf(sP[g * 128 + tt], bf16f(sU[tt * RCH + r]), v);
-            ar[c][i] = v;
+            const int r = et + 256 * i;
+            if (r >= vo.rT) continue;
+            for (int tt = 0; tt < nt; ++tt) {
+              const float u = bf16f(sU[r * UP + tt]);
+              const float4 p0 = reinterpret_cast<const float4*>(sP + (ts + tt) * GMAX)[0];
+              const float4 p1 = reinterpret_cast<const float4*>(sP + (ts + tt) * GMAX)[1];
+              const float pv[GMAX] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+              for (int g = 0; g < GMAX; ++g) ar[i][g] = fmaf(pv[g], u, ar[i][g]);
+            }
           }
         }
-        // chunks this cell does not have still take the tile's rescale
-#pragma unroll
-        for (int c = 0; c < RVMAX / RCH; ++c)
-          if (c >= nchunk)
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              const int g = (et + 256 * i) / RCH;
-              if (g < G) ar[c][i] = __fmul_rn(ar[c][i], alpha[g]);
-            }
-        if (vo.b == 0)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int g = (et + 256 * i) / D;
-            if (g < G) ae[i] = __fmul_rn(ae[i], alpha[g]);
-          }
         epi_sync();   // sP, sRed and the staged values are rewritten by the next tile
       }
       if (!ok) break;
@@ -484,16 +479,23 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
         base[et * stride + 1] = l_run[et];
       }
 #pragma unroll
-      for (int c = 0; c < RVMAX / RCH; ++c)
+      for (int i = 0; i < 2; ++i) {
+        const int r = et + 256 * i;
+        if (r < a.rpv)
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int pr = et + 256 * i, g = pr / RCH, r = c * RCH + pr % RCH;
-          if (g < G && r < a.rpv) base[g * stride + 2 + r] = ar[c][i];
-        }
+          for (int g = 0; g < GMAX; ++g)
+            if (g < G) base[g * stride + 2 + r] = (r < vo.rT) ? ar[i][g] : 0.0f;
+      }
+      // the residual state's token parts, added in a fixed order
+      epi_sync();
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int pr = et + 256 * i, g = pr / D, d = pr % D;
-        if (g < G) base[g * stride + 2 + a.rpv + d] = ae[i];
+      for (int g = 0; g < GMAX; ++g) sEred[(tpart * GMAX + g) * 128 + dcol] = ae[g];
+      epi_sync();
+      for (int e2 = et; e2 < G * D; e2 += 32 * EPI_WARPS) {
+        const int g = e2 / D, d = e2 % D;
+        float v = sEred[g * 128 + d];
+        for (int tp = 1; tp < TPARTS; ++tp) v = __fadd_rn(v, sEred[(tp * GMAX + g) * 128 + d]);
+        base[g * stride + 2 + a.rpv + d] = v;
       }
     }
   }

@@ -1,3 +1,4 @@
+#include <algorithm>
 // Batched small dense fp64 linear algebra for the randomized range finder
 // (CholeskyQR and B B^T = R^{-T} (Z^T Z) R^{-1}, "A JoLT for the KV Cache",
 // Section 3.1): every kernel runs all cells at once and spreads each matrix
@@ -465,9 +466,213 @@ __global__ void __launch_bounds__(128) k_dgemm(DgemmArgs g) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// The same product with a deeper operand pipeline: 16-byte cp.async copies
+// (no register staging) into PS stages of shared memory that keep each
+// operand in its own type (fp32 or fp64; fp32 values are widened when the
+// fragments are read, which is exact), so several K steps of loads are in
+// flight while the fp64 tensor cores work. Used when every 16-byte chunk of
+// the operands' contiguous dimension is aligned (A contiguous along m or
+// along k, B along n); the register-staged kernel above covers the rest.
+// Tile, warps, fragment order and the K order of the sums are those of
+// k_dgemm, so both give the same result bit for bit.
+constexpr int PS = 4;            // pipeline stages
+template <class AT, class BT, bool AMF>
+struct DgPipe {
+  // A stage: AMF ? [DG_K][DG_T + pad] : [DG_T][DG_K + pad]; B stage: [DG_K][DG_T + pad].
+  // Row pitches of 72 (along m or n) or 20 (along k) elements put the
+  // fragment reads of a (half-)warp on distinct banks, and keep every row a
+  // whole number of 16-byte chunks.
+  static constexpr int APAD = AMF ? 8 : 4;
+  static constexpr int A_ELEMS = AMF ? DG_K * (DG_T + APAD) : DG_T * (DG_K + APAD);
+  static constexpr int BPAD = 8;
+  static constexpr int B_ELEMS = DG_K * (DG_T + BPAD);
+  static constexpr int A_BYTES = (A_ELEMS * (int)sizeof(AT) + 15) / 16 * 16;
+  static constexpr int B_BYTES = (B_ELEMS * (int)sizeof(BT) + 15) / 16 * 16;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int SMEM = PS * STAGE;
+};
+
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src, int bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <class AT, class BT, bool AMF>
+__global__ void __launch_bounds__(128) k_dgemm_pipe(DgemmArgs g) {
+  using P = DgPipe<AT, BT, AMF>;
+  extern __shared__ __align__(16) uint8_t dsm[];
+  const int cell = (int)(blockIdx.z % g.ncells), slice = (int)(blockIdx.z / g.ncells);
+  int m0, n0;
+  if (g.sym) {
+    int b = blockIdx.x, ti = 0;
+    const int nt = (g.N + DG_T - 1) / DG_T;
+    while (ti < nt && b >= nt - ti) { b -= nt - ti; ++ti; }
+    if (ti >= nt) return;
+    m0 = ti * DG_T;
+    n0 = (ti + b) * DG_T;
+  } else {
+    m0 = blockIdx.x * DG_T;
+    n0 = blockIdx.y * DG_T;
+  }
+  const int M = g.M_of ? g.M_of[cell] : g.M_fixed;
+  const int K = g.K_of ? g.K_of[cell] : g.K_fixed;
+  if (m0 >= M || n0 >= g.N) return;
+  int k_lo = 0, k_hi = K;
+  if (g.kmode == 1) k_hi = min(K, n0 + DG_T);
+  if (g.kmode == 2) k_lo = (n0 / DG_K) * DG_K;
+  if (g.ksplit > 1) {
+    const int steps = (k_hi - k_lo + DG_K - 1) / DG_K;
+    const int per = (steps + g.ksplit - 1) / g.ksplit;
+    const int s0 = k_lo + slice * per * DG_K;
+    k_hi = min(k_hi, s0 + per * DG_K);
+    k_lo = s0;
+  }
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
+  const int gq = lane >> 2, tq = lane & 3;
+  const AT* A = reinterpret_cast<const AT*>(g.A) + (int64_t)cell * g.a_cell;
+  const BT* B = reinterpret_cast<const BT*>(g.B) + (int64_t)cell * g.b_cell;
+  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(dsm);
+  constexpr int AV = 16 / (int)sizeof(AT), BV = 16 / (int)sizeof(BT);   // elements per 16-byte chunk
+  auto load_stage = [&](int st, int kb) {
+    const uint32_t sa = sbase + st * P::STAGE, sb = sa + P::A_BYTES;
+    if (AMF) {        // A(m, k) contiguous along m: chunks of AV m-values per k row
+      constexpr int CH = DG_T / AV;
+      for (int c = tid; c < DG_K * CH; c += 128) {
+        const int kk = c / CH, mm = (c % CH) * AV;
+        const int gm = m0 + mm, gk = kb + kk;
+        int valid = (gk < k_hi) ? min(AV, M - gm) : 0;
+        if (valid < 0) valid = 0;
+        const AT* src = A + (valid ? (int64_t)gk * g.a_lk + gm : 0);
+        cp16(sa + (kk * (DG_T + P::APAD) + mm) * (int)sizeof(AT), src, valid * (int)sizeof(AT));
+      }
+    } else {          // A(m, k) contiguous along k: chunks of AV k-values per m row
+      constexpr int CH = DG_K / AV;
+      for (int c = tid; c < DG_T * CH; c += 128) {
+        const int mm = c / CH, kk = (c % CH) * AV;
+        const int gm = m0 + mm, gk = kb + kk;
+        int valid = (gm < M) ? min(AV, k_hi - gk) : 0;
+        if (valid < 0) valid = 0;
+        const AT* src = A + (valid ? (int64_t)gm * g.a_lm + gk : 0);
+        cp16(sa + (mm * (DG_K + P::APAD) + kk) * (int)sizeof(AT), src, valid * (int)sizeof(AT));
+      }
+    }
+    {                 // B(k, n) contiguous along n
+      constexpr int CH = DG_T / BV;
+      for (int c = tid; c < DG_K * CH; c += 128) {
+        const int kk = c / CH, nn = (c % CH) * BV;
+        const int gn = n0 + nn, gk = kb + kk;
+        int valid = (gk < k_hi) ? min(BV, g.N - gn) : 0;
+        if (valid < 0) valid = 0;
+        const BT* src = B + (valid ? (int64_t)gk * g.b_lk + gn : 0);
+        cp16(sb + (kk * (DG_T + P::BPAD) + nn) * (int)sizeof(BT), src, valid * (int)sizeof(BT));
+      }
+    }
+  };
+  double c[4][4][2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) c[i][j][0] = c[i][j][1] = 0.0;
+  const int nsteps = (k_hi > k_lo) ? (k_hi - k_lo + DG_K - 1) / DG_K : 0;
+#pragma unroll
+  for (int st = 0; st < PS - 1; ++st) {
+    if (st < nsteps) load_stage(st, k_lo + st * DG_K);
+    cp_commit();
+  }
+  for (int it = 0; it < nsteps; ++it) {
+    cp_wait<PS - 2>();
+    __syncthreads();
+    // refill the stage consumed PS - 1 steps ago (every thread is past it)
+    const int nxt = it + PS - 1;
+    if (nxt < nsteps) load_stage(nxt % PS, k_lo + nxt * DG_K);
+    cp_commit();
+    const uint8_t* stg = dsm + (it % PS) * P::STAGE;
+    const AT* As = reinterpret_cast<const AT*>(stg);
+    const BT* Bs = reinterpret_cast<const BT*>(stg + P::A_BYTES);
+#pragma unroll
+    for (int ks = 0; ks < DG_K / 4; ++ks) {
+      double av[4], bv[4];
+      const int kk = ks * 4 + tq;
+#pragma unroll
+      for (int f = 0; f < 4; ++f) {
+        const int mm = wm + f * 8 + gq, nn = wn + f * 8 + gq;
+        av[f] = AMF ? (double)As[kk * (DG_T + P::APAD) + mm] : (double)As[mm * (DG_K + P::APAD) + kk];
+        bv[f] = (double)Bs[kk * (DG_T + P::BPAD) + nn];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dmma(c[i][j][0], c[i][j][1], av[i], bv[j]);
+    }
+  }
+  cp_wait<0>();
+  __syncthreads();
+  double* Ts = reinterpret_cast<double*>(dsm);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int v = 0; v < 2; ++v) Ts[(wm + i * 8 + gq) * (DG_T + 1) + wn + j * 8 + 2 * tq + v] = c[i][j][v];
+  __syncthreads();
+  double* c64 = g.C64 ? g.C64 + (int64_t)slice * g.part_stride : nullptr;
+  auto store = [&](int r, int q, double v) {
+    if (c64) c64[(int64_t)cell * g.c_cell + (int64_t)r * g.c_lm + (int64_t)q * g.c_ln] = v;
+    if (g.C16) g.C16[(int64_t)cell * g.h_cell + (int64_t)r * g.h_lm + (int64_t)q * g.h_ln] = bf16_bits_from_f64(v);
+  };
+  const bool m_fast = (g.C64 ? g.c_lm : g.h_lm) == 1;
+  for (int e = tid; e < DG_T * DG_T; e += 128) {
+    int mm, nn;
+    if (m_fast) { nn = e / DG_T; mm = e % DG_T; } else { mm = e / DG_T; nn = e % DG_T; }
+    const int r = m0 + mm, q = n0 + nn;
+    if (r >= M || q >= g.N) continue;
+    const double v = Ts[mm * (DG_T + 1) + nn];
+    store(r, q, v);
+    if (g.sym && r != q) store(q, r, v);
+  }
+}
+
+template <class AT, class BT, bool AMF>
+static jolt_status launch_pipe(const DgemmArgs& g, dim3 grid, cudaStream_t s) {
+  using P = DgPipe<AT, BT, AMF>;
+  const int smem = std::max(P::SMEM, DG_T * (DG_T + 1) * 8);
+  static bool attr = false;
+  if (!attr) {
+    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_dgemm_pipe<AT, BT, AMF>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    attr = true;
+  }
+  k_dgemm_pipe<AT, BT, AMF><<<grid, 128, smem, s>>>(g);
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
 static jolt_status launch_dgemm(DgemmArgs g, int M_max, int ncells, cudaStream_t s) {
   if (M_max <= 0 || g.N <= 0 || ncells <= 0) return JOLT_OK;
   if (g.ksplit < 1) g.ksplit = 1;
+  {
+    // the pipelined kernel needs 16-byte chunks along A's and B's contiguous
+    // dimensions: unit strides there, and bases and other strides that are
+    // whole 16-byte multiples
+    const int ea = g.a64 ? 8 : 4, eb = g.b64 ? 8 : 4;
+    const bool amf = g.a_lm == 1, akf = g.a_lk == 1;
+    const int64_t a_other = amf ? g.a_lk : g.a_lm;
+    const bool a_ok = (amf || akf) && ((a_other * ea) % 16 == 0) && ((g.a_cell * ea) % 16 == 0) &&
+                      (reinterpret_cast<uintptr_t>(g.A) % 16 == 0);
+    const bool b_ok = g.b_ln == 1 && ((g.b_lk * eb) % 16 == 0) && ((g.b_cell * eb) % 16 == 0) &&
+                      (reinterpret_cast<uintptr_t>(g.B) % 16 == 0);
+    if (a_ok && b_ok) {
+      g.ncells = ncells;
+      const int mt = (M_max + DG_T - 1) / DG_T, nt = (g.N + DG_T - 1) / DG_T;
+      dim3 grid = g.sym ? dim3(nt * (nt + 1) / 2, 1, ncells * g.ksplit) : dim3(mt, nt, ncells * g.ksplit);
+      if (!g.a64 && !g.b64) return amf ? launch_pipe<float, float, true>(g, grid, s) : launch_pipe<float, float, false>(g, grid, s);
+      if (!g.a64 && g.b64) return amf ? launch_pipe<float, double, true>(g, grid, s) : launch_pipe<float, double, false>(g, grid, s);
+      if (g.a64 && g.b64) return amf ? launch_pipe<double, double, true>(g, grid, s) : launch_pipe<double, double, false>(g, grid, s);
+    }
+  }
   g.ncells = ncells;
   const int mt = (M_max + DG_T - 1) / DG_T, nt = (g.N + DG_T - 1) / DG_T;
   dim3 grid = g.sym ? dim3(nt * (nt + 1) / 2, 1, ncells * g.ksplit) : dim3(mt, nt, ncells * g.ksplit);
