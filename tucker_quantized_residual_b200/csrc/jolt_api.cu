@@ -1544,12 +1544,10 @@ extern "C" jolt_status jolt_decode_attention(const jolt_handle_t* hc, int32_t la
     const int rpk = (rk + 63) / 64 * 64, rpv = (rv + 63) / 64 * 64;
     const int64_t part_len = (int64_t)Bc * H * 64 * G * (2 + rpv + D);
     Arena A;
-    CellOut* dko = nullptr; CellOut* dvo = nullptr; uint16_t* mtk = nullptr; float* mv = nullptr; float* part = nullptr;
+    uint16_t* mtk = nullptr; float* mv = nullptr; float* part = nullptr;
     void* blk = nullptr;
     for (int pass = 0; pass < 2; ++pass) {
       A.used = 0;
-      dko = A.take<CellOut>(Bc);
-      dvo = A.take<CellOut>(Bc);
       mtk = A.take<uint16_t>((size_t)Bc * H * D * rpk);
       mv = A.take<float>((size_t)Bc * H * rpv * D);
       part = A.take<float>((size_t)part_len);
@@ -1560,10 +1558,12 @@ extern "C" jolt_status jolt_decode_attention(const jolt_handle_t* hc, int32_t la
       }
     }
     auto run = [&]() -> jolt_status {
-      JOLT_CUDA_TRY(cudaMemcpyAsync(dko, ko.data(), Bc * sizeof(CellOut), cudaMemcpyHostToDevice, s));
-      JOLT_CUDA_TRY(cudaMemcpyAsync(dvo, vo.data(), Bc * sizeof(CellOut), cudaMemcpyHostToDevice, s));
+      // the handle's own cell records, read in place: sequence b's cells of
+      // group g are 2 * n_groups records apart
       c.B = Bc; c.H = H; c.D = D; c.T = p->T; c.G = G; c.gq = p->G; c.li = li;
-      c.kout = dko; c.vout = dvo;
+      c.kout = h->d_out + ((int64_t)b0 * L.n_groups + g) * 2;
+      c.vout = c.kout + 1;
+      c.cstride = 2 * L.n_groups;
       c.cs = (L.rope_theta_k > 0) ? p->d_cs : nullptr;
       c.seed = h->seed + (uint64_t)b0;
       c.q = q + (int64_t)b0 * n_q_heads * D;

@@ -60,8 +60,9 @@ struct Maps {
 
 struct Args {
   int B, H, T, G, gq, li, nsplit, per;     // per: tokens per split (multiple of 128)
-  const CellOut* kout;     // [B] key cells of this layer's group
-  const CellOut* vout;     // [B] value cells
+  const CellOut* kout;     // key cell of this layer's group for sequence 0; sequence b at b * cstride
+  const CellOut* vout;     // value cells, same stride
+  int cstride;
   const float2* cs;        // RoPE table (keys), or null
   uint64_t seed;           // rotation seed of sequence 0 (sequence b: seed + b)
   const float* q;          // [B][H*G][D]
@@ -149,7 +150,7 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
       for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
         int b, h, s;
         item_of(a, it, b, h, s);
-        const CellOut ok_ = a.kout[b];
+        const CellOut ok_ = a.kout[b * a.cstride];
         const int tb = s * a.per, te = min(a.T, tb + a.per);
         const int nk = (ok_.rT + 63) / 64;
         for (int t0 = tb; t0 < te && ok; t0 += SBM) {
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
       for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
         int b, h, s;
         item_of(a, it, b, h, s);
-        const int rT = a.kout[b].rT;
+        const int rT = a.kout[b * a.cstride].rT;
         const int tb = s * a.per, te = min(a.T, tb + a.per);
         const int nk = (rT + 63) / 64;
         for (int t0 = tb; t0 < te && ok; t0 += SBM) {
@@ -239,7 +240,7 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
     for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
       int b, h, s;
       item_of(a, it, b, h, s);
-      const CellOut ko = a.kout[b], vo = a.vout[b];
+      const CellOut ko = a.kout[b * a.cstride], vo = a.vout[b * a.cstride];
       const int tb = s * a.per, te = min(a.T, tb + a.per);
       // queries of this KV head and the sequence's rotation signs
       epi_sync();
@@ -431,12 +432,15 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
             for (int g = 0; g < GMAX; ++g) ae[g] = fmaf(pv[g], dq, ae[g]);
           }
         }
-        // ---- rank-space values: TSUB tokens of U_T^V at a time, all ranks
-        for (int ts = 0; ts < nrows; ts += TSUB) {
+        // ---- rank-space values: all ranks, the whole tile at once when they
+        // fit the staging buffer, else TSUB tokens at a time
+        const int tsub = (vo.rT * (SBM + 2) <= RVMAX * UP) ? SBM : TSUB;
+        const int up = tsub + 2;     // odd word pitch: rank rows on distinct banks
+        for (int ts = 0; ts < nrows; ts += tsub) {
           epi_sync();   // the previous slice's readers are done with sU
-          const int nt = min(TSUB, nrows - ts);
-          for (int w = et; w < vo.rT * (TSUB / 8); w += 32 * EPI_WARPS) {
-            const int r = w / (TSUB / 8), tq = (w % (TSUB / 8)) * 8;
+          const int nt = min(tsub, nrows - ts);
+          for (int w = et; w < vo.rT * (tsub / 8); w += 32 * EPI_WARPS) {
+            const int r = w / (tsub / 8), tq = (w % (tsub / 8)) * 8;
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
             if (tq < nt) {
               const uint16_t* src = vo.ut + (int64_t)r * vo.t_pitch + t0 + ts + tq;
@@ -450,7 +454,7 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
                                tmp[4] | (uint32_t)tmp[5] << 16, tmp[6] | (uint32_t)tmp[7] << 16);
               }
             }
-            uint32_t* dst = reinterpret_cast<uint32_t*>(sU + r * UP + tq);
+            uint32_t* dst = reinterpret_cast<uint32_t*>(sU + r * up + tq);
             dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
           }
           epi_sync();
@@ -459,7 +463,7 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
             const int r = et + 256 * i;
             if (r >= vo.rT) continue;
             for (int tt = 0; tt < nt; ++tt) {
-              const float u = bf16f(sU[r * UP + tt]);
+              const float u = bf16f(sU[r * up + tt]);
               const float4 p0 = reinterpret_cast<const float4*>(sP + (ts + tt) * GMAX)[0];
               const float4 p1 = reinterpret_cast<const float4*>(sP + (ts + tt) * GMAX)[1];
               const float pv[GMAX] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
@@ -513,10 +517,10 @@ __global__ void __launch_bounds__(STHREADS, 1) k_dec_attn(const __grid_constant_
 // summed in fp64 and rounded once, as decompression forms M^.
 template <int D>
 __global__ void __launch_bounds__(D) k_dec_m(const CellOut* __restrict__ kout, const CellOut* __restrict__ vout,
-                                             int H, int li, uint16_t* __restrict__ mtk, int rpk,
+                                             int cstride, int H, int li, uint16_t* __restrict__ mtk, int rpk,
                                              float* __restrict__ mv, int rpv) {
   const int r = blockIdx.x, h = blockIdx.y, b = blockIdx.z >> 1, kind = blockIdx.z & 1;
-  const CellOut o = kind == 0 ? kout[b] : vout[b];
+  const CellOut o = kind == 0 ? kout[b * cstride] : vout[b * cstride];
   const int rp = kind == 0 ? rpk : rpv;
   if (r >= rp) return;
   const int d = threadIdx.x;
@@ -539,7 +543,7 @@ __global__ void __launch_bounds__(128) k_dec_merge(Args a, const CellOut* __rest
                                                    const float* __restrict__ mv, const uint16_t* __restrict__ tk,
                                                    const uint16_t* __restrict__ tv, int ntail, float* __restrict__ out) {
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const CellOut vo = vout[b];
+  const CellOut vo = vout[b * a.cstride];
   const int stride = 2 + a.rpv + D, G = a.G;
   __shared__ float sq[D], sres[D], srank[RVMAX], sw[64], stl[1024];
   __shared__ float sred[4];
@@ -645,12 +649,12 @@ jolt_status launch_decode_attention(const DecodeCall& c, cudaStream_t s) {
   if (nsplit > 64) { set_error("decode attention: %d splits exceed 64", nsplit); return JOLT_ERR_UNSUPPORTED_SHAPE; }
   dec::Args a{};
   a.B = B; a.H = H; a.T = T; a.G = G; a.gq = c.gq; a.li = c.li; a.nsplit = nsplit; a.per = per;
-  a.kout = c.kout; a.vout = c.vout; a.cs = c.cs; a.seed = c.seed; a.q = c.q; a.part = c.part; a.rpv = c.rpv;
+  a.kout = c.kout; a.vout = c.vout; a.cstride = c.cstride; a.cs = c.cs; a.seed = c.seed; a.q = c.q; a.part = c.part; a.rpv = c.rpv;
   a.status = c.status;
   if ((int64_t)B * H * nsplit * G * (2 + c.rpv + D) > c.part_len) { set_error("decode attention: state buffer too small"); return JOLT_ERR_CUDA; }
   dim3 gm(std::max(c.rpk, c.rpv), H, 2 * B);
-  if (D == 128) k_dec_m<128><<<gm, 128, 0, s>>>(c.kout, c.vout, H, c.li, c.mtk, c.rpk, c.mv, c.rpv);
-  else k_dec_m<64><<<gm, 64, 0, s>>>(c.kout, c.vout, H, c.li, c.mtk, c.rpk, c.mv, c.rpv);
+  if (D == 128) k_dec_m<128><<<gm, 128, 0, s>>>(c.kout, c.vout, c.cstride, H, c.li, c.mtk, c.rpk, c.mv, c.rpv);
+  else k_dec_m<64><<<gm, 64, 0, s>>>(c.kout, c.vout, c.cstride, H, c.li, c.mtk, c.rpk, c.mv, c.rpv);
   JOLT_LAUNCHED();
   dec::Maps m;
   JOLT_TRY(map_3d_box(&m.mt, c.mtk, B * H, D, c.rpk, c.rpk, 64, D));

@@ -244,8 +244,9 @@ jolt_status launch_rope_tiled(const float2* cs, int T, int D, float4* csq, cudaS
 constexpr int DEC_BMAX = 16;      // sequences per launch
 struct DecodeCall {
   int B, H, D, T, G, gq, li;      // G query heads per KV head, li = layer within its group
-  const CellOut* kout;            // [B] key cells (device)
-  const CellOut* vout;            // [B] value cells (device)
+  const CellOut* kout;            // key cell of sequence 0 (device); sequence b at b * cstride
+  const CellOut* vout;            // value cells, same stride
+  int cstride;
   const float2* cs;               // RoPE table of the keys, or null
   uint64_t seed;                  // rotation seed of sequence 0
   const float* q;                 // [B][H*G][D]
