@@ -176,6 +176,11 @@ struct jolt_plan_s {
   // GEMM tile width BN, padded extents, working buffers
   int k = 0, BN = 0, nt_k = 0, kpad = 0, rpad = 0, tp = 0, Ncmax = 0, fg_chunks = 0, fg_spc = 0, q_used = 0;
   int gemm_pair = 0;        // X W / X^T Y on CTA pairs (tcgen05 cta_group::2)
+  // k > 256 on CTA pairs: N tiles up to 512 wide (one TMEM accumulator, two
+  // MMAs per K step), so X is streamed ceil(k/512) times per pass instead of
+  // ceil(k/256); B boxes of two heights hb[0], hb[1]
+  int wide = 0, wide_nt = 0, wide_w0 = 0;
+  int wtn0[4] = {}, wta[4] = {}, wtb[4] = {}, wmap_a[4] = {}, wmap_b[4] = {}, whb[2] = {};
   // tensor-core residual/decode streams: U_T^ rows and M^T, padded to 64 ranks
   bool tc_in = false;
   int rows_u = 0, rpad_m = 0;
@@ -442,6 +447,30 @@ jolt_status jolt_plan(const jolt_layout* L, int64_t byte_budget, const jolt_opti
     p->nt_k = (p->k + p->BN - 1) / p->BN;
     p->kpad = (p->k + 63) / 64 * 64;
     p->gemm_pair = (p->BN / 2) % 8 == 0;   // BN is a multiple of 16, so always
+    if (p->gemm_pair && p->k > 256 && p->k <= 2048) {
+      const int nt = (p->k + 511) / 512;
+      const int w0 = ((p->k + nt - 1) / nt + 15) / 16 * 16;
+      int nh = 0;
+      bool ok = true;
+      for (int j = 0; j < nt && ok; ++j) {
+        const int n0 = j * w0, w = std::min(w0, p->k - n0);
+        const int a = ((w + 1) / 2 + 15) / 16 * 16, b = w - a;
+        if (a < 16 || b < 16 || a > 256 || b > 256) { ok = false; break; }
+        p->wtn0[j] = n0; p->wta[j] = a; p->wtb[j] = b;
+        int* sel[2] = {&p->wmap_a[j], &p->wmap_b[j]};
+        const int hh[2] = {a / 2, b / 2};
+        for (int t = 0; t < 2 && ok; ++t) {
+          int f = -1;
+          for (int u = 0; u < nh; ++u) if (p->whb[u] == hh[t]) f = u;
+          if (f < 0) { if (nh == 2) { ok = false; break; } p->whb[nh] = hh[t]; f = nh++; }
+          *sel[t] = f;
+        }
+      }
+      if (ok) {
+        if (nh == 1) p->whb[1] = p->whb[0];
+        p->wide = 1; p->wide_nt = nt; p->wide_w0 = w0;
+      }
+    }
     p->rpad = (p->rmax_all + 127) / 128 * 128;
     p->tp = (p->T + 7) / 8 * 8;
     const int steps = ((p->Ncmax + 127) / 128) * ((p->T + 63) / 64);
@@ -803,22 +832,37 @@ static jolt_status run_range_finder(jolt_plan_s* p, const void* k_in, const void
   }
   // W_0^T = Omega^T
   JOLT_TRY(launch_omega(p->Wt, nc, k, p->Ncmax, p->d_Nc, p->d_cb, p->d_cis, seed, s));
+  // B operand maps and N tiling of the pair passes (wide tiles when planned)
+  auto pair_tiles = [&](umma::Maps& mm, umma::Problem& q, const void* bt, int cols, int64_t pitch,
+                        bool wide) -> jolt_status {
+    q.pair = p->gemm_pair;
+    if (!wide) {
+      q.BN = p->BN; q.nt = p->nt_k;
+      return map_3d(&mm.bt, bt, nc, k, cols, pitch, p->gemm_pair ? p->BN / 2 : p->BN);
+    }
+    q.wide = 1; q.BN = p->wide_w0; q.nt = p->wide_nt;
+    for (int j = 0; j < p->wide_nt; ++j) {
+      q.tn0[j] = p->wtn0[j]; q.ta[j] = p->wta[j]; q.tb[j] = p->wtb[j];
+      q.tmap_a[j] = p->wmap_a[j]; q.tmap_b[j] = p->wmap_b[j];
+    }
+    JOLT_TRY(map_3d(&mm.bt, bt, nc, k, cols, pitch, p->whb[0]));
+    return map_3d(&mm.bt2, bt, nc, k, cols, pitch, p->whb[1]);
+  };
   auto xw = [&]() -> jolt_status {
     ProfScope ps(JOLT_STAGE_GEMM_XW, s);
     umma::Maps mm = m;
-    JOLT_TRY(map_3d(&mm.bt, p->Wt, nc, k, p->Ncmax, p->Ncmax, p->gemm_pair ? p->BN / 2 : p->BN));
     umma::Problem q = gemm_problem(p, umma::XW, status);
-    q.M = T; q.N = k; q.BN = p->BN; q.mt = (T + 127) / 128; q.nt = p->nt_k; q.pair = p->gemm_pair;
+    JOLT_TRY(pair_tiles(mm, q, p->Wt, p->Ncmax, p->Ncmax, p->wide != 0));
+    q.M = T; q.N = k; q.mt = (T + 127) / 128;
     q.out_bf16 = p->Yt; q.out_cell_stride = (int64_t)k * p->tp;
     return launch_umma(mm, q, s);
   };
   auto xty = [&]() -> jolt_status {
     ProfScope ps(JOLT_STAGE_GEMM_XTY, s);
     umma::Maps mm = m;
-    JOLT_TRY(map_3d(&mm.bt, p->Yt, nc, k, T, p->tp, p->gemm_pair ? p->BN / 2 : p->BN));
     umma::Problem q = gemm_problem(p, umma::XTY, status);
-    q.M = p->Ncmax; q.N = k; q.Kdim = T; q.BN = p->BN; q.mt = (p->Ncmax + 127) / 128; q.nt = p->nt_k;
-    q.pair = p->gemm_pair;
+    JOLT_TRY(pair_tiles(mm, q, p->Yt, T, p->tp, p->wide != 0));
+    q.M = p->Ncmax; q.N = k; q.Kdim = T; q.mt = (p->Ncmax + 127) / 128;
     q.out_f32 = p->Z; q.out_cell_stride = (int64_t)p->Ncmax * k;
     return launch_umma(mm, q, s);
   };

@@ -97,7 +97,17 @@ static int num_sms() {
 jolt_status launch_umma(const umma::Maps& maps, const umma::Problem& p, cudaStream_t s) {
   const int ntiles = p.ncells * p.mt * p.nt;
   if (ntiles == 0) return JOLT_OK;
-  if (p.BN % 16 || p.BN < 16 || p.BN > umma::BN_MAX) { set_error("bad GEMM tile width %d", p.BN); return JOLT_ERR_INVALID_ARG; }
+  const int bn_max = (p.pair && p.wide) ? 2 * umma::BN_MAX : umma::BN_MAX;
+  if (p.BN % 16 || p.BN < 16 || p.BN > bn_max) { set_error("bad GEMM tile width %d", p.BN); return JOLT_ERR_INVALID_ARG; }
+  if (p.wide) {
+    // wide tiles: CTA pairs only, at most 4 N tiles, each two MMAs 16..256
+    // wide (multiples of 16) that together fit the widest tile
+    bool ok = p.pair && p.nt >= 1 && p.nt <= 4;
+    for (int j = 0; ok && j < p.nt; ++j)
+      ok = p.ta[j] % 16 == 0 && p.tb[j] % 16 == 0 && p.ta[j] >= 16 && p.tb[j] >= 16 && p.ta[j] <= umma::BN_MAX &&
+           p.tb[j] <= umma::BN_MAX && p.ta[j] + p.tb[j] <= p.BN && p.tn0[j] + p.ta[j] + p.tb[j] <= p.N;
+    if (!ok) { set_error("bad wide GEMM tiling"); return JOLT_ERR_INVALID_ARG; }
+  }
   static bool attr = false;
   if (!attr) {
     JOLT_CUDA_TRY(cudaFuncSetAttribute(umma::k_umma_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,

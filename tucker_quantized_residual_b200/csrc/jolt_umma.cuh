@@ -74,6 +74,14 @@ struct Problem {
   uint16_t* const* wp_dst;   // WP: per-cell U^T base, row pitch t_pitch
   int* status;
   int pair;              // 1: CTA pairs (tcgen05 cta_group::2), M = 256 per pair; XW and XTY only
+  // pair mode, N tiles wider than 256: one TMEM accumulator of up to 512
+  // columns and two MMAs per 16-wide K step. N tile j covers the columns
+  // [tn0[j], tn0[j] + ta[j] + tb[j]); its MMAs are ta[j] and tb[j] wide, and
+  // each CTA loads half of each one's B rows with maps.bt (tmap 0) or
+  // maps.bt2 (tmap 1), whose boxes are that many rows high. BN is the widest
+  // tile (it sizes the pipeline stages).
+  int wide;
+  int tn0[4], ta[4], tb[4], tmap_a[4], tmap_b[4];
 };
 
 struct Maps {
@@ -81,6 +89,7 @@ struct Maps {
   CUtensorMap xv;     // X of values
   CUtensorMap bt;     // XW: W^T [cells][k][N_c]; XTY/GRAM: Y^T [cells][k][T]; WP: P^T [cells][r][k]; box {64, BN}
   CUtensorMap at;     // GRAM: Y^T, box {64, 128}; WP: Y^T read along t, box {64, 64}
+  CUtensorMap bt2;    // wide pair tiles: the second B box height (same tensor as bt)
   // pair mode: bt's box is {64, BN/2}, each CTA of a pair loads its half of the N columns
 };
 
@@ -585,7 +594,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm_pair(const __grid_cons
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
-  const int ncols = (2 * p.BN <= 64) ? 64 : (2 * p.BN <= 128) ? 128 : (2 * p.BN <= 256) ? 256 : 512;
+  // two accumulators (the epilogue of one tile overlaps the next tile's main
+  // loop) while they fit in TMEM's 512 columns; wide tiles have one
+  const int nacc = p.wide ? 1 : 2;
+  const int ncols = p.wide ? 512 : (2 * p.BN <= 64) ? 64 : (2 * p.BN <= 128) ? 128 : (2 * p.BN <= 256) ? 256 : 512;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
@@ -617,12 +629,19 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm_pair(const __grid_cons
       bool issued[MAX_STAGES];
       for (int s = 0; s < MAX_STAGES; ++s) issued[s] = false;
       bool ok = true;
-      const uint32_t stage_tx = 2u * (uint32_t)(A_BYTES + BNH * BK * 2);
       for (int tile = pair_id; tile < ntiles && ok; tile += npairs) {
         const int cell = tile / (mt2 * p.nt);
         const int r = tile - cell * (mt2 * p.nt);
         const int m0 = (r / p.nt) * (2 * BM) + (int)rank * BM;
-        const int n0 = (r % p.nt) * p.BN + (int)rank * BNH;
+        const int j = r % p.nt;
+        // B rows of this CTA: one box of BN/2 rows, or (wide) one box per MMA
+        const int n0 = p.wide ? p.tn0[j] + (int)rank * (p.ta[j] / 2) : j * p.BN + (int)rank * BNH;
+        const int n1 = p.wide ? p.tn0[j] + p.ta[j] + (int)rank * (p.tb[j] / 2) : 0;
+        const CUtensorMap* bma = (p.wide && p.tmap_a[j]) ? &maps.bt2 : &maps.bt;
+        const CUtensorMap* bmb = (p.wide && p.tmap_b[j]) ? &maps.bt2 : &maps.bt;
+        const uint32_t sb1 = p.wide ? (uint32_t)(p.ta[j] / 2) * (BK * 2) : 0u;
+        const uint32_t stage_tx =
+            2u * (uint32_t)(A_BYTES + (p.wide ? (p.ta[j] + p.tb[j]) / 2 : BNH) * BK * 2);
         const int Kc = (p.mode == XW) ? p.cell_Lg[cell] * p.H * p.D : p.Kdim;
         const int nkb = (Kc + BK - 1) / BK;
         const CUtensorMap* xm = (p.cell_kind[cell] == 0) ? &maps.xk : &maps.xv;
@@ -645,7 +664,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm_pair(const __grid_cons
               tma2_load_5d(sa + 8192 * half, xm, fb, d0, k0, lh % p.H, l0 + lh / p.H, b);
             }
           }
-          tma2_load_3d(sb, &maps.bt, fb, k0, n0, cell);
+          tma2_load_3d(sb, bma, fb, k0, n0, cell);
+          if (p.wide) tma2_load_3d(sb + sb1, bmb, fb, k0, n1, cell);
           issued[stage] = true;
           issued_phase[stage] = ph;
           if (++stage == STAGES) { stage = 0; ph ^= 1; }
@@ -668,13 +688,22 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm_pair(const __grid_cons
       int acc = 0;
       uint32_t aph[2] = {0, 0};
       const int a_mn = (p.mode == XTY) ? 1 : 0;
-      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) |
-                             ((uint32_t)(p.BN >> 3) << 17) | ((uint32_t)((2 * BM) >> 4) << 24);
+      auto idesc_n = [&](int n) {
+        return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)(n >> 3) << 17) |
+               ((uint32_t)((2 * BM) >> 4) << 24);
+      };
       bool ok = true;
       for (int tile = pair_id; tile < ntiles && ok; tile += npairs) {
         const int cell = tile / (mt2 * p.nt);
+        const int j = (tile - cell * (mt2 * p.nt)) % p.nt;
         const int Kc = (p.mode == XW) ? p.cell_Lg[cell] * p.H * p.D : p.Kdim;
         const int nkb = (Kc + BK - 1) / BK;
+        // one MMA BN wide, or (wide) two: ta[j] columns, then tb[j] columns
+        // whose B rows follow the first MMA's in shared memory
+        const int na = p.wide ? p.ta[j] : p.BN;
+        const uint32_t idesc = idesc_n(na);
+        const uint32_t idesc1 = p.wide ? idesc_n(p.tb[j]) : 0u;
+        const uint32_t sb1 = p.wide ? (uint32_t)(p.ta[j] / 2) * (BK * 2) : 0u;
         if (!mbar_wait(tempty_bar(acc), aph[acc] ^ 1, abort_flag, p.status)) break;
         fence_after();
         const uint32_t dcol = tmem + (uint32_t)(acc * p.BN);
@@ -686,7 +715,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm_pair(const __grid_cons
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t da = a_mn ? sdesc(sa + kk * 2048, 8192, 1024) : sdesc(sa + kk * 32, 16, 1024);
             const uint64_t db = sdesc(sb + kk * 32, 16, 1024);
-            mma2_bf16(dcol, da, db, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            mma2_bf16(dcol, da, db, idesc, accum);
+            if (p.wide) mma2_bf16(dcol + (uint32_t)na, da, sdesc(sb + sb1 + kk * 32, 16, 1024), idesc1, accum);
           }
           mma2_commit_both(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; ph ^= 1; }
@@ -694,7 +725,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm_pair(const __grid_cons
         if (!ok) break;
         mma2_commit_both(tfull_bar(acc));
         aph[acc] ^= 1;
-        acc ^= 1;
+        if (nacc == 2) acc ^= 1;
       }
       if (!ok) *abort_flag = 1;
     }
@@ -707,13 +738,15 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm_pair(const __grid_cons
       const int cell = tile / (mt2 * p.nt);
       const int r = tile - cell * (mt2 * p.nt);
       const int m0 = (r / p.nt) * (2 * BM) + (int)rank * BM;
-      const int n0 = (r % p.nt) * p.BN;
+      const int j = r % p.nt;
+      const int n0 = p.wide ? p.tn0[j] : j * p.BN;
+      const int wn = p.wide ? p.ta[j] + p.tb[j] : p.BN;
       const int Mc = (p.mode == XTY) ? p.cell_Lg[cell] * p.H * p.D : p.M;
       if (!mbar_wait(tfull_bar(acc), aph[acc], abort_flag, p.status)) break;
       fence_after();
       const int row = m0 + q * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.BN);
-      for (int c0 = 0; c0 < p.BN; c0 += 16) {
+      for (int c0 = 0; c0 < wn; c0 += 16) {
         float v[16];
         tmem_ld16(tbase + c0, v);
         const int n = n0 + c0;
@@ -737,7 +770,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_umma_gemm_pair(const __grid_cons
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_to_rank(tempty_bar(acc), 0));
       aph[acc] ^= 1;
-      acc ^= 1;
+      if (nacc == 2) acc ^= 1;
     }
   }
   fence_before();
