@@ -498,6 +498,259 @@ __global__ void __launch_bounds__(EIG_THREADS) k_tridiag_multi(const EighJob* __
   }
 }
 
+// ------------------------------------------ cluster tridiagonalization --
+// The same Householder reduction with the matrix held in the shared memory of
+// a cluster of CS CTAs (distributed shared memory) instead of L2: row r of the
+// lower triangle (entries 0..r) lives in CTA r mod CS, so each column costs
+// two cluster barriers and three rounds of remote shared-memory reads, and the
+// symmetric matrix-vector product and the rank-2 update read and write shared
+// memory only. Per column k (trailing indices k+1..n-1):
+//   every CTA forms v, beta from the gathered column x (redundantly, bit-
+//   identically); A: y1 = the row part of A v for its rows (entries j <= i),
+//   y2 = its rows' contribution to the column part (entries i > j) for every
+//   j, and a copy of its rows' column k+1; barrier; B: the owner of j sums
+//   p_j = beta (y1_j + sum over CTAs of y2_j), every CTA gathers column k+1;
+//   barrier; C: every CTA gathers p, forms w = p - (beta p.v / 2) v, updates
+//   its rows and, from the gathered column, the next x (the same operations
+//   as the owner's update of those entries).
+// A warp works on up to four of its rows at once (one pass over j for all
+// four), so the shared-memory loads of a pass are independent.
+// Outputs as k_tridiag: d, e, beta in work, reflector k in row k of A.
+constexpr int TC_THREADS = 512;
+constexpr size_t TC_SMEM_MAX = 227 * 1024;
+
+__device__ __forceinline__ uint32_t tc_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// generic address of the same shared-memory location in CTA `rank` of the
+// cluster (plain loads through it read that CTA's shared memory)
+__device__ __forceinline__ const double* tc_peer(const double* local, uint32_t rank) {
+  uint64_t a;
+  asm("mapa.u64 %0, %1, %2;" : "=l"(a) : "l"(reinterpret_cast<uint64_t>(local)), "r"(rank));
+  return reinterpret_cast<const double*>(a);
+}
+// every thread of every CTA of the cluster; writes before it are visible to
+// the cluster's reads after it
+__device__ __forceinline__ void tc_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// packed offset of owned row lr (global row rank + CS lr, rank + 1 + CS lr entries)
+template <int CS>
+__host__ __device__ inline int tc_off(int lr, int rank) { return lr * (rank + 1) + CS * (lr * (lr - 1) / 2); }
+template <int CS>
+__host__ __device__ inline size_t tc_lsize(int n) {
+  const size_t nmx = (n + CS - 1) / CS;
+  return nmx * CS + CS * nmx * (nmx - 1) / 2;
+}
+template <int CS>
+__host__ __device__ inline size_t tc_smem_bytes(int n) {
+  return (tc_lsize<CS>(n) + 8 * (size_t)n + 2 * (size_t)((n + CS - 1) / CS) + 32) * sizeof(double);
+}
+
+template <int CS>
+__global__ void __launch_bounds__(TC_THREADS, 1) k_tridiag_cl(const EighJob* __restrict__ jobs, int nmax) {
+  const int job = blockIdx.x / CS;
+  const int rank = (int)tc_rank();
+  const EighJob J = jobs[job];
+  const int n = J.n;              // the same for the whole cluster: every CTA returns, or none
+  if (n <= 0) return;
+  extern __shared__ double sh[];
+  // the layout depends on nmax only, so it is the same in every CTA
+  const int nmx = (nmax + CS - 1) / CS;
+  double* L = sh;                           // owned rows, packed
+  double* vv = L + tc_lsize<CS>(nmax);      // v (absolute indices)
+  double* ww = vv + nmax;                   // gathered p, then w
+  double* xx = ww + nmax;                   // x = current column below the diagonal; xx[k+1] diagonal
+  double* yp = xx + nmax;                   // this CTA's y2 (read remotely)
+  double* xs = yp + nmax;                   // this CTA's rows' column k+1 (read remotely)
+  double* pb = xs + nmax;                   // p_j of this CTA's j (read remotely)
+  double* y1 = pb + nmax;                   // row part of A v, owned rows
+  int* roff = reinterpret_cast<int*>(y1 + nmx);   // packed offset of each owned row
+  double* red = y1 + 2 * nmx;
+  double* se = red + 32;                    // e and beta of every column, written out at the end
+  double* st = se + nmax;
+  double* A = J.A;
+  double* dd = J.work;
+  double* ee = dd + n;
+  double* tau = ee + n;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5, nwarp = nt >> 5;
+  const int nown = rank < n ? (n - rank + CS - 1) / CS : 0;
+  for (int lr = tid; lr < nown; lr += nt) roff[lr] = tc_off<CS>(lr, rank);
+  // load the owned rows (lower part) and the first column (row 0 by symmetry)
+  for (int lr = warp; lr < nown; lr += nwarp) {
+    const int r = rank + CS * lr;
+    double* dst = L + tc_off<CS>(lr, rank);
+    for (int j = lane; j <= r; j += 32) dst[j] = __ldcg(A + (int64_t)r * n + j);
+  }
+  double sq = 0.0;
+  for (int r = tid; r < n; r += nt) {
+    const double x = __ldcg(A + r);         // xx[0] = A[0][0]
+    xx[r] = x;
+    if (r >= 2) sq += x * x;
+  }
+  tc_cluster_sync();
+  for (int k = 0; k + 2 < n; ++k) {
+    // ---- Householder vector of x = xx[k+1 .. n-1]
+    const double s = block_sum(sq, red);
+    const double x0 = xx[k + 1];
+    double beta = 0.0, alpha = x0;
+    if (s != 0.0) {
+      const double nrm = sqrt(x0 * x0 + s);
+      alpha = (x0 <= 0.0) ? nrm : -nrm;
+      const double v0 = x0 - alpha;
+      beta = 2.0 / (s + v0 * v0);
+      for (int r = k + 1 + tid; r < n; r += nt) vv[r] = (r == k + 1) ? v0 : xx[r];
+    } else {
+      // no reflection: v = 0 makes p, w and the update vanish exactly
+      for (int r = k + 1 + tid; r < n; r += nt) vv[r] = 0.0;
+    }
+    if (tid == 0) { se[k] = alpha; st[k] = beta; }
+    __syncthreads();
+    // ---- A: y1 (owned rows), y2 partials (all j), copy of column k+1
+    const int lr_lo = (k + 1 <= rank) ? 0 : (k + 1 - rank + CS - 1) / CS;   // first owned row >= k+1
+    for (int base = lr_lo + warp; base < nown; base += 4 * nwarp) {
+      int ro[4], rr[4];
+      int rmax = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int lr = base + i * nwarp;
+        rr[i] = lr < nown ? rank + CS * lr : -1;     // -1: no row (the j loop skips it)
+        ro[i] = lr < nown ? roff[lr] : 0;
+        rmax = max(rmax, rr[i]);
+      }
+      double acc[4] = {0.0, 0.0, 0.0, 0.0};
+      for (int j = k + 1 + lane; j <= rmax; j += 32) {
+        const double vj = vv[j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (j <= rr[i]) acc[i] += L[ro[i] + j] * vj;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = warp_sum(acc[i]);
+      if (lane < 4) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (i == lane && rr[i] >= 0) { y1[base + i * nwarp] = acc[i]; xs[rr[i]] = L[ro[i] + k + 1]; }
+      }
+    }
+    // column k of the owned rows is no longer read: it keeps reflector k
+    for (int lr = lr_lo + tid; lr < nown; lr += nt) L[roff[lr] + k] = vv[rank + CS * lr];
+    for (int j = k + 1 + tid; j < n; j += nt) {
+      int lr = (j < rank) ? 0 : (j - rank) / CS + 1;   // owned rows > j
+      // four partial sums (rows lr mod 4), added in a fixed order
+      double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+      for (; lr + 3 < nown; lr += 4) {
+        const int r = rank + CS * lr;
+        a0 += L[roff[lr] + j] * vv[r];
+        a1 += L[roff[lr + 1] + j] * vv[r + CS];
+        a2 += L[roff[lr + 2] + j] * vv[r + 2 * CS];
+        a3 += L[roff[lr + 3] + j] * vv[r + 3 * CS];
+      }
+      for (; lr < nown; ++lr) a0 += L[roff[lr] + j] * vv[rank + CS * lr];
+      yp[j] = (a0 + a1) + (a2 + a3);
+    }
+    tc_cluster_sync();
+    // ---- B: p_j for owned j; gather column k+1
+    for (int lr = lr_lo + tid; lr < nown; lr += nt) {
+      const int j = rank + CS * lr;
+      double part[CS];
+#pragma unroll
+      for (int c = 0; c < CS; ++c) part[c] = *tc_peer(yp + j, (uint32_t)c);
+      double acc = y1[lr];
+#pragma unroll
+      for (int c = 0; c < CS; ++c) acc += part[c];
+      pb[j] = beta * acc;
+    }
+    for (int r = k + 1 + tid; r < n; r += nt) xx[r] = *tc_peer(xs + r, (uint32_t)(r % CS));
+    tc_cluster_sync();
+    // ---- C: gather p, w = p - Kc v, update owned rows and the next column
+    double pv = 0.0;
+    for (int j = k + 1 + tid; j < n; j += nt) {
+      const double pj = *tc_peer(pb + j, (uint32_t)(j % CS));
+      ww[j] = pj;
+      pv += pj * vv[j];
+    }
+    const double Kc = 0.5 * beta * block_sum(pv, red);
+    for (int j = k + 1 + tid; j < n; j += nt) ww[j] -= Kc * vv[j];
+    __syncthreads();
+    for (int base = lr_lo + warp; base < nown; base += 4 * nwarp) {
+      int ro[4], rr[4];
+      double vi[4], wi[4];
+      int rmax = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int lr = base + i * nwarp;
+        rr[i] = lr < nown ? rank + CS * lr : -1;
+        ro[i] = lr < nown ? roff[lr] : 0;
+        vi[i] = lr < nown ? vv[rr[i]] : 0.0;
+        wi[i] = lr < nown ? ww[rr[i]] : 0.0;
+        rmax = max(rmax, rr[i]);
+      }
+      for (int j = k + 1 + lane; j <= rmax; j += 32) {
+        const double wj = ww[j], vj = vv[j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (j <= rr[i]) {
+            double* e = L + ro[i] + j;
+            *e = __dsub_rn(*e, __dadd_rn(__dmul_rn(vi[i], wj), __dmul_rn(wi[i], vj)));
+          }
+      }
+    }
+    const double vk = vv[k + 1], wk = ww[k + 1];
+    sq = 0.0;
+    for (int r = k + 1 + tid; r < n; r += nt) {
+      const double x = __dsub_rn(xx[r], __dadd_rn(__dmul_rn(vv[r], wk), __dmul_rn(ww[r], vk)));
+      xx[r] = x;
+      if (r >= k + 3) sq += x * x;       // the next column's sum of squares
+    }
+  }
+  __syncthreads();
+  // d from the owned diagonals; reflector k (column k of rows k+1..n-1) into
+  // row k of A; e and beta from CTA 0; the last two columns have no reflector
+  for (int lr = warp; lr < nown; lr += nwarp) {
+    const int r = rank + CS * lr;
+    const double* row = L + roff[lr];
+    const int kmax = min(r, n - 2);
+    for (int k = lane; k < kmax; k += 32) A[(int64_t)k * n + r] = row[k];
+    if (lane == 0) dd[r] = row[r];
+    if (lane == 0 && r == n - 1 && n >= 2) ee[n - 2] = row[n - 2];
+  }
+  if (rank == 0) {
+    for (int k = tid; k + 2 < n; k += nt) { ee[k] = se[k]; tau[k] = st[k]; }
+    if (tid == 0) {
+      if (n >= 2) tau[n - 2] = 0.0;
+      ee[n - 1] = 0.0;
+      tau[n - 1] = 0.0;
+    }
+  }
+  tc_cluster_sync();          // no CTA leaves while another may still read its shared memory
+}
+
+template <int CS>
+static jolt_status launch_tridiag_cl(const EighJob* jobs, int njobs, int nmax, cudaStream_t s) {
+  const size_t smem = tc_smem_bytes<CS>(nmax);
+  { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_tridiag_cl<CS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(njobs * CS);
+  cfg.blockDim = dim3(TC_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = CS;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int nm = nmax;
+  JOLT_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_tridiag_cl<CS>, jobs, nm));
+  JOLT_LAUNCHED();
+  return JOLT_OK;
+}
+
 // Number of eigenvalues of the tridiagonal (d, e) smaller than x.
 __device__ __forceinline__ int sturm_count(const double* d, const double* e, int n, double x, double pivmin) {
   int c = 0;
@@ -756,6 +1009,9 @@ __global__ void __launch_bounds__(256) k_backtr(const EighJob* __restrict__ jobs
 }
 
 jolt_status launch_tridiag(const EighJob* jobs, int njobs, int nmax, cudaStream_t s) {
+  if (njobs <= 0) return JOLT_OK;
+  // matrices that fit a cluster's shared memory: the cluster reduction
+  if (nmax >= 48 && tc_smem_bytes<6>(nmax) <= TC_SMEM_MAX) return launch_tridiag_cl<6>(jobs, njobs, nmax, s);
   const size_t smem = (size_t)(2 * nmax + 32) * sizeof(double);
   { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_tridiag, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
   k_tridiag<<<njobs, EIG_THREADS, smem, s>>>(jobs);
@@ -788,6 +1044,10 @@ static int tridiag_blocks_per_job(int njobs, int nmax, size_t smem) {
 jolt_status launch_tridiag_multi(const EighJob* jobs, int njobs, int nmax, double* scratch, unsigned int* counters,
                                  int* status, cudaStream_t s) {
   if (njobs <= 0) return JOLT_OK;
+  // the matrix fits the shared memory of a cluster: k_tridiag_cl, on the
+  // smallest cluster whose CTAs hold their rows (more clusters resident)
+  if (nmax >= 48 && tc_smem_bytes<6>(nmax) <= TC_SMEM_MAX) return launch_tridiag_cl<6>(jobs, njobs, nmax, s);
+  if (nmax >= 48 && tc_smem_bytes<8>(nmax) <= TC_SMEM_MAX) return launch_tridiag_cl<8>(jobs, njobs, nmax, s);
   const size_t smem = (size_t)(2 * nmax + 32) * sizeof(double);
   { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_tridiag_multi, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
   const int G = tridiag_blocks_per_job(njobs, nmax, smem);
