@@ -180,39 +180,37 @@ __device__ __forceinline__ double opt_err(const AllocArgs& a, const CellRD& c, i
   return __dmul_rn(a.eps2[bi], __dadd_rn(c.tT[rt], c.tD[rd]));
 }
 
-__global__ void __launch_bounds__(256) k_alloc_eval(AllocArgs a) {
-  if (a.st->phase == 3) return;
-  const int cell = blockIdx.y;
-  const CellRD c = a.cells[cell];
-  const double lam = a.st->lam;
-  const int nopt = a.n_bits * c.n_rt * a.n_rd;
-  const int per = (nopt + a.nchunk - 1) / a.nchunk;
-  const int i0 = blockIdx.x * per, i1 = min(nopt, i0 + per);
-  double best = INFINITY;
-  int bidx = 0x7fffffff;
-  for (int idx = i0 + threadIdx.x; idx < i1; idx += blockDim.x) {
-    int bi, rt, rd;
-    decode_opt(a, c, idx, bi, rt, rd);
-    double e = opt_err(a, c, bi, rt, rd);
-    double v = __dadd_rn(e, __dmul_rn(lam, (double)opt_bytes(a, c, bi, rt, rd)));
-    if (v < best) { best = v; bidx = idx; }   // ascending idx per thread: first min kept
+// The greedy search for bit width index bi: its e + lambda s and option index.
+__device__ void greedy_lane(const AllocArgs& a, const CellRD& c, double lam, int bi, double& best, int& bidx) {
+  int ti = 0, di = 0;
+  auto eval = [&](int t, int d, double& e, int64_t& s) {
+    const int rt = a.rt_grid[t], rd = a.rd_grid[d];
+    e = opt_err(a, c, bi, rt, rd);
+    s = opt_bytes(a, c, bi, rt, rd);
+    return __dadd_rn(e, __dmul_rn(lam, (double)s));
+  };
+  for (int guard = 0; guard < c.n_rt + a.n_rd; ++guard) {
+    double e0, e1, e2;
+    int64_t s0, s1, s2;
+    const double v0 = eval(ti, di, e0, s0);
+    bool c1 = false, c2 = false;
+    double r1 = 0.0, r2 = 0.0;
+    if (ti + 1 < c.n_rt) {
+      const double v1 = eval(ti + 1, di, e1, s1);
+      if (v1 < v0) { c1 = true; r1 = __ddiv_rn(__dsub_rn(e0, e1), (double)(s1 - s0)); }
+    }
+    if (di + 1 < a.n_rd) {
+      const double v2 = eval(ti, di + 1, e2, s2);
+      if (v2 < v0) { c2 = true; r2 = __ddiv_rn(__dsub_rn(e0, e2), (double)(s2 - s0)); }
+    }
+    if (!c1 && !c2) break;
+    if (c1 && (!c2 || r1 >= r2)) ++ti;
+    else ++di;
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    double ob = __shfl_xor_sync(0xffffffffu, best, o);
-    int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
-    if (ob < best || (ob == best && oi < bidx)) { best = ob; bidx = oi; }
-  }
-  __shared__ double sv[8];
-  __shared__ int si[8];
-  if ((threadIdx.x & 31) == 0) { sv[threadIdx.x >> 5] = best; si[threadIdx.x >> 5] = bidx; }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
-      if (sv[w] < best || (sv[w] == best && si[w] < bidx)) { best = sv[w]; bidx = si[w]; }
-    a.pv[cell * a.nchunk + blockIdx.x] = best;
-    a.pi[cell * a.nchunk + blockIdx.x] = bidx;
-  }
+  double e;
+  int64_t sb;
+  best = eval(ti, di, e, sb);
+  bidx = (bi * c.n_rt + ti) * a.n_rd + di;
 }
 
 // The page's greedy per-cell search ("Solving the allocation"): for each b
@@ -228,38 +226,7 @@ __global__ void __launch_bounds__(32) k_alloc_greedy(AllocArgs a) {
   const double lam = a.st->lam;
   double best = INFINITY;
   int bidx = 0x7fffffff;
-  if (lane < a.n_bits) {
-    const int bi = lane;
-    int ti = 0, di = 0;
-    auto eval = [&](int t, int d, double& e, int64_t& s) {
-      const int rt = a.rt_grid[t], rd = a.rd_grid[d];
-      e = opt_err(a, c, bi, rt, rd);
-      s = opt_bytes(a, c, bi, rt, rd);
-      return __dadd_rn(e, __dmul_rn(lam, (double)s));
-    };
-    for (int guard = 0; guard < c.n_rt + a.n_rd; ++guard) {
-      double e0, e1, e2;
-      int64_t s0, s1, s2;
-      const double v0 = eval(ti, di, e0, s0);
-      bool c1 = false, c2 = false;
-      double r1 = 0.0, r2 = 0.0;
-      if (ti + 1 < c.n_rt) {
-        const double v1 = eval(ti + 1, di, e1, s1);
-        if (v1 < v0) { c1 = true; r1 = __ddiv_rn(__dsub_rn(e0, e1), (double)(s1 - s0)); }
-      }
-      if (di + 1 < a.n_rd) {
-        const double v2 = eval(ti, di + 1, e2, s2);
-        if (v2 < v0) { c2 = true; r2 = __ddiv_rn(__dsub_rn(e0, e2), (double)(s2 - s0)); }
-      }
-      if (!c1 && !c2) break;
-      if (c1 && (!c2 || r1 >= r2)) ++ti;
-      else ++di;
-    }
-    double e;
-    int64_t sb;
-    best = eval(ti, di, e, sb);
-    bidx = (bi * c.n_rt + ti) * a.n_rd + di;
-  }
+  if (lane < a.n_bits) greedy_lane(a, c, lam, lane, best, bidx);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const double ob = __shfl_xor_sync(0xffffffffu, best, o);
@@ -269,6 +236,54 @@ __global__ void __launch_bounds__(32) k_alloc_greedy(AllocArgs a) {
   for (int k = lane; k < a.nchunk; k += 32) {
     a.pv[cell * a.nchunk + k] = (k == 0) ? best : INFINITY;
     a.pi[cell * a.nchunk + k] = (k == 0) ? bidx : 0x7fffffff;
+  }
+}
+
+// One step of the multiplier search on the total bytes S of the current
+// argmins; returns what to do with them: 0 nothing, 1 keep <- cur, 2 finish
+// with cur, 3 finish with keep, 4 keep <- cur then finish with keep.
+__device__ int alloc_step(AllocState* st, long long S, int* status) {
+  st->S = S;
+  const long long B = st->budget;
+  int act = 0;
+  if (st->phase == 0) {
+    if (S <= B) { act = 2; st->lam_final = st->lam; st->iters_final = 0; st->phase = 3; }
+    else { st->phase = 1; st->lam = st->hi; }
+  } else if (st->phase == 1) {
+    if (S > B) { atomicOr(status, DEV_ERR_INFEASIBLE); act = 2; st->lam_final = st->lam; st->iters_final = 0; st->phase = 3; }
+    else { act = 1; st->iter = 1; st->phase = 2; st->lam = sqrt(st->lo * st->hi); }
+  } else {
+    const double lo_ok = (1.0 - st->tol) * (double)B;
+    if ((double)S >= lo_ok && S <= B) {
+      act = 2; st->lam_final = st->lam; st->iters_final = st->iter; st->phase = 3;
+    } else {
+      if (S > B) st->lo = st->lam;
+      else { st->hi = st->lam; act = 1; }
+      if (st->iter >= st->max_iters) {
+        act = (act == 1) ? 4 : 3;
+        st->lam_final = st->hi; st->iters_final = st->max_iters; st->phase = 3;
+      } else {
+        st->iter += 1;
+        st->lam = sqrt(st->lo * st->hi);
+      }
+    }
+  }
+  return act;
+}
+
+// Applies a step's action to cell c: the kept argmin, or the final choice.
+__device__ void alloc_apply(const AllocArgs& a, int act, int c) {
+  if (act == 1 || act == 4) a.keep[c] = a.cur[c];
+  if (act >= 2) {
+    const int idx = (act == 2) ? a.cur[c] : a.keep[c];
+    const CellRD cc = a.cells[c];
+    int bi, rt, rd;
+    decode_opt(a, cc, idx, bi, rt, rd);
+    Choice ch;
+    ch.rT = rt; ch.rd = rd; ch.b = a.bits[bi]; ch.pad = 0;
+    ch.bytes = opt_bytes(a, cc, bi, rt, rd);
+    ch.err = opt_err(a, cc, bi, rt, rd);
+    a.out[c] = ch;
   }
 }
 
@@ -303,49 +318,171 @@ __global__ void __launch_bounds__(512) k_alloc_decide(AllocArgs a) {
   if (threadIdx.x == 0) {
     long long S = 0;
     for (int i = 0; i < (int)blockDim.x; ++i) S += sbytes[i];
-    st->S = S;
-    const long long B = st->budget;
-    int act = 0;
-    if (st->phase == 0) {
-      if (S <= B) { act = 2; st->lam_final = st->lam; st->iters_final = 0; st->phase = 3; }
-      else { st->phase = 1; st->lam = st->hi; }
-    } else if (st->phase == 1) {
-      if (S > B) { atomicOr(a.status, DEV_ERR_INFEASIBLE); act = 2; st->lam_final = st->lam; st->iters_final = 0; st->phase = 3; }
-      else { act = 1; st->iter = 1; st->phase = 2; st->lam = sqrt(st->lo * st->hi); }
-    } else {
-      const double lo_ok = (1.0 - st->tol) * (double)B;
-      if ((double)S >= lo_ok && S <= B) {
-        act = 2; st->lam_final = st->lam; st->iters_final = st->iter; st->phase = 3;
-      } else {
-        if (S > B) st->lo = st->lam;
-        else { st->hi = st->lam; act = 1; }
-        if (st->iter >= st->max_iters) {
-          act = (act == 1) ? 4 : 3;   // 4: keep<-cur then finish with keep
-          st->lam_final = st->hi; st->iters_final = st->max_iters; st->phase = 3;
-        } else {
-          st->iter += 1;
-          st->lam = sqrt(st->lo * st->hi);
-        }
-      }
-    }
+    const int act = alloc_step(st, S, a.status);
     action = act;
   }
   __syncthreads();
   const int act = action;
-  for (int c = threadIdx.x; c < a.ncells; c += blockDim.x) {
-    if (act == 1 || act == 4) a.keep[c] = a.cur[c];
-    if (act >= 2) {
-      int idx = (act == 2) ? a.cur[c] : a.keep[c];
-      const CellRD cc = a.cells[c];
-      int bi, rt, rd;
-      decode_opt(a, cc, idx, bi, rt, rd);
-      Choice ch;
-      ch.rT = rt; ch.rd = rd; ch.b = a.bits[bi]; ch.pad = 0;
-      ch.bytes = opt_bytes(a, cc, bi, rt, rd);
-      ch.err = opt_err(a, cc, bi, rt, rd);
-      a.out[c] = ch;
+  for (int c = threadIdx.x; c < a.ncells; c += blockDim.x) alloc_apply(a, act, c);
+}
+
+
+// The whole search in one block (small problems): per round, a warp per cell
+// takes the cell's argmin of e + lambda s over its options (lanes over the
+// options, first index on ties, as the chunked evaluation), the block sums
+// the bytes and thread 0 takes the bisection step. Same rounds and results
+// as the evaluate + decide launches, without a launch per round.
+__global__ void __launch_bounds__(1024) k_alloc_single(AllocArgs a, AllocState init) {
+  __shared__ AllocState st;
+  __shared__ long long sb[32];
+  __shared__ int act_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  if (threadIdx.x == 0) { st = init; st.arrive = 0u; }
+  __syncthreads();
+  for (int it = 0; it < init.max_iters + 2; ++it) {
+    const double lam = st.lam;
+    long long mine = 0;
+    for (int c = warp; c < a.ncells; c += nw) {
+      const CellRD cd = a.cells[c];
+      double best = INFINITY;
+      int bidx = 0x7fffffff;
+      if (a.greedy) {
+        if (lane < a.n_bits) greedy_lane(a, cd, lam, lane, best, bidx);
+      } else {
+        const int nopt = a.n_bits * cd.n_rt * a.n_rd;
+        for (int idx = lane; idx < nopt; idx += 32) {
+          int bi, rt, rd;
+          decode_opt(a, cd, idx, bi, rt, rd);
+          const double v = __dadd_rn(opt_err(a, cd, bi, rt, rd), __dmul_rn(lam, (double)opt_bytes(a, cd, bi, rt, rd)));
+          if (v < best) { best = v; bidx = idx; }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+        if (ob < best || (ob == best && oi < bidx)) { best = ob; bidx = oi; }
+      }
+      if (lane == 0) {
+        if (bidx < 0 || bidx >= a.n_bits * cd.n_rt * a.n_rd) {
+          bidx = 0;
+          atomicOr(a.status, DEV_ERR_NONFINITE);
+        }
+        a.cur[c] = bidx;
+        int bi, rt, rd;
+        decode_opt(a, cd, bidx, bi, rt, rd);
+        mine += opt_bytes(a, cd, bi, rt, rd);
+      }
+    }
+    if (lane == 0) sb[warp] = mine;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      long long S = 0;
+      for (int w = 0; w < nw; ++w) S += sb[w];
+      act_s = alloc_step(&st, S, a.status);
+    }
+    __syncthreads();
+    const int act = act_s;
+    for (int c = threadIdx.x; c < a.ncells; c += blockDim.x) alloc_apply(a, act, c);
+    if (st.phase == 3) break;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *a.st = st;
+}
+
+
+// One evaluation round of the enumeration, by rows: a row is a (bit width,
+// r_T grid entry) pair and its options are the r_d grid entries, so the
+// option index (bi*n_rt + ti)*n_rd + di needs no division and the byte count
+// is s0 + (bytes per unit of r_d) r_d in exact integers; e and e + lambda s
+// are rounded exactly as opt_err / opt_bytes give them. Blocks (chunk, cell)
+// write their partial argmin; the last block to finish takes the per-cell
+// argmins, the total bytes and the bisection step (alloc_step), so a round is
+// one launch.
+__global__ void __launch_bounds__(256) k_alloc_rows(AllocArgs a) {
+  AllocState* st = a.st;
+  if (st->phase == 3) return;
+  const int cell = blockIdx.y;
+  const CellRD c = a.cells[cell];
+  const double lam = st->lam;
+  const int nrows = a.n_bits * c.n_rt;
+  const int per = (nrows + a.nchunk - 1) / a.nchunk;
+  const int r0 = blockIdx.x * per, r1 = min(nrows, r0 + per);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int64_t LH = (int64_t)c.Lg * c.H;
+  double best = INFINITY;
+  int bidx = 0x7fffffff;
+  for (int r = r0 + warp; r < r1; r += nw) {
+    const int bi = r / c.n_rt, ti = r - bi * c.n_rt;
+    const int rt = a.rt_grid[ti];
+    const double eb = a.eps2[bi], tt = c.tT[rt];
+    const int64_t s0 = 2 * ((int64_t)c.T * rt) + a.rowbytes[bi] * LH * c.T;
+    const int64_t srd = 2 * (LH * rt + c.D);
+    const int rd_ok = c.Lg * c.H * rt;      // larger feature ranks are excluded (infinite error)
+    for (int di = lane; di < a.n_rd; di += 32) {
+      const int rd = a.rd_grid[di];
+      if (rd > rd_ok) continue;
+      const double e = __dmul_rn(eb, __dadd_rn(tt, c.tD[rd]));
+      const double v = __dadd_rn(e, __dmul_rn(lam, (double)(s0 + srd * rd)));
+      const int idx = r * a.n_rd + di;
+      if (v < best || (v == best && idx < bidx)) { best = v; bidx = idx; }
     }
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+    if (ob < best || (ob == best && oi < bidx)) { best = ob; bidx = oi; }
+  }
+  __shared__ double sv[8];
+  __shared__ int si[8];
+  __shared__ int last_s;
+  if (lane == 0) { sv[warp] = best; si[warp] = bidx; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < nw; ++w)
+      if (sv[w] < best || (sv[w] == best && si[w] < bidx)) { best = sv[w]; bidx = si[w]; }
+    a.pv[cell * a.nchunk + blockIdx.x] = best;
+    a.pi[cell * a.nchunk + blockIdx.x] = bidx;
+    __threadfence();
+    const unsigned n = atomicAdd(&st->arrive, 1u);
+    last_s = (n == gridDim.x * gridDim.y - 1);
+  }
+  __syncthreads();
+  if (!last_s) return;
+  __threadfence();
+  // ---- the last block: per-cell argmins, total bytes, one bisection step
+  __shared__ long long sbytes[256];
+  __shared__ int action;
+  long long mine = 0;
+  for (int cc = threadIdx.x; cc < a.ncells; cc += blockDim.x) {
+    double b2 = INFINITY;
+    int i2 = 0x7fffffff;
+    for (int k = 0; k < a.nchunk; ++k) {
+      const double v = __ldcg(a.pv + cc * a.nchunk + k);
+      const int i = __ldcg(a.pi + cc * a.nchunk + k);
+      if (v < b2 || (v == b2 && i < i2)) { b2 = v; i2 = i; }
+    }
+    if (i2 < 0 || i2 >= a.n_bits * a.cells[cc].n_rt * a.n_rd) {
+      i2 = 0;
+      atomicOr(a.status, DEV_ERR_NONFINITE);
+    }
+    a.cur[cc] = i2;
+    int bi, rt, rd;
+    decode_opt(a, a.cells[cc], i2, bi, rt, rd);
+    mine += opt_bytes(a, a.cells[cc], bi, rt, rd);
+  }
+  sbytes[threadIdx.x] = mine;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long S = 0;
+    for (int i = 0; i < (int)blockDim.x; ++i) S += sbytes[i];
+    action = alloc_step(st, S, a.status);
+    st->arrive = 0u;
+  }
+  __syncthreads();
+  const int act = action;
+  for (int cc = threadIdx.x; cc < a.ncells; cc += blockDim.x) alloc_apply(a, act, cc);
 }
 
 __global__ void k_alloc_init(AllocState* st, AllocState init) {
@@ -356,14 +493,25 @@ __global__ void k_alloc_init(AllocState* st, AllocState init) {
 // evaluate + decide; each round tries one multiplier and rounds after the
 // decision return at once.
 jolt_status launch_alloc(const AllocArgs& a, const AllocState& init, cudaStream_t s) {
-  k_alloc_init<<<1, 32, 0, s>>>(a.st, init);
+  // small searches (all options of all cells within a few per thread): one block
+  if ((int64_t)a.ncells * a.n_bits * std::max(a.n_rt_max, 1) * a.n_rd <= (int64_t)16 * 1024) {
+    k_alloc_single<<<1, 1024, 0, s>>>(a, init);
+    JOLT_LAUNCHED();
+    return JOLT_OK;
+  }
+  AllocState i0 = init;
+  i0.arrive = 0u;
+  k_alloc_init<<<1, 32, 0, s>>>(a.st, i0);
   JOLT_LAUNCHED();
   dim3 grid(a.nchunk, a.ncells);
   for (int it = 0; it < init.max_iters + 2; ++it) {
-    if (a.greedy) k_alloc_greedy<<<a.ncells, 32, 0, s>>>(a);
-    else k_alloc_eval<<<grid, 256, 0, s>>>(a);
-    JOLT_LAUNCHED();
-    k_alloc_decide<<<1, 512, 0, s>>>(a);
+    if (a.greedy) {
+      k_alloc_greedy<<<a.ncells, 32, 0, s>>>(a);
+      JOLT_LAUNCHED();
+      k_alloc_decide<<<1, 512, 0, s>>>(a);
+    } else {
+      k_alloc_rows<<<grid, 256, 0, s>>>(a);
+    }
     JOLT_LAUNCHED();
   }
   return JOLT_OK;

@@ -1025,7 +1025,7 @@ static jolt_status run_allocation(jolt_plan_s* p, int64_t budget, const double* 
   AllocArgs a{};
   a.greedy = p->opt.minimizer == JOLT_MIN_GREEDY;
   a.cells = p->d_rd_cells; a.ncells = p->ncells;
-  a.rt_grid = p->d_rt; a.rd_grid = p->d_rd; a.n_rd = (int)p->rd_grid.size();
+  a.rt_grid = p->d_rt; a.rd_grid = p->d_rd; a.n_rd = (int)p->rd_grid.size(); a.n_rt_max = (int)p->rt_grid.size();
   a.bits = p->d_bits; a.eps2 = eps2; a.rowbytes = p->d_rowbytes; a.n_bits = (int)p->bits.size();
   a.nchunk = p->achunk; a.pv = p->d_apv; a.pi = p->d_api; a.cur = p->d_cur; a.keep = p->d_keep;
   a.st = st_dev; a.out = out; a.status = status;
@@ -1155,7 +1155,7 @@ static jolt_status compress_end(jolt_handle_s* h, const void* k, const void* v, 
         AllocArgs a{};
         a.greedy = p->opt.minimizer == JOLT_MIN_GREEDY;
         a.cells = rd; a.ncells = n_total;
-        a.rt_grid = p->d_rt; a.rd_grid = p->d_rd; a.n_rd = (int)p->rd_grid.size();
+        a.rt_grid = p->d_rt; a.rd_grid = p->d_rd; a.n_rd = (int)p->rd_grid.size(); a.n_rt_max = (int)p->rt_grid.size();
         a.bits = p->d_bits; a.eps2 = p->d_eps2; a.rowbytes = p->d_rowbytes; a.n_bits = (int)p->bits.size();
         a.nchunk = p->achunk; a.pv = pv; a.pi = pi; a.cur = cur; a.keep = keep;
         a.st = ast; a.out = ch; a.status = h->d_status;

@@ -57,6 +57,7 @@ struct AllocState {
   double lam_final;
   int iters_final;
   int64_t S;
+  unsigned arrive;      // blocks of the current evaluation round that have finished
 };
 
 // The chosen option of a cell (device).
@@ -85,6 +86,7 @@ struct AllocArgs {
   Choice* out;              // [ncells]
   int* status;
   int greedy;               // 1: the page's greedy per-cell search instead of enumeration
+  int n_rt_max;             // the most r_T grid entries of any cell (sizes the search)
 };
 
 jolt_status launch_alloc(const AllocArgs& a, const AllocState& init, cudaStream_t s);
