@@ -1584,6 +1584,9 @@ extern "C" jolt_status jolt_decode_attention(const jolt_handle_t* hc, int32_t la
       c.ut[b] = ko[b].ut;
       c.rt_k[b] = ko[b].rT;
       c.tpitch[b] = ko[b].t_pitch;
+      c.uv[b] = vo[b].ut;
+      c.rt_v[b] = vo[b].rT;
+      c.tpitch_v[b] = vo[b].t_pitch;
     }
     const int rpk = (rk + 63) / 64 * 64, rpv = (rv + 63) / 64 * 64;
     const int64_t part_len = (int64_t)Bc * H * 64 * G * (2 + rpv + D);

@@ -261,6 +261,8 @@ struct DecodeCall {
   float* part; int64_t part_len;  // workspace: split states
   const uint16_t* ut[DEC_BMAX];   // U_T^ of each sequence's key cell and its shape
   int rt_k[DEC_BMAX], tpitch[DEC_BMAX];
+  const uint16_t* uv[DEC_BMAX];   // U_T^ of each sequence's value cell and its shape
+  int rt_v[DEC_BMAX], tpitch_v[DEC_BMAX];
   int* status;
 };
 jolt_status launch_decode_attention(const DecodeCall& c, cudaStream_t s);
