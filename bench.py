@@ -124,7 +124,7 @@ class ClockSampler:
 # the 64K-token cache, scaled to the full 16-cell launch by the cells it
 # processes (mean of the X W and X^T Y launches); None once the kernel has
 # changed since the capture.
-GEMM_TRAFFIC = {}
+GEMM_TRAFFIC = {"llama31_8b_64k": 9.85e9}
 
 
 def sketch_width(spec, ratio, p=8):

@@ -979,9 +979,14 @@ __global__ void __launch_bounds__(256) k_backtr(const EighJob* __restrict__ jobs
       const double* v = vbuf + (k & 1) * n;
       for (int vv = warp; vv < nb; vv += 8) {
         double* z = Zs + (int64_t)vv * n + (k + 1);
-        double acc = 0.0;
-        for (int i = lane; i < m; i += 32) acc += v[i] * z[i];
-        acc = beta * warp_sum(acc);
+        double acc0 = 0.0, acc1 = 0.0;         // two chains, added in a fixed order
+        int i = lane;
+        for (; i + 32 < m; i += 64) {
+          acc0 += v[i] * z[i];
+          acc1 += v[i + 32] * z[i + 32];
+        }
+        if (i < m) acc0 += v[i] * z[i];
+        const double acc = beta * warp_sum(acc0 + acc1);
         for (int i = lane; i < m; i += 32) z[i] -= acc * v[i];
       }
     }
@@ -1075,8 +1080,9 @@ jolt_status launch_eigvecs_n(const EighJob* jobs, int njobs, int nvec_max, int n
   if (nmax > 256 * BT_PRE) { set_error("eigenvectors need n <= %d (n=%d)", 256 * BT_PRE, nmax); return JOLT_ERR_UNSUPPORTED_SHAPE; }
   k_invit<<<dim3((nvec_max + INV_W - 1) / INV_W, njobs), INV_W, 0, s>>>(jobs, nvec);
   JOLT_LAUNCHED();
-  // vectors per block: as many as 200 KB of shared memory hold, at most 32
-  const int vb = std::max(1, std::min(32, (int)((200 * 1024) / ((size_t)nmax * sizeof(double))) - 2));
+  // vectors per block: 16 (two per warp), so that several blocks share an
+  // SM and hide each other's shared-memory latency; fewer when n is large
+  const int vb = std::max(1, std::min(16, (int)((200 * 1024) / ((size_t)nmax * sizeof(double))) - 2));
   const size_t smem = (size_t)(vb + 2) * nmax * sizeof(double);
   { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_backtr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
   k_backtr<<<dim3((nvec_max + vb - 1) / vb, njobs), 256, smem, s>>>(jobs, nvec, vb);
