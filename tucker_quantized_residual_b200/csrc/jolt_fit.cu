@@ -208,38 +208,49 @@ __global__ void k_ud_store(FitArgs a) {
   }
 }
 
-// One block per (r, lh): G^ row and M^ row.
+// One block per (CORE_R rows r, lh): G^ rows and M^ rows. The core reads
+// U_d^[d][j] across the threads j (consecutive), M^ reads U_d^ staged
+// transposed in shared memory ([j][d], consecutive across the threads d);
+// each value is the same fp64 sum in the same order (d, then j ascending) as
+// a block per row. Shared memory: 48 KB at D = 128.
+constexpr int CORE_R = 8;
 template <int D>
 __global__ void __launch_bounds__(D) k_core(FitArgs a) {
-  const int cell = blockIdx.z, lh = blockIdx.y, r = blockIdx.x;
+  const int cell = blockIdx.z, lh = blockIdx.y, r0 = blockIdx.x * CORE_R;
   const CellDesc c = a.cells[cell];
   const CellOut o = a.out[cell];
-  if (lh >= c.Lg * c.H || r >= o.rT) return;
-  __shared__ double y[D];
-  __shared__ double g[D];
+  if (lh >= c.Lg * c.H || r0 >= o.rT) return;
+  __shared__ double y[CORE_R][D];
+  __shared__ double g[CORE_R][D];
+  __shared__ uint16_t udt[D * D];    // [j][d], j < rd
+  const int rd = o.rd, nr = min(CORE_R, o.rT - r0);
   const int rmax = a.rmax_of[cell];
-  const double* yr = a.Y[cell] + ((int64_t)lh * rmax + r) * D;
-  y[threadIdx.x] = yr[threadIdx.x];
+  for (int e = threadIdx.x; e < D * rd; e += D) udt[(e % rd) * D + e / rd] = o.ud[e];
+  for (int i = 0; i < nr; ++i) y[i][threadIdx.x] = a.Y[cell][((int64_t)lh * rmax + r0 + i) * D + threadIdx.x];
   __syncthreads();
   const int j = threadIdx.x;
-  if (j < o.rd) {
-    double acc = 0.0;
-    for (int d = 0; d < D; ++d) acc += y[d] * bf16d(o.ud[d * o.rd + j]);
-    uint16_t gb = bf16_bits_from_f64(acc);
-    o.core[((int64_t)lh * o.rT + r) * o.rd + j] = gb;
-    g[j] = bf16d(gb);
+  if (j < rd) {
+    for (int i = 0; i < nr; ++i) {
+      double acc = 0.0;
+      for (int d = 0; d < D; ++d) acc += y[i][d] * bf16d(o.ud[d * rd + j]);
+      const uint16_t gb = bf16_bits_from_f64(acc);
+      o.core[((int64_t)lh * o.rT + r0 + i) * rd + j] = gb;
+      g[i][j] = bf16d(gb);
+    }
   }
   __syncthreads();
   const int d = threadIdx.x;
-  double m = 0.0;
-  for (int jj = 0; jj < o.rd; ++jj) m += g[jj] * bf16d(o.ud[d * o.rd + jj]);
-  a.M[cell][((int64_t)lh * rmax + r) * D + d] = bf16_bits_from_f64(m);
+  for (int i = 0; i < nr; ++i) {
+    double m = 0.0;
+    for (int jj = 0; jj < rd; ++jj) m += g[i][jj] * bf16d(udt[jj * D + d]);
+    a.M[cell][((int64_t)lh * rmax + r0 + i) * D + d] = bf16_bits_from_f64(m);
+  }
 }
 
 jolt_status launch_core(const FitArgs& a, int rmax_all, int lh_max, cudaStream_t s) {
   k_ud_store<<<a.ncells, 256, 0, s>>>(a);
   JOLT_LAUNCHED();
-  dim3 g(rmax_all, lh_max, a.ncells);
+  dim3 g((rmax_all + CORE_R - 1) / CORE_R, lh_max, a.ncells);
   if (a.D == 128) k_core<128><<<g, 128, 0, s>>>(a);
   else k_core<64><<<g, 64, 0, s>>>(a);
   JOLT_LAUNCHED();
@@ -274,25 +285,32 @@ jolt_status launch_copy_rt(const CellOut* out, int* rt, int ncells, cudaStream_t
 
 // Decoder product from the stored payload: M^[lh][r][d] = bf16(sum_j G^[lh][r][j] U_d^[d][j]),
 // the same fp64 sum order as at compression, so the values match bit for bit.
+// CORE_R rows per block, U_d^ staged transposed in shared memory.
 template <int D>
 __global__ void __launch_bounds__(D) k_core_m(const CellOut* __restrict__ outs, const CellDesc* __restrict__ cells,
                                               uint16_t* const* __restrict__ M, const int* __restrict__ rmax_of) {
-  const int cell = blockIdx.z, lh = blockIdx.y, r = blockIdx.x;
+  const int cell = blockIdx.z, lh = blockIdx.y, r0 = blockIdx.x * CORE_R;
   const CellDesc c = cells[cell];
   const CellOut o = outs[cell];
-  if (lh >= c.Lg * c.H || r >= o.rT) return;
-  __shared__ double g[D];
-  if ((int)threadIdx.x < o.rd) g[threadIdx.x] = bf16d(o.core[((int64_t)lh * o.rT + r) * o.rd + threadIdx.x]);
+  if (lh >= c.Lg * c.H || r0 >= o.rT) return;
+  __shared__ double g[CORE_R][D];
+  __shared__ uint16_t udt[D * D];    // [j][d]
+  const int rd = o.rd, nr = min(CORE_R, o.rT - r0);
+  for (int e = threadIdx.x; e < D * rd; e += D) udt[(e % rd) * D + e / rd] = o.ud[e];
+  for (int i = 0; i < nr; ++i)
+    if ((int)threadIdx.x < rd) g[i][threadIdx.x] = bf16d(o.core[((int64_t)lh * o.rT + r0 + i) * rd + threadIdx.x]);
   __syncthreads();
   const int d = threadIdx.x;
-  double m = 0.0;
-  for (int j = 0; j < o.rd; ++j) m += g[j] * bf16d(o.ud[d * o.rd + j]);
-  M[cell][((int64_t)lh * rmax_of[cell] + r) * D + d] = bf16_bits_from_f64(m);
+  for (int i = 0; i < nr; ++i) {
+    double m = 0.0;
+    for (int j = 0; j < rd; ++j) m += g[i][j] * bf16d(udt[j * D + d]);
+    M[cell][((int64_t)lh * rmax_of[cell] + r0 + i) * D + d] = bf16_bits_from_f64(m);
+  }
 }
 
 jolt_status launch_core_m(const CellOut* out, const CellDesc* cells, uint16_t* const* M, const int* rmax_of,
                           int ncells, int D, int rmax_all, int lh_max, cudaStream_t s) {
-  dim3 g(rmax_all, lh_max, ncells);
+  dim3 g((rmax_all + CORE_R - 1) / CORE_R, lh_max, ncells);
   if (D == 128) k_core_m<128><<<g, 128, 0, s>>>(out, cells, M, rmax_of);
   else k_core_m<64><<<g, 64, 0, s>>>(out, cells, M, rmax_of);
   JOLT_LAUNCHED();
