@@ -300,4 +300,24 @@ __device__ __forceinline__ bool dispatch_gb(int G, int B, F& f) {
   return false;
 }
 
+// ------------------------------------------------ thread-block clusters ----
+// Rank of this CTA in its cluster.
+__device__ __forceinline__ uint32_t tc_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Generic address of the same shared-memory location in CTA `rank` of the
+// cluster (plain loads through it read that CTA's shared memory).
+__device__ __forceinline__ const double* tc_peer(const double* local, uint32_t rank) {
+  uint64_t a;
+  asm("mapa.u64 %0, %1, %2;" : "=l"(a) : "l"(reinterpret_cast<uint64_t>(local)), "r"(rank));
+  return reinterpret_cast<const double*>(a);
+}
+// Every thread of every CTA of the cluster; writes before it are visible to
+// the cluster's reads after it.
+__device__ __forceinline__ void tc_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 }  // namespace jolt

@@ -519,23 +519,6 @@ __global__ void __launch_bounds__(EIG_THREADS) k_tridiag_multi(const EighJob* __
 constexpr int TC_THREADS = 512;
 constexpr size_t TC_SMEM_MAX = 227 * 1024;
 
-__device__ __forceinline__ uint32_t tc_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// generic address of the same shared-memory location in CTA `rank` of the
-// cluster (plain loads through it read that CTA's shared memory)
-__device__ __forceinline__ const double* tc_peer(const double* local, uint32_t rank) {
-  uint64_t a;
-  asm("mapa.u64 %0, %1, %2;" : "=l"(a) : "l"(reinterpret_cast<uint64_t>(local)), "r"(rank));
-  return reinterpret_cast<const double*>(a);
-}
-// every thread of every CTA of the cluster; writes before it are visible to
-// the cluster's reads after it
-__device__ __forceinline__ void tc_cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
 // packed offset of owned row lr (global row rank + CS lr, rank + 1 + CS lr entries)
 template <int CS>
 __host__ __device__ inline int tc_off(int lr, int rank) { return lr * (rank + 1) + CS * (lr * (lr - 1) / 2); }
