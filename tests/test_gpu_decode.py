@@ -137,3 +137,23 @@ def test_decode_rejects_bad_arguments():
         torch.cuda.synchronize()
         jolt.jolt_free_handle(h)
         jolt.jolt_free_plan(plan)
+
+
+@pytest.mark.parametrize("D,Hq_per", [(128, 8), (64, 3)])
+def test_decode_value_ranks_over_several_blocks(D, Hq_per):
+    """A token rank of 320 for every cell (a one-entry r_T grid), so the
+    rank-space value product spans three blocks of 128 ranks (the last one
+    partly past r_T), with 8 and 3 query heads per KV head; T = 1000 leaves a
+    ragged last tile."""
+    spec = synth.CacheSpec("dec320", 1, 4, 4, 1000, D, 4, 48, 0.8, 0.02, rope_theta_k=1e4)
+    K, V, plan, h, comp = _case(spec, 1.2, bits=(0, 4), rt_grid=(320,), rd_grid=(D // 2, D))
+    try:
+        assert all(c.r_t == 320 for c in comp.cells)
+        rng = np.random.default_rng(23)
+        for layer in (0, 2):
+            _check(comp, h, spec, layer, spec.n_heads * Hq_per, 6, rng)
+    finally:
+        torch.cuda.synchronize()
+        jolt.jolt_free_handle(h)
+        jolt.jolt_free_plan(plan)
+
