@@ -148,7 +148,7 @@ def test_decode_value_ranks_over_several_blocks(D, Hq_per):
     spec = synth.CacheSpec("dec320", 1, 4, 4, 1000, D, 4, 48, 0.8, 0.02, rope_theta_k=1e4)
     K, V, plan, h, comp = _case(spec, 1.2, bits=(0, 4), rt_grid=(320,), rd_grid=(D // 2, D))
     try:
-        assert all(c.r_t == 320 for c in comp.cells)
+        assert all(c.rT == 320 for c in comp.cells)
         rng = np.random.default_rng(23)
         for layer in (0, 2):
             _check(comp, h, spec, layer, spec.n_heads * Hq_per, 6, rng)
