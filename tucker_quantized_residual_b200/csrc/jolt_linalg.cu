@@ -734,14 +734,15 @@ static jolt_status launch_tridiag_cl(const EighJob* jobs, int njobs, int nmax, c
   return JOLT_OK;
 }
 
-// Number of eigenvalues of the tridiagonal (d, e) smaller than x.
-__device__ __forceinline__ int sturm_count(const double* d, const double* e, int n, double x, double pivmin) {
+// Number of eigenvalues of the tridiagonal (d, e) smaller than x; e2[i] is
+// the rounded square of e[i].
+__device__ __forceinline__ int sturm_count(const double* d, const double* e2, int n, double x, double pivmin) {
   int c = 0;
   double q = d[0] - x;
   if (fabs(q) < pivmin) q = -pivmin;
   c += q < 0.0;
   for (int i = 1; i < n; ++i) {
-    q = (d[i] - x) - e[i - 1] * e[i - 1] / q;
+    q = (d[i] - x) - e2[i - 1] / q;
     if (fabs(q) < pivmin) q = -pivmin;
     c += q < 0.0;
   }
@@ -762,7 +763,13 @@ __global__ void __launch_bounds__(256) k_bisect(const EighJob* __restrict__ jobs
   extern __shared__ double sh[];
   double* d = sh;
   double* e = sh + n;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) { d[i] = J.work[i]; e[i] = J.work[n + i]; }
+  double* e2 = sh + 2 * n;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    d[i] = J.work[i];
+    const double ei = J.work[n + i];
+    e[i] = ei;
+    e2[i] = ei * ei;
+  }
   __syncthreads();
   const int lane = threadIdx.x & 31, sub = lane & (BIS_L - 1), base = lane & ~(BIS_L - 1);
   const int j = blockIdx.x * (blockDim.x / BIS_L) + threadIdx.x / BIS_L;
@@ -792,7 +799,7 @@ __global__ void __launch_bounds__(256) k_bisect(const EighJob* __restrict__ jobs
     if (mid <= lo || mid >= hi) done = true;
     if (__all_sync(0xffffffffu, done)) break;
     const double x = lo + (hi - lo) * ((double)(sub + 1) / (double)(BIS_L + 1));
-    const bool above = (!done && x > lo && x < hi) ? (sturm_count(d, e, n, x, pivmin) > m) : (x >= hi);
+    const bool above = (!done && x > lo && x < hi) ? (sturm_count(d, e2, n, x, pivmin) > m) : (x >= hi);
     const unsigned bal = (__ballot_sync(0xffffffffu, above) >> base) & ((1u << BIS_L) - 1u);
     const int f = bal ? (__ffs(bal) - 1) : BIS_L;   // first point past the eigenvalue
     const double xl = __shfl_sync(0xffffffffu, x, base + (f > 0 ? f - 1 : 0));
@@ -1050,7 +1057,7 @@ jolt_status launch_tridiag_multi(const EighJob* jobs, int njobs, int nmax, doubl
 }
 
 jolt_status launch_bisect(const EighJob* jobs, int njobs, int nmax, cudaStream_t s) {
-  const size_t smem = (size_t)(2 * nmax) * sizeof(double);
+  const size_t smem = (size_t)(3 * nmax) * sizeof(double);
   { static size_t set = 0; if (smem > set) { JOLT_CUDA_TRY(cudaFuncSetAttribute(k_bisect, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); set = smem; } }
   dim3 g((nmax + 256 / BIS_L - 1) / (256 / BIS_L), njobs);   // BIS_L lanes per eigenvalue
   k_bisect<<<g, 256, smem, s>>>(jobs);

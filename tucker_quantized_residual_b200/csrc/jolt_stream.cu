@@ -511,6 +511,8 @@ __global__ void __launch_bounds__(QTHREADS, 1) k_stream(const __grid_constant__ 
           xph[xb] ^= 1;
           xb ^= 1;
           fwht_quad<C>(e, lane_base, x1, x2, j, q);
+          // times D^-1/2, then the sign: one product by +-D^-1/2 (the sign is
+          // exact, so this is the same rounded value)
 #pragma unroll
           for (int k = 0; k < 2; ++k)
 #pragma unroll
@@ -518,7 +520,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) k_stream(const __grid_constant__ 
               const float4 s4 = reinterpret_cast<const float4*>(sSign + (k ? cB : cA))[u];
               const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
-              for (int i = 0; i < 4; ++i) e[k * C + 4 * u + i] = __fmul_rn(__fmul_rn(e[k * C + 4 * u + i], rs), sv[i]);
+              for (int i = 0; i < 4; ++i) e[k * C + 4 * u + i] = __fmul_rn(e[k * C + 4 * u + i], __fmul_rn(rs, sv[i]));
             }
         } else {
 #pragma unroll
