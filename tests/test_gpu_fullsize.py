@@ -3,9 +3,11 @@ their full-size paths, against the fp64 oracle.
 
 * k = 528: one layer of 8 KV heads at D = 128 and T = 16384, so N = 1024 and
   q_cap = 512 by Eq. (5): the sketch width k = 512 + 8 rounded up to 16 is the
-  one of the 64K-token LLaMA-3.1-8B-shaped cache, the GEMM splits it into
-  three 176-column tiles, and CholeskyQR and the eigensolver run on 528 x 528
-  matrices.
+  one of the 64K-token LLaMA-3.1-8B-shaped cache, the CTA-pair GEMM splits it
+  into N tiles of 272 and 256 columns, and CholeskyQR and the eigensolver run
+  on 528 x 528 matrices.
+* k = 272: the same layer at T = 8192 (q_cap = 256): one N tile of 272
+  columns, two MMAs of 144 and 128 per K step.
 * LLaMA-2-13B shape: 4 layers of 40 KV heads (N_c = 20480) at T = 4096,
   q_cap = 128, k = 144.
 * the MoE/GQA batch: 16 sequences in one call (groups of 6 layers, 4 KV heads,
@@ -28,6 +30,7 @@ from gpu_helpers import gpu_compress, oracle_compress
 pytestmark = pytest.mark.gpu
 
 K528 = synth.SPECS["llama31_8b_64k"].replace(n_layers=1, group_size=1, seq_len=16384)
+K272 = synth.SPECS["llama31_8b_64k"].replace(n_layers=1, group_size=1, seq_len=8192)
 LLAMA2 = synth.SPECS["llama2_13b"].replace(n_layers=4)
 MOE16 = synth.SPECS["moe_t1024"].replace(n_layers=12)
 
@@ -100,6 +103,14 @@ def test_k528_spectrum_on_the_same_sketch():
 @pytest.mark.parametrize("C_ratio", [2.0, 3.0])
 def test_k528_gate(C_ratio):
     _gate(K528, C_ratio)
+
+
+def test_k272_spectrum_on_the_same_sketch():
+    _same_sketch(K272, 2.0)
+
+
+def test_k272_gate():
+    _gate(K272, 2.0)
 
 
 def test_llama2_13b_shape_spectrum_on_the_same_sketch():
