@@ -240,7 +240,9 @@ JOLT_API jolt_status jolt_decompress(const jolt_handle_t* h, void* k_out, void* 
  *     rotated), NULL when n_tail == 0; n_tail <= 1024.
  *   out: DEVICE fp32 [batch][n_q_heads][D].
  * The handle must use the Hadamard rotation (JOLT_ERR_UNSUPPORTED_SHAPE for
- * JOLT_ROT_QR_GAUSS). The first call on a handle reads the cells' layout to
+ * JOLT_ROT_QR_GAUSS), and the value cells of the layer's group a token rank
+ * r_T <= 512 (always so in randomized mode, where r_T <= q_cap <= 512;
+ * JOLT_ERR_UNSUPPORTED_SHAPE otherwise). The first call on a handle reads the cells' layout to
  * the host (synchronises the handle's stream once); later calls are
  * asynchronous. Workspace comes from the library allocator. */
 JOLT_API jolt_status jolt_decode_attention(const jolt_handle_t* h, int32_t layer, const float* q,

@@ -1588,6 +1588,11 @@ extern "C" jolt_status jolt_decode_attention(const jolt_handle_t* hc, int32_t la
       c.rt_v[b] = vo[b].rT;
       c.tpitch_v[b] = vo[b].t_pitch;
     }
+    if (rv > 512) {
+      // the rank-space value state holds at most four blocks of 128 ranks
+      set_error("fused decode attention needs the value cells' r_T <= 512 (layer %d has %d)", layer, rv);
+      return JOLT_ERR_UNSUPPORTED_SHAPE;
+    }
     const int rpk = (rk + 63) / 64 * 64, rpv = (rv + 63) / 64 * 64;
     const int64_t part_len = (int64_t)Bc * H * 64 * G * (2 + rpv + D);
     Arena A;
