@@ -32,11 +32,38 @@ def _layout(D=64, theta=0.0, groups=(0, 2)):
     return L, gs
 
 
-@pytest.mark.parametrize("bad", ["D", "bits", "group", "grid", "groups", "minimizer", "rotation"])
+@pytest.mark.parametrize("bad", ["D", "bits", "group", "grid", "groups", "minimizer", "rotation", "dtype", "stride",
+                                 "rope", "mode", "n_bits", "bits_order", "tol", "iters", "seq_base", "cap_ratio",
+                                 "rd_grid", "budget"])
 def test_plan_rejects_bad_arguments_before_touching_the_device(bad):
     L, keep = _layout()
     o, k2 = jolt.make_options()
-    if bad == "D":
+    budget = 10 ** 6
+    if bad == "dtype":
+        L.dtype = 7
+    elif bad == "stride":
+        L.stride_t = L.head_dim - 1
+    elif bad == "rope":
+        L.rope_theta_k = -1.0
+    elif bad == "mode":
+        o.mode = 5
+    elif bad == "n_bits":
+        o.n_bits = 0
+    elif bad == "bits_order":
+        o, k2 = jolt.make_options(bits=(4, 2))
+    elif bad == "tol":
+        o.budget_tol = 1.0
+    elif bad == "iters":
+        o.max_iters = 0
+    elif bad == "seq_base":
+        o.seq_base = -1
+    elif bad == "cap_ratio":
+        o.cap_ratio = float("nan")
+    elif bad == "rd_grid":
+        o, k2 = jolt.make_options(rd_grid=[0, 8])
+    elif bad == "budget":
+        budget = 0
+    elif bad == "D":
         L.head_dim = 96
     elif bad == "bits":
         o.bits[1] = 5
@@ -52,7 +79,7 @@ def test_plan_rejects_bad_arguments_before_touching_the_device(bad):
     elif bad == "rotation":
         o.rotation = 2
     with pytest.raises(jolt.JoltError) as ei:
-        jolt.jolt_plan(L, 10 ** 6, o)
+        jolt.jolt_plan(L, budget, o)
     assert ei.value.status in (1, 2)
 
 
