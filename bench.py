@@ -592,21 +592,12 @@ def run_jolt(args):
             sys.stderr.write(f"  cell g{c.group} {'KV'[c.kind]}: r_T {c.r_t} r_d {c.r_d} b {c.bits}\n")
 
     if rank == 0:
-        par = (f"one shared byte budget over {world} GPUs: rank r compresses sequences [r*{spec.batch}, "
-               f"(r+1)*{spec.batch}), one all-gather of per-cell rate-distortion records per step (NCCL)"
-               if world > 1 else "one GPU")
         line = {
             "metric": "GB/s of bf16 KV cache compressed+decompressed at 2x/3x budget; rel. Frobenius err",
             "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{args.config} ({spec.n_layers} layers / groups of {spec.group_size}, "
-                                   f"{spec.n_heads} KV heads, D={spec.head_dim}, T={spec.seq_len}, "
-                                   f"batch {spec.batch} per GPU), {args.ratio:g}x budget, {args.mode} token SVD",
-                       "global_batch": spec.batch * world, "seq_len": spec.seq_len,
-                       "parallelism": par,
-                       "l2": f"inputs {dense / 1e9:.2f} GB per GPU" + (
-                           ", larger than L2; no flush" if dense > 126e6 else ", smaller than L2")},
+            "config": arm_config(args, spec, world),
             "rel_frobenius_err": {"K": errK, "V": errV}, "bytes": nbytes, "budget": B,
             "budgets": budgets,
             "roofline": roof, "path_roofline": path_roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
@@ -679,6 +670,23 @@ def cpu_baseline(spec, ratio, T_sample=CPU_TOKENS, reps=8):
             "sample": sample_text(spec, T_sample, reps) + f", {nb / 1e6:.1f} MB dense bf16 in {total:.2f} s"}
 
 
+def arm_config(args, spec, world):
+    """The workload both arms report (the reference arm times a bounded sample
+    of it, described in its cpu_baseline)."""
+    from tucker_quantized_residual_b200 import synth
+    dense = synth.dense_bf16_bytes(spec)
+    par = (f"one shared byte budget over {world} GPUs: rank r compresses sequences [r*{spec.batch}, "
+           f"(r+1)*{spec.batch}), one all-gather of per-cell rate-distortion records per step (NCCL)"
+           if world > 1 else "one GPU")
+    return {"workload": f"{args.config} ({spec.n_layers} layers / groups of {spec.group_size}, "
+                        f"{spec.n_heads} KV heads, D={spec.head_dim}, T={spec.seq_len}, "
+                        f"batch {spec.batch} per GPU), {args.ratio:g}x budget, {args.mode} token SVD",
+            "global_batch": spec.batch * world, "seq_len": spec.seq_len,
+            "parallelism": par,
+            "l2": f"inputs {dense / 1e9:.2f} GB per GPU" + (
+                ", larger than L2; no flush" if dense > 126e6 else ", smaller than L2")}
+
+
 def run_reference(args):
     """The oracle arm: the same bounded sample as the cpu_baseline leg, on the
     host cores, one sample per step."""
@@ -687,6 +695,8 @@ def run_reference(args):
         return
     from tucker_quantized_residual_b200 import synth
     spec = synth.SPECS[args.config]
+    if args.groups:
+        spec = spec.replace(n_layers=min(spec.n_layers, args.groups * spec.group_size))
     T_sample = args.cpu_tokens
     Ks, Vs = cpu_sample(spec, T_sample)
     for _ in range(args.warmup):
@@ -703,7 +713,7 @@ def run_reference(args):
             "value": round(value, 6), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{args.config} sample, {args.ratio:g}x budget"},
+            "config": arm_config(args, spec, int(os.environ.get("WORLD_SIZE", "1"))),
             "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
                              "sample": sample_text(spec, T_sample, 1)},
             "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
