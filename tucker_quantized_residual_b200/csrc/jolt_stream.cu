@@ -11,15 +11,11 @@
 // and scales with bulk copies; warp 1 issues tcgen05.mma (backbone tile
 // 128 x D in TMEM, K = r_T rounded up to 64, fp32 accumulate).
 //
-// Warps 2..9 form the epilogue: two threads per row, from two warps on the
-// same TMEM lane quarter. Thread half h of a row owns the columns
-// [hC, hC + C) and [D/2 + hC, D/2 + hC + C), C = D/4, so each RoPE pair
-// (i, i + D/2) stays in one thread. The Walsh-Hadamard stages of span < C and
-// the stage of span D/2 run in registers; the stage of span C pairs the two
-// halves and goes through a swizzled shared-memory exchange. Every stage
-// performs the same fp32 additions as the one-row transform, so the result
-// is identical to it. Codes, scales and decoded rows are stored straight
-// from registers.
+// Warps 2..17 form the epilogue: four threads per row, from four warps on the
+// same TMEM lane quarter (details below). Every Walsh-Hadamard stage performs
+// the same fp32 additions as the one-row transform, so the result is
+// identical to it. Codes, scales and decoded rows are stored straight from
+// registers.
 #include "jolt_stream.cuh"
 
 namespace jolt {

@@ -6,7 +6,8 @@
 // owns the TMEM accumulators and one elected thread issues tcgen05.mma
 // (kind::f16, bf16 x bf16 -> fp32), warps 2..5 drain the accumulators with
 // tcgen05.ld and store. Two accumulators in TMEM let the epilogue of one tile
-// overlap the main loop of the next. Every mbarrier wait is bounded by a
+// overlap the main loop of the next (one, when the CTA-pair kernel's N tiles
+// are wider than 256 columns). Every mbarrier wait is bounded by a
 // wall-clock deadline; on expiry the kernel records a timeout in the status
 // word, stops issuing, waits (bounded) for its own loads in flight, frees its
 // TMEM and returns.
