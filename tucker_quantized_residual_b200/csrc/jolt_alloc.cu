@@ -489,9 +489,11 @@ __global__ void k_alloc_init(AllocState* st, AllocState init) {
   if (threadIdx.x == 0 && blockIdx.x == 0) *st = init;
 }
 
-// Writes the initial state (phase 0, lambda = lo), then rounds of
-// evaluate + decide; each round tries one multiplier and rounds after the
-// decision return at once.
+// Writes the initial state (phase 0, lambda = lo), then max_iters + 2 rounds,
+// each trying one multiplier: one k_alloc_rows launch (evaluation and, in its
+// last block, the decision), or k_alloc_greedy + k_alloc_decide for the
+// greedy minimizer; rounds after the final decision return at once. Small
+// searches run every round inside one k_alloc_single block.
 jolt_status launch_alloc(const AllocArgs& a, const AllocState& init, cudaStream_t s) {
   // small searches (all options of all cells within a few per thread): one block
   if ((int64_t)a.ncells * a.n_bits * std::max(a.n_rt_max, 1) * a.n_rd <= (int64_t)16 * 1024) {
