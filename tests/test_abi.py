@@ -174,3 +174,30 @@ def test_plan_reports_oom_from_a_failing_allocator_without_touching_the_device()
         assert lib.jolt_set_allocator(None, None, None) == 0
     # only one of the two callbacks is an error
     assert lib.jolt_set_allocator(C.cast(af, C.c_void_p), None, None) == 1
+
+
+@pytest.mark.parametrize("call", ["compress", "compress_begin", "decompress", "rd_table", "residual_encode",
+                                  "residual_decode", "layer_groups"])
+def test_wrappers_refuse_host_tensors_for_device_buffers(call):
+    """Every entry point hands its buffers to kernels as device addresses; the
+    binding refuses host tensors before the call (a host address read as a
+    device one is a memory fault), so no plan or handle is needed here."""
+    import torch
+    x = torch.zeros(1, 2, 2, 64, 64)
+    codes = torch.zeros(4, 32, dtype=torch.uint8)
+    scales = torch.zeros(4, 1)
+    with pytest.raises(ValueError):
+        if call == "compress":
+            jolt.jolt_compress(0, x, x, 1000, 0)
+        elif call == "compress_begin":
+            jolt.jolt_compress_begin(0, x, x, 1000, 0, None)
+        elif call == "decompress":
+            jolt.jolt_decompress(0, x, x)
+        elif call == "rd_table":
+            jolt.jolt_rd_table(0, x, x, 1, 8, 64)
+        elif call == "residual_encode":
+            jolt.jolt_residual_encode(torch.zeros(4, 64), 64, 4, 64, 0, codes, scales)
+        elif call == "residual_decode":
+            jolt.jolt_residual_decode(codes, scales, 4, 64, 4, 64, 0, torch.zeros(4, 64))
+        else:
+            jolt.jolt_layer_groups(x)

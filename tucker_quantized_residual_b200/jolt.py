@@ -146,6 +146,14 @@ def _ptr(t) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _dev(**tensors) -> None:
+    """The library reads and writes these buffers from its kernels: refuse host
+    tensors before their addresses reach the device."""
+    for name, t in tensors.items():
+        if t is not None and not getattr(t, "is_cuda", False):
+            raise ValueError(f"{name} must be a CUDA tensor (the library reads and writes it on the device)")
+
+
 # ------------------------------------------------------------------ helpers
 def make_layout(t, group_start: Sequence[int], rope_theta_k: float = 0.0) -> Tuple[jolt_layout, object]:
     """Layout of a [B, L, H, T, D] torch tensor (d contiguous). Returns the
@@ -208,6 +216,7 @@ def jolt_num_cells(plan: int) -> int:
 
 
 def jolt_compress(plan: int, k, v, byte_budget: int = 0, seed: int = 0, stream=None) -> int:
+    _dev(k=k, v=v)
     lib = load_library()
     out = C.c_void_p()
     _check(lib.jolt_compress(plan, _ptr(k), _ptr(v), int(byte_budget), int(seed), _stream(stream),
@@ -220,6 +229,7 @@ def jolt_summary_bytes(plan: int) -> int:
 
 
 def jolt_compress_begin(plan: int, k, v, byte_budget: int, seed: int, summary, stream=None) -> int:
+    _dev(k=k, v=v)
     """Phase 1 of a shared-budget compression; `summary` is a CUDA uint8
     tensor of jolt_num_cells(plan) * jolt_summary_bytes(plan) bytes."""
     need = jolt_num_cells(plan) * jolt_summary_bytes(plan)
@@ -241,6 +251,7 @@ def jolt_compress_end(handle: int, all_summaries, n_total: int, first_cell: int,
 
 
 def jolt_decompress(handle: int, k_out, v_out, out_layout: Optional[jolt_layout] = None, stream=None) -> None:
+    _dev(k_out=k_out, v_out=v_out)
     lib = load_library()
     _check(lib.jolt_decompress(handle, _ptr(k_out), _ptr(v_out),
                                C.byref(out_layout) if out_layout is not None else None, _stream(stream)))
@@ -289,6 +300,7 @@ def jolt_free_handle(handle: int) -> None:
 
 def jolt_rd_table(plan: int, k, v, n_cells: int, max_t: int, D: int, stream=None):
     """Returns (norm_sq[n], sig_t[n][max_t], n_t, sig_d[n][D]) as Python lists."""
+    _dev(k=k, v=v)
     ns = (C.c_double * n_cells)()
     st = (C.c_double * (n_cells * max_t))()
     sd = (C.c_double * (n_cells * D))()
@@ -381,6 +393,7 @@ def jolt_sketch(plan: int, seed: int, n_cells: int, stream=None):
 
 
 def jolt_residual_encode(e, D: int, bits: int, group: int, seed: int, codes, scales, stream=None) -> None:
+    _dev(e=e, codes=codes, scales=scales)
     rows = e.numel() // D
     _check(load_library().jolt_residual_encode(_ptr(e), rows, D, bits, group, int(seed), _ptr(codes),
                                                _ptr(scales), _stream(stream)))
@@ -388,6 +401,7 @@ def jolt_residual_encode(e, D: int, bits: int, group: int, seed: int, codes, sca
 
 def jolt_residual_decode(codes, scales, rows: int, D: int, bits: int, group: int, seed: int, e_hat,
                          stream=None) -> None:
+    _dev(codes=codes, scales=scales, e_hat=e_hat)
     _check(load_library().jolt_residual_decode(_ptr(codes), _ptr(scales), rows, D, bits, group, int(seed),
                                                _ptr(e_hat), _stream(stream)))
 
@@ -396,6 +410,7 @@ def jolt_layer_groups(k, rope_theta_k: float = 0.0, power_iters: int = 4, seed: 
                       stream=None) -> Tuple[List[int], List[float]]:
     """Data-driven layer grouping of a [B, L, H, T, D] device key tensor:
     (group starts including 0 and L, the L-1 consecutive-layer scores)."""
+    _dev(k=k)
     L = k.shape[1]
     lay, keep = make_layout(k, [0, L], rope_theta_k)
     starts = (C.c_int32 * (L + 1))()
